@@ -1,0 +1,220 @@
+"""CPU oracle for the block-scaled FP4 quantized linear.
+
+TEST INFRASTRUCTURE ONLY.  The test suite, the package smoke check and the
+benchmark's CPU-baseline leg are the only users; the CUDA library never loads it.
+
+`fp4_oracle.c` is the oracle proper (plain C, fp32 steps as IEEE operations, fp64
+GEMM, OpenMP over rows).  This module builds it with gcc and exposes it through
+ctypes with numpy arrays.  `oracle_np.py` is an independent NumPy restatement used
+to cross-check it on tiny shapes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp4_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+MX, NV = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile fp4_oracle.c into liboracle.so (no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+                               "-shared", "-fPIC", "-std=c11", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P, I64, F, D, U8, U16 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_double,
+                                  ctypes.c_uint8, ctypes.c_uint16)
+        sig = {
+            "orc_e2m1_decode": (D, [U8]), "orc_e2m1_encode": (U8, [F]),
+            "orc_e4m3_decode": (D, [U8]), "orc_e4m3_encode": (U8, [F]),
+            "orc_e8m0_decode": (D, [U8]), "orc_bf16_to_f32": (F, [U16]),
+            "orc_f16_to_double": (D, [U16]),
+            "orc_sf_offset": (I64, [I64, I64, I64]), "orc_sf_bytes": (I64, [I64, I64]),
+            "orc_tensor_amax": (F, [P, I64]), "orc_nv_global": (F, [F]),
+            "orc_quant_mxfp4": (None, [P, I64, I64, P, P]),
+            "orc_quant_nvfp4": (None, [P, I64, I64, F, P, P]),
+            "orc_quant_mxfp8": (None, [P, I64, I64, P, P]),
+            "orc_dequant_fp4": (None, [ctypes.c_int, P, P, I64, D, P, I64, P]),
+            "orc_dequant_mxfp8": (None, [P, P, I64, P, I64, P]),
+            "orc_linear_fp64": (None, [P, I64, P, I64, I64, P, P, P]),
+            "orc_lowrank_fp64": (None, [P, I64, P, I64, P, P, I64, I64, P, P]),
+            "orc_num_threads": (ctypes.c_int, []),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# ----------------------------------------------------------------------------- codecs
+def e2m1_encode(v: float) -> int:
+    return lib().orc_e2m1_encode(float(v))
+
+
+def e2m1_decode(c: int) -> float:
+    return lib().orc_e2m1_decode(int(c))
+
+
+def e4m3_encode(v: float) -> int:
+    return lib().orc_e4m3_encode(float(v))
+
+
+def e4m3_decode(b: int) -> float:
+    return lib().orc_e4m3_decode(int(b))
+
+
+def e8m0_decode(b: int) -> float:
+    return lib().orc_e8m0_decode(int(b))
+
+
+def sf_offset(r: int, j: int, Kg: int) -> int:
+    return lib().orc_sf_offset(r, j, Kg)
+
+
+def sf_bytes(rows: int, Kg: int) -> int:
+    return lib().orc_sf_bytes(rows, Kg)
+
+
+def group_size(fmt: int) -> int:
+    return 32 if fmt == MX else 16
+
+
+# ----------------------------------------------------------------------------- quantizers
+def tensor_amax(x_bf16: np.ndarray) -> float:
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    return lib().orc_tensor_amax(_p(x), x.size)
+
+
+def nv_global(T: float) -> float:
+    return lib().orc_nv_global(float(T))
+
+
+def quantize(fmt: int, x_bf16: np.ndarray, g: float | None = None):
+    """bf16 [rows, K] -> (codes [rows, K/2] uint8, sf flat uint8) in format fmt."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, K = x.shape
+    G = group_size(fmt)
+    codes = np.zeros((rows, K // 2), dtype=np.uint8)
+    sf = np.zeros(sf_bytes(rows, K // G), dtype=np.uint8)
+    if fmt == MX:
+        lib().orc_quant_mxfp4(_p(x), rows, K, _p(codes), _p(sf))
+    else:
+        lib().orc_quant_nvfp4(_p(x), rows, K, float(g), _p(codes), _p(sf))
+    return codes, sf
+
+
+def quantize_mxfp8(x_bf16: np.ndarray):
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, K = x.shape
+    elems = np.zeros((rows, K), dtype=np.uint8)
+    sf = np.zeros(sf_bytes(rows, K // 32), dtype=np.uint8)
+    lib().orc_quant_mxfp8(_p(x), rows, K, _p(elems), _p(sf))
+    return elems, sf
+
+
+def pack_weight(fmt: int, w_bf16: np.ndarray):
+    """Offline weight pack: (codes, sf, global).  NVFP4 global from the tensor amax."""
+    if fmt == MX:
+        c, s = quantize(MX, w_bf16)
+        return c, s, None
+    g = nv_global(tensor_amax(w_bf16))
+    c, s = quantize(NV, w_bf16, g)
+    return c, s, g
+
+
+# ----------------------------------------------------------------------------- dequant
+def dequant_fp4(fmt: int, codes, sf, K: int, g: float = 1.0, rows=None) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    ids = np.arange(codes.shape[0], dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    out = np.empty((ids.size, K), dtype=np.float64)
+    lib().orc_dequant_fp4(fmt, _p(codes), _p(sf), K, float(g), _p(ids), ids.size, _p(out))
+    return out
+
+
+def dequant_mxfp8(elems, sf, K: int, rows=None) -> np.ndarray:
+    elems = np.ascontiguousarray(elems, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    ids = np.arange(elems.shape[0], dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    out = np.empty((ids.size, K), dtype=np.float64)
+    lib().orc_dequant_mxfp8(_p(elems), _p(sf), K, _p(ids), ids.size, _p(out))
+    return out
+
+
+def linear_fp64(a_deq: np.ndarray, w_deq: np.ndarray, bias_f16=None):
+    """(Y, S): Y = a w^T + bias in fp64, S = |a| |w|^T."""
+    a = np.ascontiguousarray(a_deq, dtype=np.float64)
+    w = np.ascontiguousarray(w_deq, dtype=np.float64)
+    nrows, K = a.shape
+    N = w.shape[0]
+    Y = np.empty((nrows, N), dtype=np.float64)
+    S = np.empty((nrows, N), dtype=np.float64)
+    b = None if bias_f16 is None else np.ascontiguousarray(bias_f16, dtype=np.uint16)
+    lib().orc_linear_fp64(_p(a), nrows, _p(w), N, K, None if b is None else _p(b), _p(Y), _p(S))
+    return Y, S
+
+
+def lowrank_fp64(x_bf16, rows, l1_bf16, l2_bf16):
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    l1 = np.ascontiguousarray(l1_bf16, dtype=np.uint16)
+    l2 = np.ascontiguousarray(l2_bf16, dtype=np.uint16)
+    ids = np.ascontiguousarray(rows, dtype=np.int64)
+    K, rank = l1.shape
+    N = l2.shape[1]
+    assert rank <= 256
+    LR = np.empty((ids.size, N), dtype=np.float64)
+    LS = np.empty((ids.size, N), dtype=np.float64)
+    lib().orc_lowrank_fp64(_p(x), K, _p(ids), ids.size, _p(l1), _p(l2), rank, N, _p(LR), _p(LS))
+    return LR, LS
+
+
+def fp4_linear_rows(fmt, x_bf16, w_bf16, bias_f16, rows, g_a=None, packed_w=None):
+    """End-to-end oracle of the W4A4 linear for selected rows of x.
+
+    Returns (Y, S) in fp64.  For NVFP4, g_a is the static activation global."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    K = x.shape[1]
+    wc, ws, gw = packed_w if packed_w is not None else pack_weight(fmt, w_bf16)
+    xs = np.ascontiguousarray(x[np.asarray(rows)])
+    ac, asf = quantize(fmt, xs, g_a)
+    a = dequant_fp4(fmt, ac, asf, K, 1.0 if fmt == MX else g_a)
+    w = dequant_fp4(fmt, wc, ws, K, 1.0 if fmt == MX else gw)
+    return linear_fp64(a, w, bias_f16)
+
+
+def num_threads() -> int:
+    return lib().orc_num_threads()
+
+
+def tolerance(Y_ref: np.ndarray, S: np.ndarray) -> np.ndarray:
+    """Per-element bound: one bf16 ulp of the exact result + 1e-5 * sum_k |a_k w_k|.
+
+    ulp_bf16(y) = 2^(floor(log2|y|) - 7); for y = 0 the smallest normal bf16 ulp 2^-133."""
+    a = np.abs(Y_ref)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))
+    ulp = np.where(a > 0, np.ldexp(1.0, np.maximum(ex - 1 - 7, -133)), 2.0 ** -133)
+    return ulp + 1e-5 * S
