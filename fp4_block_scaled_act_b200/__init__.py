@@ -1,0 +1,247 @@
+"""Python binding of libfp4bsa.so, the block-scaled FP4 quantized linear for B200.
+
+Every function below has the name of the C entry point it calls (include/fp4bsa.h)
+and only marshals arguments: tensors become device pointers, the current torch CUDA
+stream becomes the stream argument, and a non-OK status raises FP4Error.  All
+arithmetic runs in the library's CUDA kernels.  There is no fallback: if the
+library is missing or the device is not sm_100, the calls raise.
+
+The helpers at the end (pack_weight, linear, w4a8_linear) allocate outputs and
+workspaces with torch and call the same entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+from ._build import LIB as _LIB_PATH
+from ._build import build
+
+MXFP4, NVFP4 = 0, 1
+_FMT = {"mxfp4": MXFP4, "nvfp4": NVFP4, MXFP4: MXFP4, NVFP4: NVFP4}
+
+STATUS = ["FP4_OK", "FP4_ERR_INVALID_ARG", "FP4_ERR_UNSUPPORTED_SHAPE", "FP4_ERR_MISALIGNED",
+          "FP4_ERR_WORKSPACE", "FP4_ERR_ARCH", "FP4_ERR_CUDA", "FP4_ERR_TIMEOUT"]
+
+# every symbol include/fp4bsa.h declares
+EXPORTS = [
+    "fp4_codes_bytes", "fp4_sf_bytes", "fp4_linear_workspace_bytes", "w4a8_workspace_bytes",
+    "fp4_tensor_amax", "fp4_pack_weight", "fp4_quantize_act", "fp4_gemm", "fp4_linear",
+    "w4a8_quantize_act", "w4a8_gemm", "w4a8_svd_linear", "fp4_sync_status", "fp4_status_string",
+    "fp4_set_wait_timeout_ns",
+]
+
+
+class FP4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        name = STATUS[status] if 0 <= status < len(STATUS) else f"status {status}"
+        super().__init__(f"{where}: {name}")
+
+
+_lib = None
+
+
+def lib():
+    """Load libfp4bsa.so (it must have been built; see build())."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: run fp4_block_scaled_act_b200.build() first")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        sig = {
+            "fp4_codes_bytes": (SZ, [I, I64, I64]),
+            "fp4_sf_bytes": (SZ, [I, I64, I64]),
+            "fp4_linear_workspace_bytes": (SZ, [I, I64, I64, I64]),
+            "w4a8_workspace_bytes": (SZ, [I64, I64, I64, I]),
+            "fp4_tensor_amax": (I, [P, I64, P, P]),
+            "fp4_pack_weight": (I, [I, P, I64, I64, P, P, P, P]),
+            "fp4_quantize_act": (I, [I, P, I64, I64, P, P, P, P]),
+            "fp4_gemm": (I, [I, P, P, I64, I64, I64, P, P, P, P, P, P, P]),
+            "fp4_linear": (I, [I, P, I64, I64, I64, P, P, P, P, P, P, P, SZ, P]),
+            "w4a8_quantize_act": (I, [P, I64, I64, P, I, P, P, P, P]),
+            "w4a8_gemm": (I, [P, P, P, I64, I64, I64, P, P, P, I, P, P, P]),
+            "w4a8_svd_linear": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, P, SZ, P]),
+            "fp4_sync_status": (I, [P]),
+            "fp4_status_string": (ctypes.c_char_p, [I]),
+            "fp4_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
+            "fp4bsa_test_skip_iteration": (None, [I]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+# ----------------------------------------------------------------------------- marshalling
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise FP4Error(status, where)
+
+
+def _fmt(fmt) -> int:
+    return _FMT[fmt]
+
+
+# ----------------------------------------------------------------------------- entry points
+def fp4_codes_bytes(fmt, rows: int, K: int) -> int:
+    return lib().fp4_codes_bytes(_fmt(fmt), rows, K)
+
+
+def fp4_sf_bytes(fmt, rows: int, K: int) -> int:
+    return lib().fp4_sf_bytes(_fmt(fmt), rows, K)
+
+
+def fp4_linear_workspace_bytes(fmt, M: int, K: int, N: int) -> int:
+    return lib().fp4_linear_workspace_bytes(_fmt(fmt), M, K, N)
+
+
+def w4a8_workspace_bytes(M: int, K: int, N: int, rank: int = 32) -> int:
+    return lib().w4a8_workspace_bytes(M, K, N, rank)
+
+
+def fp4_tensor_amax(x, n: int, amax_out, stream=None):
+    _check(lib().fp4_tensor_amax(_ptr(x), n, _ptr(amax_out), _stream(stream)), "fp4_tensor_amax")
+
+
+def fp4_pack_weight(fmt, w, N: int, K: int, w_codes, w_sf, w_global=None, stream=None):
+    _check(lib().fp4_pack_weight(_fmt(fmt), _ptr(w), N, K, _ptr(w_codes), _ptr(w_sf), _ptr(w_global),
+                                 _stream(stream)), "fp4_pack_weight")
+
+
+def fp4_quantize_act(fmt, x, M: int, K: int, a_global, x_codes, x_sf, stream=None):
+    _check(lib().fp4_quantize_act(_fmt(fmt), _ptr(x), M, K, _ptr(a_global), _ptr(x_codes), _ptr(x_sf),
+                                  _stream(stream)), "fp4_quantize_act")
+
+
+def fp4_gemm(fmt, a_codes, a_sf, M: int, K: int, N: int, w_codes, w_sf, w_global, a_global, bias, y,
+             stream=None):
+    _check(lib().fp4_gemm(_fmt(fmt), _ptr(a_codes), _ptr(a_sf), M, K, N, _ptr(w_codes), _ptr(w_sf),
+                          _ptr(w_global), _ptr(a_global), _ptr(bias), _ptr(y), _stream(stream)), "fp4_gemm")
+
+
+def fp4_linear(fmt, x, M: int, K: int, N: int, w_codes, w_sf, w_global, a_global, bias, y, workspace,
+               ws_bytes: int, stream=None):
+    _check(lib().fp4_linear(_fmt(fmt), _ptr(x), M, K, N, _ptr(w_codes), _ptr(w_sf), _ptr(w_global),
+                            _ptr(a_global), _ptr(bias), _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
+           "fp4_linear")
+
+
+def w4a8_quantize_act(x, M: int, K: int, l1, rank: int, x_e4m3, x_sf, u, stream=None):
+    _check(lib().w4a8_quantize_act(_ptr(x), M, K, _ptr(l1), rank, _ptr(x_e4m3), _ptr(x_sf), _ptr(u),
+                                   _stream(stream)), "w4a8_quantize_act")
+
+
+def w4a8_gemm(x_e4m3, x_sf, u, M: int, K: int, N: int, r_codes, r_sf, l2, rank: int, bias, y, stream=None):
+    _check(lib().w4a8_gemm(_ptr(x_e4m3), _ptr(x_sf), _ptr(u), M, K, N, _ptr(r_codes), _ptr(r_sf), _ptr(l2),
+                           rank, _ptr(bias), _ptr(y), _stream(stream)), "w4a8_gemm")
+
+
+def w4a8_svd_linear(x, M: int, K: int, N: int, r_codes, r_sf, l1, l2, rank: int, bias, y, workspace,
+                    ws_bytes: int, stream=None):
+    _check(lib().w4a8_svd_linear(_ptr(x), M, K, N, _ptr(r_codes), _ptr(r_sf), _ptr(l1), _ptr(l2), rank,
+                                 _ptr(bias), _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
+           "w4a8_svd_linear")
+
+
+def fp4_sync_status(stream=None) -> int:
+    return lib().fp4_sync_status(_stream(stream))
+
+
+def fp4_status_string(status: int) -> str:
+    return lib().fp4_status_string(status).decode()
+
+
+def fp4_set_wait_timeout_ns(ns: int):
+    lib().fp4_set_wait_timeout_ns(ns)
+
+
+# ----------------------------------------------------------------------------- helpers
+@dataclass
+class PackedWeight:
+    fmt: int
+    N: int
+    K: int
+    codes: "object"          # torch.uint8 [N, K/2]
+    sf: "object"             # torch.uint8 [sf bytes]
+    w_global: "object" = None  # torch.float32 [1] (NVFP4)
+
+
+def pack_weight(w, fmt="mxfp4", stream=None) -> PackedWeight:
+    """bf16 [N, K] weight (CUDA) -> PackedWeight (codes, scales, NVFP4 global)."""
+    import torch
+
+    f = _fmt(fmt)
+    N, K = w.shape
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    sf = torch.empty(fp4_sf_bytes(f, N, K), dtype=torch.uint8, device=w.device)
+    g = torch.empty(1, dtype=torch.float32, device=w.device) if f == NVFP4 else None
+    fp4_pack_weight(f, w, N, K, codes, sf, g, stream)
+    return PackedWeight(f, N, K, codes, sf, g)
+
+
+def quantize_act(x, fmt="mxfp4", a_global=None, stream=None):
+    """bf16 [M, K] activations (CUDA) -> (codes [M, K/2], scale factors)."""
+    import torch
+
+    f = _fmt(fmt)
+    M, K = x.shape
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    sf = torch.empty(fp4_sf_bytes(f, M, K), dtype=torch.uint8, device=x.device)
+    fp4_quantize_act(f, x, M, K, a_global, codes, sf, stream)
+    return codes, sf
+
+
+def linear(x, pw: PackedWeight, bias=None, a_global=None, y=None, workspace=None, stream=None):
+    """W4A4 quantized linear: bf16 [M, K] -> bf16 [M, N]."""
+    import torch
+
+    M, K = x.shape
+    assert K == pw.K
+    if y is None:
+        y = torch.empty((M, pw.N), dtype=torch.bfloat16, device=x.device)
+    ws = fp4_linear_workspace_bytes(pw.fmt, M, K, pw.N)
+    if workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=x.device)
+    fp4_linear(pw.fmt, x, M, K, pw.N, pw.codes, pw.sf, pw.w_global, a_global, bias, y, workspace,
+               workspace.numel(), stream)
+    return y
+
+
+def w4a8_linear(x, r: PackedWeight, l1, l2, bias=None, y=None, workspace=None, stream=None):
+    """W4A8 SVDQuant linear: bf16 [M, K] -> bf16 [M, N] (MXFP4 residual r, rank-32 L1/L2)."""
+    import torch
+
+    M, K = x.shape
+    rank = l1.shape[1]
+    if y is None:
+        y = torch.empty((M, r.N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(w4a8_workspace_bytes(M, K, r.N, rank), dtype=torch.uint8, device=x.device)
+    w4a8_svd_linear(x, M, K, r.N, r.codes, r.sf, l1, l2, rank, bias, y, workspace, workspace.numel(), stream)
+    return y

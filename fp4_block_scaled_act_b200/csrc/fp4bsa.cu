@@ -1,0 +1,347 @@
+// fp4bsa.cu -- the C ABI (include/fp4bsa.h): argument validation, TMA descriptors,
+// kernel launches and the device status word.  One translation unit holds every
+// kernel, so the status word is a plain __device__ variable.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "fp4bsa.h"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+using namespace fp4;
+
+__device__ int g_fp4_status = 0;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+uint64_t g_timeout_ns = kDefaultTimeoutNs;
+int g_skip_iter = -1;  // test hook, see fp4bsa_test_skip_iteration
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceState {
+    bool ready = false;
+    bool arch_ok = false;
+    int sm_count = 0;
+    int* status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[64];
+EncodeTiledFn g_encode = nullptr;
+
+fp4_status_t device_state(DeviceState** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP4_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& s = g_dev[dev];
+    if (!s.ready) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&s.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return FP4_ERR_CUDA;
+        s.arch_ok = (major == 10 && minor == 0);
+        if (s.arch_ok) {
+            if (cudaGetSymbolAddress(reinterpret_cast<void**>(&s.status), g_fp4_status) != cudaSuccess)
+                return FP4_ERR_CUDA;
+            if (cudaFuncSetAttribute(gemm_kernel<G_MXFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     GemmCfg<G_MXFP4>::SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm_kernel<G_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     GemmCfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm_kernel<G_W4A8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     GemmCfg<G_W4A8>::SMEM_BYTES) != cudaSuccess)
+                return FP4_ERR_CUDA;
+        }
+        if (!g_encode) {
+            cudaDriverEntryPointQueryResult q;
+            void* fn = nullptr;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                return FP4_ERR_CUDA;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        s.ready = true;
+    }
+    if (!s.arch_ok) return FP4_ERR_ARCH;
+    *out = &s;
+    return FP4_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int group_of(fp4_fmt_t fmt) { return fmt == FP4_FMT_MXFP4 ? 32 : 16; }
+inline bool fmt_ok(fp4_fmt_t fmt) { return fmt == FP4_FMT_MXFP4 || fmt == FP4_FMT_NVFP4; }
+constexpr int64_t kMaxDim = (int64_t)1 << 30;
+
+fp4_status_t check_shape(int64_t M, int64_t K, int64_t N) {
+    if (M < 1) return FP4_ERR_INVALID_ARG;
+    if (K < 128 || K % 128 != 0 || N < 128 || N % 128 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (M >= kMaxDim || K >= kMaxDim || N >= kMaxDim) return FP4_ERR_UNSUPPORTED_SHAPE;
+    return FP4_OK;
+}
+
+fp4_status_t launched() { return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA; }
+
+int quant_blocks(const DeviceState* ds, int64_t M, int64_t K) {
+    const int64_t Mpad = (M + 127) & ~int64_t(127);
+    const int64_t threads = Mpad * (K / 128) * 16;
+    int64_t blocks = (threads + (int64_t)QUANT_THREADS * QUANT_UNROLL - 1) / ((int64_t)QUANT_THREADS * QUANT_UNROLL);
+    const int64_t cap = (int64_t)ds->sm_count * 16;
+    if (blocks > cap) blocks = cap;
+    return (int)(blocks < 1 ? 1 : blocks);
+}
+
+fp4_status_t launch_quant(const DeviceState* ds, int kind, const void* x, int64_t M, int64_t K, const float* g,
+                          uint8_t* out, uint8_t* sf, cudaStream_t st) {
+    const int blocks = quant_blocks(ds, M, K);
+    const uint4* xv = static_cast<const uint4*>(x);
+    if (kind == Q_MXFP4)
+        quant_kernel<Q_MXFP4><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
+    else if (kind == Q_NVFP4)
+        quant_kernel<Q_NVFP4><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
+    else
+        quant_kernel<Q_MXFP8><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
+    return launched();
+}
+
+fp4_status_t encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t rows,
+                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
+}
+
+template <int KIND>
+fp4_status_t launch_gemm(const DeviceState* ds, const CUtensorMap& ta, const CUtensorMap& tb, GemmParams& p,
+                         cudaStream_t st) {
+    const int tiles = ((p.M + GEMM_BM - 1) / GEMM_BM) * ((p.N + GEMM_BN - 1) / GEMM_BN);
+    const int grid = tiles < ds->sm_count ? tiles : ds->sm_count;
+    p.timeout_ns = g_timeout_ns;
+    p.skip_iter = g_skip_iter;
+    p.status = ds->status;
+    gemm_kernel<KIND><<<grid, GEMM_THREADS, GemmCfg<KIND>::SMEM_BYTES, st>>>(ta, tb, p);
+    return launched();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fp4_codes_bytes(fp4_fmt_t fmt, int64_t rows, int64_t K) {
+    if (!fmt_ok(fmt) || rows < 0 || K < 0 || (K & 1)) return 0;
+    return (size_t)rows * (size_t)(K / 2);
+}
+
+size_t fp4_sf_bytes(fp4_fmt_t fmt, int64_t rows, int64_t K) {
+    if (!fmt_ok(fmt) || rows < 0 || K < 0 || K % 128 != 0) return 0;
+    const int64_t rp = (rows + 127) / 128 * 128;
+    return (size_t)rp * (size_t)(K / group_of(fmt));
+}
+
+size_t fp4_linear_workspace_bytes(fp4_fmt_t fmt, int64_t M, int64_t K, int64_t N) {
+    if (!fmt_ok(fmt) || check_shape(M, K, N) != FP4_OK) return 0;
+    return align256(fp4_codes_bytes(fmt, M, K)) + align256(fp4_sf_bytes(fmt, M, K));
+}
+
+size_t w4a8_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank) {
+    if (rank != 32 || check_shape(M, K, N) != FP4_OK) return 0;
+    return align256((size_t)M * K) + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K)) + align256((size_t)M * rank * 4);
+}
+
+fp4_status_t fp4_tensor_amax(const void* x_bf16, int64_t n, float* amax_out, void* stream) {
+    if (!x_bf16 || !amax_out || n < 1) return FP4_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || (reinterpret_cast<uintptr_t>(amax_out) & 3u)) return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    fp4_status_t s = device_state(&ds);
+    if (s != FP4_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(amax_out, 0, sizeof(float), st) != cudaSuccess) return FP4_ERR_CUDA;
+    int64_t blocks = (n / 8 + 255) / 256;
+    if (blocks > ds->sm_count * 8) blocks = ds->sm_count * 8;
+    if (blocks < 1) blocks = 1;
+    amax_kernel<<<(int)blocks, 256, 0, st>>>(static_cast<const uint16_t*>(x_bf16), n,
+                                             reinterpret_cast<unsigned int*>(amax_out));
+    return launched();
+}
+
+fp4_status_t fp4_quantize_act(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K, const float* a_global,
+                              uint8_t* x_codes, uint8_t* x_sf, void* stream) {
+    if (!fmt_ok(fmt) || !x_bf16 || !x_codes || !x_sf) return FP4_ERR_INVALID_ARG;
+    if ((fmt == FP4_FMT_NVFP4) != (a_global != nullptr)) return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, 128);
+    if (s != FP4_OK) return s;
+    if (!aligned16(x_bf16) || !aligned16(x_codes) || !aligned16(x_sf) || !aligned16(a_global))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    if ((s = device_state(&ds)) != FP4_OK) return s;
+    return launch_quant(ds, fmt == FP4_FMT_MXFP4 ? Q_MXFP4 : Q_NVFP4, x_bf16, M, K, a_global, x_codes, x_sf,
+                        static_cast<cudaStream_t>(stream));
+}
+
+fp4_status_t fp4_pack_weight(fp4_fmt_t fmt, const void* w_bf16, int64_t N, int64_t K, uint8_t* w_codes,
+                             uint8_t* w_sf, float* w_global, void* stream) {
+    if (!fmt_ok(fmt) || !w_bf16 || !w_codes || !w_sf) return FP4_ERR_INVALID_ARG;
+    if ((fmt == FP4_FMT_NVFP4) != (w_global != nullptr)) return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(N, K, 128);
+    if (s != FP4_OK) return s;
+    if (!aligned16(w_bf16) || !aligned16(w_codes) || !aligned16(w_sf) || !aligned16(w_global))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    if ((s = device_state(&ds)) != FP4_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (fmt == FP4_FMT_NVFP4) {
+        if ((s = fp4_tensor_amax(w_bf16, N * K, w_global, stream)) != FP4_OK) return s;
+        nv_global_kernel<<<1, 1, 0, st>>>(w_global);
+        if ((s = launched()) != FP4_OK) return s;
+    }
+    return launch_quant(ds, fmt == FP4_FMT_MXFP4 ? Q_MXFP4 : Q_NVFP4, w_bf16, N, K, w_global, w_codes, w_sf, st);
+}
+
+fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf, int64_t M, int64_t K, int64_t N,
+                      const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global, const float* a_global,
+                      const void* bias_f16, void* y_bf16, void* stream) {
+    if (!fmt_ok(fmt) || !a_codes || !a_sf || !w_codes || !w_sf || !y_bf16) return FP4_ERR_INVALID_ARG;
+    const bool nv = (fmt == FP4_FMT_NVFP4);
+    if (nv != (w_global != nullptr) || nv != (a_global != nullptr)) return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, N);
+    if (s != FP4_OK) return s;
+    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) || !aligned16(y_bf16) ||
+        !aligned16(bias_f16) || (reinterpret_cast<uintptr_t>(w_global) & 3u) ||
+        (reinterpret_cast<uintptr_t>(a_global) & 3u))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    if ((s = device_state(&ds)) != FP4_OK) return s;
+    CUtensorMap ta, tb;
+    if ((s = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 128, GEMM_BM)) != FP4_OK) return s;
+    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 128, GEMM_BN)) != FP4_OK) return s;
+    GemmParams p{};
+    p.M = (int)M, p.N = (int)N, p.K = (int)K;
+    p.sfa = a_sf, p.sfb = w_sf, p.g_a = a_global, p.g_w = w_global;
+    p.bias = static_cast<const __half*>(bias_f16);
+    p.y = static_cast<__nv_bfloat16*>(y_bf16);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return nv ? launch_gemm<G_NVFP4>(ds, ta, tb, p, st) : launch_gemm<G_MXFP4>(ds, ta, tb, p, st);
+}
+
+fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K, int64_t N, const uint8_t* w_codes,
+                        const uint8_t* w_sf, const float* w_global, const float* a_global, const void* bias_f16,
+                        void* y_bf16, void* workspace, size_t ws_bytes, void* stream) {
+    if (!fmt_ok(fmt) || !x_bf16 || !workspace) return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, N);
+    if (s != FP4_OK) return s;
+    if (ws_bytes < fp4_linear_workspace_bytes(fmt, M, K, N)) return FP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+    uint8_t* codes = static_cast<uint8_t*>(workspace);
+    uint8_t* sf = codes + align256(fp4_codes_bytes(fmt, M, K));
+    // validate the GEMM's arguments before launching anything
+    const bool nv = (fmt == FP4_FMT_NVFP4);
+    if (!w_codes || !w_sf || !y_bf16 || nv != (w_global != nullptr) || nv != (a_global != nullptr))
+        return FP4_ERR_INVALID_ARG;
+    if ((s = fp4_quantize_act(fmt, x_bf16, M, K, a_global, codes, sf, stream)) != FP4_OK) return s;
+    return fp4_gemm(fmt, codes, sf, M, K, N, w_codes, w_sf, w_global, a_global, bias_f16, y_bf16, stream);
+}
+
+fp4_status_t w4a8_quantize_act(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16, int rank,
+                               uint8_t* x_e4m3, uint8_t* x_sf, float* u_f32, void* stream) {
+    if (!x_bf16 || !l1_bf16 || !x_e4m3 || !x_sf || !u_f32 || rank != 32) return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, 128);
+    if (s != FP4_OK) return s;
+    if (!aligned16(x_bf16) || !aligned16(l1_bf16) || !aligned16(x_e4m3) || !aligned16(x_sf) || !aligned16(u_f32))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    if ((s = device_state(&ds)) != FP4_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = launch_quant(ds, Q_MXFP8, x_bf16, M, K, nullptr, x_e4m3, x_sf, st)) != FP4_OK) return s;
+    const int blocks = (int)((M + 31) / 32);
+    lowrank_down_kernel<32><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x_bf16),
+                                                   static_cast<const __nv_bfloat16*>(l1_bf16), M, K, u_f32);
+    return launched();
+}
+
+fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const float* u_f32, int64_t M, int64_t K,
+                       int64_t N, const uint8_t* r_codes, const uint8_t* r_sf, const void* l2_bf16, int rank,
+                       const void* bias_f16, void* y_bf16, void* stream) {
+    if (!x_e4m3 || !x_sf || !u_f32 || !r_codes || !r_sf || !l2_bf16 || !y_bf16 || rank != 32)
+        return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, N);
+    if (s != FP4_OK) return s;
+    if (!aligned16(x_e4m3) || !aligned16(x_sf) || !aligned16(u_f32) || !aligned16(r_codes) || !aligned16(r_sf) ||
+        !aligned16(l2_bf16) || !aligned16(bias_f16) || !aligned16(y_bf16))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    if ((s = device_state(&ds)) != FP4_OK) return s;
+    CUtensorMap ta, tb;
+    if ((s = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_e4m3, K, M, K, 128, GEMM_BM)) != FP4_OK) return s;
+    // packed E2M1 in global memory, unpacked to one 16-byte slot per 16 values in shared memory
+    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, r_codes, K, N, K / 2, 128, GEMM_BN)) != FP4_OK)
+        return s;
+    GemmParams p{};
+    p.M = (int)M, p.N = (int)N, p.K = (int)K;
+    p.sfa = x_sf, p.sfb = r_sf;
+    p.bias = static_cast<const __half*>(bias_f16);
+    p.y = static_cast<__nv_bfloat16*>(y_bf16);
+    p.u = u_f32;
+    p.l2 = static_cast<const __nv_bfloat16*>(l2_bf16);
+    return launch_gemm<G_W4A8>(ds, ta, tb, p, static_cast<cudaStream_t>(stream));
+}
+
+fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N, const uint8_t* r_codes,
+                             const uint8_t* r_sf, const void* l1_bf16, const void* l2_bf16, int rank,
+                             const void* bias_f16, void* y_bf16, void* workspace, size_t ws_bytes, void* stream) {
+    if (!workspace || rank != 32) return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, N);
+    if (s != FP4_OK) return s;
+    if (ws_bytes < w4a8_workspace_bytes(M, K, N, rank)) return FP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+    if (!r_codes || !r_sf || !l2_bf16 || !y_bf16) return FP4_ERR_INVALID_ARG;
+    uint8_t* xe = static_cast<uint8_t*>(workspace);
+    uint8_t* xs = xe + align256((size_t)M * K);
+    float* u = reinterpret_cast<float*>(xs + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K)));
+    if ((s = w4a8_quantize_act(x_bf16, M, K, l1_bf16, rank, xe, xs, u, stream)) != FP4_OK) return s;
+    return w4a8_gemm(xe, xs, u, M, K, N, r_codes, r_sf, l2_bf16, rank, bias_f16, y_bf16, stream);
+}
+
+fp4_status_t fp4_sync_status(void* stream) {
+    DeviceState* ds;
+    fp4_status_t s = device_state(&ds);
+    if (s != FP4_OK) return s;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP4_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_fp4_status, sizeof(int)) != cudaSuccess) return FP4_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_fp4_status, &zero, sizeof(int)) != cudaSuccess) return FP4_ERR_CUDA;
+    return word == 0 ? FP4_OK : static_cast<fp4_status_t>(word);
+}
+
+const char* fp4_status_string(fp4_status_t status) {
+    switch (status) {
+        case FP4_OK: return "FP4_OK";
+        case FP4_ERR_INVALID_ARG: return "FP4_ERR_INVALID_ARG";
+        case FP4_ERR_UNSUPPORTED_SHAPE: return "FP4_ERR_UNSUPPORTED_SHAPE";
+        case FP4_ERR_MISALIGNED: return "FP4_ERR_MISALIGNED";
+        case FP4_ERR_WORKSPACE: return "FP4_ERR_WORKSPACE";
+        case FP4_ERR_ARCH: return "FP4_ERR_ARCH";
+        case FP4_ERR_CUDA: return "FP4_ERR_CUDA";
+        case FP4_ERR_TIMEOUT: return "FP4_ERR_TIMEOUT";
+    }
+    return "FP4_ERR_UNKNOWN";
+}
+
+void fp4_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTimeoutNs; }
+
+// Test hook (not in the public header): the GEMM producer skips the given k-iteration of
+// its ring, so the MMA warp's bounded wait runs out.  -1 disables it.
+void fp4bsa_test_skip_iteration(int it) { g_skip_iter = it; }
+
+}  // extern "C"

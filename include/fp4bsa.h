@@ -1,0 +1,195 @@
+/*
+ * fp4bsa.h -- C ABI of the block-scaled FP4 quantized linear for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the quantized linear layer of the Wan2.2 diffusion transformers:
+ * bf16 activations are quantized on the fly to FP4 E2M1 with per-block scales and
+ * multiplied against pre-packed FP4 weights; an fp16 bias is added and the output is
+ * bf16.  Two FP4 formats are supported:
+ *
+ *   MXFP4  E2M1 values, two per byte, one E8M0 scale per 32 values along K
+ *          (Wan2.2-I2V-A14B-Lightning-Diffusers-MXFP4-AutoRound, "Quantization Details":
+ *           group_size 32, act_dynamic, weights "packed FP4 E2M1 (two FP4 values per
+ *           byte) with per-32 E8M0 scales"; biases kept F16).
+ *   NVFP4  E2M1 values, one FP8 E4M3 scale per 16 values, one FP32 global scale per
+ *          tensor; activations use dynamic block scales under a static, calibrated
+ *          global (Wan2.2-T2V-A14B-Diffusers-NVFP4-AutoRound, "Model Details").
+ *
+ * and a W4A8 SVDQuant linear: MXFP4 residual weight, dynamic MXFP8 (E4M3, per-32
+ * E8M0) activations, and a rank-32 low-rank correction x L1 L2 added in the epilogue
+ * (wan2.2-ti2v-w4a8-svd README, opening paragraph).
+ *
+ * ---------------------------------------------------------------------------------
+ * Conventions (apply to every call)
+ *   - Pointers marked (device) are CUDA device pointers; (host) are host pointers.
+ *     All device pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Every call that launches work is asynchronous on `stream`; no call synchronizes
+ *     except fp4_sync_status.
+ *   - Ownership: the caller allocates and frees every buffer, including workspaces.
+ *     The library allocates no device memory.  It keeps a process-wide cache of TMA
+ *     descriptors keyed by (pointer, shape) and a device status word per GPU.
+ *   - Shapes: M >= 1 (any value), K and N multiples of 128, all < 2^31 / 2.
+ *   - Errors: arguments are validated on the host before any launch; an invalid call
+ *     returns a status and launches nothing.  Launch failures return FP4_ERR_CUDA.  A
+ *     device-side wait that runs out of time records FP4_ERR_TIMEOUT in the status
+ *     word (read it with fp4_sync_status).  No C++ exception crosses this ABI.
+ *
+ * Layouts (part of the ABI; exactly what the CPU oracle in oracle/ produces):
+ *   codes  [rows][K/2] bytes, row-major; element 2i in bits 3:0, element 2i+1 in
+ *          bits 7:4 of byte i of its row.
+ *   sf     one byte per group (G = 32 for MXFP4/MXFP8, 16 for NVFP4) in 128-row x
+ *          4-group atoms of 512 bytes, rows padded to a multiple of 128:
+ *            off(r, j) = ((r/128)*(Kg/4) + j/4)*512 + (r%32)*16 + ((r%128)/32)*4 + j%4
+ *          with Kg = K/G.  Padding bytes are written as 0.
+ *   e4m3 elements (MXFP8) [rows][K] bytes, row-major.
+ *   Rounding: E2M1 and E4M3 round to nearest, ties to even, saturating (E2M1 at 6,
+ *   E4M3 at 448); the sign of zero is kept.  MX scale = 2^(floor(log2 amax) - 2)
+ *   (MXFP8: - 8) stored as E8M0; an all-zero group stores 0x00.  NVFP4:
+ *   g = T/2688 (T = tensor amax, 2688 = 6*448; T = 0 gives g = 1),
+ *   s = amax/(6 g) -> E4M3, codes = e2m1(x * (1/(dec(s) g))), each step one fp32
+ *   IEEE operation; a block whose scale is 0 stores zero codes.
+ * ---------------------------------------------------------------------------------
+ */
+#ifndef FP4BSA_H
+#define FP4BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { FP4_FMT_MXFP4 = 0, FP4_FMT_NVFP4 = 1 } fp4_fmt_t;
+
+typedef enum {
+    FP4_OK = 0,
+    FP4_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, M < 1, rank != 32 */
+    FP4_ERR_UNSUPPORTED_SHAPE = 2, /* K or N not a multiple of 128, sizes too large */
+    FP4_ERR_MISALIGNED = 3,        /* a device pointer not 16-byte aligned */
+    FP4_ERR_WORKSPACE = 4,         /* workspace smaller than the size query returned */
+    FP4_ERR_ARCH = 5,              /* current device is not sm_100 */
+    FP4_ERR_CUDA = 6,              /* a CUDA runtime or driver call failed */
+    FP4_ERR_TIMEOUT = 7            /* a device-side wait ran out of time (see fp4_sync_status) */
+} fp4_status_t;
+
+/* ----------------------------------------------------------------- size queries (host) */
+
+/* Bytes of packed E2M1 codes for a [rows, K] operand: rows * K / 2.  0 if K is odd. */
+size_t fp4_codes_bytes(fp4_fmt_t fmt, int64_t rows, int64_t K);
+
+/* Bytes of the scale-factor buffer of a [rows, K] operand in the 128x4 atom layout:
+ * ceil(rows/128)*128 * K/G (G = 32 MXFP4, 16 NVFP4).  0 on a bad fmt or K % 128 != 0. */
+size_t fp4_sf_bytes(fp4_fmt_t fmt, int64_t rows, int64_t K);
+
+/* Workspace fp4_linear needs: the quantized activation codes and scales, each
+ * 256-byte aligned.  0 on invalid arguments. */
+size_t fp4_linear_workspace_bytes(fp4_fmt_t fmt, int64_t M, int64_t K, int64_t N);
+
+/* Workspace w4a8_svd_linear needs: MXFP8 elements [M,K], their scales, and the fp32
+ * low-rank projection u = x L1 [M, rank], each 256-byte aligned. */
+size_t w4a8_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank);
+
+/* ----------------------------------------------------------------- quantization */
+
+/* Per-tensor amax: *amax_out (device fp32) = max |x_i| over n bf16 values (device).
+ * Used for the NVFP4 weight global and for calibrating the static activation global
+ * (NVFP4 card: "calibrated static global scales").  The result is order-independent. */
+fp4_status_t fp4_tensor_amax(const void* x_bf16, int64_t n, float* amax_out, void* stream);
+
+/* Offline weight pre-pack (MXFP4 / NVFP4 cards: weights stored as packed E2M1 with
+ * block scales; NVFP4 adds an FP32 global from the tensor amax).
+ *   w_bf16    (device) [N, K] bf16, torch Linear layout (out_features x in_features)
+ *   w_codes   (device, out) fp4_codes_bytes(fmt, N, K) bytes
+ *   w_sf      (device, out) fp4_sf_bytes(fmt, N, K) bytes
+ *   w_global  (device, out) NVFP4: one fp32, g_w = max|W| / 2688; MXFP4: must be NULL
+ * Same rounding as the activation quantizer; deterministic. */
+fp4_status_t fp4_pack_weight(fp4_fmt_t fmt, const void* w_bf16, int64_t N, int64_t K,
+                             uint8_t* w_codes, uint8_t* w_sf, float* w_global, void* stream);
+
+/* Dynamic activation quantization (MXFP4 card: act_dynamic, act_group_size 32; NVFP4
+ * card: dynamic block scales with a calibrated static global).
+ *   x_bf16    (device) [M, K] bf16 row-major
+ *   a_global  (device) NVFP4: the static activation global g_a (one fp32); MXFP4: NULL
+ *   x_codes   (device, out) fp4_codes_bytes(fmt, M, K) bytes
+ *   x_sf      (device, out) fp4_sf_bytes(fmt, M, K) bytes (padding rows zeroed) */
+fp4_status_t fp4_quantize_act(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K,
+                              const float* a_global, uint8_t* x_codes, uint8_t* x_sf,
+                              void* stream);
+
+/* ----------------------------------------------------------------- GEMM */
+
+/* Block-scaled FP4 x FP4 GEMM with fused epilogue on pre-quantized activations
+ * (MXFP4 card: "FlashInferMxFp4LinearKernel + cuDNN blockScaleMatMul (W4A4)"; NVFP4
+ * card: "CUTLASS NVFP4 GEMMs, not an activation quantize-dequantize emulation path"):
+ *   y[m,n] = bf16_rn( gs * sum_k deq(a[m,k]) deq(w[n,k]) + bias[n] )
+ * with gs = g_a * g_w for NVFP4 and 1 for MXFP4; the sum accumulates in fp32.
+ *   a_codes, a_sf       (device) quantized activations as fp4_quantize_act writes them
+ *   w_codes, w_sf       (device) packed weight as fp4_pack_weight writes it
+ *   w_global, a_global  (device) NVFP4 globals; both NULL for MXFP4
+ *   bias_f16            (device) [N] fp16, or NULL for no bias
+ *   y_bf16              (device, out) [M, N] bf16 row-major */
+fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf, int64_t M,
+                      int64_t K, int64_t N, const uint8_t* w_codes, const uint8_t* w_sf,
+                      const float* w_global, const float* a_global, const void* bias_f16,
+                      void* y_bf16, void* stream);
+
+/* The W4A4 quantized linear: fp4_quantize_act into `workspace`, then fp4_gemm.
+ *   x_bf16     (device) [M, K] bf16
+ *   workspace  (device) at least fp4_linear_workspace_bytes(fmt, M, K, N) bytes; its
+ *              contents on return are the quantized activations (codes, then scales)
+ * Other arguments as fp4_gemm. */
+fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K, int64_t N,
+                        const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
+                        const float* a_global, const void* bias_f16, void* y_bf16,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* ----------------------------------------------------------------- W4A8 SVDQuant */
+
+/* Activation side of the W4A8 SVDQuant linear (W4A8 README: "dynamic MXFP8
+ * activations, rank-32 low-rank correction"; the low-rank branch reads the
+ * unquantized input):
+ *   x_bf16   (device) [M, K] bf16
+ *   l1_bf16  (device) [K, rank] bf16 (proj_down with 1/s folded in)
+ *   x_e4m3   (device, out) [M, K] E4M3 bytes
+ *   x_sf     (device, out) fp4_sf_bytes(FP4_FMT_MXFP4, M, K) bytes (E8M0, per 32)
+ *   u_f32    (device, out) [M, rank] fp32, u = x L1 accumulated in fp32 */
+fp4_status_t w4a8_quantize_act(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16,
+                               int rank, uint8_t* x_e4m3, uint8_t* x_sf, float* u_f32,
+                               void* stream);
+
+/* W4A8 GEMM with low-rank epilogue: y = bf16_rn( sum_k deq8(x) deq4(r) + u L2 + bias ).
+ *   r_codes, r_sf  (device) MXFP4-packed residual weight [N, K] (fp4_pack_weight)
+ *   l2_bf16        (device) [rank, N] bf16
+ * The low-rank product u L2 is evaluated with fp32 FMAs in the epilogue. */
+fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const float* u_f32, int64_t M,
+                       int64_t K, int64_t N, const uint8_t* r_codes, const uint8_t* r_sf,
+                       const void* l2_bf16, int rank, const void* bias_f16, void* y_bf16,
+                       void* stream);
+
+/* The full W4A8 SVDQuant linear: w4a8_quantize_act into `workspace`, then w4a8_gemm.
+ * rank must be 32. */
+fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N,
+                             const uint8_t* r_codes, const uint8_t* r_sf, const void* l1_bf16,
+                             const void* l2_bf16, int rank, const void* bias_f16, void* y_bf16,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* ----------------------------------------------------------------- status */
+
+/* Synchronizes `stream`, then returns and clears the device status word of the current
+ * GPU: FP4_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
+ * FP4_ERR_CUDA if the synchronization failed, FP4_OK otherwise. */
+fp4_status_t fp4_sync_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* fp4_status_string(fp4_status_t status);
+
+/* Test hook: limit, in nanoseconds, of every device-side wait in kernels launched
+ * after this call on this process (default 2e9 = 2 s).  0 restores the default. */
+void fp4_set_wait_timeout_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4BSA_H */

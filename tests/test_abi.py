@@ -1,0 +1,106 @@
+"""The C ABI on the host (no GPU): the library loads, exports every symbol the header
+declares, answers size queries, and rejects invalid calls before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fb():
+    import fp4_block_scaled_act_b200 as fb
+
+    fb.build()
+    return fb
+
+
+def header_symbols():
+    text = open(os.path.join(ROOT, "include", "fp4bsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b((?:fp4|w4a8)_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_header_symbol(fb):
+    syms = header_symbols()
+    assert len(syms) >= 15
+    L = ctypes.CDLL(os.path.join(ROOT, "fp4_block_scaled_act_b200", "libfp4bsa.so"))
+    for s in syms:
+        assert hasattr(L, s), s
+    assert sorted(fb.EXPORTS) == syms
+
+
+def test_size_queries(fb):
+    MX, NV = fb.MXFP4, fb.NVFP4
+    assert fb.fp4_codes_bytes(MX, 75600, 5120) == 75600 * 2560
+    assert fb.fp4_sf_bytes(MX, 75600, 5120) == 75648 * 160     # rows padded to 128
+    assert fb.fp4_sf_bytes(NV, 75600, 5120) == 75648 * 320
+    assert fb.fp4_sf_bytes(MX, 1, 128) == 128 * 4
+    assert fb.fp4_sf_bytes(MX, 10, 100) == 0                    # K % 128 != 0
+    assert fb.lib().fp4_sf_bytes(7, 10, 128) == 0               # bad format
+    ws = fb.fp4_linear_workspace_bytes(MX, 75600, 5120, 13824)
+    assert ws == 193536000 + 12103680
+    assert fb.fp4_linear_workspace_bytes(MX, 0, 5120, 13824) == 0
+    assert fb.w4a8_workspace_bytes(4290, 3072, 14336, 32) > 4290 * 3072
+    assert fb.w4a8_workspace_bytes(4290, 3072, 14336, 16) == 0
+
+
+def test_bytes_per_weight_match_format(fb):
+    """Packed FP4 + scales = 0.5 + 1/32 (MXFP4) or 0.5 + 1/16 (NVFP4) bytes per weight for
+    every Wan2.2 A14B linear shape (N multiple of 128: no padding)."""
+    for N, K in ((5120, 5120), (13824, 5120), (5120, 13824)):
+        mx = fb.fp4_codes_bytes(fb.MXFP4, N, K) + fb.fp4_sf_bytes(fb.MXFP4, N, K)
+        nv = fb.fp4_codes_bytes(fb.NVFP4, N, K) + fb.fp4_sf_bytes(fb.NVFP4, N, K)
+        assert mx * 32 == N * K * 17
+        assert nv * 16 == N * K * 9
+
+
+def test_status_strings(fb):
+    for i, name in enumerate(fb.STATUS):
+        assert fb.fp4_status_string(i) == name
+
+
+def test_invalid_calls_rejected_before_launch(fb):
+    """Fake (never dereferenced) pointers: validation must fail first."""
+    L = fb.lib()
+    P = ctypes.c_void_p
+    A = 1 << 20          # 16-byte aligned fake address
+    bad = A + 8          # misaligned
+    st = P(0)
+    # bad format
+    assert L.fp4_quantize_act(5, A, 16, 256, None, A, A, st) == 1
+    # K not a multiple of 128
+    assert L.fp4_quantize_act(0, A, 16, 200, None, A, A, st) == 2
+    # M < 1
+    assert L.fp4_quantize_act(0, A, 0, 256, None, A, A, st) == 1
+    # NVFP4 without an activation global / MXFP4 with one
+    assert L.fp4_quantize_act(1, A, 16, 256, None, A, A, st) == 1
+    assert L.fp4_quantize_act(0, A, 16, 256, A, A, A, st) == 1
+    # misaligned pointer
+    assert L.fp4_quantize_act(0, bad, 16, 256, None, A, A, st) == 3
+    # null output
+    assert L.fp4_quantize_act(0, A, 16, 256, None, None, A, st) == 1
+    # GEMM: N not a multiple of 128
+    assert L.fp4_gemm(0, A, A, 16, 256, 200, A, A, None, None, None, A, st) == 2
+    assert L.fp4_gemm(0, A, A, 16, 256, 256, A, A, None, None, bad, A, st) == 3
+    # linear: workspace too small
+    assert L.fp4_linear(0, A, 16, 256, 256, A, A, None, None, None, A, A, 10, st) == 4
+    # W4A8: rank must be 32
+    assert L.w4a8_svd_linear(A, 16, 256, 256, A, A, A, A, 16, None, A, A, 1 << 30, st) == 1
+    assert L.w4a8_gemm(A, A, A, 16, 256, 384, A, A, A, 32, None, bad, st) == 3
+    # weight pack: MXFP4 must not get a global
+    assert L.fp4_pack_weight(0, A, 256, 256, A, A, A, st) == 1
+    assert L.fp4_tensor_amax(A, 0, A, st) == 1
+
+
+def test_product_path_has_no_oracle_import():
+    """The package never imports or loads the oracle."""
+    pkg = os.path.join(ROOT, "fp4_block_scaled_act_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                for pat in ("import oracle", "from oracle", "liboracle", "fp4_oracle"):
+                    assert pat not in text, (f, pat)

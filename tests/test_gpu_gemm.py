@@ -1,0 +1,192 @@
+"""GPU parity of the block-scaled GEMM and the end-to-end quantized linear.
+
+Every output element is checked against the fp64 oracle on the dequantized operands
+within |y - y_ref| <= ulp_bf16(y_ref) + 1e-5 * sum_k |a_k w_k| for small shapes (several
+tiles, ragged M and N tails, odd K stages); at the full Wan2.2 sizes, in the launch
+configuration the benchmark times, sampled rows (including every row of the ragged
+last tile) are checked the same way.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+MX, NV = oracle.MX, oracle.NV
+
+
+@pytest.fixture(scope="module")
+def fb():
+    import fp4_block_scaled_act_b200 as fb
+
+    fb.build()
+    return fb
+
+
+def _run_linear(fb, fmt, x_bits, w_bits, b_bits, g_a=None):
+    import torch
+
+    x = H.dev_bf16(x_bits)
+    pw = fb.pack_weight(H.dev_bf16(w_bits), fmt)
+    bias = H.dev_f16(b_bits) if b_bits is not None else None
+    ga = H.dev_f32([g_a]) if fmt == NV else None
+    y = fb.linear(x, pw, bias, ga)
+    st = fb.fp4_sync_status()
+    assert st == 0, fb.fp4_status_string(st)
+    torch.cuda.synchronize()
+    return y
+
+
+def _oracle(orc, fmt, x_bits, w_bits, b_bits, rows, g_a=None):
+    return orc.fp4_linear_rows(fmt, x_bits, w_bits, b_bits, rows, g_a=g_a)
+
+
+SMALL = [
+    (1, 256, 256), (128, 256, 256), (129, 512, 384), (256, 512, 512), (300, 384, 640),
+    (77, 1280, 1024), (513, 768, 256),
+]
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("M,K,N", SMALL)
+def test_linear_small_all_elements(fb, orc, fmt, M, K, N):
+    kind = "outlier" if (M, K, N) == (256, 512, 512) else "lognormal"
+    x = synth.activation(10 * M + K, M, K, kind)
+    w = synth.weight(20 * N + K, N, K)
+    b = synth.bias(N + 3, N)
+    g_a = None
+    if fmt == NV:
+        g_a = orc.nv_global(orc.tensor_amax(synth.activation(30 * M + K, 64, K, kind)))
+    y = _run_linear(fb, fmt, x, w, b, g_a)
+    rows = np.arange(M)
+    Y, S = _oracle(orc, fmt, x, w, b, rows, g_a)
+    H.check_linear(y, Y, S, rows, f"fmt={fmt} M={M} K={K} N={N}")
+
+
+def test_linear_no_bias(fb, orc):
+    M, K, N = 200, 512, 384
+    x = synth.activation(1, M, K, "lognormal")
+    w = synth.weight(2, N, K)
+    y = _run_linear(fb, MX, x, w, None)
+    Y, S = _oracle(orc, MX, x, w, None, np.arange(M))
+    H.check_linear(y, Y, S, np.arange(M), "no bias")
+
+
+def test_gemm_exact_grid_values(fb, orc):
+    """Grid-valued operands with scale 1: the exact product is representable, so y must
+    equal bf16(exact) with the error of a single rounding."""
+    rng = np.random.default_rng(3)
+    M, K, N = 130, 512, 256
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float32)
+
+    def gm(r, c):
+        v = grid[rng.integers(0, 8, size=(r, c))] * np.where(rng.random((r, c)) < 0.5, -1, 1)
+        v[:, ::32] = 6.0
+        return v.astype(np.float32)
+
+    a, w = gm(M, K), gm(N, K)
+    y = _run_linear(fb, MX, synth.f32_to_bf16_bits(a), synth.f32_to_bf16_bits(w), None)
+    exact = a.astype(np.float64) @ w.astype(np.float64).T
+    got = H.host_bf16_as_f64(y)
+    ref_bf16 = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(exact.astype(np.float32))).astype(np.float64)
+    np.testing.assert_array_equal(got, ref_bf16)
+
+
+def test_gemm_selector_weight(fb, orc):
+    """W row n holds a single 4.0 at column (5n) % K: y[:, n] = 4 * deq(a)[:, (5n) % K]."""
+    M, K, N = 256, 1024, 512
+    x = synth.activation(4, M, K, "lognormal")
+    w = np.zeros((N, K), dtype=np.float32)
+    cols = (5 * np.arange(N)) % K
+    w[np.arange(N), cols] = 4.0
+    y = _run_linear(fb, MX, x, synth.f32_to_bf16_bits(w), None)
+    codes, sf = orc.quantize(MX, x)
+    a = orc.dequant_fp4(MX, codes, sf, K)
+    exp = 4.0 * a[:, cols]
+    np.testing.assert_array_equal(H.host_bf16_as_f64(y),
+                                  synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(exp.astype(np.float32))))
+
+
+def test_gemm_determinism(fb):
+    import torch
+
+    M, K, N = 700, 1024, 768
+    x = H.dev_bf16(synth.activation(5, M, K, "lognormal"))
+    pw = fb.pack_weight(H.dev_bf16(synth.weight(6, N, K)), MX)
+    y1 = fb.linear(x, pw)
+    y2 = fb.linear(x, pw)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_gemm_entry_matches_linear(fb):
+    """fp4_gemm on separately quantized activations == fp4_linear (same kernels)."""
+    import torch
+
+    M, K, N = 333, 768, 512
+    x = H.dev_bf16(synth.activation(8, M, K, "lognormal"))
+    pw = fb.pack_weight(H.dev_bf16(synth.weight(9, N, K)), NV)
+    ga = H.dev_f32([0.01])
+    codes, sf = fb.quantize_act(x, NV, ga)
+    y1 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    fb.fp4_gemm(NV, codes, sf, M, K, N, pw.codes, pw.sf, pw.w_global, ga, None, y1)
+    y2 = fb.linear(x, pw, None, ga)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+# ------------------------------------------------------------------ full-size workloads
+FULL = [
+    # (config, fmt, M, K, N, activation kind)
+    (1, MX, 75600, 5120, 5120, "lognormal"),     # attention projection, MXFP4
+    (4, MX, 75600, 5120, 13824, "lognormal"),    # ffn up, MXFP4 (the benchmark workload)
+    (2, NV, 75600, 5120, 13824, "lognormal"),    # ffn up, NVFP4
+    (2, NV, 75600, 13824, 5120, "gelu"),         # ffn down, NVFP4
+    (4, MX, 512, 5120, 5120, "lognormal"),       # attn2 k/v on 512 text tokens
+]
+
+
+@pytest.mark.parametrize("cfg,fmt,M,K,N,kind", FULL)
+def test_linear_full_size_sampled(fb, orc, cfg, fmt, M, K, N, kind):
+    s = synth.seeds_for(cfg, layer=K // 1000 + N // 1000)
+    x = synth.activation(s["x"], M, K, kind, gain_seed=s["gain"])
+    w = synth.weight(s["w"], N, K)
+    b = synth.bias(s["bias"], N)
+    g_a = None
+    if fmt == NV:
+        cal = synth.activation(s["calib"], synth.CALIB_TOKENS, K, kind, gain_seed=s["gain"])
+        g_a = orc.nv_global(orc.tensor_amax(cal))
+    y = _run_linear(fb, fmt, x, w, b, g_a)
+    rows = H.sample_rows(M, n_random=40, seed=cfg)
+    Y, S = _oracle(orc, fmt, x, w, b, rows, g_a)
+    H.check_linear(y, Y, S, rows, f"full cfg={cfg} fmt={fmt} M={M} K={K} N={N}")
+
+
+# ------------------------------------------------------------------ bounded waits
+def test_bounded_wait_reports_timeout(fb, orc):
+    """A k-stage that is never filled (test hook) makes the MMA warp's wait run out; the
+    kernel returns, the status word reads FP4_ERR_TIMEOUT, and the next call is correct."""
+    import torch
+
+    M, K, N = 128, 512, 256
+    x = synth.activation(11, M, K, "lognormal")
+    w = synth.weight(12, N, K)
+    xd, pw = H.dev_bf16(x), fb.pack_weight(H.dev_bf16(w), MX)
+    assert fb.fp4_sync_status() == 0
+    L = fb.lib()
+    try:
+        fb.fp4_set_wait_timeout_ns(2_000_000)  # 2 ms
+        L.fp4bsa_test_skip_iteration(1)
+        fb.linear(xd, pw)
+        st = fb.fp4_sync_status()
+    finally:
+        L.fp4bsa_test_skip_iteration(-1)
+        fb.fp4_set_wait_timeout_ns(0)
+    assert fb.fp4_status_string(st) == "FP4_ERR_TIMEOUT"
+    y = fb.linear(xd, pw)
+    assert fb.fp4_sync_status() == 0
+    torch.cuda.synchronize()
+    Y, S = orc.fp4_linear_rows(MX, x, w, None, np.arange(M))
+    H.check_linear(y, Y, S, np.arange(M), "after timeout")

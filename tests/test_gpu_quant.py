@@ -1,0 +1,214 @@
+"""GPU parity of the quantization kernels against the CPU oracle (bit-exact).
+
+Codes and the whole scale-factor buffer (padding rows included) must match the
+oracle byte for byte; the NVFP4 weight global must match bit for bit.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+MX, NV = oracle.MX, oracle.NV
+
+
+@pytest.fixture(scope="module")
+def fb():
+    import fp4_block_scaled_act_b200 as fb
+
+    fb.build()
+    return fb
+
+
+def _quant_dev(fb, fmt, x_bits, g=None):
+    import torch
+
+    x = H.dev_bf16(x_bits)
+    ga = H.dev_f32([g]) if fmt == NV else None
+    codes, sf = fb.quantize_act(x, fmt, ga)
+    torch.cuda.synchronize()
+    return H.host_u8(codes), H.host_u8(sf)
+
+
+def _assert_quant(fb, orc, fmt, x_bits, g=None):
+    c_ref, s_ref = orc.quantize(fmt, x_bits, g)
+    c, s = _quant_dev(fb, fmt, x_bits, g)
+    assert c.shape == c_ref.shape and s.shape == s_ref.shape
+    if not np.array_equal(c, c_ref):
+        i = np.argwhere(c != c_ref)[0]
+        raise AssertionError(f"codes differ at {tuple(i)}: gpu {c[tuple(i)]:#04x} oracle {c_ref[tuple(i)]:#04x}")
+    if not np.array_equal(s, s_ref):
+        i = int(np.argwhere(s != s_ref)[0][0])
+        raise AssertionError(f"scale byte {i} differs: gpu {s[i]:#04x} oracle {s_ref[i]:#04x}")
+
+
+# ------------------------------------------------------------------ converter sweeps
+def test_e2m1_conversion_sweep(fb, orc):
+    """Every finite bf16 value in (-8, 8) through the device E2M1 path, scale fixed at 1.
+
+    Each 32-group holds a 6.0 so the MX scale is 2^0 and the codes are e2m1(x) itself."""
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = synth.bf16_bits_to_f32(allbits)
+    keep = np.isfinite(vals) & (np.abs(vals) < 8.0)
+    xs = allbits[keep]
+    n_per_group = 31
+    groups = -(-xs.size // n_per_group)
+    pad = np.zeros(groups * n_per_group, dtype=np.uint16)
+    pad[: xs.size] = xs
+    body = pad.reshape(groups, n_per_group)
+    six = np.full((groups, 1), synth.f32_to_bf16_bits(np.float32(6.0)), dtype=np.uint16)
+    flat = np.concatenate([six, body], axis=1).reshape(-1)
+    K = 512
+    rows = -(-flat.size // K)
+    x = np.zeros(rows * K, dtype=np.uint16)
+    x[: flat.size] = flat
+    _assert_quant(fb, orc, MX, x.reshape(rows, K))
+
+
+def test_e4m3_conversion_sweep(fb, orc):
+    """Every finite bf16 value in (-512, 512) through the device E4M3 path (MXFP8 with a
+    300.0 in each group, so the scale is 2^0 and the elements are e4m3(x))."""
+    import torch
+
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = synth.bf16_bits_to_f32(allbits)
+    xs = allbits[np.isfinite(vals) & (np.abs(vals) < 512.0)]
+    n_per_group = 31
+    groups = -(-xs.size // n_per_group)
+    pad = np.zeros(groups * n_per_group, dtype=np.uint16)
+    pad[: xs.size] = xs
+    big = np.full((groups, 1), synth.f32_to_bf16_bits(np.float32(300.0)), dtype=np.uint16)
+    flat = np.concatenate([big, pad.reshape(groups, n_per_group)], axis=1).reshape(-1)
+    K = 512
+    rows = -(-flat.size // K)
+    x = np.zeros(rows * K, dtype=np.uint16)
+    x[: flat.size] = flat
+    x = x.reshape(rows, K)
+    e_ref, s_ref = orc.quantize_mxfp8(x)
+    l1 = torch.zeros((K, 32), dtype=torch.bfloat16, device="cuda")
+    xe = torch.empty((rows, K), dtype=torch.uint8, device="cuda")
+    xs_ = torch.empty(fb.fp4_sf_bytes(MX, rows, K), dtype=torch.uint8, device="cuda")
+    u = torch.empty((rows, 32), dtype=torch.float32, device="cuda")
+    fb.w4a8_quantize_act(H.dev_bf16(x), rows, K, l1, 32, xe, xs_, u)
+    torch.cuda.synchronize()
+    e = H.host_u8(xe)
+    if not np.array_equal(e, e_ref):
+        i = np.argwhere(e != e_ref)[0]
+        raise AssertionError(f"e4m3 differs at {tuple(i)}: input {synth.bf16_bits_to_f32(x[tuple(i)])!r} "
+                             f"gpu {e[tuple(i)]:#04x} oracle {e_ref[tuple(i)]:#04x}")
+    np.testing.assert_array_equal(H.host_u8(xs_), s_ref)
+
+
+# ------------------------------------------------------------------ shapes and formats
+SHAPES = [(1, 128), (7, 256), (128, 512), (129, 384), (256, 512), (300, 640), (1000, 1280)]
+
+
+@pytest.mark.parametrize("M,K", SHAPES)
+def test_mxfp4_quant(fb, orc, M, K):
+    x = synth.activation(100 + M, M, K, "lognormal")
+    _assert_quant(fb, orc, MX, x)
+
+
+@pytest.mark.parametrize("M,K", SHAPES)
+def test_nvfp4_quant(fb, orc, M, K):
+    x = synth.activation(200 + M, M, K, "lognormal")
+    cal = synth.activation(300 + M, 256, K, "lognormal")
+    g = orc.nv_global(orc.tensor_amax(cal))     # static global from a different batch
+    _assert_quant(fb, orc, NV, x, g)
+
+
+@pytest.mark.parametrize("M,K", [(1, 128), (130, 256), (4290 // 10, 3072)])
+def test_mxfp8_quant_and_lowrank(fb, orc, M, K):
+    import torch
+
+    x = synth.activation(400 + M, M, K, "lognormal")
+    f = synth.svdquant_factors(500 + K, 256, K, calib_tokens=256)
+    e_ref, s_ref = orc.quantize_mxfp8(x)
+    xe = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    xs = torch.empty(fb.fp4_sf_bytes(MX, M, K), dtype=torch.uint8, device="cuda")
+    u = torch.empty((M, 32), dtype=torch.float32, device="cuda")
+    fb.w4a8_quantize_act(H.dev_bf16(x), M, K, H.dev_bf16(f["l1_bf16"]), 32, xe, xs, u)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(H.host_u8(xe), e_ref)
+    np.testing.assert_array_equal(H.host_u8(xs), s_ref)
+    # u = x L1 in fp32 against fp64: within fp32 accumulation error of sum_k |x_k l1_k|
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    l1 = synth.bf16_bits_to_f32(f["l1_bf16"]).astype(np.float64)
+    u_ref = xf @ l1
+    mag = np.abs(xf) @ np.abs(l1)
+    err = np.abs(u.cpu().numpy().astype(np.float64) - u_ref)
+    assert np.all(err <= 4 * K * 2.0 ** -24 * mag + 1e-30)
+
+
+def test_edge_values(fb, orc):
+    """Zeros, negative zeros, huge and tiny magnitudes, and mixed-sign groups."""
+    K = 256
+    rows = []
+    rows.append(np.zeros(K, dtype=np.float32))
+    rows.append(np.full(K, -0.0, dtype=np.float32))
+    rows.append(np.linspace(-3e38, 3e38, K).astype(np.float32))
+    rows.append((np.linspace(-1, 1, K) * 1e-38).astype(np.float32))
+    r = np.zeros(K, dtype=np.float32)
+    r[::2] = 1e-30
+    r[1::2] = -7.0
+    rows.append(r)
+    rows.append(np.where(np.arange(K) % 17 == 0, 1e4, -1e-4).astype(np.float32))
+    x = synth.f32_to_bf16_bits(np.stack(rows))
+    _assert_quant(fb, orc, MX, x)
+    for T in (2688.0, 1.0, 1e-3, 3e38):
+        _assert_quant(fb, orc, NV, x, orc.nv_global(T))
+
+
+# ------------------------------------------------------------------ amax and weight pack
+def test_tensor_amax(fb, orc):
+    import torch
+
+    for n, seed in ((1, 1), (7, 2), (4096, 3), (1_000_003, 4)):
+        x = synth.activation(seed, 1, n, "lognormal")
+        xd = H.dev_bf16(x.reshape(-1))
+        out = torch.empty(1, dtype=torch.float32, device="cuda")
+        fb.fp4_tensor_amax(xd, n, out)
+        torch.cuda.synchronize()
+        assert out.item() == orc.tensor_amax(x)
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("N,K", [(128, 128), (384, 512), (512, 512)])
+def test_pack_weight(fb, orc, fmt, N, K):
+    import torch
+
+    w = synth.weight(600 + N + K, N, K)
+    c_ref, s_ref, g_ref = orc.pack_weight(fmt, w)
+    pw = fb.pack_weight(H.dev_bf16(w), fmt)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(H.host_u8(pw.codes), c_ref)
+    np.testing.assert_array_equal(H.host_u8(pw.sf), s_ref)
+    if fmt == NV:
+        assert np.float32(pw.w_global.item()) == np.float32(g_ref)
+
+
+def test_quant_determinism(fb):
+    import torch
+
+    x = H.dev_bf16(synth.activation(7, 513, 1024, "lognormal"))
+    a = fb.quantize_act(x, MX)
+    b = fb.quantize_act(x, MX)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+# ------------------------------------------------------------------ full size (the bench workload)
+@pytest.mark.parametrize("fmt", [MX, NV])
+def test_full_size_quant(fb, orc, fmt):
+    """M = 75600 tokens, K = 5120: every code and scale byte, in the bench's launch shape."""
+    M, K = 75600, 5120
+    s = synth.seeds_for(2 if fmt == NV else 1)
+    x = synth.activation(s["x"], M, K, "lognormal", gain_seed=s["gain"])
+    g = None
+    if fmt == NV:
+        cal = synth.activation(s["calib"], synth.CALIB_TOKENS, K, "lognormal", gain_seed=s["gain"])
+        g = orc.nv_global(orc.tensor_amax(cal))
+    _assert_quant(fb, orc, fmt, x, g)
