@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A4 block-scaled FP4 quantized linear on B200.
+
+Workload: the Wan2.2-A14B FFN up-projection in MXFP4, M = 75600 tokens (a 21x45x80
+latent grid), K = 5120, N = 13824; bf16 activations N(0,1) x per-channel lognormal
+gains, bf16 weights N(0, 0.02) packed offline, fp16 bias, bf16 output.  One step is
+one quantized linear: dynamic activation quantization + block-scaled GEMM with the
+fused bias epilogue (the weight pre-pack is offline and untimed).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line.  `value` is TFLOPS (2*M*K*N per step, all ranks together)
+with inputs resident in HBM; `e2e` is the same metric through fp4_linear with the
+input copied from pinned host memory and the output copied back every step.  With
+N > 1 (torchrun) every rank runs its own batch (weak scaling, no collective on the
+data path); time is the max over ranks.  `--impl reference` times the CPU oracle on
+a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, K, N = 75600, 5120, 13824
+FMT = "mxfp4"
+WORKLOAD = "wan22_a14b_ffn_up_mxfp4"
+METRIC = "FP4 W4A4 linear TFLOPS incl. act-quant (M=75600 K=5120 N=13824), % FP4 peak"
+FLOP_PER_STEP = 2.0 * M * K * N
+NOMINAL_FP4_TFLOPS = 9000.0
+FP4_PER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor ratio on B200 (9 / 2.25 PFLOP/s)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--m", type=int, default=75600,
+                    help="tokens; smaller values run a reduced case of the same kernels (profiling only)")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=2)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if ts < t0 - 0.05 or ts > t1 + 0.1:
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ----------------------------------------------------------------------------- inputs
+def make_inputs(rank: int):
+    import synth
+
+    s = synth.seeds_for(4, layer=1)
+    x = synth.activation(s["x"] + 7919 * rank, M, K, "lognormal", gain_seed=s["gain"])
+    w = synth.weight(s["w"], N, K)
+    b = synth.bias(s["bias"], N)
+    return x, w, b
+
+
+def to_dev(bits, torch, dt):
+    return torch.from_numpy(bits.view(np.int16)).view(dt).cuda()
+
+
+# ----------------------------------------------------------------------------- cpu baseline
+def cpu_baseline(x_bits, w_bits, b_bits, target_s: float = 15.0):
+    """The oracle, as it stands, on a bounded row sample of the same workload."""
+    import oracle
+
+    wc, ws, _ = oracle.pack_weight(oracle.MX, w_bits)          # offline step, untimed
+    w_deq = oracle.dequant_fp4(oracle.MX, wc, ws, K)            # once, untimed
+
+    def run(rows):
+        xs = np.ascontiguousarray(x_bits[rows])
+        c, sf = oracle.quantize(oracle.MX, xs)
+        a = oracle.dequant_fp4(oracle.MX, c, sf, K)
+        oracle.linear_fp64(a, w_deq, b_bits)
+
+    t = time.perf_counter()
+    run(np.arange(2))
+    per_row = max((time.perf_counter() - t) / 2, 1e-4)
+    nrows = int(max(2, min(512, target_s / per_row)))
+    rows = np.linspace(0, M - 1, nrows).astype(np.int64)
+    t = time.perf_counter()
+    run(rows)
+    dt = time.perf_counter() - t
+    return {"value": 2.0 * nrows * K * N / dt / 1e12, "unit": "TFLOPS", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{nrows} of {M} rows: MXFP4 quantize + dequantize + fp64 GEMM over full K={K}, N={N} "
+                      f"({dt:.1f} s); weight pack and dequantize excluded (offline)"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def reference_arm(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    import synth
+
+    oracle.build()
+    s = synth.seeds_for(4, layer=1)
+    w = synth.weight(s["w"], N, K)
+    b = synth.bias(s["bias"], N)
+    wc, ws, _ = oracle.pack_weight(oracle.MX, w)
+    w_deq = oracle.dequant_fp4(oracle.MX, wc, ws, K)
+    # one step = the quantized linear for a bounded row sample of the workload
+    total_steps = args.steps + args.warmup
+    probe = synth.activation(s["x"], 1, K, "lognormal", gain_seed=s["gain"])
+    t = time.perf_counter()
+    c, sf = oracle.quantize(oracle.MX, probe)
+    oracle.linear_fp64(oracle.dequant_fp4(oracle.MX, c, sf, K), w_deq, b)
+    per_row = time.perf_counter() - t
+    budget = 150.0
+    rows_per_step = int(max(1, min(64, budget / max(total_steps, 1) / max(per_row, 1e-4))))
+    x = synth.activation(s["x"], rows_per_step * 8, K, "lognormal", gain_seed=s["gain"])
+
+    def step(i):
+        r0 = (i * rows_per_step) % (x.shape[0] - rows_per_step + 1)
+        xs = np.ascontiguousarray(x[r0:r0 + rows_per_step])
+        c, sf = oracle.quantize(oracle.MX, xs)
+        oracle.linear_fp64(oracle.dequant_fp4(oracle.MX, c, sf, K), w_deq, b)
+
+    for i in range(args.warmup):
+        step(i)
+    t = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t
+    flops = 2.0 * rows_per_step * K * N * args.steps
+    value = flops / dt / 1e12
+    sample = (f"{rows_per_step} row(s) of the {M}x{K}x{N} workload per step: MXFP4 quantize + "
+              f"dequantize + fp64 GEMM (weight packed once, untimed)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / max(args.steps, 1) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "fmt": FMT},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- native arm
+def native_arm(args):
+    import torch
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    import fp4_block_scaled_act_b200 as fb
+
+    fb.lib()  # fails loudly if the CUDA library is missing
+    x_bits, w_bits, b_bits = make_inputs(rank)
+    x = to_dev(x_bits, torch, torch.bfloat16)
+    bias = to_dev(b_bits, torch, torch.float16)
+    pw = fb.pack_weight(to_dev(w_bits, torch, torch.bfloat16), FMT)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws_bytes = fb.fp4_linear_workspace_bytes(FMT, M, K, N)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    codes = ws[: fb.fp4_codes_bytes(FMT, M, K)]
+    sf_off = (codes.numel() + 255) // 256 * 256
+    sf = ws[sf_off: sf_off + fb.fp4_sf_bytes(FMT, M, K)]
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        # fp4_linear is exactly these two launches; calling them separately lets the
+        # events time each kernel on the launching stream
+        if ev is not None:
+            ev[0].record(stream)
+        fb.fp4_quantize_act(FMT, x, M, K, None, codes, sf)
+        if ev is not None:
+            ev[1].record(stream)
+        fb.fp4_gemm(FMT, codes, sf, M, K, N, pw.codes, pw.sf, None, None, bias, y)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = fb.fp4_sync_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {fb.fp4_status_string(st)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local])
+                          if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
+    clocks.start()
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    w0 = time.time()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    w1 = time.time()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop(w0, w1)
+    st = fb.fp4_sync_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {fb.fp4_status_string(st)}")
+    total_ms = t_start.elapsed_time(t_end)
+    q_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    g_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    if dist:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = t.item()
+    ms_per_step = total_ms / args.steps
+    value = FLOP_PER_STEP * world * args.steps / (total_ms / 1e3) / 1e12
+
+    # ---- end to end through the public API, host buffers (pinned), copies inside the timing
+    x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    x_e2e = torch.empty_like(x)
+
+    def e2e_step():
+        x_e2e.copy_(x_host, non_blocking=True)
+        fb.fp4_linear(FMT, x_e2e, M, K, N, pw.codes, pw.sf, None, None, bias, y, ws, ws_bytes)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    e2e_value = FLOP_PER_STEP * world * args.e2e_steps / (e2e_ms / 1e3) / 1e12
+
+    # ---- roofline of the dominant kernel (the GEMM), live CUDA-event durations
+    pk, pk_kind = peaks()
+    g_avg = sum(g_ms) / len(g_ms)
+    q_avg = sum(q_ms) / len(q_ms)
+    gemm_tflops = FLOP_PER_STEP / (g_avg / 1e3) / 1e12
+    fp4_peak = pk["bf16_tflops"] * FP4_PER_BF16
+    q_bytes = 2 * M * K + M * K // 2 + ((M + 127) // 128 * 128) * (K // 32)
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if os.path.exists(tr_path):
+        traffic = json.load(open(tr_path)).get("bytes_per_launch")
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp4", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "fmt": FMT, "tokens_per_gpu": M,
+                   "parallelism": f"dp{world} (independent batches)" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (X 774 MB, Y 2.09 GB), no flush"},
+        "pct_nominal_fp4_peak": 100.0 * value / world / NOMINAL_FP4_TFLOPS,
+        "roofline": {"bound": "tensor", "kernel": "gemm_kernel<MXFP4>", "achieved": gemm_tflops,
+                     "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
+                     "peak_source": f"{pk_kind} bf16 burst {pk['bf16_tflops']} x {FP4_PER_BF16:g} (nominal FP4/BF16)",
+                     "traffic": traffic,
+                     "algorithmic_flop_per_launch": FLOP_PER_STEP, "avg_launch_ms": g_avg},
+        "kernels": {"quant_ms": q_avg, "quant_gbs": q_bytes / (q_avg / 1e3) / 1e9,
+                    "quant_hbm_frac": q_bytes / (q_avg / 1e3) / 1e9 / pk["hbm_gbs"], "gemm_ms": g_avg},
+        "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": x_bits.nbytes,
+                "d2h_bytes_per_step": M * N * 2, "steps": args.e2e_steps},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x_bits, w_bits, b_bits)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    global M, WORKLOAD, FLOP_PER_STEP
+    args = parse()
+    if args.m != M:
+        M = args.m
+        WORKLOAD = f"ffn_up_mxfp4_m{M}"
+        FLOP_PER_STEP = 2.0 * M * K * N
+    if args.impl == "reference":
+        return reference_arm(args)
+    return native_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -276,8 +276,9 @@ fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const float* 
         return FP4_ERR_INVALID_ARG;
     fp4_status_t s = check_shape(M, K, N);
     if (s != FP4_OK) return s;
-    if (!aligned16(x_e4m3) || !aligned16(x_sf) || !aligned16(u_f32) || !aligned16(r_codes) || !aligned16(r_sf) ||
-        !aligned16(l2_bf16) || !aligned16(bias_f16) || !aligned16(y_bf16))
+    // the unpacking tensor map needs a 32-byte aligned residual-weight base
+    if (!aligned16(x_e4m3) || !aligned16(x_sf) || !aligned16(u_f32) || (reinterpret_cast<uintptr_t>(r_codes) & 31u) ||
+        !aligned16(r_sf) || !aligned16(l2_bf16) || !aligned16(bias_f16) || !aligned16(y_bf16))
         return FP4_ERR_MISALIGNED;
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;

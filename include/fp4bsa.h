@@ -159,7 +159,8 @@ fp4_status_t w4a8_quantize_act(const void* x_bf16, int64_t M, int64_t K, const v
                                void* stream);
 
 /* W4A8 GEMM with low-rank epilogue: y = bf16_rn( sum_k deq8(x) deq4(r) + u L2 + bias ).
- *   r_codes, r_sf  (device) MXFP4-packed residual weight [N, K] (fp4_pack_weight)
+ *   r_codes, r_sf  (device) MXFP4-packed residual weight [N, K] (fp4_pack_weight);
+ *                  r_codes must be 32-byte aligned
  *   l2_bf16        (device) [rank, N] bf16
  * The low-rank product u L2 is evaluated with fp32 FMAs in the epilogue. */
 fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const float* u_f32, int64_t M,
