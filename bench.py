@@ -269,8 +269,8 @@ def native_arm(args):
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local])
-                          if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    clocks = ClockSampler(vis.split(",")[local].strip() if vis else str(local))
     clocks.start()
     time.sleep(0.3)
     if dist:
