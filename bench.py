@@ -137,6 +137,22 @@ def to_dev(bits, torch, dt):
     return torch.from_numpy(bits.view(np.int16)).view(dt).cuda()
 
 
+def gemm_traffic():
+    """DRAM bytes per launch of the GEMM from the committed ncu summary, or None when the
+    kernel source changed since those counters were taken."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "gemm_mxfp4_ffn_up_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    fields = dict(l.split(":", 1) for l in open(path) if ":" in l)
+    src = b"".join(open(os.path.join(ROOT, "fp4_block_scaled_act_b200", "csrc", f), "rb").read()
+                   for f in ("gemm.cuh", "ptx.cuh"))
+    if hashlib.sha1(src).hexdigest()[:12] != fields.get("source_sha1", "").strip():
+        return None
+    return float(fields["bytes_per_launch"])
+
+
 # ----------------------------------------------------------------------------- cpu baseline
 def cpu_baseline(x_bits, w_bits, b_bits, target_s: float = 15.0):
     """The oracle, as it stands, on a bounded row sample of the same workload."""
@@ -334,10 +350,7 @@ def native_arm(args):
     gemm_tflops = FLOP_PER_STEP / (g_avg / 1e3) / 1e12
     fp4_peak = pk["bf16_tflops"] * FP4_PER_BF16
     q_bytes = 2 * M * K + M * K // 2 + ((M + 127) // 128 * 128) * (K // 32)
-    traffic = None
-    tr_path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
-    if os.path.exists(tr_path):
-        traffic = json.load(open(tr_path)).get("bytes_per_launch")
+    traffic = gemm_traffic()
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
