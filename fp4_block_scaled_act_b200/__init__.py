@@ -30,7 +30,7 @@ EXPORTS = [
     "fp4_codes_bytes", "fp4_sf_bytes", "fp4_linear_workspace_bytes", "w4a8_workspace_bytes",
     "fp4_tensor_amax", "fp4_pack_weight", "fp4_quantize_act", "fp4_gemm", "fp4_linear",
     "w4a8_quantize_act", "w4a8_gemm", "w4a8_svd_linear", "fp4_sync_status", "fp4_status_string",
-    "fp4_set_wait_timeout_ns",
+    "fp4_set_wait_timeout_ns", "fp4_linear_noalloc",
 ]
 
 
@@ -62,6 +62,7 @@ def lib():
             "fp4_quantize_act": (I, [I, P, I64, I64, P, P, P, P]),
             "fp4_gemm": (I, [I, P, P, I64, I64, I64, P, P, P, P, P, P, P]),
             "fp4_linear": (I, [I, P, I64, I64, I64, P, P, P, P, P, P, P, SZ, P]),
+            "fp4_linear_noalloc": (I, [I, P, I64, I64, I64, P, P, P, P, P, P, P]),
             "w4a8_quantize_act": (I, [P, I64, I64, P, I, P, P, P, P]),
             "w4a8_gemm": (I, [P, P, P, I64, I64, I64, P, P, P, I, P, P, P]),
             "w4a8_svd_linear": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, P, SZ, P]),
@@ -150,6 +151,14 @@ def fp4_linear(fmt, x, M: int, K: int, N: int, w_codes, w_sf, w_global, a_global
     _check(lib().fp4_linear(_fmt(fmt), _ptr(x), M, K, N, _ptr(w_codes), _ptr(w_sf), _ptr(w_global),
                             _ptr(a_global), _ptr(bias), _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
            "fp4_linear")
+
+
+def fp4_linear_noalloc(fmt, x, M: int, K: int, N: int, w_codes, w_sf, w_global, a_global, bias, y,
+                       stream=None):
+    """fp4_linear without a workspace argument, for callers that cannot allocate device
+    memory: the quantized activations use the library's built-in 16 MiB device array."""
+    _check(lib().fp4_linear_noalloc(_fmt(fmt), _ptr(x), M, K, N, _ptr(w_codes), _ptr(w_sf), _ptr(w_global),
+                                    _ptr(a_global), _ptr(bias), _ptr(y), _stream(stream)), "fp4_linear_noalloc")
 
 
 def w4a8_quantize_act(x, M: int, K: int, l1, rank: int, x_e4m3, x_sf, u, stream=None):

@@ -341,6 +341,49 @@ const char* fp4_status_string(fp4_status_t status) {
 
 void fp4_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTimeoutNs; }
 
+// ---------------------------------------------------------------------------------------
+// Allocation-free variant of fp4_linear.  Some callers cannot call cudaMalloc: code that
+// runs inside another framework's memory pool or a plugin whose host forbids device
+// allocations, or a real-time loop where an allocation could block.  For them the
+// quantized activations live in this library's own device array instead of a
+// caller-provided workspace.  The array is FP4_NOALLOC_SCRATCH_BYTES on every GPU that
+// loads the library, for the life of the process; all calls share it, so calls that
+// overlap on the GPU (different streams, or different host threads on one device) race.
+// Nothing in it needs clearing: the quantizer rewrites every byte the GEMM reads.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FP4_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {};
+}  // namespace
+
+fp4_status_t fp4_linear_noalloc(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K, int64_t N,
+                                const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
+                                const float* a_global, const void* bias_f16, void* y_bf16, void* stream) {
+    if (!fmt_ok(fmt)) return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, N);
+    if (s != FP4_OK) return s;
+    if (fp4_linear_workspace_bytes(fmt, M, K, N) > (size_t)FP4_NOALLOC_SCRATCH_BYTES) return FP4_ERR_WORKSPACE;
+    DeviceState* ds;
+    if ((s = device_state(&ds)) != FP4_OK) return s;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP4_ERR_CUDA;
+    void* scratch = nullptr;
+    {
+        // once per device, with that device current: the array's name is only a host-side
+        // stand-in, so its device address has to be looked up
+        std::lock_guard<std::mutex> lock(g_scratch_mu);
+        if (!g_scratch_addr[dev]) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return FP4_ERR_CUDA;
+            g_scratch_addr[dev] = p;
+        }
+        scratch = g_scratch_addr[dev];
+    }
+    return fp4_linear(fmt, x_bf16, M, K, N, w_codes, w_sf, w_global, a_global, bias_f16, y_bf16, scratch,
+                      (size_t)FP4_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 // Test hook (not in the public header): the GEMM producer skips the given k-iteration of
 // its ring, so the MMA warp's bounded wait runs out.  -1 disables it.
 void fp4bsa_test_skip_iteration(int it) { g_skip_iter = it; }

@@ -144,6 +144,30 @@ fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K,
                         const float* a_global, const void* bias_f16, void* y_bf16,
                         void* workspace, size_t ws_bytes, void* stream);
 
+/* Size of the device array fp4_linear_noalloc uses in place of a workspace. */
+#define FP4_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* fp4_linear for callers that cannot allocate device memory (a plugin whose host owns
+ * every allocation, code running under another framework's memory pool, a real-time
+ * loop that must not block in an allocator).  The paper has no counterpart: this is a
+ * packaging variant of fp4_linear, not part of the method.
+ *   Same arguments and result as fp4_linear, minus the workspace: the quantized
+ *   activations go to a library-owned device array of FP4_NOALLOC_SCRATCH_BYTES
+ *   (16 MiB) that exists on every GPU that loads the library until the process exits.
+ *   The call allocates nothing (no cudaMalloc/cudaFree, no allocating library routine).
+ *   The first call on a device looks up that array's device address (with the device
+ *   current); make that first call before any stream capture.
+ *   Returns FP4_ERR_WORKSPACE, launching nothing, when
+ *   fp4_linear_workspace_bytes(fmt, M, K, N) exceeds FP4_NOALLOC_SCRATCH_BYTES
+ *   (e.g. MXFP4 with K = 5120 fits up to 6168 rows).
+ *   Every call shares the one array, and it keeps the last call's contents: calls that
+ *   overlap on the GPU (other streams, other host threads on the same device) race and
+ *   must be serialized by the caller.  No part of the array needs clearing between calls. */
+fp4_status_t fp4_linear_noalloc(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K, int64_t N,
+                                const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
+                                const float* a_global, const void* bias_f16, void* y_bf16,
+                                void* stream);
+
 /* ----------------------------------------------------------------- W4A8 SVDQuant */
 
 /* Activation side of the W4A8 SVDQuant linear (W4A8 README: "dynamic MXFP8
