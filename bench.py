@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm-ctas", type=int, default=0, choices=[0, 1, 2],
+                    help="GEMM kernel: 0/1 the 1-CTA 128x256 tile (default), 2 the 2-CTA 256x256 tile")
     ap.add_argument("--m", type=int, default=75600,
                     help="tokens; smaller values run a reduced case of the same kernels (profiling only)")
     return ap.parse_args()
@@ -137,12 +139,13 @@ def to_dev(bits, torch, dt):
     return torch.from_numpy(bits.view(np.int16)).view(dt).cuda()
 
 
-def gemm_traffic():
-    """DRAM bytes per launch of the GEMM from the committed ncu summary, or None when the
-    kernel source changed since those counters were taken."""
+def gemm_traffic(pair: bool):
+    """DRAM bytes per launch of the timed GEMM kernel from the committed ncu summary, or
+    None when the kernel source changed since those counters were taken."""
     import hashlib
 
-    path = os.path.join(ROOT, "profiles", "gemm_mxfp4_ffn_up_traffic.txt")
+    name = "gemm2_mxfp4_ffn_up_traffic.txt" if pair else "gemm_mxfp4_ffn_up_traffic.txt"
+    path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
         return None
     fields = dict(l.split(":", 1) for l in open(path) if ":" in l)
@@ -253,6 +256,8 @@ def native_arm(args):
     import fp4_block_scaled_act_b200 as fb
 
     fb.lib()  # fails loudly if the CUDA library is missing
+    fb.lib().fp4bsa_set_gemm_ctas(args.gemm_ctas)
+    pair = args.gemm_ctas == 2 and M > 128
     x_bits, w_bits, b_bits = make_inputs(rank)
     x = to_dev(x_bits, torch, torch.bfloat16)
     bias = to_dev(b_bits, torch, torch.float16)
@@ -350,7 +355,7 @@ def native_arm(args):
     gemm_tflops = FLOP_PER_STEP / (g_avg / 1e3) / 1e12
     fp4_peak = pk["bf16_tflops"] * FP4_PER_BF16
     q_bytes = 2 * M * K + M * K // 2 + ((M + 127) // 128 * 128) * (K // 32)
-    traffic = gemm_traffic()
+    traffic = gemm_traffic(pair)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
@@ -360,7 +365,8 @@ def native_arm(args):
                    "parallelism": f"dp{world} (independent batches)" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (X 774 MB, Y 2.09 GB), no flush"},
         "pct_nominal_fp4_peak": 100.0 * value / world / NOMINAL_FP4_TFLOPS,
-        "roofline": {"bound": "tensor", "kernel": "gemm_kernel<MXFP4>", "achieved": gemm_tflops,
+        "roofline": {"bound": "tensor", "kernel": "gemm2_kernel<MXFP4> (2-CTA 256x256)" if pair
+                     else "gemm_kernel<MXFP4> (1-CTA 128x256)", "achieved": gemm_tflops,
                      "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
                      "peak_source": f"{pk_kind} bf16 burst {pk['bf16_tflops']} x {FP4_PER_BF16:g} (nominal FP4/BF16)",
                      "traffic": traffic,

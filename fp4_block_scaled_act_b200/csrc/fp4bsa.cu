@@ -19,6 +19,7 @@ namespace {
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 uint64_t g_timeout_ns = kDefaultTimeoutNs;
 int g_skip_iter = -1;  // test hook, see fp4bsa_test_skip_iteration
+int g_gemm_ctas = 0;   // tuning hook: 0 auto (the 1-CTA kernel, fastest measured), 1 or 2 to force
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -28,8 +29,24 @@ struct DeviceState {
     bool ready = false;
     bool arch_ok = false;
     int sm_count = 0;
+    int pairs[3] = {0, 0, 0};  // co-resident CTA pairs of gemm2_kernel<kind>
+    int quant_occ[3] = {1, 1, 1};  // resident CTAs per SM of quant_kernel<kind>
     int* status = nullptr;
 };
+
+template <int KIND>
+int max_pairs(int sm_count) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sm_count & ~1);
+    cfg.blockDim = dim3(Gemm2Cfg<KIND>::THREADS);
+    cfg.dynamicSmemBytes = Gemm2Cfg<KIND>::SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void*)gemm2_kernel<KIND>, &cfg) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = sm_count / 2;
+    }
+    return n;
+}
 
 std::mutex g_mu;
 DeviceState g_dev[64];
@@ -55,8 +72,24 @@ fp4_status_t device_state(DeviceState** out) {
                 cudaFuncSetAttribute(gemm_kernel<G_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      GemmCfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm_kernel<G_W4A8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     GemmCfg<G_W4A8>::SMEM_BYTES) != cudaSuccess)
+                                     GemmCfg<G_W4A8>::SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm2_kernel<G_MXFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Gemm2Cfg<G_MXFP4>::SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm2_kernel<G_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Gemm2Cfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm2_kernel<G_W4A8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Gemm2Cfg<G_W4A8>::SMEM_BYTES) != cudaSuccess)
                 return FP4_ERR_CUDA;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.quant_occ[Q_MXFP4], quant_kernel<Q_MXFP4>,
+                                                              QUANT_THREADS, 0) != cudaSuccess ||
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.quant_occ[Q_NVFP4], quant_kernel<Q_NVFP4>,
+                                                              QUANT_THREADS, 0) != cudaSuccess ||
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.quant_occ[Q_MXFP8], quant_kernel<Q_MXFP8>,
+                                                              QUANT_THREADS, 0) != cudaSuccess)
+                return FP4_ERR_CUDA;
+            s.pairs[G_MXFP4] = max_pairs<G_MXFP4>(s.sm_count);
+            s.pairs[G_NVFP4] = max_pairs<G_NVFP4>(s.sm_count);
+            s.pairs[G_W4A8] = max_pairs<G_W4A8>(s.sm_count);
         }
         if (!g_encode) {
             cudaDriverEntryPointQueryResult q;
@@ -83,23 +116,27 @@ fp4_status_t check_shape(int64_t M, int64_t K, int64_t N) {
     if (M < 1) return FP4_ERR_INVALID_ARG;
     if (K < 128 || K % 128 != 0 || N < 128 || N % 128 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
     if (M >= kMaxDim || K >= kMaxDim || N >= kMaxDim) return FP4_ERR_UNSUPPORTED_SHAPE;
+    // the quantizer numbers 128-element units with 32-bit indices
+    if ((M + 127) / 128 * 128 * (K / 128) >= ((int64_t)1 << 31)) return FP4_ERR_UNSUPPORTED_SHAPE;
     return FP4_OK;
 }
 
 fp4_status_t launched() { return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA; }
 
-int quant_blocks(const DeviceState* ds, int64_t M, int64_t K) {
+// One resident wave of quantize CTAs, each taking a contiguous range of 128-element units.
+int quant_blocks(const DeviceState* ds, int kind, int64_t M, int64_t K) {
     const int64_t Mpad = (M + 127) & ~int64_t(127);
-    const int64_t threads = Mpad * (K / 128) * 16;
-    int64_t blocks = (threads + (int64_t)QUANT_THREADS * QUANT_UNROLL - 1) / ((int64_t)QUANT_THREADS * QUANT_UNROLL);
-    const int64_t cap = (int64_t)ds->sm_count * 16;
+    const int64_t units = Mpad * (K / 128);
+    const int64_t span = (QUANT_THREADS / 16) * QUANT_UNROLL;
+    int64_t blocks = (units + span - 1) / span;
+    const int64_t cap = (int64_t)ds->sm_count * (ds->quant_occ[kind] > 0 ? ds->quant_occ[kind] : 1);
     if (blocks > cap) blocks = cap;
     return (int)(blocks < 1 ? 1 : blocks);
 }
 
 fp4_status_t launch_quant(const DeviceState* ds, int kind, const void* x, int64_t M, int64_t K, const float* g,
                           uint8_t* out, uint8_t* sf, cudaStream_t st) {
-    const int blocks = quant_blocks(ds, M, K);
+    const int blocks = quant_blocks(ds, kind, M, K);
     const uint4* xv = static_cast<const uint4*>(x);
     if (kind == Q_MXFP4)
         quant_kernel<Q_MXFP4><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
@@ -111,13 +148,14 @@ fp4_status_t launch_quant(const DeviceState* ds, int kind, const void* x, int64_
 }
 
 fp4_status_t encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t rows,
-                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                       CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     const cuuint64_t dims[2] = {inner, rows};
     const cuuint64_t strides[1] = {row_bytes};
     const cuuint32_t box[2] = {box_inner, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
 }
@@ -131,6 +169,31 @@ fp4_status_t launch_gemm(const DeviceState* ds, const CUtensorMap& ta, const CUt
     p.skip_iter = g_skip_iter;
     p.status = ds->status;
     gemm_kernel<KIND><<<grid, GEMM_THREADS, GemmCfg<KIND>::SMEM_BYTES, st>>>(ta, tb, p);
+    return launched();
+}
+
+// Scale-factor buffer seen by TMA as rows of 512-byte atoms (128 x u32), `atoms` per box.
+fp4_status_t encode_sf(CUtensorMap* m, const uint8_t* sf, int64_t rows, int64_t K, int group, int atoms) {
+    const uint64_t total_atoms = (uint64_t)((rows + 127) / 128) * (uint64_t)(K / (group * 4));
+    return encode_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, sf, 128, total_atoms, 512, 128, (uint32_t)atoms,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// 2-CTA GEMM: A box 128 rows, B box 128 rows (half of the 256-wide N tile) per CTA.
+template <int KIND>
+fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CUtensorMap& tb, const uint8_t* sfa,
+                          const uint8_t* sfb, GemmParams& p, cudaStream_t st) {
+    using C = Gemm2Cfg<KIND>;
+    CUtensorMap tsa, tsb;
+    fp4_status_t s;
+    if ((s = encode_sf(&tsa, sfa, p.M, p.K, C::G, C::ATOMS)) != FP4_OK) return s;
+    if ((s = encode_sf(&tsb, sfb, p.N, p.K, C::G, C::ATOMS)) != FP4_OK) return s;
+    const int tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
+    const int pairs = tiles < ds->pairs[KIND] ? tiles : ds->pairs[KIND];
+    p.timeout_ns = g_timeout_ns;
+    p.skip_iter = g_skip_iter;
+    p.status = ds->status;
+    gemm2_kernel<KIND><<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, p);
     return launched();
 }
 
@@ -222,15 +285,22 @@ fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf
         return FP4_ERR_MISALIGNED;
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;
+    // 1-CTA 128x256 tiles unless the 2-CTA 256x256 kernel is forced (tuning hook)
+    const bool pair = g_gemm_ctas == 2 && M > GEMM_BM;
     CUtensorMap ta, tb;
     if ((s = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 128, GEMM_BM)) != FP4_OK) return s;
-    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 128, GEMM_BN)) != FP4_OK) return s;
+    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 128, pair ? 128 : GEMM_BN)) !=
+        FP4_OK)
+        return s;
     GemmParams p{};
     p.M = (int)M, p.N = (int)N, p.K = (int)K;
     p.sfa = a_sf, p.sfb = w_sf, p.g_a = a_global, p.g_w = w_global;
     p.bias = static_cast<const __half*>(bias_f16);
     p.y = static_cast<__nv_bfloat16*>(y_bf16);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (pair)
+        return nv ? launch_gemm2<G_NVFP4>(ds, ta, tb, a_sf, w_sf, p, st)
+                  : launch_gemm2<G_MXFP4>(ds, ta, tb, a_sf, w_sf, p, st);
     return nv ? launch_gemm<G_NVFP4>(ds, ta, tb, p, st) : launch_gemm<G_MXFP4>(ds, ta, tb, p, st);
 }
 
@@ -282,10 +352,12 @@ fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const float* 
         return FP4_ERR_MISALIGNED;
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;
+    const bool pair = g_gemm_ctas == 2 && M > GEMM_BM;
     CUtensorMap ta, tb;
     if ((s = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_e4m3, K, M, K, 128, GEMM_BM)) != FP4_OK) return s;
     // packed E2M1 in global memory, unpacked to one 16-byte slot per 16 values in shared memory
-    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, r_codes, K, N, K / 2, 128, GEMM_BN)) != FP4_OK)
+    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, r_codes, K, N, K / 2, 128,
+                       pair ? 128 : GEMM_BN)) != FP4_OK)
         return s;
     GemmParams p{};
     p.M = (int)M, p.N = (int)N, p.K = (int)K;
@@ -294,6 +366,7 @@ fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const float* 
     p.y = static_cast<__nv_bfloat16*>(y_bf16);
     p.u = u_f32;
     p.l2 = static_cast<const __nv_bfloat16*>(l2_bf16);
+    if (pair) return launch_gemm2<G_W4A8>(ds, ta, tb, x_sf, r_sf, p, static_cast<cudaStream_t>(stream));
     return launch_gemm<G_W4A8>(ds, ta, tb, p, static_cast<cudaStream_t>(stream));
 }
 
@@ -383,6 +456,10 @@ fp4_status_t fp4_linear_noalloc(fp4_fmt_t fmt, const void* x_bf16, int64_t M, in
     return fp4_linear(fmt, x_bf16, M, K, N, w_codes, w_sf, w_global, a_global, bias_f16, y_bf16, scratch,
                       (size_t)FP4_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+// Tuning hook (not in the public header): 0 or 1 use the 1-CTA 128x256 kernel, 2 the
+// 2-CTA 256x256 kernel (for M > 128).
+void fp4bsa_set_gemm_ctas(int ctas) { g_gemm_ctas = (ctas == 1 || ctas == 2) ? ctas : 0; }
 
 // Test hook (not in the public header): the GEMM producer skips the given k-iteration of
 // its ring, so the MMA warp's bounded wait runs out.  -1 disables it.

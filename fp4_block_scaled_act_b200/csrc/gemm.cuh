@@ -77,6 +77,82 @@ FP4_DEV void gemm_fail(const GemmParams& p, volatile int* abort) {
     atomicCAS(p.status, 0, STATUS_TIMEOUT);
 }
 
+// Add the W4A8 low-rank term, scale, add bias, round to bf16 and store 128 columns of one
+// output row held in registers (acc[c][j] = column col0 + 32c + j).
+template <int KIND>
+FP4_DEV void epilogue_store(const GemmParams& p, uint32_t (&acc)[4][32], int row, int col0, float gs) {
+    if (row >= p.M || col0 >= p.N) return;
+    const int N = p.N;
+    if (KIND == G_W4A8) {
+        // acc += u[row, r] * L2[r, cols] for r = 0..31, one rank at a time (fp32 FMAs)
+        const float* urow = p.u + (size_t)row * 32;
+#pragma unroll 1
+        for (int r = 0; r < 32; ++r) {
+            const float ur = urow[r];
+            const __nv_bfloat16* l2r = p.l2 + (size_t)r * N + col0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                    const uint4 lv = *reinterpret_cast<const uint4*>(l2r + c * 32 + j);
+                    const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        acc[c][j + 2 * i] = __float_as_uint(
+                            __fmaf_rn(ur, __uint_as_float(lw[i] << 16), __uint_as_float(acc[c][j + 2 * i])));
+                        acc[c][j + 2 * i + 1] = __float_as_uint(__fmaf_rn(
+                            ur, __uint_as_float(lw[i] & 0xFFFF0000u), __uint_as_float(acc[c][j + 2 * i + 1])));
+                    }
+                }
+            }
+        }
+    }
+    __nv_bfloat16* yrow = p.y + (size_t)row * N + col0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+            const int col = col0 + c * 32 + j;
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(acc[c][j + i]) * gs;
+            if (p.bias) {
+                const uint4 bv = *reinterpret_cast<const uint4*>(p.bias + col);
+                const __half2* bh = reinterpret_cast<const __half2*>(&bv);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 bf = __half22float2(bh[i]);
+                    v[2 * i] += bf.x;
+                    v[2 * i + 1] += bf.y;
+                }
+            }
+            uint4 o;
+            uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+                ow[i] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(yrow + c * 32 + j) = o;
+        }
+    }
+}
+
+// Which TMEM scale atom and which byte of it MMA number k of a stage reads.
+template <int KIND>
+FP4_DEV void sf_select(int k, int& atom, int& sf_id) {
+    if (KIND == G_MXFP4) {  // 2 E8M0 scales (K = 64) per MMA: byte pair 0-1 or 2-3
+        atom = k >> 1;
+        sf_id = (k & 1) * 2;
+    } else if (KIND == G_NVFP4) {  // 4 E4M3 scales (K = 64) per MMA: the whole word
+        atom = k;
+        sf_id = 0;
+    } else {  // W4A8: 1 E8M0 scale (K = 32) per MMA
+        atom = 0;
+        sf_id = k;
+    }
+}
+
 template <int KIND>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
@@ -224,16 +300,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                     for (int k = 0; k < n_mma; ++k) {
                         // scale-factor selection: which atom (TMEM column group) and which byte
                         int atom, sf_id;
-                        if (KIND == G_MXFP4) {
-                            atom = k >> 1;
-                            sf_id = (k & 1) * 2;
-                        } else if (KIND == G_NVFP4) {
-                            atom = k;
-                            sf_id = 0;
-                        } else {
-                            atom = 0;
-                            sf_id = k;
-                        }
+                        sf_select<KIND>(k, atom, sf_id);
                         const uint32_t idesc = C::IDESC | ((uint32_t)sf_id << 29) | ((uint32_t)sf_id << 4);
                         const uint64_t adesc = smem_desc(a_base + k * 32, 0, 1024, 2);
                         const uint64_t bdesc = smem_desc(b_base + k * 32, 0, 1024, 2);
@@ -283,60 +350,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(tmem_empty);
 
-            const int row = mb * GEMM_BM + q * 32 + lane;
-            const int col0 = nb * GEMM_BN + h * 128;
-            if (row < M && col0 < N) {
-                float ur[32];
-                if (KIND == G_W4A8) {
-                    const float4* up = reinterpret_cast<const float4*>(p.u + (size_t)row * 32);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 t = up[i];
-                        ur[4 * i] = t.x, ur[4 * i + 1] = t.y, ur[4 * i + 2] = t.z, ur[4 * i + 3] = t.w;
-                    }
-                }
-                __nv_bfloat16* yrow = p.y + (size_t)row * N + col0;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        const int col = col0 + c * 32 + j;
-                        float v[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(acc[c][j + i]) * gs;
-                        if (KIND == G_W4A8) {
-#pragma unroll
-                            for (int r = 0; r < 32; ++r) {
-                                const uint4 lv = *reinterpret_cast<const uint4*>(p.l2 + (size_t)r * N + col);
-                                const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    v[2 * i] = __fmaf_rn(ur[r], __uint_as_float(lw[i] << 16), v[2 * i]);
-                                    v[2 * i + 1] = __fmaf_rn(ur[r], __uint_as_float(lw[i] & 0xFFFF0000u), v[2 * i + 1]);
-                                }
-                            }
-                        }
-                        if (p.bias) {
-                            const uint4 bv = *reinterpret_cast<const uint4*>(p.bias + col);
-                            const __half2* bh = reinterpret_cast<const __half2*>(&bv);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const float2 bf = __half22float2(bh[i]);
-                                v[2 * i] += bf.x;
-                                v[2 * i + 1] += bf.y;
-                            }
-                        }
-                        uint4 o;
-                        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-                            ow[i] = *reinterpret_cast<uint32_t*>(&b2);
-                        }
-                        *reinterpret_cast<uint4*>(yrow + c * 32 + j) = o;
-                    }
-                }
-            }
+            epilogue_store<KIND>(p, acc, mb * GEMM_BM + q * 32 + lane, nb * GEMM_BN + h * 128, gs);
         }
     }
 
@@ -345,6 +359,380 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
+    }
+}
+
+// =======================================================================================
+// 2-CTA variant (cta_group::2): a cluster of two CTAs on an SM pair computes a 256 x 256
+// tile with M = 256 MMAs issued by the pair leader (CTA rank 0).  Each CTA loads its own
+// 128 rows of A and 128 of the 256 B rows; the tensor core combines both halves of B.
+// Per SM that is 256 operand rows per K stage instead of 384 for a 1-CTA 128 x 256 tile.
+//
+// Scale factors.  The MMA reads, in each 32-lane TMEM sub-partition, the scales of that
+// sub-partition's rows, so every 512-byte scale atom has to be present in all four
+// sub-partitions.  Copying it with the multicast shape (32x128b.warpx4) costs the tensor
+// pipe several times more than a plain 128x256b copy of the same TMEM bytes.  Here an
+// expander warp writes each atom four times into shared memory (one copy per 32-lane
+// quarter), so the MMA thread moves two atoms per 128x256b copy: 3 copies per K stage
+// for MXFP4 instead of 6 multicast ones.  Both CTAs hold the scales of all 256 B rows.
+//
+// Accumulators.  Two 256-column accumulators overlap by 64 columns ([0,256) and
+// [192,448)), leaving [448,512) for the scale columns.  The epilogue drains the overlap
+// chunk first and releases it, so the next tile's MMAs start after a 64-column drain.
+//
+// Synchronization.
+//   full[s]      (leader)  A/B bytes of both CTAs; the leader alone expects them
+//   sf_full[s]   (local)   this CTA's raw scale atoms
+//   empty[s]     (both)    the leader's commit (MMAs and scale copies of stage s done)
+//   sf_ready[x]  (leader)  expanded scales of both CTAs in slot x
+//   tmem_full[b] (both)    accumulator b complete
+//   acc_free[b]  (leader)  accumulator b fully drained by both CTAs (16 warps)
+//   ovl_free     (leader)  overlap chunk of the last tile drained (8 warps)
+// =======================================================================================
+template <int KIND>
+struct Gemm2Cfg {
+    using C1 = GemmCfg<KIND>;
+    static constexpr int BK = C1::BK, G = C1::G, MMA_K = C1::MMA_K, ATOMS = C1::ATOMS;
+    static constexpr int A_BYTES = 128 * 128;
+    static constexpr int B_BYTES = 128 * 128;  // this CTA's half of the 256 B rows
+    static constexpr int RSFA_BYTES = ATOMS * 512;        // raw atoms, this CTA's 128 A rows
+    static constexpr int RSFB_BYTES = 2 * ATOMS * 512;    // raw atoms, all 256 B rows
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RSFA_BYTES + RSFB_BYTES;
+    static constexpr int STAGES = (KIND == G_NVFP4) ? 4 : (KIND == G_W4A8 ? 6 : 5);
+    // expanded scales: every atom replicated 4x (2 KB); a 128x256b copy takes two of them
+    static constexpr int XSFA_BYTES = ATOMS * 2048;       // atom pairs (2a, 2a+1) per 4 KB
+    static constexpr int XSFB_BYTES = ATOMS * 4096;       // per atom: row block 0 | row block 1
+    static constexpr int XSF_BYTES = XSFA_BYTES + XSFB_BYTES;
+    static constexpr int XBUFS = (KIND == G_NVFP4) ? 2 : 3;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + XBUFS * XSF_BYTES + 512;
+    static constexpr uint32_t AB_TX = A_BYTES + ((KIND == G_W4A8) ? B_BYTES / 2 : B_BYTES);
+    static constexpr uint32_t SF_TX = RSFA_BYTES + RSFB_BYTES;
+    static constexpr int SF_COLS = ATOMS * 12;            // SFA 4/atom + SFB 8/atom
+    static constexpr int ACC1_COL = 192;                  // second accumulator: [192, 448)
+    static constexpr int SF_COL0 = 448;
+    static constexpr int SF_TBUFS = (64 / SF_COLS) >= 2 ? 2 : 1;
+    static constexpr int THREADS = 352;
+    static constexpr uint32_t IDESC = (C1::A_FMT << 7) | (C1::B_FMT << 10) | ((uint32_t)(256 >> 3) << 17) |
+                                      (C1::SCALE_FMT << 23) | ((uint32_t)(256 >> 4) << 24);
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert(SF_COL0 + SF_TBUFS * SF_COLS <= GEMM_TMEM_COLS, "TMEM budget");
+};
+
+FP4_DEV void gemm2_fail(const GemmParams& p, volatile int* abort, uint32_t peer_abort) {
+    *abort = 1;
+    st_cluster_u32(peer_abort, 1u);
+    atomicCAS(p.status, 0, STATUS_TIMEOUT);
+}
+
+// Arrive on a barrier of the pair leader: a local arrive in the leader, a remote relaxed
+// arrive in the follower (used after TMEM reads that tcgen05.wait::ld has completed).
+FP4_DEV void arrive_leader_relaxed(uint64_t* bar, uint32_t rank) {
+    if (rank == 0)
+        mbar_arrive(bar);
+    else
+        mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(bar), 0));
+}
+
+template <int KIND>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THREADS, 1)
+    gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB, GemmParams p) {
+    using C = Gemm2Cfg<KIND>;
+    constexpr int S = C::STAGES;
+    constexpr int X = C::XBUFS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + S * C::A_BYTES;
+    uint8_t* sRSFA = sB + S * C::B_BYTES;
+    uint8_t* sRSFB = sRSFA + S * C::RSFA_BYTES;
+    uint8_t* sXSF = sRSFB + S * C::RSFB_BYTES;           // X slots of XSF_BYTES
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sXSF + X * C::XSF_BYTES);
+    uint64_t* full = bars;
+    uint64_t* sf_full = full + S;
+    uint64_t* empty = sf_full + S;
+    uint64_t* sf_ready = empty + S;
+    uint64_t* tmem_full = sf_ready + X;                   // [2]
+    uint64_t* acc_free = tmem_full + 2;                   // [2]
+    uint64_t* ovl_free = acc_free + 2;
+    uint64_t* mma_done = ovl_free + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const uint32_t peer_abort = mapa_shared(smem_u32((const void*)abort), rank ^ 1u);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&sf_full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int x = 0; x < X; ++x) mbar_init(&sf_ready[x], 2);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tmem_full[b], 1);
+            mbar_init(&acc_free[b], 16);
+        }
+        mbar_init(ovl_free, 8);
+        mbar_init(mma_done, 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmSFA);
+        prefetch_tmap(&tmSFB);
+    }
+    __syncwarp();
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_holder, GEMM_TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncwarp();  // the cluster barrier is .aligned: every warp converged
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const int M = p.M, N = p.N, K = p.K;
+    const int num_m = (M + 255) / 256;
+    const int num_n = (N + 255) / 256;
+    const int num_tiles = num_m * num_n;
+    const int num_kb = (K + C::BK - 1) / C::BK;
+    const int apr = K / (C::G * 4);  // scale atoms per 128-row block
+    const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+
+    if (warp == 0) {
+        // ============================================================ producer (both CTAs)
+        if (lane == 0) {
+            const uint64_t pol_a = policy_evict_normal();
+            const uint64_t pol_b = policy_evict_last();
+            int it = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+                const int mb = tile / num_n, nb = tile % num_n;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (uint32_t)(it / S) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, p.timeout_ns, abort)) {
+                        gemm2_fail(p, abort, peer_abort);
+                        ok = false;
+                        break;
+                    }
+                    if (it == p.skip_iter) continue;  // test hook: this stage is never filled
+                    // A/B of both CTAs land on the leader's barrier; only the leader expects them
+                    // (a remote arrive with release semantics would fence every stage)
+                    const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::AB_TX);
+                    mbar_arrive_expect_tx(&sf_full[s], C::SF_TX);
+                    const int ax = (KIND == G_W4A8) ? kb * C::BK : kb * (C::BK / 2);
+                    const int bx = (KIND == G_W4A8) ? kb * C::BK : kb * (C::BK / 2);
+                    tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, bar, ax, mb * 256 + (int)rank * 128, pol_a);
+                    tma_load_2d_pair(sB + s * C::B_BYTES, &tmB, bar, bx, nb * 256 + (int)rank * 128, pol_b);
+                    tma_load_2d(sRSFA + s * C::RSFA_BYTES, &tmSFA, &sf_full[s], 0,
+                                (mb * 2 + (int)rank) * apr + kb * C::ATOMS, pol_a);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+                        tma_load_2d(sRSFB + s * C::RSFB_BYTES + j * C::ATOMS * 512, &tmSFB, &sf_full[s], 0,
+                                    (nb * 2 + j) * apr + kb * C::ATOMS, pol_b);
+                }
+            }
+            // drain what this CTA issued: its scale loads, and (leader) both CTAs' A/B
+            for (int j = max(0, it - S); j < it; ++j) {
+                if (j == p.skip_iter) continue;
+                if (!mbar_wait_drain(&sf_full[j % S], (uint32_t)(j / S) & 1u, p.timeout_ns))
+                    gemm2_fail(p, abort, peer_abort);
+                if (rank == 0 && !mbar_wait_drain(&full[j % S], (uint32_t)(j / S) & 1u, p.timeout_ns))
+                    gemm2_fail(p, abort, peer_abort);
+            }
+        }
+    } else if (warp == 10) {
+        // ============================================================ scale expander (both CTAs)
+        int it = 0;
+        bool ok = true;
+        for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int s = it % S;
+                const int x = it % X;
+                bool got = mbar_wait(&sf_full[s], (uint32_t)(it / S) & 1u, p.timeout_ns, abort);
+                // slot x is free once the copies of iteration it - X (same slot) are done
+                if (got && it >= X)
+                    got = mbar_wait(&empty[(it - X) % S], (uint32_t)((it - X) / S) & 1u, p.timeout_ns, abort);
+                if (!__all_sync(0xffffffffu, got)) {
+                    if (lane == 0) gemm2_fail(p, abort, peer_abort);
+                    ok = false;
+                    break;
+                }
+                const uint4* rsfa = reinterpret_cast<const uint4*>(sRSFA + s * C::RSFA_BYTES);
+                const uint4* rsfb = reinterpret_cast<const uint4*>(sRSFB + s * C::RSFB_BYTES);
+                uint8_t* xsfa = sXSF + x * C::XSF_BYTES;
+                uint8_t* xsfb = xsfa + C::XSFA_BYTES;
+#pragma unroll
+                for (int a = 0; a < C::ATOMS; ++a) {
+                    // lane l moves 16 bytes of the atom: quarter q gets a full copy
+                    const uint4 v = rsfa[a * 32 + lane];
+                    uint8_t* dst = xsfa + (a >> 1) * 4096 + (a & 1) * 2048 + lane * 16;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(dst + q * 512) = v;
+                }
+#pragma unroll
+                for (int rb = 0; rb < 2; ++rb) {
+#pragma unroll
+                    for (int a = 0; a < C::ATOMS; ++a) {
+                        const uint4 v = rsfb[(rb * C::ATOMS + a) * 32 + lane];
+                        uint8_t* dst = xsfb + a * 4096 + rb * 2048 + lane * 16;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(dst + q * 512) = v;
+                    }
+                }
+                fence_proxy_async_smem();  // generic-proxy writes -> visible to tcgen05.cp
+                __syncwarp();
+                // relaxed: a release.cluster arrive would put a cluster-scope fence in every stage
+                // (measured: half the throughput).  The writes are this CTA's own shared memory,
+                // read only by this SM's tensor core, and the proxy fence above has made them
+                // visible to the async proxy before the arrive is issued.
+                if (lane == 0) {
+                    if (rank == 0)
+                        mbar_arrive(&sf_ready[x]);
+                    else
+                        mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&sf_ready[x]), 0));
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ============================================================ MMA issuer (leader)
+        if (rank == 0 && lane == 0) {
+            int it = 0, tcount = 0;
+            bool issued = false, ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++tcount) {
+                const int b = tcount & 1;
+                // accumulator b drained (tile tcount-2) and the overlap of tile tcount-1 drained
+                bool got = mbar_wait(&acc_free[b], (((uint32_t)tcount >> 1) & 1u) ^ 1u, p.timeout_ns, abort);
+                if (got && tcount > 0) got = mbar_wait(ovl_free, (uint32_t)(tcount - 1) & 1u, p.timeout_ns, abort);
+                if (!got) {
+                    gemm2_fail(p, abort, peer_abort);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t dacc = tmem_base + (uint32_t)(b * C::ACC1_COL);
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % S;
+                    const int x = it % X;
+                    if (!mbar_wait(&full[s], (uint32_t)(it / S) & 1u, p.timeout_ns, abort) ||
+                        !mbar_wait(&sf_ready[x], (uint32_t)(it / X) & 1u, p.timeout_ns, abort)) {
+                        gemm2_fail(p, abort, peer_abort);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int k_elems = min(C::BK, K - kb * C::BK);
+                    const int n_mma = k_elems / C::MMA_K;
+                    const uint32_t sf_col = C::SF_COL0 + (uint32_t)(it % C::SF_TBUFS) * C::SF_COLS;
+                    const uint32_t tsfa = tmem_base + sf_col;
+                    const uint32_t tsfb = tmem_base + sf_col + C::ATOMS * 4;
+                    const uint32_t xsfa = smem_u32(sXSF + x * C::XSF_BYTES);
+                    const uint32_t xsfb = xsfa + C::XSFA_BYTES;
+                    // canonical no-swizzle K-major source: 16-byte column chunks 2048 bytes apart
+                    if (C::ATOMS == 1) {
+                        tmem_cp_128x128b_pair(tsfa, smem_desc(xsfa, 0, 128, 0));
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < C::ATOMS / 2; ++c)
+                            tmem_cp_128x256b_pair(tsfa + c * 8, smem_desc(xsfa + c * 4096, 2048, 128, 0));
+                    }
+#pragma unroll
+                    for (int a = 0; a < C::ATOMS; ++a)
+                        tmem_cp_128x256b_pair(tsfb + a * 8, smem_desc(xsfb + a * 4096, 2048, 128, 0));
+                    const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
+                    const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
+                    for (int k = 0; k < n_mma; ++k) {
+                        int atom, sf_id;
+                        sf_select<KIND>(k, atom, sf_id);
+                        const uint32_t idesc = C::IDESC | ((uint32_t)sf_id << 29) | ((uint32_t)sf_id << 4);
+                        const uint64_t adesc = smem_desc(a_base + k * 32, 0, 1024, 2);
+                        const uint64_t bdesc = smem_desc(b_base + k * 32, 0, 1024, 2);
+                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                        if (KIND == G_MXFP4)
+                            mma2_mxf4nvf4_block32(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                        else if (KIND == G_NVFP4)
+                            mma2_mxf4nvf4_block16(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                        else
+                            mma2_mxf8f6f4_block32(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                    }
+                    tc_commit_pair(&empty[s], 0x3);
+                    issued = true;
+                }
+                if (!ok) break;
+                tc_commit_pair(&tmem_full[b], 0x3);
+            }
+            if (issued) {
+                tc_commit_pair(mma_done, 0x1);
+                if (!mbar_wait_drain(mma_done, 0, p.timeout_ns)) gemm2_fail(p, abort, peer_abort);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ============================================================ epilogue (both CTAs)
+        const int q = warp & 3;
+        const int h = (warp - 2) >> 2;
+        float gs = 1.0f;
+        if (KIND == G_NVFP4) gs = __fmul_rn(*p.g_a, *p.g_w);
+        int tcount = 0;
+        for (int tile = pair; tile < num_tiles; tile += num_pairs, ++tcount) {
+            const int mb = tile / num_n, nb = tile % num_n;
+            const int b = tcount & 1;
+            const bool got = mbar_wait(&tmem_full[b], ((uint32_t)tcount >> 1) & 1u, p.timeout_ns, abort);
+            if (!__all_sync(0xffffffffu, got)) {
+                if (lane == 0) gemm2_fail(p, abort, peer_abort);
+                break;
+            }
+            tc_fence_after();
+            uint32_t acc[4][32];
+            const uint32_t taddr =
+                tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC1_COL) + (uint32_t)(h * 128);
+            // the 64 columns shared by both accumulators: tile columns 192..255 of accumulator 0
+            // (half 1, chunks 2-3) or 0..63 of accumulator 1 (half 0, chunks 0-1)
+            const bool holds_overlap = (h == (b == 0 ? 1 : 0));
+            if (holds_overlap) {
+                if (b == 0) {
+                    tmem_ld_32x32b_x32(taddr + 2 * 32, acc[2]);
+                    tmem_ld_32x32b_x32(taddr + 3 * 32, acc[3]);
+                } else {
+                    tmem_ld_32x32b_x32(taddr + 0 * 32, acc[0]);
+                    tmem_ld_32x32b_x32(taddr + 1 * 32, acc[1]);
+                }
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) arrive_leader_relaxed(ovl_free, rank);
+                if (b == 0) {
+                    tmem_ld_32x32b_x32(taddr + 0 * 32, acc[0]);
+                    tmem_ld_32x32b_x32(taddr + 1 * 32, acc[1]);
+                } else {
+                    tmem_ld_32x32b_x32(taddr + 2 * 32, acc[2]);
+                    tmem_ld_32x32b_x32(taddr + 3 * 32, acc[3]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(taddr + c * 32, acc[c]);
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_leader_relaxed(&acc_free[b], rank);
+            epilogue_store<KIND>(p, acc, mb * 256 + (int)rank * 128 + q * 32 + lane, nb * GEMM_BN + h * 128, gs);
+        }
+    }
+
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, GEMM_TMEM_COLS);
     }
 }
 

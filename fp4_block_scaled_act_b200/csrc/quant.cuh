@@ -49,13 +49,21 @@ template <int KIND>
 __global__ void __launch_bounds__(QUANT_THREADS) quant_kernel(const uint4* __restrict__ x, int64_t M, int64_t K,
                                                               const float* __restrict__ g_ptr,
                                                               uint8_t* __restrict__ out, uint8_t* __restrict__ sf) {
-    const int64_t units_per_row = K >> 7;
-    const int64_t Mpad = (M + 127) & ~int64_t(127);
-    const int64_t total_units = Mpad * units_per_row;
+    // Each CTA owns a contiguous range of units; per pass its 16 half-warps take 16
+    // consecutive units, QUANT_UNROLL passes are loaded before any is processed.  Row and
+    // chunk of a unit are advanced incrementally (no per-unit division).
+    constexpr uint32_t UPB = QUANT_THREADS / 16;  // units per pass
+    const uint32_t upr = (uint32_t)(K >> 7);
+    const uint32_t Mpad = (uint32_t)((M + 127) & ~int64_t(127));
+    const uint32_t total = Mpad * upr;  // even: Mpad is a multiple of 128
+    const uint32_t span = UPB * QUANT_UNROLL;
+    const uint32_t per_cta = ((total + gridDim.x - 1) / gridDim.x + span - 1) / span * span;
+    const uint32_t u_begin = blockIdx.x * per_cta;
+    const uint32_t u_end = min(total, u_begin + per_cta);
     const int lane = threadIdx.x & 31;
     const int part = lane & 15;
-    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t stride_units = ((int64_t)gridDim.x * blockDim.x) >> 4;
+    const uint32_t my = threadIdx.x >> 4;
+    const uint32_t adv_rows = UPB / upr, adv_chunk = UPB % upr;
 
     float g = 1.0f, six_g = 6.0f;
     if (KIND == Q_NVFP4) {
@@ -63,24 +71,30 @@ __global__ void __launch_bounds__(QUANT_THREADS) quant_kernel(const uint4* __res
         six_g = __fmul_rn(6.0f, g);
     }
     // atoms (4 groups) per 128-row block along K
-    const int64_t atoms_per_rowblock = (KIND == Q_NVFP4) ? (K >> 6) : (K >> 7);
+    const uint32_t apr = (KIND == Q_NVFP4) ? (uint32_t)(K >> 6) : upr;
 
-    for (int64_t u0 = tid >> 4; u0 < total_units; u0 += stride_units * QUANT_UNROLL) {
+    uint32_t row = (u_begin + my) / upr;
+    uint32_t chunk = (u_begin + my) - row * upr;
+    for (uint32_t ub = u_begin; ub < u_end; ub += span) {
         uint4 raw[QUANT_UNROLL];
-        bool live[QUANT_UNROLL];
+        uint32_t rows[QUANT_UNROLL], chunks[QUANT_UNROLL];
 #pragma unroll
         for (int it = 0; it < QUANT_UNROLL; ++it) {
-            const int64_t u = u0 + it * stride_units;
-            const int64_t row = u / units_per_row;
-            live[it] = (u < total_units) && (row < M);
-            raw[it] = live[it] ? __ldcs(x + u * 16 + part) : make_uint4(0, 0, 0, 0);
+            rows[it] = row;
+            chunks[it] = chunk;
+            const uint32_t u = ub + it * UPB + my;
+            raw[it] = (u < u_end && row < (uint32_t)M) ? __ldcs(x + (size_t)u * 16 + part) : make_uint4(0, 0, 0, 0);
+            chunk += adv_chunk;
+            row += adv_rows;
+            if (chunk >= upr) {
+                chunk -= upr;
+                ++row;
+            }
         }
 #pragma unroll
         for (int it = 0; it < QUANT_UNROLL; ++it) {
-            const int64_t u = u0 + it * stride_units;
-            if (u >= total_units) break;  // uniform across the warp (total_units is even)
-            const int64_t row = u / units_per_row;
-            const int64_t chunk = u - row * units_per_row;
+            const uint32_t u = ub + it * UPB + my;
+            if (u >= u_end) break;  // uniform across the warp (ranges are even)
             float v[8];
             bf16x8_to_f32(raw[it], v);
             float amax = 0.0f;
@@ -109,41 +123,34 @@ __global__ void __launch_bounds__(QUANT_THREADS) quant_kernel(const uint4* __res
                 for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], inv);
             }
 
-            if (live[it]) {
+            if (rows[it] < (uint32_t)M) {
                 if (KIND == Q_MXFP8) {
                     uint2 w;
                     w.x = cvt_e4m3x2(v[0], v[1]) | (cvt_e4m3x2(v[2], v[3]) << 16);
                     w.y = cvt_e4m3x2(v[4], v[5]) | (cvt_e4m3x2(v[6], v[7]) << 16);
-                    reinterpret_cast<uint2*>(out)[u * 16 + part] = w;
+                    reinterpret_cast<uint2*>(out)[(size_t)u * 16 + part] = w;
                 } else {
-                    reinterpret_cast<uint32_t*>(out)[u * 16 + part] = cvt_e2m1x8(v);
+                    reinterpret_cast<uint32_t*>(out)[(size_t)u * 16 + part] = cvt_e2m1x8(v);
                 }
             }
 
-            // gather the unit's scale bytes into 32-bit words (padding rows give zeros)
-            const int half = lane & 16;
+            // gather the unit's scale bytes into 32-bit words (padding rows give zeros):
+            // every lane of a group holds its group's byte; shift it to the group's slot and
+            // OR across the 4 groups of a word
+            uint32_t word;
             if (KIND == Q_NVFP4) {
-                // groups 0..7 live in parts 0,2,..,14; word w holds groups 4w..4w+3
-                const int wsel = (part >> 3);
-                uint32_t word = 0;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t b = __shfl_sync(0xffffffffu, sfb, half + wsel * 8 + 2 * i);
-                    word |= b << (8 * i);
-                }
+                word = sfb << (8 * ((part >> 1) & 3));  // groups of 2 lanes, words of 8 lanes
+                word |= __shfl_xor_sync(0xffffffffu, word, 2);
+                word |= __shfl_xor_sync(0xffffffffu, word, 4);
                 if ((part & 7) == 0)
-                    *reinterpret_cast<uint32_t*>(sf + sf_word_offset(row, chunk * 2 + wsel, atoms_per_rowblock)) =
+                    *reinterpret_cast<uint32_t*>(sf + sf_word_offset(rows[it], chunks[it] * 2 + (part >> 3), apr)) =
                         word;
             } else {
-                // groups 0..3 live in parts 0,4,8,12
-                uint32_t word = 0;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t b = __shfl_sync(0xffffffffu, sfb, half + 4 * i);
-                    word |= b << (8 * i);
-                }
+                word = sfb << (8 * (part >> 2));        // groups of 4 lanes, one word per unit
+                word |= __shfl_xor_sync(0xffffffffu, word, 4);
+                word |= __shfl_xor_sync(0xffffffffu, word, 8);
                 if (part == 0)
-                    *reinterpret_cast<uint32_t*>(sf + sf_word_offset(row, chunk, atoms_per_rowblock)) = word;
+                    *reinterpret_cast<uint32_t*>(sf + sf_word_offset(rows[it], chunks[it], apr)) = word;
             }
         }
     }
