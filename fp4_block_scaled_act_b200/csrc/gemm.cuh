@@ -77,10 +77,10 @@ FP4_DEV void gemm_fail(const GemmParams& p, volatile int* abort) {
     atomicCAS(p.status, 0, STATUS_TIMEOUT);
 }
 
-// Add the W4A8 low-rank term, scale, add bias, round to bf16 and store 128 columns of one
-// output row held in registers (acc[c][j] = column col0 + 32c + j).
-template <int KIND>
-FP4_DEV void epilogue_store(const GemmParams& p, uint32_t (&acc)[4][32], int row, int col0, float gs) {
+// Add the W4A8 low-rank term, scale, add bias, round to bf16 and store NC x 32 columns of
+// one output row held in registers (acc[c][j] = column col0 + 32c + j).
+template <int KIND, int NC>
+FP4_DEV void epilogue_store(const GemmParams& p, uint32_t (&acc)[NC][32], int row, int col0, float gs) {
     if (row >= p.M || col0 >= p.N) return;
     const int N = p.N;
     if (KIND == G_W4A8) {
@@ -91,7 +91,7 @@ FP4_DEV void epilogue_store(const GemmParams& p, uint32_t (&acc)[4][32], int row
             const float ur = urow[r];
             const __nv_bfloat16* l2r = p.l2 + (size_t)r * N + col0;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < NC; ++c) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 8) {
                     const uint4 lv = *reinterpret_cast<const uint4*>(l2r + c * 32 + j);
@@ -109,7 +109,7 @@ FP4_DEV void epilogue_store(const GemmParams& p, uint32_t (&acc)[4][32], int row
     }
     __nv_bfloat16* yrow = p.y + (size_t)row * N + col0;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < NC; ++c) {
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
             const int col = col0 + c * 32 + j;
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(tmem_empty);
 
-            epilogue_store<KIND>(p, acc, mb * GEMM_BM + q * 32 + lane, nb * GEMM_BN + h * 128, gs);
+            epilogue_store<KIND, 4>(p, acc, mb * GEMM_BM + q * 32 + lane, nb * GEMM_BN + h * 128, gs);
         }
     }
 
@@ -366,56 +366,64 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // 2-CTA variant (cta_group::2): a cluster of two CTAs on an SM pair computes a 256 x 256
 // tile with M = 256 MMAs issued by the pair leader (CTA rank 0).  Each CTA loads its own
 // 128 rows of A and 128 of the 256 B rows; the tensor core combines both halves of B.
-// Per SM that is 256 operand rows per K stage instead of 384 for a 1-CTA 128 x 256 tile.
+// Per SM and K stage that is 256 operand rows instead of 384 for a 1-CTA 128 x 256
+// tile, so both the L2 -> shared-memory stream and the shared-memory reads of the MMA
+// shrink by a third.
 //
-// Scale factors.  The MMA reads, in each 32-lane TMEM sub-partition, the scales of that
-// sub-partition's rows, so every 512-byte scale atom has to be present in all four
-// sub-partitions.  Copying it with the multicast shape (32x128b.warpx4) costs the tensor
-// pipe several times more than a plain 128x256b copy of the same TMEM bytes.  Here an
-// expander warp writes each atom four times into shared memory (one copy per 32-lane
-// quarter), so the MMA thread moves two atoms per 128x256b copy: 3 copies per K stage
-// for MXFP4 instead of 6 multicast ones.  Both CTAs hold the scales of all 256 B rows.
+// Scale factors go to TMEM without tcgen05.cp: four "scale writer" warps, one per 32-lane
+// TMEM quarter, read the raw 512-byte atoms from shared memory and store them with
+// tcgen05.st in the layout the MMA reads: lane 32q+i, column xa+4a+g holds word g of row i
+// of A atom a (the scales of A row 32g+i), and column xb+8a+4rb+g holds word g of row i of
+// B atom a in row block rb, in every quarter q.  The tensor pipe then runs MMAs only, and
+// shared memory sees only the raw atoms.  Both CTAs hold the scales of all 256 B rows.
+// The writers load a stage's words before waiting for its TMEM buffer to be free, so only
+// the TMEM store and the arrive follow that wait.
 //
-// Accumulators.  Two 256-column accumulators overlap by 64 columns ([0,256) and
-// [192,448)), leaving [448,512) for the scale columns.  The epilogue drains the overlap
-// chunk first and releases it, so the next tile's MMAs start after a 64-column drain.
+// Accumulators: two 256-column accumulators overlap by 64 columns ([0,256), [192,448));
+// the epilogue drains the shared 64 columns first, so the next tile's MMAs wait for a
+// 64-column drain only.  Columns [448,512) hold the scale buffers.
 //
-// Synchronization.
+// Warps (448 threads): 0 TMA producer, 1 TMEM owner + MMA issuer (leader), 2-9 epilogue
+// (64 columns at a time), 10-13 scale writers.
+// Synchronization:
 //   full[s]      (leader)  A/B bytes of both CTAs; the leader alone expects them
 //   sf_full[s]   (local)   this CTA's raw scale atoms
-//   empty[s]     (both)    the leader's commit (MMAs and scale copies of stage s done)
-//   sf_ready[x]  (leader)  expanded scales of both CTAs in slot x
+//   empty[s]     (both)    the leader's commit (MMAs of stage s done)
+//   sf_ready[t]  (leader)  scale buffer t written in both CTAs (8 writer warps)
 //   tmem_full[b] (both)    accumulator b complete
 //   acc_free[b]  (leader)  accumulator b fully drained by both CTAs (16 warps)
-//   ovl_free     (leader)  overlap chunk of the last tile drained (8 warps)
+//   ovl_free     (leader)  overlap columns of the last tile drained (8 warps)
 // =======================================================================================
 template <int KIND>
 struct Gemm2Cfg {
     using C1 = GemmCfg<KIND>;
-    static constexpr int BK = C1::BK, G = C1::G, MMA_K = C1::MMA_K, ATOMS = C1::ATOMS;
-    static constexpr int A_BYTES = 128 * 128;
-    static constexpr int B_BYTES = 128 * 128;  // this CTA's half of the 256 B rows
-    static constexpr int RSFA_BYTES = ATOMS * 512;        // raw atoms, this CTA's 128 A rows
-    static constexpr int RSFB_BYTES = 2 * ATOMS * 512;    // raw atoms, all 256 B rows
+    // NVFP4 takes 128 K per stage (64-byte swizzle) so its scale footprint matches MXFP4's
+    static constexpr int BK = (KIND == G_NVFP4) ? 128 : C1::BK;
+    static constexpr int G = C1::G, MMA_K = C1::MMA_K;
+    static constexpr int ATOMS = BK / (G * 4);
+    static constexpr int ROW_BYTES = (KIND == G_NVFP4) ? 64 : 128;     // per operand row per stage
+    static constexpr uint32_t SWZ = (ROW_BYTES == 128) ? 2u : 4u;      // descriptor layout
+    static constexpr int SBO = 8 * ROW_BYTES;
+    static constexpr int N_MMA = BK / MMA_K;
+    static constexpr int A_BYTES = 128 * ROW_BYTES;
+    static constexpr int B_BYTES = 128 * ROW_BYTES;  // this CTA's half of the 256 B rows
+    static constexpr int RSFA_BYTES = ATOMS * 512;    // raw atoms, this CTA's 128 A rows
+    static constexpr int RSFB_BYTES = 2 * ATOMS * 512;  // raw atoms, all 256 B rows
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RSFA_BYTES + RSFB_BYTES;
-    static constexpr int STAGES = (KIND == G_NVFP4) ? 4 : (KIND == G_W4A8 ? 6 : 5);
-    // expanded scales: every atom replicated 4x (2 KB); a 128x256b copy takes two of them
-    static constexpr int XSFA_BYTES = ATOMS * 2048;       // atom pairs (2a, 2a+1) per 4 KB
-    static constexpr int XSFB_BYTES = ATOMS * 4096;       // per atom: row block 0 | row block 1
-    static constexpr int XSF_BYTES = XSFA_BYTES + XSFB_BYTES;
-    static constexpr int XBUFS = (KIND == G_NVFP4) ? 2 : 3;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + XBUFS * XSF_BYTES + 512;
+    static constexpr int STAGES = (KIND == G_NVFP4) ? 10 : 6;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512;
     static constexpr uint32_t AB_TX = A_BYTES + ((KIND == G_W4A8) ? B_BYTES / 2 : B_BYTES);
     static constexpr uint32_t SF_TX = RSFA_BYTES + RSFB_BYTES;
-    static constexpr int SF_COLS = ATOMS * 12;            // SFA 4/atom + SFB 8/atom
-    static constexpr int ACC1_COL = 192;                  // second accumulator: [192, 448)
+    static constexpr int ACC1_COL = 192;
     static constexpr int SF_COL0 = 448;
-    static constexpr int SF_TBUFS = (64 / SF_COLS) >= 2 ? 2 : 1;
-    static constexpr int THREADS = 352;
+    static constexpr int SFA_COLS = 4 * ATOMS;        // A: 4 columns per atom
+    static constexpr int SF_COLS = SFA_COLS + 8 * ATOMS;  // B: 8 columns per atom
+    static constexpr int TB = (64 / SF_COLS) >= 4 ? 4 : (64 / SF_COLS);  // scale buffers
+    static constexpr int THREADS = 448;
     static constexpr uint32_t IDESC = (C1::A_FMT << 7) | (C1::B_FMT << 10) | ((uint32_t)(256 >> 3) << 17) |
                                       (C1::SCALE_FMT << 23) | ((uint32_t)(256 >> 4) << 24);
     static_assert(SMEM_BYTES <= 232448, "shared memory");
-    static_assert(SF_COL0 + SF_TBUFS * SF_COLS <= GEMM_TMEM_COLS, "TMEM budget");
+    static_assert(TB >= 2 && SF_COL0 + TB * SF_COLS <= GEMM_TMEM_COLS, "TMEM budget");
 };
 
 FP4_DEV void gemm2_fail(const GemmParams& p, volatile int* abort, uint32_t peer_abort) {
@@ -425,7 +433,8 @@ FP4_DEV void gemm2_fail(const GemmParams& p, volatile int* abort, uint32_t peer_
 }
 
 // Arrive on a barrier of the pair leader: a local arrive in the leader, a remote relaxed
-// arrive in the follower (used after TMEM reads that tcgen05.wait::ld has completed).
+// arrive in the follower (used after TMEM loads/stores that tcgen05.wait has completed, so
+// no memory write needs publishing; a release.cluster arrive would fence every call).
 FP4_DEV void arrive_leader_relaxed(uint64_t* bar, uint32_t rank) {
     if (rank == 0)
         mbar_arrive(bar);
@@ -439,20 +448,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                  const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB, GemmParams p) {
     using C = Gemm2Cfg<KIND>;
     constexpr int S = C::STAGES;
-    constexpr int X = C::XBUFS;
+    constexpr int TB = C::TB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + S * C::A_BYTES;
     uint8_t* sRSFA = sB + S * C::B_BYTES;
     uint8_t* sRSFB = sRSFA + S * C::RSFA_BYTES;
-    uint8_t* sXSF = sRSFB + S * C::RSFB_BYTES;           // X slots of XSF_BYTES
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sXSF + X * C::XSF_BYTES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sRSFB + S * C::RSFB_BYTES);
     uint64_t* full = bars;
     uint64_t* sf_full = full + S;
     uint64_t* empty = sf_full + S;
-    uint64_t* sf_ready = empty + S;
-    uint64_t* tmem_full = sf_ready + X;                   // [2]
+    uint64_t* sf_ready = empty + S;                       // [TB]
+    uint64_t* tmem_full = sf_ready + TB;                  // [2]
     uint64_t* acc_free = tmem_full + 2;                   // [2]
     uint64_t* ovl_free = acc_free + 2;
     uint64_t* mma_done = ovl_free + 1;
@@ -470,7 +478,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             mbar_init(&sf_full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int x = 0; x < X; ++x) mbar_init(&sf_ready[x], 2);
+        for (int t = 0; t < TB; ++t) mbar_init(&sf_ready[t], 8);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tmem_full[b], 1);
             mbar_init(&acc_free[b], 16);
@@ -524,12 +532,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                     }
                     if (it == p.skip_iter) continue;  // test hook: this stage is never filled
                     // A/B of both CTAs land on the leader's barrier; only the leader expects them
-                    // (a remote arrive with release semantics would fence every stage)
                     const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
                     if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::AB_TX);
                     mbar_arrive_expect_tx(&sf_full[s], C::SF_TX);
-                    const int ax = (KIND == G_W4A8) ? kb * C::BK : kb * (C::BK / 2);
-                    const int bx = (KIND == G_W4A8) ? kb * C::BK : kb * (C::BK / 2);
+                    // x: bytes of the row for packed FP4 and E4M3, elements for the W4A8 unpacking map
+                    const int ax = kb * C::ROW_BYTES;
+                    const int bx = (KIND == G_W4A8) ? kb * C::BK : kb * C::ROW_BYTES;
                     tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, bar, ax, mb * 256 + (int)rank * 128, pol_a);
                     tma_load_2d_pair(sB + s * C::B_BYTES, &tmB, bar, bx, nb * 256 + (int)rank * 128, pol_b);
                     tma_load_2d(sRSFA + s * C::RSFA_BYTES, &tmSFA, &sf_full[s], 0,
@@ -549,18 +557,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                     gemm2_fail(p, abort, peer_abort);
             }
         }
-    } else if (warp == 10) {
-        // ============================================================ scale expander (both CTAs)
+    } else if (warp >= 10) {
+        // ============================================================ scale writers (both CTAs)
+        const int quarter = warp & 3;
+        const uint32_t tlane = tmem_base + ((uint32_t)(quarter * 32) << 16);
         int it = 0;
         bool ok = true;
         for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
             for (int kb = 0; kb < num_kb; ++kb, ++it) {
                 const int s = it % S;
-                const int x = it % X;
+                const int t = it % TB;
                 bool got = mbar_wait(&sf_full[s], (uint32_t)(it / S) & 1u, p.timeout_ns, abort);
-                // slot x is free once the copies of iteration it - X (same slot) are done
-                if (got && it >= X)
-                    got = mbar_wait(&empty[(it - X) % S], (uint32_t)((it - X) / S) & 1u, p.timeout_ns, abort);
                 if (!__all_sync(0xffffffffu, got)) {
                     if (lane == 0) gemm2_fail(p, abort, peer_abort);
                     ok = false;
@@ -568,38 +575,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 }
                 const uint4* rsfa = reinterpret_cast<const uint4*>(sRSFA + s * C::RSFA_BYTES);
                 const uint4* rsfb = reinterpret_cast<const uint4*>(sRSFB + s * C::RSFB_BYTES);
-                uint8_t* xsfa = sXSF + x * C::XSF_BYTES;
-                uint8_t* xsfb = xsfa + C::XSFA_BYTES;
+                // lane i takes row i of every atom: words 0-3 = the scales of rows i, 32+i, 64+i, 96+i
+                uint32_t va[4 * C::ATOMS];
+                uint32_t vb[8 * C::ATOMS];
 #pragma unroll
                 for (int a = 0; a < C::ATOMS; ++a) {
-                    // lane l moves 16 bytes of the atom: quarter q gets a full copy
-                    const uint4 v = rsfa[a * 32 + lane];
-                    uint8_t* dst = xsfa + (a >> 1) * 4096 + (a & 1) * 2048 + lane * 16;
+                    const uint4 w = rsfa[a * 32 + lane];
+                    va[4 * a] = w.x, va[4 * a + 1] = w.y, va[4 * a + 2] = w.z, va[4 * a + 3] = w.w;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(dst + q * 512) = v;
-                }
-#pragma unroll
-                for (int rb = 0; rb < 2; ++rb) {
-#pragma unroll
-                    for (int a = 0; a < C::ATOMS; ++a) {
-                        const uint4 v = rsfb[(rb * C::ATOMS + a) * 32 + lane];
-                        uint8_t* dst = xsfb + a * 4096 + rb * 2048 + lane * 16;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(dst + q * 512) = v;
+                    for (int rb = 0; rb < 2; ++rb) {
+                        const uint4 z = rsfb[(rb * C::ATOMS + a) * 32 + lane];
+                        vb[8 * a + 4 * rb] = z.x, vb[8 * a + 4 * rb + 1] = z.y;
+                        vb[8 * a + 4 * rb + 2] = z.z, vb[8 * a + 4 * rb + 3] = z.w;
                     }
                 }
-                fence_proxy_async_smem();  // generic-proxy writes -> visible to tcgen05.cp
-                __syncwarp();
-                // relaxed: a release.cluster arrive would put a cluster-scope fence in every stage
-                // (measured: half the throughput).  The writes are this CTA's own shared memory,
-                // read only by this SM's tensor core, and the proxy fence above has made them
-                // visible to the async proxy before the arrive is issued.
-                if (lane == 0) {
-                    if (rank == 0)
-                        mbar_arrive(&sf_ready[x]);
-                    else
-                        mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&sf_ready[x]), 0));
+                // buffer t is free once the MMAs of iteration it - TB (same buffer) are done
+                got = it < TB || mbar_wait(&empty[(it - TB) % S], (uint32_t)((it - TB) / S) & 1u, p.timeout_ns, abort);
+                if (!__all_sync(0xffffffffu, got)) {
+                    if (lane == 0) gemm2_fail(p, abort, peer_abort);
+                    ok = false;
+                    break;
                 }
+                const uint32_t xa = C::SF_COL0 + (uint32_t)(t * C::SF_COLS);
+                const uint32_t xb = xa + C::SFA_COLS;
+                if constexpr (C::ATOMS == 2) {
+                    tmem_st_32x32b_x8(tlane + xa, va);
+                    tmem_st_32x32b_x16(tlane + xb, vb);
+                } else {
+                    tmem_st_32x32b_x4(tlane + xa, va);
+                    tmem_st_32x32b_x8(tlane + xb, vb);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) arrive_leader_relaxed(&sf_ready[t], rank);
             }
         }
     } else if (warp == 1) {
@@ -620,9 +629,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 const uint32_t dacc = tmem_base + (uint32_t)(b * C::ACC1_COL);
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int s = it % S;
-                    const int x = it % X;
+                    const int t = it % TB;
                     if (!mbar_wait(&full[s], (uint32_t)(it / S) & 1u, p.timeout_ns, abort) ||
-                        !mbar_wait(&sf_ready[x], (uint32_t)(it / X) & 1u, p.timeout_ns, abort)) {
+                        !mbar_wait(&sf_ready[t], (uint32_t)(it / TB) & 1u, p.timeout_ns, abort)) {
                         gemm2_fail(p, abort, peer_abort);
                         ok = false;
                         break;
@@ -630,30 +639,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                     tc_fence_after();
                     const int k_elems = min(C::BK, K - kb * C::BK);
                     const int n_mma = k_elems / C::MMA_K;
-                    const uint32_t sf_col = C::SF_COL0 + (uint32_t)(it % C::SF_TBUFS) * C::SF_COLS;
-                    const uint32_t tsfa = tmem_base + sf_col;
-                    const uint32_t tsfb = tmem_base + sf_col + C::ATOMS * 4;
-                    const uint32_t xsfa = smem_u32(sXSF + x * C::XSF_BYTES);
-                    const uint32_t xsfb = xsfa + C::XSFA_BYTES;
-                    // canonical no-swizzle K-major source: 16-byte column chunks 2048 bytes apart
-                    if (C::ATOMS == 1) {
-                        tmem_cp_128x128b_pair(tsfa, smem_desc(xsfa, 0, 128, 0));
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < C::ATOMS / 2; ++c)
-                            tmem_cp_128x256b_pair(tsfa + c * 8, smem_desc(xsfa + c * 4096, 2048, 128, 0));
-                    }
-#pragma unroll
-                    for (int a = 0; a < C::ATOMS; ++a)
-                        tmem_cp_128x256b_pair(tsfb + a * 8, smem_desc(xsfb + a * 4096, 2048, 128, 0));
+                    const uint32_t tsfa = tmem_base + C::SF_COL0 + (uint32_t)(t * C::SF_COLS);
+                    const uint32_t tsfb = tsfa + C::SFA_COLS;
                     const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
                     const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
                     for (int k = 0; k < n_mma; ++k) {
                         int atom, sf_id;
                         sf_select<KIND>(k, atom, sf_id);
                         const uint32_t idesc = C::IDESC | ((uint32_t)sf_id << 29) | ((uint32_t)sf_id << 4);
-                        const uint64_t adesc = smem_desc(a_base + k * 32, 0, 1024, 2);
-                        const uint64_t bdesc = smem_desc(b_base + k * 32, 0, 1024, 2);
+                        const uint64_t adesc = smem_desc(a_base + k * 32, 0, C::SBO, C::SWZ);
+                        const uint64_t bdesc = smem_desc(b_base + k * 32, 0, C::SBO, C::SWZ);
                         const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
                         if (KIND == G_MXFP4)
                             mma2_mxf4nvf4_block32(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
@@ -674,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             }
         }
         __syncwarp();
-    } else {
+    } else if (warp >= 2) {
         // ============================================================ epilogue (both CTAs)
         const int q = warp & 3;
         const int h = (warp - 2) >> 2;
@@ -690,40 +685,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 break;
             }
             tc_fence_after();
-            uint32_t acc[4][32];
             const uint32_t taddr =
                 tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC1_COL) + (uint32_t)(h * 128);
-            // the 64 columns shared by both accumulators: tile columns 192..255 of accumulator 0
-            // (half 1, chunks 2-3) or 0..63 of accumulator 1 (half 0, chunks 0-1)
+            const int row = mb * 256 + (int)rank * 128 + q * 32 + lane;
+            const int col0 = nb * GEMM_BN + h * 128;
+            // the 64 columns shared by both accumulators are tile columns 192..255 of
+            // accumulator 0 (half 1, chunks 2-3) or 0..63 of accumulator 1 (half 0, chunks 0-1):
+            // their holders drain them first and release them
             const bool holds_overlap = (h == (b == 0 ? 1 : 0));
+            const int first = holds_overlap ? (b == 0 ? 2 : 0) : 0;
+            const int second = 2 - first;
+            uint32_t acc[2][32];
+            tmem_ld_32x32b_x32(taddr + first * 32, acc[0]);
+            tmem_ld_32x32b_x32(taddr + (first + 1) * 32, acc[1]);
+            tmem_wait_ld();
             if (holds_overlap) {
-                if (b == 0) {
-                    tmem_ld_32x32b_x32(taddr + 2 * 32, acc[2]);
-                    tmem_ld_32x32b_x32(taddr + 3 * 32, acc[3]);
-                } else {
-                    tmem_ld_32x32b_x32(taddr + 0 * 32, acc[0]);
-                    tmem_ld_32x32b_x32(taddr + 1 * 32, acc[1]);
-                }
-                tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) arrive_leader_relaxed(ovl_free, rank);
-                if (b == 0) {
-                    tmem_ld_32x32b_x32(taddr + 0 * 32, acc[0]);
-                    tmem_ld_32x32b_x32(taddr + 1 * 32, acc[1]);
-                } else {
-                    tmem_ld_32x32b_x32(taddr + 2 * 32, acc[2]);
-                    tmem_ld_32x32b_x32(taddr + 3 * 32, acc[3]);
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(taddr + c * 32, acc[c]);
             }
+            epilogue_store<KIND, 2>(p, acc, row, col0 + first * 32, gs);
+            tmem_ld_32x32b_x32(taddr + second * 32, acc[0]);
+            tmem_ld_32x32b_x32(taddr + (second + 1) * 32, acc[1]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) arrive_leader_relaxed(&acc_free[b], rank);
-            epilogue_store<KIND>(p, acc, mb * 256 + (int)rank * 128 + q * 32 + lane, nb * GEMM_BN + h * 128, gs);
+            epilogue_store<KIND, 2>(p, acc, row, col0 + second * 32, gs);
         }
     }
 
