@@ -188,12 +188,17 @@ fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CU
     fp4_status_t s;
     if ((s = encode_sf(&tsa, sfa, p.M, p.K, C::G, C::ATOMS)) != FP4_OK) return s;
     if ((s = encode_sf(&tsb, sfb, p.N, p.K, C::G, C::ATOMS)) != FP4_OK) return s;
+    // output: bf16 [M, N], stored by the epilogue in 32-row x 64-column boxes (128-byte swizzle)
+    CUtensorMap ty;
+    if ((s = encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.y, (uint64_t)p.N, (uint64_t)p.M,
+                       (uint64_t)p.N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
+        return s;
     const int tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
     const int pairs = tiles < ds->pairs[KIND] ? tiles : ds->pairs[KIND];
     p.timeout_ns = g_timeout_ns;
     p.skip_iter = g_skip_iter;
     p.status = ds->status;
-    gemm2_kernel<KIND><<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, p);
+    gemm2_kernel<KIND><<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, ty, p);
     return launched();
 }
 

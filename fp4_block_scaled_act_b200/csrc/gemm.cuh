@@ -77,11 +77,11 @@ FP4_DEV void gemm_fail(const GemmParams& p, volatile int* abort) {
     atomicCAS(p.status, 0, STATUS_TIMEOUT);
 }
 
-// Add the W4A8 low-rank term, scale, add bias, round to bf16 and store NC x 32 columns of
-// one output row held in registers (acc[c][j] = column col0 + 32c + j).
+// Add the W4A8 low-rank term, scale, add bias and round to bf16 NC x 32 columns of one
+// output row held in registers (acc[c][j] = column col0 + 32c + j, fp32 bits; row < M).
+// On return acc[c][w], w < 16, holds columns 32c + 2w and 32c + 2w + 1 as a bf16 pair.
 template <int KIND, int NC>
-FP4_DEV void epilogue_store(const GemmParams& p, uint32_t (&acc)[NC][32], int row, int col0, float gs) {
-    if (row >= p.M || col0 >= p.N) return;
+FP4_DEV void epilogue_pack(const GemmParams& p, uint32_t (&acc)[NC][32], int row, int col0, float gs) {
     const int N = p.N;
     if (KIND == G_W4A8) {
         // acc += u[row, r] * L2[r, cols] for r = 0..31, one rank at a time (fp32 FMAs)
@@ -107,17 +107,15 @@ FP4_DEV void epilogue_store(const GemmParams& p, uint32_t (&acc)[NC][32], int ro
             }
         }
     }
-    __nv_bfloat16* yrow = p.y + (size_t)row * N + col0;
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
-            const int col = col0 + c * 32 + j;
             float v[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(acc[c][j + i]) * gs;
             if (p.bias) {
-                const uint4 bv = *reinterpret_cast<const uint4*>(p.bias + col);
+                const uint4 bv = *reinterpret_cast<const uint4*>(p.bias + col0 + c * 32 + j);
                 const __half2* bh = reinterpret_cast<const __half2*>(&bv);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -126,16 +124,27 @@ FP4_DEV void epilogue_store(const GemmParams& p, uint32_t (&acc)[NC][32], int ro
                     v[2 * i + 1] += bf.y;
                 }
             }
-            uint4 o;
-            uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-                ow[i] = *reinterpret_cast<uint32_t*>(&b2);
+                acc[c][j / 2 + i] = *reinterpret_cast<uint32_t*>(&b2);
             }
-            *reinterpret_cast<uint4*>(yrow + c * 32 + j) = o;
         }
     }
+}
+
+// Pack one row's NC 32-column chunks and store them straight to global memory (1-CTA kernel).
+template <int KIND, int NC>
+FP4_DEV void epilogue_store(const GemmParams& p, uint32_t (&acc)[NC][32], int row, int col0, float gs) {
+    if (row >= p.M || col0 >= p.N) return;
+    epilogue_pack<KIND, NC>(p, acc, row, col0, gs);
+    __nv_bfloat16* yrow = p.y + (size_t)row * p.N + col0;
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+            *reinterpret_cast<uint4*>(yrow + c * 32 + g * 8) =
+                make_uint4(acc[c][4 * g], acc[c][4 * g + 1], acc[c][4 * g + 2], acc[c][4 * g + 3]);
 }
 
 // Which TMEM scale atom and which byte of it MMA number k of a stage reads.
@@ -383,8 +392,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // the epilogue drains the shared 64 columns first, so the next tile's MMAs wait for a
 // 64-column drain only.  Columns [448,512) hold the scale buffers.
 //
-// Warps (448 threads): 0 TMA producer, 1 TMEM owner + MMA issuer (leader), 2-9 epilogue
-// (64 columns at a time), 10-13 scale writers.
+// Warps (480 threads): 0 TMA producer, 1 TMEM owner + MMA issuer (leader), 2-9 epilogue
+// (64 columns at a time), 10-13 scale writers, 14 stage coordinator (leader).
+// The tensor pipe queues very little ahead of the issuing thread, so every cycle that
+// thread spends between two MMAs is a bubble, and an mbarrier test from it costs on the
+// order of a hundred cycles while the tensor core streams shared memory.  The MMA warp
+// therefore tests no mbarrier: the coordinator does the waits and hands each stage over
+// with a hardware named barrier (bar.arrive / bar.sync), which does not touch shared
+// memory.
 // Synchronization:
 //   full[s]      (leader)  A/B bytes of both CTAs; the leader alone expects them
 //   sf_full[s]   (local)   this CTA's raw scale atoms
@@ -410,8 +425,9 @@ struct Gemm2Cfg {
     static constexpr int RSFA_BYTES = ATOMS * 512;    // raw atoms, this CTA's 128 A rows
     static constexpr int RSFB_BYTES = 2 * ATOMS * 512;  // raw atoms, all 256 B rows
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RSFA_BYTES + RSFB_BYTES;
-    static constexpr int STAGES = (KIND == G_NVFP4) ? 10 : 6;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512;
+    static constexpr int STAGES = (KIND == G_NVFP4) ? 10 : 5;
+    static constexpr int EPI_BYTES = 8 * 32 * 128;    // a 32 x 64 bf16 staging tile per epilogue warp
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + 512;
     static constexpr uint32_t AB_TX = A_BYTES + ((KIND == G_W4A8) ? B_BYTES / 2 : B_BYTES);
     static constexpr uint32_t SF_TX = RSFA_BYTES + RSFB_BYTES;
     static constexpr int ACC1_COL = 192;
@@ -419,12 +435,32 @@ struct Gemm2Cfg {
     static constexpr int SFA_COLS = 4 * ATOMS;        // A: 4 columns per atom
     static constexpr int SF_COLS = SFA_COLS + 8 * ATOMS;  // B: 8 columns per atom
     static constexpr int TB = (64 / SF_COLS) >= 4 ? 4 : (64 / SF_COLS);  // scale buffers
-    static constexpr int THREADS = 448;
+    static constexpr int THREADS = 480;
     static constexpr uint32_t IDESC = (C1::A_FMT << 7) | (C1::B_FMT << 10) | ((uint32_t)(256 >> 3) << 17) |
                                       (C1::SCALE_FMT << 23) | ((uint32_t)(256 >> 4) << 24);
     static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert((STAGES * (A_BYTES + B_BYTES)) % 1024 == 0, "staging tiles 1024-byte aligned");
     static_assert(TB >= 2 && SF_COL0 + TB * SF_COLS <= GEMM_TMEM_COLS, "TMEM budget");
 };
+
+// Pair-kernel epilogue: pack one row's 64 columns and write them, as 128 bytes, into row
+// `r` of the warp's 32 x 128-byte staging tile in the 128-byte-swizzled layout the output
+// tensor map reads (16-byte granule g of row r at granule g ^ (r % 8)).  Rows at or beyond
+// M are not computed; the TMA store clips them.
+template <int KIND>
+FP4_DEV void epilogue_stage(const GemmParams& p, uint32_t (&acc)[2][32], int row, int col0, float gs, uint8_t* tile,
+                            int r) {
+    if (row >= p.M) return;
+    epilogue_pack<KIND, 2>(p, acc, row, col0, gs);
+    const uint32_t base = smem_u32(tile) + (uint32_t)r * 128u;
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+            const uint32_t g = (uint32_t)(c * 4 + g4) ^ ((uint32_t)r & 7u);
+            st_shared_v4(base + g * 16u, acc[c][4 * g4], acc[c][4 * g4 + 1], acc[c][4 * g4 + 2], acc[c][4 * g4 + 3]);
+        }
+}
 
 FP4_DEV void gemm2_fail(const GemmParams& p, volatile int* abort, uint32_t peer_abort) {
     *abort = 1;
@@ -445,7 +481,8 @@ FP4_DEV void arrive_leader_relaxed(uint64_t* bar, uint32_t rank) {
 template <int KIND>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THREADS, 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB, GemmParams p) {
+                 const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+                 const __grid_constant__ CUtensorMap tmY, GemmParams p) {
     using C = Gemm2Cfg<KIND>;
     constexpr int S = C::STAGES;
     constexpr int TB = C::TB;
@@ -453,7 +490,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + S * C::A_BYTES;
-    uint8_t* sRSFA = sB + S * C::B_BYTES;
+    uint8_t* sEpi = sB + S * C::B_BYTES;                  // 8 staging tiles of 4 KB
+    uint8_t* sRSFA = sEpi + C::EPI_BYTES;
     uint8_t* sRSFB = sRSFA + S * C::RSFA_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sRSFB + S * C::RSFB_BYTES);
     uint64_t* full = bars;
@@ -493,6 +531,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         prefetch_tmap(&tmB);
         prefetch_tmap(&tmSFA);
         prefetch_tmap(&tmSFB);
+        prefetch_tmap(&tmY);
     }
     __syncwarp();
     if (warp == 1) {
@@ -557,7 +596,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                     gemm2_fail(p, abort, peer_abort);
             }
         }
-    } else if (warp >= 10) {
+    } else if (warp >= 10 && warp < 14) {
         // ============================================================ scale writers (both CTAs)
         const int quarter = warp & 3;
         const uint32_t tlane = tmem_base + ((uint32_t)(quarter * 32) << 16);
@@ -613,66 +652,98 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         }
     } else if (warp == 1) {
         // ============================================================ MMA issuer (leader)
-        if (rank == 0 && lane == 0) {
-            int it = 0, tcount = 0;
+        // The whole warp runs the loop so that it can take the named barrier each stage;
+        // lane 0 issues.  Per stage it touches no shared memory at all: the coordinator
+        // warp has checked everything the stage needs before releasing it, and the abort
+        // flag is read once per tile (the coordinator releases every stage of a tile even
+        // after a failure, so the warp always reaches that check).
+        if (rank == 0) {
+            uint32_t it = 0;
+            int tcount = 0;
             bool issued = false, ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++tcount) {
+                const int b = tcount & 1;
+                const uint32_t dacc = tmem_base + (uint32_t)(b * C::ACC1_COL);
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    named_bar_sync(1u + it % TB, 64u);
+                    if (lane == 0) {
+                        tc_fence_after();
+                        const int s = (int)(it % S);
+                        const int t = (int)(it % TB);
+                        const int n_mma = min(C::BK, K - kb * C::BK) / C::MMA_K;
+                        const uint32_t tsfa = tmem_base + C::SF_COL0 + (uint32_t)(t * C::SF_COLS);
+                        const uint32_t tsfb = tsfa + C::SFA_COLS;
+                        const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
+                        const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
+                        for (int k = 0; k < n_mma; ++k) {
+                            int atom, sf_id;
+                            sf_select<KIND>(k, atom, sf_id);
+                            const uint32_t idesc = C::IDESC | ((uint32_t)sf_id << 29) | ((uint32_t)sf_id << 4);
+                            const uint64_t adesc = smem_desc(a_base + k * 32, 0, C::SBO, C::SWZ);
+                            const uint64_t bdesc = smem_desc(b_base + k * 32, 0, C::SBO, C::SWZ);
+                            const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                            if (KIND == G_MXFP4)
+                                mma2_mxf4nvf4_block32(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                            else if (KIND == G_NVFP4)
+                                mma2_mxf4nvf4_block16(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                            else
+                                mma2_mxf8f6f4_block32(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                        }
+                        tc_commit_pair(&empty[s], 0x3);
+                    }
+                    __syncwarp();
+                    issued = true;
+                }
+                if (lane == 0) tc_commit_pair(&tmem_full[b], 0x3);
+                __syncwarp();
+                if (__any_sync(0xffffffffu, *abort != 0)) ok = false;
+            }
+            if (issued) {
+                if (lane == 0) tc_commit_pair(mma_done, 0x1);
+                __syncwarp();
+                const bool drained = mbar_wait_drain(mma_done, 0, p.timeout_ns);
+                if (!__all_sync(0xffffffffu, drained) && lane == 0) gemm2_fail(p, abort, peer_abort);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 14) {
+        // ============================================================ stage coordinator (leader)
+        // Waits, in the MMA warp's order, for everything a stage needs (the accumulator
+        // and the overlap at a tile's first stage; A/B bytes of both CTAs; both CTAs'
+        // scale buffer) and then releases the stage with named barrier 1 + it % TB.  After
+        // a failure it still releases the remaining stages of that tile without waiting,
+        // so the MMA warp, which checks the abort flag at the end of each tile, never
+        // waits on a barrier that nobody arrives at.  The ring of TB barrier ids cannot be lapped:
+        // the scale buffer of stage it + TB is free only after the MMA warp has passed
+        // stage it.
+        if (rank == 0) {
+            uint32_t it = 0;
+            int tcount = 0;
+            bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++tcount) {
                 const int b = tcount & 1;
                 // accumulator b drained (tile tcount-2) and the overlap of tile tcount-1 drained
                 bool got = mbar_wait(&acc_free[b], (((uint32_t)tcount >> 1) & 1u) ^ 1u, p.timeout_ns, abort);
                 if (got && tcount > 0) got = mbar_wait(ovl_free, (uint32_t)(tcount - 1) & 1u, p.timeout_ns, abort);
-                if (!got) {
-                    gemm2_fail(p, abort, peer_abort);
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t dacc = tmem_base + (uint32_t)(b * C::ACC1_COL);
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
-                    const int s = it % S;
-                    const int t = it % TB;
-                    if (!mbar_wait(&full[s], (uint32_t)(it / S) & 1u, p.timeout_ns, abort) ||
-                        !mbar_wait(&sf_ready[t], (uint32_t)(it / TB) & 1u, p.timeout_ns, abort)) {
-                        gemm2_fail(p, abort, peer_abort);
+                    if (got) got = mbar_wait(&full[it % S], (it / S) & 1u, p.timeout_ns, abort);
+                    if (got) got = mbar_wait(&sf_ready[it % TB], (it / TB) & 1u, p.timeout_ns, abort);
+                    got = __all_sync(0xffffffffu, got);
+                    if (!got && ok) {
+                        if (lane == 0) gemm2_fail(p, abort, peer_abort);
                         ok = false;
-                        break;
                     }
-                    tc_fence_after();
-                    const int k_elems = min(C::BK, K - kb * C::BK);
-                    const int n_mma = k_elems / C::MMA_K;
-                    const uint32_t tsfa = tmem_base + C::SF_COL0 + (uint32_t)(t * C::SF_COLS);
-                    const uint32_t tsfb = tsfa + C::SFA_COLS;
-                    const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
-                    const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
-                    for (int k = 0; k < n_mma; ++k) {
-                        int atom, sf_id;
-                        sf_select<KIND>(k, atom, sf_id);
-                        const uint32_t idesc = C::IDESC | ((uint32_t)sf_id << 29) | ((uint32_t)sf_id << 4);
-                        const uint64_t adesc = smem_desc(a_base + k * 32, 0, C::SBO, C::SWZ);
-                        const uint64_t bdesc = smem_desc(b_base + k * 32, 0, C::SBO, C::SWZ);
-                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-                        if (KIND == G_MXFP4)
-                            mma2_mxf4nvf4_block32(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
-                        else if (KIND == G_NVFP4)
-                            mma2_mxf4nvf4_block16(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
-                        else
-                            mma2_mxf8f6f4_block32(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
-                    }
-                    tc_commit_pair(&empty[s], 0x3);
-                    issued = true;
+                    __syncwarp();
+                    named_bar_arrive(1u + it % TB, 64u);
                 }
-                if (!ok) break;
-                tc_commit_pair(&tmem_full[b], 0x3);
-            }
-            if (issued) {
-                tc_commit_pair(mma_done, 0x1);
-                if (!mbar_wait_drain(mma_done, 0, p.timeout_ns)) gemm2_fail(p, abort, peer_abort);
             }
         }
-        __syncwarp();
     } else if (warp >= 2) {
         // ============================================================ epilogue (both CTAs)
         const int q = warp & 3;
         const int h = (warp - 2) >> 2;
+        uint8_t* stile = sEpi + (warp - 2) * 4096;
+        uint32_t acc[2][32];
         float gs = 1.0f;
         if (KIND == G_NVFP4) gs = __fmul_rn(*p.g_a, *p.g_w);
         int tcount = 0;
@@ -687,15 +758,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             tc_fence_after();
             const uint32_t taddr =
                 tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * C::ACC1_COL) + (uint32_t)(h * 128);
-            const int row = mb * 256 + (int)rank * 128 + q * 32 + lane;
+            const int row0 = mb * 256 + (int)rank * 128 + q * 32;
+            const int row = row0 + lane;
             const int col0 = nb * GEMM_BN + h * 128;
+            // pack 64 columns into the staging tile and hand them to one TMA store (which
+            // clips rows at or beyond M); the tile is reused once the previous store has read it
+            auto stage_store = [&](int chunk) {
+                if (col0 >= p.N) return;
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+                epilogue_stage<KIND>(p, acc, row, col0 + chunk * 32, gs, stile, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && row0 < p.M) {
+                    tma_store_2d(&tmY, stile, col0 + chunk * 32, row0);
+                    bulk_commit_group();
+                }
+            };
             // the 64 columns shared by both accumulators are tile columns 192..255 of
             // accumulator 0 (half 1, chunks 2-3) or 0..63 of accumulator 1 (half 0, chunks 0-1):
             // their holders drain them first and release them
             const bool holds_overlap = (h == (b == 0 ? 1 : 0));
             const int first = holds_overlap ? (b == 0 ? 2 : 0) : 0;
             const int second = 2 - first;
-            uint32_t acc[2][32];
             tmem_ld_32x32b_x32(taddr + first * 32, acc[0]);
             tmem_ld_32x32b_x32(taddr + (first + 1) * 32, acc[1]);
             tmem_wait_ld();
@@ -704,15 +789,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 __syncwarp();
                 if (lane == 0) arrive_leader_relaxed(ovl_free, rank);
             }
-            epilogue_store<KIND, 2>(p, acc, row, col0 + first * 32, gs);
+            stage_store(first);
             tmem_ld_32x32b_x32(taddr + second * 32, acc[0]);
             tmem_ld_32x32b_x32(taddr + (second + 1) * 32, acc[1]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) arrive_leader_relaxed(&acc_free[b], rank);
-            epilogue_store<KIND, 2>(p, acc, row, col0 + second * 32, gs);
+            stage_store(second);
         }
+        // the staging tile must outlive the stores that read it
+        if (lane == 0) bulk_wait_group0();
+        __syncwarp();
     }
 
     tc_fence_before();
