@@ -50,7 +50,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm-ctas", type=int, default=0, choices=[0, 1, 2],
-                    help="GEMM kernel: 0/1 the 1-CTA 128x256 tile (default), 2 the 2-CTA 256x256 tile")
+                    help="GEMM kernel: 0 auto (2-CTA 256x256 tile for M > 128), 1 force the 1-CTA 128x256 tile, 2 force 2-CTA")
     ap.add_argument("--m", type=int, default=75600,
                     help="tokens; smaller values run a reduced case of the same kernels (profiling only)")
     return ap.parse_args()
@@ -257,7 +257,7 @@ def native_arm(args):
 
     fb.lib()  # fails loudly if the CUDA library is missing
     fb.lib().fp4bsa_set_gemm_ctas(args.gemm_ctas)
-    pair = args.gemm_ctas == 2 and M > 128
+    pair = args.gemm_ctas != 1 and M > 128
     x_bits, w_bits, b_bits = make_inputs(rank)
     x = to_dev(x_bits, torch, torch.bfloat16)
     bias = to_dev(b_bits, torch, torch.float16)

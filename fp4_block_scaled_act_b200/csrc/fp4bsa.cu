@@ -19,7 +19,7 @@ namespace {
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 uint64_t g_timeout_ns = kDefaultTimeoutNs;
 int g_skip_iter = -1;  // test hook, see fp4bsa_test_skip_iteration
-int g_gemm_ctas = 0;   // tuning hook: 0 auto (the 1-CTA kernel, fastest measured), 1 or 2 to force
+int g_gemm_ctas = 0;   // tuning hook: 0 auto (2-CTA kernel for M > 128), 1 or 2 to force
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -290,8 +290,9 @@ fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf
         return FP4_ERR_MISALIGNED;
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;
-    // 1-CTA 128x256 tiles unless the 2-CTA 256x256 kernel is forced (tuning hook)
-    const bool pair = g_gemm_ctas == 2 && M > GEMM_BM;
+    // 2-CTA 256x256 tiles (faster at every M measured) unless M fits one 128-row tile or
+    // the 1-CTA kernel is forced (tuning hook)
+    const bool pair = g_gemm_ctas != 1 && M > GEMM_BM;
     // the 2-CTA NVFP4 kernel stages 128 K (64 bytes per row, 64-byte swizzle)
     const uint32_t box_inner = (pair && nv) ? 64 : 128;
     const CUtensorMapSwizzle swz = (pair && nv) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
@@ -362,7 +363,7 @@ fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const float* 
         return FP4_ERR_MISALIGNED;
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;
-    const bool pair = g_gemm_ctas == 2 && M > GEMM_BM;
+    const bool pair = g_gemm_ctas != 1 && M > GEMM_BM;
     CUtensorMap ta, tb;
     if ((s = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_e4m3, K, M, K, 128, GEMM_BM)) != FP4_OK) return s;
     // packed E2M1 in global memory, unpacked to one 16-byte slot per 16 values in shared memory
@@ -467,8 +468,8 @@ fp4_status_t fp4_linear_noalloc(fp4_fmt_t fmt, const void* x_bf16, int64_t M, in
                       (size_t)FP4_NOALLOC_SCRATCH_BYTES, stream);
 }
 
-// Tuning hook (not in the public header): 0 or 1 use the 1-CTA 128x256 kernel, 2 the
-// 2-CTA 256x256 kernel (for M > 128).
+// Tuning hook (not in the public header): 1 forces the 1-CTA 128x256 kernel; 0 (default)
+// and 2 use the 2-CTA 256x256 kernel whenever M > 128.
 void fp4bsa_set_gemm_ctas(int ctas) { g_gemm_ctas = (ctas == 1 || ctas == 2) ? ctas : 0; }
 
 // Test hook (not in the public header): the GEMM producer skips the given k-iteration of

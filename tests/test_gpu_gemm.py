@@ -6,6 +6,8 @@ tiles, ragged M and N tails, odd K stages); at the full Wan2.2 sizes, in the lau
 configuration the benchmark times, sampled rows (including every row of the ragged
 last tile) are checked the same way.
 """
+import contextlib
+
 import numpy as np
 import pytest
 
@@ -167,8 +169,9 @@ def test_linear_full_size_sampled(fb, orc, cfg, fmt, M, K, N, kind):
 # ------------------------------------------------------------------ bounded waits
 @pytest.mark.parametrize("M", [128, 256])
 def test_bounded_wait_reports_timeout(fb, orc, M):
-    """A k-stage that is never filled (test hook) makes the MMA warp's wait run out; the
-    kernel returns, the status word reads FP4_ERR_TIMEOUT, and the next call is correct."""
+    """A k-stage that is never filled (test hook) makes the kernel's bounded wait run out
+    (M = 128: 1-CTA kernel, M = 256: 2-CTA kernel); the kernel returns, the status word
+    reads FP4_ERR_TIMEOUT, and the next call is correct."""
     import torch
 
     K, N = 512, 256
@@ -227,59 +230,65 @@ def test_w4a8_full_size_sampled(fb, orc):
     _w4a8_check(fb, orc, M, K, N, seed=3001, rows=rows, calib=2048)
 
 
-# ------------------------------------------------------------------ 2-CTA kernel (tuning hook)
+# ------------------------------------------------------------------ each GEMM kernel, forced
+# The library picks the cta_group::2 256x256 kernel for M > 128 and the 1-CTA 128x256
+# kernel otherwise; a tuning hook forces either, so both stay covered on ragged shapes.
+@contextlib.contextmanager
+def _gemm_ctas(fb, ctas):
+    L = fb.lib()
+    L.fp4bsa_set_gemm_ctas(ctas)
+    try:
+        yield L
+    finally:
+        L.fp4bsa_set_gemm_ctas(0)
+
+
+@pytest.mark.parametrize("ctas", [1, 2])
 @pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("M,K,N", [(129, 512, 384), (300, 768, 512), (600, 1280, 1024)])
-def test_pair_kernel_all_elements(fb, orc, fmt, M, K, N):
-    """The cta_group::2 256x256 kernel (reachable through the tuning hook) on ragged shapes."""
-    L = fb.lib()
+def test_each_kernel_all_elements(fb, orc, ctas, fmt, M, K, N):
     x = synth.activation(40 * M + K, M, K, "lognormal")
     w = synth.weight(50 * N + K, N, K)
     b = synth.bias(N + 9, N)
     g_a = orc.nv_global(orc.tensor_amax(x)) if fmt == NV else None
-    try:
-        L.fp4bsa_set_gemm_ctas(2)
+    with _gemm_ctas(fb, ctas):
         y = _run_linear(fb, fmt, x, w, b, g_a)
-    finally:
-        L.fp4bsa_set_gemm_ctas(0)
     rows = np.arange(M)
     Y, S = _oracle(orc, fmt, x, w, b, rows, g_a)
-    H.check_linear(y, Y, S, rows, f"pair fmt={fmt} M={M} K={K} N={N}")
+    H.check_linear(y, Y, S, rows, f"ctas={ctas} fmt={fmt} M={M} K={K} N={N}")
 
 
-def test_pair_kernel_w4a8(fb, orc):
-    L = fb.lib()
-    try:
-        L.fp4bsa_set_gemm_ctas(2)
+@pytest.mark.parametrize("ctas", [1, 2])
+def test_each_kernel_w4a8(fb, orc, ctas):
+    with _gemm_ctas(fb, ctas):
         _w4a8_check(fb, orc, 300, 1024, 512, seed=7777)
-    finally:
-        L.fp4bsa_set_gemm_ctas(0)
 
 
-def test_pair_kernel_timeout(fb, orc):
+@pytest.mark.parametrize("ctas", [1, 2])
+def test_each_kernel_timeout(fb, orc, ctas):
+    """A stage that is never filled makes the kernel's bounded wait run out; the status
+    word reads FP4_ERR_TIMEOUT and the next call on the same context is correct."""
     import torch
 
     M, K, N = 256, 512, 256
     x = synth.activation(13, M, K, "lognormal")
     w = synth.weight(14, N, K)
     xd, pw = H.dev_bf16(x), fb.pack_weight(H.dev_bf16(w), MX)
-    L = fb.lib()
     assert fb.fp4_sync_status() == 0
-    try:
-        L.fp4bsa_set_gemm_ctas(2)
-        fb.fp4_set_wait_timeout_ns(2_000_000)
-        L.fp4bsa_test_skip_iteration(1)
-        fb.linear(xd, pw)
-        st = fb.fp4_sync_status()
-        L.fp4bsa_test_skip_iteration(-1)
-        fb.fp4_set_wait_timeout_ns(0)
-        y = fb.linear(xd, pw)
-        st2 = fb.fp4_sync_status()
-    finally:
-        L.fp4bsa_test_skip_iteration(-1)
-        fb.fp4_set_wait_timeout_ns(0)
-        L.fp4bsa_set_gemm_ctas(0)
+    with _gemm_ctas(fb, ctas) as L:
+        try:
+            fb.fp4_set_wait_timeout_ns(2_000_000)
+            L.fp4bsa_test_skip_iteration(1)
+            fb.linear(xd, pw)
+            st = fb.fp4_sync_status()
+            L.fp4bsa_test_skip_iteration(-1)
+            fb.fp4_set_wait_timeout_ns(0)
+            y = fb.linear(xd, pw)
+            st2 = fb.fp4_sync_status()
+        finally:
+            L.fp4bsa_test_skip_iteration(-1)
+            fb.fp4_set_wait_timeout_ns(0)
     assert fb.fp4_status_string(st) == "FP4_ERR_TIMEOUT" and st2 == 0
     torch.cuda.synchronize()
     Y, S = orc.fp4_linear_rows(MX, x, w, None, np.arange(M))
-    H.check_linear(y, Y, S, np.arange(M), "pair after timeout")
+    H.check_linear(y, Y, S, np.arange(M), f"ctas={ctas} after timeout")
