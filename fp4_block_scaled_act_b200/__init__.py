@@ -6,8 +6,8 @@ stream becomes the stream argument, and a non-OK status raises FP4Error.  All
 arithmetic runs in the library's CUDA kernels.  There is no fallback: if the
 library is missing or the device is not sm_100, the calls raise.
 
-The helpers at the end (pack_weight, linear, w4a8_linear) allocate outputs and
-workspaces with torch and call the same entry points.
+The helpers at the end (pack_weight, quantize_act, linear, pack_lowrank_up, w4a8_linear)
+allocate outputs and workspaces with torch and call the same entry points.
 """
 from __future__ import annotations
 
@@ -30,7 +30,7 @@ EXPORTS = [
     "fp4_codes_bytes", "fp4_sf_bytes", "fp4_linear_workspace_bytes", "w4a8_workspace_bytes",
     "fp4_tensor_amax", "fp4_pack_weight", "fp4_quantize_act", "fp4_gemm", "fp4_linear",
     "w4a8_quantize_act", "w4a8_gemm", "w4a8_svd_linear", "fp4_sync_status", "fp4_status_string",
-    "fp4_set_wait_timeout_ns", "fp4_linear_noalloc",
+    "fp4_set_wait_timeout_ns", "fp4_linear_noalloc", "w4a8_pack_lowrank_up",
 ]
 
 
@@ -64,6 +64,7 @@ def lib():
             "fp4_linear": (I, [I, P, I64, I64, I64, P, P, P, P, P, P, P, SZ, P]),
             "fp4_linear_noalloc": (I, [I, P, I64, I64, I64, P, P, P, P, P, P, P]),
             "w4a8_quantize_act": (I, [P, I64, I64, P, I, P, P, P, P]),
+            "w4a8_pack_lowrank_up": (I, [P, I64, I, P, P]),
             "w4a8_gemm": (I, [P, P, P, I64, I64, I64, P, P, P, I, P, P, P]),
             "w4a8_svd_linear": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, P, SZ, P]),
             "fp4_sync_status": (I, [P]),
@@ -162,19 +163,24 @@ def fp4_linear_noalloc(fmt, x, M: int, K: int, N: int, w_codes, w_sf, w_global, 
                                     _ptr(a_global), _ptr(bias), _ptr(y), _stream(stream)), "fp4_linear_noalloc")
 
 
-def w4a8_quantize_act(x, M: int, K: int, l1, rank: int, x_e4m3, x_sf, u, stream=None):
-    _check(lib().w4a8_quantize_act(_ptr(x), M, K, _ptr(l1), rank, _ptr(x_e4m3), _ptr(x_sf), _ptr(u),
+def w4a8_quantize_act(x, M: int, K: int, l1, rank: int, x_e4m3, x_sf, u_pair, stream=None):
+    _check(lib().w4a8_quantize_act(_ptr(x), M, K, _ptr(l1), rank, _ptr(x_e4m3), _ptr(x_sf), _ptr(u_pair),
                                    _stream(stream)), "w4a8_quantize_act")
 
 
-def w4a8_gemm(x_e4m3, x_sf, u, M: int, K: int, N: int, r_codes, r_sf, l2, rank: int, bias, y, stream=None):
-    _check(lib().w4a8_gemm(_ptr(x_e4m3), _ptr(x_sf), _ptr(u), M, K, N, _ptr(r_codes), _ptr(r_sf), _ptr(l2),
-                           rank, _ptr(bias), _ptr(y), _stream(stream)), "w4a8_gemm")
+def w4a8_pack_lowrank_up(l2, N: int, rank: int, l2t, stream=None):
+    _check(lib().w4a8_pack_lowrank_up(_ptr(l2), N, rank, _ptr(l2t), _stream(stream)), "w4a8_pack_lowrank_up")
 
 
-def w4a8_svd_linear(x, M: int, K: int, N: int, r_codes, r_sf, l1, l2, rank: int, bias, y, workspace,
+def w4a8_gemm(x_e4m3, x_sf, u_pair, M: int, K: int, N: int, r_codes, r_sf, l2t, rank: int, bias, y,
+              stream=None):
+    _check(lib().w4a8_gemm(_ptr(x_e4m3), _ptr(x_sf), _ptr(u_pair), M, K, N, _ptr(r_codes), _ptr(r_sf),
+                           _ptr(l2t), rank, _ptr(bias), _ptr(y), _stream(stream)), "w4a8_gemm")
+
+
+def w4a8_svd_linear(x, M: int, K: int, N: int, r_codes, r_sf, l1, l2t, rank: int, bias, y, workspace,
                     ws_bytes: int, stream=None):
-    _check(lib().w4a8_svd_linear(_ptr(x), M, K, N, _ptr(r_codes), _ptr(r_sf), _ptr(l1), _ptr(l2), rank,
+    _check(lib().w4a8_svd_linear(_ptr(x), M, K, N, _ptr(r_codes), _ptr(r_sf), _ptr(l1), _ptr(l2t), rank,
                                  _ptr(bias), _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
            "w4a8_svd_linear")
 
@@ -243,8 +249,19 @@ def linear(x, pw: PackedWeight, bias=None, a_global=None, y=None, workspace=None
     return y
 
 
-def w4a8_linear(x, r: PackedWeight, l1, l2, bias=None, y=None, workspace=None, stream=None):
-    """W4A8 SVDQuant linear: bf16 [M, K] -> bf16 [M, N] (MXFP4 residual r, rank-32 L1/L2)."""
+def pack_lowrank_up(l2, stream=None):
+    """bf16 [rank, N] low-rank up-projection (CUDA) -> packed bf16 [N, rank] for the GEMM."""
+    import torch
+
+    rank, N = l2.shape
+    l2t = torch.empty((N, rank), dtype=torch.bfloat16, device=l2.device)
+    w4a8_pack_lowrank_up(l2, N, rank, l2t, stream)
+    return l2t
+
+
+def w4a8_linear(x, r: PackedWeight, l1, l2t, bias=None, y=None, workspace=None, stream=None):
+    """W4A8 SVDQuant linear: bf16 [M, K] -> bf16 [M, N] (MXFP4 residual r, rank-32 L1 [K, rank]
+    and packed L2 [N, rank] from pack_lowrank_up)."""
     import torch
 
     M, K = x.shape
@@ -253,5 +270,5 @@ def w4a8_linear(x, r: PackedWeight, l1, l2, bias=None, y=None, workspace=None, s
         y = torch.empty((M, r.N), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
         workspace = torch.empty(w4a8_workspace_bytes(M, K, r.N, rank), dtype=torch.uint8, device=x.device)
-    w4a8_svd_linear(x, M, K, r.N, r.codes, r.sf, l1, l2, rank, bias, y, workspace, workspace.numel(), stream)
+    w4a8_svd_linear(x, M, K, r.N, r.codes, r.sf, l1, l2t, rank, bias, y, workspace, workspace.numel(), stream)
     return y

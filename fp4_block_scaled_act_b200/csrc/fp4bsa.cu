@@ -71,8 +71,6 @@ fp4_status_t device_state(DeviceState** out) {
                                      GemmCfg<G_MXFP4>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm_kernel<G_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      GemmCfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess ||
-                cudaFuncSetAttribute(gemm_kernel<G_W4A8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     GemmCfg<G_W4A8>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm2_kernel<G_MXFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Gemm2Cfg<G_MXFP4>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm2_kernel<G_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -180,9 +178,11 @@ fp4_status_t encode_sf(CUtensorMap* m, const uint8_t* sf, int64_t rows, int64_t 
 }
 
 // 2-CTA GEMM: A box 128 rows, B box 128 rows (half of the 256-wide N tile) per CTA.
+// tu / tl: the W4A8 low-rank operands (u pair, packed L2); other kinds pass any map.
 template <int KIND>
 fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CUtensorMap& tb, const uint8_t* sfa,
-                          const uint8_t* sfb, GemmParams& p, cudaStream_t st) {
+                          const uint8_t* sfb, GemmParams& p, cudaStream_t st, const CUtensorMap* tu = nullptr,
+                          const CUtensorMap* tl = nullptr) {
     using C = Gemm2Cfg<KIND>;
     CUtensorMap tsa, tsb;
     fp4_status_t s;
@@ -198,7 +198,8 @@ fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CU
     p.timeout_ns = g_timeout_ns;
     p.skip_iter = g_skip_iter;
     p.status = ds->status;
-    gemm2_kernel<KIND><<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, ty, p);
+    gemm2_kernel<KIND><<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, ty, tu ? *tu : ta,
+                                                                   tl ? *tl : tb, p);
     return launched();
 }
 
@@ -334,67 +335,83 @@ fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K,
 }
 
 fp4_status_t w4a8_quantize_act(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16, int rank,
-                               uint8_t* x_e4m3, uint8_t* x_sf, float* u_f32, void* stream) {
-    if (!x_bf16 || !l1_bf16 || !x_e4m3 || !x_sf || !u_f32 || rank != 32) return FP4_ERR_INVALID_ARG;
+                               uint8_t* x_e4m3, uint8_t* x_sf, void* u_pair, void* stream) {
+    if (!x_bf16 || !l1_bf16 || !x_e4m3 || !x_sf || !u_pair || rank != 32) return FP4_ERR_INVALID_ARG;
     fp4_status_t s = check_shape(M, K, 128);
     if (s != FP4_OK) return s;
-    if (!aligned16(x_bf16) || !aligned16(l1_bf16) || !aligned16(x_e4m3) || !aligned16(x_sf) || !aligned16(u_f32))
+    if (!aligned16(x_bf16) || !aligned16(l1_bf16) || !aligned16(x_e4m3) || !aligned16(x_sf) || !aligned16(u_pair))
         return FP4_ERR_MISALIGNED;
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((s = launch_quant(ds, Q_MXFP8, x_bf16, M, K, nullptr, x_e4m3, x_sf, st)) != FP4_OK) return s;
-    const int blocks = (int)((M + 31) / 32);
-    lowrank_down_kernel<32><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x_bf16),
-                                                   static_cast<const __nv_bfloat16*>(l1_bf16), M, K, u_f32);
+    const int blocks = (int)((M + LR_ROWS - 1) / LR_ROWS);
+    lowrank_down_kernel<<<blocks, LR_THREADS, 0, st>>>(static_cast<const __nv_bfloat16*>(x_bf16),
+                                                       static_cast<const __nv_bfloat16*>(l1_bf16), (int)M, (int)K,
+                                                       static_cast<__nv_bfloat16*>(u_pair));
     return launched();
 }
 
-fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const float* u_f32, int64_t M, int64_t K,
-                       int64_t N, const uint8_t* r_codes, const uint8_t* r_sf, const void* l2_bf16, int rank,
+fp4_status_t w4a8_pack_lowrank_up(const void* l2_bf16, int64_t N, int rank, void* l2t_bf16, void* stream) {
+    if (!l2_bf16 || !l2t_bf16 || rank != 32) return FP4_ERR_INVALID_ARG;
+    if (N < 128 || N % 128 != 0 || N >= kMaxDim) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(l2_bf16) || !aligned16(l2t_bf16)) return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    fp4_status_t s = device_state(&ds);
+    if (s != FP4_OK) return s;
+    transpose_rank_kernel<<<(int)(N / 128), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16*>(l2_bf16), (int)N, static_cast<__nv_bfloat16*>(l2t_bf16));
+    return launched();
+}
+
+fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const void* u_pair, int64_t M, int64_t K,
+                       int64_t N, const uint8_t* r_codes, const uint8_t* r_sf, const void* l2t_bf16, int rank,
                        const void* bias_f16, void* y_bf16, void* stream) {
-    if (!x_e4m3 || !x_sf || !u_f32 || !r_codes || !r_sf || !l2_bf16 || !y_bf16 || rank != 32)
+    if (!x_e4m3 || !x_sf || !u_pair || !r_codes || !r_sf || !l2t_bf16 || !y_bf16 || rank != 32)
         return FP4_ERR_INVALID_ARG;
     fp4_status_t s = check_shape(M, K, N);
     if (s != FP4_OK) return s;
     // the unpacking tensor map needs a 32-byte aligned residual-weight base
-    if (!aligned16(x_e4m3) || !aligned16(x_sf) || !aligned16(u_f32) || (reinterpret_cast<uintptr_t>(r_codes) & 31u) ||
-        !aligned16(r_sf) || !aligned16(l2_bf16) || !aligned16(bias_f16) || !aligned16(y_bf16))
+    if (!aligned16(x_e4m3) || !aligned16(x_sf) || !aligned16(u_pair) || (reinterpret_cast<uintptr_t>(r_codes) & 31u) ||
+        !aligned16(r_sf) || !aligned16(l2t_bf16) || !aligned16(bias_f16) || !aligned16(y_bf16))
         return FP4_ERR_MISALIGNED;
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;
-    const bool pair = g_gemm_ctas != 1 && M > GEMM_BM;
-    CUtensorMap ta, tb;
+    // always the 2-CTA kernel: its low-rank stage runs on the tensor core
+    CUtensorMap ta, tb, tu, tl;
     if ((s = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_e4m3, K, M, K, 128, GEMM_BM)) != FP4_OK) return s;
     // packed E2M1 in global memory, unpacked to one 16-byte slot per 16 values in shared memory
-    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, r_codes, K, N, K / 2, 128,
-                       pair ? 128 : GEMM_BN)) != FP4_OK)
+    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, r_codes, K, N, K / 2, 128, 128)) != FP4_OK)
+        return s;
+    // u pair [M, 64] bf16 (128-byte rows) and packed L2 [N, 32] bf16 (64-byte rows)
+    if ((s = encode_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, u_pair, 2 * (uint64_t)rank, M, 4 * (uint64_t)rank,
+                       2 * rank, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
+        return s;
+    if ((s = encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l2t_bf16, (uint64_t)rank, N, 2 * (uint64_t)rank, rank,
+                       128, CU_TENSOR_MAP_SWIZZLE_64B)) != FP4_OK)
         return s;
     GemmParams p{};
     p.M = (int)M, p.N = (int)N, p.K = (int)K;
     p.sfa = x_sf, p.sfb = r_sf;
     p.bias = static_cast<const __half*>(bias_f16);
     p.y = static_cast<__nv_bfloat16*>(y_bf16);
-    p.u = u_f32;
-    p.l2 = static_cast<const __nv_bfloat16*>(l2_bf16);
-    if (pair) return launch_gemm2<G_W4A8>(ds, ta, tb, x_sf, r_sf, p, static_cast<cudaStream_t>(stream));
-    return launch_gemm<G_W4A8>(ds, ta, tb, p, static_cast<cudaStream_t>(stream));
+    return launch_gemm2<G_W4A8>(ds, ta, tb, x_sf, r_sf, p, static_cast<cudaStream_t>(stream), &tu, &tl);
 }
 
 fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N, const uint8_t* r_codes,
-                             const uint8_t* r_sf, const void* l1_bf16, const void* l2_bf16, int rank,
+                             const uint8_t* r_sf, const void* l1_bf16, const void* l2t_bf16, int rank,
                              const void* bias_f16, void* y_bf16, void* workspace, size_t ws_bytes, void* stream) {
     if (!workspace || rank != 32) return FP4_ERR_INVALID_ARG;
     fp4_status_t s = check_shape(M, K, N);
     if (s != FP4_OK) return s;
     if (ws_bytes < w4a8_workspace_bytes(M, K, N, rank)) return FP4_ERR_WORKSPACE;
     if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
-    if (!r_codes || !r_sf || !l2_bf16 || !y_bf16) return FP4_ERR_INVALID_ARG;
+    if (!r_codes || !r_sf || !l2t_bf16 || !y_bf16) return FP4_ERR_INVALID_ARG;
     uint8_t* xe = static_cast<uint8_t*>(workspace);
     uint8_t* xs = xe + align256((size_t)M * K);
-    float* u = reinterpret_cast<float*>(xs + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K)));
+    uint8_t* u = xs + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K));
     if ((s = w4a8_quantize_act(x_bf16, M, K, l1_bf16, rank, xe, xs, u, stream)) != FP4_OK) return s;
-    return w4a8_gemm(xe, xs, u, M, K, N, r_codes, r_sf, l2_bf16, rank, bias_f16, y_bf16, stream);
+    return w4a8_gemm(xe, xs, u, M, K, N, r_codes, r_sf, l2t_bf16, rank, bias_f16, y_bf16, stream);
 }
 
 fp4_status_t fp4_sync_status(void* stream) {

@@ -65,8 +65,6 @@ struct GemmParams {
     const float* g_w;
     const __half* bias;       // [N] or null
     __nv_bfloat16* y;         // [M, N]
-    const float* u;           // W4A8: [M, 32] fp32
-    const __nv_bfloat16* l2;  // W4A8: [32, N] bf16
     uint64_t timeout_ns;
     int skip_iter;            // test hook: producer skips this k-iteration (-1: none)
     int* status;              // device status word
@@ -77,36 +75,12 @@ FP4_DEV void gemm_fail(const GemmParams& p, volatile int* abort) {
     atomicCAS(p.status, 0, STATUS_TIMEOUT);
 }
 
-// Add the W4A8 low-rank term, scale, add bias and round to bf16 NC x 32 columns of one
-// output row held in registers (acc[c][j] = column col0 + 32c + j, fp32 bits; row < M).
+// Scale, add bias and round to bf16 NC x 32 columns of one output row held in registers
+// (acc[c][j] = column col0 + 32c + j, fp32 bits; row < M).  The W4A8 low-rank term is
+// already in the accumulator (a tensor-core stage of the pair kernel).
 // On return acc[c][w], w < 16, holds columns 32c + 2w and 32c + 2w + 1 as a bf16 pair.
 template <int KIND, int NC>
 FP4_DEV void epilogue_pack(const GemmParams& p, uint32_t (&acc)[NC][32], int row, int col0, float gs) {
-    const int N = p.N;
-    if (KIND == G_W4A8) {
-        // acc += u[row, r] * L2[r, cols] for r = 0..31, one rank at a time (fp32 FMAs)
-        const float* urow = p.u + (size_t)row * 32;
-#pragma unroll 1
-        for (int r = 0; r < 32; ++r) {
-            const float ur = urow[r];
-            const __nv_bfloat16* l2r = p.l2 + (size_t)r * N + col0;
-#pragma unroll
-            for (int c = 0; c < NC; ++c) {
-#pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    const uint4 lv = *reinterpret_cast<const uint4*>(l2r + c * 32 + j);
-                    const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        acc[c][j + 2 * i] = __float_as_uint(
-                            __fmaf_rn(ur, __uint_as_float(lw[i] << 16), __uint_as_float(acc[c][j + 2 * i])));
-                        acc[c][j + 2 * i + 1] = __float_as_uint(__fmaf_rn(
-                            ur, __uint_as_float(lw[i] & 0xFFFF0000u), __uint_as_float(acc[c][j + 2 * i + 1])));
-                    }
-                }
-            }
-        }
-    }
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
 #pragma unroll
@@ -436,6 +410,12 @@ struct Gemm2Cfg {
     static constexpr int SF_COLS = SFA_COLS + 8 * ATOMS;  // B: 8 columns per atom
     static constexpr int TB = (64 / SF_COLS) >= 4 ? 4 : (64 / SF_COLS);  // scale buffers
     static constexpr int THREADS = 480;
+    // W4A8 low-rank stage (one per tile, after the K stages): A = the u pair, 128 rows x 64
+    // bf16 (128-byte rows, 128-byte swizzle); B = packed L2, 128 rows x 32 bf16 (64-byte
+    // rows, 64-byte swizzle); four kind::f16 MMAs of K = 16 (u_hi x L2, then u_lo x L2).
+    static constexpr uint32_t LR_TX = 128 * 128 + 128 * 64;
+    static constexpr uint32_t IDESC_LR = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
+                                         ((uint32_t)(256 >> 4) << 24);
     static constexpr uint32_t IDESC = (C1::A_FMT << 7) | (C1::B_FMT << 10) | ((uint32_t)(256 >> 3) << 17) |
                                       (C1::SCALE_FMT << 23) | ((uint32_t)(256 >> 4) << 24);
     static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -482,7 +462,8 @@ template <int KIND>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THREADS, 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                 const __grid_constant__ CUtensorMap tmY, GemmParams p) {
+                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmU,
+                 const __grid_constant__ CUtensorMap tmL, GemmParams p) {
     using C = Gemm2Cfg<KIND>;
     constexpr int S = C::STAGES;
     constexpr int TB = C::TB;
@@ -532,6 +513,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         prefetch_tmap(&tmSFA);
         prefetch_tmap(&tmSFB);
         prefetch_tmap(&tmY);
+        if (KIND == G_W4A8) {
+            prefetch_tmap(&tmU);
+            prefetch_tmap(&tmL);
+        }
     }
     __syncwarp();
     if (warp == 1) {
@@ -549,6 +534,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
     const int num_n = (N + 255) / 256;
     const int num_tiles = num_m * num_n;
     const int num_kb = (K + C::BK - 1) / C::BK;
+    // stages per tile: the K blocks, then (W4A8) the low-rank stage kb == num_kb
+    const int spt = num_kb + (KIND == G_W4A8 ? 1 : 0);
     const int apr = K / (C::G * 4);  // scale atoms per 128-row block
     const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
 
@@ -561,7 +548,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
                 const int mb = tile / num_n, nb = tile % num_n;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = 0; kb < spt; ++kb, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (uint32_t)(it / S) & 1u;
                     if (!mbar_wait(&empty[s], ph ^ 1u, p.timeout_ns, abort)) {
@@ -572,6 +559,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                     if (it == p.skip_iter) continue;  // test hook: this stage is never filled
                     // A/B of both CTAs land on the leader's barrier; only the leader expects them
                     const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+                    if (KIND == G_W4A8 && kb == num_kb) {
+                        // low-rank stage: u pair rows and packed-L2 rows; no scale atoms, but
+                        // sf_full still completes a phase so its parity keeps counting stages
+                        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::LR_TX);
+                        mbar_arrive(&sf_full[s]);
+                        tma_load_2d_pair(sA + s * C::A_BYTES, &tmU, bar, 0, mb * 256 + (int)rank * 128, pol_a);
+                        tma_load_2d_pair(sB + s * C::B_BYTES, &tmL, bar, 0, nb * 256 + (int)rank * 128, pol_b);
+                        continue;
+                    }
                     if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::AB_TX);
                     mbar_arrive_expect_tx(&sf_full[s], C::SF_TX);
                     // x: bytes of the row for packed FP4 and E4M3, elements for the W4A8 unpacking map
@@ -603,7 +599,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         int it = 0;
         bool ok = true;
         for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+            for (int kb = 0; kb < spt; ++kb, ++it) {
                 const int s = it % S;
                 const int t = it % TB;
                 bool got = mbar_wait(&sf_full[s], (uint32_t)(it / S) & 1u, p.timeout_ns, abort);
@@ -637,7 +633,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 }
                 const uint32_t xa = C::SF_COL0 + (uint32_t)(t * C::SF_COLS);
                 const uint32_t xb = xa + C::SFA_COLS;
-                if constexpr (C::ATOMS == 2) {
+                // the W4A8 low-rank stage reads no scales: its buffer turn passes unwritten
+                if (KIND == G_W4A8 && kb == num_kb) {
+                } else if constexpr (C::ATOMS == 2) {
                     tmem_st_32x32b_x8(tlane + xa, va);
                     tmem_st_32x32b_x16(tlane + xb, vb);
                 } else {
@@ -664,9 +662,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++tcount) {
                 const int b = tcount & 1;
                 const uint32_t dacc = tmem_base + (uint32_t)(b * C::ACC1_COL);
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = 0; kb < spt; ++kb, ++it) {
                     named_bar_sync(1u + it % TB, 64u);
-                    if (lane == 0) {
+                    if (lane == 0 && KIND == G_W4A8 && kb == num_kb) {
+                        // low-rank stage: acc += u_hi L2 + u_lo L2 (bf16 x bf16 -> fp32)
+                        tc_fence_after();
+                        const int s = (int)(it % S);
+                        const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
+                        const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t adesc = smem_desc(a_base + k * 32, 0, 1024, 2u);
+                            const uint64_t bdesc = smem_desc(b_base + (k & 1) * 32, 0, 512, 4u);
+                            mma2_f16(dacc, adesc, bdesc, C::IDESC_LR, 1u);
+                        }
+                        tc_commit_pair(&empty[s], 0x3);
+                    } else if (lane == 0) {
                         tc_fence_after();
                         const int s = (int)(it % S);
                         const int t = (int)(it % TB);
@@ -725,7 +736,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 // accumulator b drained (tile tcount-2) and the overlap of tile tcount-1 drained
                 bool got = mbar_wait(&acc_free[b], (((uint32_t)tcount >> 1) & 1u) ^ 1u, p.timeout_ns, abort);
                 if (got && tcount > 0) got = mbar_wait(ovl_free, (uint32_t)(tcount - 1) & 1u, p.timeout_ns, abort);
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = 0; kb < spt; ++kb, ++it) {
                     if (got) got = mbar_wait(&full[it % S], (it / S) & 1u, p.timeout_ns, abort);
                     if (got) got = mbar_wait(&sf_ready[it % TB], (it / TB) & 1u, p.timeout_ns, abort);
                     got = __all_sync(0xffffffffu, got);

@@ -359,6 +359,14 @@ FP4_DEV void mma2_mxf8f6f4_block32(uint32_t d, uint64_t a, uint64_t b, uint32_t 
         "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
         : "memory");
 }
+// Dense bf16 x bf16 -> fp32 MMA of the pair (kind::f16, K = 16 per instruction).
+FP4_DEV void mma2_f16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
 // arrive on the mbarrier at the same shared-memory offset in every CTA of `cta_mask`
 // once all tcgen05 operations issued so far by this thread are complete
 FP4_DEV void tc_commit_pair(uint64_t* bar, uint16_t cta_mask) {

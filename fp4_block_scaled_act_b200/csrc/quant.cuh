@@ -192,45 +192,129 @@ __global__ void nv_global_kernel(float* g) {
 }
 
 // ---------------------------------------------------------------- low-rank down-projection
-// u[m, r] = sum_k x[m, k] * L1[k, r] in fp32, fixed summation order (k ascending), for the
-// W4A8 SVDQuant linear.  Block: 256 threads, 32 rows x RANK outputs; K staged in chunks.
-template <int RANK>
-__global__ void __launch_bounds__(256) lowrank_down_kernel(const __nv_bfloat16* __restrict__ x,
-                                                           const __nv_bfloat16* __restrict__ l1, int64_t M,
-                                                           int64_t K, float* __restrict__ u) {
-    constexpr int ROWS = 32, KC = 64;
-    constexpr int RPT = ROWS * RANK / 256;  // rows per thread
-    __shared__ float xs[ROWS][KC + 1];
-    __shared__ float ls[KC][RANK];
-    const int r = threadIdx.x % RANK;
-    const int rg = threadIdx.x / RANK;  // 0 .. 256/RANK-1
-    const int64_t m0 = (int64_t)blockIdx.x * ROWS;
-    float acc[RPT];
+// W4A8 SVDQuant: u[m, r] = sum_k x[m, k] * L1[k, r] (rank 32) with bf16 inputs and fp32
+// accumulation, on the warp-level tensor-core MMA (mma.sync m16n8k16): a skinny,
+// HBM-bound contraction (the kernel is bound by reading X), for which the warp-level MMA
+// is ample.  The result is stored as a bf16 pair per value, hi = bf16(u), lo = bf16(u - hi)
+// (u_pair[m][r] = hi, u_pair[m][32 + r] = lo), so the GEMM can add u L2 on the tensor core
+// as u_hi L2 + u_lo L2 with |u - hi - lo| <= 2^-18 |u|.
+// Block: 256 threads = 8 warps x 16 rows = 128 rows, all 32 ranks; K in 64-element chunks,
+// double-buffered with cp.async.
+constexpr int LR_ROWS = 128, LR_THREADS = 256, LR_KC = 64;
+constexpr int LR_XP = LR_KC + 8;  // padded X row (elements): conflict-free ldmatrix
+constexpr int LR_LP = 32 + 8;     // padded L1 row
+
+FP4_DEV void cp_async16(void* dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+FP4_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+FP4_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__global__ void __launch_bounds__(LR_THREADS) lowrank_down_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                  const __nv_bfloat16* __restrict__ l1, int M,
+                                                                  int K, __nv_bfloat16* __restrict__ u_pair) {
+    __shared__ __align__(16) __nv_bfloat16 xs[2][LR_ROWS][LR_XP];
+    __shared__ __align__(16) __nv_bfloat16 ls[2][LR_KC][LR_LP];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int m0 = blockIdx.x * LR_ROWS;
+    const int nkc = K / LR_KC;
+
+    auto load = [&](int kc, int st) {
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) acc[i] = 0.0f;
-    for (int64_t k0 = 0; k0 < K; k0 += KC) {
-        for (int i = threadIdx.x; i < ROWS * KC; i += 256) {
-            const int rr = i / KC, kk = i % KC;
-            const int64_t m = m0 + rr;
-            xs[rr][kk] = (m < M) ? __bfloat162float(x[m * K + k0 + kk]) : 0.0f;
+        for (int i = 0; i < 4; ++i) {  // X: 128 rows x 8 pieces of 16 bytes
+            const int idx = tid + i * LR_THREADS;
+            const int row = idx >> 3, c = idx & 7;
+            const bool ok = m0 + row < M;
+            const __nv_bfloat16* src = ok ? x + (size_t)(m0 + row) * K + kc * LR_KC + c * 8 : x;
+            cp_async16(&xs[st][row][c * 8], src, ok);
         }
-        for (int i = threadIdx.x; i < KC * RANK; i += 256) {
-            const int kk = i / RANK, rr = i % RANK;
-            ls[kk][rr] = __bfloat162float(l1[(k0 + kk) * RANK + rr]);
+        {  // L1: 64 rows x 4 pieces of 16 bytes
+            const int row = tid >> 2, c = tid & 3;
+            cp_async16(&ls[st][row][c * 8], l1 + (size_t)(kc * LR_KC + row) * 32 + c * 8, true);
+        }
+        cp_async_commit();
+    };
+
+    float acc[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[j][e] = 0.0f;
+
+    load(0, 0);
+    for (int kc = 0; kc < nkc; ++kc) {
+        const int st = kc & 1;
+        if (kc + 1 < nkc) {
+            load(kc + 1, st ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
         __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < KC; ++kk) {
-            const float l = ls[kk][r];
 #pragma unroll
-            for (int i = 0; i < RPT; ++i) acc[i] = __fmaf_rn(xs[rg * RPT + i][kk], l, acc[i]);
+        for (int ks = 0; ks < LR_KC / 16; ++ks) {
+            uint32_t a[4];
+            const uint32_t aaddr = smem_u32(&xs[st][warp * 16 + (lane & 15)][ks * 16 + (lane >> 4) * 8]);
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                         : "r"(aaddr));
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t b[4];
+                const uint32_t baddr = smem_u32(&ls[st][ks * 16 + (lane & 15)][np * 16 + (lane >> 4) * 8]);
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
+                             : "r"(baddr));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float* d = acc[np * 2 + h];
+                    asm volatile(
+                        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                        "{%8, %9}, {%0, %1, %2, %3};"
+                        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[2 * h]), "r"(b[2 * h + 1]));
+                }
+            }
         }
         __syncthreads();
     }
+    // accumulator fragment: acc[j][0..1] -> row lane/4, acc[j][2..3] -> row lane/4 + 8,
+    // columns 8j + 2(lane%4) + {0, 1}
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int64_t m = m0 + rg * RPT + i;
-        if (m < M) u[m * RANK + r] = acc[i];
+    for (int half = 0; half < 2; ++half) {
+        const int m = m0 + warp * 16 + (lane >> 2) + half * 8;
+        if (m >= M) continue;
+        __nv_bfloat16* row = u_pair + (size_t)m * 64;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = j * 8 + 2 * (lane & 3);
+            const float u0 = acc[j][2 * half], u1 = acc[j][2 * half + 1];
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(u0), h1 = __float2bfloat16_rn(u1);
+            const __nv_bfloat16 l0 = __float2bfloat16_rn(u0 - __bfloat162float(h0));
+            const __nv_bfloat16 l1v = __float2bfloat16_rn(u1 - __bfloat162float(h1));
+            *reinterpret_cast<__nv_bfloat162*>(row + c) = __halves2bfloat162(h0, h1);
+            *reinterpret_cast<__nv_bfloat162*>(row + 32 + c) = __halves2bfloat162(l0, l1v);
+        }
+    }
+}
+
+// W4A8: L2 [32, N] bf16 (rank-major) -> packed L2 [N, 32] bf16, the K-major operand of the
+// GEMM's low-rank stage.  Block: 128 columns.
+__global__ void __launch_bounds__(256) transpose_rank_kernel(const __nv_bfloat16* __restrict__ l2, int N,
+                                                             __nv_bfloat16* __restrict__ l2t) {
+    __shared__ __nv_bfloat16 t[32][128 + 2];
+    const int n0 = blockIdx.x * 128;
+    for (int i = threadIdx.x; i < 32 * 128; i += 256) {
+        const int r = i / 128, c = i % 128;
+        t[r][c] = l2[(size_t)r * N + n0 + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 32 * 128; i += 256) {
+        const int c = i / 32, r = i % 32;
+        l2t[(size_t)(n0 + c) * 32 + r] = t[r][c];
     }
 }
 

@@ -177,26 +177,37 @@ fp4_status_t fp4_linear_noalloc(fp4_fmt_t fmt, const void* x_bf16, int64_t M, in
  *   l1_bf16  (device) [K, rank] bf16 (proj_down with 1/s folded in)
  *   x_e4m3   (device, out) [M, K] E4M3 bytes
  *   x_sf     (device, out) fp4_sf_bytes(FP4_FMT_MXFP4, M, K) bytes (E8M0, per 32)
- *   u_f32    (device, out) [M, rank] fp32, u = x L1 accumulated in fp32 */
+ *   u_pair   (device, out) [M, 2 * rank] bf16: u = x L1 accumulated in fp32, stored as
+ *            hi = bf16_rn(u) in columns [0, rank) and lo = bf16_rn(u - hi) in columns
+ *            [rank, 2 rank), so hi + lo equals u within 2^-18 |u| (M * rank * 4 bytes,
+ *            the size of an fp32 [M, rank] array). */
 fp4_status_t w4a8_quantize_act(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16,
-                               int rank, uint8_t* x_e4m3, uint8_t* x_sf, float* u_f32,
+                               int rank, uint8_t* x_e4m3, uint8_t* x_sf, void* u_pair,
                                void* stream);
+
+/* Offline pack of the low-rank up-projection for the GEMM (like fp4_pack_weight):
+ *   l2_bf16   (device) [rank, N] bf16 (proj_up, rank-major as the checkpoint stores it)
+ *   l2t_bf16  (device, out) [N, rank] bf16, the transpose.  N multiple of 128, rank 32. */
+fp4_status_t w4a8_pack_lowrank_up(const void* l2_bf16, int64_t N, int rank, void* l2t_bf16,
+                                  void* stream);
 
 /* W4A8 GEMM with low-rank epilogue: y = bf16_rn( sum_k deq8(x) deq4(r) + u L2 + bias ).
  *   r_codes, r_sf  (device) MXFP4-packed residual weight [N, K] (fp4_pack_weight);
  *                  r_codes must be 32-byte aligned
- *   l2_bf16        (device) [rank, N] bf16
- * The low-rank product u L2 is evaluated with fp32 FMAs in the epilogue. */
-fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const float* u_f32, int64_t M,
+ *   u_pair         (device) [M, 2 * rank] bf16 from w4a8_quantize_act
+ *   l2t_bf16       (device) [N, rank] bf16 from w4a8_pack_lowrank_up
+ * The low-rank product is accumulated on the tensor core into the same fp32 accumulator,
+ * as (u_hi L2 + u_lo L2), before the bias and the bf16 rounding. */
+fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const void* u_pair, int64_t M,
                        int64_t K, int64_t N, const uint8_t* r_codes, const uint8_t* r_sf,
-                       const void* l2_bf16, int rank, const void* bias_f16, void* y_bf16,
+                       const void* l2t_bf16, int rank, const void* bias_f16, void* y_bf16,
                        void* stream);
 
 /* The full W4A8 SVDQuant linear: w4a8_quantize_act into `workspace`, then w4a8_gemm.
- * rank must be 32. */
+ * l2t_bf16 is the packed [N, rank] up-projection; rank must be 32. */
 fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N,
                              const uint8_t* r_codes, const uint8_t* r_sf, const void* l1_bf16,
-                             const void* l2_bf16, int rank, const void* bias_f16, void* y_bf16,
+                             const void* l2t_bf16, int rank, const void* bias_f16, void* y_bf16,
                              void* workspace, size_t ws_bytes, void* stream);
 
 /* ----------------------------------------------------------------- status */

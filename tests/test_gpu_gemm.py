@@ -204,7 +204,8 @@ def _w4a8_check(fb, orc, M, K, N, seed, rows=None, calib=256):
     x = synth.activation(seed + 1, M, K, "lognormal", gain_seed=seed + 5)
     b = synth.bias(seed + 2, N)
     rp = fb.pack_weight(H.dev_bf16(f["r_bf16"]), MX)
-    y = fb.w4a8_linear(H.dev_bf16(x), rp, H.dev_bf16(f["l1_bf16"]), H.dev_bf16(f["l2_bf16"]), H.dev_f16(b))
+    l2t = fb.pack_lowrank_up(H.dev_bf16(f["l2_bf16"]))
+    y = fb.w4a8_linear(H.dev_bf16(x), rp, H.dev_bf16(f["l1_bf16"]), l2t, H.dev_f16(b))
     st = fb.fp4_sync_status()
     assert st == 0, fb.fp4_status_string(st)
     torch.cuda.synchronize()
@@ -259,7 +260,8 @@ def test_each_kernel_all_elements(fb, orc, ctas, fmt, M, K, N):
 
 
 @pytest.mark.parametrize("ctas", [1, 2])
-def test_each_kernel_w4a8(fb, orc, ctas):
+def test_w4a8_ignores_the_kernel_hook(fb, orc, ctas):
+    """W4A8 always runs the 2-CTA kernel (its low-rank stage is a tensor-core stage there)."""
     with _gemm_ctas(fb, ctas):
         _w4a8_check(fb, orc, 300, 1024, 512, seed=7777)
 

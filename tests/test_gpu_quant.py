@@ -91,7 +91,7 @@ def test_e4m3_conversion_sweep(fb, orc):
     l1 = torch.zeros((K, 32), dtype=torch.bfloat16, device="cuda")
     xe = torch.empty((rows, K), dtype=torch.uint8, device="cuda")
     xs_ = torch.empty(fb.fp4_sf_bytes(MX, rows, K), dtype=torch.uint8, device="cuda")
-    u = torch.empty((rows, 32), dtype=torch.float32, device="cuda")
+    u = torch.empty((rows, 64), dtype=torch.bfloat16, device="cuda")
     fb.w4a8_quantize_act(H.dev_bf16(x), rows, K, l1, 32, xe, xs_, u)
     torch.cuda.synchronize()
     e = H.host_u8(xe)
@@ -129,18 +129,23 @@ def test_mxfp8_quant_and_lowrank(fb, orc, M, K):
     e_ref, s_ref = orc.quantize_mxfp8(x)
     xe = torch.empty((M, K), dtype=torch.uint8, device="cuda")
     xs = torch.empty(fb.fp4_sf_bytes(MX, M, K), dtype=torch.uint8, device="cuda")
-    u = torch.empty((M, 32), dtype=torch.float32, device="cuda")
+    u = torch.empty((M, 64), dtype=torch.bfloat16, device="cuda")
     fb.w4a8_quantize_act(H.dev_bf16(x), M, K, H.dev_bf16(f["l1_bf16"]), 32, xe, xs, u)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(H.host_u8(xe), e_ref)
     np.testing.assert_array_equal(H.host_u8(xs), s_ref)
-    # u = x L1 in fp32 against fp64: within fp32 accumulation error of sum_k |x_k l1_k|
+    # u = x L1 accumulated in fp32, carried as the bf16 pair hi + lo: against fp64, within
+    # the fp32 accumulation error of sum_k |x_k l1_k| plus the pair's 2^-18 |u|
     xf = synth.bf16_bits_to_f32(x).astype(np.float64)
     l1 = synth.bf16_bits_to_f32(f["l1_bf16"]).astype(np.float64)
     u_ref = xf @ l1
     mag = np.abs(xf) @ np.abs(l1)
-    err = np.abs(u.cpu().numpy().astype(np.float64) - u_ref)
-    assert np.all(err <= 4 * K * 2.0 ** -24 * mag + 1e-30)
+    pair = u.float().cpu().numpy().astype(np.float64)
+    hi, lo = pair[:, :32], pair[:, 32:]
+    err = np.abs(hi + lo - u_ref)
+    assert np.all(err <= 4 * K * 2.0 ** -24 * mag + 2.0 ** -17 * np.abs(u_ref) + 1e-30)
+    # a valid split: lo is below half an ulp of hi (bf16: 2^-8 relative)
+    assert np.all(np.abs(lo) <= 2.0 ** -8 * np.abs(hi) + 1e-30)
 
 
 def test_edge_values(fb, orc):
@@ -212,3 +217,15 @@ def test_full_size_quant(fb, orc, fmt):
         cal = synth.activation(s["calib"], synth.CALIB_TOKENS, K, "lognormal", gain_seed=s["gain"])
         g = orc.nv_global(orc.tensor_amax(cal))
     _assert_quant(fb, orc, fmt, x, g)
+
+
+def test_pack_lowrank_up_is_the_transpose(fb):
+    """w4a8_pack_lowrank_up: [rank, N] -> [N, rank], bit-exact."""
+    import torch
+
+    N = 384
+    l2 = synth.svdquant_factors(77, N, 256, calib_tokens=64)["l2_bf16"]
+    l2t = fb.pack_lowrank_up(H.dev_bf16(l2))
+    torch.cuda.synchronize()
+    got = l2t.view(torch.int16).cpu().numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, np.ascontiguousarray(l2.T))
