@@ -294,15 +294,11 @@ fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf
     // 2-CTA 256x256 tiles (faster at every M measured) unless M fits one 128-row tile or
     // the 1-CTA kernel is forced (tuning hook)
     const bool pair = g_gemm_ctas != 1 && M > GEMM_BM;
-    // the 2-CTA NVFP4 kernel stages 128 K (64 bytes per row, 64-byte swizzle)
-    const uint32_t box_inner = (pair && nv) ? 64 : 128;
-    const CUtensorMapSwizzle swz = (pair && nv) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     CUtensorMap ta, tb;
-    if ((s = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, box_inner, GEMM_BM, swz)) !=
-        FP4_OK)
+    if ((s = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 128, GEMM_BM)) != FP4_OK)
         return s;
-    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, box_inner,
-                       pair ? 128 : GEMM_BN, swz)) != FP4_OK)
+    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 128, pair ? 128 : GEMM_BN)) !=
+        FP4_OK)
         return s;
     GemmParams p{};
     p.M = (int)M, p.N = (int)N, p.K = (int)K;

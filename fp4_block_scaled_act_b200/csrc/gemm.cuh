@@ -386,12 +386,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 template <int KIND>
 struct Gemm2Cfg {
     using C1 = GemmCfg<KIND>;
-    // NVFP4 takes 128 K per stage (64-byte swizzle) so its scale footprint matches MXFP4's
-    static constexpr int BK = (KIND == G_NVFP4) ? 128 : C1::BK;
+    // 128-byte operand rows (128-byte swizzle) for every kind: with 64-byte rows (64-byte
+    // swizzle) a 256x256x64 MMA was measured at ~290 cycles instead of ~160
+    static constexpr int BK = C1::BK;
     static constexpr int G = C1::G, MMA_K = C1::MMA_K;
-    static constexpr int ATOMS = BK / (G * 4);
-    static constexpr int ROW_BYTES = (KIND == G_NVFP4) ? 64 : 128;     // per operand row per stage
-    static constexpr uint32_t SWZ = (ROW_BYTES == 128) ? 2u : 4u;      // descriptor layout
+    static constexpr int ATOMS = BK / (G * 4);  // scale atoms per stage: MX 2, NV 4, W4A8 1
+    static constexpr int ROW_BYTES = 128;       // per operand row per stage
+    static constexpr uint32_t SWZ = 2u;         // descriptor layout: 128-byte swizzle
     static constexpr int SBO = 8 * ROW_BYTES;
     static constexpr int N_MMA = BK / MMA_K;
     static constexpr int A_BYTES = 128 * ROW_BYTES;
@@ -399,16 +400,19 @@ struct Gemm2Cfg {
     static constexpr int RSFA_BYTES = ATOMS * 512;    // raw atoms, this CTA's 128 A rows
     static constexpr int RSFB_BYTES = 2 * ATOMS * 512;  // raw atoms, all 256 B rows
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RSFA_BYTES + RSFB_BYTES;
-    static constexpr int STAGES = (KIND == G_NVFP4) ? 10 : 5;
+    static constexpr int STAGES = 5;
     static constexpr int EPI_BYTES = 8 * 32 * 128;    // a 32 x 64 bf16 staging tile per epilogue warp
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + 512;
     static constexpr uint32_t AB_TX = A_BYTES + ((KIND == G_W4A8) ? B_BYTES / 2 : B_BYTES);
     static constexpr uint32_t SF_TX = RSFA_BYTES + RSFB_BYTES;
-    static constexpr int ACC1_COL = 192;
-    static constexpr int SF_COL0 = 448;
+    // NVFP4 stages carry 4 scale atoms (48 TMEM columns): its accumulators overlap by 96
+    // columns to leave room for two scale buffers; the others overlap by 64
+    static constexpr int ACC1_COL = (KIND == G_NVFP4) ? 160 : 192;
+    static constexpr int SF_COL0 = ACC1_COL + 256;
+    static constexpr int OVL = 256 - ACC1_COL;
     static constexpr int SFA_COLS = 4 * ATOMS;        // A: 4 columns per atom
     static constexpr int SF_COLS = SFA_COLS + 8 * ATOMS;  // B: 8 columns per atom
-    static constexpr int TB = (64 / SF_COLS) >= 4 ? 4 : (64 / SF_COLS);  // scale buffers
+    static constexpr int TB = ((GEMM_TMEM_COLS - SF_COL0) / SF_COLS) >= 4 ? 4 : ((GEMM_TMEM_COLS - SF_COL0) / SF_COLS);
     static constexpr int THREADS = 480;
     // W4A8 low-rank stage (one per tile, after the K stages): A = the u pair, 128 rows x 64
     // bf16 (128-byte rows, 128-byte swizzle); B = packed L2, 128 rows x 32 bf16 (64-byte
@@ -421,6 +425,7 @@ struct Gemm2Cfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert((STAGES * (A_BYTES + B_BYTES)) % 1024 == 0, "staging tiles 1024-byte aligned");
     static_assert(TB >= 2 && SF_COL0 + TB * SF_COLS <= GEMM_TMEM_COLS, "TMEM budget");
+    static_assert(OVL == 64 || OVL == 96, "epilogue overlap handling");
 };
 
 // Pair-kernel epilogue: pack one row's 64 columns and write them, as 128 bytes, into row
@@ -635,6 +640,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 const uint32_t xb = xa + C::SFA_COLS;
                 // the W4A8 low-rank stage reads no scales: its buffer turn passes unwritten
                 if (KIND == G_W4A8 && kb == num_kb) {
+                } else if constexpr (C::ATOMS == 4) {
+                    tmem_st_32x32b_x16(tlane + xa, *reinterpret_cast<const uint32_t(*)[16]>(va));
+                    tmem_st_32x32b_x16(tlane + xb, *reinterpret_cast<const uint32_t(*)[16]>(vb));
+                    tmem_st_32x32b_x16(tlane + xb + 16, *reinterpret_cast<const uint32_t(*)[16]>(vb + 16));
                 } else if constexpr (C::ATOMS == 2) {
                     tmem_st_32x32b_x8(tlane + xa, va);
                     tmem_st_32x32b_x16(tlane + xb, vb);
@@ -786,16 +795,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                     bulk_commit_group();
                 }
             };
-            // the 64 columns shared by both accumulators are tile columns 192..255 of
-            // accumulator 0 (half 1, chunks 2-3) or 0..63 of accumulator 1 (half 0, chunks 0-1):
-            // their holders drain them first and release them
+            // the OVL columns shared by both accumulators are the last OVL tile columns of
+            // accumulator 0 (half 1) or the first OVL of accumulator 1 (half 0): their holders
+            // drain them first and release them -- after the first chunk pair when OVL = 64,
+            // after both pairs when OVL = 96 (NVFP4)
             const bool holds_overlap = (h == (b == 0 ? 1 : 0));
             const int first = holds_overlap ? (b == 0 ? 2 : 0) : 0;
             const int second = 2 - first;
             tmem_ld_32x32b_x32(taddr + first * 32, acc[0]);
             tmem_ld_32x32b_x32(taddr + (first + 1) * 32, acc[1]);
             tmem_wait_ld();
-            if (holds_overlap) {
+            if (holds_overlap && C::OVL <= 64) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) arrive_leader_relaxed(ovl_free, rank);
@@ -806,6 +816,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
+            if (holds_overlap && C::OVL > 64 && lane == 0) arrive_leader_relaxed(ovl_free, rank);
             if (lane == 0) arrive_leader_relaxed(&acc_free[b], rank);
             stage_store(second);
         }
