@@ -6,7 +6,8 @@ stream becomes the stream argument, and a non-OK status raises FP4Error.  All
 arithmetic runs in the library's CUDA kernels.  There is no fallback: if the
 library is missing or the device is not sm_100, the calls raise.
 
-The helpers at the end (pack_weight, quantize_act, linear, pack_lowrank_up, w4a8_linear)
+The helpers at the end (pack_weight, quantize_act, linear, pack_lowrank_up, w4a8_linear,
+w4a4_linear)
 allocate outputs and workspaces with torch and call the same entry points.
 """
 from __future__ import annotations
@@ -31,6 +32,7 @@ EXPORTS = [
     "fp4_tensor_amax", "fp4_pack_weight", "fp4_quantize_act", "fp4_gemm", "fp4_linear",
     "w4a8_quantize_act", "w4a8_gemm", "w4a8_svd_linear", "fp4_sync_status", "fp4_status_string",
     "fp4_set_wait_timeout_ns", "fp4_linear_noalloc", "w4a8_pack_lowrank_up",
+    "w4a4_workspace_bytes", "w4a4_quantize_act", "w4a4_gemm", "w4a4_svd_linear",
 ]
 
 
@@ -65,6 +67,10 @@ def lib():
             "fp4_linear_noalloc": (I, [I, P, I64, I64, I64, P, P, P, P, P, P, P]),
             "w4a8_quantize_act": (I, [P, I64, I64, P, I, P, P, P, P]),
             "w4a8_pack_lowrank_up": (I, [P, I64, I, P, P]),
+            "w4a4_workspace_bytes": (SZ, [I64, I64, I64, I]),
+            "w4a4_quantize_act": (I, [P, I64, I64, P, I, P, P, P, P]),
+            "w4a4_gemm": (I, [P, P, P, I64, I64, I64, P, P, P, I, P, P, P]),
+            "w4a4_svd_linear": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, P, SZ, P]),
             "w4a8_gemm": (I, [P, P, P, I64, I64, I64, P, P, P, I, P, P, P]),
             "w4a8_svd_linear": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, P, SZ, P]),
             "fp4_sync_status": (I, [P]),
@@ -185,6 +191,28 @@ def w4a8_svd_linear(x, M: int, K: int, N: int, r_codes, r_sf, l1, l2t, rank: int
            "w4a8_svd_linear")
 
 
+def w4a4_workspace_bytes(M: int, K: int, N: int, rank: int = 32) -> int:
+    return lib().w4a4_workspace_bytes(M, K, N, rank)
+
+
+def w4a4_quantize_act(x, M: int, K: int, l1, rank: int, x_codes, x_sf, u_pair, stream=None):
+    _check(lib().w4a4_quantize_act(_ptr(x), M, K, _ptr(l1), rank, _ptr(x_codes), _ptr(x_sf), _ptr(u_pair),
+                                   _stream(stream)), "w4a4_quantize_act")
+
+
+def w4a4_gemm(x_codes, x_sf, u_pair, M: int, K: int, N: int, r_codes, r_sf, l2t, rank: int, bias, y,
+              stream=None):
+    _check(lib().w4a4_gemm(_ptr(x_codes), _ptr(x_sf), _ptr(u_pair), M, K, N, _ptr(r_codes), _ptr(r_sf),
+                           _ptr(l2t), rank, _ptr(bias), _ptr(y), _stream(stream)), "w4a4_gemm")
+
+
+def w4a4_svd_linear(x, M: int, K: int, N: int, r_codes, r_sf, l1, l2t, rank: int, bias, y, workspace,
+                    ws_bytes: int, stream=None):
+    _check(lib().w4a4_svd_linear(_ptr(x), M, K, N, _ptr(r_codes), _ptr(r_sf), _ptr(l1), _ptr(l2t), rank,
+                                 _ptr(bias), _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
+           "w4a4_svd_linear")
+
+
 def fp4_sync_status(stream=None) -> int:
     return lib().fp4_sync_status(_stream(stream))
 
@@ -271,4 +299,19 @@ def w4a8_linear(x, r: PackedWeight, l1, l2t, bias=None, y=None, workspace=None, 
     if workspace is None:
         workspace = torch.empty(w4a8_workspace_bytes(M, K, r.N, rank), dtype=torch.uint8, device=x.device)
     w4a8_svd_linear(x, M, K, r.N, r.codes, r.sf, l1, l2t, rank, bias, y, workspace, workspace.numel(), stream)
+    return y
+
+
+def w4a4_linear(x, r: PackedWeight, l1, l2t, bias=None, y=None, workspace=None, stream=None):
+    """W4A4 SVDQuant linear: bf16 [M, K] -> bf16 [M, N] (MXFP4 activations and residual r,
+    rank-32 L1 [K, rank] and packed L2 [N, rank] from pack_lowrank_up)."""
+    import torch
+
+    M, K = x.shape
+    rank = l1.shape[1]
+    if y is None:
+        y = torch.empty((M, r.N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(w4a4_workspace_bytes(M, K, r.N, rank), dtype=torch.uint8, device=x.device)
+    w4a4_svd_linear(x, M, K, r.N, r.codes, r.sf, l1, l2t, rank, bias, y, workspace, workspace.numel(), stream)
     return y

@@ -29,7 +29,7 @@ struct DeviceState {
     bool ready = false;
     bool arch_ok = false;
     int sm_count = 0;
-    int pairs[3] = {0, 0, 0};  // co-resident CTA pairs of gemm2_kernel<kind>
+    int pairs[4] = {0, 0, 0, 0};  // co-resident CTA pairs of gemm2_kernel<kind>
     int quant_occ[3] = {1, 1, 1};  // resident CTAs per SM of quant_kernel<kind>
     int* status = nullptr;
 };
@@ -76,7 +76,9 @@ fp4_status_t device_state(DeviceState** out) {
                 cudaFuncSetAttribute(gemm2_kernel<G_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Gemm2Cfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm2_kernel<G_W4A8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     Gemm2Cfg<G_W4A8>::SMEM_BYTES) != cudaSuccess)
+                                     Gemm2Cfg<G_W4A8>::SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm2_kernel<G_SVD4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Gemm2Cfg<G_SVD4>::SMEM_BYTES) != cudaSuccess)
                 return FP4_ERR_CUDA;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.quant_occ[Q_MXFP4], quant_kernel<Q_MXFP4>,
                                                               QUANT_THREADS, 0) != cudaSuccess ||
@@ -88,6 +90,7 @@ fp4_status_t device_state(DeviceState** out) {
             s.pairs[G_MXFP4] = max_pairs<G_MXFP4>(s.sm_count);
             s.pairs[G_NVFP4] = max_pairs<G_NVFP4>(s.sm_count);
             s.pairs[G_W4A8] = max_pairs<G_W4A8>(s.sm_count);
+            s.pairs[G_SVD4] = max_pairs<G_SVD4>(s.sm_count);
         }
         if (!g_encode) {
             cudaDriverEntryPointQueryResult q;
@@ -225,7 +228,15 @@ size_t fp4_linear_workspace_bytes(fp4_fmt_t fmt, int64_t M, int64_t K, int64_t N
 
 size_t w4a8_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank) {
     if (rank != 32 || check_shape(M, K, N) != FP4_OK) return 0;
+    // E4M3 codes, E8M0 scales, u pair (M x 2 rank bf16)
     return align256((size_t)M * K) + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K)) + align256((size_t)M * rank * 4);
+}
+
+size_t w4a4_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank) {
+    if (rank != 32 || check_shape(M, K, N) != FP4_OK) return 0;
+    // MXFP4 codes, E8M0 scales, u pair (M x 2 rank bf16)
+    return align256(fp4_codes_bytes(FP4_FMT_MXFP4, M, K)) + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K)) +
+           align256((size_t)M * rank * 4);
 }
 
 fp4_status_t fp4_tensor_amax(const void* x_bf16, int64_t n, float* amax_out, void* stream) {
@@ -408,6 +419,70 @@ fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N
     uint8_t* u = xs + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K));
     if ((s = w4a8_quantize_act(x_bf16, M, K, l1_bf16, rank, xe, xs, u, stream)) != FP4_OK) return s;
     return w4a8_gemm(xe, xs, u, M, K, N, r_codes, r_sf, l2t_bf16, rank, bias_f16, y_bf16, stream);
+}
+
+fp4_status_t w4a4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16, int rank,
+                               uint8_t* x_codes, uint8_t* x_sf, void* u_pair, void* stream) {
+    if (!x_bf16 || !l1_bf16 || !x_codes || !x_sf || !u_pair || rank != 32) return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, 128);
+    if (s != FP4_OK) return s;
+    if (!aligned16(x_bf16) || !aligned16(l1_bf16) || !aligned16(x_codes) || !aligned16(x_sf) || !aligned16(u_pair))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    if ((s = device_state(&ds)) != FP4_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = launch_quant(ds, Q_MXFP4, x_bf16, M, K, nullptr, x_codes, x_sf, st)) != FP4_OK) return s;
+    const int blocks = (int)((M + LR_ROWS - 1) / LR_ROWS);
+    lowrank_down_kernel<<<blocks, LR_THREADS, 0, st>>>(static_cast<const __nv_bfloat16*>(x_bf16),
+                                                       static_cast<const __nv_bfloat16*>(l1_bf16), (int)M, (int)K,
+                                                       static_cast<__nv_bfloat16*>(u_pair));
+    return launched();
+}
+
+fp4_status_t w4a4_gemm(const uint8_t* x_codes, const uint8_t* x_sf, const void* u_pair, int64_t M, int64_t K,
+                       int64_t N, const uint8_t* r_codes, const uint8_t* r_sf, const void* l2t_bf16, int rank,
+                       const void* bias_f16, void* y_bf16, void* stream) {
+    if (!x_codes || !x_sf || !u_pair || !r_codes || !r_sf || !l2t_bf16 || !y_bf16 || rank != 32)
+        return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, N);
+    if (s != FP4_OK) return s;
+    if (!aligned16(x_codes) || !aligned16(x_sf) || !aligned16(u_pair) || !aligned16(r_codes) || !aligned16(r_sf) ||
+        !aligned16(l2t_bf16) || !aligned16(bias_f16) || !aligned16(y_bf16))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    if ((s = device_state(&ds)) != FP4_OK) return s;
+    CUtensorMap ta, tb, tu, tl;
+    if ((s = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, x_codes, K / 2, M, K / 2, 128, GEMM_BM)) != FP4_OK)
+        return s;
+    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, r_codes, K / 2, N, K / 2, 128, 128)) != FP4_OK) return s;
+    if ((s = encode_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, u_pair, 2 * (uint64_t)rank, M, 4 * (uint64_t)rank,
+                       2 * rank, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
+        return s;
+    if ((s = encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l2t_bf16, (uint64_t)rank, N, 2 * (uint64_t)rank, rank,
+                       128, CU_TENSOR_MAP_SWIZZLE_64B)) != FP4_OK)
+        return s;
+    GemmParams p{};
+    p.M = (int)M, p.N = (int)N, p.K = (int)K;
+    p.sfa = x_sf, p.sfb = r_sf;
+    p.bias = static_cast<const __half*>(bias_f16);
+    p.y = static_cast<__nv_bfloat16*>(y_bf16);
+    return launch_gemm2<G_SVD4>(ds, ta, tb, x_sf, r_sf, p, static_cast<cudaStream_t>(stream), &tu, &tl);
+}
+
+fp4_status_t w4a4_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N, const uint8_t* r_codes,
+                             const uint8_t* r_sf, const void* l1_bf16, const void* l2t_bf16, int rank,
+                             const void* bias_f16, void* y_bf16, void* workspace, size_t ws_bytes, void* stream) {
+    if (!workspace || rank != 32) return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, N);
+    if (s != FP4_OK) return s;
+    if (ws_bytes < w4a4_workspace_bytes(M, K, N, rank)) return FP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+    if (!r_codes || !r_sf || !l2t_bf16 || !y_bf16) return FP4_ERR_INVALID_ARG;
+    uint8_t* xc = static_cast<uint8_t*>(workspace);
+    uint8_t* xs = xc + align256(fp4_codes_bytes(FP4_FMT_MXFP4, M, K));
+    uint8_t* u = xs + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K));
+    if ((s = w4a4_quantize_act(x_bf16, M, K, l1_bf16, rank, xc, xs, u, stream)) != FP4_OK) return s;
+    return w4a4_gemm(xc, xs, u, M, K, N, r_codes, r_sf, l2t_bf16, rank, bias_f16, y_bf16, stream);
 }
 
 fp4_status_t fp4_sync_status(void* stream) {

@@ -25,7 +25,9 @@
 
 namespace fp4 {
 
-enum GemmKind { G_MXFP4 = 0, G_NVFP4 = 1, G_W4A8 = 2 };
+// G_SVD4: W4A4 SVDQuant, MXFP4 activations x MXFP4 residual (the MXFP4 main loop) plus the
+// low-rank stage of the 2-CTA kernel, like G_W4A8.
+enum GemmKind { G_MXFP4 = 0, G_NVFP4 = 1, G_W4A8 = 2, G_SVD4 = 3 };
 
 constexpr int GEMM_THREADS = 320;
 constexpr int GEMM_BM = 128;
@@ -124,7 +126,7 @@ FP4_DEV void epilogue_store(const GemmParams& p, uint32_t (&acc)[NC][32], int ro
 // Which TMEM scale atom and which byte of it MMA number k of a stage reads.
 template <int KIND>
 FP4_DEV void sf_select(int k, int& atom, int& sf_id) {
-    if (KIND == G_MXFP4) {  // 2 E8M0 scales (K = 64) per MMA: byte pair 0-1 or 2-3
+    if (KIND == G_MXFP4 || KIND == G_SVD4) {  // 2 E8M0 scales (K = 64) per MMA: byte pair 0-1 or 2-3
         atom = k >> 1;
         sf_id = (k & 1) * 2;
     } else if (KIND == G_NVFP4) {  // 4 E4M3 scales (K = 64) per MMA: the whole word
@@ -518,7 +520,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         prefetch_tmap(&tmSFA);
         prefetch_tmap(&tmSFB);
         prefetch_tmap(&tmY);
-        if (KIND == G_W4A8) {
+        if (KIND == G_W4A8 || KIND == G_SVD4) {
             prefetch_tmap(&tmU);
             prefetch_tmap(&tmL);
         }
@@ -539,8 +541,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
     const int num_n = (N + 255) / 256;
     const int num_tiles = num_m * num_n;
     const int num_kb = (K + C::BK - 1) / C::BK;
-    // stages per tile: the K blocks, then (W4A8) the low-rank stage kb == num_kb
-    const int spt = num_kb + (KIND == G_W4A8 ? 1 : 0);
+    // stages per tile: the K blocks, then (W4A8, W4A4 SVDQuant) the low-rank stage kb == num_kb
+    constexpr bool HAS_LR = (KIND == G_W4A8 || KIND == G_SVD4);
+    const int spt = num_kb + (HAS_LR ? 1 : 0);
     const int apr = K / (C::G * 4);  // scale atoms per 128-row block
     const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
 
@@ -564,7 +567,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                     if (it == p.skip_iter) continue;  // test hook: this stage is never filled
                     // A/B of both CTAs land on the leader's barrier; only the leader expects them
                     const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
-                    if (KIND == G_W4A8 && kb == num_kb) {
+                    if (HAS_LR && kb == num_kb) {
                         // low-rank stage: u pair rows and packed-L2 rows; no scale atoms, but
                         // sf_full still completes a phase so its parity keeps counting stages
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::LR_TX);
@@ -639,7 +642,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 const uint32_t xa = C::SF_COL0 + (uint32_t)(t * C::SF_COLS);
                 const uint32_t xb = xa + C::SFA_COLS;
                 // the W4A8 low-rank stage reads no scales: its buffer turn passes unwritten
-                if (KIND == G_W4A8 && kb == num_kb) {
+                if (HAS_LR && kb == num_kb) {
                 } else if constexpr (C::ATOMS == 4) {
                     tmem_st_32x32b_x16(tlane + xa, *reinterpret_cast<const uint32_t(*)[16]>(va));
                     tmem_st_32x32b_x16(tlane + xb, *reinterpret_cast<const uint32_t(*)[16]>(vb));
@@ -673,7 +676,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 const uint32_t dacc = tmem_base + (uint32_t)(b * C::ACC1_COL);
                 for (int kb = 0; kb < spt; ++kb, ++it) {
                     named_bar_sync(1u + it % TB, 64u);
-                    if (lane == 0 && KIND == G_W4A8 && kb == num_kb) {
+                    if (lane == 0 && HAS_LR && kb == num_kb) {
                         // low-rank stage: acc += u_hi L2 + u_lo L2 (bf16 x bf16 -> fp32)
                         tc_fence_after();
                         const int s = (int)(it % S);
@@ -702,7 +705,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                             const uint64_t adesc = smem_desc(a_base + k * 32, 0, C::SBO, C::SWZ);
                             const uint64_t bdesc = smem_desc(b_base + k * 32, 0, C::SBO, C::SWZ);
                             const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-                            if (KIND == G_MXFP4)
+                            if (KIND == G_MXFP4 || KIND == G_SVD4)
                                 mma2_mxf4nvf4_block32(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
                             else if (KIND == G_NVFP4)
                                 mma2_mxf4nvf4_block16(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);

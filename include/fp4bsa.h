@@ -210,6 +210,39 @@ fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N
                              const void* l2t_bf16, int rank, const void* bias_f16, void* y_bf16,
                              void* workspace, size_t ws_bytes, void* stream);
 
+/* ----------------------------------------------------------------- W4A4 SVDQuant */
+
+/* The W4A8 README's experimental W4A4 variant ("Experimental W4A4 (MXFP4 activations)"):
+ * the same calibrated factors (MXFP4 residual R, rank-32 L1 / L2), with the activations
+ * quantized to MXFP4 instead of MXFP8; the low-rank branch still reads the unquantized
+ * input.  y = bf16_rn( sum_k deq4(x) deq4(r) + u L2 + bias ). */
+
+/* Workspace for w4a4_svd_linear: MXFP4 codes + scales of x and the u pair (0 if invalid). */
+size_t w4a4_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank);
+
+/* Activation side: MXFP4 codes and scales of x (exactly fp4_quantize_act with
+ * FP4_FMT_MXFP4) and the u pair of x L1 (exactly as w4a8_quantize_act writes it).
+ *   x_codes  (device, out) [M, K/2]; x_sf (device, out) fp4_sf_bytes(FP4_FMT_MXFP4, M, K)
+ *   u_pair   (device, out) [M, 2 * rank] bf16 */
+fp4_status_t w4a4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16,
+                               int rank, uint8_t* x_codes, uint8_t* x_sf, void* u_pair,
+                               void* stream);
+
+/* W4A4 SVDQuant GEMM: MXFP4 x MXFP4 block-scaled main loop plus the tensor-core low-rank
+ * stage (u_hi L2 + u_lo L2) into the same fp32 accumulator, + bias, bf16 out.
+ *   r_codes, r_sf  MXFP4-packed residual [N, K] (fp4_pack_weight)
+ *   l2t_bf16       packed [N, rank] up-projection (w4a8_pack_lowrank_up) */
+fp4_status_t w4a4_gemm(const uint8_t* x_codes, const uint8_t* x_sf, const void* u_pair, int64_t M,
+                       int64_t K, int64_t N, const uint8_t* r_codes, const uint8_t* r_sf,
+                       const void* l2t_bf16, int rank, const void* bias_f16, void* y_bf16,
+                       void* stream);
+
+/* The full W4A4 SVDQuant linear: w4a4_quantize_act into `workspace`, then w4a4_gemm. */
+fp4_status_t w4a4_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N,
+                             const uint8_t* r_codes, const uint8_t* r_sf, const void* l1_bf16,
+                             const void* l2t_bf16, int rank, const void* bias_f16, void* y_bf16,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /* ----------------------------------------------------------------- status */
 
 /* Synchronizes `stream`, then returns and clears the device status word of the current

@@ -20,7 +20,7 @@ def fb():
 def header_symbols():
     text = open(os.path.join(ROOT, "include", "fp4bsa.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b((?:fp4|w4a8)_[a-z0-9_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b((?:fp4|w4a8|w4a4)_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_exports_every_header_symbol(fb):
@@ -45,6 +45,11 @@ def test_size_queries(fb):
     assert fb.fp4_linear_workspace_bytes(MX, 0, 5120, 13824) == 0
     assert fb.w4a8_workspace_bytes(4290, 3072, 14336, 32) > 4290 * 3072
     assert fb.w4a8_workspace_bytes(4290, 3072, 14336, 16) == 0
+    # W4A4 SVDQuant: MXFP4 codes + scales + the u pair, each 256-byte aligned
+    a256 = lambda n: (n + 255) // 256 * 256
+    assert fb.w4a4_workspace_bytes(4290, 3072, 14336, 32) == (
+        a256(4290 * 1536) + a256(fb.fp4_sf_bytes(MX, 4290, 3072)) + a256(4290 * 32 * 4))
+    assert fb.w4a4_workspace_bytes(4290, 3072, 14336, 16) == 0
 
 
 def test_bytes_per_weight_match_format(fb):
@@ -93,6 +98,12 @@ def test_invalid_calls_rejected_before_launch(fb):
     assert L.w4a8_pack_lowrank_up(A, 384, 16, A, st) == 1
     assert L.w4a8_pack_lowrank_up(A, 200, 32, A, st) == 2
     assert L.w4a8_pack_lowrank_up(bad, 384, 32, A, st) == 3
+    # W4A4 SVDQuant: rank, shape, alignment, workspace
+    assert L.w4a4_svd_linear(A, 16, 256, 256, A, A, A, A, 16, None, A, A, 1 << 30, st) == 1
+    assert L.w4a4_gemm(A, A, A, 16, 256, 200, A, A, A, 32, None, A, st) == 2
+    assert L.w4a4_gemm(A, A, A, 16, 256, 384, A, A, A, 32, None, bad, st) == 3
+    assert L.w4a4_svd_linear(A, 16, 256, 256, A, A, A, A, 32, None, A, A, 10, st) == 4
+    assert L.w4a4_quantize_act(A, 16, 256, A, 32, A, A, None, st) == 1
     # weight pack: MXFP4 must not get a global
     assert L.fp4_pack_weight(0, A, 256, 256, A, A, A, st) == 1
     assert L.fp4_tensor_amax(A, 0, A, st) == 1

@@ -231,6 +231,42 @@ def test_w4a8_full_size_sampled(fb, orc):
     _w4a8_check(fb, orc, M, K, N, seed=3001, rows=rows, calib=2048)
 
 
+# ------------------------------------------------------------------ W4A4 SVDQuant linear
+# The W4A8 README's experimental W4A4 variant: MXFP4 activations on the same factors.
+def _w4a4_check(fb, orc, M, K, N, seed, rows=None, calib=256):
+    import torch
+
+    f = synth.svdquant_factors(seed, N, K, calib_tokens=calib)
+    x = synth.activation(seed + 1, M, K, "lognormal", gain_seed=seed + 5)
+    b = synth.bias(seed + 2, N)
+    rp = fb.pack_weight(H.dev_bf16(f["r_bf16"]), MX)
+    l2t = fb.pack_lowrank_up(H.dev_bf16(f["l2_bf16"]))
+    y = fb.w4a4_linear(H.dev_bf16(x), rp, H.dev_bf16(f["l1_bf16"]), l2t, H.dev_f16(b))
+    st = fb.fp4_sync_status()
+    assert st == 0, fb.fp4_status_string(st)
+    torch.cuda.synchronize()
+    rows = np.arange(M) if rows is None else rows
+    xc, xs = orc.quantize(MX, np.ascontiguousarray(x[rows]))
+    a = orc.dequant_fp4(MX, xc, xs, K)
+    rc, rs, _ = orc.pack_weight(MX, f["r_bf16"])
+    w = orc.dequant_fp4(MX, rc, rs, K)
+    Y, S = orc.linear_fp64(a, w, b)
+    LR, LS = orc.lowrank_fp64(x, rows, f["l1_bf16"], f["l2_bf16"])
+    return H.check_linear(y, Y + LR, S + LS, rows, f"w4a4 M={M} K={K} N={N}")
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 256, 256), (130, 512, 384), (300, 1024, 512)])
+def test_w4a4_small_all_elements(fb, orc, M, K, N):
+    _w4a4_check(fb, orc, M, K, N, seed=8000 + M)
+
+
+def test_w4a4_full_size_sampled(fb, orc):
+    """TI2V-5B-shaped W4A4 SVDQuant linear: M = 4290, K = 3072, N = 14336, rank 32."""
+    M, K, N = 4290, 3072, 14336
+    rows = H.sample_rows(M, n_random=48, seed=4)
+    _w4a4_check(fb, orc, M, K, N, seed=4001, rows=rows, calib=2048)
+
+
 # ------------------------------------------------------------------ each GEMM kernel, forced
 # The library picks the cta_group::2 256x256 kernel for M > 128 and the 1-CTA 128x256
 # kernel otherwise; a tuning hook forces either, so both stay covered on ragged shapes.

@@ -229,3 +229,27 @@ def test_pack_lowrank_up_is_the_transpose(fb):
     torch.cuda.synchronize()
     got = l2t.view(torch.int16).cpu().numpy().view(np.uint16)
     np.testing.assert_array_equal(got, np.ascontiguousarray(l2.T))
+
+
+@pytest.mark.parametrize("M,K", [(130, 512), (300, 1024)])
+def test_w4a4_quantize_act(fb, orc, M, K):
+    """W4A4 SVDQuant activation side: MXFP4 codes and scales bit-exact, the u pair as in W4A8."""
+    import torch
+
+    x = synth.activation(900 + M, M, K, "lognormal")
+    f = synth.svdquant_factors(901 + K, 256, K, calib_tokens=256)
+    c_ref, s_ref = orc.quantize(MX, x)
+    xc = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    xs = torch.empty(fb.fp4_sf_bytes(MX, M, K), dtype=torch.uint8, device="cuda")
+    u = torch.empty((M, 64), dtype=torch.bfloat16, device="cuda")
+    fb.w4a4_quantize_act(H.dev_bf16(x), M, K, H.dev_bf16(f["l1_bf16"]), 32, xc, xs, u)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(H.host_u8(xc), c_ref)
+    np.testing.assert_array_equal(H.host_u8(xs), s_ref)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    l1 = synth.bf16_bits_to_f32(f["l1_bf16"]).astype(np.float64)
+    u_ref = xf @ l1
+    mag = np.abs(xf) @ np.abs(l1)
+    pair = u.float().cpu().numpy().astype(np.float64)
+    err = np.abs(pair[:, :32] + pair[:, 32:] - u_ref)
+    assert np.all(err <= 4 * K * 2.0 ** -24 * mag + 2.0 ** -17 * np.abs(u_ref) + 1e-30)
