@@ -56,6 +56,8 @@ def lib():
             "orc_linear_fp64": (None, [P, I64, P, I64, I64, P, P, P]),
             "orc_lowrank_fp64": (None, [P, I64, P, I64, P, P, I64, I64, P, P]),
             "orc_num_threads": (ctypes.c_int, []),
+            "orc_gelu_f64": (D, [D]), "orc_exp_f32": (F, [F]), "orc_gelu_f32": (F, [F]),
+            "orc_gelu_bf16": (None, [P, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -125,6 +127,35 @@ def quantize(fmt: int, x_bf16: np.ndarray, g: float | None = None):
     else:
         lib().orc_quant_nvfp4(_p(x), rows, K, float(g), _p(codes), _p(sf))
     return codes, sf
+
+
+def gelu_f64(z: float) -> float:
+    """Plain GELU-tanh definition in fp64 (R10)."""
+    return lib().orc_gelu_f64(float(z))
+
+
+def exp_f32(a: float) -> float:
+    """The fixed fp32 exp of R10 (Cody-Waite reduction + degree-7 Taylor)."""
+    return lib().orc_exp_f32(float(a))
+
+
+def gelu_f32(z: float) -> float:
+    """The fixed fp32 GELU-tanh evaluation of R10."""
+    return lib().orc_gelu_f32(float(z))
+
+
+def gelu_bf16(z_bf16: np.ndarray) -> np.ndarray:
+    """h = bf16_rn(gelu_f32(z)) element-wise, bf16 bits in and out (R10)."""
+    z = np.ascontiguousarray(z_bf16, dtype=np.uint16)
+    h = np.zeros_like(z)
+    lib().orc_gelu_bf16(_p(z), z.size, _p(h))
+    return h
+
+
+def gelu_quantize(fmt: int, z_bf16: np.ndarray, g: float | None = None):
+    """The down projection's input from the bf16 up-projection output z: GELU-tanh,
+    bf16 rounding, then the format's quantizer (R10 then c-3 / c-4)."""
+    return quantize(fmt, gelu_bf16(z_bf16), g)
 
 
 def quantize_mxfp8(x_bf16: np.ndarray):

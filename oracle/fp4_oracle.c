@@ -34,6 +34,13 @@
  *        off(r, j) = ((r/128)*(Kg/4) + j/4)*512 + (r%32)*16 + ((r%128)/32)*4 + j%4,
  *      rows padded to a multiple of 128 with zero bytes.
  *   R7 W4A8 low-rank term uses the unquantized bf16 input: u = x L1 (fp64).
+ *   R10 the activation between the FFN's two quantized linears (ffn.net.0.proj ->
+ *      ffn.net.2 in the MXFP4 pages' coverage lists) is the tanh-approximated GELU,
+ *        gelu(z) = 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))),
+ *      applied to the bf16 up-projection output z in fp32 and rounded to bf16 before the
+ *      down projection quantizes it.  Because that bf16 value decides integer codes, its
+ *      fp32 evaluation is fixed here (see orc_gelu_f32) and the GPU evaluates the same
+ *      steps; orc_gelu_f64 is the plain definition the fp32 steps are checked against.
  *
  * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC (no fast-math), so every
  * float operation is one IEEE round-to-nearest operation.
@@ -165,6 +172,70 @@ float orc_tensor_amax(const uint16_t* x, int64_t n) {
 float orc_nv_global(float T) {
     if (T == 0.0f) return 1.0f;
     return T / 2688.0f;
+}
+
+/* ------------------------------------------------------------------------------------
+ * GELU-tanh (R10).
+ * ---------------------------------------------------------------------------------- */
+
+/* Plain definition in fp64 (the reference the fp32 evaluation is checked against). */
+double orc_gelu_f64(double z) {
+    const double k = sqrt(2.0 / 3.14159265358979323846);
+    return 0.5 * z * (1.0 + tanh(k * (z + 0.044715 * z * z * z)));
+}
+
+/* exp(a) in fp32 for a in [-87, 88], every step one IEEE fp32 operation:
+ * Cody-Waite argument reduction (W. J. Cody, W. Waite, Software Manual for the Elementary
+ * Functions, 1980): n = floor(a / ln2 + 1/2), r = (a - n ln2_hi) - n ln2_lo, where ln2_hi
+ * has 16 significant bits so n ln2_hi is exact; exp(r), |r| <= ln2/2, by the degree-7
+ * Taylor polynomial in Horner form (truncation below 2^-27); then the exact scaling by
+ * 2^n. */
+float orc_exp_f32(float a) {
+    /* fp32 constants written exactly: 1/ln2, ln2 in two parts, 1/k! for k = 7..3 */
+    const float inv_ln2 = 0x1.715476p+0f;
+    const float ln2_hi = 0x1.62e4p-1f;  /* 0.693145751953125, 16 significant bits */
+    const float ln2_lo = 0x1.7f7d1cp-20f; /* fp32(ln2 - ln2_hi) */
+    const float t = a * inv_ln2;
+    const float fn = floorf(t + 0.5f);
+    const float r = (a - fn * ln2_hi) - fn * ln2_lo;
+    float p = 0x1.a01a02p-13f;      /* 1/5040 */
+    p = p * r + 0x1.6c16c2p-10f;    /* 1/720 */
+    p = p * r + 0x1.111112p-7f;     /* 1/120 */
+    p = p * r + 0x1.555556p-5f;     /* 1/24 */
+    p = p * r + 0x1.555556p-3f;     /* 1/6 */
+    p = p * r + 0.5f;
+    p = p * r + 1.0f;
+    p = p * r + 1.0f;
+    return (float)ldexp((double)p, (int)fn); /* p * 2^n, exact: the result is a normal float */
+}
+
+/* GELU-tanh in fp32, in this fixed order (R10), using 0.5 (1 + tanh(v)) = 1 / (1 + exp(-2v)):
+ *   q = 0.044715 * (z * z);  w = (q + 1) * z;  a = w * (-2 sqrt(2/pi))
+ *   a > 88:  gelu = z * 0 (a signed zero: exp(-2v) overflows, the true value is below 2^-120)
+ *   else:    gelu = z / (1 + exp_f32(max(a, -87)))   (exp(-87) < 2^-125: 1 + it rounds to 1) */
+float orc_gelu_f32(float z) {
+    const float c = 0x1.6e4e26p-5f;   /* fp32(0.044715) */
+    const float k2 = -0x1.988454p+0f; /* fp32(-2 sqrt(2/pi)) */
+    const float q = c * (z * z);
+    const float w = (q + 1.0f) * z;
+    float a = w * k2;
+    if (a > 88.0f) return z * 0.0f;
+    if (a < -87.0f) a = -87.0f;
+    return z / (1.0f + orc_exp_f32(a));
+}
+
+/* IEEE round-to-nearest-even fp32 -> bf16 (finite inputs). */
+static uint16_t f32_to_bf16_rn(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+/* h = bf16_rn(gelu_f32(z)) element-wise: the down projection's input (R10). */
+void orc_gelu_bf16(const uint16_t* z, int64_t n, uint16_t* h) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) h[i] = f32_to_bf16_rn(orc_gelu_f32(orc_bf16_to_f32(z[i])));
 }
 
 /* ------------------------------------------------------------------------------------

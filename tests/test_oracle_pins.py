@@ -343,3 +343,121 @@ def test_wan_a14b_byte_count():
     mx_bytes = params // 2 + params // 32
     assert mx_bytes == 7_464_550_400
     assert abs(mx_bytes / 1e9 - 7.45) < 0.02
+
+
+# ------------------------------------------------------------------ GELU-tanh (R10)
+# The activation between ffn.net.0.proj and ffn.net.2 (the MXFP4 cards' coverage lists):
+# 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))).  The oracle evaluates it in fp32 in a
+# fixed order with its own exp; these pins tie that evaluation to the definition.
+def _f32(v):
+    return float(np.float32(v))
+
+
+def _gelu_arg(z):
+    """a = -2 sqrt(2/pi) (z + 0.044715 z^3), the exp argument of the fp32 evaluation."""
+    return -2.0 * math.sqrt(2.0 / math.pi) * (z + 0.044715 * z ** 3)
+
+
+def test_exp_f32_against_math_exp(orc):
+    """Cody-Waite reduction + degree-7 Taylor: within 2^-22 relative over [-87, 88]."""
+    rng = np.random.default_rng(11)
+    pts = np.concatenate([np.linspace(-87.0, 88.0, 20001), rng.uniform(-87.0, 88.0, 5000),
+                          [0.0, -0.0, 1e-8, -1e-8, 0.34657359, -0.34657359]]).astype(np.float32)
+    worst = 0.0
+    for a in pts:
+        a = float(a)
+        ref = math.exp(a)
+        worst = max(worst, abs(orc.exp_f32(a) - ref) / ref)
+    assert worst <= 2.0 ** -22, worst
+    assert orc.exp_f32(0.0) == 1.0
+    for k in range(-120, 121, 7):  # exp(k ln2) = 2^k, exactly representable
+        a = _f32(k * math.log(2.0))
+        assert abs(orc.exp_f32(a) / math.exp(a) - 1.0) <= 2.0 ** -22
+
+
+def test_gelu_f32_against_tanh_definition(orc):
+    """Where 1 + tanh(v) does not cancel in fp64 (z >= -5) the plain definition is the
+    reference; the fp32 evaluation is within (2|a| + 16) 2^-23 relative of it."""
+    for z in np.linspace(-5.0, 14.0, 19001).astype(np.float32):
+        z = float(z)
+        ref = orc.gelu_f64(z)
+        got = orc.gelu_f32(z)
+        tol = (2.0 * abs(_gelu_arg(z)) + 16.0) * 2.0 ** -23 * abs(ref) + 2.0 ** -126
+        assert abs(got - ref) <= tol, (z, got, ref)
+
+
+def test_gelu_f32_against_library_gelu(orc):
+    """PyTorch's own tanh-approximated GELU in fp64 (a library routine) on random bf16
+    inputs of both signs, within the same bound."""
+    import torch
+
+    rng = np.random.default_rng(12)
+    z = np.concatenate([rng.normal(0.0, 2.0, 4000), rng.uniform(-5.0, 12.0, 2000)])
+    zb = synth.f32_to_bf16_bits(z.astype(np.float32))
+    zf = synth.bf16_bits_to_f32(zb).astype(np.float64)
+    ref = torch.nn.functional.gelu(torch.from_numpy(zf), approximate="tanh").numpy()
+    for zi, ri in zip(zf, ref):
+        if zi < -5.0:
+            continue  # fp64 cancellation in 1 + tanh
+        got = orc.gelu_f32(float(zi))
+        tol = (2.0 * abs(_gelu_arg(zi)) + 16.0) * 2.0 ** -23 * abs(ri) + 2.0 ** -126
+        assert abs(got - ri) <= tol, (zi, got, ri)
+
+
+def test_gelu_f32_tail_against_sigmoid_identity(orc):
+    """On the negative tail the fp64 reference is the exact identity
+    0.5 (1 + tanh(v)) = 1 / (1 + exp(-2v)), itself checked against tanh where both are
+    accurate; the fp32 result is a signed zero once exp(-2v) leaves fp32 (true value
+    below 2^-120)."""
+    for z in np.linspace(-5.0, 5.0, 1001):
+        v = math.sqrt(2.0 / math.pi) * (z + 0.044715 * z ** 3)
+        assert abs(0.5 * (1.0 + math.tanh(v)) - 1.0 / (1.0 + math.exp(-2.0 * v))) <= 1e-15
+    for z in np.linspace(-10.02, -5.0, 5021).astype(np.float32):
+        z = float(z)
+        a = _gelu_arg(z)
+        got = orc.gelu_f32(z)
+        if got == 0.0:
+            assert math.copysign(1.0, got) == -1.0 and a > 87.9
+            assert abs(z / (1.0 + math.exp(a))) < 2.0 ** -120
+            continue
+        ref = z / (1.0 + math.exp(a))
+        assert abs(got - ref) <= (2.0 * abs(a) + 16.0) * 2.0 ** -23 * abs(ref), (z, got, ref)
+    assert math.copysign(1.0, orc.gelu_f32(-11.0)) == -1.0 and orc.gelu_f32(-11.0) == 0.0
+    assert orc.gelu_f32(-3.0e38) == 0.0
+
+
+def test_gelu_f32_special_values(orc):
+    assert orc.gelu_f32(0.0) == 0.0
+    for z in (12.0, 20.0, 1000.0, 3.0e38):  # sigmoid(2v) rounds to 1 in fp32
+        assert orc.gelu_f32(z) == _f32(z)
+    # GELU-tanh(1) = 0.84119199... (the tanh-approximation's value, fp64 definition)
+    assert abs(orc.gelu_f32(1.0) - 0.8411919906082768) <= 2.0 ** -21
+    # odd part: gelu(z) - gelu(-z) = z
+    for z in (0.25, 0.75, 1.5, 2.5, 4.0):
+        assert abs(orc.gelu_f32(z) - orc.gelu_f32(-z) - z) <= 2.0 ** -20 * z
+
+
+def test_gelu_bf16_rounding(orc):
+    """gelu_bf16 rounds the fp32 result to nearest even bf16, brute-forced on small inputs."""
+    import struct
+
+    def bf16_rn(f):
+        u = struct.unpack("<I", struct.pack("<f", f))[0]
+        lower = u & 0xFFFF
+        hi = u >> 16
+        if lower > 0x8000 or (lower == 0x8000 and (hi & 1)):
+            hi += 1
+        return hi & 0xFFFF
+
+    rng = np.random.default_rng(13)
+    z = synth.f32_to_bf16_bits(rng.normal(0.0, 3.0, 3000).astype(np.float32))
+    h = orc.gelu_bf16(z)
+    zf = synth.bf16_bits_to_f32(z)
+    for zi, hi in zip(zf, h):
+        assert int(hi) == bf16_rn(orc.gelu_f32(float(zi)))
+    # the composition used for the fused path: GELU, bf16, then the MXFP4 quantizer
+    zz = z[:2 * 128].reshape(2, 128)
+    c1, s1 = orc.gelu_quantize(orc.MX, zz)
+    c2, s2 = orc.quantize(orc.MX, orc.gelu_bf16(zz))
+    np.testing.assert_array_equal(c1, c2)
+    np.testing.assert_array_equal(s1, s2)
