@@ -7,7 +7,7 @@ arithmetic runs in the library's CUDA kernels.  There is no fallback: if the
 library is missing or the device is not sm_100, the calls raise.
 
 The helpers at the end (pack_weight, quantize_act, linear, pack_lowrank_up, w4a8_linear,
-w4a4_linear)
+w4a4_linear, gelu_quantize_act, linear_gelu_quant)
 allocate outputs and workspaces with torch and call the same entry points.
 """
 from __future__ import annotations
@@ -33,6 +33,7 @@ EXPORTS = [
     "w4a8_quantize_act", "w4a8_gemm", "w4a8_svd_linear", "fp4_sync_status", "fp4_status_string",
     "fp4_set_wait_timeout_ns", "fp4_linear_noalloc", "w4a8_pack_lowrank_up",
     "w4a4_workspace_bytes", "w4a4_quantize_act", "w4a4_gemm", "w4a4_svd_linear",
+    "fp4_gelu_quantize_act", "fp4_gemm_gelu_quant", "fp4_linear_gelu_quant",
 ]
 
 
@@ -68,6 +69,9 @@ def lib():
             "w4a8_quantize_act": (I, [P, I64, I64, P, I, P, P, P, P]),
             "w4a8_pack_lowrank_up": (I, [P, I64, I, P, P]),
             "w4a4_workspace_bytes": (SZ, [I64, I64, I64, I]),
+            "fp4_gelu_quantize_act": (I, [I, P, I64, I64, P, P, P, P]),
+            "fp4_gemm_gelu_quant": (I, [I, P, P, I64, I64, I64, P, P, P, P, P, P, P, P, P]),
+            "fp4_linear_gelu_quant": (I, [I, P, I64, I64, I64, P, P, P, P, P, P, P, P, P, SZ, P]),
             "w4a4_quantize_act": (I, [P, I64, I64, P, I, P, P, P, P]),
             "w4a4_gemm": (I, [P, P, P, I64, I64, I64, P, P, P, I, P, P, P]),
             "w4a4_svd_linear": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, P, SZ, P]),
@@ -167,6 +171,25 @@ def fp4_linear_noalloc(fmt, x, M: int, K: int, N: int, w_codes, w_sf, w_global, 
     memory: the quantized activations use the library's built-in 16 MiB device array."""
     _check(lib().fp4_linear_noalloc(_fmt(fmt), _ptr(x), M, K, N, _ptr(w_codes), _ptr(w_sf), _ptr(w_global),
                                     _ptr(a_global), _ptr(bias), _ptr(y), _stream(stream)), "fp4_linear_noalloc")
+
+
+def fp4_gelu_quantize_act(fmt, z, M: int, K: int, a_global, x_codes, x_sf, stream=None):
+    _check(lib().fp4_gelu_quantize_act(_fmt(fmt), _ptr(z), M, K, _ptr(a_global), _ptr(x_codes), _ptr(x_sf),
+                                       _stream(stream)), "fp4_gelu_quantize_act")
+
+
+def fp4_gemm_gelu_quant(fmt, a_codes, a_sf, M: int, K: int, N: int, w_codes, w_sf, w_global, a_global, bias,
+                        h_global, h_codes, h_sf, stream=None):
+    _check(lib().fp4_gemm_gelu_quant(_fmt(fmt), _ptr(a_codes), _ptr(a_sf), M, K, N, _ptr(w_codes), _ptr(w_sf),
+                                     _ptr(w_global), _ptr(a_global), _ptr(bias), _ptr(h_global), _ptr(h_codes),
+                                     _ptr(h_sf), _stream(stream)), "fp4_gemm_gelu_quant")
+
+
+def fp4_linear_gelu_quant(fmt, x, M: int, K: int, N: int, w_codes, w_sf, w_global, a_global, bias, h_global,
+                          h_codes, h_sf, workspace, ws_bytes: int, stream=None):
+    _check(lib().fp4_linear_gelu_quant(_fmt(fmt), _ptr(x), M, K, N, _ptr(w_codes), _ptr(w_sf), _ptr(w_global),
+                                       _ptr(a_global), _ptr(bias), _ptr(h_global), _ptr(h_codes), _ptr(h_sf),
+                                       _ptr(workspace), ws_bytes, _stream(stream)), "fp4_linear_gelu_quant")
 
 
 def w4a8_quantize_act(x, M: int, K: int, l1, rank: int, x_e4m3, x_sf, u_pair, stream=None):
@@ -315,3 +338,32 @@ def w4a4_linear(x, r: PackedWeight, l1, l2t, bias=None, y=None, workspace=None, 
         workspace = torch.empty(w4a4_workspace_bytes(M, K, r.N, rank), dtype=torch.uint8, device=x.device)
     w4a4_svd_linear(x, M, K, r.N, r.codes, r.sf, l1, l2t, rank, bias, y, workspace, workspace.numel(), stream)
     return y
+
+
+def gelu_quantize_act(z, fmt="mxfp4", a_global=None, stream=None):
+    """bf16 up-projection output z [M, K] (CUDA) -> (codes, scale factors) of
+    bf16(gelu_tanh(z)) in fmt, the down projection's quantized input."""
+    import torch
+
+    f = _fmt(fmt)
+    M, K = z.shape
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=z.device)
+    sf = torch.empty(fp4_sf_bytes(f, M, K), dtype=torch.uint8, device=z.device)
+    fp4_gelu_quantize_act(f, z, M, K, a_global, codes, sf, stream)
+    return codes, sf
+
+
+def linear_gelu_quant(x, pw: PackedWeight, bias=None, a_global=None, h_global=None, workspace=None, stream=None):
+    """Up projection + GELU-tanh + quantize in one GEMM: bf16 x [M, K] -> (codes [M, N/2],
+    scale factors) of h = bf16(gelu_tanh(bf16(x W^T + bias))) in the weight's format."""
+    import torch
+
+    M, K = x.shape
+    N = pw.N
+    codes = torch.empty((M, N // 2), dtype=torch.uint8, device=x.device)
+    sf = torch.empty(fp4_sf_bytes(pw.fmt, M, N), dtype=torch.uint8, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(fp4_linear_workspace_bytes(pw.fmt, M, K, N), dtype=torch.uint8, device=x.device)
+    fp4_linear_gelu_quant(pw.fmt, x, M, K, N, pw.codes, pw.sf, pw.w_global, a_global, bias, h_global, codes, sf,
+                          workspace, workspace.numel(), stream)
+    return codes, sf

@@ -78,7 +78,11 @@ fp4_status_t device_state(DeviceState** out) {
                 cudaFuncSetAttribute(gemm2_kernel<G_W4A8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Gemm2Cfg<G_W4A8>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm2_kernel<G_SVD4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     Gemm2Cfg<G_SVD4>::SMEM_BYTES) != cudaSuccess)
+                                     Gemm2Cfg<G_SVD4>::SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm2_kernel<G_MXFP4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Gemm2Cfg<G_MXFP4>::SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm2_kernel<G_NVFP4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Gemm2Cfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess)
                 return FP4_ERR_CUDA;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.quant_occ[Q_MXFP4], quant_kernel<Q_MXFP4>,
                                                               QUANT_THREADS, 0) != cudaSuccess ||
@@ -135,11 +139,16 @@ int quant_blocks(const DeviceState* ds, int kind, int64_t M, int64_t K) {
     return (int)(blocks < 1 ? 1 : blocks);
 }
 
+// gelu: quantize bf16_rn(gelu_tanh(x)) instead of x (MXFP4 / NVFP4 only)
 fp4_status_t launch_quant(const DeviceState* ds, int kind, const void* x, int64_t M, int64_t K, const float* g,
-                          uint8_t* out, uint8_t* sf, cudaStream_t st) {
+                          uint8_t* out, uint8_t* sf, cudaStream_t st, bool gelu = false) {
     const int blocks = quant_blocks(ds, kind, M, K);
     const uint4* xv = static_cast<const uint4*>(x);
-    if (kind == Q_MXFP4)
+    if (gelu && kind == Q_MXFP4)
+        quant_kernel<Q_MXFP4, true><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
+    else if (gelu)
+        quant_kernel<Q_NVFP4, true><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
+    else if (kind == Q_MXFP4)
         quant_kernel<Q_MXFP4><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
     else if (kind == Q_NVFP4)
         quant_kernel<Q_NVFP4><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
@@ -182,7 +191,8 @@ fp4_status_t encode_sf(CUtensorMap* m, const uint8_t* sf, int64_t rows, int64_t 
 
 // 2-CTA GEMM: A box 128 rows, B box 128 rows (half of the 256-wide N tile) per CTA.
 // tu / tl: the W4A8 low-rank operands (u pair, packed L2); other kinds pass any map.
-template <int KIND>
+// OUTQ != 0: the fused GELU + quantize output (p.h_codes / p.h_sf) instead of p.y.
+template <int KIND, int OUTQ = 0>
 fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CUtensorMap& tb, const uint8_t* sfa,
                           const uint8_t* sfb, GemmParams& p, cudaStream_t st, const CUtensorMap* tu = nullptr,
                           const CUtensorMap* tl = nullptr) {
@@ -192,17 +202,17 @@ fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CU
     if ((s = encode_sf(&tsa, sfa, p.M, p.K, C::G, C::ATOMS)) != FP4_OK) return s;
     if ((s = encode_sf(&tsb, sfb, p.N, p.K, C::G, C::ATOMS)) != FP4_OK) return s;
     // output: bf16 [M, N], stored by the epilogue in 32-row x 64-column boxes (128-byte swizzle)
-    CUtensorMap ty;
-    if ((s = encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.y, (uint64_t)p.N, (uint64_t)p.M,
-                       (uint64_t)p.N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
+    CUtensorMap ty = ta;
+    if (OUTQ == 0 && (s = encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.y, (uint64_t)p.N, (uint64_t)p.M,
+                                    (uint64_t)p.N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
         return s;
     const int tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
     const int pairs = tiles < ds->pairs[KIND] ? tiles : ds->pairs[KIND];
     p.timeout_ns = g_timeout_ns;
     p.skip_iter = g_skip_iter;
     p.status = ds->status;
-    gemm2_kernel<KIND><<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, ty, tu ? *tu : ta,
-                                                                   tl ? *tl : tb, p);
+    gemm2_kernel<KIND, OUTQ><<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, ty, tu ? *tu : ta,
+                                                                         tl ? *tl : tb, p);
     return launched();
 }
 
@@ -267,6 +277,20 @@ fp4_status_t fp4_quantize_act(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int6
     if ((s = device_state(&ds)) != FP4_OK) return s;
     return launch_quant(ds, fmt == FP4_FMT_MXFP4 ? Q_MXFP4 : Q_NVFP4, x_bf16, M, K, a_global, x_codes, x_sf,
                         static_cast<cudaStream_t>(stream));
+}
+
+fp4_status_t fp4_gelu_quantize_act(fp4_fmt_t fmt, const void* z_bf16, int64_t M, int64_t K,
+                                   const float* a_global, uint8_t* x_codes, uint8_t* x_sf, void* stream) {
+    if (!fmt_ok(fmt) || !z_bf16 || !x_codes || !x_sf) return FP4_ERR_INVALID_ARG;
+    if ((fmt == FP4_FMT_NVFP4) != (a_global != nullptr)) return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, 128);
+    if (s != FP4_OK) return s;
+    if (!aligned16(z_bf16) || !aligned16(x_codes) || !aligned16(x_sf) || (reinterpret_cast<uintptr_t>(a_global) & 3u))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    if ((s = device_state(&ds)) != FP4_OK) return s;
+    return launch_quant(ds, fmt == FP4_FMT_MXFP4 ? Q_MXFP4 : Q_NVFP4, z_bf16, M, K, a_global, x_codes, x_sf,
+                        static_cast<cudaStream_t>(stream), true);
 }
 
 fp4_status_t fp4_pack_weight(fp4_fmt_t fmt, const void* w_bf16, int64_t N, int64_t K, uint8_t* w_codes,
@@ -339,6 +363,57 @@ fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K,
         return FP4_ERR_INVALID_ARG;
     if ((s = fp4_quantize_act(fmt, x_bf16, M, K, a_global, codes, sf, stream)) != FP4_OK) return s;
     return fp4_gemm(fmt, codes, sf, M, K, N, w_codes, w_sf, w_global, a_global, bias_f16, y_bf16, stream);
+}
+
+fp4_status_t fp4_gemm_gelu_quant(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf, int64_t M, int64_t K,
+                                 int64_t N, const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
+                                 const float* a_global, const void* bias_f16, const float* h_global,
+                                 uint8_t* h_codes, uint8_t* h_sf, void* stream) {
+    if (!fmt_ok(fmt) || !a_codes || !a_sf || !w_codes || !w_sf || !h_codes || !h_sf) return FP4_ERR_INVALID_ARG;
+    const bool nv = fmt == FP4_FMT_NVFP4;
+    if (nv != (w_global != nullptr) || nv != (a_global != nullptr) || nv != (h_global != nullptr))
+        return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, N);
+    if (s != FP4_OK) return s;
+    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) || !aligned16(bias_f16) ||
+        !aligned16(h_codes) || !aligned16(h_sf) || (reinterpret_cast<uintptr_t>(w_global) & 3u) ||
+        (reinterpret_cast<uintptr_t>(a_global) & 3u) || (reinterpret_cast<uintptr_t>(h_global) & 3u))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    if ((s = device_state(&ds)) != FP4_OK) return s;
+    // always the 2-CTA kernel (its epilogue warps each own 64 columns of a row)
+    CUtensorMap ta, tb;
+    if ((s = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 128, GEMM_BM)) != FP4_OK)
+        return s;
+    if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, K / 2, N, K / 2, 128, 128)) != FP4_OK) return s;
+    GemmParams p{};
+    p.M = (int)M, p.N = (int)N, p.K = (int)K;
+    p.sfa = a_sf, p.sfb = w_sf, p.g_a = a_global, p.g_w = w_global;
+    p.bias = static_cast<const __half*>(bias_f16);
+    p.h_codes = h_codes, p.h_sf = h_sf, p.g_h = h_global;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return nv ? launch_gemm2<G_NVFP4, 2>(ds, ta, tb, a_sf, w_sf, p, st)
+              : launch_gemm2<G_MXFP4, 1>(ds, ta, tb, a_sf, w_sf, p, st);
+}
+
+fp4_status_t fp4_linear_gelu_quant(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K, int64_t N,
+                                   const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
+                                   const float* a_global, const void* bias_f16, const float* h_global,
+                                   uint8_t* h_codes, uint8_t* h_sf, void* workspace, size_t ws_bytes, void* stream) {
+    if (!fmt_ok(fmt) || !x_bf16 || !workspace) return FP4_ERR_INVALID_ARG;
+    fp4_status_t s = check_shape(M, K, N);
+    if (s != FP4_OK) return s;
+    if (ws_bytes < fp4_linear_workspace_bytes(fmt, M, K, N)) return FP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+    uint8_t* codes = static_cast<uint8_t*>(workspace);
+    uint8_t* sf = codes + align256(fp4_codes_bytes(fmt, M, K));
+    const bool nv = fmt == FP4_FMT_NVFP4;
+    if (!w_codes || !w_sf || !h_codes || !h_sf || nv != (w_global != nullptr) || nv != (a_global != nullptr) ||
+        nv != (h_global != nullptr))
+        return FP4_ERR_INVALID_ARG;
+    if ((s = fp4_quantize_act(fmt, x_bf16, M, K, a_global, codes, sf, stream)) != FP4_OK) return s;
+    return fp4_gemm_gelu_quant(fmt, codes, sf, M, K, N, w_codes, w_sf, w_global, a_global, bias_f16, h_global,
+                               h_codes, h_sf, stream);
 }
 
 fp4_status_t w4a8_quantize_act(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16, int rank,

@@ -21,7 +21,9 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "gelu.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace fp4 {
 
@@ -67,6 +69,9 @@ struct GemmParams {
     const float* g_w;
     const __half* bias;       // [N] or null
     __nv_bfloat16* y;         // [M, N]
+    uint8_t* h_codes;         // fused GELU + quantize output: FP4 codes [M, N/2]
+    uint8_t* h_sf;            //   and scale bytes (128x4 atoms over [M, N])
+    const float* g_h;         //   NVFP4 global of that output (device scalar) or null
     uint64_t timeout_ns;
     int skip_iter;            // test hook: producer skips this k-iteration (-1: none)
     int* status;              // device status word
@@ -449,6 +454,66 @@ FP4_DEV void epilogue_stage(const GemmParams& p, uint32_t (&acc)[2][32], int row
         }
 }
 
+// Fused down-projection input (OUTQ 1: MXFP4, 2: NVFP4).  Columns col0 .. col0+63 of one
+// row, rounded to bf16 z by epilogue_pack, become h = bf16_rn(gelu_tanh(z)) (gelu.cuh) and
+// are quantized in the output format's groups along N (MXFP4: 2 groups of 32 with an E8M0
+// scale, NVFP4: 4 groups of 16 with an E4M3 scale under the global g_h) by the same steps
+// as quant_kernel: codes to h_codes[row][col / 2], scale bytes into the 128x4 atoms of the
+// [M, N] activation.  Each thread owns its row, so no group spans threads.  Rows in
+// [M, Mpad) store zero scale bytes (the layout's padding), rows >= Mpad nothing.
+template <int KIND, int OUTQ>
+FP4_DEV void epilogue_gelu_quant(const GemmParams& p, uint32_t (&acc)[2][32], int row, int col0, float gs, float g_h,
+                                 float six_g_h) {
+    const int Mpad = (p.M + 127) & ~127;
+    if (row >= Mpad || col0 >= p.N) return;
+    constexpr int G = (OUTQ == 1) ? 32 : 16;
+    const int64_t apr = p.N / (G * 4);                 // scale atoms per 128-row block
+    const int j0 = col0 / G;                           // first group of the 64 columns
+    uint8_t* word = p.h_sf + sf_word_offset(row, j0 >> 2, apr);
+    uint32_t sfw = 0;                                  // this pair's scale bytes in their word slots
+    if (row < p.M) {
+        epilogue_pack<KIND, 2>(p, acc, row, col0, gs);  // acc[c][w], w < 16: bf16 pairs of z
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            float h[32];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+                h[2 * w] = gelu_bf16_f32(__uint_as_float(acc[c][w] << 16));
+                h[2 * w + 1] = gelu_bf16_f32(__uint_as_float(acc[c][w] & 0xFFFF0000u));
+            }
+            uint32_t cw[4];
+#pragma unroll
+            for (int g = 0; g < 32 / G; ++g) {
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < G; ++i) amax = fmaxf(amax, fabsf(h[g * G + i]));
+                uint32_t sfb;
+                if (OUTQ == 1) {
+                    sfb = mx_scale_byte<2>(amax);
+                    const float inv = mx_inv_scale(sfb);
+#pragma unroll
+                    for (int i = 0; i < G; ++i) h[g * G + i] = __fmul_rn(h[g * G + i], inv);
+                } else {
+                    sfb = cvt_e4m3x2(__fdiv_rn(amax, six_g_h), 0.0f) & 0xFFu;
+                    const float d = __fmul_rn(e4m3_to_f32(sfb), g_h);
+                    const float r = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+#pragma unroll
+                    for (int i = 0; i < G; ++i) h[g * G + i] = (d == 0.0f) ? 0.0f : __fmul_rn(h[g * G + i], r);
+                }
+                sfw |= sfb << (8 * ((j0 + c * (32 / G) + g) & 3));
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cw[q] = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(h + 8 * q));
+            *reinterpret_cast<uint4*>(p.h_codes + (size_t)row * (p.N / 2) + col0 / 2 + 16 * c) =
+                make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        }
+    }
+    if (OUTQ == 1)  // groups j0, j0 + 1: one half of the atom word
+        *reinterpret_cast<uint16_t*>(word + (j0 & 3)) = (uint16_t)(sfw >> (8 * (j0 & 3)));
+    else            // groups j0 .. j0 + 3: the whole word
+        *reinterpret_cast<uint32_t*>(word) = sfw;
+}
+
 FP4_DEV void gemm2_fail(const GemmParams& p, volatile int* abort, uint32_t peer_abort) {
     *abort = 1;
     st_cluster_u32(peer_abort, 1u);
@@ -465,7 +530,9 @@ FP4_DEV void arrive_leader_relaxed(uint64_t* bar, uint32_t rank) {
         mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(bar), 0));
 }
 
-template <int KIND>
+// OUTQ 0: bf16 output through the TMA-store epilogue; 1 / 2: the fused GELU + MXFP4 /
+// NVFP4 quantize epilogue (epilogue_gelu_quant) in place of the bf16 output.
+template <int KIND, int OUTQ = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THREADS, 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
@@ -769,6 +836,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         uint32_t acc[2][32];
         float gs = 1.0f;
         if (KIND == G_NVFP4) gs = __fmul_rn(*p.g_a, *p.g_w);
+        float g_h = 1.0f, six_g_h = 6.0f;
+        if (OUTQ == 2) {
+            g_h = *p.g_h;
+            six_g_h = __fmul_rn(6.0f, g_h);
+        }
         int tcount = 0;
         for (int tile = pair; tile < num_tiles; tile += num_pairs, ++tcount) {
             const int mb = tile / num_n, nb = tile % num_n;
@@ -787,6 +859,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             // pack 64 columns into the staging tile and hand them to one TMA store (which
             // clips rows at or beyond M); the tile is reused once the previous store has read it
             auto stage_store = [&](int chunk) {
+                if (OUTQ != 0) {
+                    epilogue_gelu_quant<KIND, OUTQ>(p, acc, row, col0 + chunk * 32, gs, g_h, six_g_h);
+                    return;
+                }
                 if (col0 >= p.N) return;
                 if (lane == 0) bulk_wait_group_read0();
                 __syncwarp();

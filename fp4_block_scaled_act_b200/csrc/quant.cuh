@@ -11,6 +11,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "gelu.cuh"
 #include "ptx.cuh"
 
 namespace fp4 {
@@ -45,7 +46,9 @@ FP4_DEV uint32_t mx_scale_byte(float amax) {
 // 2^-e for e = byte - 127, exact (byte <= 252 keeps the result a normal float).
 FP4_DEV float mx_inv_scale(uint32_t byte) { return __uint_as_float((254u - byte) << 23); }
 
-template <int KIND>
+// GELU = true: the input is the bf16 up-projection output z and the quantized value is
+// bf16_rn(gelu_tanh(z)) (gelu.cuh), the down projection's activation.
+template <int KIND, bool GELU = false>
 __global__ void __launch_bounds__(QUANT_THREADS) quant_kernel(const uint4* __restrict__ x, int64_t M, int64_t K,
                                                               const float* __restrict__ g_ptr,
                                                               uint8_t* __restrict__ out, uint8_t* __restrict__ sf) {
@@ -97,6 +100,10 @@ __global__ void __launch_bounds__(QUANT_THREADS) quant_kernel(const uint4* __res
             if (u >= u_end) break;  // uniform across the warp (ranges are even)
             float v[8];
             bf16x8_to_f32(raw[it], v);
+            if (GELU) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = gelu_bf16_f32(v[i]);
+            }
             float amax = 0.0f;
 #pragma unroll
             for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));

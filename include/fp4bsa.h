@@ -168,6 +168,51 @@ fp4_status_t fp4_linear_noalloc(fp4_fmt_t fmt, const void* x_bf16, int64_t M, in
                                 const float* a_global, const void* bias_f16, void* y_bf16,
                                 void* stream);
 
+/* ----------------------------------------------------------------- fused FFN activation */
+
+/* The Wan2.2 FFN applies GELU-tanh between its two quantized linears (ffn.net.0.proj ->
+ * ffn.net.2, MXFP4 card Quantization Details coverage list).  These calls produce the
+ * down projection's quantized input, h = bf16_rn(gelu_tanh(z)) with z the bf16
+ * up-projection output, without writing z to memory.  gelu_tanh(z) is
+ * 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))) evaluated in fp32 in a fixed order:
+ *   q = 0.044715 (z z); w = (q + 1) z; a = -2 sqrt(2/pi) w;
+ *   a > 88: z * 0;  otherwise z / (1 + exp(max(a, -87)))
+ * with exp by Cody-Waite reduction (n = floor(a / ln2 + 1/2), ln2 split into a 16-bit and
+ * a remainder part) and the degree-7 Taylor polynomial, each step one IEEE fp32
+ * operation, so the codes are reproducible bit for bit.  h is then quantized exactly as
+ * fp4_quantize_act quantizes x (same formats, layouts and NVFP4 global rule). */
+
+/* Standalone: z_bf16 [M, K] bf16 (the up-projection output) -> codes [M, K/2] and scale
+ * factors of h in `fmt`; a_global is the down projection's static activation global
+ * (NVFP4) or NULL (MXFP4). */
+fp4_status_t fp4_gelu_quantize_act(fp4_fmt_t fmt, const void* z_bf16, int64_t M, int64_t K,
+                                   const float* a_global, uint8_t* x_codes, uint8_t* x_sf,
+                                   void* stream);
+
+/* The up projection with the activation fused into its epilogue: same operands as
+ * fp4_gemm (a_codes, a_sf [M, K]; w_codes, w_sf [N, K]; NVFP4 globals; bias [N] or NULL),
+ * but instead of y it writes z = bf16_rn(acc (g_a g_w) + bias), h = bf16_rn(gelu_tanh(z)),
+ * quantized in the same format `fmt`:
+ *   h_global (device) NVFP4: the down projection's static activation global; MXFP4: NULL
+ *   h_codes  (device, out) [M, N/2];  h_sf (device, out) fp4_sf_bytes(fmt, M, N) bytes
+ * i.e. exactly the x_codes / x_sf that fp4_quantize_act would produce from h, ready as the
+ * A operand of the down projection (K' = N).  Always the 2-CTA kernel. */
+fp4_status_t fp4_gemm_gelu_quant(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf,
+                                 int64_t M, int64_t K, int64_t N, const uint8_t* w_codes,
+                                 const uint8_t* w_sf, const float* w_global,
+                                 const float* a_global, const void* bias_f16,
+                                 const float* h_global, uint8_t* h_codes, uint8_t* h_sf,
+                                 void* stream);
+
+/* fp4_quantize_act of x into `workspace` (fp4_linear_workspace_bytes), then
+ * fp4_gemm_gelu_quant. */
+fp4_status_t fp4_linear_gelu_quant(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K,
+                                   int64_t N, const uint8_t* w_codes, const uint8_t* w_sf,
+                                   const float* w_global, const float* a_global,
+                                   const void* bias_f16, const float* h_global,
+                                   uint8_t* h_codes, uint8_t* h_sf, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
 /* ----------------------------------------------------------------- W4A8 SVDQuant */
 
 /* Activation side of the W4A8 SVDQuant linear (W4A8 README: "dynamic MXFP8

@@ -104,6 +104,14 @@ def test_invalid_calls_rejected_before_launch(fb):
     assert L.w4a4_gemm(A, A, A, 16, 256, 384, A, A, A, 32, None, bad, st) == 3
     assert L.w4a4_svd_linear(A, 16, 256, 256, A, A, A, A, 32, None, A, A, 10, st) == 4
     assert L.w4a4_quantize_act(A, 16, 256, A, 32, A, A, None, st) == 1
+    # fused GELU + quantize: NVFP4 needs the output global, MXFP4 must not get one
+    assert L.fp4_gemm_gelu_quant(1, A, A, 16, 256, 256, A, A, A, A, None, None, A, A, st) == 1
+    assert L.fp4_gemm_gelu_quant(0, A, A, 16, 256, 256, A, A, None, None, None, A, A, A, st) == 1
+    assert L.fp4_gemm_gelu_quant(0, A, A, 16, 256, 200, A, A, None, None, None, None, A, A, st) == 2
+    assert L.fp4_gemm_gelu_quant(0, A, A, 16, 256, 256, A, A, None, None, None, None, bad, A, st) == 3
+    assert L.fp4_linear_gelu_quant(0, A, 16, 256, 256, A, A, None, None, None, None, A, A, A, 10, st) == 4
+    assert L.fp4_gelu_quantize_act(1, A, 16, 256, None, A, A, st) == 1
+    assert L.fp4_gelu_quantize_act(0, A, 16, 200, None, A, A, st) == 2
     # weight pack: MXFP4 must not get a global
     assert L.fp4_pack_weight(0, A, 256, 256, A, A, A, st) == 1
     assert L.fp4_tensor_amax(A, 0, A, st) == 1

@@ -231,6 +231,52 @@ def test_w4a8_full_size_sampled(fb, orc):
     _w4a8_check(fb, orc, M, K, N, seed=3001, rows=rows, calib=2048)
 
 
+# ------------------------------------------------------------------ up projection + GELU + quantize
+# The FFN's up projection with GELU-tanh and the down projection's quantizer fused into its
+# epilogue.  z (the bf16 GEMM result) is only known to the GEMM tolerance, so the output is
+# checked for validity (tests/gpu_helpers.check_gelu_quant) and for its agreement rate with
+# the oracle's own choice of z.
+def _gelu_linear_case(fb, orc, fmt, M, K, N, x, w, b, rows, what):
+    import torch
+
+    g_a = orc.nv_global(orc.tensor_amax(x)) if fmt == NV else None
+    Y, S = _oracle(orc, fmt, x, w, b, rows, g_a)
+    g_h = None
+    if fmt == NV:  # the down projection's static global, from the oracle's own output
+        zb = H._bf16_bracket(Y)[0]
+        g_h = orc.nv_global(orc.tensor_amax(orc.gelu_bf16(zb)))
+    pw = fb.pack_weight(H.dev_bf16(w), fmt)
+    codes, sf = fb.linear_gelu_quant(H.dev_bf16(x), pw, H.dev_f16(b) if b is not None else None,
+                                     H.dev_f32([g_a]) if fmt == NV else None,
+                                     H.dev_f32([g_h]) if fmt == NV else None)
+    st = fb.fp4_sync_status()
+    assert st == 0, fb.fp4_status_string(st)
+    torch.cuda.synchronize()
+    agree = H.check_gelu_quant(fmt, codes, sf, Y, S, rows, M, N, g_h, what)
+    assert agree > 0.99, (what, agree)
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("M,K,N", [(1, 256, 256), (129, 512, 384), (300, 768, 512), (600, 1280, 1024)])
+def test_linear_gelu_quant_small(fb, orc, fmt, M, K, N):
+    x = synth.activation(60 * M + K, M, K, "lognormal")
+    w = synth.weight(70 * N + K, N, K)
+    b = synth.bias(N + 11, N)
+    _gelu_linear_case(fb, orc, fmt, M, K, N, x, w, b, np.arange(M), f"gelu fmt={fmt} M={M} K={K} N={N}")
+
+
+@pytest.mark.parametrize("cfg,fmt", [(2, NV), (4, MX)])
+def test_linear_gelu_quant_full_size_sampled(fb, orc, cfg, fmt):
+    """ffn up projection 75600 x 5120 -> 13824 with GELU and the down projection's quantizer."""
+    M, K, N = 75600, 5120, 13824
+    s = synth.seeds_for(cfg, layer=K // 1000 + N // 1000)
+    x = synth.activation(s["x"], M, K, "lognormal", gain_seed=s["gain"])
+    w = synth.weight(s["w"], N, K)
+    b = synth.bias(s["bias"], N)
+    rows = H.sample_rows(M, n_random=24, seed=cfg + 50)
+    _gelu_linear_case(fb, orc, fmt, M, K, N, x, w, b, rows, f"gelu full cfg={cfg} fmt={fmt}")
+
+
 # ------------------------------------------------------------------ W4A4 SVDQuant linear
 # The W4A8 README's experimental W4A4 variant: MXFP4 activations on the same factors.
 def _w4a4_check(fb, orc, M, K, N, seed, rows=None, calib=256):

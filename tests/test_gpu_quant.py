@@ -253,3 +253,48 @@ def test_w4a4_quantize_act(fb, orc, M, K):
     pair = u.float().cpu().numpy().astype(np.float64)
     err = np.abs(pair[:, :32] + pair[:, 32:] - u_ref)
     assert np.all(err <= 4 * K * 2.0 ** -24 * mag + 2.0 ** -17 * np.abs(u_ref) + 1e-30)
+
+
+# ------------------------------------------------------------------ GELU-tanh + quantize (R10)
+def _gelu_sweep_bits():
+    """Every bf16 value with |z| <= 16, both signs, in rows of 256 (zero padded)."""
+    pos = np.arange(0x0000, 0x4181, dtype=np.uint16)  # 0x4180 = 16.0
+    z = np.concatenate([pos, pos | np.uint16(0x8000)])
+    pad = (-z.size) % 256
+    return np.concatenate([z, np.zeros(pad, dtype=np.uint16)]).reshape(-1, 256)
+
+
+def _gelu_case(fb, orc, fmt, z):
+    import torch
+
+    M, K = z.shape
+    g = orc.nv_global(orc.tensor_amax(orc.gelu_bf16(z))) if fmt == NV else None
+    c_ref, s_ref = orc.gelu_quantize(fmt, z, g)
+    codes, sf = fb.gelu_quantize_act(H.dev_bf16(z), fmt, H.dev_f32([g]) if fmt == NV else None)
+    torch.cuda.synchronize()
+    got_c, got_s = H.host_u8(codes), H.host_u8(sf)
+    if not np.array_equal(got_c, c_ref):
+        i = tuple(np.argwhere(got_c != c_ref)[0])
+        zf = synth.bf16_bits_to_f32(z)
+        raise AssertionError(f"fmt={fmt}: codes differ at {i} (z near {zf[i[0], 2 * i[1]]!r})")
+    np.testing.assert_array_equal(got_s, s_ref)
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+def test_gelu_quantize_act_every_bf16_in_range(fb, orc, fmt):
+    """bf16(gelu_tanh(z)) quantized, bit-exact against the oracle for every bf16 |z| <= 16."""
+    _gelu_case(fb, orc, fmt, _gelu_sweep_bits())
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("M,K,sigma", [(1, 256, 0.3), (130, 512, 1.0), (300, 13824, 3.0)])
+def test_gelu_quantize_act_shapes(fb, orc, fmt, M, K, sigma):
+    rng = np.random.default_rng(M + K)
+    z = synth.f32_to_bf16_bits((rng.normal(0.0, sigma, (M, K))).astype(np.float32))
+    _gelu_case(fb, orc, fmt, z)
+
+
+def test_gelu_quantize_act_full_size_nvfp4(fb, orc):
+    """The ffn down projection's input at the full shape (M = 75600, K = 13824), NVFP4."""
+    z = synth.activation(7100, 75600, 13824, "lognormal")
+    _gelu_case(fb, orc, NV, z)
