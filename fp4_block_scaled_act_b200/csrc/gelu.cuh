@@ -5,46 +5,72 @@
 //   gelu(z) = 0.5 z (1 + tanh(v)),  v = sqrt(2/pi) (z + 0.044715 z^3).
 // The down projection quantizes bf16_rn(gelu(z)), so the integer codes depend on every
 // rounding of this evaluation; it is therefore written out step by step (no library
-// transcendental, no contracted multiply-add) as
-//   q = 0.044715 (z z);  w = (q + 1) z;  a = w (-2 sqrt(2/pi))          [a = -2v]
-//   a > 88:  gelu = z * 0     (exp(a) leaves fp32; the true value is below 2^-120)
-//   else:    gelu = z / (1 + exp(max(a, -87)))    using 0.5 (1 + tanh v) = 1 / (1 + exp(-2v))
-// with exp by Cody-Waite argument reduction (W. J. Cody and W. Waite, "Software Manual
-// for the Elementary Functions", 1980): n = floor(a / ln2 + 1/2), r = (a - n ln2_hi) -
-// n ln2_lo with a 16-bit ln2_hi (so n ln2_hi is exact), exp(r) for |r| <= ln2/2 by the
-// degree-7 Taylor polynomial in Horner form, then the exact scaling by 2^n (a normal
-// float for a in [-87, 88]).  Every constant is written exactly as an fp32 hex literal.
+// transcendental or division; every operation, fused multiply-add included, one IEEE
+// fp32 operation, so a plain C restatement reproduces it bit for bit):
+//   q = z z;  p = q 0.044715;  w = fma(p, z, z)                  [w = z + 0.044715 z^3]
+//   t = w (-2 sqrt(2/pi) / ln 2)                                 [exp(-2v) = 2^t]
+//   t > 125:  gelu = z * 0   (the true value is below 2^-118 |z|)
+//   else:     t = max(t, -126)
+//             2^t: n = (t + 1.5 2^23) - 1.5 2^23 (t rounded to the nearest integer, ties
+//             to even, by two additions), f = t - n (exact, |f| <= 1/2), 2^f by the
+//             degree-6 Taylor polynomial in ln2 f (Horner with fma; relative error below
+//             2^-22 on |f| <= 1/2), times 2^n exactly
+//             d = 1 + 2^t;  y = 1/d by Newton-Raphson: y0 from the exponent bits
+//             (bits(y0) = 0x7EF311C7 - bits(d), within 1/8 of 1/d), three steps
+//             r = fma(-d, y, 1), y = fma(y, r, y) (each squares the relative error)
+//             gelu = z y           using 0.5 (1 + tanh v) = 1 / (1 + exp(-2v))
+// Pairs of values are evaluated with the packed f32x2 operations of sm_100 (each lane an
+// IEEE fp32 operation).  Every constant is written exactly as an fp32 hex literal.
 #pragma once
 #include "ptx.cuh"
 
 namespace fp4 {
 
-FP4_DEV float exp_cw_f32(float a) {
-    const float t = __fmul_rn(a, 0x1.715476p+0f);  // 1/ln2
-    const float fn = floorf(__fadd_rn(t, 0.5f));
-    const float r = __fsub_rn(__fsub_rn(a, __fmul_rn(fn, 0x1.62e4p-1f)), __fmul_rn(fn, 0x1.7f7d1cp-20f));
-    float p = 0x1.a01a02p-13f;                          // 1/7!
-    p = __fadd_rn(__fmul_rn(p, r), 0x1.6c16c2p-10f);    // 1/6!
-    p = __fadd_rn(__fmul_rn(p, r), 0x1.111112p-7f);     // 1/5!
-    p = __fadd_rn(__fmul_rn(p, r), 0x1.555556p-5f);     // 1/4!
-    p = __fadd_rn(__fmul_rn(p, r), 0x1.555556p-3f);     // 1/3!
-    p = __fadd_rn(__fmul_rn(p, r), 0.5f);
-    p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-    p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-    const int n = (int)fn;  // in [-126, 127] for a in [-87, 88]
-    return __fmul_rn(p, __int_as_float((n + 127) << 23));
+// bf16_rn of a finite fp32 value, returned as fp32 (round to nearest even on the bits)
+FP4_DEV float bf16_rn_f32(float g) {
+    uint32_t u = __float_as_uint(g);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return __uint_as_float(u & 0xFFFF0000u);
 }
 
-FP4_DEV float gelu_tanh_f32(float z) {
-    const float q = __fmul_rn(0x1.6e4e26p-5f, __fmul_rn(z, z));  // 0.044715 z^2
-    const float w = __fmul_rn(__fadd_rn(q, 1.0f), z);
-    float a = __fmul_rn(w, -0x1.988454p+0f);  // -2 sqrt(2/pi)
-    if (a > 88.0f) return __fmul_rn(z, 0.0f);
-    a = fmaxf(a, -87.0f);
-    return __fdiv_rn(z, __fadd_rn(1.0f, exp_cw_f32(a)));
+// h = bf16_rn(gelu_tanh(z)) for the pair (z0, z1)
+FP4_DEV void gelu_bf16_x2(float z0, float z1, float& h0, float& h1) {
+    const uint64_t z = f2_pack(z0, z1);
+    const uint64_t p = f2_mul(f2_mul(z, z), f2_splat(0x1.6e4e26p-5f));  // 0.044715 z^2
+    const uint64_t w = f2_fma(p, z, z);                                  // z + 0.044715 z^3
+    float t0, t1;
+    f2_unpack(f2_mul(w, f2_splat(-0x1.26aec2p+1f)), t0, t1);            // -2 sqrt(2/pi) / ln2
+    const bool cut0 = t0 > 125.0f, cut1 = t1 > 125.0f;
+    const uint64_t t = f2_pack(fminf(fmaxf(t0, -126.0f), 125.0f), fminf(fmaxf(t1, -126.0f), 125.0f));
+    // 2^t
+    const uint64_t big = f2_add(t, f2_splat(0x1.8p23f));
+    const uint64_t f = f2_sub(t, f2_sub(big, f2_splat(0x1.8p23f)));
+    uint64_t e = f2_splat(0x1.430912p-13f);                // (ln2)^6 / 6!
+    e = f2_fma(e, f, f2_splat(0x1.5d87fep-10f));           // (ln2)^5 / 5!
+    e = f2_fma(e, f, f2_splat(0x1.3b2ab6p-7f));            // (ln2)^4 / 4!
+    e = f2_fma(e, f, f2_splat(0x1.c6b08ep-5f));            // (ln2)^3 / 3!
+    e = f2_fma(e, f, f2_splat(0x1.ebfbe0p-3f));            // (ln2)^2 / 2!
+    e = f2_fma(e, f, f2_splat(0x1.62e430p-1f));            // ln2
+    e = f2_fma(e, f, f2_splat(1.0f));
+    float b0, b1;
+    f2_unpack(big, b0, b1);  // n in the low mantissa bits of big
+    const uint64_t s2 = f2_pack(__uint_as_float((__float_as_uint(b0) - 0x4B400000u + 127u) << 23),
+                                __uint_as_float((__float_as_uint(b1) - 0x4B400000u + 127u) << 23));
+    const uint64_t d = f2_add(f2_splat(1.0f), f2_mul(e, s2));
+    // y = 1/d by Newton-Raphson from the exponent-bit guess
+    float d0, d1;
+    f2_unpack(d, d0, d1);
+    uint64_t y = f2_pack(__uint_as_float(0x7EF311C7u - __float_as_uint(d0)),
+                         __uint_as_float(0x7EF311C7u - __float_as_uint(d1)));
+    const uint64_t nd = d ^ 0x8000000080000000ull;  // -d, exactly
+#pragma unroll
+    for (int i = 0; i < 3; ++i) y = f2_fma(y, f2_fma(nd, y, f2_splat(1.0f)), y);
+    float g0, g1;
+    f2_unpack(f2_mul(z, y), g0, g1);
+    if (cut0) g0 = __fmul_rn(z0, 0.0f);
+    if (cut1) g1 = __fmul_rn(z1, 0.0f);
+    h0 = bf16_rn_f32(g0);
+    h1 = bf16_rn_f32(g1);
 }
-
-// bf16_rn(gelu(z)) as an fp32 value
-FP4_DEV float gelu_bf16_f32(float z) { return __bfloat162float(__float2bfloat16_rn(gelu_tanh_f32(z))); }
 
 }  // namespace fp4

@@ -477,10 +477,9 @@ FP4_DEV void epilogue_gelu_quant(const GemmParams& p, uint32_t (&acc)[2][32], in
         for (int c = 0; c < 2; ++c) {
             float h[32];
 #pragma unroll
-            for (int w = 0; w < 16; ++w) {
-                h[2 * w] = gelu_bf16_f32(__uint_as_float(acc[c][w] << 16));
-                h[2 * w + 1] = gelu_bf16_f32(__uint_as_float(acc[c][w] & 0xFFFF0000u));
-            }
+            for (int w = 0; w < 16; ++w)
+                gelu_bf16_x2(__uint_as_float(acc[c][w] << 16), __uint_as_float(acc[c][w] & 0xFFFF0000u), h[2 * w],
+                             h[2 * w + 1]);
             uint32_t cw[4];
 #pragma unroll
             for (int g = 0; g < 32 / G; ++g) {

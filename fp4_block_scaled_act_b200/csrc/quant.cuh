@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(QUANT_THREADS) quant_kernel(const uint4* __res
             bf16x8_to_f32(raw[it], v);
             if (GELU) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = gelu_bf16_f32(v[i]);
+                for (int i = 0; i < 8; i += 2) gelu_bf16_x2(v[i], v[i + 1], v[i], v[i + 1]);
             }
             float amax = 0.0f;
 #pragma unroll

@@ -56,7 +56,7 @@ def lib():
             "orc_linear_fp64": (None, [P, I64, P, I64, I64, P, P, P]),
             "orc_lowrank_fp64": (None, [P, I64, P, I64, P, P, I64, I64, P, P]),
             "orc_num_threads": (ctypes.c_int, []),
-            "orc_gelu_f64": (D, [D]), "orc_exp_f32": (F, [F]), "orc_gelu_f32": (F, [F]),
+            "orc_gelu_f64": (D, [D]), "orc_exp2_f32": (F, [F]), "orc_recip_f32": (F, [F]), "orc_gelu_f32": (F, [F]),
             "orc_gelu_bf16": (None, [P, I64, P]),
         }
         for name, (res, args) in sig.items():
@@ -134,9 +134,14 @@ def gelu_f64(z: float) -> float:
     return lib().orc_gelu_f64(float(z))
 
 
-def exp_f32(a: float) -> float:
-    """The fixed fp32 exp of R10 (Cody-Waite reduction + degree-7 Taylor)."""
-    return lib().orc_exp_f32(float(a))
+def exp2_f32(t: float) -> float:
+    """The fixed fp32 2^t of R10 (floor reduction + degree-6 Taylor in ln2 f, fma Horner)."""
+    return lib().orc_exp2_f32(float(t))
+
+
+def recip_f32(d: float) -> float:
+    """The fixed fp32 Newton-Raphson reciprocal of R10."""
+    return lib().orc_recip_f32(float(d))
 
 
 def gelu_f32(z: float) -> float:

@@ -41,6 +41,8 @@
  *      down projection quantizes it.  Because that bf16 value decides integer codes, its
  *      fp32 evaluation is fixed here (see orc_gelu_f32) and the GPU evaluates the same
  *      steps; orc_gelu_f64 is the plain definition the fp32 steps are checked against.
+ *      fmaf below is the C99 correctly rounded fused multiply-add (one IEEE operation),
+ *      not a contraction; -ffp-contract=off keeps every other expression unfused.
  *
  * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC (no fast-math), so every
  * float operation is one IEEE round-to-nearest operation.
@@ -184,44 +186,54 @@ double orc_gelu_f64(double z) {
     return 0.5 * z * (1.0 + tanh(k * (z + 0.044715 * z * z * z)));
 }
 
-/* exp(a) in fp32 for a in [-87, 88], every step one IEEE fp32 operation:
- * Cody-Waite argument reduction (W. J. Cody, W. Waite, Software Manual for the Elementary
- * Functions, 1980): n = floor(a / ln2 + 1/2), r = (a - n ln2_hi) - n ln2_lo, where ln2_hi
- * has 16 significant bits so n ln2_hi is exact; exp(r), |r| <= ln2/2, by the degree-7
- * Taylor polynomial in Horner form (truncation below 2^-27); then the exact scaling by
- * 2^n. */
-float orc_exp_f32(float a) {
-    /* fp32 constants written exactly: 1/ln2, ln2 in two parts, 1/k! for k = 7..3 */
-    const float inv_ln2 = 0x1.715476p+0f;
-    const float ln2_hi = 0x1.62e4p-1f;  /* 0.693145751953125, 16 significant bits */
-    const float ln2_lo = 0x1.7f7d1cp-20f; /* fp32(ln2 - ln2_hi) */
-    const float t = a * inv_ln2;
-    const float fn = floorf(t + 0.5f);
-    const float r = (a - fn * ln2_hi) - fn * ln2_lo;
-    float p = 0x1.a01a02p-13f;      /* 1/5040 */
-    p = p * r + 0x1.6c16c2p-10f;    /* 1/720 */
-    p = p * r + 0x1.111112p-7f;     /* 1/120 */
-    p = p * r + 0x1.555556p-5f;     /* 1/24 */
-    p = p * r + 0x1.555556p-3f;     /* 1/6 */
-    p = p * r + 0.5f;
-    p = p * r + 1.0f;
-    p = p * r + 1.0f;
-    return (float)ldexp((double)p, (int)fn); /* p * 2^n, exact: the result is a normal float */
+/* 2^t in fp32 for t in [-126, 127], every step one IEEE fp32 operation (fmaf is one
+ * correctly rounded fused multiply-add): n = (t + 1.5 2^23) - 1.5 2^23, t rounded to the
+ * nearest integer (ties to even) by two additions, f = t - n (exact, |f| <= 1/2),
+ * 2^f = exp(f ln2) by its degree-6 Taylor polynomial in Horner form with the coefficients
+ * (ln2)^k / k! rounded to fp32 (truncation below 2^-23 on |f| <= 1/2), then the exact
+ * scaling by 2^n (the result is a normal float). */
+float orc_exp2_f32(float t) {
+    const float big = t + 0x1.8p23f;
+    const float fn = big - 0x1.8p23f;
+    const float f = t - fn;
+    float p = 0x1.430912p-13f;        /* (ln2)^6 / 6! */
+    p = fmaf(p, f, 0x1.5d87fep-10f);  /* (ln2)^5 / 5! */
+    p = fmaf(p, f, 0x1.3b2ab6p-7f);   /* (ln2)^4 / 4! */
+    p = fmaf(p, f, 0x1.c6b08ep-5f);   /* (ln2)^3 / 3! */
+    p = fmaf(p, f, 0x1.ebfbe0p-3f);   /* (ln2)^2 / 2! */
+    p = fmaf(p, f, 0x1.62e430p-1f);   /* ln2 */
+    p = fmaf(p, f, 1.0f);
+    return (float)ldexp((double)p, (int)fn); /* p * 2^n, exact */
 }
 
-/* GELU-tanh in fp32, in this fixed order (R10), using 0.5 (1 + tanh(v)) = 1 / (1 + exp(-2v)):
- *   q = 0.044715 * (z * z);  w = (q + 1) * z;  a = w * (-2 sqrt(2/pi))
- *   a > 88:  gelu = z * 0 (a signed zero: exp(-2v) overflows, the true value is below 2^-120)
- *   else:    gelu = z / (1 + exp_f32(max(a, -87)))   (exp(-87) < 2^-125: 1 + it rounds to 1) */
+/* 1/d in fp32 for d in [1, 2^126) by Newton-Raphson: the initial guess takes its bits
+ * from d's (bits(y0) = 0x7EF311C7 - bits(d): the exponent negated, within 1/8 of 1/d),
+ * then three steps r = fma(-d, y, 1), y = fma(y, r, y), each squaring the relative error
+ * (below 2^-23 after three). */
+float orc_recip_f32(float d) {
+    uint32_t u;
+    memcpy(&u, &d, 4);
+    u = 0x7EF311C7u - u;
+    float y;
+    memcpy(&y, &u, 4);
+    for (int i = 0; i < 3; ++i) y = fmaf(y, fmaf(-d, y, 1.0f), y);
+    return y;
+}
+
+/* GELU-tanh in fp32, in this fixed order (R10), using 0.5 (1 + tanh(v)) = 1 / (1 + exp(-2v))
+ * and exp(-2v) = 2^t:
+ *   q = z z;  p = q 0.044715;  w = fma(p, z, z);  t = w * (-2 sqrt(2/pi) / ln2)
+ *   t > 125:  gelu = z * 0 (a signed zero; the true value is below 2^-118 |z|)
+ *   else:     gelu = z * recip(1 + exp2_f32(max(t, -126))) */
 float orc_gelu_f32(float z) {
     const float c = 0x1.6e4e26p-5f;   /* fp32(0.044715) */
-    const float k2 = -0x1.988454p+0f; /* fp32(-2 sqrt(2/pi)) */
-    const float q = c * (z * z);
-    const float w = (q + 1.0f) * z;
-    float a = w * k2;
-    if (a > 88.0f) return z * 0.0f;
-    if (a < -87.0f) a = -87.0f;
-    return z / (1.0f + orc_exp_f32(a));
+    const float k = -0x1.26aec2p+1f;  /* fp32(-2 sqrt(2/pi) / ln2) */
+    const float p = (z * z) * c;
+    const float w = fmaf(p, z, z);
+    float t = w * k;
+    if (t > 125.0f) return z * 0.0f;
+    if (t < -126.0f) t = -126.0f;
+    return z * orc_recip_f32(1.0f + orc_exp2_f32(t));
 }
 
 /* IEEE round-to-nearest-even fp32 -> bf16 (finite inputs). */

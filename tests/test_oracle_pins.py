@@ -358,21 +358,32 @@ def _gelu_arg(z):
     return -2.0 * math.sqrt(2.0 / math.pi) * (z + 0.044715 * z ** 3)
 
 
-def test_exp_f32_against_math_exp(orc):
-    """Cody-Waite reduction + degree-7 Taylor: within 2^-22 relative over [-87, 88]."""
+def test_exp2_f32_against_math(orc):
+    """floor reduction + degree-6 Taylor in ln2 f (fma Horner): within 2^-21.5 relative of
+    2^t over [-126, 127], and exact at integers (f = 0 gives the polynomial's 1)."""
     rng = np.random.default_rng(11)
-    pts = np.concatenate([np.linspace(-87.0, 88.0, 20001), rng.uniform(-87.0, 88.0, 5000),
-                          [0.0, -0.0, 1e-8, -1e-8, 0.34657359, -0.34657359]]).astype(np.float32)
+    pts = np.concatenate([np.linspace(-126.0, 127.0, 20001), rng.uniform(-126.0, 127.0, 5000),
+                          [0.0, -0.0, 1e-8, -1e-8, 0.5, -0.5, 0.49999997, -0.49999997]]).astype(np.float32)
     worst = 0.0
-    for a in pts:
-        a = float(a)
-        ref = math.exp(a)
-        worst = max(worst, abs(orc.exp_f32(a) - ref) / ref)
-    assert worst <= 2.0 ** -22, worst
-    assert orc.exp_f32(0.0) == 1.0
-    for k in range(-120, 121, 7):  # exp(k ln2) = 2^k, exactly representable
-        a = _f32(k * math.log(2.0))
-        assert abs(orc.exp_f32(a) / math.exp(a) - 1.0) <= 2.0 ** -22
+    for t in pts:
+        t = float(t)
+        ref = 2.0 ** t
+        worst = max(worst, abs(orc.exp2_f32(t) - ref) / ref)
+    assert worst <= 2.0 ** -21.5, worst
+    for n in range(-126, 128):
+        assert orc.exp2_f32(float(n)) == 2.0 ** n
+
+
+def test_recip_f32_newton(orc):
+    """Newton-Raphson 1/d from the exponent-bit guess: within 2^-23 relative over
+    [1, 2^125], and exact where 1/d is a power of two reached by the iteration."""
+    rng = np.random.default_rng(14)
+    ds = np.concatenate([np.exp2(np.linspace(0.0, 125.0, 50001)), rng.uniform(1.0, 4.0, 5000),
+                         [1.0, 1.5, 2.0, 3.0, 1.0000001, 1.9999999]]).astype(np.float32)
+    worst = max(abs(orc.recip_f32(float(d)) * float(d) - 1.0) for d in ds)
+    assert worst <= 2.0 ** -23, worst
+    for k in range(0, 126, 5):
+        assert orc.recip_f32(2.0 ** k) == 2.0 ** -k
 
 
 def test_gelu_f32_against_tanh_definition(orc):
@@ -407,8 +418,8 @@ def test_gelu_f32_against_library_gelu(orc):
 def test_gelu_f32_tail_against_sigmoid_identity(orc):
     """On the negative tail the fp64 reference is the exact identity
     0.5 (1 + tanh(v)) = 1 / (1 + exp(-2v)), itself checked against tanh where both are
-    accurate; the fp32 result is a signed zero once exp(-2v) leaves fp32 (true value
-    below 2^-120)."""
+    accurate; the fp32 result is a signed zero once 2^t passes 2^125 (true value below
+    2^-118 |z|)."""
     for z in np.linspace(-5.0, 5.0, 1001):
         v = math.sqrt(2.0 / math.pi) * (z + 0.044715 * z ** 3)
         assert abs(0.5 * (1.0 + math.tanh(v)) - 1.0 / (1.0 + math.exp(-2.0 * v))) <= 1e-15
@@ -417,8 +428,8 @@ def test_gelu_f32_tail_against_sigmoid_identity(orc):
         a = _gelu_arg(z)
         got = orc.gelu_f32(z)
         if got == 0.0:
-            assert math.copysign(1.0, got) == -1.0 and a > 87.9
-            assert abs(z / (1.0 + math.exp(a))) < 2.0 ** -120
+            assert math.copysign(1.0, got) == -1.0 and a > 86.6  # t = a / ln2 > 125
+            assert abs(z / (1.0 + math.exp(a))) < 2.0 ** -118 * abs(z)
             continue
         ref = z / (1.0 + math.exp(a))
         assert abs(got - ref) <= (2.0 * abs(a) + 16.0) * 2.0 ** -23 * abs(ref), (z, got, ref)
