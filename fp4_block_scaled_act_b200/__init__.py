@@ -82,6 +82,8 @@ def lib():
             "fp4_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
             "fp4bsa_test_skip_iteration": (None, [I]),
             "fp4bsa_set_gemm_ctas": (None, [I]),
+            "fp4bsa_set_stream_k": (None, [I]),
+            "fp4bsa_set_pdl": (None, [I]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "fp4bsa.h"
@@ -157,9 +158,38 @@ fp4_status_t launch_quant(const DeviceState* ds, int kind, const void* x, int64_
     return launched();
 }
 
+// Encoded tensor maps are cached per host thread, keyed by every encode argument: a map
+// holds only an address, a shape and a box (no memory contents), so a cached map stays
+// valid for as long as the same arguments are passed, and encoding (a driver call of a
+// few microseconds) happens once per distinct buffer and shape.
+struct TmapKey {
+    const void* ptr;
+    uint64_t inner, rows, row_bytes;
+    uint32_t box_inner, box_rows;
+    int dt, swz;
+    bool operator==(const TmapKey& o) const {
+        return ptr == o.ptr && inner == o.inner && rows == o.rows && row_bytes == o.row_bytes &&
+               box_inner == o.box_inner && box_rows == o.box_rows && dt == o.dt && swz == o.swz;
+    }
+};
+constexpr int kTmapCache = 64;
+struct TmapCache {
+    TmapKey key[kTmapCache];
+    CUtensorMap map[kTmapCache];
+    int n = 0, next = 0;
+};
+thread_local TmapCache t_tmaps;
+
 fp4_status_t encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t rows,
                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
                        CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+    const TmapKey key{ptr, inner, rows, row_bytes, box_inner, box_rows, (int)dt, (int)swz};
+    TmapCache& c = t_tmaps;
+    for (int i = 0; i < c.n; ++i)
+        if (c.key[i] == key) {
+            *m = c.map[i];
+            return FP4_OK;
+        }
     const cuuint64_t dims[2] = {inner, rows};
     const cuuint64_t strides[1] = {row_bytes};
     const cuuint32_t box[2] = {box_inner, box_rows};
@@ -167,7 +197,11 @@ fp4_status_t encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, 
     CUresult r = g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
+    if (r != CUDA_SUCCESS) return FP4_ERR_CUDA;
+    const int slot = (c.n < kTmapCache) ? c.n++ : (c.next++ % kTmapCache);
+    c.key[slot] = key;
+    c.map[slot] = *m;
+    return FP4_OK;
 }
 
 template <int KIND>
@@ -189,13 +223,60 @@ fp4_status_t encode_sf(CUtensorMap* m, const uint8_t* sf, int64_t rows, int64_t 
                      CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// ---------------------------------------------------------------- stream-K plan (small M)
+// With fewer 256x256 tiles than two rounds of pairs, the 2-CTA kernel can spread the
+// flattened (tile, K block) space evenly over the pairs (stream-K); tiles split between
+// pairs are summed through fp32 slabs in the linear's workspace.  The workspace is sized
+// for kPlanPairs (a B200's 148 SMs); a device whose pair count needs more slabs per tile
+// runs whole tiles instead.
+constexpr int kPlanPairs = 74;
+int g_stream_k = 0;
+int g_pdl = 1;  // tuning hook: programmatic launch of fp4_linear's short GEMMs after the quantize (1 on, 0 off)  // tuning / test hook: 0 default (off), 1 never, 2 whenever the workspace allows
+
+int64_t sk_kstart(int64_t p, int64_t total, int P) { return p * total / P; }
+int64_t sk_pair_of(int64_t k, int64_t total, int P) {
+    int64_t q = k * P / total;
+    while (q + 1 < P && sk_kstart(q + 1, total, P) <= k) ++q;
+    while (q > 0 && sk_kstart(q, total, P) > k) --q;
+    return q;
+}
+// largest number of pairs sharing one tile
+int sk_seg_max(int64_t tiles, int64_t num_kb, int P) {
+    const int64_t total = tiles * num_kb;
+    int64_t m = 1;
+    for (int64_t t = 0; t < tiles; ++t)
+        m = std::max(m, sk_pair_of(t * num_kb + num_kb - 1, total, P) - sk_pair_of(t * num_kb, total, P) + 1);
+    return (int)m;
+}
+// K blocks of the 2-CTA MXFP4 / NVFP4 kernel (256 K per stage, the last may be half)
+int64_t sk_num_kb(int64_t K) { return (K + 255) / 256; }
+// Every pair's share must hold at least one K block (tiles * K blocks >= pairs): a pair
+// with an empty share would be counted among a tile's segments without ever arriving.
+// Only on request (hook): measured on B200, the small problems it targets are bound by
+// the kernel's fixed launch / prologue / pipeline-fill cost, and the slab round trip and
+// unit hand-offs made stream-K slower than whole tiles for every text-token shape tried.
+bool sk_wanted(int64_t M, int64_t K, int64_t N) {
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    if (g_stream_k == 1 || sk_num_kb(K) < 4 || tiles * sk_num_kb(K) < kPlanPairs) return false;
+    return g_stream_k == 2;
+}
+size_t sk_bytes(int64_t M, int64_t K, int64_t N) {
+    if (!sk_wanted(M, K, N)) return 0;
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    return align256((size_t)tiles * sk_seg_max(tiles, sk_num_kb(K), kPlanPairs) * 65536 * 4) +
+           align256((size_t)tiles * 64);
+}
+
 // 2-CTA GEMM: A box 128 rows, B box 128 rows (half of the 256-wide N tile) per CTA.
 // tu / tl: the W4A8 low-rank operands (u pair, packed L2); other kinds pass any map.
 // OUTQ != 0: the fused GELU + quantize output (p.h_codes / p.h_sf) instead of p.y.
+// pdl: launch with programmatic stream serialization, so the kernel's launch and prologue
+// overlap the previous kernel on the stream (its producer waits before reading A); used
+// right after our own quantize kernel, which does not touch the GEMM's output.
 template <int KIND, int OUTQ = 0>
 fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CUtensorMap& tb, const uint8_t* sfa,
                           const uint8_t* sfb, GemmParams& p, cudaStream_t st, const CUtensorMap* tu = nullptr,
-                          const CUtensorMap* tl = nullptr) {
+                          const CUtensorMap* tl = nullptr, bool pdl = false) {
     using C = Gemm2Cfg<KIND>;
     CUtensorMap tsa, tsb;
     fp4_status_t s;
@@ -207,12 +288,24 @@ fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CU
                                     (uint64_t)p.N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
         return s;
     const int tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
-    const int pairs = tiles < ds->pairs[KIND] ? tiles : ds->pairs[KIND];
+    // stream-K keeps every pair busy; whole tiles need no more pairs than tiles
+    const int pairs = (p.stream_k || tiles >= ds->pairs[KIND]) ? ds->pairs[KIND] : tiles;
     p.timeout_ns = g_timeout_ns;
     p.skip_iter = g_skip_iter;
     p.status = ds->status;
-    gemm2_kernel<KIND, OUTQ><<<2 * pairs, C::THREADS, C::SMEM_BYTES, st>>>(ta, tb, tsa, tsb, ty, tu ? *tu : ta,
-                                                                         tl ? *tl : tb, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, gemm2_kernel<KIND, OUTQ>, ta, tb, tsa, tsb, ty, tu ? *tu : ta, tl ? *tl : tb, p) !=
+        cudaSuccess)
+        return FP4_ERR_CUDA;
     return launched();
 }
 
@@ -233,7 +326,8 @@ size_t fp4_sf_bytes(fp4_fmt_t fmt, int64_t rows, int64_t K) {
 
 size_t fp4_linear_workspace_bytes(fp4_fmt_t fmt, int64_t M, int64_t K, int64_t N) {
     if (!fmt_ok(fmt) || check_shape(M, K, N) != FP4_OK) return 0;
-    return align256(fp4_codes_bytes(fmt, M, K)) + align256(fp4_sf_bytes(fmt, M, K));
+    // quantized activations, then (small M) the stream-K partial slabs and counters
+    return align256(fp4_codes_bytes(fmt, M, K)) + align256(fp4_sf_bytes(fmt, M, K)) + sk_bytes(M, K, N);
 }
 
 size_t w4a8_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank) {
@@ -312,9 +406,15 @@ fp4_status_t fp4_pack_weight(fp4_fmt_t fmt, const void* w_bf16, int64_t N, int64
     return launch_quant(ds, fmt == FP4_FMT_MXFP4 ? Q_MXFP4 : Q_NVFP4, w_bf16, N, K, w_global, w_codes, w_sf, st);
 }
 
-fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf, int64_t M, int64_t K, int64_t N,
-                      const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global, const float* a_global,
-                      const void* bias_f16, void* y_bf16, void* stream) {
+}  // extern "C"
+
+namespace {
+// fp4_gemm, optionally with a stream-K workspace (sk_ws: slabs then counters, sk_ws_bytes
+// as sized by sk_bytes) that fp4_linear passes for small M.
+fp4_status_t gemm_impl(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf, int64_t M, int64_t K, int64_t N,
+                       const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global, const float* a_global,
+                       const void* bias_f16, void* y_bf16, void* stream, uint8_t* sk_ws, size_t sk_ws_bytes,
+                       bool pdl = false) {
     if (!fmt_ok(fmt) || !a_codes || !a_sf || !w_codes || !w_sf || !y_bf16) return FP4_ERR_INVALID_ARG;
     const bool nv = (fmt == FP4_FMT_NVFP4);
     if (nv != (w_global != nullptr) || nv != (a_global != nullptr)) return FP4_ERR_INVALID_ARG;
@@ -326,9 +426,21 @@ fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf
         return FP4_ERR_MISALIGNED;
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;
+    // stream-K over the 2-CTA kernel when the linear provided its workspace and the pair
+    // count of this device fits the slabs it was sized for
+    bool sk = false;
+    int seg_max = 1;
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    if (sk_ws && sk_ws_bytes > 0 && g_gemm_ctas != 1) {
+        const int P = ds->pairs[nv ? G_NVFP4 : G_MXFP4];
+        if (tiles * sk_num_kb(K) >= P) {
+            seg_max = sk_seg_max(tiles, sk_num_kb(K), P);
+            sk = (size_t)tiles * seg_max * 65536 * 4 + (size_t)tiles * 64 <= sk_ws_bytes;
+        }
+    }
     // 2-CTA 256x256 tiles (faster at every M measured) unless M fits one 128-row tile or
     // the 1-CTA kernel is forced (tuning hook)
-    const bool pair = g_gemm_ctas != 1 && M > GEMM_BM;
+    const bool pair = sk || (g_gemm_ctas != 1 && M > GEMM_BM);
     CUtensorMap ta, tb;
     if ((s = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K / 2, M, K / 2, 128, GEMM_BM)) != FP4_OK)
         return s;
@@ -341,10 +453,28 @@ fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf
     p.bias = static_cast<const __half*>(bias_f16);
     p.y = static_cast<__nv_bfloat16*>(y_bf16);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (sk) {
+        const size_t slab_bytes = align256((size_t)tiles * seg_max * 65536 * 4);
+        p.stream_k = 1;
+        p.seg_max = seg_max;
+        p.partials = reinterpret_cast<float*>(sk_ws);
+        p.counters = reinterpret_cast<int*>(sk_ws + slab_bytes);
+        if (cudaMemsetAsync(p.counters, 0, (size_t)tiles * 64, st) != cudaSuccess) return FP4_ERR_CUDA;
+    }
     if (pair)
-        return nv ? launch_gemm2<G_NVFP4>(ds, ta, tb, a_sf, w_sf, p, st)
-                  : launch_gemm2<G_MXFP4>(ds, ta, tb, a_sf, w_sf, p, st);
+        return nv ? launch_gemm2<G_NVFP4>(ds, ta, tb, a_sf, w_sf, p, st, nullptr, nullptr, pdl)
+                  : launch_gemm2<G_MXFP4>(ds, ta, tb, a_sf, w_sf, p, st, nullptr, nullptr, pdl);
     return nv ? launch_gemm<G_NVFP4>(ds, ta, tb, p, st) : launch_gemm<G_MXFP4>(ds, ta, tb, p, st);
+}
+}  // namespace
+
+extern "C" {
+
+fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf, int64_t M, int64_t K, int64_t N,
+                      const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global, const float* a_global,
+                      const void* bias_f16, void* y_bf16, void* stream) {
+    return gemm_impl(fmt, a_codes, a_sf, M, K, N, w_codes, w_sf, w_global, a_global, bias_f16, y_bf16, stream,
+                     nullptr, 0);
 }
 
 fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K, int64_t N, const uint8_t* w_codes,
@@ -362,7 +492,14 @@ fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K,
     if (!w_codes || !w_sf || !y_bf16 || nv != (w_global != nullptr) || nv != (a_global != nullptr))
         return FP4_ERR_INVALID_ARG;
     if ((s = fp4_quantize_act(fmt, x_bf16, M, K, a_global, codes, sf, stream)) != FP4_OK) return s;
-    return fp4_gemm(fmt, codes, sf, M, K, N, w_codes, w_sf, w_global, a_global, bias_f16, y_bf16, stream);
+    // small M: the stream-K slabs follow the quantized activations
+    const size_t sk = sk_bytes(M, K, N);
+    uint8_t* sk_ws = sk ? sf + align256(fp4_sf_bytes(fmt, M, K)) : nullptr;
+    // short GEMMs (at most two rounds of 256x256 tiles on a B200) overlap their launch and
+    // prologue with the quantize kernel; measured 5-7 % faster there, and no gain on long ones
+    const bool pdl = g_pdl != 0 && ((M + 255) / 256) * ((N + 255) / 256) <= 2 * kPlanPairs;
+    return gemm_impl(fmt, codes, sf, M, K, N, w_codes, w_sf, w_global, a_global, bias_f16, y_bf16, stream, sk_ws, sk,
+                     pdl);
 }
 
 fp4_status_t fp4_gemm_gelu_quant(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf, int64_t M, int64_t K,
@@ -634,6 +771,15 @@ fp4_status_t fp4_linear_noalloc(fp4_fmt_t fmt, const void* x_bf16, int64_t M, in
 // Tuning hook (not in the public header): 1 forces the 1-CTA 128x256 kernel; 0 (default)
 // and 2 use the 2-CTA 256x256 kernel whenever M > 128.
 void fp4bsa_set_gemm_ctas(int ctas) { g_gemm_ctas = (ctas == 1 || ctas == 2) ? ctas : 0; }
+
+// Tuning / test hook (not in the public header): stream-K for fp4_linear: 0 default (off),
+// 1 never, 2 whenever the workspace allows (tiles x K blocks >= pairs).  The workspace
+// size query follows the same setting.
+void fp4bsa_set_stream_k(int mode) { g_stream_k = (mode == 1 || mode == 2) ? mode : 0; }
+
+// Tuning hook (not in the public header): 1 (default) launches fp4_linear's 2-CTA GEMM with
+// programmatic dependent launch after its quantize kernel, 0 with a plain launch.
+void fp4bsa_set_pdl(int on) { g_pdl = on ? 1 : 0; }
 
 // Test hook (not in the public header): the GEMM producer skips the given k-iteration of
 // its ring, so the MMA warp's bounded wait runs out.  -1 disables it.

@@ -72,6 +72,10 @@ struct GemmParams {
     uint8_t* h_codes;         // fused GELU + quantize output: FP4 codes [M, N/2]
     uint8_t* h_sf;            //   and scale bytes (128x4 atoms over [M, N])
     const float* g_h;         //   NVFP4 global of that output (device scalar) or null
+    int stream_k;             // 2-CTA kernel: stream-K schedule (small M) instead of whole tiles
+    int seg_max;              //   partial slabs per tile in `partials`
+    float* partials;          //   fp32 [tiles][seg_max][256][256] partial sums of split tiles
+    int* counters;            //   [tiles][16] arrivals per 32 x 128 region (zero before launch)
     uint64_t timeout_ns;
     int skip_iter;            // test hook: producer skips this k-iteration (-1: none)
     int* status;              // device status word
@@ -513,6 +517,50 @@ FP4_DEV void epilogue_gelu_quant(const GemmParams& p, uint32_t (&acc)[2][32], in
         *reinterpret_cast<uint32_t*>(word) = sfw;
 }
 
+// Work schedule of the 2-CTA kernel.  Whole tiles round-robin over the pairs, or (stream-K,
+// for problems with fewer tiles than two rounds of pairs) each pair takes an equal,
+// contiguous share of the flattened (tile, K block) space, cut at tile ends into units.
+// A tile split over several pairs is summed through fp32 partial slabs (epilogue).
+struct Sched {
+    int num_tiles, num_kb, num_pairs, pair;
+    bool sk;
+    int lo, hi, t;
+    FP4_DEV int kstart(int p) const { return (int)((int64_t)p * num_tiles * num_kb / num_pairs); }
+    // the pair whose share contains flattened K block k
+    FP4_DEV int pair_of(int k) const {
+        int q = (int)(((int64_t)k * num_pairs) / ((int64_t)num_tiles * num_kb));
+        while (q + 1 < num_pairs && kstart(q + 1) <= k) ++q;
+        while (q > 0 && kstart(q) > k) --q;
+        return q;
+    }
+    FP4_DEV void begin() {
+        if (sk) {
+            lo = kstart(pair);
+            hi = kstart(pair + 1);
+        } else {
+            t = pair;
+        }
+    }
+    FP4_DEV bool get(int& tile, int& kb0, int& kb1) const {
+        if (sk) {
+            if (lo >= hi) return false;
+            tile = lo / num_kb;
+            kb0 = lo - tile * num_kb;
+            kb1 = min(num_kb, kb0 + (hi - lo));
+            return true;
+        }
+        if (t >= num_tiles) return false;
+        tile = t;
+        kb0 = 0;
+        kb1 = num_kb;
+        return true;
+    }
+    FP4_DEV void step(int kb0, int kb1) {
+        if (sk) lo += kb1 - kb0;
+        else t += num_pairs;
+    }
+};
+
 FP4_DEV void gemm2_fail(const GemmParams& p, volatile int* abort, uint32_t peer_abort) {
     *abort = 1;
     st_cluster_u32(peer_abort, 1u);
@@ -607,22 +655,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
     const int num_n = (N + 255) / 256;
     const int num_tiles = num_m * num_n;
     const int num_kb = (K + C::BK - 1) / C::BK;
-    // stages per tile: the K blocks, then (W4A8, W4A4 SVDQuant) the low-rank stage kb == num_kb
+    // stages per unit: its K blocks, then (W4A8, W4A4 SVDQuant) the low-rank stage kb == num_kb
+    // (those kinds always run whole tiles)
     constexpr bool HAS_LR = (KIND == G_W4A8 || KIND == G_SVD4);
-    const int spt = num_kb + (HAS_LR ? 1 : 0);
     const int apr = K / (C::G * 4);  // scale atoms per 128-row block
     const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+    const Sched sched0{num_tiles, num_kb, num_pairs, pair, p.stream_k != 0, 0, 0, 0};
 
     if (warp == 0) {
         // ============================================================ producer (both CTAs)
         if (lane == 0) {
+            // the activations may come from the kernel just before us (programmatic launch)
+            griddep_wait();
             const uint64_t pol_a = policy_evict_normal();
             const uint64_t pol_b = policy_evict_last();
             int it = 0;
             bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+            Sched sc = sched0;
+            sc.begin();
+            int tile, kb0, kb1;
+            while (ok && sc.get(tile, kb0, kb1)) {
                 const int mb = tile / num_n, nb = tile % num_n;
-                for (int kb = 0; kb < spt; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (uint32_t)(it / S) & 1u;
                     if (!mbar_wait(&empty[s], ph ^ 1u, p.timeout_ns, abort)) {
@@ -656,6 +710,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                         tma_load_2d(sRSFB + s * C::RSFB_BYTES + j * C::ATOMS * 512, &tmSFB, &sf_full[s], 0,
                                     (nb * 2 + j) * apr + kb * C::ATOMS, pol_b);
                 }
+                sc.step(kb0, kb1);
             }
             // drain what this CTA issued: its scale loads, and (leader) both CTAs' A/B
             for (int j = max(0, it - S); j < it; ++j) {
@@ -672,8 +727,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         const uint32_t tlane = tmem_base + ((uint32_t)(quarter * 32) << 16);
         int it = 0;
         bool ok = true;
-        for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-            for (int kb = 0; kb < spt; ++kb, ++it) {
+        Sched sc = sched0;
+        sc.begin();
+        int tile, kb0, kb1;
+        while (ok && sc.get(tile, kb0, kb1)) {
+            for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
                 const int s = it % S;
                 const int t = it % TB;
                 bool got = mbar_wait(&sf_full[s], (uint32_t)(it / S) & 1u, p.timeout_ns, abort);
@@ -725,6 +783,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 __syncwarp();
                 if (lane == 0) arrive_leader_relaxed(&sf_ready[t], rank);
             }
+            sc.step(kb0, kb1);
         }
     } else if (warp == 1) {
         // ============================================================ MMA issuer (leader)
@@ -737,10 +796,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             uint32_t it = 0;
             int tcount = 0;
             bool issued = false, ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++tcount) {
+            Sched sc = sched0;
+            sc.begin();
+            int tile, kb0, kb1;
+            for (; ok && sc.get(tile, kb0, kb1); sc.step(kb0, kb1), ++tcount) {
                 const int b = tcount & 1;
                 const uint32_t dacc = tmem_base + (uint32_t)(b * C::ACC1_COL);
-                for (int kb = 0; kb < spt; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
                     named_bar_sync(1u + it % TB, 64u);
                     if (lane == 0 && HAS_LR && kb == num_kb) {
                         // low-rank stage: acc += u_hi L2 + u_lo L2 (bf16 x bf16 -> fp32)
@@ -770,7 +832,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                             const uint32_t idesc = C::IDESC | ((uint32_t)sf_id << 29) | ((uint32_t)sf_id << 4);
                             const uint64_t adesc = smem_desc(a_base + k * 32, 0, C::SBO, C::SWZ);
                             const uint64_t bdesc = smem_desc(b_base + k * 32, 0, C::SBO, C::SWZ);
-                            const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                            const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
                             if (KIND == G_MXFP4 || KIND == G_SVD4)
                                 mma2_mxf4nvf4_block32(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
                             else if (KIND == G_NVFP4)
@@ -809,12 +871,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             uint32_t it = 0;
             int tcount = 0;
             bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += num_pairs, ++tcount) {
+            Sched sc = sched0;
+            sc.begin();
+            int tile, kb0, kb1;
+            for (; ok && sc.get(tile, kb0, kb1); sc.step(kb0, kb1), ++tcount) {
                 const int b = tcount & 1;
-                // accumulator b drained (tile tcount-2) and the overlap of tile tcount-1 drained
+                // accumulator b drained (unit tcount-2) and the overlap of unit tcount-1 drained
                 bool got = mbar_wait(&acc_free[b], (((uint32_t)tcount >> 1) & 1u) ^ 1u, p.timeout_ns, abort);
                 if (got && tcount > 0) got = mbar_wait(ovl_free, (uint32_t)(tcount - 1) & 1u, p.timeout_ns, abort);
-                for (int kb = 0; kb < spt; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
                     if (got) got = mbar_wait(&full[it % S], (it / S) & 1u, p.timeout_ns, abort);
                     if (got) got = mbar_wait(&sf_ready[it % TB], (it / TB) & 1u, p.timeout_ns, abort);
                     got = __all_sync(0xffffffffu, got);
@@ -841,7 +906,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             six_g_h = __fmul_rn(6.0f, g_h);
         }
         int tcount = 0;
-        for (int tile = pair; tile < num_tiles; tile += num_pairs, ++tcount) {
+        Sched sc = sched0;
+        sc.begin();
+        int tile, kb0, kb1;
+        for (; sc.get(tile, kb0, kb1); sc.step(kb0, kb1), ++tcount) {
             const int mb = tile / num_n, nb = tile % num_n;
             const int b = tcount & 1;
             const bool got = mbar_wait(&tmem_full[b], ((uint32_t)tcount >> 1) & 1u, p.timeout_ns, abort);
@@ -855,9 +923,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             const int row0 = mb * 256 + (int)rank * 128 + q * 32;
             const int row = row0 + lane;
             const int col0 = nb * GEMM_BN + h * 128;
+            // stream-K: the tile's segments (pairs whose share meets it) and this unit's index
+            int nseg = 1, seg = 0;
+            if (p.stream_k) {
+                const int pf = sc.pair_of(tile * num_kb);
+                nseg = sc.pair_of(tile * num_kb + num_kb - 1) - pf + 1;
+                seg = pair - pf;
+            }
+            // this warp's 32 x 128 region of the tile's fp32 partial slabs, stored lane-major
+            // (float4 (chunk, j4, lane) at ((chunk * 8 + j4) * 32 + lane) * 4) so every warp
+            // instruction writes or reads 512 contiguous bytes; the summing warp has the same
+            // rows and lanes, so only it needs to know the layout
+            float* slab0 = p.partials + (size_t)tile * p.seg_max * 65536 + ((int)rank * 8 + (warp - 2)) * 4096 + lane * 4;
             // pack 64 columns into the staging tile and hand them to one TMA store (which
             // clips rows at or beyond M); the tile is reused once the previous store has read it
-            auto stage_store = [&](int chunk) {
+            auto emit = [&](int chunk) {
                 if (OUTQ != 0) {
                     epilogue_gelu_quant<KIND, OUTQ>(p, acc, row, col0 + chunk * 32, gs, g_h, six_g_h);
                     return;
@@ -872,6 +952,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                     tma_store_2d(&tmY, stile, col0 + chunk * 32, row0);
                     bulk_commit_group();
                 }
+            };
+            // a split tile: this segment's fp32 sums of the 64 columns go to its slab
+            auto stage_store = [&](int chunk) {
+                if (nseg == 1) {
+                    emit(chunk);
+                    return;
+                }
+                float* dst = slab0 + (size_t)seg * 65536;
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4*>(dst + (((chunk + c) * 8 + j / 4) * 32) * 4) =
+                            make_float4(__uint_as_float(acc[c][j]), __uint_as_float(acc[c][j + 1]),
+                                        __uint_as_float(acc[c][j + 2]), __uint_as_float(acc[c][j + 3]));
             };
             // the OVL columns shared by both accumulators are the last OVL tile columns of
             // accumulator 0 (half 1) or the first OVL of accumulator 1 (half 0): their holders
@@ -897,6 +992,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             if (holds_overlap && C::OVL > 64 && lane == 0) arrive_leader_relaxed(ovl_free, rank);
             if (lane == 0) arrive_leader_relaxed(&acc_free[b], rank);
             stage_store(second);
+            if (nseg > 1) {
+                // the last of the tile's segments to arrive sums the slabs in segment order
+                // (a fixed order, so the result does not depend on which one is last) and
+                // runs the epilogue; nobody waits for anybody
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) last = atomicAdd(p.counters + tile * 16 + (int)rank * 8 + (warp - 2), 1) == nseg - 1;
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last) {
+                    __threadfence();
+#pragma unroll 1
+                    for (int pr = 0; pr < 4; pr += 2) {
+                        // segment-outer: 16 independent float4 loads per segment in flight
+#pragma unroll 1
+                        for (int sg = 0; sg < nseg; ++sg) {
+                            const float* src = slab0 + (size_t)sg * 65536;
+#pragma unroll
+                            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                                for (int j = 0; j < 32; j += 4) {
+                                    const float4 v =
+                                        __ldcg(reinterpret_cast<const float4*>(src + (((pr + c) * 8 + j / 4) * 32) * 4));
+                                    if (sg == 0) {
+                                        acc[c][j] = __float_as_uint(v.x), acc[c][j + 1] = __float_as_uint(v.y);
+                                        acc[c][j + 2] = __float_as_uint(v.z), acc[c][j + 3] = __float_as_uint(v.w);
+                                    } else {
+                                        acc[c][j] = __float_as_uint(__fadd_rn(__uint_as_float(acc[c][j]), v.x));
+                                        acc[c][j + 1] = __float_as_uint(__fadd_rn(__uint_as_float(acc[c][j + 1]), v.y));
+                                        acc[c][j + 2] = __float_as_uint(__fadd_rn(__uint_as_float(acc[c][j + 2]), v.z));
+                                        acc[c][j + 3] = __float_as_uint(__fadd_rn(__uint_as_float(acc[c][j + 3]), v.w));
+                                    }
+                                }
+                        }
+                        emit(pr);
+                    }
+                }
+            }
         }
         // the staging tile must outlive the stores that read it
         if (lane == 0) bulk_wait_group0();

@@ -65,6 +65,13 @@ FP4_DEV bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) 
     }
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start while the previous kernel on the stream runs; griddep_wait blocks the calling
+// thread until that kernel has completed and its memory is visible (a no-op otherwise).
+// griddep_launch_dependents lets such a dependent kernel be scheduled early.
+FP4_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+FP4_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Named (hardware) CTA barriers: `count` threads, whole warps, converged.
 FP4_DEV void named_bar_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

@@ -55,6 +55,9 @@ __global__ void __launch_bounds__(QUANT_THREADS) quant_kernel(const uint4* __res
     // Each CTA owns a contiguous range of units; per pass its 16 half-warps take 16
     // consecutive units, QUANT_UNROLL passes are loaded before any is processed.  Row and
     // chunk of a unit are advanced incrementally (no per-unit division).
+    // a GEMM launched after us with programmatic serialization may be scheduled now (its
+    // prologue overlaps our work; it still waits for our completion before reading)
+    griddep_launch_dependents();
     constexpr uint32_t UPB = QUANT_THREADS / 16;  // units per pass
     const uint32_t upr = (uint32_t)(K >> 7);
     const uint32_t Mpad = (uint32_t)((M + 127) & ~int64_t(127));

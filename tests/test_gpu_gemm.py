@@ -313,6 +313,56 @@ def test_w4a4_full_size_sampled(fb, orc):
     _w4a4_check(fb, orc, M, K, N, seed=4001, rows=rows, calib=2048)
 
 
+# ------------------------------------------------------------------ small-M stream-K schedule
+# fp4_linear can run small problems as stream-K (a tuning hook turns it on; measured slower
+# than whole tiles on B200): tiles shared by pairs are summed through fp32 slabs in a fixed
+# segment order.
+@contextlib.contextmanager
+def _stream_k(fb, mode):
+    L = fb.lib()
+    L.fp4bsa_set_stream_k(mode)
+    try:
+        yield L
+    finally:
+        L.fp4bsa_set_stream_k(0)
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("M,K,N", [(1, 5120, 1024), (77, 2560, 2048), (129, 5120, 1024), (300, 2432, 1024),
+                                   (512, 5120, 1280)])
+def test_stream_k_all_elements(fb, orc, fmt, M, K, N):
+    """Stream-K (forced on) against the oracle on every element, ragged M and K % 256 = 128."""
+    x = synth.activation(80 * M + K, M, K, "lognormal")
+    w = synth.weight(90 * N + K, N, K)
+    b = synth.bias(N + 13, N)
+    g_a = orc.nv_global(orc.tensor_amax(x)) if fmt == NV else None
+    with _stream_k(fb, 2):
+        y = _run_linear(fb, fmt, x, w, b, g_a)
+    rows = np.arange(M)
+    Y, S = _oracle(orc, fmt, x, w, b, rows, g_a)
+    H.check_linear(y, Y, S, rows, f"stream-K fmt={fmt} M={M} K={K} N={N}")
+
+
+def test_stream_k_deterministic_and_close_to_whole_tiles(fb, orc):
+    """Two stream-K runs are bit-identical; whole tiles give the same result within tolerance."""
+    import torch
+
+    M, K, N = 512, 5120, 5120  # the attn2 k/v shape (text tokens)
+    x = synth.activation(4242, M, K, "lognormal")
+    w = synth.weight(4243, N, K)
+    b = synth.bias(4244, N)
+    with _stream_k(fb, 2):
+        y1 = _run_linear(fb, MX, x, w, b)
+        y2 = _run_linear(fb, MX, x, w, b)
+    assert torch.equal(y1, y2)
+    with _stream_k(fb, 1):
+        y3 = _run_linear(fb, MX, x, w, b)
+    rows = np.arange(M)
+    Y, S = _oracle(orc, MX, x, w, b, rows)
+    H.check_linear(y1, Y, S, rows, "stream-K attn2 k/v")
+    H.check_linear(y3, Y, S, rows, "whole tiles attn2 k/v")
+
+
 # ------------------------------------------------------------------ each GEMM kernel, forced
 # The library picks the cta_group::2 256x256 kernel for M > 128 and the 1-CTA 128x256
 # kernel otherwise; a tuning hook forces either, so both stay covered on ragged shapes.
