@@ -10,7 +10,7 @@ fused bias epilogue (the weight pre-pack is offline and untimed).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
 Prints one JSON line.  `value` is TFLOPS (2*M*K*N per step, all ranks together)
-with inputs resident in HBM; `e2e` is the same metric through fp4_linear with the
+with inputs resident in HBM; `e2e` is the same metric through fp4_linear (linear_host) with the
 input copied from pinned host memory and the output copied back every step.  With
 N > 1 (torchrun) every rank runs its own batch (weak scaling, no collective on the
 data path); time is the max over ranks.  `--impl reference` times the CPU oracle on
@@ -321,14 +321,13 @@ def native_arm(args):
     value = FLOP_PER_STEP * world * args.steps / (total_ms / 1e3) / 1e12
 
     # ---- end to end through the public API, host buffers (pinned), copies inside the timing
+    # (fb.linear_host: row chunks through fp4_linear with both copy directions overlapped)
     x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    x_e2e = torch.empty_like(x)
+    pipe = fb.HostPipeline(FMT, min(M, 8192), K, N)
 
     def e2e_step():
-        x_e2e.copy_(x_host, non_blocking=True)
-        fb.fp4_linear(FMT, x_e2e, M, K, N, pw.codes, pw.sf, None, None, bias, y, ws, ws_bytes)
-        y_host.copy_(y, non_blocking=True)
+        fb.linear_host(x_host, pw, pipe, bias, None, y_host)
 
     for _ in range(2):
         e2e_step()

@@ -7,7 +7,7 @@ arithmetic runs in the library's CUDA kernels.  There is no fallback: if the
 library is missing or the device is not sm_100, the calls raise.
 
 The helpers at the end (pack_weight, quantize_act, linear, pack_lowrank_up, w4a8_linear,
-w4a4_linear, gelu_quantize_act, linear_gelu_quant)
+w4a4_linear, gelu_quantize_act, linear_gelu_quant, linear_host)
 allocate outputs and workspaces with torch and call the same entry points.
 """
 from __future__ import annotations
@@ -369,3 +369,65 @@ def linear_gelu_quant(x, pw: PackedWeight, bias=None, a_global=None, h_global=No
     fp4_linear_gelu_quant(pw.fmt, x, M, K, N, pw.codes, pw.sf, pw.w_global, a_global, bias, h_global, codes, sf,
                           workspace, workspace.numel(), stream)
     return codes, sf
+
+
+class HostPipeline:
+    """Reusable device buffers, streams and events for linear_host: two sets of per-chunk
+    device buffers (x rows, y rows, quantize workspace) so that the host->device copy of
+    chunk i + 1, the linear of chunk i and the device->host copy of chunk i - 1 run
+    concurrently on three streams."""
+
+    def __init__(self, fmt, chunk_rows: int, K: int, N: int, device="cuda"):
+        import torch
+
+        self.fmt = _fmt(fmt)
+        self.chunk_rows, self.K, self.N = chunk_rows, K, N
+        ws = fp4_linear_workspace_bytes(self.fmt, chunk_rows, K, N)
+        self.x = [torch.empty((chunk_rows, K), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        self.y = [torch.empty((chunk_rows, N), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        self.ws = [torch.empty(ws, dtype=torch.uint8, device=device) for _ in range(2)]
+        self.streams = [torch.cuda.Stream(device=device) for _ in range(3)]
+        self.ev_x = [torch.cuda.Event() for _ in range(2)]   # chunk copied in
+        self.ev_c = [torch.cuda.Event() for _ in range(2)]   # chunk computed (x read, y written)
+        self.ev_y = [torch.cuda.Event() for _ in range(2)]   # chunk copied out
+
+
+def linear_host(x_host, pw: PackedWeight, pipe: HostPipeline, bias=None, a_global=None, y_host=None):
+    """Host-to-host W4A4 linear: pinned bf16 x [M, K] in host memory -> pinned bf16 y
+    [M, N] in host memory, in row chunks of pipe.chunk_rows through fp4_linear, with the
+    copies in both directions overlapped with the GEMMs (see HostPipeline).  The work is
+    ordered after everything already on the current stream, and the current stream waits
+    for the last copy, so an event recorded on it afterwards marks completion."""
+    import torch
+
+    M, K = x_host.shape
+    assert K == pipe.K and pw.N == pipe.N and pw.fmt == pipe.fmt
+    if y_host is None:
+        y_host = torch.empty((M, pw.N), dtype=torch.bfloat16, pin_memory=True)
+    cur = torch.cuda.current_stream()
+    s_in, s_mm, s_out = pipe.streams
+    for s in pipe.streams:
+        s.wait_stream(cur)
+    C = pipe.chunk_rows
+    for i, r0 in enumerate(range(0, M, C)):
+        r1 = min(M, r0 + C)
+        rows, b = r1 - r0, i % 2
+        xd, yd = pipe.x[b][:rows], pipe.y[b][:rows]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(pipe.ev_c[b])        # chunk i - 2 no longer reads x[b]
+            xd.copy_(x_host[r0:r1], non_blocking=True)
+            pipe.ev_x[b].record(s_in)
+        with torch.cuda.stream(s_mm):
+            s_mm.wait_event(pipe.ev_x[b])
+            if i >= 2:
+                s_mm.wait_event(pipe.ev_y[b])        # chunk i - 2 copied y[b] out
+            fp4_linear(pipe.fmt, xd, rows, K, pipe.N, pw.codes, pw.sf, pw.w_global, a_global, bias, yd,
+                       pipe.ws[b], pipe.ws[b].numel(), s_mm)
+            pipe.ev_c[b].record(s_mm)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(pipe.ev_c[b])
+            y_host[r0:r1].copy_(yd, non_blocking=True)
+            pipe.ev_y[b].record(s_out)
+    cur.wait_stream(s_out)
+    return y_host

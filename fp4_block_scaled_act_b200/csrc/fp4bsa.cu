@@ -83,6 +83,10 @@ fp4_status_t device_state(DeviceState** out) {
                 cudaFuncSetAttribute(gemm2_kernel<G_MXFP4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Gemm2Cfg<G_MXFP4>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm2_kernel<G_NVFP4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Gemm2Cfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm2_kernel<G_MXFP4, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Gemm2Cfg<G_MXFP4>::SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm2_kernel<G_NVFP4, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Gemm2Cfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess)
                 return FP4_ERR_CUDA;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.quant_occ[Q_MXFP4], quant_kernel<Q_MXFP4>,
@@ -273,7 +277,7 @@ size_t sk_bytes(int64_t M, int64_t K, int64_t N) {
 // pdl: launch with programmatic stream serialization, so the kernel's launch and prologue
 // overlap the previous kernel on the stream (its producer waits before reading A); used
 // right after our own quantize kernel, which does not touch the GEMM's output.
-template <int KIND, int OUTQ = 0>
+template <int KIND, int OUTQ = 0, bool SK = false>
 fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CUtensorMap& tb, const uint8_t* sfa,
                           const uint8_t* sfb, GemmParams& p, cudaStream_t st, const CUtensorMap* tu = nullptr,
                           const CUtensorMap* tl = nullptr, bool pdl = false) {
@@ -289,7 +293,7 @@ fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CU
         return s;
     const int tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
     // stream-K keeps every pair busy; whole tiles need no more pairs than tiles
-    const int pairs = (p.stream_k || tiles >= ds->pairs[KIND]) ? ds->pairs[KIND] : tiles;
+    const int pairs = (SK || tiles >= ds->pairs[KIND]) ? ds->pairs[KIND] : tiles;
     p.timeout_ns = g_timeout_ns;
     p.skip_iter = g_skip_iter;
     p.status = ds->status;
@@ -303,7 +307,7 @@ fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CU
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, gemm2_kernel<KIND, OUTQ>, ta, tb, tsa, tsb, ty, tu ? *tu : ta, tl ? *tl : tb, p) !=
+    if (cudaLaunchKernelEx(&cfg, gemm2_kernel<KIND, OUTQ, SK>, ta, tb, tsa, tsb, ty, tu ? *tu : ta, tl ? *tl : tb, p) !=
         cudaSuccess)
         return FP4_ERR_CUDA;
     return launched();
@@ -455,12 +459,14 @@ fp4_status_t gemm_impl(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_s
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (sk) {
         const size_t slab_bytes = align256((size_t)tiles * seg_max * 65536 * 4);
-        p.stream_k = 1;
         p.seg_max = seg_max;
         p.partials = reinterpret_cast<float*>(sk_ws);
         p.counters = reinterpret_cast<int*>(sk_ws + slab_bytes);
         if (cudaMemsetAsync(p.counters, 0, (size_t)tiles * 64, st) != cudaSuccess) return FP4_ERR_CUDA;
     }
+    if (sk)
+        return nv ? launch_gemm2<G_NVFP4, 0, true>(ds, ta, tb, a_sf, w_sf, p, st, nullptr, nullptr, pdl)
+                  : launch_gemm2<G_MXFP4, 0, true>(ds, ta, tb, a_sf, w_sf, p, st, nullptr, nullptr, pdl);
     if (pair)
         return nv ? launch_gemm2<G_NVFP4>(ds, ta, tb, a_sf, w_sf, p, st, nullptr, nullptr, pdl)
                   : launch_gemm2<G_MXFP4>(ds, ta, tb, a_sf, w_sf, p, st, nullptr, nullptr, pdl);

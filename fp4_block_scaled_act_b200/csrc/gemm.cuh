@@ -72,8 +72,7 @@ struct GemmParams {
     uint8_t* h_codes;         // fused GELU + quantize output: FP4 codes [M, N/2]
     uint8_t* h_sf;            //   and scale bytes (128x4 atoms over [M, N])
     const float* g_h;         //   NVFP4 global of that output (device scalar) or null
-    int stream_k;             // 2-CTA kernel: stream-K schedule (small M) instead of whole tiles
-    int seg_max;              //   partial slabs per tile in `partials`
+    int seg_max;              // stream-K (2-CTA kernel): partial slabs per tile in `partials`
     float* partials;          //   fp32 [tiles][seg_max][256][256] partial sums of split tiles
     int* counters;            //   [tiles][16] arrivals per 32 x 128 region (zero before launch)
     uint64_t timeout_ns;
@@ -579,7 +578,9 @@ FP4_DEV void arrive_leader_relaxed(uint64_t* bar, uint32_t rank) {
 
 // OUTQ 0: bf16 output through the TMA-store epilogue; 1 / 2: the fused GELU + MXFP4 /
 // NVFP4 quantize epilogue (epilogue_gelu_quant) in place of the bf16 output.
-template <int KIND, int OUTQ = 0>
+// SK: the stream-K schedule (small problems, opt-in); a separate instantiation so the
+// default kernel carries none of its registers.
+template <int KIND, int OUTQ = 0, bool SK = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THREADS, 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
@@ -660,7 +661,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
     constexpr bool HAS_LR = (KIND == G_W4A8 || KIND == G_SVD4);
     const int apr = K / (C::G * 4);  // scale atoms per 128-row block
     const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
-    const Sched sched0{num_tiles, num_kb, num_pairs, pair, p.stream_k != 0, 0, 0, 0};
+    const Sched sched0{num_tiles, num_kb, num_pairs, pair, SK, 0, 0, 0};
 
     if (warp == 0) {
         // ============================================================ producer (both CTAs)
@@ -925,7 +926,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             const int col0 = nb * GEMM_BN + h * 128;
             // stream-K: the tile's segments (pairs whose share meets it) and this unit's index
             int nseg = 1, seg = 0;
-            if (p.stream_k) {
+            if constexpr (SK) {
                 const int pf = sc.pair_of(tile * num_kb);
                 nseg = sc.pair_of(tile * num_kb + num_kb - 1) - pf + 1;
                 seg = pair - pf;
@@ -955,7 +956,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             };
             // a split tile: this segment's fp32 sums of the 64 columns go to its slab
             auto stage_store = [&](int chunk) {
-                if (nseg == 1) {
+                if (!SK || nseg == 1) {
                     emit(chunk);
                     return;
                 }
@@ -992,7 +993,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             if (holds_overlap && C::OVL > 64 && lane == 0) arrive_leader_relaxed(ovl_free, rank);
             if (lane == 0) arrive_leader_relaxed(&acc_free[b], rank);
             stage_store(second);
-            if (nseg > 1) {
+            if (SK && nseg > 1) {
                 // the last of the tile's segments to arrive sums the slabs in segment order
                 // (a fixed order, so the result does not depend on which one is last) and
                 // runs the epilogue; nobody waits for anybody

@@ -426,3 +426,26 @@ def test_each_kernel_timeout(fb, orc, ctas):
     torch.cuda.synchronize()
     Y, S = orc.fp4_linear_rows(MX, x, w, None, np.arange(M))
     H.check_linear(y, Y, S, np.arange(M), f"ctas={ctas} after timeout")
+
+
+# ------------------------------------------------------------------ host-to-host pipeline
+@pytest.mark.parametrize("fmt", [MX, NV])
+def test_linear_host_chunks(fb, orc, fmt):
+    """linear_host: pinned host x -> pinned host y in row chunks (ragged last chunk) with
+    overlapped copies, against the oracle on every row."""
+    import torch
+
+    M, K, N = 700, 1024, 512
+    x = synth.activation(5151 + fmt, M, K, "lognormal")
+    w = synth.weight(5152, N, K)
+    b = synth.bias(5153, N)
+    g_a = orc.nv_global(orc.tensor_amax(x)) if fmt == NV else None
+    pw = fb.pack_weight(H.dev_bf16(w), fmt)
+    x_host = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
+    pipe = fb.HostPipeline(fmt, 256, K, N)
+    y_host = fb.linear_host(x_host, pw, pipe, H.dev_f16(b), H.dev_f32([g_a]) if fmt == NV else None)
+    torch.cuda.synchronize()
+    assert fb.fp4_sync_status() == 0
+    rows = np.arange(M)
+    Y, S = _oracle(orc, fmt, x, w, b, rows, g_a)
+    H.check_linear(y_host, Y, S, rows, f"linear_host fmt={fmt}")
