@@ -1,19 +1,21 @@
-// gemm.cuh -- persistent block-scaled GEMM for sm_100a (tcgen05 + TMA), fused epilogue.
+// gemm.cuh -- persistent block-scaled GEMMs for sm_100a (tcgen05 + TMA), fused epilogues.
 //
 //   y[m, n] = bf16_rn( gs * sum_k deq(a[m, k]) * deq(w[n, k]) (+ u[m,:] L2[:, n]) + bias[n] )
 //
-// Tile 128 x 256 (M x N), one CTA per SM, tiles assigned round-robin (tile t -> CTA
-// t mod grid), N fastest so concurrently running CTAs share the activation rows in L2.
+// Two kernels:
+//   gemm2_kernel  (default for M > 128, and every W4A8 / W4A4-SVDQuant / fused-activation
+//                 call) -- a cta_group::2 pair of CTAs computes a 256 x 256 tile; see the
+//                 block comment above Gemm2Cfg for its warp roles, TMEM layout and schedule.
+//   gemm_kernel   (M <= 128, or forced) -- one CTA per SM, 128 x 256 tiles, described below.
 // Per K-stage the operands take one 128-byte swizzle atom per row:
-//   W4A4 (kind::mxf4nvf4): 256 packed E2M1 values, 4 MMAs of K = 64
+//   FP4 x FP4 (kind::mxf4nvf4): 256 packed E2M1 values, 4 MMAs of K = 64
 //   W4A8 (kind::mxf8f6f4): 128 E4M3 / unpacked E2M1 values, 4 MMAs of K = 32
-// Warp roles (320 threads):
+// gemm_kernel warp roles (320 threads):
 //   warp 0      TMA producer: A/B tiles (tensor maps) + scale-factor atoms (bulk copies)
 //   warp 1      TMEM owner and MMA issuer: tcgen05.cp scale atoms into TMEM, then
 //               tcgen05.mma block_scale into a 128 x 256 fp32 accumulator in TMEM
 //   warps 2..9  epilogue: drain the accumulator to registers (freeing TMEM for the next
-//               tile's MMAs at once), then scale, add bias (and the low-rank term), round
-//               to bf16 and store
+//               tile's MMAs at once), then scale, add bias, round to bf16 and store
 // Every mbarrier wait is bounded; a wait that runs out sets the device status word and
 // the shared abort flag, and all roles leave their loops, drain in-flight copies/MMAs and
 // free TMEM before the CTA exits.
