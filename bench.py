@@ -141,19 +141,29 @@ def to_dev(bits, torch, dt):
 
 def gemm_traffic(pair: bool):
     """DRAM bytes per launch of the timed GEMM kernel from the committed ncu summary, or
-    None when the kernel source changed since those counters were taken."""
-    import hashlib
-
+    None when the kernel code changed since those counters were taken."""
     name = "gemm2_mxfp4_ffn_up_traffic.txt" if pair else "gemm_mxfp4_ffn_up_traffic.txt"
     path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
         return None
     fields = dict(l.split(":", 1) for l in open(path) if ":" in l)
-    src = b"".join(open(os.path.join(ROOT, "fp4_block_scaled_act_b200", "csrc", f), "rb").read()
-                   for f in ("gemm.cuh", "ptx.cuh"))
-    if hashlib.sha1(src).hexdigest()[:12] != fields.get("source_sha1", "").strip():
+    if kernel_code_digest() != fields.get("code_sha1", "").strip():
         return None
     return float(fields["bytes_per_launch"])
+
+
+def kernel_code_digest() -> str:
+    """sha1 (12 hex digits) of the GEMM kernel sources with // comments and blank lines
+    removed: an edit to the code invalidates recorded counters, an edit to a comment does not."""
+    import hashlib
+
+    h = hashlib.sha1()
+    for f in ("gemm.cuh", "ptx.cuh"):
+        for line in open(os.path.join(ROOT, "fp4_block_scaled_act_b200", "csrc", f), encoding="utf-8"):
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                h.update(code.encode() + b"\n")
+    return h.hexdigest()[:12]
 
 
 # ----------------------------------------------------------------------------- cpu baseline

@@ -35,6 +35,18 @@ struct DeviceState {
     int* status = nullptr;
 };
 
+// The pair kernels move registers between warpgroups with setmaxnreg; the split is sized
+// for exactly Gemm2Cfg::REG_LAUNCH registers per thread at launch, and with fewer the
+// epilogue warps' increase could never be satisfied.  Checked before any pair launch.
+bool launch_regs_are(const void* kernel, int want) {
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, kernel) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.numRegs == want;
+}
+
 template <int KIND>
 int max_pairs(int sm_count) {
     cudaLaunchConfig_t cfg = {};
@@ -89,6 +101,16 @@ fp4_status_t device_state(DeviceState** out) {
                 cudaFuncSetAttribute(gemm2_kernel<G_NVFP4, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Gemm2Cfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess)
                 return FP4_ERR_CUDA;
+            {
+                constexpr int R = (int)Gemm2Cfg<G_MXFP4>::REG_LAUNCH;
+                const void* pair_kernels[] = {
+                    (const void*)gemm2_kernel<G_MXFP4>,          (const void*)gemm2_kernel<G_NVFP4>,
+                    (const void*)gemm2_kernel<G_W4A8>,           (const void*)gemm2_kernel<G_SVD4>,
+                    (const void*)gemm2_kernel<G_MXFP4, 1>,       (const void*)gemm2_kernel<G_NVFP4, 2>,
+                    (const void*)gemm2_kernel<G_MXFP4, 0, true>, (const void*)gemm2_kernel<G_NVFP4, 0, true>};
+                for (const void* k : pair_kernels)
+                    if (!launch_regs_are(k, R)) return FP4_ERR_ARCH;
+            }
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.quant_occ[Q_MXFP4], quant_kernel<Q_MXFP4>,
                                                               QUANT_THREADS, 0) != cudaSuccess ||
                 cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.quant_occ[Q_NVFP4], quant_kernel<Q_NVFP4>,

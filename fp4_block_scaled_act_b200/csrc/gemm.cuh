@@ -374,18 +374,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // The writers load a stage's words before waiting for its TMEM buffer to be free, so only
 // the TMEM store and the arrive follow that wait.
 //
-// Accumulators: two 256-column accumulators overlap by 64 columns ([0,256), [192,448));
-// the epilogue drains the shared 64 columns first, so the next tile's MMAs wait for a
-// 64-column drain only.  Columns [448,512) hold the scale buffers.
+// Accumulators: two 256-column accumulators overlapping by 64 columns ([0,256),
+// [192,448)) -- 96 for NVFP4 with a fused epilogue -- drained 64 columns at a time with
+// the shared columns first, so the next tile's MMAs wait for that part only; the scale
+// buffers follow the second accumulator.  NVFP4 with plain bf16 output uses one
+// accumulator [0,256) instead: each epilogue warp copies its 32 x 128 share to registers
+// with four tcgen05.ld and hands the accumulator back at once, and columns [256,512) hold
+// four scale buffers.
 //
-// Warps (480 threads): 0 TMA producer, 1 TMEM owner + MMA issuer (leader), 2-9 epilogue
-// (64 columns at a time), 10-13 scale writers, 14 stage coordinator (leader).
+// Warps (512 threads, four warpgroups): 0 TMA producer, 1 TMEM owner + MMA issuer
+// (leader), 2 stage coordinator (leader), 3 idle, 4-7 scale writers, 8-15 epilogue.  The
+// control warpgroups (0-7) drop to REG_LO registers per thread with setmaxnreg and the
+// epilogue warpgroups rise to REG_HI, so a 128-column drain fits in registers.
 // The tensor pipe queues very little ahead of the issuing thread, so every cycle that
-// thread spends between two MMAs is a bubble, and an mbarrier test from it costs on the
-// order of a hundred cycles while the tensor core streams shared memory.  The MMA warp
-// therefore tests no mbarrier: the coordinator does the waits and hands each stage over
-// with a hardware named barrier (bar.arrive / bar.sync), which does not touch shared
-// memory.
+// thread spends between two MMAs is a bubble.  The MMA warp therefore tests no mbarrier:
+// the coordinator does the waits and hands each stage over with a hardware named barrier
+// (bar.arrive / bar.sync), which does not touch shared memory.
 // Synchronization:
 //   full[s]      (leader)  A/B bytes of both CTAs; the leader alone expects them
 //   sf_full[s]   (local)   this CTA's raw scale atoms
@@ -393,9 +397,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 //   sf_ready[t]  (leader)  scale buffer t written in both CTAs (8 writer warps)
 //   tmem_full[b] (both)    accumulator b complete
 //   acc_free[b]  (leader)  accumulator b fully drained by both CTAs (16 warps)
-//   ovl_free     (leader)  overlap columns of the last tile drained (8 warps)
+//   ovl_free     (leader)  overlap columns of the last tile drained (8 warps; with one
+//                          accumulator, all of it copied out by all 16 epilogue warps)
 // =======================================================================================
-template <int KIND>
+template <int KIND, int OUTQ = 0>
 struct Gemm2Cfg {
     using C1 = GemmCfg<KIND>;
     // 128-byte operand rows (128-byte swizzle) for every kind: with 64-byte rows (64-byte
@@ -407,6 +412,7 @@ struct Gemm2Cfg {
     static constexpr uint32_t SWZ = 2u;         // descriptor layout: 128-byte swizzle
     static constexpr int SBO = 8 * ROW_BYTES;
     static constexpr int N_MMA = BK / MMA_K;
+    static_assert(N_MMA == 4, "the MMA warp issues a stage as four unrolled MMAs");
     static constexpr int A_BYTES = 128 * ROW_BYTES;
     static constexpr int B_BYTES = 128 * ROW_BYTES;  // this CTA's half of the 256 B rows
     static constexpr int RSFA_BYTES = ATOMS * 512;    // raw atoms, this CTA's 128 A rows
@@ -417,15 +423,25 @@ struct Gemm2Cfg {
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + 512;
     static constexpr uint32_t AB_TX = A_BYTES + ((KIND == G_W4A8) ? B_BYTES / 2 : B_BYTES);
     static constexpr uint32_t SF_TX = RSFA_BYTES + RSFB_BYTES;
-    // NVFP4 stages carry 4 scale atoms (48 TMEM columns): its accumulators overlap by 96
-    // columns to leave room for two scale buffers; the others overlap by 64
-    static constexpr int ACC1_COL = (KIND == G_NVFP4) ? 160 : 192;
-    static constexpr int SF_COL0 = ACC1_COL + 256;
+    // TMEM columns.  Two accumulators overlapping by OVL columns, drained 64 columns at a
+    // time with the shared columns first: NVFP4 stages carry 4 scale atoms (48 columns),
+    // so its accumulators overlap by 96 to leave room for two scale buffers; the others
+    // overlap by 64.  NVFP4 with plain bf16 output (OUTQ 0) instead keeps one accumulator
+    // [0,256), which the epilogue copies to registers in one go, and four scale buffers
+    // from column 256: measured faster there than waiting for a 96-column drain, while for
+    // MXFP4 the 128 KB burst of TMEM reads costs more MMA time than the 64-column overlap.
+    static constexpr bool SINGLE = (OUTQ == 0) && (KIND == G_NVFP4);
+    static constexpr int ACC1_COL = SINGLE ? 0 : (KIND == G_NVFP4) ? 160 : 192;
+    static constexpr int SF_COL0 = SINGLE ? 256 : ACC1_COL + 256;
     static constexpr int OVL = 256 - ACC1_COL;
     static constexpr int SFA_COLS = 4 * ATOMS;        // A: 4 columns per atom
     static constexpr int SF_COLS = SFA_COLS + 8 * ATOMS;  // B: 8 columns per atom
     static constexpr int TB = ((GEMM_TMEM_COLS - SF_COL0) / SF_COLS) >= 4 ? 4 : ((GEMM_TMEM_COLS - SF_COL0) / SF_COLS);
-    static constexpr int THREADS = 480;
+    // 16 warps in four warpgroups; the two control warpgroups (warps 0-7) hand registers to
+    // the two epilogue warpgroups (8-15).  Launched with 128 registers per thread.
+    static constexpr int THREADS = 512;
+    static constexpr uint32_t REG_LAUNCH = 128, REG_LO = 80, REG_HI = 176;
+    static_assert(256 * REG_LO + 256 * REG_HI == THREADS * REG_LAUNCH, "register split must match the launch");
     // W4A8 low-rank stage (one per tile, after the K stages): A = the u pair, 128 rows x 64
     // bf16 (128-byte rows, 128-byte swizzle); B = packed L2, 128 rows x 32 bf16 (64-byte
     // rows, 64-byte swizzle); four kind::f16 MMAs of K = 16 (u_hi x L2, then u_lo x L2).
@@ -437,7 +453,7 @@ struct Gemm2Cfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert((STAGES * (A_BYTES + B_BYTES)) % 1024 == 0, "staging tiles 1024-byte aligned");
     static_assert(TB >= 2 && SF_COL0 + TB * SF_COLS <= GEMM_TMEM_COLS, "TMEM budget");
-    static_assert(OVL == 64 || OVL == 96, "epilogue overlap handling");
+    static_assert(SINGLE || OVL == 64 || OVL == 96, "epilogue overlap handling");
 };
 
 // Pair-kernel epilogue: pack one row's 64 columns and write them, as 128 bytes, into row
@@ -588,7 +604,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                  const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                  const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmU,
                  const __grid_constant__ CUtensorMap tmL, GemmParams p) {
-    using C = Gemm2Cfg<KIND>;
+    using C = Gemm2Cfg<KIND, OUTQ>;
     constexpr int S = C::STAGES;
     constexpr int TB = C::TB;
     extern __shared__ uint8_t smem_raw[];
@@ -626,7 +642,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             mbar_init(&tmem_full[b], 1);
             mbar_init(&acc_free[b], 16);
         }
-        mbar_init(ovl_free, 8);
+        mbar_init(ovl_free, C::SINGLE ? 16 : 8);
         mbar_init(mma_done, 1);
         *abort = 0;
         fence_mbar_init();
@@ -665,242 +681,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
     const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
     const Sched sched0{num_tiles, num_kb, num_pairs, pair, SK, 0, 0, 0};
 
-    if (warp == 0) {
-        // ============================================================ producer (both CTAs)
-        if (lane == 0) {
-            // the activations may come from the kernel just before us (programmatic launch)
-            griddep_wait();
-            const uint64_t pol_a = policy_evict_normal();
-            const uint64_t pol_b = policy_evict_last();
-            int it = 0;
-            bool ok = true;
-            Sched sc = sched0;
-            sc.begin();
-            int tile, kb0, kb1;
-            while (ok && sc.get(tile, kb0, kb1)) {
-                const int mb = tile / num_n, nb = tile % num_n;
-                for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (uint32_t)(it / S) & 1u;
-                    if (!mbar_wait(&empty[s], ph ^ 1u, p.timeout_ns, abort)) {
-                        gemm2_fail(p, abort, peer_abort);
-                        ok = false;
-                        break;
-                    }
-                    if (it == p.skip_iter) continue;  // test hook: this stage is never filled
-                    // A/B of both CTAs land on the leader's barrier; only the leader expects them
-                    const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
-                    if (HAS_LR && kb == num_kb) {
-                        // low-rank stage: u pair rows and packed-L2 rows; no scale atoms, but
-                        // sf_full still completes a phase so its parity keeps counting stages
-                        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::LR_TX);
-                        mbar_arrive(&sf_full[s]);
-                        tma_load_2d_pair(sA + s * C::A_BYTES, &tmU, bar, 0, mb * 256 + (int)rank * 128, pol_a);
-                        tma_load_2d_pair(sB + s * C::B_BYTES, &tmL, bar, 0, nb * 256 + (int)rank * 128, pol_b);
-                        continue;
-                    }
-                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::AB_TX);
-                    mbar_arrive_expect_tx(&sf_full[s], C::SF_TX);
-                    // x: bytes of the row for packed FP4 and E4M3, elements for the W4A8 unpacking map
-                    const int ax = kb * C::ROW_BYTES;
-                    const int bx = (KIND == G_W4A8) ? kb * C::BK : kb * C::ROW_BYTES;
-                    tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, bar, ax, mb * 256 + (int)rank * 128, pol_a);
-                    tma_load_2d_pair(sB + s * C::B_BYTES, &tmB, bar, bx, nb * 256 + (int)rank * 128, pol_b);
-                    tma_load_2d(sRSFA + s * C::RSFA_BYTES, &tmSFA, &sf_full[s], 0,
-                                (mb * 2 + (int)rank) * apr + kb * C::ATOMS, pol_a);
-#pragma unroll
-                    for (int j = 0; j < 2; ++j)
-                        tma_load_2d(sRSFB + s * C::RSFB_BYTES + j * C::ATOMS * 512, &tmSFB, &sf_full[s], 0,
-                                    (nb * 2 + j) * apr + kb * C::ATOMS, pol_b);
-                }
-                sc.step(kb0, kb1);
-            }
-            // drain what this CTA issued: its scale loads, and (leader) both CTAs' A/B
-            for (int j = max(0, it - S); j < it; ++j) {
-                if (j == p.skip_iter) continue;
-                if (!mbar_wait_drain(&sf_full[j % S], (uint32_t)(j / S) & 1u, p.timeout_ns))
-                    gemm2_fail(p, abort, peer_abort);
-                if (rank == 0 && !mbar_wait_drain(&full[j % S], (uint32_t)(j / S) & 1u, p.timeout_ns))
-                    gemm2_fail(p, abort, peer_abort);
-            }
-        }
-    } else if (warp >= 10 && warp < 14) {
-        // ============================================================ scale writers (both CTAs)
-        const int quarter = warp & 3;
-        const uint32_t tlane = tmem_base + ((uint32_t)(quarter * 32) << 16);
-        int it = 0;
-        bool ok = true;
-        Sched sc = sched0;
-        sc.begin();
-        int tile, kb0, kb1;
-        while (ok && sc.get(tile, kb0, kb1)) {
-            for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
-                const int s = it % S;
-                const int t = it % TB;
-                bool got = mbar_wait(&sf_full[s], (uint32_t)(it / S) & 1u, p.timeout_ns, abort);
-                if (!__all_sync(0xffffffffu, got)) {
-                    if (lane == 0) gemm2_fail(p, abort, peer_abort);
-                    ok = false;
-                    break;
-                }
-                const uint4* rsfa = reinterpret_cast<const uint4*>(sRSFA + s * C::RSFA_BYTES);
-                const uint4* rsfb = reinterpret_cast<const uint4*>(sRSFB + s * C::RSFB_BYTES);
-                // lane i takes row i of every atom: words 0-3 = the scales of rows i, 32+i, 64+i, 96+i
-                uint32_t va[4 * C::ATOMS];
-                uint32_t vb[8 * C::ATOMS];
-#pragma unroll
-                for (int a = 0; a < C::ATOMS; ++a) {
-                    const uint4 w = rsfa[a * 32 + lane];
-                    va[4 * a] = w.x, va[4 * a + 1] = w.y, va[4 * a + 2] = w.z, va[4 * a + 3] = w.w;
-#pragma unroll
-                    for (int rb = 0; rb < 2; ++rb) {
-                        const uint4 z = rsfb[(rb * C::ATOMS + a) * 32 + lane];
-                        vb[8 * a + 4 * rb] = z.x, vb[8 * a + 4 * rb + 1] = z.y;
-                        vb[8 * a + 4 * rb + 2] = z.z, vb[8 * a + 4 * rb + 3] = z.w;
-                    }
-                }
-                // buffer t is free once the MMAs of iteration it - TB (same buffer) are done
-                got = it < TB || mbar_wait(&empty[(it - TB) % S], (uint32_t)((it - TB) / S) & 1u, p.timeout_ns, abort);
-                if (!__all_sync(0xffffffffu, got)) {
-                    if (lane == 0) gemm2_fail(p, abort, peer_abort);
-                    ok = false;
-                    break;
-                }
-                const uint32_t xa = C::SF_COL0 + (uint32_t)(t * C::SF_COLS);
-                const uint32_t xb = xa + C::SFA_COLS;
-                // the W4A8 low-rank stage reads no scales: its buffer turn passes unwritten
-                if (HAS_LR && kb == num_kb) {
-                } else if constexpr (C::ATOMS == 4) {
-                    tmem_st_32x32b_x16(tlane + xa, *reinterpret_cast<const uint32_t(*)[16]>(va));
-                    tmem_st_32x32b_x16(tlane + xb, *reinterpret_cast<const uint32_t(*)[16]>(vb));
-                    tmem_st_32x32b_x16(tlane + xb + 16, *reinterpret_cast<const uint32_t(*)[16]>(vb + 16));
-                } else if constexpr (C::ATOMS == 2) {
-                    tmem_st_32x32b_x8(tlane + xa, va);
-                    tmem_st_32x32b_x16(tlane + xb, vb);
-                } else {
-                    tmem_st_32x32b_x4(tlane + xa, va);
-                    tmem_st_32x32b_x8(tlane + xb, vb);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) arrive_leader_relaxed(&sf_ready[t], rank);
-            }
-            sc.step(kb0, kb1);
-        }
-    } else if (warp == 1) {
-        // ============================================================ MMA issuer (leader)
-        // The whole warp runs the loop so that it can take the named barrier each stage;
-        // lane 0 issues.  Per stage it touches no shared memory at all: the coordinator
-        // warp has checked everything the stage needs before releasing it, and the abort
-        // flag is read once per tile (the coordinator releases every stage of a tile even
-        // after a failure, so the warp always reaches that check).
-        if (rank == 0) {
-            uint32_t it = 0;
-            int tcount = 0;
-            bool issued = false, ok = true;
-            Sched sc = sched0;
-            sc.begin();
-            int tile, kb0, kb1;
-            for (; ok && sc.get(tile, kb0, kb1); sc.step(kb0, kb1), ++tcount) {
-                const int b = tcount & 1;
-                const uint32_t dacc = tmem_base + (uint32_t)(b * C::ACC1_COL);
-                for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
-                    named_bar_sync(1u + it % TB, 64u);
-                    if (lane == 0 && HAS_LR && kb == num_kb) {
-                        // low-rank stage: acc += u_hi L2 + u_lo L2 (bf16 x bf16 -> fp32)
-                        tc_fence_after();
-                        const int s = (int)(it % S);
-                        const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
-                        const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint64_t adesc = smem_desc(a_base + k * 32, 0, 1024, 2u);
-                            const uint64_t bdesc = smem_desc(b_base + (k & 1) * 32, 0, 512, 4u);
-                            mma2_f16(dacc, adesc, bdesc, C::IDESC_LR, 1u);
-                        }
-                        tc_commit_pair(&empty[s], 0x3);
-                    } else if (lane == 0) {
-                        tc_fence_after();
-                        const int s = (int)(it % S);
-                        const int t = (int)(it % TB);
-                        const int n_mma = min(C::BK, K - kb * C::BK) / C::MMA_K;
-                        const uint32_t tsfa = tmem_base + C::SF_COL0 + (uint32_t)(t * C::SF_COLS);
-                        const uint32_t tsfb = tsfa + C::SFA_COLS;
-                        const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
-                        const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
-                        for (int k = 0; k < n_mma; ++k) {
-                            int atom, sf_id;
-                            sf_select<KIND>(k, atom, sf_id);
-                            const uint32_t idesc = C::IDESC | ((uint32_t)sf_id << 29) | ((uint32_t)sf_id << 4);
-                            const uint64_t adesc = smem_desc(a_base + k * 32, 0, C::SBO, C::SWZ);
-                            const uint64_t bdesc = smem_desc(b_base + k * 32, 0, C::SBO, C::SWZ);
-                            const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
-                            if (KIND == G_MXFP4 || KIND == G_SVD4)
-                                mma2_mxf4nvf4_block32(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
-                            else if (KIND == G_NVFP4)
-                                mma2_mxf4nvf4_block16(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
-                            else
-                                mma2_mxf8f6f4_block32(dacc, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
-                        }
-                        tc_commit_pair(&empty[s], 0x3);
-                    }
-                    __syncwarp();
-                    issued = true;
-                }
-                if (lane == 0) tc_commit_pair(&tmem_full[b], 0x3);
-                __syncwarp();
-                if (__any_sync(0xffffffffu, *abort != 0)) ok = false;
-            }
-            if (issued) {
-                if (lane == 0) tc_commit_pair(mma_done, 0x1);
-                __syncwarp();
-                const bool drained = mbar_wait_drain(mma_done, 0, p.timeout_ns);
-                if (!__all_sync(0xffffffffu, drained) && lane == 0) gemm2_fail(p, abort, peer_abort);
-            }
-        }
-        __syncwarp();
-    } else if (warp == 14) {
-        // ============================================================ stage coordinator (leader)
-        // Waits, in the MMA warp's order, for everything a stage needs (the accumulator
-        // and the overlap at a tile's first stage; A/B bytes of both CTAs; both CTAs'
-        // scale buffer) and then releases the stage with named barrier 1 + it % TB.  After
-        // a failure it still releases the remaining stages of that tile without waiting,
-        // so the MMA warp, which checks the abort flag at the end of each tile, never
-        // waits on a barrier that nobody arrives at.  The ring of TB barrier ids cannot be lapped:
-        // the scale buffer of stage it + TB is free only after the MMA warp has passed
-        // stage it.
-        if (rank == 0) {
-            uint32_t it = 0;
-            int tcount = 0;
-            bool ok = true;
-            Sched sc = sched0;
-            sc.begin();
-            int tile, kb0, kb1;
-            for (; ok && sc.get(tile, kb0, kb1); sc.step(kb0, kb1), ++tcount) {
-                const int b = tcount & 1;
-                // accumulator b drained (unit tcount-2) and the overlap of unit tcount-1 drained
-                bool got = mbar_wait(&acc_free[b], (((uint32_t)tcount >> 1) & 1u) ^ 1u, p.timeout_ns, abort);
-                if (got && tcount > 0) got = mbar_wait(ovl_free, (uint32_t)(tcount - 1) & 1u, p.timeout_ns, abort);
-                for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
-                    if (got) got = mbar_wait(&full[it % S], (it / S) & 1u, p.timeout_ns, abort);
-                    if (got) got = mbar_wait(&sf_ready[it % TB], (it / TB) & 1u, p.timeout_ns, abort);
-                    got = __all_sync(0xffffffffu, got);
-                    if (!got && ok) {
-                        if (lane == 0) gemm2_fail(p, abort, peer_abort);
-                        ok = false;
-                    }
-                    __syncwarp();
-                    named_bar_arrive(1u + it % TB, 64u);
-                }
-            }
-        }
-    } else if (warp >= 2) {
+    if (warp >= 8) {
+        // the two epilogue warpgroups take the registers the control warps give up
+        setmaxnreg_inc<C::REG_HI>();
         // ============================================================ epilogue (both CTAs)
+        // Epilogue warp ew = warp - 8 drains TMEM lane quarter warp % 4 (the only quarter a
+        // warp can reach) and column half ew / 4 of every tile: 32 rows x 128 columns.
+        const int ew = warp - 8;
         const int q = warp & 3;
-        const int h = (warp - 2) >> 2;
-        uint8_t* stile = sEpi + (warp - 2) * 4096;
-        uint32_t acc[2][32];
+        const int h = ew >> 2;
+        uint8_t* stile = sEpi + ew * 4096;
+        // acc: the 64-column pair being written; acc2: the second pair of a one-go drain
+        uint32_t acc[2][32], acc2[2][32];
         float gs = 1.0f;
         if (KIND == G_NVFP4) gs = __fmul_rn(*p.g_a, *p.g_w);
         float g_h = 1.0f, six_g_h = 6.0f;
@@ -937,18 +729,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             // (float4 (chunk, j4, lane) at ((chunk * 8 + j4) * 32 + lane) * 4) so every warp
             // instruction writes or reads 512 contiguous bytes; the summing warp has the same
             // rows and lanes, so only it needs to know the layout
-            float* slab0 = p.partials + (size_t)tile * p.seg_max * 65536 + ((int)rank * 8 + (warp - 2)) * 4096 + lane * 4;
+            float* slab0 = p.partials + (size_t)tile * p.seg_max * 65536 + ((int)rank * 8 + ew) * 4096 + lane * 4;
             // pack 64 columns into the staging tile and hand them to one TMA store (which
             // clips rows at or beyond M); the tile is reused once the previous store has read it
-            auto emit = [&](int chunk) {
+            auto emit = [&](uint32_t (&a)[2][32], int chunk) {
                 if (OUTQ != 0) {
-                    epilogue_gelu_quant<KIND, OUTQ>(p, acc, row, col0 + chunk * 32, gs, g_h, six_g_h);
+                    epilogue_gelu_quant<KIND, OUTQ>(p, a, row, col0 + chunk * 32, gs, g_h, six_g_h);
                     return;
                 }
                 if (col0 >= p.N) return;
                 if (lane == 0) bulk_wait_group_read0();
                 __syncwarp();
-                epilogue_stage<KIND>(p, acc, row, col0 + chunk * 32, gs, stile, lane);
+                epilogue_stage<KIND>(p, a, row, col0 + chunk * 32, gs, stile, lane);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0 && row0 < p.M) {
@@ -957,9 +749,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 }
             };
             // a split tile: this segment's fp32 sums of the 64 columns go to its slab
-            auto stage_store = [&](int chunk) {
+            auto stage_store = [&](uint32_t (&a)[2][32], int chunk) {
                 if (!SK || nseg == 1) {
-                    emit(chunk);
+                    emit(a, chunk);
                     return;
                 }
                 float* dst = slab0 + (size_t)seg * 65536;
@@ -968,33 +760,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4*>(dst + (((chunk + c) * 8 + j / 4) * 32) * 4) =
-                            make_float4(__uint_as_float(acc[c][j]), __uint_as_float(acc[c][j + 1]),
-                                        __uint_as_float(acc[c][j + 2]), __uint_as_float(acc[c][j + 3]));
+                            make_float4(__uint_as_float(a[c][j]), __uint_as_float(a[c][j + 1]),
+                                        __uint_as_float(a[c][j + 2]), __uint_as_float(a[c][j + 3]));
             };
-            // the OVL columns shared by both accumulators are the last OVL tile columns of
-            // accumulator 0 (half 1) or the first OVL of accumulator 1 (half 0): their holders
-            // drain them first and release them -- after the first chunk pair when OVL = 64,
-            // after both pairs when OVL = 96 (NVFP4)
-            const bool holds_overlap = (h == (b == 0 ? 1 : 0));
-            const int first = holds_overlap ? (b == 0 ? 2 : 0) : 0;
-            const int second = 2 - first;
-            tmem_ld_32x32b_x32(taddr + first * 32, acc[0]);
-            tmem_ld_32x32b_x32(taddr + (first + 1) * 32, acc[1]);
-            tmem_wait_ld();
-            if (holds_overlap && C::OVL <= 64) {
+            if constexpr (C::SINGLE) {
+                // one accumulator: the warp's 128 columns go to registers at once and the
+                // accumulator is handed back before any of them is converted
+                tmem_ld_32x32b_x32(taddr, acc[0]);
+                tmem_ld_32x32b_x32(taddr + 32, acc[1]);
+                tmem_ld_32x32b_x32(taddr + 64, acc2[0]);
+                tmem_ld_32x32b_x32(taddr + 96, acc2[1]);
+                tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) arrive_leader_relaxed(ovl_free, rank);
+                if (lane == 0) {
+                    arrive_leader_relaxed(ovl_free, rank);
+                    arrive_leader_relaxed(&acc_free[b], rank);
+                }
+                stage_store(acc, 0);
+                stage_store(acc2, 2);
+            } else {
+                // the OVL columns shared by both accumulators are the last OVL tile columns of
+                // accumulator 0 (half 1) or the first OVL of accumulator 1 (half 0): their holders
+                // drain them first and release them -- after the first chunk pair when OVL = 64,
+                // after both pairs when OVL = 96 (NVFP4)
+                const bool holds_overlap = (h == (b == 0 ? 1 : 0));
+                const int first = holds_overlap ? (b == 0 ? 2 : 0) : 0;
+                const int second = 2 - first;
+                tmem_ld_32x32b_x32(taddr + first * 32, acc[0]);
+                tmem_ld_32x32b_x32(taddr + (first + 1) * 32, acc[1]);
+                tmem_wait_ld();
+                if (holds_overlap && C::OVL <= 64) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) arrive_leader_relaxed(ovl_free, rank);
+                }
+                stage_store(acc, first);
+                tmem_ld_32x32b_x32(taddr + second * 32, acc[0]);
+                tmem_ld_32x32b_x32(taddr + (second + 1) * 32, acc[1]);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (holds_overlap && C::OVL > 64 && lane == 0) arrive_leader_relaxed(ovl_free, rank);
+                if (lane == 0) arrive_leader_relaxed(&acc_free[b], rank);
+                stage_store(acc, second);
             }
-            stage_store(first);
-            tmem_ld_32x32b_x32(taddr + second * 32, acc[0]);
-            tmem_ld_32x32b_x32(taddr + (second + 1) * 32, acc[1]);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (holds_overlap && C::OVL > 64 && lane == 0) arrive_leader_relaxed(ovl_free, rank);
-            if (lane == 0) arrive_leader_relaxed(&acc_free[b], rank);
-            stage_store(second);
             if (SK && nseg > 1) {
                 // the last of the tile's segments to arrive sums the slabs in segment order
                 // (a fixed order, so the result does not depend on which one is last) and
@@ -1002,7 +812,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 __threadfence();
                 __syncwarp();
                 int last = 0;
-                if (lane == 0) last = atomicAdd(p.counters + tile * 16 + (int)rank * 8 + (warp - 2), 1) == nseg - 1;
+                if (lane == 0) last = atomicAdd(p.counters + tile * 16 + (int)rank * 8 + ew, 1) == nseg - 1;
                 last = __shfl_sync(0xffffffffu, last, 0);
                 if (last) {
                     __threadfence();
@@ -1029,7 +839,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                                     }
                                 }
                         }
-                        emit(pr);
+                        emit(acc, pr);
                     }
                 }
             }
@@ -1037,6 +847,252 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         // the staging tile must outlive the stores that read it
         if (lane == 0) bulk_wait_group0();
         __syncwarp();
+    } else {
+        // warps 0-7: producer, MMA issuer, coordinator, an idle warp and the scale writers
+        setmaxnreg_dec<C::REG_LO>();
+        if (warp == 0) {
+            // ============================================================ producer (both CTAs)
+            if (lane == 0) {
+                // the activations may come from the kernel just before us (programmatic launch)
+                griddep_wait();
+                const uint64_t pol_a = policy_evict_normal();
+                const uint64_t pol_b = policy_evict_last();
+                int it = 0;
+                bool ok = true;
+                Sched sc = sched0;
+                sc.begin();
+                int tile, kb0, kb1;
+                while (ok && sc.get(tile, kb0, kb1)) {
+                    const int mb = tile / num_n, nb = tile % num_n;
+                    for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
+                        const int s = it % S;
+                        const uint32_t ph = (uint32_t)(it / S) & 1u;
+                        if (!mbar_wait(&empty[s], ph ^ 1u, p.timeout_ns, abort)) {
+                            gemm2_fail(p, abort, peer_abort);
+                            ok = false;
+                            break;
+                        }
+                        if (it == p.skip_iter) continue;  // test hook: this stage is never filled
+                        // A/B of both CTAs land on the leader's barrier; only the leader expects them
+                        const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+                        if (HAS_LR && kb == num_kb) {
+                            // low-rank stage: u pair rows and packed-L2 rows; no scale atoms, but
+                            // sf_full still completes a phase so its parity keeps counting stages
+                            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::LR_TX);
+                            mbar_arrive(&sf_full[s]);
+                            tma_load_2d_pair(sA + s * C::A_BYTES, &tmU, bar, 0, mb * 256 + (int)rank * 128, pol_a);
+                            tma_load_2d_pair(sB + s * C::B_BYTES, &tmL, bar, 0, nb * 256 + (int)rank * 128, pol_b);
+                            continue;
+                        }
+                        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::AB_TX);
+                        mbar_arrive_expect_tx(&sf_full[s], C::SF_TX);
+                        // x: bytes of the row for packed FP4 and E4M3, elements for the W4A8 unpacking map
+                        const int ax = kb * C::ROW_BYTES;
+                        const int bx = (KIND == G_W4A8) ? kb * C::BK : kb * C::ROW_BYTES;
+                        tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, bar, ax, mb * 256 + (int)rank * 128, pol_a);
+                        tma_load_2d_pair(sB + s * C::B_BYTES, &tmB, bar, bx, nb * 256 + (int)rank * 128, pol_b);
+                        tma_load_2d(sRSFA + s * C::RSFA_BYTES, &tmSFA, &sf_full[s], 0,
+                                    (mb * 2 + (int)rank) * apr + kb * C::ATOMS, pol_a);
+    #pragma unroll
+                        for (int j = 0; j < 2; ++j)
+                            tma_load_2d(sRSFB + s * C::RSFB_BYTES + j * C::ATOMS * 512, &tmSFB, &sf_full[s], 0,
+                                        (nb * 2 + j) * apr + kb * C::ATOMS, pol_b);
+                    }
+                    sc.step(kb0, kb1);
+                }
+                // drain what this CTA issued: its scale loads, and (leader) both CTAs' A/B
+                for (int j = max(0, it - S); j < it; ++j) {
+                    if (j == p.skip_iter) continue;
+                    if (!mbar_wait_drain(&sf_full[j % S], (uint32_t)(j / S) & 1u, p.timeout_ns))
+                        gemm2_fail(p, abort, peer_abort);
+                    if (rank == 0 && !mbar_wait_drain(&full[j % S], (uint32_t)(j / S) & 1u, p.timeout_ns))
+                        gemm2_fail(p, abort, peer_abort);
+                }
+            }
+        } else if (warp >= 4) {
+            // ============================================================ scale writers (both CTAs)
+            const int quarter = warp & 3;
+            const uint32_t tlane = tmem_base + ((uint32_t)(quarter * 32) << 16);
+            int it = 0;
+            bool ok = true;
+            Sched sc = sched0;
+            sc.begin();
+            int tile, kb0, kb1;
+            while (ok && sc.get(tile, kb0, kb1)) {
+                for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
+                    const int s = it % S;
+                    const int t = it % TB;
+                    bool got = mbar_wait(&sf_full[s], (uint32_t)(it / S) & 1u, p.timeout_ns, abort);
+                    if (!__all_sync(0xffffffffu, got)) {
+                        if (lane == 0) gemm2_fail(p, abort, peer_abort);
+                        ok = false;
+                        break;
+                    }
+                    const uint4* rsfa = reinterpret_cast<const uint4*>(sRSFA + s * C::RSFA_BYTES);
+                    const uint4* rsfb = reinterpret_cast<const uint4*>(sRSFB + s * C::RSFB_BYTES);
+                    // lane i takes row i of every atom: words 0-3 = the scales of rows i, 32+i, 64+i, 96+i
+                    uint32_t va[4 * C::ATOMS];
+                    uint32_t vb[8 * C::ATOMS];
+    #pragma unroll
+                    for (int a = 0; a < C::ATOMS; ++a) {
+                        const uint4 w = rsfa[a * 32 + lane];
+                        va[4 * a] = w.x, va[4 * a + 1] = w.y, va[4 * a + 2] = w.z, va[4 * a + 3] = w.w;
+    #pragma unroll
+                        for (int rb = 0; rb < 2; ++rb) {
+                            const uint4 z = rsfb[(rb * C::ATOMS + a) * 32 + lane];
+                            vb[8 * a + 4 * rb] = z.x, vb[8 * a + 4 * rb + 1] = z.y;
+                            vb[8 * a + 4 * rb + 2] = z.z, vb[8 * a + 4 * rb + 3] = z.w;
+                        }
+                    }
+                    // buffer t is free once the MMAs of iteration it - TB (same buffer) are done
+                    got = it < TB || mbar_wait(&empty[(it - TB) % S], (uint32_t)((it - TB) / S) & 1u, p.timeout_ns, abort);
+                    if (!__all_sync(0xffffffffu, got)) {
+                        if (lane == 0) gemm2_fail(p, abort, peer_abort);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t xa = C::SF_COL0 + (uint32_t)(t * C::SF_COLS);
+                    const uint32_t xb = xa + C::SFA_COLS;
+                    // the W4A8 low-rank stage reads no scales: its buffer turn passes unwritten
+                    if (HAS_LR && kb == num_kb) {
+                    } else if constexpr (C::ATOMS == 4) {
+                        tmem_st_32x32b_x16(tlane + xa, *reinterpret_cast<const uint32_t(*)[16]>(va));
+                        tmem_st_32x32b_x16(tlane + xb, *reinterpret_cast<const uint32_t(*)[16]>(vb));
+                        tmem_st_32x32b_x16(tlane + xb + 16, *reinterpret_cast<const uint32_t(*)[16]>(vb + 16));
+                    } else if constexpr (C::ATOMS == 2) {
+                        tmem_st_32x32b_x8(tlane + xa, va);
+                        tmem_st_32x32b_x16(tlane + xb, vb);
+                    } else {
+                        tmem_st_32x32b_x4(tlane + xa, va);
+                        tmem_st_32x32b_x8(tlane + xb, vb);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) arrive_leader_relaxed(&sf_ready[t], rank);
+                }
+                sc.step(kb0, kb1);
+            }
+        } else if (warp == 1) {
+            // ============================================================ MMA issuer (leader)
+            // The whole warp runs the loop so that it can take the named barrier each stage;
+            // lane 0 issues.  Per stage it touches no shared memory at all: the coordinator
+            // warp has checked everything the stage needs before releasing it, and the abort
+            // flag is read once per tile (the coordinator releases every stage of a tile even
+            // after a failure, so the warp always reaches that check).
+            // The issuing thread's own latency decides the MMA rate: with the stage's four MMAs
+            // unrolled and every operand a running value or a constant offset, a stage issues
+            // at the tensor pipe's 128 cycles per 256x256x64 MMA; recomputing descriptors,
+            // scale ids and slot indices per MMA was measured at ~150.
+            if (rank == 0) {
+                uint32_t it = 0;
+                int tcount = 0;
+                bool issued = false, ok = true;
+                int s = 0, t = 0;  // it % S and it % TB
+                const uint64_t adesc0 = smem_desc(smem_u32(sA), 0, C::SBO, C::SWZ);
+                const uint64_t bdesc0 = smem_desc(smem_u32(sB), 0, C::SBO, C::SWZ);
+                Sched sc = sched0;
+                sc.begin();
+                int tile, kb0, kb1;
+                for (; ok && sc.get(tile, kb0, kb1); sc.step(kb0, kb1), ++tcount) {
+                    const int b = tcount & 1;
+                    const uint32_t dacc = tmem_base + (uint32_t)(b * C::ACC1_COL);
+                    for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
+                        named_bar_sync(1u + (uint32_t)t, 64u);
+                        if (lane == 0 && HAS_LR && kb == num_kb) {
+                            // low-rank stage: acc += u_hi L2 + u_lo L2 (bf16 x bf16 -> fp32)
+                            tc_fence_after();
+                            const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
+                            const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
+    #pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const uint64_t adesc = smem_desc(a_base + k * 32, 0, 1024, 2u);
+                                const uint64_t bdesc = smem_desc(b_base + (k & 1) * 32, 0, 512, 4u);
+                                mma2_f16(dacc, adesc, bdesc, C::IDESC_LR, 1u);
+                            }
+                            tc_commit_pair(&empty[s], 0x3);
+                        } else if (lane == 0) {
+                            tc_fence_after();
+                            // slot s's descriptors: slot 0's plus s * bytes / 16 in the start-address
+                            // field; MMA k reads the 32 bytes at k * 32 of every 128-byte row
+                            const uint64_t adesc = adesc0 + (uint64_t)(s * (C::A_BYTES >> 4));
+                            const uint64_t bdesc = bdesc0 + (uint64_t)(s * (C::B_BYTES >> 4));
+                            const uint32_t tsfa = tmem_base + C::SF_COL0 + (uint32_t)(t * C::SF_COLS);
+                            const uint32_t tsfb = tsfa + C::SFA_COLS;
+                            const uint32_t acc0 = kb > kb0 ? 1u : 0u;
+                            // a last stage of K % BK = 128 (FP4 kinds) holds two MMAs
+                            const bool half = (KIND != G_W4A8) && (K - kb * C::BK < C::BK);
+    #pragma unroll
+                            for (int k = 0; k < C::N_MMA; ++k) {
+                                if (k >= 2 && half) break;
+                                int atom, sf_id;
+                                sf_select<KIND>(k, atom, sf_id);
+                                const uint32_t idesc = C::IDESC | ((uint32_t)sf_id << 29) | ((uint32_t)sf_id << 4);
+                                const uint32_t acc = k > 0 ? 1u : acc0;
+                                const uint64_t ad = adesc + (uint64_t)(k * 2), bd = bdesc + (uint64_t)(k * 2);
+                                if (KIND == G_MXFP4 || KIND == G_SVD4)
+                                    mma2_mxf4nvf4_block32(dacc, ad, bd, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                                else if (KIND == G_NVFP4)
+                                    mma2_mxf4nvf4_block16(dacc, ad, bd, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                                else
+                                    mma2_mxf8f6f4_block32(dacc, ad, bd, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                            }
+                            tc_commit_pair(&empty[s], 0x3);
+                        }
+                        __syncwarp();
+                        issued = true;
+                        if (++s == S) s = 0;
+                        if (++t == TB) t = 0;
+                    }
+                    if (lane == 0) tc_commit_pair(&tmem_full[b], 0x3);
+                    __syncwarp();
+                    if (__any_sync(0xffffffffu, *abort != 0)) ok = false;
+                }
+                if (issued) {
+                    if (lane == 0) tc_commit_pair(mma_done, 0x1);
+                    __syncwarp();
+                    const bool drained = mbar_wait_drain(mma_done, 0, p.timeout_ns);
+                    if (!__all_sync(0xffffffffu, drained) && lane == 0) gemm2_fail(p, abort, peer_abort);
+                }
+            }
+            __syncwarp();
+        } else if (warp == 2) {
+            // ============================================================ stage coordinator (leader)
+            // Waits, in the MMA warp's order, for everything a stage needs (the accumulator
+            // and the overlap at a tile's first stage; A/B bytes of both CTAs; both CTAs'
+            // scale buffer) and then releases the stage with named barrier 1 + it % TB.  After
+            // a failure it still releases the remaining stages of that tile without waiting,
+            // so the MMA warp, which checks the abort flag at the end of each tile, never
+            // waits on a barrier that nobody arrives at.  The ring of TB barrier ids cannot be lapped:
+            // the scale buffer of stage it + TB is free only after the MMA warp has passed
+            // stage it.
+            if (rank == 0) {
+                uint32_t it = 0;
+                int tcount = 0;
+                bool ok = true;
+                Sched sc = sched0;
+                sc.begin();
+                int tile, kb0, kb1;
+                for (; ok && sc.get(tile, kb0, kb1); sc.step(kb0, kb1), ++tcount) {
+                    const int b = tcount & 1;
+                    // accumulator b drained (unit tcount-2) and the overlap of unit tcount-1 drained
+                    // (with one accumulator the "overlap" is all of it: every epilogue warp arrives)
+                    bool got = mbar_wait(&acc_free[b], (((uint32_t)tcount >> 1) & 1u) ^ 1u, p.timeout_ns, abort);
+                    if (got && tcount > 0) got = mbar_wait(ovl_free, (uint32_t)(tcount - 1) & 1u, p.timeout_ns, abort);
+                    for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
+                        if (got) got = mbar_wait(&full[it % S], (it / S) & 1u, p.timeout_ns, abort);
+                        if (got) got = mbar_wait(&sf_ready[it % TB], (it / TB) & 1u, p.timeout_ns, abort);
+                        got = __all_sync(0xffffffffu, got);
+                        if (!got && ok) {
+                            if (lane == 0) gemm2_fail(p, abort, peer_abort);
+                            ok = false;
+                        }
+                        __syncwarp();
+                        named_bar_arrive(1u + it % TB, 64u);
+                    }
+                }
+            }
+        }
     }
 
     tc_fence_before();

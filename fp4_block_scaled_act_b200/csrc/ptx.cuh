@@ -80,6 +80,18 @@ FP4_DEV void named_bar_arrive(uint32_t id, uint32_t count) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Warpgroup register reallocation (all four warps of a warpgroup execute it together):
+// dec returns registers to the CTA's pool, inc waits until the pool can supply them.  The
+// increments of a kernel must be covered by the registers it was launched with.
+template <uint32_t R>
+FP4_DEV void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+FP4_DEV void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+
 // Packed fp32 pairs (sm_100 f32x2): each lane of the pair is one IEEE fp32 operation.
 FP4_DEV uint64_t f2_pack(float lo, float hi) {
     uint64_t r;
