@@ -375,17 +375,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // the TMEM store and the arrive follow that wait.
 //
 // Accumulators: two 256-column accumulators overlapping by 64 columns ([0,256),
-// [192,448)) -- 96 for NVFP4 with a fused epilogue -- drained 64 columns at a time with
-// the shared columns first, so the next tile's MMAs wait for that part only; the scale
-// buffers follow the second accumulator.  NVFP4 with plain bf16 output uses one
-// accumulator [0,256) instead: each epilogue warp copies its 32 x 128 share to registers
-// with four tcgen05.ld and hands the accumulator back at once, and columns [256,512) hold
-// four scale buffers.
+// [192,448)), or by 96 for NVFP4; the epilogue drains the shared columns first, so the
+// next tile's MMAs wait for that part only.  The scale buffers follow the second
+// accumulator.
 //
 // Warps (512 threads, four warpgroups): 0 TMA producer, 1 TMEM owner + MMA issuer
 // (leader), 2 stage coordinator (leader), 3 idle, 4-7 scale writers, 8-15 epilogue.  The
 // control warpgroups (0-7) drop to REG_LO registers per thread with setmaxnreg and the
-// epilogue warpgroups rise to REG_HI, so a 128-column drain fits in registers.
+// epilogue warpgroups rise to REG_HI: the fused epilogues run without spilling, and an
+// NVFP4 overlap holder can copy its whole 128-column share before converting any.
 // The tensor pipe queues very little ahead of the issuing thread, so every cycle that
 // thread spends between two MMAs is a bubble.  The MMA warp therefore tests no mbarrier:
 // the coordinator does the waits and hands each stage over with a hardware named barrier
@@ -397,8 +395,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 //   sf_ready[t]  (leader)  scale buffer t written in both CTAs (8 writer warps)
 //   tmem_full[b] (both)    accumulator b complete
 //   acc_free[b]  (leader)  accumulator b fully drained by both CTAs (16 warps)
-//   ovl_free     (leader)  overlap columns of the last tile drained (8 warps; with one
-//                          accumulator, all of it copied out by all 16 epilogue warps)
+//   ovl_free     (leader)  overlap columns of the last tile drained (8 warps)
 // =======================================================================================
 template <int KIND, int OUTQ = 0>
 struct Gemm2Cfg {
@@ -423,17 +420,17 @@ struct Gemm2Cfg {
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + 512;
     static constexpr uint32_t AB_TX = A_BYTES + ((KIND == G_W4A8) ? B_BYTES / 2 : B_BYTES);
     static constexpr uint32_t SF_TX = RSFA_BYTES + RSFB_BYTES;
-    // TMEM columns.  Two accumulators overlapping by OVL columns, drained 64 columns at a
-    // time with the shared columns first: NVFP4 stages carry 4 scale atoms (48 columns),
-    // so its accumulators overlap by 96 to leave room for two scale buffers; the others
-    // overlap by 64.  NVFP4 with plain bf16 output (OUTQ 0) instead keeps one accumulator
-    // [0,256), which the epilogue copies to registers in one go, and four scale buffers
-    // from column 256: measured faster there than waiting for a 96-column drain, while for
-    // MXFP4 the 128 KB burst of TMEM reads costs more MMA time than the 64-column overlap.
-    static constexpr bool SINGLE = (OUTQ == 0) && (KIND == G_NVFP4);
-    static constexpr int ACC1_COL = SINGLE ? 0 : (KIND == G_NVFP4) ? 160 : 192;
-    static constexpr int SF_COL0 = SINGLE ? 256 : ACC1_COL + 256;
+    // TMEM columns: two accumulators overlapping by OVL columns, the shared columns drained
+    // first.  NVFP4 stages carry 4 scale atoms (48 columns), so its accumulators overlap by
+    // 96 to leave room for two scale buffers; the others overlap by 64, which the holders
+    // drain as their first 64-column pair.  A 96-column overlap spans both pairs: with
+    // plain bf16 output (HOLD_ALL) its holders copy all four chunks to registers before
+    // converting any, so the overlap is released after the copy rather than after a pair
+    // has been written; the fused epilogues need those registers for their arithmetic.
+    static constexpr int ACC1_COL = (KIND == G_NVFP4) ? 160 : 192;
+    static constexpr int SF_COL0 = ACC1_COL + 256;
     static constexpr int OVL = 256 - ACC1_COL;
+    static constexpr bool HOLD_ALL = (OUTQ == 0) && (OVL > 64);
     static constexpr int SFA_COLS = 4 * ATOMS;        // A: 4 columns per atom
     static constexpr int SF_COLS = SFA_COLS + 8 * ATOMS;  // B: 8 columns per atom
     static constexpr int TB = ((GEMM_TMEM_COLS - SF_COL0) / SF_COLS) >= 4 ? 4 : ((GEMM_TMEM_COLS - SF_COL0) / SF_COLS);
@@ -453,7 +450,7 @@ struct Gemm2Cfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert((STAGES * (A_BYTES + B_BYTES)) % 1024 == 0, "staging tiles 1024-byte aligned");
     static_assert(TB >= 2 && SF_COL0 + TB * SF_COLS <= GEMM_TMEM_COLS, "TMEM budget");
-    static_assert(SINGLE || OVL == 64 || OVL == 96, "epilogue overlap handling");
+    static_assert(OVL == 64 || OVL == 96, "epilogue overlap handling");
 };
 
 // Pair-kernel epilogue: pack one row's 64 columns and write them, as 128 bytes, into row
@@ -642,7 +639,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             mbar_init(&tmem_full[b], 1);
             mbar_init(&acc_free[b], 16);
         }
-        mbar_init(ovl_free, C::SINGLE ? 16 : 8);
+        mbar_init(ovl_free, 8);
         mbar_init(mma_done, 1);
         *abort = 0;
         fence_mbar_init();
@@ -691,7 +688,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         const int q = warp & 3;
         const int h = ew >> 2;
         uint8_t* stile = sEpi + ew * 4096;
-        // acc: the 64-column pair being written; acc2: the second pair of a one-go drain
+        // acc: the 64-column pair being written; acc2: an overlap holder's second pair (HOLD_ALL)
         uint32_t acc[2][32], acc2[2][32];
         float gs = 1.0f;
         if (KIND == G_NVFP4) gs = __fmul_rn(*p.g_a, *p.g_w);
@@ -763,13 +760,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                             make_float4(__uint_as_float(a[c][j]), __uint_as_float(a[c][j + 1]),
                                         __uint_as_float(a[c][j + 2]), __uint_as_float(a[c][j + 3]));
             };
-            if constexpr (C::SINGLE) {
-                // one accumulator: the warp's 128 columns go to registers at once and the
-                // accumulator is handed back before any of them is converted
-                tmem_ld_32x32b_x32(taddr, acc[0]);
-                tmem_ld_32x32b_x32(taddr + 32, acc[1]);
-                tmem_ld_32x32b_x32(taddr + 64, acc2[0]);
-                tmem_ld_32x32b_x32(taddr + 96, acc2[1]);
+            // the OVL columns shared by both accumulators are the last OVL tile columns of
+            // accumulator 0 (half 1) or the first OVL of accumulator 1 (half 0): their holders
+            // drain them first and release them -- after the first chunk pair when OVL = 64,
+            // after copying all four chunks with HOLD_ALL, else after both pairs
+            const bool holds_overlap = (h == (b == 0 ? 1 : 0));
+            const int first = holds_overlap ? (b == 0 ? 2 : 0) : 0;
+            const int second = 2 - first;
+            tmem_ld_32x32b_x32(taddr + first * 32, acc[0]);
+            tmem_ld_32x32b_x32(taddr + (first + 1) * 32, acc[1]);
+            if (C::HOLD_ALL && holds_overlap) {
+                tmem_ld_32x32b_x32(taddr + second * 32, acc2[0]);
+                tmem_ld_32x32b_x32(taddr + (second + 1) * 32, acc2[1]);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
@@ -777,18 +779,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                     arrive_leader_relaxed(ovl_free, rank);
                     arrive_leader_relaxed(&acc_free[b], rank);
                 }
-                stage_store(acc, 0);
-                stage_store(acc2, 2);
+                stage_store(acc, first);
+                stage_store(acc2, second);
             } else {
-                // the OVL columns shared by both accumulators are the last OVL tile columns of
-                // accumulator 0 (half 1) or the first OVL of accumulator 1 (half 0): their holders
-                // drain them first and release them -- after the first chunk pair when OVL = 64,
-                // after both pairs when OVL = 96 (NVFP4)
-                const bool holds_overlap = (h == (b == 0 ? 1 : 0));
-                const int first = holds_overlap ? (b == 0 ? 2 : 0) : 0;
-                const int second = 2 - first;
-                tmem_ld_32x32b_x32(taddr + first * 32, acc[0]);
-                tmem_ld_32x32b_x32(taddr + (first + 1) * 32, acc[1]);
                 tmem_wait_ld();
                 if (holds_overlap && C::OVL <= 64) {
                     tc_fence_before();
@@ -1076,7 +1069,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 for (; ok && sc.get(tile, kb0, kb1); sc.step(kb0, kb1), ++tcount) {
                     const int b = tcount & 1;
                     // accumulator b drained (unit tcount-2) and the overlap of unit tcount-1 drained
-                    // (with one accumulator the "overlap" is all of it: every epilogue warp arrives)
                     bool got = mbar_wait(&acc_free[b], (((uint32_t)tcount >> 1) & 1u) ^ 1u, p.timeout_ns, abort);
                     if (got && tcount > 0) got = mbar_wait(ovl_free, (uint32_t)(tcount - 1) & 1u, p.timeout_ns, abort);
                     for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
