@@ -125,14 +125,33 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- inputs
-def make_inputs(rank: int):
+def make_inputs(rank: int, m: int | None = None, k: int | None = None, n: int | None = None):
+    """Rank r's batch: its own activations (weak scaling: every rank a different batch of the
+    same size), the shared weight and bias.  Sizes default to the workload's."""
     import synth
 
+    m, k, n = (M if m is None else m), (K if k is None else k), (N if n is None else n)
     s = synth.seeds_for(4, layer=1)
-    x = synth.activation(s["x"] + 7919 * rank, M, K, "lognormal", gain_seed=s["gain"])
-    w = synth.weight(s["w"], N, K)
-    b = synth.bias(s["bias"], N)
+    x = synth.activation(s["x"] + 7919 * rank, m, k, "lognormal", gain_seed=s["gain"])
+    w = synth.weight(s["w"], n, k)
+    b = synth.bias(s["bias"], n)
     return x, w, b
+
+
+def max_over_ranks(x: float, dist=None, device="cuda") -> float:
+    """The largest x over all ranks: a job's time is its slowest rank's."""
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_tflops(flop_per_rank_step: float, world: int, steps: int, slowest_ms: float) -> float:
+    """Whole-job throughput: the work of all ranks over the slowest rank's timed region."""
+    return flop_per_rank_step * world * steps / (slowest_ms / 1e3) / 1e12
 
 
 def to_dev(bits, torch, dt):
@@ -323,12 +342,9 @@ def native_arm(args):
     total_ms = t_start.elapsed_time(t_end)
     q_ms = [e[0].elapsed_time(e[1]) for e in evs]
     g_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    if dist:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = t.item()
+    total_ms = max_over_ranks(total_ms, dist)
     ms_per_step = total_ms / args.steps
-    value = FLOP_PER_STEP * world * args.steps / (total_ms / 1e3) / 1e12
+    value = job_tflops(FLOP_PER_STEP, world, args.steps, total_ms)
 
     # ---- end to end through the public API, host buffers (pinned), copies inside the timing
     # (fb.linear_host: row chunks through fp4_linear with both copy directions overlapped)
@@ -351,11 +367,8 @@ def native_arm(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
-    e2e_value = FLOP_PER_STEP * world * args.e2e_steps / (e2e_ms / 1e3) / 1e12
+    e2e_ms = max_over_ranks(e2e_ms, dist)
+    e2e_value = job_tflops(FLOP_PER_STEP, world, args.e2e_steps, e2e_ms)
 
     # ---- roofline of the dominant kernel (the GEMM), live CUDA-event durations
     pk, pk_kind = peaks()

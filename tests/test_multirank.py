@@ -1,0 +1,91 @@
+"""Multi-rank host logic of bench.py, on CPU with world-size-2 gloo ranks.
+
+The data-parallel path shards by batch: every rank quantizes and multiplies its own
+activations against the shared weight, with no collective on the data path.  The only
+cross-rank steps are the barriers around the timed region and the maximum over ranks of
+its duration; the job's throughput is the work of all ranks over that maximum.
+"""
+import argparse
+import datetime
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, times, out_q):
+    import torch.distributed as dist
+
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import bench
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        dist.barrier()
+        slowest = bench.max_over_ranks(times[rank], dist, "cpu")
+        value = bench.job_tflops(1e12, world, 10, slowest)
+        dist.barrier()
+        out_q.put((rank, slowest, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_slowest_time_and_count_all_work():
+    import torch.multiprocessing as mp
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    times = [3.0, 5.0]  # ms of each rank's timed region
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, times, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(60)
+    assert [p.exitcode for p in procs] == [0, 0]
+    for rank, slowest, value in res:
+        assert slowest == 5.0
+        # 1 TFLOP per rank-step, 2 ranks, 10 steps, over the slowest rank's 5 ms
+        assert value == pytest.approx(4000.0)
+
+
+def test_single_rank_needs_no_process_group():
+    import bench
+
+    assert bench.max_over_ranks(2.5) == 2.5
+    assert bench.job_tflops(2.0e12, 1, 4, 8.0) == pytest.approx(1000.0)
+
+
+def test_each_rank_gets_its_own_batch_and_the_shared_weight():
+    import bench
+
+    x0, w0, b0 = bench.make_inputs(0, 8, 128, 16)
+    x1, w1, b1 = bench.make_inputs(1, 8, 128, 16)
+    x0_again, _, _ = bench.make_inputs(0, 8, 128, 16)
+    assert x0.shape == (8, 128) and w0.shape == (16, 128) and b0.shape == (16,)
+    assert not np.array_equal(x0, x1)
+    assert np.array_equal(x0, x0_again)
+    assert np.array_equal(w0, w1) and np.array_equal(b0, b1)
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    import bench
+
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    args = argparse.Namespace(gpus=2, steps=1, warmup=0, impl="reference")
+    assert bench.reference_arm(args) == 0
+    assert capsys.readouterr().out == ""
