@@ -688,6 +688,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         const int q = warp & 3;
         const int h = ew >> 2;
         uint8_t* stile = sEpi + ew * 4096;
+        // Y is streamed out (2 GB at the FFN shape): evict-first lines drain to DRAM during
+        // the GEMM instead of being written back while the next kernel streams its input
+        const uint64_t pol_y = policy_evict_first();
         // acc: the 64-column pair being written; acc2: an overlap holder's second pair (HOLD_ALL)
         uint32_t acc[2][32], acc2[2][32];
         float gs = 1.0f;
@@ -741,7 +744,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0 && row0 < p.M) {
-                    tma_store_2d(&tmY, stile, col0 + chunk * 32, row0);
+                    tma_store_2d_hint(&tmY, stile, col0 + chunk * 32, row0, pol_y);
                     bulk_commit_group();
                 }
             };

@@ -148,6 +148,12 @@ FP4_DEV void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y)
                  "r"(smem_u32(src)), "r"(x), "r"(y)
                  : "memory");
 }
+// Same, with an L2 cache policy for the written lines (e.g. evict_first for a streamed output).
+FP4_DEV void tma_store_2d_hint(const CUtensorMap* map, const void* src, int x, int y, uint64_t policy) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(map),
+                 "r"(smem_u32(src)), "r"(x), "r"(y), "l"(policy)
+                 : "memory");
+}
 FP4_DEV void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 FP4_DEV void bulk_wait_group_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 FP4_DEV void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
