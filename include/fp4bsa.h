@@ -94,7 +94,8 @@ size_t w4a8_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank);
 
 /* Per-tensor amax: *amax_out (device fp32) = max |x_i| over n bf16 values (device).
  * Used for the NVFP4 weight global and for calibrating the static activation global
- * (NVFP4 card: "calibrated static global scales").  The result is order-independent. */
+ * (NVFP4 card, Model Details: the activation globals are static, set by calibration).
+ * The result is order-independent. */
 fp4_status_t fp4_tensor_amax(const void* x_bf16, int64_t n, float* amax_out, void* stream);
 
 /* Offline weight pre-pack (MXFP4 / NVFP4 cards: weights stored as packed E2M1 with
@@ -119,9 +120,9 @@ fp4_status_t fp4_quantize_act(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int6
 
 /* ----------------------------------------------------------------- GEMM */
 
-/* Block-scaled FP4 x FP4 GEMM with fused epilogue on pre-quantized activations
- * (MXFP4 card: "FlashInferMxFp4LinearKernel + cuDNN blockScaleMatMul (W4A4)"; NVFP4
- * card: "CUTLASS NVFP4 GEMMs, not an activation quantize-dequantize emulation path"):
+/* Block-scaled FP4 x FP4 GEMM with fused epilogue on pre-quantized activations (the
+ * MXFP4 card runs its W4A4 linears on a block-scaled FP4 matmul; the NVFP4 card, How to
+ * Use, stresses that real FP4 GEMMs run, not a quantize-dequantize emulation):
  *   y[m,n] = bf16_rn( gs * sum_k deq(a[m,k]) deq(w[n,k]) + bias[n] )
  * with gs = g_a * g_w for NVFP4 and 1 for MXFP4; the sum accumulates in fp32.
  *   a_codes, a_sf       (device) quantized activations as fp4_quantize_act writes them
@@ -257,7 +258,7 @@ fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N
 
 /* ----------------------------------------------------------------- W4A4 SVDQuant */
 
-/* The W4A8 README's experimental W4A4 variant ("Experimental W4A4 (MXFP4 activations)"):
+/* The W4A8 README's experimental W4A4 variant (Quick start: MXFP4 activations):
  * the same calibrated factors (MXFP4 residual R, rank-32 L1 / L2), with the activations
  * quantized to MXFP4 instead of MXFP8; the low-rank branch still reads the unquantized
  * input.  y = bf16_rn( sum_k deq4(x) deq4(r) + u L2 + bias ). */

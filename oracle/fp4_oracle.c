@@ -62,8 +62,8 @@
  * Element and scale codecs
  * ---------------------------------------------------------------------------------- */
 
-/* The eight E2M1 magnitudes: 1 sign, 2 exponent, 1 mantissa bit (MXFP4 page,
- * "packed FP4 E2M1"). Index = the 3 low bits of the code. */
+/* The eight E2M1 magnitudes: 1 sign, 2 exponent, 1 mantissa bit (MXFP4 page: weights
+ * stored as packed 4-bit E2M1 codes). Index = the 3 low bits of the code. */
 static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
 
 double orc_e2m1_decode(uint8_t code) {
