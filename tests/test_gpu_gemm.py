@@ -449,3 +449,42 @@ def test_linear_host_chunks(fb, orc, fmt):
     rows = np.arange(M)
     Y, S = _oracle(orc, fmt, x, w, b, rows, g_a)
     H.check_linear(y_host, Y, S, rows, f"linear_host fmt={fmt}")
+
+
+# ------------------------------------------------------------------ several tiles per CTA pair
+# 9 x 17 = 153 output tiles of 256 x 256 for 74 pairs: every pair runs two or three tiles, so
+# both accumulators, the hand-over of their shared columns between consecutive tiles and (NVFP4
+# with bf16 output) the overlap holders' copy-all release are exercised on every element; M and
+# N both end in a ragged tile.
+MANY = (2300, 512, 4224)
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+def test_pair_kernel_many_tiles_all_elements(fb, orc, fmt):
+    M, K, N = MANY
+    x = synth.activation(90 * M + K, M, K, "lognormal")
+    w = synth.weight(91 * N + K, N, K)
+    b = synth.bias(N + 13, N)
+    g_a = orc.nv_global(orc.tensor_amax(x)) if fmt == NV else None
+    with _gemm_ctas(fb, 2):
+        y = _run_linear(fb, fmt, x, w, b, g_a)
+    rows = np.arange(M)
+    Y, S = _oracle(orc, fmt, x, w, b, rows, g_a)
+    H.check_linear(y, Y, S, rows, f"many tiles fmt={fmt}")
+
+
+def test_w4a8_many_tiles_all_elements(fb, orc):
+    _w4a8_check(fb, orc, *MANY, seed=7100)
+
+
+def test_w4a4_many_tiles_all_elements(fb, orc):
+    _w4a4_check(fb, orc, *MANY, seed=8100)
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+def test_linear_gelu_quant_many_tiles(fb, orc, fmt):
+    M, K, N = MANY
+    x = synth.activation(92 * M + K, M, K, "lognormal")
+    w = synth.weight(93 * N + K, N, K)
+    b = synth.bias(N + 17, N)
+    _gelu_linear_case(fb, orc, fmt, M, K, N, x, w, b, np.arange(M), f"gelu many tiles fmt={fmt}")
