@@ -290,22 +290,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                                 tsfb + a * 8 + rb * 4,
                                 smem_desc(smem_u32(sSFB + s * C::SFB_BYTES + (rb * C::ATOMS + a) * 512), 0, 128, 0));
                     }
-                    const uint32_t a_base = smem_u32(sA + s * C::A_BYTES);
-                    const uint32_t b_base = smem_u32(sB + s * C::B_BYTES);
-                    for (int k = 0; k < n_mma; ++k) {
+                    // the stage's MMAs, unrolled with every operand a constant offset (the issuing
+                    // thread's own latency sets the MMA rate); MMA k reads 32 bytes at k * 32 of
+                    // every 128-byte row, and a last stage of K % 256 = 128 holds two MMAs
+                    const uint64_t adesc = smem_desc(smem_u32(sA + s * C::A_BYTES), 0, 1024, 2);
+                    const uint64_t bdesc = smem_desc(smem_u32(sB + s * C::B_BYTES), 0, 1024, 2);
+                    const uint32_t acc0 = kb > 0 ? 1u : 0u;
+                    static_assert(C::BK / C::MMA_K == 4, "four MMAs per stage");
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        if (k >= n_mma) break;
                         // scale-factor selection: which atom (TMEM column group) and which byte
                         int atom, sf_id;
                         sf_select<KIND>(k, atom, sf_id);
                         const uint32_t idesc = C::IDESC | ((uint32_t)sf_id << 29) | ((uint32_t)sf_id << 4);
-                        const uint64_t adesc = smem_desc(a_base + k * 32, 0, 1024, 2);
-                        const uint64_t bdesc = smem_desc(b_base + k * 32, 0, 1024, 2);
-                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                        const uint64_t ad = adesc + (uint64_t)(k * 2), bd = bdesc + (uint64_t)(k * 2);
+                        const uint32_t acc = k > 0 ? 1u : acc0;
                         if (KIND == G_MXFP4)
-                            mma_mxf4nvf4_block32(tmem_base, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                            mma_mxf4nvf4_block32(tmem_base, ad, bd, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
                         else if (KIND == G_NVFP4)
-                            mma_mxf4nvf4_block16(tmem_base, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                            mma_mxf4nvf4_block16(tmem_base, ad, bd, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
                         else
-                            mma_mxf8f6f4_block32(tmem_base, adesc, bdesc, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
+                            mma_mxf8f6f4_block32(tmem_base, ad, bd, idesc, acc, tsfa + atom * 4, tsfb + atom * 8);
                     }
                     tc_commit(&empty[s]);
                     issued = true;
