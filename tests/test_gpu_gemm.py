@@ -488,3 +488,44 @@ def test_linear_gelu_quant_many_tiles(fb, orc, fmt):
     w = synth.weight(93 * N + K, N, K)
     b = synth.bias(N + 17, N)
     _gelu_linear_case(fb, orc, fmt, M, K, N, x, w, b, np.arange(M), f"gelu many tiles fmt={fmt}")
+
+
+# ------------------------------------------------------------------ CUDA-graph capture
+# The library allocates nothing, synchronizes nothing and copies nothing between host and
+# device inside a call, so a quantized linear can be captured once and replayed (the way
+# launch-bound text-token calls amortize their fixed cost).  The captured graph holds the
+# quantize kernel and the GEMM (with its programmatic launch edge); each replay reads
+# whatever the input buffer holds at that moment.
+@pytest.mark.parametrize("fmt", [MX, NV])
+def test_linear_replays_in_a_cuda_graph(fb, orc, fmt):
+    import torch
+
+    M, K, N = 512, 1024, 768
+    w = synth.weight(95 * N + K, N, K)
+    b = synth.bias(N + 19, N)
+    xs = [synth.activation(96 * M + K + i, M, K, "lognormal") for i in range(2)]
+    g_a = orc.nv_global(max(orc.tensor_amax(xi) for xi in xs)) if fmt == NV else None
+    pw = fb.pack_weight(H.dev_bf16(w), fmt)
+    bias = H.dev_f16(b)
+    ga = H.dev_f32([g_a]) if fmt == NV else None
+    x = H.dev_bf16(xs[0])
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(fb.fp4_linear_workspace_bytes(fmt, M, K, N), dtype=torch.uint8, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fb.linear(x, pw, bias, ga, y, ws)  # eager first call: one-time device setup
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        fb.linear(x, pw, bias, ga, y, ws)
+    rows = np.arange(M)
+    for i, xi in enumerate(xs):
+        x.copy_(H.dev_bf16(xi))
+        y.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        st = fb.fp4_sync_status()
+        assert st == 0, fb.fp4_status_string(st)
+        Y, S = _oracle(orc, fmt, xi, w, b, rows, g_a)
+        H.check_linear(y, Y, S, rows, f"graph replay {i} fmt={fmt}")
