@@ -111,6 +111,9 @@ fp4_status_t device_state(DeviceState** out) {
                 for (const void* k : pair_kernels)
                     if (!launch_regs_are(k, R)) return FP4_ERR_ARCH;
             }
+            if (cudaFuncSetAttribute(lowrank_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LR_SMEM_BYTES) !=
+                cudaSuccess)
+                return FP4_ERR_CUDA;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.quant_occ[Q_MXFP4], quant_kernel<Q_MXFP4>,
                                                               QUANT_THREADS, 0) != cudaSuccess ||
                 cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.quant_occ[Q_NVFP4], quant_kernel<Q_NVFP4>,
@@ -276,6 +279,38 @@ int sk_seg_max(int64_t tiles, int64_t num_kb, int P) {
 }
 // K blocks of the 2-CTA MXFP4 / NVFP4 kernel (256 K per stage, the last may be half)
 int64_t sk_num_kb(int64_t K) { return (K + 255) / 256; }
+
+// Low-rank down-projection u = x L1 (W4A8 / W4A4 SVDQuant): with few 128-row blocks (the
+// 4290-token W4A8 shape has 34) K is split over up to 8 blocks per row block, whose fp32
+// partial sums a second kernel adds in split order.  Only the full linears, which own a
+// workspace, split; the split is a function of (M, K) alone, so the workspace size is too.
+int lr_split(int64_t M, int64_t K) {
+    const int64_t blocks = (M + LR_ROWS - 1) / LR_ROWS, nkc = K / LR_KC;
+    if (blocks >= 64) return 1;
+    for (int sp : {8, 4, 2})
+        if (nkc % sp == 0 && nkc / sp >= 2) return sp;
+    return 1;
+}
+size_t lr_partial_bytes(int64_t M, int64_t K) {
+    const int sp = lr_split(M, K);
+    const int64_t mpad = (M + LR_ROWS - 1) / LR_ROWS * LR_ROWS;
+    return sp > 1 ? align256((size_t)sp * mpad * 32 * sizeof(float)) : 0;
+}
+void launch_lowrank(const void* x_bf16, const void* l1_bf16, int64_t M, int64_t K, void* u_pair, float* partial,
+                    cudaStream_t st) {
+    const int blocks = (int)((M + LR_ROWS - 1) / LR_ROWS);
+    const auto x = static_cast<const __nv_bfloat16*>(x_bf16);
+    const auto l1 = static_cast<const __nv_bfloat16*>(l1_bf16);
+    const auto u = static_cast<__nv_bfloat16*>(u_pair);
+    const int sp = partial ? lr_split(M, K) : 1;
+    if (sp == 1) {
+        lowrank_down_kernel<<<blocks, LR_THREADS, LR_SMEM_BYTES, st>>>(x, l1, (int)M, (int)K, u, nullptr, 0);
+        return;
+    }
+    lowrank_down_kernel<<<dim3(blocks, sp), LR_THREADS, LR_SMEM_BYTES, st>>>(x, l1, (int)M, (int)K, u, partial,
+                                                                           (int)(K / LR_KC / sp));
+    lowrank_reduce_kernel<<<(int)((M * 32 + 255) / 256), 256, 0, st>>>(partial, (int)M, blocks * LR_ROWS, sp, u);
+}
 // Every pair's share must hold at least one K block (tiles * K blocks >= pairs): a pair
 // with an empty share would be counted among a tile's segments without ever arriving.
 // Only on request (hook): measured on B200, the small problems it targets are bound by
@@ -358,15 +393,16 @@ size_t fp4_linear_workspace_bytes(fp4_fmt_t fmt, int64_t M, int64_t K, int64_t N
 
 size_t w4a8_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank) {
     if (rank != 32 || check_shape(M, K, N) != FP4_OK) return 0;
-    // E4M3 codes, E8M0 scales, u pair (M x 2 rank bf16)
-    return align256((size_t)M * K) + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K)) + align256((size_t)M * rank * 4);
+    // E4M3 codes, E8M0 scales, u pair (M x 2 rank bf16), split-K partials of u
+    return align256((size_t)M * K) + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K)) + align256((size_t)M * rank * 4) +
+           lr_partial_bytes(M, K);
 }
 
 size_t w4a4_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank) {
     if (rank != 32 || check_shape(M, K, N) != FP4_OK) return 0;
-    // MXFP4 codes, E8M0 scales, u pair (M x 2 rank bf16)
+    // MXFP4 codes, E8M0 scales, u pair (M x 2 rank bf16), split-K partials of u
     return align256(fp4_codes_bytes(FP4_FMT_MXFP4, M, K)) + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K)) +
-           align256((size_t)M * rank * 4);
+           align256((size_t)M * rank * 4) + lr_partial_bytes(M, K);
 }
 
 fp4_status_t fp4_tensor_amax(const void* x_bf16, int64_t n, float* amax_out, void* stream) {
@@ -581,8 +617,10 @@ fp4_status_t fp4_linear_gelu_quant(fp4_fmt_t fmt, const void* x_bf16, int64_t M,
                                h_codes, h_sf, stream);
 }
 
-fp4_status_t w4a8_quantize_act(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16, int rank,
-                               uint8_t* x_e4m3, uint8_t* x_sf, void* u_pair, void* stream) {
+}  // extern "C"
+namespace {
+fp4_status_t w4a8_quantize_impl(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16, int rank,
+                               uint8_t* x_e4m3, uint8_t* x_sf, void* u_pair, float* partial, void* stream) {
     if (!x_bf16 || !l1_bf16 || !x_e4m3 || !x_sf || !u_pair || rank != 32) return FP4_ERR_INVALID_ARG;
     fp4_status_t s = check_shape(M, K, 128);
     if (s != FP4_OK) return s;
@@ -592,11 +630,14 @@ fp4_status_t w4a8_quantize_act(const void* x_bf16, int64_t M, int64_t K, const v
     if ((s = device_state(&ds)) != FP4_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((s = launch_quant(ds, Q_MXFP8, x_bf16, M, K, nullptr, x_e4m3, x_sf, st)) != FP4_OK) return s;
-    const int blocks = (int)((M + LR_ROWS - 1) / LR_ROWS);
-    lowrank_down_kernel<<<blocks, LR_THREADS, 0, st>>>(static_cast<const __nv_bfloat16*>(x_bf16),
-                                                       static_cast<const __nv_bfloat16*>(l1_bf16), (int)M, (int)K,
-                                                       static_cast<__nv_bfloat16*>(u_pair));
+    launch_lowrank(x_bf16, l1_bf16, M, K, u_pair, partial, st);
     return launched();
+}
+}  // namespace
+extern "C" {
+fp4_status_t w4a8_quantize_act(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16, int rank,
+                               uint8_t* x_e4m3, uint8_t* x_sf, void* u_pair, void* stream) {
+    return w4a8_quantize_impl(x_bf16, M, K, l1_bf16, rank, x_e4m3, x_sf, u_pair, nullptr, stream);
 }
 
 fp4_status_t w4a8_pack_lowrank_up(const void* l2_bf16, int64_t N, int rank, void* l2t_bf16, void* stream) {
@@ -657,12 +698,15 @@ fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N
     uint8_t* xe = static_cast<uint8_t*>(workspace);
     uint8_t* xs = xe + align256((size_t)M * K);
     uint8_t* u = xs + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K));
-    if ((s = w4a8_quantize_act(x_bf16, M, K, l1_bf16, rank, xe, xs, u, stream)) != FP4_OK) return s;
+    float* partial = lr_partial_bytes(M, K) ? reinterpret_cast<float*>(u + align256((size_t)M * rank * 4)) : nullptr;
+    if ((s = w4a8_quantize_impl(x_bf16, M, K, l1_bf16, rank, xe, xs, u, partial, stream)) != FP4_OK) return s;
     return w4a8_gemm(xe, xs, u, M, K, N, r_codes, r_sf, l2t_bf16, rank, bias_f16, y_bf16, stream);
 }
 
-fp4_status_t w4a4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16, int rank,
-                               uint8_t* x_codes, uint8_t* x_sf, void* u_pair, void* stream) {
+}  // extern "C"
+namespace {
+fp4_status_t w4a4_quantize_impl(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16, int rank,
+                               uint8_t* x_codes, uint8_t* x_sf, void* u_pair, float* partial, void* stream) {
     if (!x_bf16 || !l1_bf16 || !x_codes || !x_sf || !u_pair || rank != 32) return FP4_ERR_INVALID_ARG;
     fp4_status_t s = check_shape(M, K, 128);
     if (s != FP4_OK) return s;
@@ -672,11 +716,14 @@ fp4_status_t w4a4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const v
     if ((s = device_state(&ds)) != FP4_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((s = launch_quant(ds, Q_MXFP4, x_bf16, M, K, nullptr, x_codes, x_sf, st)) != FP4_OK) return s;
-    const int blocks = (int)((M + LR_ROWS - 1) / LR_ROWS);
-    lowrank_down_kernel<<<blocks, LR_THREADS, 0, st>>>(static_cast<const __nv_bfloat16*>(x_bf16),
-                                                       static_cast<const __nv_bfloat16*>(l1_bf16), (int)M, (int)K,
-                                                       static_cast<__nv_bfloat16*>(u_pair));
+    launch_lowrank(x_bf16, l1_bf16, M, K, u_pair, partial, st);
     return launched();
+}
+}  // namespace
+extern "C" {
+fp4_status_t w4a4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const void* l1_bf16, int rank,
+                               uint8_t* x_codes, uint8_t* x_sf, void* u_pair, void* stream) {
+    return w4a4_quantize_impl(x_bf16, M, K, l1_bf16, rank, x_codes, x_sf, u_pair, nullptr, stream);
 }
 
 fp4_status_t w4a4_gemm(const uint8_t* x_codes, const uint8_t* x_sf, const void* u_pair, int64_t M, int64_t K,
@@ -721,7 +768,8 @@ fp4_status_t w4a4_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N
     uint8_t* xc = static_cast<uint8_t*>(workspace);
     uint8_t* xs = xc + align256(fp4_codes_bytes(FP4_FMT_MXFP4, M, K));
     uint8_t* u = xs + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K));
-    if ((s = w4a4_quantize_act(x_bf16, M, K, l1_bf16, rank, xc, xs, u, stream)) != FP4_OK) return s;
+    float* partial = lr_partial_bytes(M, K) ? reinterpret_cast<float*>(u + align256((size_t)M * rank * 4)) : nullptr;
+    if ((s = w4a4_quantize_impl(x_bf16, M, K, l1_bf16, rank, xc, xs, u, partial, stream)) != FP4_OK) return s;
     return w4a4_gemm(xc, xs, u, M, K, N, r_codes, r_sf, l2t_bf16, rank, bias_f16, y_bf16, stream);
 }
 

@@ -208,11 +208,14 @@ __global__ void nv_global_kernel(float* g) {
 // is ample.  The result is stored as a bf16 pair per value, hi = bf16(u), lo = bf16(u - hi)
 // (u_pair[m][r] = hi, u_pair[m][32 + r] = lo), so the GEMM can add u L2 on the tensor core
 // as u_hi L2 + u_lo L2 with |u - hi - lo| <= 2^-18 |u|.
-// Block: 256 threads = 8 warps x 16 rows = 128 rows, all 32 ranks; K in 64-element chunks,
-// double-buffered with cp.async.
-constexpr int LR_ROWS = 128, LR_THREADS = 256, LR_KC = 64;
+// Block: 256 threads = 8 warps x 16 rows = 128 rows, all 32 ranks; K in 64-element chunks
+// through a ring of LR_STAGES cp.async stages.  At the W4A8 shape (4290 rows) only 34 blocks
+// exist, each streaming 786 KB of X, so bytes in flight per SM set the speed: with two
+// stages the kernel took 33 us (about 32 GB/s per SM), hence a deep ring.
+constexpr int LR_ROWS = 128, LR_THREADS = 256, LR_KC = 64, LR_STAGES = 6;
 constexpr int LR_XP = LR_KC + 8;  // padded X row (elements): conflict-free ldmatrix
 constexpr int LR_LP = 32 + 8;     // padded L1 row
+constexpr int LR_SMEM_BYTES = LR_STAGES * (LR_ROWS * LR_XP + LR_KC * LR_LP) * 2;  // dynamic shared memory
 
 FP4_DEV void cp_async16(void* dst, const void* src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
@@ -223,14 +226,21 @@ FP4_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memo
 template <int N>
 FP4_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// Split K (partial != nullptr): block (i, j) covers chunks [j * kc_per_split, (j + 1) *
+// kc_per_split) of row block i and writes its fp32 sums to partial[j][m][r] (rows padded to
+// whole blocks); lowrank_reduce_kernel adds the splits in index order.  Otherwise the block
+// covers all of K and writes the pair itself.
 __global__ void __launch_bounds__(LR_THREADS) lowrank_down_kernel(const __nv_bfloat16* __restrict__ x,
                                                                   const __nv_bfloat16* __restrict__ l1, int M,
-                                                                  int K, __nv_bfloat16* __restrict__ u_pair) {
-    __shared__ __align__(16) __nv_bfloat16 xs[2][LR_ROWS][LR_XP];
-    __shared__ __align__(16) __nv_bfloat16 ls[2][LR_KC][LR_LP];
+                                                                  int K, __nv_bfloat16* __restrict__ u_pair,
+                                                                  float* __restrict__ partial, int kc_per_split) {
+    extern __shared__ __align__(16) uint8_t lr_smem[];
+    auto xs = reinterpret_cast<__nv_bfloat16(*)[LR_ROWS][LR_XP]>(lr_smem);
+    auto ls = reinterpret_cast<__nv_bfloat16(*)[LR_KC][LR_LP]>(lr_smem + LR_STAGES * LR_ROWS * LR_XP * 2);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int m0 = blockIdx.x * LR_ROWS;
-    const int nkc = K / LR_KC;
+    const int nkc = partial ? kc_per_split : K / LR_KC;
+    const int kc0 = partial ? (int)blockIdx.y * kc_per_split : 0;
 
     auto load = [&](int kc, int st) {
 #pragma unroll
@@ -238,12 +248,12 @@ __global__ void __launch_bounds__(LR_THREADS) lowrank_down_kernel(const __nv_bfl
             const int idx = tid + i * LR_THREADS;
             const int row = idx >> 3, c = idx & 7;
             const bool ok = m0 + row < M;
-            const __nv_bfloat16* src = ok ? x + (size_t)(m0 + row) * K + kc * LR_KC + c * 8 : x;
+            const __nv_bfloat16* src = ok ? x + (size_t)(m0 + row) * K + (kc0 + kc) * LR_KC + c * 8 : x;
             cp_async16(&xs[st][row][c * 8], src, ok);
         }
         {  // L1: 64 rows x 4 pieces of 16 bytes
             const int row = tid >> 2, c = tid & 3;
-            cp_async16(&ls[st][row][c * 8], l1 + (size_t)(kc * LR_KC + row) * 32 + c * 8, true);
+            cp_async16(&ls[st][row][c * 8], l1 + (size_t)((kc0 + kc) * LR_KC + row) * 32 + c * 8, true);
         }
         cp_async_commit();
     };
@@ -254,16 +264,26 @@ __global__ void __launch_bounds__(LR_THREADS) lowrank_down_kernel(const __nv_bfl
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[j][e] = 0.0f;
 
-    load(0, 0);
+    // prologue: chunks 0 .. LR_STAGES - 2 in flight (one commit group per chunk; empty groups
+    // past the end keep the count uniform, so "chunk kc landed" is "at most LR_STAGES - 2
+    // groups pending")
+#pragma unroll
+    for (int c = 0; c < LR_STAGES - 1; ++c) {
+        if (c < nkc)
+            load(c, c);
+        else
+            cp_async_commit();
+    }
     for (int kc = 0; kc < nkc; ++kc) {
-        const int st = kc & 1;
-        if (kc + 1 < nkc) {
-            load(kc + 1, st ^ 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
+        const int st = kc % LR_STAGES;
+        cp_async_wait<LR_STAGES - 2>();
         __syncthreads();
+        // refill the stage chunk kc - 1 used: every thread is past it (the barrier above)
+        const int nk = kc + LR_STAGES - 1;
+        if (nk < nkc)
+            load(nk, nk % LR_STAGES);
+        else
+            cp_async_commit();
 #pragma unroll
         for (int ks = 0; ks < LR_KC / 16; ++ks) {
             uint32_t a[4];
@@ -289,10 +309,22 @@ __global__ void __launch_bounds__(LR_THREADS) lowrank_down_kernel(const __nv_bfl
                 }
             }
         }
-        __syncthreads();
     }
     // accumulator fragment: acc[j][0..1] -> row lane/4, acc[j][2..3] -> row lane/4 + 8,
     // columns 8j + 2(lane%4) + {0, 1}
+    if (partial) {
+        const size_t mpad = (size_t)gridDim.x * LR_ROWS;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int m = m0 + warp * 16 + (lane >> 2) + half * 8;
+            float* row = partial + ((size_t)blockIdx.y * mpad + m) * 32;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<float2*>(row + j * 8 + 2 * (lane & 3)) =
+                    make_float2(acc[j][2 * half], acc[j][2 * half + 1]);
+        }
+        return;
+    }
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         const int m = m0 + warp * 16 + (lane >> 2) + half * 8;
@@ -309,6 +341,21 @@ __global__ void __launch_bounds__(LR_THREADS) lowrank_down_kernel(const __nv_bfl
             *reinterpret_cast<__nv_bfloat162*>(row + 32 + c) = __halves2bfloat162(l0, l1v);
         }
     }
+}
+
+// u[m][r] = the splits' partial sums added in split order (a fixed order: the result does not
+// depend on scheduling), stored as the bf16 pair hi, lo like lowrank_down_kernel.
+__global__ void __launch_bounds__(256) lowrank_reduce_kernel(const float* __restrict__ partial, int M, int mpad,
+                                                             int splits, __nv_bfloat16* __restrict__ u_pair) {
+    const int i = blockIdx.x * 256 + threadIdx.x;  // (row, rank)
+    if (i >= M * 32) return;
+    float u = partial[i];
+    for (int j = 1; j < splits; ++j) u = __fadd_rn(u, partial[(size_t)j * mpad * 32 + i]);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(u);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(u - __bfloat162float(hi));
+    const int m = i >> 5, r = i & 31;
+    u_pair[(size_t)m * 64 + r] = hi;
+    u_pair[(size_t)m * 64 + 32 + r] = lo;
 }
 
 // W4A8: L2 [32, N] bf16 (rank-major) -> packed L2 [N, 32] bf16, the K-major operand of the

@@ -86,8 +86,9 @@ size_t fp4_sf_bytes(fp4_fmt_t fmt, int64_t rows, int64_t K);
  * 256-byte aligned.  0 on invalid arguments. */
 size_t fp4_linear_workspace_bytes(fp4_fmt_t fmt, int64_t M, int64_t K, int64_t N);
 
-/* Workspace w4a8_svd_linear needs: MXFP8 elements [M,K], their scales, and the fp32
- * low-rank projection u = x L1 [M, rank], each 256-byte aligned. */
+/* Workspace w4a8_svd_linear needs: MXFP8 elements [M,K], their scales, the low-rank
+ * projection u = x L1 as its bf16 pair [M, 2 rank] and, when x has fewer than 64 blocks of
+ * 128 rows, fp32 partial sums of u for a K-split projection; each 256-byte aligned. */
 size_t w4a8_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank);
 
 /* ----------------------------------------------------------------- quantization */
@@ -249,7 +250,8 @@ fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const void* u
                        const void* l2t_bf16, int rank, const void* bias_f16, void* y_bf16,
                        void* stream);
 
-/* The full W4A8 SVDQuant linear: w4a8_quantize_act into `workspace`, then w4a8_gemm.
+/* The full W4A8 SVDQuant linear: w4a8_quantize_act into `workspace` (with few rows, u = x L1
+ * split over K into the workspace's partial sums, added in a fixed order), then w4a8_gemm.
  * l2t_bf16 is the packed [N, rank] up-projection; rank must be 32. */
 fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N,
                              const uint8_t* r_codes, const uint8_t* r_sf, const void* l1_bf16,
@@ -263,7 +265,9 @@ fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N
  * quantized to MXFP4 instead of MXFP8; the low-rank branch still reads the unquantized
  * input.  y = bf16_rn( sum_k deq4(x) deq4(r) + u L2 + bias ). */
 
-/* Workspace for w4a4_svd_linear: MXFP4 codes + scales of x and the u pair (0 if invalid). */
+/* Workspace for w4a4_svd_linear: MXFP4 codes + scales of x, the u pair and, when x has
+ * fewer than 64 blocks of 128 rows, fp32 partial sums of u for a K-split u = x L1 (0 if
+ * invalid). */
 size_t w4a4_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank);
 
 /* Activation side: MXFP4 codes and scales of x (exactly fp4_quantize_act with

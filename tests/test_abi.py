@@ -45,10 +45,15 @@ def test_size_queries(fb):
     assert fb.fp4_linear_workspace_bytes(MX, 0, 5120, 13824) == 0
     assert fb.w4a8_workspace_bytes(4290, 3072, 14336, 32) > 4290 * 3072
     assert fb.w4a8_workspace_bytes(4290, 3072, 14336, 16) == 0
-    # W4A4 SVDQuant: MXFP4 codes + scales + the u pair, each 256-byte aligned
+    # W4A4 SVDQuant: MXFP4 codes + scales + the u pair, each 256-byte aligned, and (34 row
+    # blocks of 128 < 64: u = x L1 split 8 ways over K = 3072) fp32 partials of u for 8 splits
+    # of the 4352 padded rows
     a256 = lambda n: (n + 255) // 256 * 256
     assert fb.w4a4_workspace_bytes(4290, 3072, 14336, 32) == (
-        a256(4290 * 1536) + a256(fb.fp4_sf_bytes(MX, 4290, 3072)) + a256(4290 * 32 * 4))
+        a256(4290 * 1536) + a256(fb.fp4_sf_bytes(MX, 4290, 3072)) + a256(4290 * 32 * 4) + a256(8 * 4352 * 32 * 4))
+    # 591 row blocks: no split, no partials
+    assert fb.w4a4_workspace_bytes(75600, 5120, 13824, 32) == (
+        a256(75600 * 2560) + a256(fb.fp4_sf_bytes(MX, 75600, 5120)) + a256(75600 * 32 * 4))
     assert fb.w4a4_workspace_bytes(4290, 3072, 14336, 16) == 0
 
 
