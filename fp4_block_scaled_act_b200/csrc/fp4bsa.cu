@@ -343,10 +343,12 @@ fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CU
     fp4_status_t s;
     if ((s = encode_sf(&tsa, sfa, p.M, p.K, C::G, C::ATOMS)) != FP4_OK) return s;
     if ((s = encode_sf(&tsb, sfb, p.N, p.K, C::G, C::ATOMS)) != FP4_OK) return s;
-    // output: bf16 [M, N], stored by the epilogue in 32-row x 64-column boxes (128-byte swizzle)
+    // output: bf16 [M, N], stored by the epilogue in 32-row boxes of EPI_COLS columns (64:
+    // 128-byte swizzle, 32: 64-byte swizzle)
     CUtensorMap ty = ta;
     if (OUTQ == 0 && (s = encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.y, (uint64_t)p.N, (uint64_t)p.M,
-                                    (uint64_t)p.N * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
+                                    (uint64_t)p.N * 2, C::EPI_COLS, 32,
+                                    C::EPI_COLS == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B)) != FP4_OK)
         return s;
     const int tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
     // stream-K keeps every pair busy; whole tiles need no more pairs than tiles

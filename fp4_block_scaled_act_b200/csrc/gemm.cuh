@@ -40,6 +40,7 @@ constexpr int GEMM_STAGES = 4;
 constexpr int GEMM_ACC_COLS = 256;
 constexpr int GEMM_TMEM_COLS = 512;
 constexpr int STATUS_TIMEOUT = 7;
+constexpr int STATUS_LAYOUT = 5;  // FP4_ERR_ARCH: the device did not honour a shared-memory alignment
 
 template <int KIND>
 struct GemmCfg {
@@ -421,9 +422,18 @@ struct Gemm2Cfg {
     static constexpr int RSFA_BYTES = ATOMS * 512;    // raw atoms, this CTA's 128 A rows
     static constexpr int RSFB_BYTES = 2 * ATOMS * 512;  // raw atoms, all 256 B rows
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RSFA_BYTES + RSFB_BYTES;
-    static constexpr int STAGES = 5;
-    static constexpr int EPI_BYTES = 8 * 32 * 128;    // a 32 x 64 bf16 staging tile per epilogue warp
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + 512;
+    // Operand ring depth.  MXFP4 with 4 stages measured 13 % slower than with 5, and the
+    // same with 6 (interleaved, bit-identical output); W4A8 with 6 runs 1.5-3.5 % faster
+    // than with 5.  NVFP4's 6 KB of scale atoms per stage leave no room for a sixth.  With
+    // six stages the epilogue's per-warp Y staging tile is 32 x 32 bf16 (64-byte rows,
+    // 64-byte swizzle), else 32 x 64 (128-byte swizzle).
+    static constexpr int STAGES = (KIND == G_W4A8) ? 6 : 5;
+    static constexpr int EPI_COLS = (STAGES == 6) ? 32 : 64;
+    static constexpr int EPI_TILE = 32 * EPI_COLS * 2;
+    static constexpr int EPI_BYTES = 8 * EPI_TILE;
+    // the dynamic shared array is declared 1024-byte aligned (checked at run time), so the
+    // layout needs no alignment slack
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 512;
     static constexpr uint32_t AB_TX = A_BYTES + ((KIND == G_W4A8) ? B_BYTES / 2 : B_BYTES);
     static constexpr uint32_t SF_TX = RSFA_BYTES + RSFB_BYTES;
     // TMEM columns: two accumulators overlapping by OVL columns, the shared columns drained
@@ -476,6 +486,18 @@ FP4_DEV void epilogue_stage(const GemmParams& p, uint32_t (&acc)[2][32], int row
             const uint32_t g = (uint32_t)(c * 4 + g4) ^ ((uint32_t)r & 7u);
             st_shared_v4(base + g * 16u, acc[c][4 * g4], acc[c][4 * g4 + 1], acc[c][4 * g4 + 2], acc[c][4 * g4 + 3]);
         }
+}
+
+// 32 packed bf16 columns of row r (16 words, from epilogue_pack) into a 32 x 32 staging
+// tile with 64-byte rows under the 64-byte swizzle: 16-byte chunk g of row r lands in slot
+// g ^ ((r >> 1) & 3), so each group of 8 lanes covers all 32 banks
+FP4_DEV void epilogue_stage_32(const uint32_t (&w)[32], uint8_t* tile, int r) {
+    const uint32_t base = smem_u32(tile) + (uint32_t)r * 64u;
+#pragma unroll
+    for (int g4 = 0; g4 < 4; ++g4) {
+        const uint32_t g = (uint32_t)g4 ^ (((uint32_t)r >> 1) & 3u);
+        st_shared_v4(base + g * 16u, w[4 * g4], w[4 * g4 + 1], w[4 * g4 + 2], w[4 * g4 + 3]);
+    }
 }
 
 // Fused down-projection input (OUTQ 1: MXFP4, 2: NVFP4).  Columns col0 .. col0+63 of one
@@ -610,11 +632,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
     using C = Gemm2Cfg<KIND, OUTQ>;
     constexpr int S = C::STAGES;
     constexpr int TB = C::TB;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA = smem;
+    extern __shared__ __align__(1024) uint8_t smem2_raw[];
+    // 128-byte-swizzled operand tiles need 1024-byte alignment; both CTAs see the same
+    // layout, so both leave here together, before any barrier
+    if ((smem_u32(smem2_raw) & 1023u) != 0) {
+        if (threadIdx.x == 0) atomicCAS(p.status, 0, STATUS_LAYOUT);
+        return;
+    }
+    uint8_t* sA = smem2_raw;
     uint8_t* sB = sA + S * C::A_BYTES;
-    uint8_t* sEpi = sB + S * C::B_BYTES;                  // 8 staging tiles of 4 KB
+    uint8_t* sEpi = sB + S * C::B_BYTES;                  // 8 per-warp Y staging tiles
     uint8_t* sRSFA = sEpi + C::EPI_BYTES;
     uint8_t* sRSFB = sRSFA + S * C::RSFA_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sRSFB + S * C::RSFB_BYTES);
@@ -693,7 +720,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         const int ew = warp - 8;
         const int q = warp & 3;
         const int h = ew >> 2;
-        uint8_t* stile = sEpi + ew * 4096;
+        uint8_t* stile = sEpi + ew * C::EPI_TILE;
         // Y is streamed out (2 GB at the FFN shape): evict-first lines drain to DRAM during
         // the GEMM instead of being written back while the next kernel streams its input
         const uint64_t pol_y = policy_evict_first();
@@ -744,14 +771,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                     return;
                 }
                 if (col0 >= p.N) return;
-                if (lane == 0) bulk_wait_group_read0();
-                __syncwarp();
-                epilogue_stage<KIND>(p, a, row, col0 + chunk * 32, gs, stile, lane);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0 && row0 < p.M) {
-                    tma_store_2d_hint(&tmY, stile, col0 + chunk * 32, row0, pol_y);
-                    bulk_commit_group();
+                if constexpr (C::EPI_COLS == 64) {
+                    if (lane == 0) bulk_wait_group_read0();
+                    __syncwarp();
+                    epilogue_stage<KIND>(p, a, row, col0 + chunk * 32, gs, stile, lane);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && row0 < p.M) {
+                        tma_store_2d_hint(&tmY, stile, col0 + chunk * 32, row0, pol_y);
+                        bulk_commit_group();
+                    }
+                } else {
+                    // one 32-column store per chunk through the half-size tile
+                    if (row < p.M) epilogue_pack<KIND, 2>(p, a, row, col0 + chunk * 32, gs);
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        if (lane == 0) bulk_wait_group_read0();
+                        __syncwarp();
+                        if (row < p.M) epilogue_stage_32(a[c], stile, lane);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0 && row0 < p.M) {
+                            tma_store_2d_hint(&tmY, stile, col0 + (chunk + c) * 32, row0, pol_y);
+                            bulk_commit_group();
+                        }
+                    }
                 }
             };
             // a split tile: this segment's fp32 sums of the 64 columns go to its slab
