@@ -39,8 +39,6 @@ constexpr int GEMM_BN = 256;
 constexpr int GEMM_STAGES = 4;
 constexpr int GEMM_ACC_COLS = 256;
 constexpr int GEMM_TMEM_COLS = 512;
-constexpr int STATUS_TIMEOUT = 7;
-constexpr int STATUS_LAYOUT = 5;  // FP4_ERR_ARCH: the device did not honour a shared-memory alignment
 
 template <int KIND>
 struct GemmCfg {

@@ -17,6 +17,10 @@ FP4_DEV uint64_t globaltimer() {
     return t;
 }
 
+// Device status word values (the ABI's fp4_status_t codes)
+constexpr int STATUS_TIMEOUT = 7;  // FP4_ERR_TIMEOUT: a bounded wait ran out
+constexpr int STATUS_LAYOUT = 5;   // FP4_ERR_ARCH: the device did not honour a shared-memory alignment
+
 // ------------------------------------------------------------------ mbarrier
 FP4_DEV void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
