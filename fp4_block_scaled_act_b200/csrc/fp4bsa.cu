@@ -111,8 +111,12 @@ fp4_status_t device_state(DeviceState** out) {
                 for (const void* k : pair_kernels)
                     if (!launch_regs_are(k, R)) return FP4_ERR_ARCH;
             }
-            if (cudaFuncSetAttribute(lowrank_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LR_SMEM_BYTES) !=
-                cudaSuccess)
+            if (cudaFuncSetAttribute(lowrank_down_kernel<Q_MXFP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     LR_SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(lowrank_down_kernel<LR_NO_QUANT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     LR_SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(lowrank_down_kernel<Q_MXFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     LR_SMEM_BYTES) != cudaSuccess)
                 return FP4_ERR_CUDA;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.quant_occ[Q_MXFP4], quant_kernel<Q_MXFP4>,
                                                               QUANT_THREADS, 0) != cudaSuccess ||
@@ -284,9 +288,10 @@ int64_t sk_num_kb(int64_t K) { return (K + 255) / 256; }
 // 4290-token W4A8 shape has 34) K is split over up to 8 blocks per row block, whose fp32
 // partial sums a second kernel adds in split order.  Only the full linears, which own a
 // workspace, split; the split is a function of (M, K) alone, so the workspace size is too.
+constexpr int kLowrankFuseBlocks = 64;  // row blocks from which one pass streams X at full speed
 int lr_split(int64_t M, int64_t K) {
     const int64_t blocks = (M + LR_ROWS - 1) / LR_ROWS, nkc = K / LR_KC;
-    if (blocks >= 64) return 1;
+    if (blocks >= kLowrankFuseBlocks) return 1;
     for (int sp : {8, 4, 2})
         if (nkc % sp == 0 && nkc / sp >= 2) return sp;
     return 1;
@@ -296,20 +301,34 @@ size_t lr_partial_bytes(int64_t M, int64_t K) {
     const int64_t mpad = (M + LR_ROWS - 1) / LR_ROWS * LR_ROWS;
     return sp > 1 ? align256((size_t)sp * mpad * 32 * sizeof(float)) : 0;
 }
-void launch_lowrank(const void* x_bf16, const void* l1_bf16, int64_t M, int64_t K, void* u_pair, float* partial,
-                    cudaStream_t st) {
+// X -> (codes, scales) in format QK and u = X L1, in one pass over X.  With few row blocks
+// and no room for a K split (the standalone quantize calls take no workspace), the
+// 34-odd blocks of one pass cannot stream X fast enough, so the quantizer runs as its own
+// grid first (at 4290 x 3072: 42 us for the two launches against 53 us fused).
+template <int QK>
+fp4_status_t launch_lowrank(const DeviceState* ds, const void* x_bf16, const void* l1_bf16, int64_t M, int64_t K,
+                            void* u_pair, float* partial, uint8_t* codes, uint8_t* sf, cudaStream_t st) {
     const int blocks = (int)((M + LR_ROWS - 1) / LR_ROWS);
     const auto x = static_cast<const __nv_bfloat16*>(x_bf16);
     const auto l1 = static_cast<const __nv_bfloat16*>(l1_bf16);
     const auto u = static_cast<__nv_bfloat16*>(u_pair);
     const int sp = partial ? lr_split(M, K) : 1;
-    if (sp == 1) {
-        lowrank_down_kernel<<<blocks, LR_THREADS, LR_SMEM_BYTES, st>>>(x, l1, (int)M, (int)K, u, nullptr, 0);
-        return;
+    if (sp == 1 && blocks < kLowrankFuseBlocks) {
+        fp4_status_t s = launch_quant(ds, QK, x_bf16, M, K, nullptr, codes, sf, st);
+        if (s != FP4_OK) return s;
+        lowrank_down_kernel<LR_NO_QUANT><<<blocks, LR_THREADS, LR_SMEM_BYTES, st>>>(x, l1, (int)M, (int)K, u,
+                                                                                   nullptr, 0, nullptr, nullptr);
+        return launched();
     }
-    lowrank_down_kernel<<<dim3(blocks, sp), LR_THREADS, LR_SMEM_BYTES, st>>>(x, l1, (int)M, (int)K, u, partial,
-                                                                           (int)(K / LR_KC / sp));
+    if (sp == 1) {
+        lowrank_down_kernel<QK><<<blocks, LR_THREADS, LR_SMEM_BYTES, st>>>(x, l1, (int)M, (int)K, u, nullptr, 0,
+                                                                          codes, sf);
+        return launched();
+    }
+    lowrank_down_kernel<QK><<<dim3(blocks, sp), LR_THREADS, LR_SMEM_BYTES, st>>>(
+        x, l1, (int)M, (int)K, u, partial, (int)(K / LR_KC / sp), codes, sf);
     lowrank_reduce_kernel<<<(int)((M * 32 + 255) / 256), 256, 0, st>>>(partial, (int)M, blocks * LR_ROWS, sp, u);
+    return launched();
 }
 // Every pair's share must hold at least one K block (tiles * K blocks >= pairs): a pair
 // with an empty share would be counted among a tile's segments without ever arriving.
@@ -631,9 +650,7 @@ fp4_status_t w4a8_quantize_impl(const void* x_bf16, int64_t M, int64_t K, const 
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if ((s = launch_quant(ds, Q_MXFP8, x_bf16, M, K, nullptr, x_e4m3, x_sf, st)) != FP4_OK) return s;
-    launch_lowrank(x_bf16, l1_bf16, M, K, u_pair, partial, st);
-    return launched();
+    return launch_lowrank<Q_MXFP8>(ds, x_bf16, l1_bf16, M, K, u_pair, partial, x_e4m3, x_sf, st);
 }
 }  // namespace
 extern "C" {
@@ -717,9 +734,7 @@ fp4_status_t w4a4_quantize_impl(const void* x_bf16, int64_t M, int64_t K, const 
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if ((s = launch_quant(ds, Q_MXFP4, x_bf16, M, K, nullptr, x_codes, x_sf, st)) != FP4_OK) return s;
-    launch_lowrank(x_bf16, l1_bf16, M, K, u_pair, partial, st);
-    return launched();
+    return launch_lowrank<Q_MXFP4>(ds, x_bf16, l1_bf16, M, K, u_pair, partial, x_codes, x_sf, st);
 }
 }  // namespace
 extern "C" {

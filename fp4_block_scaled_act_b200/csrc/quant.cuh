@@ -216,6 +216,7 @@ constexpr int LR_ROWS = 128, LR_THREADS = 256, LR_KC = 64, LR_STAGES = 6;
 constexpr int LR_XP = LR_KC + 8;  // padded X row (elements): conflict-free ldmatrix
 constexpr int LR_LP = 32 + 8;     // padded L1 row
 constexpr int LR_SMEM_BYTES = LR_STAGES * (LR_ROWS * LR_XP + LR_KC * LR_LP) * 2;  // dynamic shared memory
+constexpr int LR_NO_QUANT = -1;
 
 FP4_DEV void cp_async16(void* dst, const void* src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
@@ -230,10 +231,19 @@ FP4_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) :
 // kc_per_split) of row block i and writes its fp32 sums to partial[j][m][r] (rows padded to
 // whole blocks); lowrank_reduce_kernel adds the splits in index order.  Otherwise the block
 // covers all of K and writes the pair itself.
+// The same pass can quantize X (QK = Q_MXFP8 for W4A8, Q_MXFP4 for W4A4 SVDQuant; LR_NO_QUANT
+// for the projection alone): every chunk,
+// once it has fed the MMAs, is read back from its stage by groups of 32 (thread t: group t & 1
+// of row t >> 1) and turned into codes and E8M0 scale bytes by the steps quant_kernel takes,
+// so X crosses HBM once for both results.  Rows in [M, Mpad) get zero scale bytes.
+template <int QK>
 __global__ void __launch_bounds__(LR_THREADS) lowrank_down_kernel(const __nv_bfloat16* __restrict__ x,
                                                                   const __nv_bfloat16* __restrict__ l1, int M,
                                                                   int K, __nv_bfloat16* __restrict__ u_pair,
-                                                                  float* __restrict__ partial, int kc_per_split) {
+                                                                  float* __restrict__ partial, int kc_per_split,
+                                                                  uint8_t* __restrict__ codes,
+                                                                  uint8_t* __restrict__ sf) {
+    static_assert(QK == Q_MXFP8 || QK == Q_MXFP4 || QK == LR_NO_QUANT, "MX activations or none");
     extern __shared__ __align__(16) uint8_t lr_smem[];
     auto xs = reinterpret_cast<__nv_bfloat16(*)[LR_ROWS][LR_XP]>(lr_smem);
     auto ls = reinterpret_cast<__nv_bfloat16(*)[LR_KC][LR_LP]>(lr_smem + LR_STAGES * LR_ROWS * LR_XP * 2);
@@ -308,6 +318,51 @@ __global__ void __launch_bounds__(LR_THREADS) lowrank_down_kernel(const __nv_bfl
                         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[2 * h]), "r"(b[2 * h + 1]));
                 }
             }
+        }
+        // quantize the chunk from the stage (it is refilled only after the next barrier)
+        if constexpr (QK != LR_NO_QUANT) {
+            const int qr = tid >> 1, qg = tid & 1;
+            const int m = m0 + qr;
+            const int col = (kc0 + kc) * LR_KC + qg * 32;  // the group's first column
+            const uint4* src = reinterpret_cast<const uint4*>(&xs[st][qr][qg * 32]);
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float w[8];
+                bf16x8_to_f32(src[i], w);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[8 * i + e] = w[e];
+            }
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            const uint32_t sfb = mx_scale_byte<(QK == Q_MXFP4) ? 2 : 8>(amax);
+            const float inv = mx_inv_scale(sfb);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], inv);
+            if (m < M) {
+                if (QK == Q_MXFP8) {
+                    uint32_t c[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        c[i] = cvt_e4m3x2(v[4 * i], v[4 * i + 1]) | (cvt_e4m3x2(v[4 * i + 2], v[4 * i + 3]) << 16);
+                    uint4* dst = reinterpret_cast<uint4*>(codes + (size_t)m * K + col);
+                    dst[0] = make_uint4(c[0], c[1], c[2], c[3]);
+                    dst[1] = make_uint4(c[4], c[5], c[6], c[7]);
+                } else {
+                    uint32_t c[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float e8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) e8[e] = v[8 * i + e];
+                        c[i] = cvt_e2m1x8(e8);
+                    }
+                    *reinterpret_cast<uint4*>(codes + (size_t)m * (K / 2) + col / 2) = make_uint4(c[0], c[1], c[2], c[3]);
+                }
+            }
+            const int j = col >> 5;  // group index in the row: byte j & 3 of atom word j >> 2
+            sf[sf_word_offset(m, j >> 2, K >> 7) + (j & 3)] = (uint8_t)sfb;
         }
     }
     // accumulator fragment: acc[j][0..1] -> row lane/4, acc[j][2..3] -> row lane/4 + 8,

@@ -219,7 +219,8 @@ def _w4a8_check(fb, orc, M, K, N, seed, rows=None, calib=256):
     return H.check_linear(y, Y + LR, S + LS, rows, f"w4a8 M={M} K={K} N={N}")
 
 
-@pytest.mark.parametrize("M,K,N", [(1, 256, 256), (130, 512, 384), (300, 1024, 512)])
+# 8300 rows (65 blocks of 128): the activation side runs as one quantize + project pass
+@pytest.mark.parametrize("M,K,N", [(1, 256, 256), (130, 512, 384), (300, 1024, 512), (8300, 256, 256)])
 def test_w4a8_small_all_elements(fb, orc, M, K, N):
     _w4a8_check(fb, orc, M, K, N, seed=7000 + M)
 
@@ -301,7 +302,7 @@ def _w4a4_check(fb, orc, M, K, N, seed, rows=None, calib=256):
     return H.check_linear(y, Y + LR, S + LS, rows, f"w4a4 M={M} K={K} N={N}")
 
 
-@pytest.mark.parametrize("M,K,N", [(1, 256, 256), (130, 512, 384), (300, 1024, 512)])
+@pytest.mark.parametrize("M,K,N", [(1, 256, 256), (130, 512, 384), (300, 1024, 512), (8300, 256, 256)])
 def test_w4a4_small_all_elements(fb, orc, M, K, N):
     _w4a4_check(fb, orc, M, K, N, seed=8000 + M)
 

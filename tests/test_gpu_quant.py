@@ -68,9 +68,12 @@ def test_e2m1_conversion_sweep(fb, orc):
     _assert_quant(fb, orc, MX, x.reshape(rows, K))
 
 
-def test_e4m3_conversion_sweep(fb, orc):
+@pytest.mark.parametrize("min_rows", [0, 8200], ids=["separate-kernels", "fused-with-lowrank"])
+def test_e4m3_conversion_sweep(fb, orc, min_rows):
     """Every finite bf16 value in (-512, 512) through the device E4M3 path (MXFP8 with a
-    300.0 in each group, so the scale is 2^0 and the elements are e4m3(x))."""
+    300.0 in each group, so the scale is 2^0 and the elements are e4m3(x)).  Padded with zero
+    rows to 8200 (65 blocks of 128), the call quantizes inside the low-rank projection's pass
+    instead of in its own kernel."""
     import torch
 
     allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
@@ -83,7 +86,7 @@ def test_e4m3_conversion_sweep(fb, orc):
     big = np.full((groups, 1), synth.f32_to_bf16_bits(np.float32(300.0)), dtype=np.uint16)
     flat = np.concatenate([big, pad.reshape(groups, n_per_group)], axis=1).reshape(-1)
     K = 512
-    rows = -(-flat.size // K)
+    rows = max(-(-flat.size // K), min_rows)
     x = np.zeros(rows * K, dtype=np.uint16)
     x[: flat.size] = flat
     x = x.reshape(rows, K)
@@ -120,7 +123,8 @@ def test_nvfp4_quant(fb, orc, M, K):
     _assert_quant(fb, orc, NV, x, g)
 
 
-@pytest.mark.parametrize("M,K", [(1, 128), (130, 256), (4290 // 10, 3072)])
+# 8300 rows = 65 blocks of 128 (the last ragged): one pass quantizes and projects
+@pytest.mark.parametrize("M,K", [(1, 128), (130, 256), (4290 // 10, 3072), (8300, 384)])
 def test_mxfp8_quant_and_lowrank(fb, orc, M, K):
     import torch
 
@@ -231,7 +235,7 @@ def test_pack_lowrank_up_is_the_transpose(fb):
     np.testing.assert_array_equal(got, np.ascontiguousarray(l2.T))
 
 
-@pytest.mark.parametrize("M,K", [(130, 512), (300, 1024)])
+@pytest.mark.parametrize("M,K", [(130, 512), (300, 1024), (8300, 384)])
 def test_w4a4_quantize_act(fb, orc, M, K):
     """W4A4 SVDQuant activation side: MXFP4 codes and scales bit-exact, the u pair as in W4A8."""
     import torch
