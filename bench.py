@@ -5,9 +5,11 @@ Workload: the Wan2.2-A14B FFN up-projection in MXFP4, M = 75600 tokens (a 21x45x
 latent grid), K = 5120, N = 13824; bf16 activations N(0,1) x per-channel lognormal
 gains, bf16 weights N(0, 0.02) packed offline, fp16 bias, bf16 output.  One step is
 one quantized linear: dynamic activation quantization + block-scaled GEMM with the
-fused bias epilogue (the weight pre-pack is offline and untimed).
+fused bias epilogue (the weight pre-pack is offline and untimed).  `--fmt nvfp4` runs
+the same layer in NVFP4 (the T2V-A14B NVFP4 card's format), its static activation
+global calibrated once, untimed, on a separate batch of the same layer.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--fmt nvfp4]
 
 Prints one JSON line.  `value` is TFLOPS (2*M*K*N per step, all ranks together)
 with inputs resident in HBM; `e2e` is the same metric through fp4_linear (linear_host) with the
@@ -51,6 +53,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm-ctas", type=int, default=0, choices=[0, 1, 2],
                     help="GEMM kernel: 0 auto (2-CTA 256x256 tile for M > 128), 1 force the 1-CTA 128x256 tile, 2 force 2-CTA")
+    ap.add_argument("--fmt", default="mxfp4", choices=["mxfp4", "nvfp4"])
     ap.add_argument("--m", type=int, default=75600,
                     help="tokens; smaller values run a reduced case of the same kernels (profiling only)")
     return ap.parse_args()
@@ -138,6 +141,19 @@ def make_inputs(rank: int, m: int | None = None, k: int | None = None, n: int | 
     return x, w, b
 
 
+def nv_static_global(k: int | None = None) -> float:
+    """NVFP4 activation global of the layer, calibrated once (untimed) on a separate
+    4096-token batch: its tensor amax T over the largest E2M1 x E4M3 product, T / 2688 in
+    fp32 (1 if T = 0)."""
+    import synth
+
+    k = K if k is None else k
+    s = synth.seeds_for(4, layer=1)
+    cal = synth.activation(s["x"] + 104729, 4096, k, "lognormal", gain_seed=s["gain"])
+    t = np.float32(np.max(np.abs(synth.bf16_bits_to_f32(cal))))
+    return float(t / np.float32(2688.0)) if t > 0 else 1.0
+
+
 def max_over_ranks(x: float, dist=None, device="cuda") -> float:
     """The largest x over all ranks: a job's time is its slowest rank's."""
     if dist is None:
@@ -190,13 +206,15 @@ def cpu_baseline(x_bits, w_bits, b_bits, target_s: float = 15.0):
     """The oracle, as it stands, on a bounded row sample of the same workload."""
     import oracle
 
-    wc, ws, _ = oracle.pack_weight(oracle.MX, w_bits)          # offline step, untimed
-    w_deq = oracle.dequant_fp4(oracle.MX, wc, ws, K)            # once, untimed
+    f = oracle.MX if FMT == "mxfp4" else oracle.NV
+    g_a = nv_static_global() if f == oracle.NV else 1.0
+    wc, ws, g_w = oracle.pack_weight(f, w_bits)                 # offline step, untimed
+    w_deq = oracle.dequant_fp4(f, wc, ws, K, g_w or 1.0)        # once, untimed
 
     def run(rows):
         xs = np.ascontiguousarray(x_bits[rows])
-        c, sf = oracle.quantize(oracle.MX, xs)
-        a = oracle.dequant_fp4(oracle.MX, c, sf, K)
+        c, sf = oracle.quantize(f, xs, g_a)
+        a = oracle.dequant_fp4(f, c, sf, K, g_a)
         oracle.linear_fp64(a, w_deq, b_bits)
 
     t = time.perf_counter()
@@ -209,7 +227,7 @@ def cpu_baseline(x_bits, w_bits, b_bits, target_s: float = 15.0):
     dt = time.perf_counter() - t
     return {"value": 2.0 * nrows * K * N / dt / 1e12, "unit": "TFLOPS", "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": f"{nrows} of {M} rows: MXFP4 quantize + dequantize + fp64 GEMM over full K={K}, N={N} "
+            "sample": f"{nrows} of {M} rows: {FMT.upper()} quantize + dequantize + fp64 GEMM over full K={K}, N={N} "
                       f"({dt:.1f} s); weight pack and dequantize excluded (offline)"}
 
 
@@ -225,14 +243,16 @@ def reference_arm(args):
     s = synth.seeds_for(4, layer=1)
     w = synth.weight(s["w"], N, K)
     b = synth.bias(s["bias"], N)
-    wc, ws, _ = oracle.pack_weight(oracle.MX, w)
-    w_deq = oracle.dequant_fp4(oracle.MX, wc, ws, K)
+    f = oracle.MX if FMT == "mxfp4" else oracle.NV
+    g_a = nv_static_global() if f == oracle.NV else 1.0
+    wc, ws, g_w = oracle.pack_weight(f, w)
+    w_deq = oracle.dequant_fp4(f, wc, ws, K, g_w or 1.0)
     # one step = the quantized linear for a bounded row sample of the workload
     total_steps = args.steps + args.warmup
     probe = synth.activation(s["x"], 1, K, "lognormal", gain_seed=s["gain"])
     t = time.perf_counter()
-    c, sf = oracle.quantize(oracle.MX, probe)
-    oracle.linear_fp64(oracle.dequant_fp4(oracle.MX, c, sf, K), w_deq, b)
+    c, sf = oracle.quantize(f, probe, g_a)
+    oracle.linear_fp64(oracle.dequant_fp4(f, c, sf, K, g_a), w_deq, b)
     per_row = time.perf_counter() - t
     budget = 150.0
     rows_per_step = int(max(1, min(64, budget / max(total_steps, 1) / max(per_row, 1e-4))))
@@ -241,8 +261,8 @@ def reference_arm(args):
     def step(i):
         r0 = (i * rows_per_step) % (x.shape[0] - rows_per_step + 1)
         xs = np.ascontiguousarray(x[r0:r0 + rows_per_step])
-        c, sf = oracle.quantize(oracle.MX, xs)
-        oracle.linear_fp64(oracle.dequant_fp4(oracle.MX, c, sf, K), w_deq, b)
+        c, sf = oracle.quantize(f, xs, g_a)
+        oracle.linear_fp64(oracle.dequant_fp4(f, c, sf, K, g_a), w_deq, b)
 
     for i in range(args.warmup):
         step(i)
@@ -252,7 +272,7 @@ def reference_arm(args):
     dt = time.perf_counter() - t
     flops = 2.0 * rows_per_step * K * N * args.steps
     value = flops / dt / 1e12
-    sample = (f"{rows_per_step} row(s) of the {M}x{K}x{N} workload per step: MXFP4 quantize + "
+    sample = (f"{rows_per_step} row(s) of the {M}x{K}x{N} workload per step: {FMT.upper()} quantize + "
               f"dequantize + fp64 GEMM (weight packed once, untimed)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
@@ -291,6 +311,9 @@ def native_arm(args):
     x = to_dev(x_bits, torch, torch.bfloat16)
     bias = to_dev(b_bits, torch, torch.float16)
     pw = fb.pack_weight(to_dev(w_bits, torch, torch.bfloat16), FMT)
+    # NVFP4: the layer's static activation global (device scalar), calibrated untimed
+    a_global = (torch.tensor([nv_static_global()], dtype=torch.float32, device="cuda")
+                if FMT == "nvfp4" else None)
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     ws_bytes = fb.fp4_linear_workspace_bytes(FMT, M, K, N)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
@@ -304,10 +327,10 @@ def native_arm(args):
         # events time each kernel on the launching stream
         if ev is not None:
             ev[0].record(stream)
-        fb.fp4_quantize_act(FMT, x, M, K, None, codes, sf)
+        fb.fp4_quantize_act(FMT, x, M, K, a_global, codes, sf)
         if ev is not None:
             ev[1].record(stream)
-        fb.fp4_gemm(FMT, codes, sf, M, K, N, pw.codes, pw.sf, None, None, bias, y)
+        fb.fp4_gemm(FMT, codes, sf, M, K, N, pw.codes, pw.sf, pw.w_global, a_global, bias, y)
         if ev is not None:
             ev[2].record(stream)
 
@@ -353,7 +376,7 @@ def native_arm(args):
     pipe = fb.HostPipeline(FMT, min(M, 8192), K, N)
 
     def e2e_step():
-        fb.linear_host(x_host, pw, pipe, bias, None, y_host)
+        fb.linear_host(x_host, pw, pipe, bias, a_global, y_host)
 
     for _ in range(2):
         e2e_step()
@@ -379,8 +402,8 @@ def native_arm(args):
     # denominator is the sustained measured peak; the burst fraction is reported beside it
     fp4_peak = pk["bf16_tflops_sustained"] * FP4_PER_BF16
     fp4_peak_burst = pk["bf16_tflops"] * FP4_PER_BF16
-    q_bytes = 2 * M * K + M * K // 2 + ((M + 127) // 128 * 128) * (K // 32)
-    traffic = gemm_traffic(pair)
+    q_bytes = 2 * M * K + M * K // 2 + ((M + 127) // 128 * 128) * (K // (32 if FMT == "mxfp4" else 16))
+    traffic = gemm_traffic(pair) if FMT == "mxfp4" else None  # counters recorded for MXFP4
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
@@ -390,8 +413,8 @@ def native_arm(args):
                    "parallelism": f"dp{world} (independent batches)" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (X 774 MB, Y 2.09 GB), no flush"},
         "pct_nominal_fp4_peak": 100.0 * value / world / NOMINAL_FP4_TFLOPS,
-        "roofline": {"bound": "tensor", "kernel": "gemm2_kernel<MXFP4> (2-CTA 256x256)" if pair
-                     else "gemm_kernel<MXFP4> (1-CTA 128x256)", "achieved": gemm_tflops,
+        "roofline": {"bound": "tensor", "kernel": f"gemm2_kernel<{FMT.upper()}> (2-CTA 256x256)" if pair
+                     else f"gemm_kernel<{FMT.upper()}> (1-CTA 128x256)", "achieved": gemm_tflops,
                      "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
                      "peak_source": f"{pk_kind} bf16 sustained {pk['bf16_tflops_sustained']} x {FP4_PER_BF16:g} "
                                     f"(nominal FP4/BF16; the GEMM runs inside a ~1 s loop of steps)",
@@ -416,11 +439,14 @@ def native_arm(args):
 
 
 def main():
-    global M, WORKLOAD, FLOP_PER_STEP
+    global M, WORKLOAD, FLOP_PER_STEP, FMT
     args = parse()
+    if args.fmt != FMT:
+        FMT = args.fmt
+        WORKLOAD = f"wan22_t2v_a14b_ffn_up_{FMT}"
     if args.m != M:
         M = args.m
-        WORKLOAD = f"ffn_up_mxfp4_m{M}"
+        WORKLOAD = f"ffn_up_{FMT}_m{M}"
         FLOP_PER_STEP = 2.0 * M * K * N
     if args.impl == "reference":
         return reference_arm(args)
