@@ -72,9 +72,18 @@ __global__ void __launch_bounds__(QUANT_THREADS, 4) quant_kernel(const uint4* __
     const uint32_t adv_rows = UPB / upr, adv_chunk = UPB % upr;
 
     float g = 1.0f, six_g = 6.0f;
+    // NVFP4: the group's decoded scale d = e4m3(sf) * g takes one of at most 127 values per
+    // tensor (sf = 0 .. 0x7E, amax >= 0), so the reciprocal 1 / d is tabulated once per CTA
+    // by the same operations; 0 marks d = 0 (no finite d > 0 has a zero reciprocal)
+    __shared__ float nv_rcp[128];
     if (KIND == Q_NVFP4) {
         g = *g_ptr;
         six_g = __fmul_rn(6.0f, g);
+        if (threadIdx.x < 128) {
+            const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
+            nv_rcp[threadIdx.x] = d == 0.0f ? 0.0f : __frcp_rn(d);
+        }
+        __syncthreads();
     }
     // atoms (4 groups) per 128-row block along K
     const uint32_t apr = (KIND == Q_NVFP4) ? (uint32_t)(K >> 6) : upr;
@@ -117,12 +126,11 @@ __global__ void __launch_bounds__(QUANT_THREADS, 4) quant_kernel(const uint4* __
             if (KIND == Q_NVFP4) {
                 const float s = __fdiv_rn(amax, six_g);
                 sfb = cvt_e4m3x2(s, 0.0f) & 0xFFu;
-                const float d = __fmul_rn(e4m3_to_f32(sfb), g);
-                if (d == 0.0f) {
+                const float r = nv_rcp[sfb & 0x7Fu];  // sfb <= 0x7E: s >= 0, satfinite
+                if (r == 0.0f) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) v[i] = 0.0f;
                 } else {
-                    const float r = __frcp_rn(d);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], r);
                 }
