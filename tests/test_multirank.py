@@ -89,3 +89,16 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     args = argparse.Namespace(gpus=2, steps=1, warmup=0, impl="reference")
     assert bench.reference_arm(args) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_nvfp4_bench_global_matches_the_oracle():
+    """bench.py --fmt nvfp4 calibrates the layer's static activation global on the host; it
+    must be the oracle's global of the same calibration batch."""
+    import bench
+    import oracle
+    import synth
+
+    k = 256
+    s = synth.seeds_for(4, layer=1)
+    cal = synth.activation(s["x"] + 104729, 4096, k, "lognormal", gain_seed=s["gain"])
+    assert bench.nv_static_global(k) == oracle.nv_global(oracle.tensor_amax(cal))
