@@ -402,6 +402,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 //   acc_free[b]  (leader)  accumulator b fully drained by both CTAs (16 warps)
 //   ovl_free     (leader)  overlap columns of the last tile drained (8 warps)
 // =======================================================================================
+// named barrier of the 8 epilogue warps (the MMA hand-off ring uses ids 1 .. TB <= 4)
+constexpr uint32_t EPI_TABLE_BAR = 8;
+
 template <int KIND, int OUTQ = 0>
 struct Gemm2Cfg {
     using C1 = GemmCfg<KIND>;
@@ -431,7 +434,8 @@ struct Gemm2Cfg {
     static constexpr int EPI_BYTES = 8 * EPI_TILE;
     // the dynamic shared array is declared 1024-byte aligned (checked at run time), so the
     // layout needs no alignment slack
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 512;
+    // + barriers; NVFP4 also keeps the fused epilogue's 128-entry reciprocal table after them
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 512 + (KIND == G_NVFP4 ? 512 : 0);
     static constexpr uint32_t AB_TX = A_BYTES + ((KIND == G_W4A8) ? B_BYTES / 2 : B_BYTES);
     static constexpr uint32_t SF_TX = RSFA_BYTES + RSFB_BYTES;
     // TMEM columns: two accumulators overlapping by OVL columns, the shared columns drained
@@ -507,7 +511,7 @@ FP4_DEV void epilogue_stage_32(const uint32_t (&w)[32], uint8_t* tile, int r) {
 // [M, Mpad) store zero scale bytes (the layout's padding), rows >= Mpad nothing.
 template <int KIND, int OUTQ>
 FP4_DEV void epilogue_gelu_quant(const GemmParams& p, uint32_t (&acc)[2][32], int row, int col0, float gs, float g_h,
-                                 float six_g_h) {
+                                 float six_g_h, const float* rcp_tab) {
     const int Mpad = (p.M + 127) & ~127;
     if (row >= Mpad || col0 >= p.N) return;
     constexpr int G = (OUTQ == 1) ? 32 : 16;
@@ -538,10 +542,10 @@ FP4_DEV void epilogue_gelu_quant(const GemmParams& p, uint32_t (&acc)[2][32], in
                     for (int i = 0; i < G; ++i) h[g * G + i] = __fmul_rn(h[g * G + i], inv);
                 } else {
                     sfb = cvt_e4m3x2(__fdiv_rn(amax, six_g_h), 0.0f) & 0xFFu;
-                    const float d = __fmul_rn(e4m3_to_f32(sfb), g_h);
-                    const float r = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+                    // 1 / (e4m3(sfb) * g_h), tabulated per E4M3 code; 0 marks a zero scale
+                    const float r = rcp_tab[sfb & 0x7Fu];
 #pragma unroll
-                    for (int i = 0; i < G; ++i) h[g * G + i] = (d == 0.0f) ? 0.0f : __fmul_rn(h[g * G + i], r);
+                    for (int i = 0; i < G; ++i) h[g * G + i] = (r == 0.0f) ? 0.0f : __fmul_rn(h[g * G + i], r);
                 }
                 sfw |= sfb << (8 * ((j0 + c * (32 / G) + g) & 3));
             }
@@ -643,6 +647,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
     uint8_t* sRSFA = sEpi + C::EPI_BYTES;
     uint8_t* sRSFB = sRSFA + S * C::RSFA_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sRSFB + S * C::RSFB_BYTES);
+    // fused NVFP4 epilogue: reciprocals of the decoded scales, 128 floats after the barriers
+    float* rcp_tab = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 512);
     uint64_t* full = bars;
     uint64_t* sf_full = full + S;
     uint64_t* empty = sf_full + S;
@@ -730,6 +736,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         if (OUTQ == 2) {
             g_h = *p.g_h;
             six_g_h = __fmul_rn(6.0f, g_h);
+            // the decoded group scale d = e4m3(sf) * g_h has at most 127 values: tabulate 1 / d
+            // once (0 for d = 0) by the operations the quantizer uses, then sync the 8 warps
+            const int et = ew * 32 + lane;
+            if (et < 128) {
+                const float d = __fmul_rn(e4m3_to_f32((uint32_t)et), g_h);
+                rcp_tab[et] = d == 0.0f ? 0.0f : __frcp_rn(d);
+            }
+            named_bar_sync(EPI_TABLE_BAR, 256u);
         }
         int tcount = 0;
         Sched sc = sched0;
@@ -765,7 +779,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             // clips rows at or beyond M); the tile is reused once the previous store has read it
             auto emit = [&](uint32_t (&a)[2][32], int chunk) {
                 if (OUTQ != 0) {
-                    epilogue_gelu_quant<KIND, OUTQ>(p, a, row, col0 + chunk * 32, gs, g_h, six_g_h);
+                    epilogue_gelu_quant<KIND, OUTQ>(p, a, row, col0 + chunk * 32, gs, g_h, six_g_h, rcp_tab);
                     return;
                 }
                 if (col0 >= p.N) return;
