@@ -107,6 +107,15 @@ def test_mxfp4_worked(orc, case):
         assert not un[len(case["codes"]):32].any()
 
 
+@pytest.mark.parametrize("case", GOLD["mxfp8_groups"]["cases"], ids=lambda c: c["why"][:30])
+def test_mxfp8_worked(orc, case):
+    x = _group(case["x"], 32)
+    for elems, sf in (orc.quantize_mxfp8(x), onp.quant_mxfp8(x)):
+        assert sf[orc.sf_offset(0, 0, 4)] == case["sf"], case["why"]
+        assert list(elems[0, : len(case["codes"])]) == case["codes"], case["why"]
+        assert not elems[0, len(case["codes"]):32].any()
+
+
 @pytest.mark.parametrize("case", GOLD["nvfp4_blocks"]["cases"], ids=lambda c: c["why"][:30])
 def test_nvfp4_worked(orc, case):
     x = _group(case["x"], 16)
