@@ -263,8 +263,8 @@ fp4_status_t encode_sf(CUtensorMap* m, const uint8_t* sf, int64_t rows, int64_t 
 // for kPlanPairs (a B200's 148 SMs); a device whose pair count needs more slabs per tile
 // runs whole tiles instead.
 constexpr int kPlanPairs = 74;
-int g_stream_k = 0;
-int g_pdl = 1;  // tuning hook: programmatic launch of fp4_linear's short GEMMs after the quantize (1 on, 0 off)  // tuning / test hook: 0 default (off), 1 never, 2 whenever the workspace allows
+int g_stream_k = 0;  // tuning / test hook: 0 default (off), 1 never, 2 whenever the workspace allows
+int g_pdl = 1;       // tuning hook: programmatic launch of fp4_linear's short GEMMs after the quantize (1 on, 0 off)
 
 int64_t sk_kstart(int64_t p, int64_t total, int P) { return p * total / P; }
 int64_t sk_pair_of(int64_t k, int64_t total, int P) {
