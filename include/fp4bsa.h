@@ -217,9 +217,9 @@ fp4_status_t fp4_linear_gelu_quant(fp4_fmt_t fmt, const void* x_bf16, int64_t M,
 
 /* ----------------------------------------------------------------- W4A8 SVDQuant */
 
-/* Activation side of the W4A8 SVDQuant linear (W4A8 README: "dynamic MXFP8
- * activations, rank-32 low-rank correction"; the low-rank branch reads the
- * unquantized input):
+/* Activation side of the W4A8 SVDQuant linear (W4A8 README, W4A8 format: the activations
+ * are quantized to MXFP8 at run time and a rank-32 low-rank branch, which reads the
+ * unquantized input, corrects the product):
  *   x_bf16   (device) [M, K] bf16
  *   l1_bf16  (device) [K, rank] bf16 (proj_down with 1/s folded in)
  *   x_e4m3   (device, out) [M, K] E4M3 bytes
