@@ -1,4 +1,5 @@
-"""Multi-rank host logic of bench.py, on CPU with world-size-2 gloo ranks.
+"""Host logic of bench.py on CPU: multi-rank timing with world-size-2 gloo ranks, the
+NVFP4 calibration, and the reference arm's JSON line.
 
 The data-parallel path shards by batch: every rank quantizes and multiplies its own
 activations against the shared weight, with no collective on the data path.  The only
@@ -102,3 +103,28 @@ def test_nvfp4_bench_global_matches_the_oracle():
     s = synth.seeds_for(4, layer=1)
     cal = synth.activation(s["x"] + 104729, 4096, k, "lognormal", gain_seed=s["gain"])
     assert bench.nv_static_global(k) == oracle.nv_global(oracle.tensor_amax(cal))
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_reference_arm_json_line(fmt):
+    """bench.py --impl reference on rank 0: one JSON line, the native arm's metric, unit and
+    workload, the oracle as its own cpu_baseline and e2e (no host-device copies)."""
+    import json
+    import subprocess
+
+    import bench
+
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0", "--fmt", fmt], capture_output=True, text=True, timeout=300,
+                         env={**os.environ, "RANK": "0", "WORLD_SIZE": "1"})
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "TFLOPS"
+    assert d["higher_is_better"] is True and d["steps"] == 1 and d["warmup"] == 0
+    assert d["config"]["fmt"] == fmt and (d["config"]["M"], d["config"]["K"], d["config"]["N"]) == (75600, 5120, 13824)
+    assert d["value"] > 0
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and isinstance(cb["cores"], int) and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
