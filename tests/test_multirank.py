@@ -128,3 +128,76 @@ def test_reference_arm_json_line(fmt):
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and isinstance(cb["cores"], int) and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def _shard_main(rank, world, port, out_q):
+    """Rank r quantizes and multiplies its own 256-row shard; rank 0 gathers the shards."""
+    import torch
+    import torch.distributed as dist
+
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import oracle
+    import synth
+
+    oracle.build()
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        M, K, N = 512, 256, 128
+        x = synth.activation(71, M, K, "lognormal", gain_seed=72)
+        w = synth.weight(73, N, K)
+        b = synth.bias(74, N)
+        g_a = oracle.nv_global(oracle.tensor_amax(x))
+        rows = np.arange(rank * M // world, (rank + 1) * M // world)
+        res = []
+        for fmt in (oracle.MX, oracle.NV):
+            g = g_a if fmt == oracle.NV else None
+            c, s = oracle.quantize(fmt, np.ascontiguousarray(x[rows]), g)
+            y, _ = oracle.fp4_linear_rows(fmt, x, w, b, rows, g_a=g)
+            for part in (torch.from_numpy(c.astype(np.int32)), torch.from_numpy(s.astype(np.int32)),
+                         torch.from_numpy(y)):
+                got = [torch.empty_like(part) for _ in range(world)]
+                dist.all_gather(got, part)
+                res.append([t.numpy() for t in got])
+        if rank == 0:
+            out_q.put(res)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_row_shards_concatenate_to_the_whole():
+    """The path shards by rows with no collective on the data: two gloo ranks, 256 rows each
+    (whole 128-row scale blocks), give exactly the codes and scale bytes of the unsharded
+    512-row quantize, and the unsharded GEMM rows, in both formats."""
+    import torch.multiprocessing as mp
+
+    import oracle
+    import synth
+
+    oracle.build()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = q.get(timeout=180)
+    for p in procs:
+        p.join(60)
+    assert [p.exitcode for p in procs] == [0, 0]
+    M, K, N = 512, 256, 128
+    x = synth.activation(71, M, K, "lognormal", gain_seed=72)
+    w = synth.weight(73, N, K)
+    b = synth.bias(74, N)
+    g_a = oracle.nv_global(oracle.tensor_amax(x))
+    for i, fmt in enumerate((oracle.MX, oracle.NV)):
+        g = g_a if fmt == oracle.NV else None
+        c, s = oracle.quantize(fmt, x, g)
+        y, S = oracle.fp4_linear_rows(fmt, x, w, b, np.arange(M), g_a=g)
+        cs, ss, ys = res[3 * i: 3 * i + 3]
+        np.testing.assert_array_equal(np.concatenate(cs).astype(np.uint8), c)
+        np.testing.assert_array_equal(np.concatenate(ss).astype(np.uint8), s)
+        # the same rows in fp64; only the product's summation blocking may differ
+        assert np.all(np.abs(np.concatenate(ys) - y) <= 1e-12 * S)
