@@ -1,0 +1,135 @@
+"""CPU models of the GPU kernels' index arithmetic (in place of a sanitizer, which this GPU
+pool does not offer): each test restates one kernel's work assignment as written in
+fp4_block_scaled_act_b200/csrc and checks, over many shapes, that every unit of work is
+done exactly once, that positions computed incrementally equal the direct ones, and that
+every load and store stays inside its buffer.  A change to a kernel's indexing must be
+mirrored here."""
+import itertools
+
+import pytest
+
+QUANT_THREADS, QUANT_UNROLL = 256, 6           # quant.cuh
+LR_ROWS, LR_THREADS, LR_KC = 128, 256, 64       # quant.cuh (low-rank projection)
+SMS, QUANT_OCC = 148, 4                         # B200; resident quantize CTAs per SM
+
+
+def sf_word_offset(r, atom_k, apr):
+    """quant.cuh: byte offset of the 32-bit scale word of row r, atom atom_k."""
+    return ((r >> 7) * apr + atom_k) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4
+
+
+def quant_blocks(M, K):
+    """fp4bsa.cu: one resident wave, at most one CTA per span of units."""
+    units = (M + 127) // 128 * 128 * (K // 128)
+    span = (QUANT_THREADS // 16) * QUANT_UNROLL
+    return max(1, min(-(-units // span), SMS * QUANT_OCC))
+
+
+def quant_walk(M, K, G):
+    """quant_kernel: yields (u, row, chunk) per unit a half-warp processes, checking loads."""
+    grid = quant_blocks(M, K)
+    UPB = QUANT_THREADS // 16
+    upr = K >> 7
+    Mpad = (M + 127) // 128 * 128
+    total = Mpad * upr
+    span = UPB * QUANT_UNROLL
+    per_cta = (-(-total // grid) + span - 1) // span * span
+    adv_rows, adv_chunk = UPB // upr, UPB % upr
+    for b in range(grid):
+        u_begin = b * per_cta
+        u_end = min(total, u_begin + per_cta)
+        for my in range(UPB):
+            row, chunk = divmod(u_begin + my, upr)
+            for ub in range(u_begin, u_end, span):
+                seen = []
+                for it in range(QUANT_UNROLL):
+                    u = ub + it * UPB + my
+                    seen.append((u, row, chunk))
+                    chunk += adv_chunk
+                    row += adv_rows
+                    if chunk >= upr:
+                        chunk -= upr
+                        row += 1
+                for u, r, c in seen:
+                    if u >= u_end:
+                        break
+                    yield u, r, c
+
+
+SHAPES = list(itertools.product([1, 7, 128, 129, 300, 4290], [128, 256, 384, 3072, 5120]))
+
+
+@pytest.mark.parametrize("M,K", SHAPES)
+def test_quant_kernel_covers_every_unit_once_in_bounds(M, K):
+    upr = K >> 7
+    Mpad = (M + 127) // 128 * 128
+    code_words = M * K // 8                       # uint32 words of [M, K/2] codes
+    for G in (32, 16):
+        apr = upr if G == 32 else K >> 6          # atoms (4 groups) per 128-row block
+        sf_size = Mpad * K // G
+        units, words = set(), set()
+        for u, r, c in quant_walk(M, K, G):
+            assert (r, c) == divmod(u, upr)
+            assert u not in units
+            units.add(u)
+            if r < M:                             # code store: 16 words per unit
+                assert u * 16 + 15 < code_words
+            # scale words: one per unit (MX), two (NV, groups of 8 lanes)
+            for half in ((0,) if G == 32 else (0, 1)):
+                off = sf_word_offset(r, c if G == 32 else c * 2 + half, apr)
+                assert 0 <= off and off + 4 <= sf_size and off % 4 == 0
+                assert off not in words
+                words.add(off)
+        assert units == set(range(Mpad * upr))
+        assert len(words) * 4 == sf_size         # the whole scale buffer, padding rows included
+
+
+def lr_split(M, K):
+    """fp4bsa.cu: K split for few 128-row blocks."""
+    blocks, nkc = (M + 127) // 128, K // 64
+    if blocks >= 64:
+        return 1
+    for sp in (8, 4, 2):
+        if nkc % sp == 0 and nkc // sp >= 2:
+            return sp
+    return 1
+
+
+@pytest.mark.parametrize("M,K", SHAPES + [(8300, 384), (75600, 5120)])
+def test_lowrank_pass_covers_every_chunk_once_in_bounds(M, K):
+    """lowrank_down_kernel (split or not, with the fused MX quantize): each (row block, K
+    chunk) is projected and quantized by exactly one block; X loads stay in [M, K] (rows past
+    M are zero-filled, not read); code and scale stores stay in their buffers."""
+    blocks = (M + LR_ROWS - 1) // LR_ROWS
+    for partial in (False, True):
+        sp = lr_split(M, K) if partial else 1
+        nkc_all = K // LR_KC
+        kps = nkc_all // sp if sp > 1 else nkc_all
+        done = set()
+        for bx in range(blocks if M < 2000 else min(blocks, 3)):
+            m0 = bx * LR_ROWS
+            for by in range(sp):
+                kc0 = by * kps if sp > 1 else 0
+                for kc in range(kps):
+                    key = (bx, kc0 + kc)
+                    assert key not in done
+                    done.add(key)
+                    for tid in range(LR_THREADS):             # X loads: 128 rows x 8 pieces
+                        for i in range(4):
+                            idx = tid + i * LR_THREADS
+                            row, c = idx >> 3, idx & 7
+                            if m0 + row < M:
+                                off = (m0 + row) * K + (kc0 + kc) * LR_KC + c * 8
+                                assert off + 8 <= M * K
+                        row, c = tid >> 2, tid & 3            # L1 loads: 64 rows x 4 pieces
+                        assert ((kc0 + kc) * LR_KC + row) * 32 + c * 8 + 8 <= K * 32
+                        qr, qg = tid >> 1, tid & 1            # fused quantize: group qg of row qr
+                        m, col = m0 + qr, (kc0 + kc) * LR_KC + qg * 32
+                        if m < M:
+                            assert m * K + col + 32 <= M * K              # MXFP8 codes
+                            assert m * (K // 2) + col // 2 + 16 <= M * K // 2   # MXFP4 codes
+                        j = col >> 5
+                        off = sf_word_offset(m, j >> 2, K >> 7) + (j & 3)
+                        assert off < (M + 127) // 128 * 128 * K // 32
+        if M < 2000:
+            assert done == {(b, k) for b in range(blocks) for k in range(nkc_all)}
