@@ -133,3 +133,59 @@ def test_lowrank_pass_covers_every_chunk_once_in_bounds(M, K):
                         assert off < (M + 127) // 128 * 128 * K // 32
         if M < 2000:
             assert done == {(b, k) for b in range(blocks) for k in range(nkc_all)}
+
+
+# ------------------------------------------------------------------ stream-K schedule
+def sk_kstart(p, total, P):
+    """fp4bsa.cu / gemm.cuh Sched::kstart: first flattened K block of pair p's share."""
+    return p * total // P
+
+
+def sk_pair_of(k, total, P):
+    """fp4bsa.cu sk_pair_of / gemm.cuh Sched::pair_of: the pair whose share holds block k."""
+    q = k * P // total
+    while q + 1 < P and sk_kstart(q + 1, total, P) <= k:
+        q += 1
+    while q > 0 and sk_kstart(q, total, P) > k:
+        q -= 1
+    return q
+
+
+def sk_seg_max(tiles, num_kb, P):
+    """fp4bsa.cu: the slab count per tile the workspace is sized for."""
+    total = tiles * num_kb
+    return max([1] + [sk_pair_of(t * num_kb + num_kb - 1, total, P) - sk_pair_of(t * num_kb, total, P) + 1
+                      for t in range(tiles)])
+
+
+@pytest.mark.parametrize("M,K,N", [(512, 5120, 5120), (512, 5120, 13824), (300, 384, 256), (1, 1024, 512),
+                                   (256, 2048, 1024), (4096, 5120, 13824), (129, 640, 384)])
+@pytest.mark.parametrize("P", [74, 70, 37])
+def test_stream_k_schedule_covers_every_block_once_within_the_slabs(M, K, N, P):
+    tiles = -(-M // 256) * -(-N // 256)
+    num_kb = -(-K // 256)
+    total = tiles * num_kb
+    if total < P:            # the host runs whole tiles then (every share must be non-empty)
+        return
+    seg_max = sk_seg_max(tiles, num_kb, P)
+    done = {}
+    for pair in range(P):
+        lo, hi = sk_kstart(pair, total, P), sk_kstart(pair + 1, total, P)
+        assert hi > lo                                        # no empty share
+        while lo < hi:                                        # Sched::get / step
+            tile = lo // num_kb
+            kb0 = lo - tile * num_kb
+            kb1 = min(num_kb, kb0 + (hi - lo))
+            pf = sk_pair_of(tile * num_kb, total, P)
+            nseg = sk_pair_of(tile * num_kb + num_kb - 1, total, P) - pf + 1
+            seg = pair - pf
+            assert 0 <= seg < nseg <= seg_max                 # slab (tile, seg) inside the workspace
+            for kb in range(kb0, kb1):
+                assert (tile, kb) not in done
+                done[(tile, kb)] = pair
+                assert sk_pair_of(tile * num_kb + kb, total, P) == pair
+            for rank in range(2):                             # arrival counters: 16 per tile
+                for ew in range(8):
+                    assert tile * 16 + rank * 8 + ew < tiles * 16
+            lo += kb1 - kb0
+    assert len(done) == total
