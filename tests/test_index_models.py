@@ -189,3 +189,38 @@ def test_stream_k_schedule_covers_every_block_once_within_the_slabs(M, K, N, P):
                     assert tile * 16 + rank * 8 + ew < tiles * 16
             lo += kb1 - kb0
     assert len(done) == total
+
+
+# ------------------------------------------------------------------ fused GELU + quantize epilogue
+@pytest.mark.parametrize("M,N", [(1, 256), (129, 384), (300, 512), (600, 1024), (257, 128)])
+@pytest.mark.parametrize("G", [32, 16])
+def test_fused_epilogue_writes_every_code_and_scale_byte_once(M, N, G):
+    """gemm2_kernel with OUTQ != 0 (epilogue_gelu_quant): per 256 x 256 tile, CTA rank r,
+    lane quarter q, lane and column half h, a thread owns row mb*256 + 128r + 32q + lane and
+    two 64-column pairs from nb*256 + 128h.  Codes of rows < M, scale bytes of rows < Mpad
+    (zeros in the padding), nothing past them."""
+    Mpad = (M + 127) // 128 * 128
+    apr = N // (G * 4)
+    codes, sf = {}, {}
+    for mb in range(-(-M // 256)):
+        for nb in range(-(-N // 256)):
+            for r, q, lane, h in itertools.product(range(2), range(4), range(32), range(2)):
+                row = mb * 256 + 128 * r + 32 * q + lane
+                for pair in range(2):
+                    col0 = nb * 256 + 128 * h + 64 * pair
+                    if row >= Mpad or col0 >= N:
+                        continue
+                    j0 = col0 // G
+                    word = sf_word_offset(row, j0 >> 2, apr)
+                    if row < M:
+                        for c in range(2):                  # two 16-byte stores of 32 codes
+                            base = row * (N // 2) + col0 // 2 + 16 * c
+                            for b in range(base, base + 16):
+                                assert b not in codes and b < M * N // 2
+                                codes[b] = 1
+                    span = range(word + (j0 & 3), word + (j0 & 3) + 2) if G == 32 else range(word, word + 4)
+                    for b in span:                          # MX: half a word, NV: the whole word
+                        assert b not in sf and b < Mpad * N // G
+                        sf[b] = 1
+    assert len(codes) == M * N // 2
+    assert len(sf) == Mpad * N // G
