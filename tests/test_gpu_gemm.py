@@ -232,6 +232,12 @@ def test_w4a8_full_size_sampled(fb, orc):
     _w4a8_check(fb, orc, M, K, N, seed=3001, rows=rows, calib=2048)
 
 
+def test_w4a8_full_size_every_element(fb, orc):
+    """The W4A8 configuration at its full size, every element of Y against the oracle (the
+    fp64 oracle of 4290 x 3072 x 14336 takes under a minute on the host)."""
+    _w4a8_check(fb, orc, 4290, 3072, 14336, seed=3011, calib=2048)
+
+
 # ------------------------------------------------------------------ up projection + GELU + quantize
 # The FFN's up projection with GELU-tanh and the down projection's quantizer fused into its
 # epilogue.  z (the bf16 GEMM result) is only known to the GEMM tolerance, so the output is
