@@ -3,8 +3,8 @@
 TEST INFRASTRUCTURE ONLY.  The test suite, the package smoke check and the
 benchmark's CPU-baseline leg are the only users; the CUDA library never loads it.
 
-`fp4_oracle.c` is the oracle proper (plain C, fp32 steps as IEEE operations, fp64
-GEMM, OpenMP over rows).  This module builds it with gcc and exposes it through
+`fp4_oracle.c` is the oracle proper (plain C, fp32 steps as IEEE operations where the
+format fixes them, fp64 GELU and GEMM, OpenMP over rows).  This module builds it with gcc and exposes it through
 ctypes with numpy arrays.  `oracle_np.py` is an independent NumPy restatement used
 to cross-check it on tiny shapes.
 """
@@ -56,7 +56,7 @@ def lib():
             "orc_linear_fp64": (None, [P, I64, P, I64, I64, P, P, P]),
             "orc_lowrank_fp64": (None, [P, I64, P, I64, P, P, I64, I64, P, P]),
             "orc_num_threads": (ctypes.c_int, []),
-            "orc_gelu_f64": (D, [D]), "orc_exp2_f32": (F, [F]), "orc_recip_f32": (F, [F]), "orc_gelu_f32": (F, [F]),
+            "orc_gelu_f64": (D, [D]), "orc_f64_to_bf16_rn": (U16, [D]),
             "orc_gelu_bf16": (None, [P, I64, P]),
         }
         for name, (res, args) in sig.items():
@@ -134,23 +134,13 @@ def gelu_f64(z: float) -> float:
     return lib().orc_gelu_f64(float(z))
 
 
-def exp2_f32(t: float) -> float:
-    """The fixed fp32 2^t of R10 (floor reduction + degree-6 Taylor in ln2 f, fma Horner)."""
-    return lib().orc_exp2_f32(float(t))
-
-
-def recip_f32(d: float) -> float:
-    """The fixed fp32 Newton-Raphson reciprocal of R10."""
-    return lib().orc_recip_f32(float(d))
-
-
-def gelu_f32(z: float) -> float:
-    """The fixed fp32 GELU-tanh evaluation of R10."""
-    return lib().orc_gelu_f32(float(z))
+def f64_to_bf16_rn(x: float) -> int:
+    """Bits of the bf16 nearest to the double x (ties to even, subnormals kept)."""
+    return int(lib().orc_f64_to_bf16_rn(float(x)))
 
 
 def gelu_bf16(z_bf16: np.ndarray) -> np.ndarray:
-    """h = bf16_rn(gelu_f32(z)) element-wise, bf16 bits in and out (R10)."""
+    """h = bf16_rn(gelu(z)) element-wise, gelu in fp64; bf16 bits in and out (R10)."""
     z = np.ascontiguousarray(z_bf16, dtype=np.uint16)
     h = np.zeros_like(z)
     lib().orc_gelu_bf16(_p(z), z.size, _p(h))
@@ -240,6 +230,31 @@ def fp4_linear_rows(fmt, x_bf16, w_bf16, bias_f16, rows, g_a=None, packed_w=None
     a = dequant_fp4(fmt, ac, asf, K, 1.0 if fmt == MX else g_a)
     w = dequant_fp4(fmt, wc, ws, K, 1.0 if fmt == MX else gw)
     return linear_fp64(a, w, bias_f16)
+
+
+def svd_linear_rows(act: str, x_bf16, r_packed, l1_bf16, l2_bf16, bias_f16, rows):
+    """End-to-end oracle of the SVDQuant linear (W4A8 README) for selected rows of x:
+    the activations quantized dynamically (act = "mxfp8" for W4A8, "mxfp4" for the W4A4
+    variant) and dequantized, times the dequantized MXFP4 residual r_packed = (codes, sf)
+    in fp64, plus the low-rank term (x L1) L2 on the unquantized x (R7) and the bias.
+    Returns (Y, S): S sums |a_k r_k| and |u_r L2[r, n]| for the tolerance."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    K = x.shape[1]
+    rows = np.asarray(rows)
+    xs = np.ascontiguousarray(x[rows])
+    if act == "mxfp8":
+        e, sf = quantize_mxfp8(xs)
+        a = dequant_mxfp8(e, sf, K)
+    elif act == "mxfp4":
+        c, sf = quantize(MX, xs)
+        a = dequant_fp4(MX, c, sf, K)
+    else:
+        raise ValueError(act)
+    rc, rs = r_packed
+    w = dequant_fp4(MX, rc, rs, K)
+    Y, S = linear_fp64(a, w, bias_f16)
+    LR, LS = lowrank_fp64(x, rows, l1_bf16, l2_bf16)
+    return Y + LR, S + LS
 
 
 def num_threads() -> int:

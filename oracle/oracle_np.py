@@ -10,6 +10,8 @@ repeat in the other:
   * The scale-factor swizzle is built by reshaping and transposing the [rows, K/G]
     scale matrix into 128x4 atoms, instead of a closed-form offset.
   * The GEMM is a library matmul in float64.
+  * GELU-tanh goes through logaddexp, and bf16 rounding picks the nearer of two
+    neighbouring codes, instead of the C oracle's tanh / exp split and rint.
 
 Sources: MXFP4 format (Wan2.2-I2V-A14B-Lightning MXFP4 card, Quantization
 Details); NVFP4 format (Wan2.2-T2V-A14B NVFP4 card, Model Details); W4A8 SVDQuant
@@ -161,6 +163,36 @@ def quant_nvfp4(x_bf16, g):
         q = (xg * r[:, :, None]).astype(np.float32)
     codes = np.where(d[:, :, None] == 0, np.uint8(0), e2m1_encode(np.where(d[:, :, None] == 0, 0, q)))
     return pack_nibbles(codes.reshape(x.shape)), swizzle_sf(sf)
+
+
+# ---------------------------------------------------------------- GELU-tanh (R10) --
+def gelu_f64(z):
+    """gelu(z) = 0.5 z (1 + tanh(v)), v = sqrt(2/pi) (z + 0.044715 z^3), written as
+    z / (1 + e^{-2v}) = z exp(-log(1 + e^{-2v})) with logaddexp (no cancellation for
+    either sign of v): a different route from the C oracle's tanh/exp split."""
+    z = np.asarray(z, dtype=np.float64)
+    v = np.sqrt(2.0 / np.pi) * (z + 0.044715 * z ** 3)
+    return z * np.exp(-np.logaddexp(0.0, -2.0 * v))
+
+
+def f64_to_bf16_rn(x):
+    """Nearest bf16 (ties to the even code) to each finite double: take the two bf16
+    neighbours of x from its fp32 bits (truncation and the next code up) and keep the
+    closer one.  The differences are exact (Sterbenz), so the choice is exact."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    t = (a.astype(np.float32).view(np.uint32) >> 16).astype(np.int64)
+    # a.astype(float32) may have rounded up past a: step down while the candidate exceeds a
+    lo = t.copy()
+    for _ in range(2):
+        lo = np.where(bf16_to_f32(lo.astype(np.uint16)).astype(np.float64) > a, lo - 1, lo)
+    hi = lo + 1
+    vlo = bf16_to_f32(lo.astype(np.uint16)).astype(np.float64)
+    vhi = bf16_to_f32(np.minimum(hi, 0x7F80).astype(np.uint16)).astype(np.float64)
+    dlo, dhi = a - vlo, vhi - a
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (lo % 2 == 1))
+    mag = np.where(a == 0, 0, np.where(pick_hi, hi, lo))
+    return (mag | (np.signbit(x).astype(np.int64) << 15)).astype(np.uint16)
 
 
 # ---------------------------------------------------------------- dequant + GEMM --

@@ -116,6 +116,34 @@ def test_mxfp8_worked(orc, case):
         assert not elems[0, len(case["codes"]):32].any()
 
 
+@pytest.mark.parametrize("case", GOLD["mxfp8_groups"]["cases"], ids=lambda c: c["why"][:30])
+def test_mxfp8_dequant_worked(orc, case):
+    """orc_dequant_mxfp8 (and the NumPy restatement) turn the worked groups' bytes back into
+    the hand-computed values."""
+    x = _group(case["x"], 32)
+    elems, sf = orc.quantize_mxfp8(x)
+    n = len(case["dequant"])
+    got = orc.dequant_mxfp8(elems, sf, 128)[0]
+    assert list(got[:n]) == case["dequant"], case["why"]
+    assert not got[n:32].any()
+    assert list(onp.dequant_mxfp8(elems, sf, 1, 128)[0, :n]) == case["dequant"]
+
+
+def test_mxfp8_dequant_matches_numpy(orc):
+    """orc_dequant_mxfp8 against the NumPy restatement on random bytes (every E4M3 code but
+    NaN, every scale byte from 100 to 154), selected rows included."""
+    rng = np.random.default_rng(31)
+    rows, K = 300, 256
+    codes = rng.integers(0, 256, size=(rows, K), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0
+    sfm = rng.integers(100, 155, size=(rows, K // 32), dtype=np.uint8)
+    sf = onp.swizzle_sf(sfm)
+    ref = onp.dequant_mxfp8(codes, sf, rows, K)
+    np.testing.assert_array_equal(orc.dequant_mxfp8(codes, sf, K), ref)
+    sel = np.array([0, 5, 127, 128, 299])
+    np.testing.assert_array_equal(orc.dequant_mxfp8(codes, sf, K, rows=sel), ref[sel])
+
+
 @pytest.mark.parametrize("case", GOLD["nvfp4_blocks"]["cases"], ids=lambda c: c["why"][:30])
 def test_nvfp4_worked(orc, case):
     x = _group(case["x"], 16)
@@ -341,6 +369,54 @@ def test_lowrank_oracle_matches_numpy(orc):
     np.testing.assert_allclose(LS, np.abs(u) @ np.abs(l2), rtol=1e-10, atol=1e-12)
 
 
+@pytest.mark.parametrize("K", [128, 256])
+def test_svd_linear_oracle_brute_force(orc, K):
+    """The composed SVDQuant oracle (W4A8: MXFP8 activations, W4A4: MXFP4 activations, MXFP4
+    residual, rank-32 low-rank term on the unquantized input, bias) against the same steps
+    composed from the NumPy restatement, for every M, N in 1..8."""
+    rng = np.random.default_rng(K + 7)
+    rank = 32
+    for M in range(1, 9):
+        for N in range(1, 9):
+            x = bf16(rng.standard_normal((M, K)) * rng.lognormal(0, 1.5, size=K))
+            r = bf16(rng.standard_normal((N, K)) * 0.02)
+            l1 = bf16(rng.standard_normal((K, rank)) * 0.05)
+            l2 = bf16(rng.standard_normal((rank, N)) * 0.05)
+            b = synth.f32_to_f16_bits(rng.standard_normal(N).astype(np.float32) * 0.01)
+            rc, rs, _ = orc.pack_weight(orc.MX, r)
+            xf = onp.bf16_to_f32(x).astype(np.float64)
+            lr = (xf @ onp.bf16_to_f32(l1).astype(np.float64)) @ onp.bf16_to_f32(l2).astype(np.float64)
+            lrs = np.abs(xf @ onp.bf16_to_f32(l1).astype(np.float64)) @ np.abs(onp.bf16_to_f32(l2).astype(np.float64))
+            wc, wsf = onp.quant_mxfp4(r)
+            w = onp.dequant_fp4("mx", wc, wsf, N, K)
+            for act in ("mxfp8", "mxfp4"):
+                Y, S = orc.svd_linear_rows(act, x, (rc, rs), l1, l2, b, np.arange(M))
+                if act == "mxfp8":
+                    e, sf = onp.quant_mxfp8(x)
+                    a = onp.dequant_mxfp8(e, sf, M, K)
+                else:
+                    c, sf = onp.quant_mxfp4(x)
+                    a = onp.dequant_fp4("mx", c, sf, M, K)
+                Y2, S2 = onp.linear_fp64(a, w, b)
+                Y2, S2 = Y2 + lr, S2 + lrs
+                assert np.all(np.abs(Y - Y2) <= 1e-12 * S2 + 1e-300), (act, M, N)
+                np.testing.assert_allclose(S, S2, rtol=1e-12, atol=1e-300)
+
+
+def test_svd_linear_oracle_selects_rows(orc):
+    """Rows selected out of order give the same values as the full result."""
+    f = synth.svdquant_factors(3004, 128, 256, rank=32, calib_tokens=128)
+    x = synth.activation(11, 40, 256, "lognormal")
+    rc, rs, _ = orc.pack_weight(orc.MX, f["r_bf16"])
+    b = synth.bias(5, 128)
+    for act in ("mxfp8", "mxfp4"):
+        Y, S = orc.svd_linear_rows(act, x, (rc, rs), f["l1_bf16"], f["l2_bf16"], b, np.arange(40))
+        sel = np.array([39, 0, 17, 17, 3])
+        Ys, Ss = orc.svd_linear_rows(act, x, (rc, rs), f["l1_bf16"], f["l2_bf16"], b, sel)
+        np.testing.assert_array_equal(Ys, Y[sel])
+        np.testing.assert_array_equal(Ss, S[sel])
+
+
 def test_wan_a14b_byte_count():
     """400 quantized linears per transformer (MXFP4 card, Coverage); packed FP4 + per-32
     E8M0 scales take 0.5 + 1/32 bytes per weight.  The card quotes about 7.45 GiB; the
@@ -356,128 +432,105 @@ def test_wan_a14b_byte_count():
 
 # ------------------------------------------------------------------ GELU-tanh (R10)
 # The activation between ffn.net.0.proj and ffn.net.2 (the MXFP4 cards' coverage lists):
-# 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))).  The oracle evaluates it in fp32 in a
-# fixed order with its own exp; these pins tie that evaluation to the definition.
-def _f32(v):
-    return float(np.float32(v))
+# gelu(z) = 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))).  The oracle is that definition
+# in fp64 (the exp identity where 1 + tanh cancels), rounded to the nearest bf16.  These
+# pins tie it to a library GELU, to the independent NumPy route, to exact identities, and
+# the bf16 rounding to exact rational arithmetic.
+def _gelu_erf(z):
+    """The exact GELU, z Phi(z), that the tanh form approximates."""
+    return 0.5 * z * (1.0 + math.erf(z / math.sqrt(2.0)))
 
 
-def _gelu_arg(z):
-    """a = -2 sqrt(2/pi) (z + 0.044715 z^3), the exp argument of the fp32 evaluation."""
-    return -2.0 * math.sqrt(2.0 / math.pi) * (z + 0.044715 * z ** 3)
-
-
-def test_exp2_f32_against_math(orc):
-    """floor reduction + degree-6 Taylor in ln2 f (fma Horner): within 2^-21.5 relative of
-    2^t over [-126, 127], and exact at integers (f = 0 gives the polynomial's 1)."""
-    rng = np.random.default_rng(11)
-    pts = np.concatenate([np.linspace(-126.0, 127.0, 20001), rng.uniform(-126.0, 127.0, 5000),
-                          [0.0, -0.0, 1e-8, -1e-8, 0.5, -0.5, 0.49999997, -0.49999997]]).astype(np.float32)
-    worst = 0.0
-    for t in pts:
-        t = float(t)
-        ref = 2.0 ** t
-        worst = max(worst, abs(orc.exp2_f32(t) - ref) / ref)
-    assert worst <= 2.0 ** -21.5, worst
-    for n in range(-126, 128):
-        assert orc.exp2_f32(float(n)) == 2.0 ** n
-
-
-def test_recip_f32_newton(orc):
-    """Newton-Raphson 1/d from the exponent-bit guess: within 2^-23 relative over
-    [1, 2^125], and exact where 1/d is a power of two reached by the iteration."""
-    rng = np.random.default_rng(14)
-    ds = np.concatenate([np.exp2(np.linspace(0.0, 125.0, 50001)), rng.uniform(1.0, 4.0, 5000),
-                         [1.0, 1.5, 2.0, 3.0, 1.0000001, 1.9999999]]).astype(np.float32)
-    worst = max(abs(orc.recip_f32(float(d)) * float(d) - 1.0) for d in ds)
-    assert worst <= 2.0 ** -23, worst
-    for k in range(0, 126, 5):
-        assert orc.recip_f32(2.0 ** k) == 2.0 ** -k
-
-
-def test_gelu_f32_against_tanh_definition(orc):
-    """Where 1 + tanh(v) does not cancel in fp64 (z >= -5) the plain definition is the
-    reference; the fp32 evaluation is within (2|a| + 16) 2^-23 relative of it."""
-    for z in np.linspace(-5.0, 14.0, 19001).astype(np.float32):
-        z = float(z)
-        ref = orc.gelu_f64(z)
-        got = orc.gelu_f32(z)
-        tol = (2.0 * abs(_gelu_arg(z)) + 16.0) * 2.0 ** -23 * abs(ref) + 2.0 ** -126
-        assert abs(got - ref) <= tol, (z, got, ref)
-
-
-def test_gelu_f32_against_library_gelu(orc):
-    """PyTorch's own tanh-approximated GELU in fp64 (a library routine) on random bf16
-    inputs of both signs, within the same bound."""
+def test_gelu_f64_against_library_gelu(orc):
+    """PyTorch's tanh-approximated GELU in fp64 (a library routine) where its 1 + tanh does
+    not cancel (z >= -5: 1 + tanh(v) >= 1e-7, so its own relative error stays below 1e-8)."""
     import torch
 
     rng = np.random.default_rng(12)
-    z = np.concatenate([rng.normal(0.0, 2.0, 4000), rng.uniform(-5.0, 12.0, 2000)])
-    zb = synth.f32_to_bf16_bits(z.astype(np.float32))
-    zf = synth.bf16_bits_to_f32(zb).astype(np.float64)
-    ref = torch.nn.functional.gelu(torch.from_numpy(zf), approximate="tanh").numpy()
-    for zi, ri in zip(zf, ref):
-        if zi < -5.0:
-            continue  # fp64 cancellation in 1 + tanh
-        got = orc.gelu_f32(float(zi))
-        tol = (2.0 * abs(_gelu_arg(zi)) + 16.0) * 2.0 ** -23 * abs(ri) + 2.0 ** -126
-        assert abs(got - ri) <= tol, (zi, got, ri)
+    z = np.concatenate([np.linspace(-5.0, 14.0, 19001), rng.normal(0.0, 2.0, 4000).clip(-5.0, None)])
+    ref = torch.nn.functional.gelu(torch.from_numpy(z), approximate="tanh").numpy()
+    got = np.array([orc.gelu_f64(float(v)) for v in z])
+    tol = np.where(z >= -2.0, 1e-14, 1e-8) * np.abs(ref) + 1e-300
+    assert np.all(np.abs(got - ref) <= tol), np.max(np.abs(got - ref) / (np.abs(ref) + 1e-300))
 
 
-def test_gelu_f32_tail_against_sigmoid_identity(orc):
-    """On the negative tail the fp64 reference is the exact identity
-    0.5 (1 + tanh(v)) = 1 / (1 + exp(-2v)), itself checked against tanh where both are
-    accurate; the fp32 result is a signed zero once 2^t passes 2^125 (true value below
-    2^-118 |z|)."""
-    for z in np.linspace(-5.0, 5.0, 1001):
-        v = math.sqrt(2.0 / math.pi) * (z + 0.044715 * z ** 3)
-        assert abs(0.5 * (1.0 + math.tanh(v)) - 1.0 / (1.0 + math.exp(-2.0 * v))) <= 1e-15
-    for z in np.linspace(-10.02, -5.0, 5021).astype(np.float32):
-        z = float(z)
-        a = _gelu_arg(z)
-        got = orc.gelu_f32(z)
-        if got == 0.0:
-            assert math.copysign(1.0, got) == -1.0 and a > 86.6  # t = a / ln2 > 125
-            assert abs(z / (1.0 + math.exp(a))) < 2.0 ** -118 * abs(z)
-            continue
-        ref = z / (1.0 + math.exp(a))
-        assert abs(got - ref) <= (2.0 * abs(a) + 16.0) * 2.0 ** -23 * abs(ref), (z, got, ref)
-    assert math.copysign(1.0, orc.gelu_f32(-11.0)) == -1.0 and orc.gelu_f32(-11.0) == 0.0
-    assert orc.gelu_f32(-3.0e38) == 0.0
+def test_gelu_f64_matches_numpy_route_every_bf16(orc):
+    """Every finite bf16 z: the C oracle's tanh / exp split and the NumPy logaddexp route
+    agree to 1e-12 relative (normal doubles), and give the same bf16 h for every z."""
+    z = np.arange(65536, dtype=np.uint16)
+    exp_field = (z >> 7) & 0xFF
+    z = z[exp_field != 0xFF]                            # finite values only
+    zf = synth.bf16_bits_to_f32(z).astype(np.float64)
+    g_np = onp.gelu_f64(zf)
+    g_c = np.array([orc.gelu_f64(float(v)) for v in zf[::5]])
+    # relative agreement where the values are normal doubles; fp64 subnormals (|g| < 2^-1022,
+    # z below about -26) carry fewer bits and both round to a zero bf16
+    normal = np.abs(g_np[::5]) >= 2.0 ** -1000
+    rel = np.abs(g_c - g_np[::5])[normal] / np.abs(g_np[::5])[normal]
+    assert rel.max() <= 1e-12, rel.max()
+    assert np.all(np.abs(g_c - g_np[::5])[~normal] <= 2.0 ** -1000)
+    np.testing.assert_array_equal(orc.gelu_bf16(z), onp.f64_to_bf16_rn(g_np))
 
 
-def test_gelu_f32_special_values(orc):
-    assert orc.gelu_f32(0.0) == 0.0
-    for z in (12.0, 20.0, 1000.0, 3.0e38):  # sigmoid(2v) rounds to 1 in fp32
-        assert orc.gelu_f32(z) == _f32(z)
-    # GELU-tanh(1) = 0.84119199... (the tanh-approximation's value, fp64 definition)
-    assert abs(orc.gelu_f32(1.0) - 0.8411919906082768) <= 2.0 ** -21
-    # odd part: gelu(z) - gelu(-z) = z
-    for z in (0.25, 0.75, 1.5, 2.5, 4.0):
-        assert abs(orc.gelu_f32(z) - orc.gelu_f32(-z) - z) <= 2.0 ** -20 * z
+def test_gelu_f64_identities(orc):
+    """gelu(z) - gelu(-z) = z (the two sides take different branches for z != 0); gelu(0) = 0;
+    gelu(z) = z once tanh(v) rounds to 1; a signed zero once e^{-2v} overflows; within 1e-3
+    of the exact GELU z Phi(z) that the tanh form approximates."""
+    for z in np.linspace(0.0, 30.0, 3001)[1:]:
+        assert abs(orc.gelu_f64(z) - orc.gelu_f64(-z) - z) <= 4e-16 * z, z
+    assert orc.gelu_f64(0.0) == 0.0
+    for z in (20.0, 100.0, 3.0e38):
+        assert orc.gelu_f64(z) == z
+    for z in (-40.0, -1e3, -3.0e38):
+        g = orc.gelu_f64(z)
+        assert g == 0.0 and math.copysign(1.0, g) == -1.0
+    for z in np.linspace(-8.0, 8.0, 1601):
+        assert abs(orc.gelu_f64(z) - _gelu_erf(z)) <= 1e-3, z
+    # worked values of the definition: gelu(1) = 0.5 (1 + tanh(sqrt(2/pi) 1.044715)), gelu(-1) = gelu(1) - 1
+    assert abs(orc.gelu_f64(1.0) - 0.8411919906082768) <= 1e-15
+    assert abs(orc.gelu_f64(-1.0) + 0.15880800939172324) <= 1e-15
 
 
-def test_gelu_bf16_rounding(orc):
-    """gelu_bf16 rounds the fp32 result to nearest even bf16, brute-forced on small inputs."""
-    import struct
+def test_f64_to_bf16_rn_exact(orc):
+    """Nearest bf16 with ties to the even code, against exact rational arithmetic, on random
+    doubles, exact midpoints, subnormals, the smallest normal and the largest finite value."""
+    from fractions import Fraction
 
-    def bf16_rn(f):
-        u = struct.unpack("<I", struct.pack("<f", f))[0]
-        lower = u & 0xFFFF
-        hi = u >> 16
-        if lower > 0x8000 or (lower == 0x8000 and (hi & 1)):
-            hi += 1
-        return hi & 0xFFFF
+    def bf16_value(b):
+        return Fraction(float(synth.bf16_bits_to_f32(np.array([b], dtype=np.uint16))[0]))
 
+    def nearest(x):
+        xf = Fraction(x)
+        a = abs(xf)
+        best = None
+        t = int(np.float32(abs(x)).view(np.uint32) >> 16) if abs(x) < 3.4e38 else 0x7F7F
+        for c in range(max(0, t - 2), min(0x7F7F, t + 3) + 1):
+            d = abs(bf16_value(c) - a)
+            if best is None or d < best[0] or (d == best[0] and c % 2 == 0):
+                best = (d, c)
+        return best[1] | (0x8000 if math.copysign(1.0, x) < 0 else 0)
+
+    rng = np.random.default_rng(21)
+    xs = list(rng.normal(0, 1, 300) * np.exp2(rng.integers(-140, 120, 300)))
+    for b in rng.integers(1, 0x7F7E, 200):                 # exact midpoints between neighbours
+        lo, hi = bf16_value(int(b)), bf16_value(int(b) + 1)
+        xs.append(float((lo + hi) / 2))
+        xs.append(-float((lo + hi) / 2))
+    xs += [2.0 ** -133, 3 * 2.0 ** -134, 2.0 ** -134, 2.0 ** -126, float.fromhex("0x1.fep127"), float.fromhex("0x1.fdp127"), 1.0, -0.0, 0.0]
+    for x in xs:
+        got = orc.f64_to_bf16_rn(float(x))
+        assert got == nearest(float(x)), (x, hex(got), hex(nearest(float(x))))
+        assert got == int(onp.f64_to_bf16_rn(np.array([x]))[0]), x
+    assert orc.f64_to_bf16_rn(float.fromhex("0x1.ffp127")) == 0x7F80       # the tie above the largest finite value
+
+
+def test_gelu_quantize_composition(orc):
+    """gelu_quantize is gelu_bf16 then the format's quantizer."""
     rng = np.random.default_rng(13)
-    z = synth.f32_to_bf16_bits(rng.normal(0.0, 3.0, 3000).astype(np.float32))
-    h = orc.gelu_bf16(z)
-    zf = synth.bf16_bits_to_f32(z)
-    for zi, hi in zip(zf, h):
-        assert int(hi) == bf16_rn(orc.gelu_f32(float(zi)))
-    # the composition used for the fused path: GELU, bf16, then the MXFP4 quantizer
-    zz = z[:2 * 128].reshape(2, 128)
-    c1, s1 = orc.gelu_quantize(orc.MX, zz)
-    c2, s2 = orc.quantize(orc.MX, orc.gelu_bf16(zz))
-    np.testing.assert_array_equal(c1, c2)
-    np.testing.assert_array_equal(s1, s2)
+    z = synth.f32_to_bf16_bits(rng.normal(0.0, 3.0, 512).astype(np.float32)).reshape(2, 256)
+    for fmt in (orc.MX, orc.NV):
+        g = None if fmt == orc.MX else orc.nv_global(orc.tensor_amax(orc.gelu_bf16(z)))
+        c1, s1 = orc.gelu_quantize(fmt, z, g)
+        c2, s2 = orc.quantize(fmt, orc.gelu_bf16(z), g)
+        np.testing.assert_array_equal(c1, c2)
+        np.testing.assert_array_equal(s1, s2)
