@@ -65,6 +65,12 @@ def check_linear(y_dev, Y_ref: np.ndarray, S: np.ndarray, rows: np.ndarray, what
 
 
 # ------------------------------------------------------------------ fused GELU + quantize
+# The library evaluates GELU-tanh in fp32 (gelu.cuh) and rounds it to bf16; the oracle takes
+# the definition in fp64 and rounds that.  The library states the bound
+#   |gelu_f32(z) - gelu(z)| <= (2 |a| + 16) 2^-23 |gelu(z)| + 2^-126,  a = -2 sqrt(2/pi) (z + 0.044715 z^3)
+# and returns a zero of z's sign once a / ln2 > 125; test_gelu_f32_error_bound checks that bound
+# on the GPU for every finite bf16 z.  Its h may therefore be any bf16 between the roundings of
+# the bound's two ends; the checks below accept exactly those values.
 def _ordered(bits):
     """bf16 bits -> integers in value order (+0 and -0 both 0)."""
     b = np.asarray(bits).astype(np.int32)
@@ -78,6 +84,73 @@ def _from_ordered(o):
 
 def _bf16_f64(bits):
     return synth.bf16_bits_to_f32(np.asarray(bits, dtype=np.uint16)).astype(np.float64)
+
+
+def gelu_error_bound(zf):
+    """The library's stated bound on its fp32 GELU at the (exact) inputs zf, and whether the
+    input is past its cut-off (a / ln2 > 125, where it returns a signed zero)."""
+    from oracle import oracle_np as onp
+
+    zf = np.asarray(zf, dtype=np.float64)
+    with np.errstate(over="ignore", invalid="ignore"):
+        a = 2.0 * np.sqrt(2.0 / np.pi) * (zf + 0.044715 * zf ** 3) * -1.0
+        g = onp.gelu_f64(zf)
+        e = (2.0 * np.abs(a) + 16.0) * 2.0 ** -23 * np.abs(g) + 2.0 ** -126
+    cut = a / np.log(2.0) > 124.99
+    return g, e, cut
+
+
+_TAB = None
+
+
+def _gelu_h_tables():
+    """Over the ordered bf16 domain o in [-32767, 32767] (index o + 32767): the smallest and
+    largest bf16 value of h the library may return for input z(o), and sparse tables for
+    range minima / maxima over runs of consecutive z."""
+    global _TAB
+    if _TAB is None:
+        from oracle import oracle_np as onp
+
+        o = np.arange(-32767, 32768)
+        zb = _from_ordered(o)
+        fin = ((zb >> 7) & 0xFF) != 0xFF
+        zf0 = np.where(fin, _bf16_f64(np.where(fin, zb, 0)), 0.0)
+        g, e, cut = gelu_error_bound(zf0)
+        lo = np.where(cut, np.minimum(g - e, 0.0), g - e)
+        hi = np.where(cut, np.maximum(g + e, 0.0), g + e)
+        with np.errstate(over="ignore"):
+            h_lo = _bf16_f64(onp.f64_to_bf16_rn(lo))
+            h_hi = _bf16_f64(onp.f64_to_bf16_rn(hi))
+        h_lo = np.where(fin, h_lo, -np.inf)
+        h_hi = np.where(fin, h_hi, np.inf)
+        mins, maxs = [h_lo], [h_hi]
+        k = 1
+        while k < h_lo.size:
+            pm, px = mins[-1], maxs[-1]
+            mins.append(np.minimum(pm[:-k], pm[k:]))
+            maxs.append(np.maximum(px[:-k], px[k:]))
+            k *= 2
+        _TAB = (mins, maxs)
+    return _TAB
+
+
+def gelu_h_interval(z_lo_bits, z_hi_bits):
+    """For brackets [z_lo, z_hi] of bf16 inputs (bits, z_lo <= z_hi in value): the smallest and
+    largest h the library may return for any z in the bracket."""
+    mins, maxs = _gelu_h_tables()
+    l = _ordered(z_lo_bits) + 32767
+    r = _ordered(z_hi_bits) + 32767
+    n = r - l + 1
+    assert np.all(n >= 1)
+    k = np.floor(np.log2(n)).astype(np.int64)
+    hmin = np.empty(l.shape)
+    hmax = np.empty(l.shape)
+    for kk in np.unique(k):
+        m = k == kk
+        w = 1 << int(kk)
+        hmin[m] = np.minimum(mins[kk][l[m]], mins[kk][r[m] - w + 1])
+        hmax[m] = np.maximum(maxs[kk][l[m]], maxs[kk][r[m] - w + 1])
+    return hmin, hmax
 
 
 def _bf16_bracket(v):
@@ -98,45 +171,21 @@ def _bf16_bracket(v):
     return lo_b, hi_b
 
 
-def check_gelu_quant(fmt, codes_dev, sf_dev, Y_ref, S, rows, M, N, g_h, what):
-    """Validity of the fused up-projection output h = quant(bf16(gelu(z))), z the bf16 GEMM
-    result.  z is only known to the GEMM tolerance (|z - Y| <= ulp_bf16(Y) + 1e-5 S), so
-    for every element the oracle brackets the admissible bf16 z, maps the bracket through
-    the oracle's bf16 GELU (monotone on each side of its minimum near z = -0.752, whose
-    value is included when the bracket straddles it) to an interval [h_min, h_max], and
-    requires: each group's scale byte lies between the scales of the smallest and largest
-    admissible group amax, and each code lies, given the GPU's own scale, between the codes
-    of h_min and h_max.  Padding rows' scale bytes must be zero.  Returns the fraction of
-    codes equal to the quantization of the oracle's own bf16(gelu(bf16(Y)))."""
+def check_quant_of_interval(fmt, codes, sf_rows, hmin, hmax, g_h, what, row_ids=None):
+    """Codes [R, N/2] and scale bytes [R, N/G] (unswizzled) of R rows are admissible for some h
+    with hmin <= h <= hmax element-wise: each group's scale byte lies between the scales of the
+    smallest and largest admissible group amax, and each code lies, given that scale, between
+    the codes of hmin and hmax."""
     from oracle import oracle_np as onp
 
     G = 32 if fmt == oracle.MX else 16
-    T = oracle.tolerance(Y_ref, S)
-    zl = _bf16_bracket(Y_ref - T)[1]
-    zh = _bf16_bracket(Y_ref + T)[0]
-    hl = _bf16_f64(oracle.gelu_bf16(zl))
-    hh = _bf16_f64(oracle.gelu_bf16(zh))
-    hmin, hmax = np.minimum(hl, hh), np.maximum(hl, hh)
-    # the bf16 GELU's minimum region
-    o0, o1 = _ordered(_bf16_bracket(np.array([-0.80]))[0])[0], _ordered(_bf16_bracket(np.array([-0.70]))[1])[0]
-    zt_b = _from_ordered(np.arange(o0, o1 + 1))
-    zt, ht = _bf16_f64(zt_b), _bf16_f64(oracle.gelu_bf16(zt_b))
-    zlv, zhv = _bf16_f64(zl), _bf16_f64(zh)
-    span = (zlv <= zt.max()) & (zhv >= zt.min())
-    if span.any():
-        idx = np.nonzero(span)
-        inside = (zt[None, :] >= zlv[idx][:, None]) & (zt[None, :] <= zhv[idx][:, None])
-        hm = np.where(inside, ht[None, :], np.inf).min(axis=1)
-        hmin[idx] = np.minimum(hmin[idx], hm)
+    R, N = hmin.shape
     mag_lo = np.where((hmin <= 0) & (hmax >= 0), 0.0, np.minimum(np.abs(hmin), np.abs(hmax)))
     mag_hi = np.maximum(np.abs(hmin), np.abs(hmax))
-    R = len(rows)
     a_lo = mag_lo.reshape(R, N // G, G).max(-1)
     a_hi = mag_hi.reshape(R, N // G, G).max(-1)
-    Mpad = -(-M // 128) * 128
-    sf_all = onp.unswizzle_sf(host_u8(sf_dev), Mpad, N // G)
-    assert np.all(sf_all[M:] == 0), f"{what}: nonzero scale bytes in padding rows"
-    sf = sf_all[rows].astype(np.int64)
+    sf = sf_rows.astype(np.int64)
+    rid = np.arange(R) if row_ids is None else np.asarray(row_ids)
 
     def scaled(h, per_group):
         return (h.reshape(R, N // G, G) * per_group[..., None]).reshape(R, N)
@@ -160,19 +209,70 @@ def check_gelu_quant(fmt, codes_dev, sf_dev, Y_ref, S, rows, M, N, g_h, what):
         s_hi = (hmax.astype(np.float32).reshape(R, N // G, G) * r[..., None]).reshape(R, N)
         zero = np.repeat(d == 0, G, axis=1)
     bad_sf = (sf < b_lo) | (sf > b_hi)
-    assert not bad_sf.any(), (f"{what}: {bad_sf.sum()} scale bytes outside their admissible range; first "
-                              f"{np.argwhere(bad_sf)[0]}")
-    codes = onp.unpack_nibbles(host_u8(codes_dev)[rows])
-    q = onp.e2m1_decode(codes)
+    if bad_sf.any():
+        i = tuple(np.argwhere(bad_sf)[0])
+        raise AssertionError(f"{what}: {bad_sf.sum()} scale bytes outside their admissible range; first at row "
+                             f"{rid[i[0]]} group {i[1]}: byte {sf[i]} range [{b_lo[i]}, {b_hi[i]}]")
+    q = onp.e2m1_decode(onp.unpack_nibbles(codes))
     q_lo = np.where(zero, 0.0, onp.e2m1_decode(onp.e2m1_encode(s_lo)))
     q_hi = np.where(zero, 0.0, onp.e2m1_decode(onp.e2m1_encode(s_hi)))
     bad = (q < q_lo) | (q > q_hi)
     if bad.any():
         i = tuple(np.argwhere(bad)[0])
         raise AssertionError(f"{what}: {bad.sum()} / {bad.size} codes outside their admissible range; first at "
-                             f"row {rows[i[0]]} col {i[1]}: code value {q[i]} range [{q_lo[i]}, {q_hi[i]}]")
+                             f"row {rid[i[0]]} col {i[1]}: code value {q[i]} range [{q_lo[i]}, {q_hi[i]}]")
+
+
+def check_gelu_quant(fmt, codes_dev, sf_dev, Y_ref, S, rows, M, N, g_h, what):
+    """Validity of the fused up-projection output h = quant(bf16(gelu(z))), z the bf16 GEMM
+    result.  z is only known to the GEMM tolerance (|z - Y| <= ulp_bf16(Y) + 1e-5 S), so for
+    every element the admissible bf16 z form a bracket, mapped through the library's GELU
+    bound (gelu_h_interval) to an interval [h_min, h_max]; the codes and scales must be
+    admissible for it (check_quant_of_interval).  Padding rows' scale bytes must be zero.
+    Returns the fraction of codes equal to the oracle's quantization of bf16(gelu(bf16(Y)))."""
+    from oracle import oracle_np as onp
+
+    G = 32 if fmt == oracle.MX else 16
+    T = oracle.tolerance(Y_ref, S)
+    zl = _bf16_bracket(Y_ref - T)[1]
+    zh = _bf16_bracket(Y_ref + T)[0]
+    hmin, hmax = gelu_h_interval(zl, zh)
+    R = len(rows)
+    Mpad = -(-M // 128) * 128
+    sf_all = onp.unswizzle_sf(host_u8(sf_dev), Mpad, N // G)
+    assert np.all(sf_all[M:] == 0), f"{what}: nonzero scale bytes in padding rows"
+    codes = host_u8(codes_dev)[rows]
+    check_quant_of_interval(fmt, codes, sf_all[rows], hmin, hmax, g_h, what, row_ids=rows)
     # agreement with the oracle's own choice z = bf16(Y)
     zb = _bf16_bracket(Y_ref)
     zn = np.where(np.abs(_bf16_f64(zb[0]) - Y_ref) <= np.abs(_bf16_f64(zb[1]) - Y_ref), zb[0], zb[1])
     c_ref, _ = oracle.gelu_quantize(fmt, zn.reshape(R, N), g_h)
-    return float((onp.unpack_nibbles(c_ref) == codes).mean())
+    return float((onp.unpack_nibbles(c_ref) == onp.unpack_nibbles(codes)).mean())
+
+
+def check_gelu_quant_exact(fmt, codes_dev, sf_dev, z_bits, g_h, what, chunk=4096):
+    """fp4_gelu_quantize_act of an exactly known bf16 z [M, K]: rows whose codes and scale bytes
+    equal the oracle's (bf16(gelu_f64(z)) quantized) pass at once; every other row must be
+    admissible for the library's GELU bound (check_quant_of_interval).  Padding rows' scale
+    bytes must be zero.  Returns the fraction of rows that differ from the oracle."""
+    from oracle import oracle_np as onp
+
+    M, K = z_bits.shape
+    G = 32 if fmt == oracle.MX else 16
+    Mpad = -(-M // 128) * 128
+    codes = host_u8(codes_dev).reshape(M, K // 2)
+    sf_all = onp.unswizzle_sf(host_u8(sf_dev), Mpad, K // G)
+    assert np.all(sf_all[M:] == 0), f"{what}: nonzero scale bytes in padding rows"
+    differ = 0
+    for r0 in range(0, M, chunk):
+        r1 = min(M, r0 + chunk)
+        c_ref, s_ref = oracle.gelu_quantize(fmt, z_bits[r0:r1], g_h)
+        s_ref = onp.unswizzle_sf(s_ref, r1 - r0, K // G)
+        bad = np.nonzero((c_ref != codes[r0:r1]).any(1) | (s_ref != sf_all[r0:r1]).any(1))[0]
+        if bad.size:
+            differ += bad.size
+            zb = z_bits[r0 + bad]
+            hmin, hmax = gelu_h_interval(zb, zb)
+            check_quant_of_interval(fmt, codes[r0 + bad], sf_all[r0 + bad], hmin, hmax, g_h, what,
+                                    row_ids=r0 + bad)
+    return differ / M
