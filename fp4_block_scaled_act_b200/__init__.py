@@ -6,7 +6,7 @@ stream becomes the stream argument, and a non-OK status raises FP4Error.  All
 arithmetic runs in the library's CUDA kernels.  There is no fallback: if the
 library is missing or the device is not sm_100, the calls raise.
 
-The helpers at the end (pack_weight, quantize_act, linear, pack_lowrank_up, w4a8_linear,
+The helpers at the end (pack_weight, calibrate_act_global, quantize_act, linear, w4a8_linear,
 w4a4_linear, gelu_quantize_act, linear_gelu_quant, linear_host)
 allocate outputs and workspaces with torch and call the same entry points.
 """
@@ -31,9 +31,9 @@ EXPORTS = [
     "fp4_codes_bytes", "fp4_sf_bytes", "fp4_linear_workspace_bytes", "w4a8_workspace_bytes",
     "fp4_tensor_amax", "fp4_pack_weight", "fp4_quantize_act", "fp4_gemm", "fp4_linear",
     "w4a8_quantize_act", "w4a8_gemm", "w4a8_svd_linear", "fp4_sync_status", "fp4_status_string",
-    "fp4_set_wait_timeout_ns", "fp4_linear_noalloc", "w4a8_pack_lowrank_up",
+    "fp4_set_wait_timeout_ns", "fp4_linear_noalloc",
     "w4a4_workspace_bytes", "w4a4_quantize_act", "w4a4_gemm", "w4a4_svd_linear",
-    "fp4_gelu_quantize_act", "fp4_gemm_gelu_quant", "fp4_linear_gelu_quant",
+    "fp4_gelu_quantize_act", "fp4_gemm_gelu_quant", "fp4_linear_gelu_quant", "fp4_calibrate_act_global",
 ]
 
 
@@ -62,12 +62,12 @@ def lib():
             "w4a8_workspace_bytes": (SZ, [I64, I64, I64, I]),
             "fp4_tensor_amax": (I, [P, I64, P, P]),
             "fp4_pack_weight": (I, [I, P, I64, I64, P, P, P, P]),
+            "fp4_calibrate_act_global": (I, [P, I64, P, P, P]),
             "fp4_quantize_act": (I, [I, P, I64, I64, P, P, P, P]),
             "fp4_gemm": (I, [I, P, P, I64, I64, I64, P, P, P, P, P, P, P]),
             "fp4_linear": (I, [I, P, I64, I64, I64, P, P, P, P, P, P, P, SZ, P]),
             "fp4_linear_noalloc": (I, [I, P, I64, I64, I64, P, P, P, P, P, P, P]),
             "w4a8_quantize_act": (I, [P, I64, I64, P, I, P, P, P, P]),
-            "w4a8_pack_lowrank_up": (I, [P, I64, I, P, P]),
             "w4a4_workspace_bytes": (SZ, [I64, I64, I64, I]),
             "fp4_gelu_quantize_act": (I, [I, P, I64, I64, P, P, P, P]),
             "fp4_gemm_gelu_quant": (I, [I, P, P, I64, I64, I64, P, P, P, P, P, P, P, P, P]),
@@ -84,6 +84,8 @@ def lib():
             "fp4bsa_set_gemm_ctas": (None, [I]),
             "fp4bsa_set_stream_k": (None, [I]),
             "fp4bsa_set_pdl": (None, [I]),
+            "fp4bsa_test_gelu_f32": (I, [P, I64, P, P]),
+            "fp4bsa_clock_probe": (I, [P, I, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -144,6 +146,11 @@ def fp4_tensor_amax(x, n: int, amax_out, stream=None):
     _check(lib().fp4_tensor_amax(_ptr(x), n, _ptr(amax_out), _stream(stream)), "fp4_tensor_amax")
 
 
+def fp4_calibrate_act_global(x, n: int, amax_inout, g_out, stream=None):
+    _check(lib().fp4_calibrate_act_global(_ptr(x), n, _ptr(amax_inout), _ptr(g_out), _stream(stream)),
+           "fp4_calibrate_act_global")
+
+
 def fp4_pack_weight(fmt, w, N: int, K: int, w_codes, w_sf, w_global=None, stream=None):
     _check(lib().fp4_pack_weight(_fmt(fmt), _ptr(w), N, K, _ptr(w_codes), _ptr(w_sf), _ptr(w_global),
                                  _stream(stream)), "fp4_pack_weight")
@@ -199,19 +206,15 @@ def w4a8_quantize_act(x, M: int, K: int, l1, rank: int, x_e4m3, x_sf, u_pair, st
                                    _stream(stream)), "w4a8_quantize_act")
 
 
-def w4a8_pack_lowrank_up(l2, N: int, rank: int, l2t, stream=None):
-    _check(lib().w4a8_pack_lowrank_up(_ptr(l2), N, rank, _ptr(l2t), _stream(stream)), "w4a8_pack_lowrank_up")
-
-
-def w4a8_gemm(x_e4m3, x_sf, u_pair, M: int, K: int, N: int, r_codes, r_sf, l2t, rank: int, bias, y,
+def w4a8_gemm(x_e4m3, x_sf, u_pair, M: int, K: int, N: int, r_codes, r_sf, l2, rank: int, bias, y,
               stream=None):
     _check(lib().w4a8_gemm(_ptr(x_e4m3), _ptr(x_sf), _ptr(u_pair), M, K, N, _ptr(r_codes), _ptr(r_sf),
-                           _ptr(l2t), rank, _ptr(bias), _ptr(y), _stream(stream)), "w4a8_gemm")
+                           _ptr(l2), rank, _ptr(bias), _ptr(y), _stream(stream)), "w4a8_gemm")
 
 
-def w4a8_svd_linear(x, M: int, K: int, N: int, r_codes, r_sf, l1, l2t, rank: int, bias, y, workspace,
+def w4a8_svd_linear(x, M: int, K: int, N: int, r_codes, r_sf, l1, l2, rank: int, bias, y, workspace,
                     ws_bytes: int, stream=None):
-    _check(lib().w4a8_svd_linear(_ptr(x), M, K, N, _ptr(r_codes), _ptr(r_sf), _ptr(l1), _ptr(l2t), rank,
+    _check(lib().w4a8_svd_linear(_ptr(x), M, K, N, _ptr(r_codes), _ptr(r_sf), _ptr(l1), _ptr(l2), rank,
                                  _ptr(bias), _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
            "w4a8_svd_linear")
 
@@ -225,15 +228,15 @@ def w4a4_quantize_act(x, M: int, K: int, l1, rank: int, x_codes, x_sf, u_pair, s
                                    _stream(stream)), "w4a4_quantize_act")
 
 
-def w4a4_gemm(x_codes, x_sf, u_pair, M: int, K: int, N: int, r_codes, r_sf, l2t, rank: int, bias, y,
+def w4a4_gemm(x_codes, x_sf, u_pair, M: int, K: int, N: int, r_codes, r_sf, l2, rank: int, bias, y,
               stream=None):
     _check(lib().w4a4_gemm(_ptr(x_codes), _ptr(x_sf), _ptr(u_pair), M, K, N, _ptr(r_codes), _ptr(r_sf),
-                           _ptr(l2t), rank, _ptr(bias), _ptr(y), _stream(stream)), "w4a4_gemm")
+                           _ptr(l2), rank, _ptr(bias), _ptr(y), _stream(stream)), "w4a4_gemm")
 
 
-def w4a4_svd_linear(x, M: int, K: int, N: int, r_codes, r_sf, l1, l2t, rank: int, bias, y, workspace,
+def w4a4_svd_linear(x, M: int, K: int, N: int, r_codes, r_sf, l1, l2, rank: int, bias, y, workspace,
                     ws_bytes: int, stream=None):
-    _check(lib().w4a4_svd_linear(_ptr(x), M, K, N, _ptr(r_codes), _ptr(r_sf), _ptr(l1), _ptr(l2t), rank,
+    _check(lib().w4a4_svd_linear(_ptr(x), M, K, N, _ptr(r_codes), _ptr(r_sf), _ptr(l1), _ptr(l2), rank,
                                  _ptr(bias), _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
            "w4a4_svd_linear")
 
@@ -248,6 +251,18 @@ def fp4_status_string(status: int) -> str:
 
 def fp4_set_wait_timeout_ns(ns: int):
     lib().fp4_set_wait_timeout_ns(ns)
+
+
+def fp4bsa_clock_probe(out, blocks: int, stream=None):
+    """Measurement hook: out (int64 [3 * blocks], device) = (SM id, SM cycle counter, global
+    ns timer) per block, recorded by a tiny kernel on `stream`."""
+    _check(lib().fp4bsa_clock_probe(_ptr(out), blocks, _stream(stream)), "fp4bsa_clock_probe")
+
+
+def fp4bsa_test_gelu_f32(z, n: int, g, stream=None):
+    """Test hook: g (fp32, device) = the library's fp32 GELU-tanh of each bf16 z (device),
+    before the bf16 rounding the fused activation applies."""
+    _check(lib().fp4bsa_test_gelu_f32(_ptr(z), n, _ptr(g), _stream(stream)), "fp4bsa_test_gelu_f32")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -272,6 +287,20 @@ def pack_weight(w, fmt="mxfp4", stream=None) -> PackedWeight:
     g = torch.empty(1, dtype=torch.float32, device=w.device) if f == NVFP4 else None
     fp4_pack_weight(f, w, N, K, codes, sf, g, stream)
     return PackedWeight(f, N, K, codes, sf, g)
+
+
+def calibrate_act_global(batches, stream=None):
+    """NVFP4 static activation global from one or more bf16 calibration batches (CUDA):
+    returns (g_a, amax) as one-element fp32 device tensors."""
+    import torch
+
+    batches = [batches] if hasattr(batches, "is_cuda") else list(batches)
+    dev = batches[0].device
+    amax = torch.zeros(1, dtype=torch.float32, device=dev)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    for b in batches:
+        fp4_calibrate_act_global(b, b.numel(), amax, g, stream)
+    return g, amax
 
 
 def quantize_act(x, fmt="mxfp4", a_global=None, stream=None):
@@ -302,19 +331,9 @@ def linear(x, pw: PackedWeight, bias=None, a_global=None, y=None, workspace=None
     return y
 
 
-def pack_lowrank_up(l2, stream=None):
-    """bf16 [rank, N] low-rank up-projection (CUDA) -> packed bf16 [N, rank] for the GEMM."""
-    import torch
-
-    rank, N = l2.shape
-    l2t = torch.empty((N, rank), dtype=torch.bfloat16, device=l2.device)
-    w4a8_pack_lowrank_up(l2, N, rank, l2t, stream)
-    return l2t
-
-
-def w4a8_linear(x, r: PackedWeight, l1, l2t, bias=None, y=None, workspace=None, stream=None):
+def w4a8_linear(x, r: PackedWeight, l1, l2, bias=None, y=None, workspace=None, stream=None):
     """W4A8 SVDQuant linear: bf16 [M, K] -> bf16 [M, N] (MXFP4 residual r, rank-32 L1 [K, rank]
-    and packed L2 [N, rank] from pack_lowrank_up)."""
+    and L2 [rank, N] as stored)."""
     import torch
 
     M, K = x.shape
@@ -323,13 +342,13 @@ def w4a8_linear(x, r: PackedWeight, l1, l2t, bias=None, y=None, workspace=None, 
         y = torch.empty((M, r.N), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
         workspace = torch.empty(w4a8_workspace_bytes(M, K, r.N, rank), dtype=torch.uint8, device=x.device)
-    w4a8_svd_linear(x, M, K, r.N, r.codes, r.sf, l1, l2t, rank, bias, y, workspace, workspace.numel(), stream)
+    w4a8_svd_linear(x, M, K, r.N, r.codes, r.sf, l1, l2, rank, bias, y, workspace, workspace.numel(), stream)
     return y
 
 
-def w4a4_linear(x, r: PackedWeight, l1, l2t, bias=None, y=None, workspace=None, stream=None):
+def w4a4_linear(x, r: PackedWeight, l1, l2, bias=None, y=None, workspace=None, stream=None):
     """W4A4 SVDQuant linear: bf16 [M, K] -> bf16 [M, N] (MXFP4 activations and residual r,
-    rank-32 L1 [K, rank] and packed L2 [N, rank] from pack_lowrank_up)."""
+    rank-32 L1 [K, rank] and L2 [rank, N] as stored)."""
     import torch
 
     M, K = x.shape
@@ -338,7 +357,7 @@ def w4a4_linear(x, r: PackedWeight, l1, l2t, bias=None, y=None, workspace=None, 
         y = torch.empty((M, r.N), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
         workspace = torch.empty(w4a4_workspace_bytes(M, K, r.N, rank), dtype=torch.uint8, device=x.device)
-    w4a4_svd_linear(x, M, K, r.N, r.codes, r.sf, l1, l2t, rank, bias, y, workspace, workspace.numel(), stream)
+    w4a4_svd_linear(x, M, K, r.N, r.codes, r.sf, l1, l2, rank, bias, y, workspace, workspace.numel(), stream)
     return y
 
 

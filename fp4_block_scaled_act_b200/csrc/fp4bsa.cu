@@ -348,7 +348,7 @@ size_t sk_bytes(int64_t M, int64_t K, int64_t N) {
 }
 
 // 2-CTA GEMM: A box 128 rows, B box 128 rows (half of the 256-wide N tile) per CTA.
-// tu / tl: the W4A8 low-rank operands (u pair, packed L2); other kinds pass any map.
+// tu / tl: the W4A8 low-rank operands (u pair, L2 [rank, N]); other kinds pass any map.
 // OUTQ != 0: the fused GELU + quantize output (p.h_codes / p.h_sf) instead of p.y.
 // pdl: launch with programmatic stream serialization, so the kernel's launch and prologue
 // overlap the previous kernel on the stream (its producer waits before reading A); used
@@ -439,6 +439,27 @@ fp4_status_t fp4_tensor_amax(const void* x_bf16, int64_t n, float* amax_out, voi
     if (blocks < 1) blocks = 1;
     amax_kernel<<<(int)blocks, 256, 0, st>>>(static_cast<const uint16_t*>(x_bf16), n,
                                              reinterpret_cast<unsigned int*>(amax_out));
+    return launched();
+}
+
+fp4_status_t fp4_calibrate_act_global(const void* x_bf16, int64_t n, float* amax_inout, float* g_out,
+                                      void* stream) {
+    if (!x_bf16 || !amax_inout || !g_out || n < 1) return FP4_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || (reinterpret_cast<uintptr_t>(amax_inout) & 3u) ||
+        (reinterpret_cast<uintptr_t>(g_out) & 3u))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    fp4_status_t s = device_state(&ds);
+    if (s != FP4_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int64_t blocks = (n / 8 + 255) / 256;
+    if (blocks > ds->sm_count * 8) blocks = ds->sm_count * 8;
+    if (blocks < 1) blocks = 1;
+    // the running amax is raised in place (max is order-independent), then g = T / 2688
+    amax_kernel<<<(int)blocks, 256, 0, st>>>(static_cast<const uint16_t*>(x_bf16), n,
+                                             reinterpret_cast<unsigned int*>(amax_inout));
+    if ((s = launched()) != FP4_OK) return s;
+    nv_global_from_kernel<<<1, 1, 0, st>>>(amax_inout, g_out);
     return launched();
 }
 
@@ -659,28 +680,16 @@ fp4_status_t w4a8_quantize_act(const void* x_bf16, int64_t M, int64_t K, const v
     return w4a8_quantize_impl(x_bf16, M, K, l1_bf16, rank, x_e4m3, x_sf, u_pair, nullptr, stream);
 }
 
-fp4_status_t w4a8_pack_lowrank_up(const void* l2_bf16, int64_t N, int rank, void* l2t_bf16, void* stream) {
-    if (!l2_bf16 || !l2t_bf16 || rank != 32) return FP4_ERR_INVALID_ARG;
-    if (N < 128 || N % 128 != 0 || N >= kMaxDim) return FP4_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(l2_bf16) || !aligned16(l2t_bf16)) return FP4_ERR_MISALIGNED;
-    DeviceState* ds;
-    fp4_status_t s = device_state(&ds);
-    if (s != FP4_OK) return s;
-    transpose_rank_kernel<<<(int)(N / 128), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const __nv_bfloat16*>(l2_bf16), (int)N, static_cast<__nv_bfloat16*>(l2t_bf16));
-    return launched();
-}
-
 fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const void* u_pair, int64_t M, int64_t K,
-                       int64_t N, const uint8_t* r_codes, const uint8_t* r_sf, const void* l2t_bf16, int rank,
+                       int64_t N, const uint8_t* r_codes, const uint8_t* r_sf, const void* l2_bf16, int rank,
                        const void* bias_f16, void* y_bf16, void* stream) {
-    if (!x_e4m3 || !x_sf || !u_pair || !r_codes || !r_sf || !l2t_bf16 || !y_bf16 || rank != 32)
+    if (!x_e4m3 || !x_sf || !u_pair || !r_codes || !r_sf || !l2_bf16 || !y_bf16 || rank != 32)
         return FP4_ERR_INVALID_ARG;
     fp4_status_t s = check_shape(M, K, N);
     if (s != FP4_OK) return s;
     // the unpacking tensor map needs a 32-byte aligned residual-weight base
     if (!aligned16(x_e4m3) || !aligned16(x_sf) || !aligned16(u_pair) || (reinterpret_cast<uintptr_t>(r_codes) & 31u) ||
-        !aligned16(r_sf) || !aligned16(l2t_bf16) || !aligned16(bias_f16) || !aligned16(y_bf16))
+        !aligned16(r_sf) || !aligned16(l2_bf16) || !aligned16(bias_f16) || !aligned16(y_bf16))
         return FP4_ERR_MISALIGNED;
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;
@@ -690,12 +699,12 @@ fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const void* u
     // packed E2M1 in global memory, unpacked to one 16-byte slot per 16 values in shared memory
     if ((s = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, r_codes, K, N, K / 2, 128, 128)) != FP4_OK)
         return s;
-    // u pair [M, 64] bf16 (128-byte rows) and packed L2 [N, 32] bf16 (64-byte rows)
+    // u pair [M, 64] bf16 (128-byte rows) and L2 [32, N] bf16 as stored, in 64-column boxes
     if ((s = encode_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, u_pair, 2 * (uint64_t)rank, M, 4 * (uint64_t)rank,
                        2 * rank, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
         return s;
-    if ((s = encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l2t_bf16, (uint64_t)rank, N, 2 * (uint64_t)rank, rank,
-                       128, CU_TENSOR_MAP_SWIZZLE_64B)) != FP4_OK)
+    if ((s = encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l2_bf16, (uint64_t)N, (uint64_t)rank, 2 * (uint64_t)N, 64,
+                       (uint32_t)rank, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
         return s;
     GemmParams p{};
     p.M = (int)M, p.N = (int)N, p.K = (int)K;
@@ -706,20 +715,20 @@ fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const void* u
 }
 
 fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N, const uint8_t* r_codes,
-                             const uint8_t* r_sf, const void* l1_bf16, const void* l2t_bf16, int rank,
+                             const uint8_t* r_sf, const void* l1_bf16, const void* l2_bf16, int rank,
                              const void* bias_f16, void* y_bf16, void* workspace, size_t ws_bytes, void* stream) {
     if (!workspace || rank != 32) return FP4_ERR_INVALID_ARG;
     fp4_status_t s = check_shape(M, K, N);
     if (s != FP4_OK) return s;
     if (ws_bytes < w4a8_workspace_bytes(M, K, N, rank)) return FP4_ERR_WORKSPACE;
     if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
-    if (!r_codes || !r_sf || !l2t_bf16 || !y_bf16) return FP4_ERR_INVALID_ARG;
+    if (!r_codes || !r_sf || !l2_bf16 || !y_bf16) return FP4_ERR_INVALID_ARG;
     uint8_t* xe = static_cast<uint8_t*>(workspace);
     uint8_t* xs = xe + align256((size_t)M * K);
     uint8_t* u = xs + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K));
     float* partial = lr_partial_bytes(M, K) ? reinterpret_cast<float*>(u + align256((size_t)M * rank * 4)) : nullptr;
     if ((s = w4a8_quantize_impl(x_bf16, M, K, l1_bf16, rank, xe, xs, u, partial, stream)) != FP4_OK) return s;
-    return w4a8_gemm(xe, xs, u, M, K, N, r_codes, r_sf, l2t_bf16, rank, bias_f16, y_bf16, stream);
+    return w4a8_gemm(xe, xs, u, M, K, N, r_codes, r_sf, l2_bf16, rank, bias_f16, y_bf16, stream);
 }
 
 }  // extern "C"
@@ -744,14 +753,14 @@ fp4_status_t w4a4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const v
 }
 
 fp4_status_t w4a4_gemm(const uint8_t* x_codes, const uint8_t* x_sf, const void* u_pair, int64_t M, int64_t K,
-                       int64_t N, const uint8_t* r_codes, const uint8_t* r_sf, const void* l2t_bf16, int rank,
+                       int64_t N, const uint8_t* r_codes, const uint8_t* r_sf, const void* l2_bf16, int rank,
                        const void* bias_f16, void* y_bf16, void* stream) {
-    if (!x_codes || !x_sf || !u_pair || !r_codes || !r_sf || !l2t_bf16 || !y_bf16 || rank != 32)
+    if (!x_codes || !x_sf || !u_pair || !r_codes || !r_sf || !l2_bf16 || !y_bf16 || rank != 32)
         return FP4_ERR_INVALID_ARG;
     fp4_status_t s = check_shape(M, K, N);
     if (s != FP4_OK) return s;
     if (!aligned16(x_codes) || !aligned16(x_sf) || !aligned16(u_pair) || !aligned16(r_codes) || !aligned16(r_sf) ||
-        !aligned16(l2t_bf16) || !aligned16(bias_f16) || !aligned16(y_bf16))
+        !aligned16(l2_bf16) || !aligned16(bias_f16) || !aligned16(y_bf16))
         return FP4_ERR_MISALIGNED;
     DeviceState* ds;
     if ((s = device_state(&ds)) != FP4_OK) return s;
@@ -762,8 +771,8 @@ fp4_status_t w4a4_gemm(const uint8_t* x_codes, const uint8_t* x_sf, const void* 
     if ((s = encode_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, u_pair, 2 * (uint64_t)rank, M, 4 * (uint64_t)rank,
                        2 * rank, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
         return s;
-    if ((s = encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l2t_bf16, (uint64_t)rank, N, 2 * (uint64_t)rank, rank,
-                       128, CU_TENSOR_MAP_SWIZZLE_64B)) != FP4_OK)
+    if ((s = encode_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l2_bf16, (uint64_t)N, (uint64_t)rank, 2 * (uint64_t)N, 64,
+                       (uint32_t)rank, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
         return s;
     GemmParams p{};
     p.M = (int)M, p.N = (int)N, p.K = (int)K;
@@ -774,20 +783,20 @@ fp4_status_t w4a4_gemm(const uint8_t* x_codes, const uint8_t* x_sf, const void* 
 }
 
 fp4_status_t w4a4_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N, const uint8_t* r_codes,
-                             const uint8_t* r_sf, const void* l1_bf16, const void* l2t_bf16, int rank,
+                             const uint8_t* r_sf, const void* l1_bf16, const void* l2_bf16, int rank,
                              const void* bias_f16, void* y_bf16, void* workspace, size_t ws_bytes, void* stream) {
     if (!workspace || rank != 32) return FP4_ERR_INVALID_ARG;
     fp4_status_t s = check_shape(M, K, N);
     if (s != FP4_OK) return s;
     if (ws_bytes < w4a4_workspace_bytes(M, K, N, rank)) return FP4_ERR_WORKSPACE;
     if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
-    if (!r_codes || !r_sf || !l2t_bf16 || !y_bf16) return FP4_ERR_INVALID_ARG;
+    if (!r_codes || !r_sf || !l2_bf16 || !y_bf16) return FP4_ERR_INVALID_ARG;
     uint8_t* xc = static_cast<uint8_t*>(workspace);
     uint8_t* xs = xc + align256(fp4_codes_bytes(FP4_FMT_MXFP4, M, K));
     uint8_t* u = xs + align256(fp4_sf_bytes(FP4_FMT_MXFP4, M, K));
     float* partial = lr_partial_bytes(M, K) ? reinterpret_cast<float*>(u + align256((size_t)M * rank * 4)) : nullptr;
     if ((s = w4a4_quantize_impl(x_bf16, M, K, l1_bf16, rank, xc, xs, u, partial, stream)) != FP4_OK) return s;
-    return w4a4_gemm(xc, xs, u, M, K, N, r_codes, r_sf, l2t_bf16, rank, bias_f16, y_bf16, stream);
+    return w4a4_gemm(xc, xs, u, M, K, N, r_codes, r_sf, l2_bf16, rank, bias_f16, y_bf16, stream);
 }
 
 fp4_status_t fp4_sync_status(void* stream) {
@@ -879,3 +888,52 @@ void fp4bsa_set_pdl(int on) { g_pdl = on ? 1 : 0; }
 void fp4bsa_test_skip_iteration(int it) { g_skip_iter = it; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Test hook (not in the public header): the fp32 GELU-tanh value, before its bf16 rounding,
+// that the fused epilogue and fp4_gelu_quantize_act compute for each bf16 input, so the
+// tests can hold it against its stated error bound.  z_bf16 [n] and g_f32 [n] are device
+// arrays; n even.
+__global__ void gelu_probe_kernel(const uint32_t* z2, int64_t pairs, float2* g2) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < pairs; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t w = z2[i];
+        float g0, g1;
+        gelu_f32_x2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u), g0, g1);
+        g2[i] = make_float2(g0, g1);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Measurement hook (not in the public header): each block's first thread records its SM id,
+// that SM's cycle counter and the global nanosecond timer: out[3 b + 0..2].  Two probes
+// around a timed region give every SM's average clock over it (cycles / nanoseconds), which
+// nvidia-smi's periodic samples can miss when the clock moves within a short region.
+__global__ void clock_probe_kernel(unsigned long long* out) {
+    if (threadIdx.x == 0) {
+        unsigned int sm;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+        out[3 * blockIdx.x + 0] = sm;
+        out[3 * blockIdx.x + 1] = (unsigned long long)clock64();
+        out[3 * blockIdx.x + 2] = globaltimer();
+    }
+}
+
+extern "C" fp4_status_t fp4bsa_clock_probe(uint64_t* out, int blocks, void* stream) {
+    if (!out || blocks < 1 || blocks > 4096) return FP4_ERR_INVALID_ARG;
+    clock_probe_kernel<<<blocks, 32, 0, (cudaStream_t)stream>>>(reinterpret_cast<unsigned long long*>(out));
+    return launched();
+}
+
+extern "C" fp4_status_t fp4bsa_test_gelu_f32(const void* z_bf16, int64_t n, float* g_f32, void* stream) {
+    if (!z_bf16 || !g_f32 || n < 2 || (n & 1)) return FP4_ERR_INVALID_ARG;
+    if (((uintptr_t)z_bf16 & 3u) || ((uintptr_t)g_f32 & 7u)) return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    fp4_status_t s = device_state(&ds);
+    if (s != FP4_OK) return s;
+    if (!ds->arch_ok) return FP4_ERR_ARCH;
+    const int64_t pairs = n / 2;
+    const int blocks = (int)std::min<int64_t>((pairs + 255) / 256, (int64_t)ds->sm_count * 8);
+    gelu_probe_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(static_cast<const uint32_t*>(z_bf16), pairs,
+                                                               reinterpret_cast<float2*>(g_f32));
+    return launched();
+}

@@ -458,11 +458,14 @@ struct Gemm2Cfg {
     static constexpr uint32_t REG_LAUNCH = 128, REG_LO = 80, REG_HI = 176;
     static_assert(256 * REG_LO + 256 * REG_HI == THREADS * REG_LAUNCH, "register split must match the launch");
     // W4A8 low-rank stage (one per tile, after the K stages): A = the u pair, 128 rows x 64
-    // bf16 (128-byte rows, 128-byte swizzle); B = packed L2, 128 rows x 32 bf16 (64-byte
-    // rows, 64-byte swizzle); four kind::f16 MMAs of K = 16 (u_hi x L2, then u_lo x L2).
-    static constexpr uint32_t LR_TX = 128 * 128 + 128 * 64;
-    static constexpr uint32_t IDESC_LR = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
-                                         ((uint32_t)(256 >> 4) << 24);
+    // bf16 (128-byte rows, 128-byte swizzle, K-major); B = L2 as stored, [rank = 32][N] bf16,
+    // read MN-major: this CTA's 128 columns as two 64-column blocks of 32 K rows x 128 bytes
+    // (128-byte swizzle; K rows 8 at a time 1024 bytes apart, the second block 4096 bytes
+    // on); four kind::f16 MMAs of K = 16 (u_hi x L2, then u_lo x L2), B transposed (bit 16).
+    static constexpr uint32_t LR_TX = 128 * 128 + 2 * 32 * 128;
+    static constexpr uint32_t LR_B_LBO = 32 * 128, LR_B_SBO = 8 * 128;
+    static constexpr uint32_t IDESC_LR = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                                         ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
     static constexpr uint32_t IDESC = (C1::A_FMT << 7) | (C1::B_FMT << 10) | ((uint32_t)(256 >> 3) << 17) |
                                       (C1::SCALE_FMT << 23) | ((uint32_t)(256 >> 4) << 24);
     static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -939,7 +942,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                             if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::LR_TX);
                             mbar_arrive(&sf_full[s]);
                             tma_load_2d_pair(sA + s * C::A_BYTES, &tmU, bar, 0, mb * 256 + (int)rank * 128, pol_a);
-                            tma_load_2d_pair(sB + s * C::B_BYTES, &tmL, bar, 0, nb * 256 + (int)rank * 128, pol_b);
+                            // L2 [32][N]: this CTA's 128 columns as two 64-column boxes of 32 rows
+                            tma_load_2d_pair(sB + s * C::B_BYTES, &tmL, bar, nb * 256 + (int)rank * 128, 0, pol_b);
+                            tma_load_2d_pair(sB + s * C::B_BYTES + C::LR_B_LBO, &tmL, bar,
+                                             nb * 256 + (int)rank * 128 + 64, 0, pol_b);
                             continue;
                         }
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::AB_TX);
@@ -1065,7 +1071,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
     #pragma unroll
                             for (int k = 0; k < 4; ++k) {
                                 const uint64_t adesc = smem_desc(a_base + k * 32, 0, 1024, 2u);
-                                const uint64_t bdesc = smem_desc(b_base + (k & 1) * 32, 0, 512, 4u);
+                                const uint64_t bdesc =
+                                    smem_desc(b_base + (k & 1) * 2 * C::LR_B_SBO, C::LR_B_LBO, C::LR_B_SBO, 2u);
                                 mma2_f16(dacc, adesc, bdesc, C::IDESC_LR, 1u);
                             }
                             tc_commit_pair(&empty[s], 0x3);

@@ -203,11 +203,14 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
     }
 }
 
-// In place: amax bits -> NVFP4 global g = T / 2688 (T = 0 gives 1).
-__global__ void nv_global_kernel(float* g) {
-    const float T = *g;
-    *g = (T == 0.0f) ? 1.0f : __fdiv_rn(T, 2688.0f);
-}
+// NVFP4 global g = T / 2688 (T = 0 gives 1), one IEEE fp32 division.
+FP4_DEV float nv_global_of(float T) { return (T == 0.0f) ? 1.0f : __fdiv_rn(T, 2688.0f); }
+
+// In place: amax bits -> NVFP4 global.
+__global__ void nv_global_kernel(float* g) { *g = nv_global_of(*g); }
+
+// g_out = NVFP4 global of the amax in *amax (kept).
+__global__ void nv_global_from_kernel(const float* amax, float* g_out) { *g_out = nv_global_of(*amax); }
 
 // ---------------------------------------------------------------- low-rank down-projection
 // W4A8 SVDQuant: u[m, r] = sum_k x[m, k] * L1[k, r] (rank 32) with bf16 inputs and fp32
@@ -419,23 +422,6 @@ __global__ void __launch_bounds__(256) lowrank_reduce_kernel(const float* __rest
     const int m = i >> 5, r = i & 31;
     u_pair[(size_t)m * 64 + r] = hi;
     u_pair[(size_t)m * 64 + 32 + r] = lo;
-}
-
-// W4A8: L2 [32, N] bf16 (rank-major) -> packed L2 [N, 32] bf16, the K-major operand of the
-// GEMM's low-rank stage.  Block: 128 columns.
-__global__ void __launch_bounds__(256) transpose_rank_kernel(const __nv_bfloat16* __restrict__ l2, int N,
-                                                             __nv_bfloat16* __restrict__ l2t) {
-    __shared__ __nv_bfloat16 t[32][128 + 2];
-    const int n0 = blockIdx.x * 128;
-    for (int i = threadIdx.x; i < 32 * 128; i += 256) {
-        const int r = i / 128, c = i % 128;
-        t[r][c] = l2[(size_t)r * N + n0 + c];
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < 32 * 128; i += 256) {
-        const int c = i / 32, r = i % 32;
-        l2t[(size_t)(n0 + c) * 32 + r] = t[r][c];
-    }
 }
 
 }  // namespace fp4

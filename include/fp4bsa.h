@@ -99,6 +99,18 @@ size_t w4a8_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank);
  * The result is order-independent. */
 fp4_status_t fp4_tensor_amax(const void* x_bf16, int64_t n, float* amax_out, void* stream);
 
+/* Static activation global for NVFP4, from calibration (NVFP4 card, Model Details: the
+ * activation global scales are static, set once from calibration data, while the block
+ * scales stay dynamic).  Call it once per calibration batch of the layer's input:
+ *   x_bf16      (device) n bf16 values of one calibration batch
+ *   amax_inout  (device, in/out) one fp32: the running tensor amax over the batches seen so
+ *               far; set it to 0 before the first batch.  Raised to max(amax_inout, max|x_i|).
+ *   g_out       (device, out) one fp32: g_a = amax_inout / 2688 in fp32 (1 if it is 0), the
+ *               a_global that fp4_quantize_act and fp4_linear take.
+ * The result is order-independent (a max) and bit-exact with the format rule above. */
+fp4_status_t fp4_calibrate_act_global(const void* x_bf16, int64_t n, float* amax_inout, float* g_out,
+                                      void* stream);
+
 /* Offline weight pre-pack (MXFP4 / NVFP4 cards: weights stored as packed E2M1 with
  * block scales; NVFP4 adds an FP32 global from the tensor amax).
  *   w_bf16    (device) [N, K] bf16, torch Linear layout (out_features x in_features)
@@ -151,8 +163,8 @@ fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K,
 
 /* fp4_linear for callers that cannot allocate device memory (a plugin whose host owns
  * every allocation, code running under another framework's memory pool, a real-time
- * loop that must not block in an allocator).  The paper has no counterpart: this is a
- * packaging variant of fp4_linear, not part of the method.
+ * loop that must not block in an allocator).  The model-card pages this library follows
+ * have no counterpart to it: it is a packaging variant of fp4_linear, not part of the method.
  *   Same arguments and result as fp4_linear, minus the workspace: the quantized
  *   activations go to a library-owned device array of FP4_NOALLOC_SCRATCH_BYTES
  *   (16 MiB) that exists on every GPU that loads the library until the process exits.
@@ -161,7 +173,8 @@ fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K,
  *   current); make that first call before any stream capture.
  *   Returns FP4_ERR_WORKSPACE, launching nothing, when
  *   fp4_linear_workspace_bytes(fmt, M, K, N) exceeds FP4_NOALLOC_SCRATCH_BYTES
- *   (e.g. MXFP4 with K = 5120 fits up to 6168 rows).
+ *   (e.g. MXFP4 with K = 5120 fits up to 6161 rows: 6161 x 2560 code bytes plus
+ *   49 x 128 x 160 scale bytes = 16,775,680 bytes).
  *   Every call shares the one array, and it keeps the last call's contents: calls that
  *   overlap on the GPU (other streams, other host threads on the same device) race and
  *   must be serialized by the caller.  No part of the array needs clearing between calls. */
@@ -175,14 +188,17 @@ fp4_status_t fp4_linear_noalloc(fp4_fmt_t fmt, const void* x_bf16, int64_t M, in
 /* The Wan2.2 FFN applies GELU-tanh between its two quantized linears (ffn.net.0.proj ->
  * ffn.net.2, MXFP4 card Quantization Details coverage list).  These calls produce the
  * down projection's quantized input, h = bf16_rn(gelu_tanh(z)) with z the bf16
- * up-projection output, without writing z to memory.  gelu_tanh(z) is
- * 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))) evaluated in fp32 in a fixed order:
- *   q = 0.044715 (z z); w = (q + 1) z; a = -2 sqrt(2/pi) w;
- *   a > 88: z * 0;  otherwise z / (1 + exp(max(a, -87)))
- * with exp by Cody-Waite reduction (n = floor(a / ln2 + 1/2), ln2 split into a 16-bit and
- * a remainder part) and the degree-7 Taylor polynomial, each step one IEEE fp32
- * operation, so the codes are reproducible bit for bit.  h is then quantized exactly as
- * fp4_quantize_act quantizes x (same formats, layouts and NVFP4 global rule). */
+ * up-projection output, without writing z to memory, where
+ *   gelu_tanh(z) = 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))).
+ * The library evaluates it in fp32 as z / (1 + 2^t), t = -2 sqrt(2/pi) (z + 0.044715 z^3) / ln 2:
+ * 2^t by rounding t to an integer n and a degree-6 Taylor polynomial of 2^(t - n), the
+ * reciprocal by three Newton-Raphson steps from a guess taken from the bits of 1 + 2^t; for
+ * t > 125 the result is a zero of z's sign.  Its error against the exact value is at most
+ * (2 |a| + 16) 2^-23 |gelu(z)| + 2^-126 with a = t ln 2, and h is its nearest bf16, so h is
+ * the correctly rounded bf16 of gelu_tanh(z) except where that value lies within the bound
+ * of a rounding midpoint, where h may be the other neighbour (a few in a thousand inputs).
+ * The evaluation is deterministic: the same z always gives the same h.  h is then quantized
+ * exactly as fp4_quantize_act quantizes x (same formats, layouts and NVFP4 global rule). */
 
 /* Standalone: z_bf16 [M, K] bf16 (the up-projection output) -> codes [M, K/2] and scale
  * factors of h in `fmt`; a_global is the down projection's static activation global
@@ -232,30 +248,31 @@ fp4_status_t w4a8_quantize_act(const void* x_bf16, int64_t M, int64_t K, const v
                                int rank, uint8_t* x_e4m3, uint8_t* x_sf, void* u_pair,
                                void* stream);
 
-/* Offline pack of the low-rank up-projection for the GEMM (like fp4_pack_weight):
- *   l2_bf16   (device) [rank, N] bf16 (proj_up, rank-major as the checkpoint stores it)
- *   l2t_bf16  (device, out) [N, rank] bf16, the transpose.  N multiple of 128, rank 32. */
-fp4_status_t w4a8_pack_lowrank_up(const void* l2_bf16, int64_t N, int rank, void* l2t_bf16,
-                                  void* stream);
-
-/* W4A8 GEMM with low-rank epilogue: y = bf16_rn( sum_k deq8(x) deq4(r) + u L2 + bias ).
+/* W4A8 GEMM with low-rank epilogue (W4A8 README, W4A8 format: MXFP4 residual times MXFP8
+ * activations plus the rank-32 correction):
+ *   y = bf16_rn( sum_k deq8(x) deq4(r) + u L2 + bias ).
  *   r_codes, r_sf  (device) MXFP4-packed residual weight [N, K] (fp4_pack_weight);
  *                  r_codes must be 32-byte aligned
  *   u_pair         (device) [M, 2 * rank] bf16 from w4a8_quantize_act
- *   l2t_bf16       (device) [N, rank] bf16 from w4a8_pack_lowrank_up
+ *   l2_bf16        (device) [rank, N] bf16, the low-rank up-projection (proj_up) as stored,
+ *                  row-major; read as it is, with no packing step
+ *   bias_f16       (device) [N] fp16 or NULL;  y_bf16 (device, out) [M, N] bf16
  * The low-rank product is accumulated on the tensor core into the same fp32 accumulator,
  * as (u_hi L2 + u_lo L2), before the bias and the bf16 rounding. */
 fp4_status_t w4a8_gemm(const uint8_t* x_e4m3, const uint8_t* x_sf, const void* u_pair, int64_t M,
                        int64_t K, int64_t N, const uint8_t* r_codes, const uint8_t* r_sf,
-                       const void* l2t_bf16, int rank, const void* bias_f16, void* y_bf16,
+                       const void* l2_bf16, int rank, const void* bias_f16, void* y_bf16,
                        void* stream);
 
-/* The full W4A8 SVDQuant linear: w4a8_quantize_act into `workspace` (with few rows, u = x L1
- * split over K into the workspace's partial sums, added in a fixed order), then w4a8_gemm.
- * l2t_bf16 is the packed [N, rank] up-projection; rank must be 32. */
+/* The full W4A8 SVDQuant linear (W4A8 README, opening paragraph and W4A8 format):
+ * w4a8_quantize_act into `workspace` (with few rows, u = x L1 split over K into the
+ * workspace's partial sums, added in a fixed order), then w4a8_gemm.
+ *   x_bf16 [M, K]; r_codes, r_sf: the MXFP4 residual [N, K]; l1_bf16 [K, rank] (proj_down,
+ *   1/s folded in); l2_bf16 [rank, N] (proj_up); rank must be 32; bias [N] fp16 or NULL;
+ *   workspace of at least w4a8_workspace_bytes(M, K, N, rank) bytes. */
 fp4_status_t w4a8_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N,
                              const uint8_t* r_codes, const uint8_t* r_sf, const void* l1_bf16,
-                             const void* l2t_bf16, int rank, const void* bias_f16, void* y_bf16,
+                             const void* l2_bf16, int rank, const void* bias_f16, void* y_bf16,
                              void* workspace, size_t ws_bytes, void* stream);
 
 /* ----------------------------------------------------------------- W4A4 SVDQuant */
@@ -281,16 +298,16 @@ fp4_status_t w4a4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const v
 /* W4A4 SVDQuant GEMM: MXFP4 x MXFP4 block-scaled main loop plus the tensor-core low-rank
  * stage (u_hi L2 + u_lo L2) into the same fp32 accumulator, + bias, bf16 out.
  *   r_codes, r_sf  MXFP4-packed residual [N, K] (fp4_pack_weight)
- *   l2t_bf16       packed [N, rank] up-projection (w4a8_pack_lowrank_up) */
+ *   l2_bf16        [rank, N] bf16 up-projection, as stored */
 fp4_status_t w4a4_gemm(const uint8_t* x_codes, const uint8_t* x_sf, const void* u_pair, int64_t M,
                        int64_t K, int64_t N, const uint8_t* r_codes, const uint8_t* r_sf,
-                       const void* l2t_bf16, int rank, const void* bias_f16, void* y_bf16,
+                       const void* l2_bf16, int rank, const void* bias_f16, void* y_bf16,
                        void* stream);
 
 /* The full W4A4 SVDQuant linear: w4a4_quantize_act into `workspace`, then w4a4_gemm. */
 fp4_status_t w4a4_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N,
                              const uint8_t* r_codes, const uint8_t* r_sf, const void* l1_bf16,
-                             const void* l2t_bf16, int rank, const void* bias_f16, void* y_bf16,
+                             const void* l2_bf16, int rank, const void* bias_f16, void* y_bf16,
                              void* workspace, size_t ws_bytes, void* stream);
 
 /* ----------------------------------------------------------------- status */

@@ -100,9 +100,6 @@ def test_invalid_calls_rejected_before_launch(fb):
     # W4A8: rank must be 32
     assert L.w4a8_svd_linear(A, 16, 256, 256, A, A, A, A, 16, None, A, A, 1 << 30, st) == 1
     assert L.w4a8_gemm(A, A, A, 16, 256, 384, A, A, A, 32, None, bad, st) == 3
-    assert L.w4a8_pack_lowrank_up(A, 384, 16, A, st) == 1
-    assert L.w4a8_pack_lowrank_up(A, 200, 32, A, st) == 2
-    assert L.w4a8_pack_lowrank_up(bad, 384, 32, A, st) == 3
     # W4A4 SVDQuant: rank, shape, alignment, workspace
     assert L.w4a4_svd_linear(A, 16, 256, 256, A, A, A, A, 16, None, A, A, 1 << 30, st) == 1
     assert L.w4a4_gemm(A, A, A, 16, 256, 200, A, A, A, 32, None, A, st) == 2

@@ -147,6 +147,13 @@ FULL = [
     (2, NV, 75600, 5120, 13824, "lognormal"),    # ffn up, NVFP4
     (2, NV, 75600, 13824, 5120, "gelu"),         # ffn down, NVFP4
     (4, MX, 512, 5120, 5120, "lognormal"),       # attn2 k/v on 512 text tokens
+    # the rest of the Wan2.2 block's ten linears in both formats
+    (4, NV, 75600, 5120, 5120, "lognormal"),     # attn1 q/k/v/out, attn2 q/out, NVFP4
+    (4, NV, 512, 5120, 5120, "lognormal"),       # attn2 k/v on 512 text tokens, NVFP4
+    (4, MX, 75600, 13824, 5120, "gelu"),         # ffn down, MXFP4
+    # the M sweep at 5120 -> 13824 (512 and 4096 are checked on every element below)
+    (4, MX, 16384, 5120, 13824, "lognormal"),
+    (4, NV, 16384, 5120, 13824, "lognormal"),
 ]
 
 
@@ -164,6 +171,25 @@ def test_linear_full_size_sampled(fb, orc, cfg, fmt, M, K, N, kind):
     rows = H.sample_rows(M, n_random=40, seed=cfg)
     Y, S = _oracle(orc, fmt, x, w, b, rows, g_a)
     H.check_linear(y, Y, S, rows, f"full cfg={cfg} fmt={fmt} M={M} K={K} N={N}")
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
+@pytest.mark.parametrize("M", [512, 4096])
+def test_linear_m_sweep_every_element(fb, orc, fmt, M):
+    """The M sweep's smaller points at 5120 -> 13824, every element of Y against the oracle."""
+    K, N = 5120, 13824
+    s = synth.seeds_for(4, layer=K // 1000 + N // 1000)
+    x = synth.activation(s["x"] + M, M, K, "lognormal", gain_seed=s["gain"])
+    w = synth.weight(s["w"], N, K)
+    b = synth.bias(s["bias"], N)
+    g_a = None
+    if fmt == NV:
+        cal = synth.activation(s["calib"], synth.CALIB_TOKENS, K, "lognormal", gain_seed=s["gain"])
+        g_a = orc.nv_global(orc.tensor_amax(cal))
+    y = _run_linear(fb, fmt, x, w, b, g_a)
+    rows = np.arange(M)
+    Y, S = _oracle(orc, fmt, x, w, b, rows, g_a)
+    H.check_linear(y, Y, S, rows, f"M sweep fmt={fmt} M={M} every element")
 
 
 # ------------------------------------------------------------------ bounded waits
@@ -204,19 +230,14 @@ def _w4a8_check(fb, orc, M, K, N, seed, rows=None, calib=256):
     x = synth.activation(seed + 1, M, K, "lognormal", gain_seed=seed + 5)
     b = synth.bias(seed + 2, N)
     rp = fb.pack_weight(H.dev_bf16(f["r_bf16"]), MX)
-    l2t = fb.pack_lowrank_up(H.dev_bf16(f["l2_bf16"]))
-    y = fb.w4a8_linear(H.dev_bf16(x), rp, H.dev_bf16(f["l1_bf16"]), l2t, H.dev_f16(b))
+    y = fb.w4a8_linear(H.dev_bf16(x), rp, H.dev_bf16(f["l1_bf16"]), H.dev_bf16(f["l2_bf16"]), H.dev_f16(b))
     st = fb.fp4_sync_status()
     assert st == 0, fb.fp4_status_string(st)
     torch.cuda.synchronize()
     rows = np.arange(M) if rows is None else rows
-    xe, xs = orc.quantize_mxfp8(np.ascontiguousarray(x[rows]))
-    a = orc.dequant_mxfp8(xe, xs, K)
     rc, rs, _ = orc.pack_weight(MX, f["r_bf16"])
-    w = orc.dequant_fp4(MX, rc, rs, K)
-    Y, S = orc.linear_fp64(a, w, b)
-    LR, LS = orc.lowrank_fp64(x, rows, f["l1_bf16"], f["l2_bf16"])
-    return H.check_linear(y, Y + LR, S + LS, rows, f"w4a8 M={M} K={K} N={N}")
+    Y, S = orc.svd_linear_rows("mxfp8", x, (rc, rs), f["l1_bf16"], f["l2_bf16"], b, rows)
+    return H.check_linear(y, Y, S, rows, f"w4a8 M={M} K={K} N={N}")
 
 
 # 8300 rows (65 blocks of 128): the activation side runs as one quantize + project pass
@@ -293,19 +314,14 @@ def _w4a4_check(fb, orc, M, K, N, seed, rows=None, calib=256):
     x = synth.activation(seed + 1, M, K, "lognormal", gain_seed=seed + 5)
     b = synth.bias(seed + 2, N)
     rp = fb.pack_weight(H.dev_bf16(f["r_bf16"]), MX)
-    l2t = fb.pack_lowrank_up(H.dev_bf16(f["l2_bf16"]))
-    y = fb.w4a4_linear(H.dev_bf16(x), rp, H.dev_bf16(f["l1_bf16"]), l2t, H.dev_f16(b))
+    y = fb.w4a4_linear(H.dev_bf16(x), rp, H.dev_bf16(f["l1_bf16"]), H.dev_bf16(f["l2_bf16"]), H.dev_f16(b))
     st = fb.fp4_sync_status()
     assert st == 0, fb.fp4_status_string(st)
     torch.cuda.synchronize()
     rows = np.arange(M) if rows is None else rows
-    xc, xs = orc.quantize(MX, np.ascontiguousarray(x[rows]))
-    a = orc.dequant_fp4(MX, xc, xs, K)
     rc, rs, _ = orc.pack_weight(MX, f["r_bf16"])
-    w = orc.dequant_fp4(MX, rc, rs, K)
-    Y, S = orc.linear_fp64(a, w, b)
-    LR, LS = orc.lowrank_fp64(x, rows, f["l1_bf16"], f["l2_bf16"])
-    return H.check_linear(y, Y + LR, S + LS, rows, f"w4a4 M={M} K={K} N={N}")
+    Y, S = orc.svd_linear_rows("mxfp4", x, (rc, rs), f["l1_bf16"], f["l2_bf16"], b, rows)
+    return H.check_linear(y, Y, S, rows, f"w4a4 M={M} K={K} N={N}")
 
 
 @pytest.mark.parametrize("M,K,N", [(1, 256, 256), (130, 512, 384), (300, 1024, 512), (8300, 256, 256)])
