@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads timed after the headline (NVFP4, fused FFN, W4A8, text tokens)")
     ap.add_argument("--gemm-ctas", type=int, default=0, choices=[0, 1, 2],
                     help="GEMM kernel: 0 auto (2-CTA 256x256 tile for M > 128), 1 force the 1-CTA 128x256 tile, 2 force 2-CTA")
     ap.add_argument("--fmt", default="mxfp4", choices=["mxfp4", "nvfp4"])
@@ -141,17 +143,29 @@ def make_inputs(rank: int, m: int | None = None, k: int | None = None, n: int | 
     return x, w, b
 
 
-def nv_static_global(k: int | None = None) -> float:
-    """NVFP4 activation global of the layer, calibrated once (untimed) on a separate
-    4096-token batch: its tensor amax T over the largest E2M1 x E4M3 product, T / 2688 in
-    fp32 (1 if T = 0)."""
+def nv_calibration_batch(k: int | None = None):
+    """The layer's NVFP4 calibration batch: 4096 tokens from a separate seed, same gains."""
     import synth
 
     k = K if k is None else k
     s = synth.seeds_for(4, layer=1)
-    cal = synth.activation(s["x"] + 104729, 4096, k, "lognormal", gain_seed=s["gain"])
-    t = np.float32(np.max(np.abs(synth.bf16_bits_to_f32(cal))))
-    return float(t / np.float32(2688.0)) if t > 0 else 1.0
+    return synth.activation(s["x"] + 104729, 4096, k, "lognormal", gain_seed=s["gain"])
+
+
+def nv_static_global(fb, torch, k: int | None = None):
+    """NVFP4 static activation global of the layer (device fp32 [1]), calibrated once,
+    untimed, by the library's fp4_calibrate_act_global on the calibration batch."""
+    cal = to_dev(nv_calibration_batch(k), torch, torch.bfloat16)
+    g, _ = fb.calibrate_act_global(cal)
+    torch.cuda.synchronize()
+    return g
+
+
+def oracle_static_global(k: int | None = None) -> float:
+    """The same global by the CPU oracle (for the oracle-timing legs)."""
+    import oracle
+
+    return oracle.nv_global(oracle.tensor_amax(nv_calibration_batch(k)))
 
 
 def max_over_ranks(x: float, dist=None, device="cuda") -> float:
@@ -168,6 +182,35 @@ def max_over_ranks(x: float, dist=None, device="cuda") -> float:
 def job_tflops(flop_per_rank_step: float, world: int, steps: int, slowest_ms: float) -> float:
     """Whole-job throughput: the work of all ranks over the slowest rank's timed region."""
     return flop_per_rank_step * world * steps / (slowest_ms / 1e3) / 1e12
+
+
+def config_dict(gpus: int) -> dict:
+    """The workload's config, identical in both arms."""
+    return {"workload": WORKLOAD, "M": M, "K": K, "N": N, "fmt": FMT, "tokens_per_gpu": M,
+            "parallelism": f"dp{gpus} (independent batches)" if gpus > 1 else "single GPU",
+            "l2": "inputs larger than L2 (X 774 MB, Y 2.09 GB), no flush"}
+
+
+def probe_clocks(fb, torch, blocks: int = 1024):
+    """Record (SM id, SM cycle counter, ns timer) from `blocks` tiny blocks on the current stream."""
+    buf = torch.zeros(3 * blocks, dtype=torch.int64, device="cuda")
+    fb.fp4bsa_clock_probe(buf, blocks)
+    return buf
+
+
+def probe_mhz(before, after):
+    """Median over SMs of each SM's average clock between two probes (cycles / ns), in MHz."""
+    b = before.view(-1, 3).cpu().numpy()
+    a = after.view(-1, 3).cpu().numpy()
+    first = {}
+    for sm, c, t in b:
+        first.setdefault(int(sm), (int(c), int(t)))
+    last = {}
+    for sm, c, t in a:
+        last[int(sm)] = (int(c), int(t))
+    f = [(last[sm][0] - c0) / (last[sm][1] - t0) * 1e3 for sm, (c0, t0) in first.items()
+         if sm in last and last[sm][1] > t0]
+    return (float(statistics.median(f)), len(f)) if f else (None, 0)
 
 
 def to_dev(bits, torch, dt):
@@ -207,7 +250,7 @@ def cpu_baseline(x_bits, w_bits, b_bits, target_s: float = 15.0):
     import oracle
 
     f = oracle.MX if FMT == "mxfp4" else oracle.NV
-    g_a = nv_static_global() if f == oracle.NV else 1.0
+    g_a = oracle_static_global() if f == oracle.NV else 1.0
     wc, ws, g_w = oracle.pack_weight(f, w_bits)                 # offline step, untimed
     w_deq = oracle.dequant_fp4(f, wc, ws, K, g_w or 1.0)        # once, untimed
 
@@ -244,7 +287,7 @@ def reference_arm(args):
     w = synth.weight(s["w"], N, K)
     b = synth.bias(s["bias"], N)
     f = oracle.MX if FMT == "mxfp4" else oracle.NV
-    g_a = nv_static_global() if f == oracle.NV else 1.0
+    g_a = oracle_static_global() if f == oracle.NV else 1.0
     wc, ws, g_w = oracle.pack_weight(f, w)
     w_deq = oracle.dequant_fp4(f, wc, ws, K, g_w or 1.0)
     # one step = the quantized linear for a bounded row sample of the workload
@@ -278,13 +321,128 @@ def reference_arm(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / max(args.steps, 1) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "fmt": FMT},
+        "data": "synthetic", "config": config_dict(args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ----------------------------------------------------------------------------- other workloads
+def extra_workloads(fb, torch, args, steps: int = 20, warmup: int = 3):
+    """The other Wan2.2 / TI2V-5B configurations of the path, each timed on its own after the
+    headline (CUDA events on the launching stream, inputs resident in HBM and larger than L2
+    except the text-token and W4A8 shapes).  Inputs are seeded synthetic tensors drawn on the
+    device with the workload's distributions: x ~ N(0,1) times a per-channel lognormal(0,1)
+    gain, weights ~ N(0, 0.02), bias ~ N(0, 0.01); the fused FFN's z is the up projection's own
+    output; the W4A8 factors are N(0, 0.02) residual and N(0, 0.05) low-rank factors (timing
+    does not depend on how they were obtained)."""
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(20261202)
+    stream = torch.cuda.current_stream()
+
+    def act(m, k):
+        gain = torch.exp(torch.randn(k, generator=gen, device="cuda"))
+        return (torch.randn(m, k, generator=gen, device="cuda") * gain).to(torch.bfloat16)
+
+    def wgt(n, k, sd=0.02):
+        return (torch.randn(n, k, generator=gen, device="cuda") * sd).to(torch.bfloat16)
+
+    def bias(n):
+        return (torch.randn(n, generator=gen, device="cuda") * 0.01).to(torch.float16)
+
+    def timed(fn, flop, n=steps):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0 = probe_clocks(fb, torch)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        p1 = probe_clocks(fb, torch)
+        torch.cuda.synchronize()
+        st = fb.fp4_sync_status()
+        if st != 0:
+            raise RuntimeError(f"device status: {fb.fp4_status_string(st)}")
+        ms = e0.elapsed_time(e1) / n
+        mhz, _ = probe_mhz(p0, p1)
+        return {"ms": ms, "tflops": flop / (ms / 1e3) / 1e12,
+                "pct_nominal": 100.0 * flop / (ms / 1e3) / 1e12 / (NOMINAL_FP4_TFLOPS if flop else 1),
+                "sm_mhz_in_kernel": mhz}
+
+    out = {}
+    Mx, Kx, Nx = 75600, 5120, 13824
+    x = act(Mx, Kx)
+    b_up = bias(Nx)
+    # NVFP4 ffn up projection (quantize + GEMM), static activation global from a separate batch
+    ga, _ = fb.calibrate_act_global(act(4096, Kx))
+    pw_nv = fb.pack_weight(wgt(Nx, Kx), "nvfp4")
+    y = torch.empty((Mx, Nx), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(fb.fp4_linear_workspace_bytes("nvfp4", Mx, Kx, Nx), dtype=torch.uint8, device="cuda")
+    out["nvfp4_ffn_up_75600x5120x13824"] = timed(
+        lambda: fb.fp4_linear("nvfp4", x, Mx, Kx, Nx, pw_nv.codes, pw_nv.sf, pw_nv.w_global, ga, b_up, y, ws,
+                              ws.numel()), 2.0 * Mx * Kx * Nx)
+    # the fused FFN activation: up projection + GELU-tanh + the down projection's quantize
+    for fmt in ("mxfp4", "nvfp4"):
+        pw = pw_nv if fmt == "nvfp4" else fb.pack_weight(wgt(Nx, Kx), "mxfp4")
+        hc = torch.empty((Mx, Nx // 2), dtype=torch.uint8, device="cuda")
+        hs = torch.empty(fb.fp4_sf_bytes(fmt, Mx, Nx), dtype=torch.uint8, device="cuda")
+        hg = torch.tensor([0.01], device="cuda") if fmt == "nvfp4" else None
+        a_g = ga if fmt == "nvfp4" else None
+        out[f"{fmt}_ffn_up_gelu_quant_75600x5120x13824"] = timed(
+            lambda: fb.fp4_linear_gelu_quant(fmt, x, Mx, Kx, Nx, pw.codes, pw.sf, pw.w_global, a_g, b_up, hg, hc,
+                                             hs, ws, ws.numel()), 2.0 * Mx * Kx * Nx)
+        del hc, hs
+    del y, pw_nv
+    # MXFP4 attention projection (75600 x 5120 -> 5120) and the text-token k/v (512 rows)
+    pw_a = fb.pack_weight(wgt(5120, 5120), "mxfp4")
+    b_a = bias(5120)
+    ya = torch.empty((Mx, 5120), dtype=torch.bfloat16, device="cuda")
+    out["mxfp4_attn_75600x5120x5120"] = timed(
+        lambda: fb.fp4_linear("mxfp4", x, Mx, 5120, 5120, pw_a.codes, pw_a.sf, None, None, b_a, ya, ws,
+                              ws.numel()), 2.0 * Mx * 5120 * 5120)
+    del ya, x
+    xt = act(512, 5120)
+    yt = torch.empty((512, 5120), dtype=torch.bfloat16, device="cuda")
+    wst = torch.empty(fb.fp4_linear_workspace_bytes("mxfp4", 512, 5120, 5120), dtype=torch.uint8, device="cuda")
+    call_t = lambda: fb.fp4_linear("mxfp4", xt, 512, 5120, 5120, pw_a.codes, pw_a.sf, None, None, b_a, yt, wst,
+                                   wst.numel())
+    out["mxfp4_text_kv_512x5120x5120_eager"] = timed(call_t, 2.0 * 512 * 5120 * 5120, n=200)
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        call_t()
+    side.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        call_t()
+    out["mxfp4_text_kv_512x5120x5120_graph"] = timed(graph.replay, 2.0 * 512 * 5120 * 5120, n=200)
+    del graph
+    # W4A8 SVDQuant linear at the TI2V-5B shape (MXFP8 activations, rank 32)
+    Mw, Kw, Nw, r = 4290, 3072, 14336, 32
+    xw = act(Mw, Kw)
+    rp = fb.pack_weight(wgt(Nw, Kw), "mxfp4")
+    l1 = wgt(Kw, r, 0.05)
+    l2 = wgt(r, Nw, 0.05)
+    bw = bias(Nw)
+    yw = torch.empty((Mw, Nw), dtype=torch.bfloat16, device="cuda")
+    wsw = torch.empty(fb.w4a8_workspace_bytes(Mw, Kw, Nw, r), dtype=torch.uint8, device="cuda")
+    flop_w = 2.0 * Mw * Kw * Nw + 2.0 * Mw * Kw * r + 2.0 * Mw * r * Nw
+    out["w4a8_svd_linear_4290x3072x14336"] = timed(
+        lambda: fb.w4a8_svd_linear(xw, Mw, Kw, Nw, rp.codes, rp.sf, l1, l2, r, bw, yw, wsw, wsw.numel()), flop_w,
+        n=100)
+    wsw4 = torch.empty(fb.w4a4_workspace_bytes(Mw, Kw, Nw, r), dtype=torch.uint8, device="cuda")
+    out["w4a4_svd_linear_4290x3072x14336"] = timed(
+        lambda: fb.w4a4_svd_linear(xw, Mw, Kw, Nw, rp.codes, rp.sf, l1, l2, r, bw, yw, wsw4, wsw4.numel()), flop_w,
+        n=100)
+    for k, v in out.items():
+        v["note"] = "pct_nominal: of 9 PFLOP/s dense FP4" + (" (W4A8 runs at the FP8 rate, nominal 4.5)"
+                                                             if k.startswith("w4a8") else "")
+    return out
 
 
 # ----------------------------------------------------------------------------- native arm
@@ -312,8 +470,7 @@ def native_arm(args):
     bias = to_dev(b_bits, torch, torch.float16)
     pw = fb.pack_weight(to_dev(w_bits, torch, torch.bfloat16), FMT)
     # NVFP4: the layer's static activation global (device scalar), calibrated untimed
-    a_global = (torch.tensor([nv_static_global()], dtype=torch.float32, device="cuda")
-                if FMT == "nvfp4" else None)
+    a_global = nv_static_global(fb, torch) if FMT == "nvfp4" else None
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     ws_bytes = fb.fp4_linear_workspace_bytes(FMT, M, K, N)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
@@ -350,15 +507,18 @@ def native_arm(args):
         dist.barrier()
     torch.cuda.synchronize()
     w0 = time.time()
+    pr0 = probe_clocks(fb, torch)
     t_start.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t_end.record(stream)
+    pr1 = probe_clocks(fb, torch)
     torch.cuda.synchronize()
     w1 = time.time()
     if dist:
         dist.barrier()
     clk = clocks.stop(w0, w1)
+    clk["sm_mhz_in_kernel"], clk["sm_probed"] = probe_mhz(pr0, pr1)
     st = fb.fp4_sync_status()
     if st != 0:
         raise RuntimeError(f"device status after timing: {fb.fp4_status_string(st)}")
@@ -398,36 +558,51 @@ def native_arm(args):
     g_avg = sum(g_ms) / len(g_ms)
     q_avg = sum(q_ms) / len(q_ms)
     gemm_tflops = FLOP_PER_STEP / (g_avg / 1e3) / 1e12
-    # the GEMM is timed inside a long loop of steps (about a second at the power cap), so its
-    # denominator is the sustained measured peak; the burst fraction is reported beside it
-    fp4_peak = pk["bf16_tflops_sustained"] * FP4_PER_BF16
-    fp4_peak_burst = pk["bf16_tflops"] * FP4_PER_BF16
+    # denominator: the FP4 peak derived from the measured bf16 GEMM rate (x4, the nominal
+    # FP4 / BF16 ratio) -- its sustained figure only when this run's timed region itself
+    # lasted seconds under the power cap, else the burst figure
+    region_s = total_ms / 1e3
+    sustained = region_s >= 2.0 and "sw_power_cap" in (clk.get("reasons") or [])
+    bf16 = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    fp4_peak = bf16 * FP4_PER_BF16
+    # the tensor pipe's own rate: 32768 FP4 FLOP per clock per SM (a 256x256x64 block-scaled
+    # MMA every 128 cycles per SM pair), at the SM clock measured inside the timed region
+    sms = torch.cuda.get_device_properties(local).multi_processor_count
+    mhz = clk.get("sm_mhz_in_kernel")
+    pipe_frac = FLOP_PER_STEP / (g_avg / 1e3) / (mhz * 1e6 * 32768 * sms) if mhz else None
     q_bytes = 2 * M * K + M * K // 2 + ((M + 127) // 128 * 128) * (K // (32 if FMT == "mxfp4" else 16))
+    q_gbs = q_bytes / (q_avg / 1e3) / 1e9
     traffic = gemm_traffic(pair) if FMT == "mxfp4" else None  # counters recorded for MXFP4
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp4", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "fmt": FMT, "tokens_per_gpu": M,
-                   "parallelism": f"dp{world} (independent batches)" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (X 774 MB, Y 2.09 GB), no flush"},
+        "config": config_dict(args.gpus),
         "pct_nominal_fp4_peak": 100.0 * value / world / NOMINAL_FP4_TFLOPS,
         "roofline": {"bound": "tensor", "kernel": f"gemm2_kernel<{FMT.upper()}> (2-CTA 256x256)" if pair
                      else f"gemm_kernel<{FMT.upper()}> (1-CTA 128x256)", "achieved": gemm_tflops,
                      "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
-                     "peak_source": f"{pk_kind} bf16 sustained {pk['bf16_tflops_sustained']} x {FP4_PER_BF16:g} "
-                                    f"(nominal FP4/BF16; the GEMM runs inside a ~1 s loop of steps)",
-                     "frac_of_burst_peak": gemm_tflops / fp4_peak_burst,
+                     "peak_source": f"{pk_kind} bf16 {'sustained' if sustained else 'burst'} {bf16} x "
+                                    f"{FP4_PER_BF16:g} (nominal FP4/BF16); timed region {region_s:.3f} s, "
+                                    f"power cap {'seen' if 'sw_power_cap' in (clk.get('reasons') or []) else 'not seen'}",
+                     "frac_of_nominal_9pf": gemm_tflops / NOMINAL_FP4_TFLOPS,
+                     "tensor_pipe_frac_at_measured_clock": pipe_frac,
                      "traffic": traffic,
-                     "algorithmic_flop_per_launch": FLOP_PER_STEP, "avg_launch_ms": g_avg},
-        "kernels": {"quant_ms": q_avg, "quant_gbs": q_bytes / (q_avg / 1e3) / 1e9,
-                    "quant_hbm_frac": q_bytes / (q_avg / 1e3) / 1e9 / pk["hbm_gbs"], "gemm_ms": g_avg},
+                     "algorithmic_flop_per_launch": FLOP_PER_STEP, "avg_launch_ms": g_avg,
+                     "quant": {"bound": "hbm", "kernel": f"quant_kernel<{FMT.upper()}>", "achieved": q_gbs,
+                               "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": q_gbs / pk["hbm_gbs"],
+                               "algorithmic_bytes_per_launch": q_bytes, "avg_launch_ms": q_avg}},
+        "kernels": {"quant_ms": q_avg, "quant_gbs": q_gbs, "quant_hbm_frac": q_gbs / pk["hbm_gbs"], "gemm_ms": g_avg},
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": x_bits.nbytes,
                 "d2h_bytes_per_step": M * N * 2, "steps": args.e2e_steps},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }
+    if not args.no_extra and world == 1:
+        del x, y, ws, codes, sf
+        torch.cuda.empty_cache()
+        line["extra"] = extra_workloads(fb, torch, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(x_bits, w_bits, b_bits)
     if dist:

@@ -92,9 +92,10 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     assert capsys.readouterr().out == ""
 
 
-def test_nvfp4_bench_global_matches_the_oracle():
-    """bench.py --fmt nvfp4 calibrates the layer's static activation global on the host; it
-    must be the oracle's global of the same calibration batch."""
+def test_nvfp4_bench_oracle_global_is_the_calibration_batch_global():
+    """bench.py --fmt nvfp4: the oracle legs use the oracle's global of the same 4096-token
+    calibration batch that the native arm hands to fp4_calibrate_act_global (the native side
+    is checked bit for bit on the GPU in test_gpu_quant.py)."""
     import bench
     import oracle
     import synth
@@ -102,7 +103,8 @@ def test_nvfp4_bench_global_matches_the_oracle():
     k = 256
     s = synth.seeds_for(4, layer=1)
     cal = synth.activation(s["x"] + 104729, 4096, k, "lognormal", gain_seed=s["gain"])
-    assert bench.nv_static_global(k) == oracle.nv_global(oracle.tensor_amax(cal))
+    np.testing.assert_array_equal(bench.nv_calibration_batch(k), cal)
+    assert bench.oracle_static_global(k) == oracle.nv_global(oracle.tensor_amax(cal))
 
 
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
