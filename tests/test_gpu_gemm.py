@@ -48,6 +48,8 @@ def _oracle(orc, fmt, x_bits, w_bits, b_bits, rows, g_a=None):
 SMALL = [
     (1, 256, 256), (128, 256, 256), (129, 512, 384), (256, 512, 512), (300, 384, 640),
     (77, 1280, 1024), (513, 768, 256),
+    # K % 512 = 128 and K = 128: a last (or only) MXFP4 stage of two MMAs
+    (300, 640, 384), (260, 128, 256),
 ]
 
 
