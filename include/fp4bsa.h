@@ -75,18 +75,22 @@ typedef enum {
 
 /* ----------------------------------------------------------------- size queries (host) */
 
-/* Bytes of packed E2M1 codes for a [rows, K] operand: rows * K / 2.  0 if K is odd. */
+/* Bytes of packed E2M1 codes for a [rows, K] operand: rows * K / 2 (MXFP4 card, Quantization
+ * Details: two FP4 E2M1 values per byte).  0 if K is odd. */
 size_t fp4_codes_bytes(fp4_fmt_t fmt, int64_t rows, int64_t K);
 
 /* Bytes of the scale-factor buffer of a [rows, K] operand in the 128x4 atom layout:
- * ceil(rows/128)*128 * K/G (G = 32 MXFP4, 16 NVFP4).  0 on a bad fmt or K % 128 != 0. */
+ * ceil(rows/128)*128 * K/G (G = 32 MXFP4, one E8M0 per 32 values, MXFP4 card Quantization
+ * Details; G = 16 NVFP4, one E4M3 per 16 values, NVFP4 card Model Details).  0 on a bad fmt
+ * or K % 128 != 0. */
 size_t fp4_sf_bytes(fp4_fmt_t fmt, int64_t rows, int64_t K);
 
-/* Workspace fp4_linear needs: the quantized activation codes and scales, each
- * 256-byte aligned.  0 on invalid arguments. */
+/* Workspace fp4_linear needs: the dynamically quantized activations (MXFP4 card: act_dynamic;
+ * NVFP4 card: dynamic block scales), codes then scales, each 256-byte aligned.  0 on
+ * invalid arguments. */
 size_t fp4_linear_workspace_bytes(fp4_fmt_t fmt, int64_t M, int64_t K, int64_t N);
 
-/* Workspace w4a8_svd_linear needs: MXFP8 elements [M,K], their scales, the low-rank
+/* Workspace w4a8_svd_linear needs (W4A8 README, W4A8 format): MXFP8 elements [M,K], their scales, the low-rank
  * projection u = x L1 as its bf16 pair [M, 2 rank] and, when x has fewer than 64 blocks of
  * 128 rows, fp32 partial sums of u for a K-split projection; each 256-byte aligned. */
 size_t w4a8_workspace_bytes(int64_t M, int64_t K, int64_t N, int rank);
@@ -148,7 +152,9 @@ fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf
                       const float* w_global, const float* a_global, const void* bias_f16,
                       void* y_bf16, void* stream);
 
-/* The W4A4 quantized linear: fp4_quantize_act into `workspace`, then fp4_gemm.
+/* The W4A4 quantized linear, one call per linear layer (MXFP4 card, Quantization Details: the
+ * transformer blocks' linears run with W4A4 MXFP4; NVFP4 card, Model Details): fp4_quantize_act
+ * into `workspace`, then fp4_gemm.
  *   x_bf16     (device) [M, K] bf16
  *   workspace  (device) at least fp4_linear_workspace_bytes(fmt, M, K, N) bytes; its
  *              contents on return are the quantized activations (codes, then scales)
@@ -311,6 +317,9 @@ fp4_status_t w4a4_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N
                              void* workspace, size_t ws_bytes, void* stream);
 
 /* ----------------------------------------------------------------- status */
+
+/* The status calls below are part of this library's error model, not of the method: the
+ * model-card pages describe no library interface, so they have no counterpart there. */
 
 /* Synchronizes `stream`, then returns and clears the device status word of the current
  * GPU: FP4_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
