@@ -93,9 +93,9 @@ fp4_status_t device_state(DeviceState** out) {
                 cudaFuncSetAttribute(gemm2_kernel<G_SVD4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Gemm2Cfg<G_SVD4>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm2_kernel<G_MXFP4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     Gemm2Cfg<G_MXFP4>::SMEM_BYTES) != cudaSuccess ||
+                                     Gemm2Cfg<G_MXFP4, 1>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm2_kernel<G_NVFP4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     Gemm2Cfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess ||
+                                     Gemm2Cfg<G_NVFP4, 2>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm2_kernel<G_MXFP4, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Gemm2Cfg<G_MXFP4>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm2_kernel<G_NVFP4, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -357,7 +357,8 @@ template <int KIND, int OUTQ = 0, bool SK = false>
 fp4_status_t launch_gemm2(const DeviceState* ds, const CUtensorMap& ta, const CUtensorMap& tb, const uint8_t* sfa,
                           const uint8_t* sfb, GemmParams& p, cudaStream_t st, const CUtensorMap* tu = nullptr,
                           const CUtensorMap* tl = nullptr, bool pdl = false) {
-    using C = Gemm2Cfg<KIND>;
+    // the launch's shared-memory size is the kernel's own configuration (kind and output)
+    using C = Gemm2Cfg<KIND, OUTQ>;
     CUtensorMap tsa, tsb;
     fp4_status_t s;
     if ((s = encode_sf(&tsa, sfa, p.M, p.K, C::G, C::ATOMS)) != FP4_OK) return s;

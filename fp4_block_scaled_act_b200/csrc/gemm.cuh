@@ -377,15 +377,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // B atom a in row block rb, in every quarter q.  The tensor pipe then runs MMAs only, and
 // shared memory sees only the raw atoms.  Both CTAs hold the scales of all 256 B rows.
 // The writers load a stage's words before waiting for its TMEM buffer to be free, so only
-// the TMEM store and the arrive follow that wait.
+// the TMEM store and the arrive follow that wait.  A scale-ring slot goes back to the scale
+// producer only after the TMEM stores have consumed its words: handed back as soon as the
+// shared-memory loads were issued, a slot was refilled by the next TMA load before those
+// loads had read it whenever the writers then waited long for their TMEM buffer (the MMA
+// stalled behind the fused GELU epilogue), and stages ran with the wrong scales.
 //
-// Accumulators: two 256-column accumulators overlapping by 64 columns ([0,256),
-// [192,448)), or by 96 for NVFP4; the epilogue drains the shared columns first, so the
-// next tile's MMAs wait for that part only.  The scale buffers follow the second
-// accumulator.
+// Accumulators: two 256-column accumulators overlapping by 96 columns ([0,256),
+// [160,416)), or by 64 for the W4A8 kernel and the fused GELU epilogues ([192,448)); the
+// epilogue drains the shared columns first, so the next tile's MMAs wait for that part
+// only.  The TMEM scale buffers follow the second accumulator: four for the plain-output
+// kinds with two scale atoms per stage (MXFP4, W4A4 SVDQuant) and for W4A8 (one atom), two
+// for NVFP4 (four atoms) and for the fused GELU epilogues.
 //
-// Warps (512 threads, four warpgroups): 0 TMA producer, 1 TMEM owner + MMA issuer
-// (leader), 2 stage coordinator (leader), 3 idle, 4-7 scale writers, 8-15 epilogue.  The
+// Warps (512 threads, four warpgroups): 0 operand TMA producer, 1 TMEM owner + MMA issuer
+// (leader), 2 stage coordinator (leader), 3 scale TMA producer, 4-7 scale writers, 8-15
+// epilogue.  The
 // control warpgroups (0-7) drop to REG_LO registers per thread with setmaxnreg and the
 // epilogue warpgroups rise to REG_HI: the fused epilogues run without spilling, and an
 // NVFP4 overlap holder can copy its whole 128-column share before converting any.
@@ -395,8 +402,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // (bar.arrive / bar.sync), which does not touch shared memory.
 // Synchronization:
 //   full[s]      (leader)  A/B bytes of both CTAs; the leader alone expects them
-//   sf_full[s]   (local)   this CTA's raw scale atoms
 //   empty[s]     (both)    the leader's commit (MMAs of stage s done)
+//   sc_full[j]   (local)   this CTA's raw scale atoms in scale-ring slot j
+//   sc_empty[j]  (local)   slot j read by this CTA's 4 writer warps (separate scale ring;
+//                          NVFP4's scale slots ride in the operand ring and are recycled
+//                          with empty[s], loaded by the operand producer)
 //   sf_ready[t]  (leader)  scale buffer t written in both CTAs (8 writer warps)
 //   tmem_full[b] (both)    accumulator b complete
 //   acc_free[b]  (leader)  accumulator b fully drained by both CTAs (16 warps)
@@ -422,20 +432,31 @@ struct Gemm2Cfg {
     static constexpr int B_BYTES = 128 * ROW_BYTES;  // this CTA's half of the 256 B rows
     static constexpr int RSFA_BYTES = ATOMS * 512;    // raw atoms, this CTA's 128 A rows
     static constexpr int RSFB_BYTES = 2 * ATOMS * 512;  // raw atoms, all 256 B rows
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + RSFA_BYTES + RSFB_BYTES;
-    // Operand ring depth.  MXFP4 with 4 stages measured 13 % slower than with 5, and the
-    // same with 6 (interleaved, bit-identical output); W4A8 with 6 runs 1.5-3.5 % faster
-    // than with 5.  NVFP4's 6 KB of scale atoms per stage leave no room for a sixth.  With
-    // six stages the epilogue's per-warp Y staging tile is 32 x 32 bf16 (64-byte rows,
-    // 64-byte swizzle), else 32 x 64 (128-byte swizzle).
+    // Two rings.  The operand ring (A and B tiles of a stage) is refilled when the MMAs of
+    // the stage it held are done; the scale ring (the raw scale atoms of a stage) is
+    // refilled as soon as the scale writers have read a slot into registers, so the scale
+    // atoms run ahead of the operands and their slots cost no operand-ring space.
+    // Operand tiles arrive over a TMA path whose latency under this load (~2000 cycles,
+    // measured) makes the number of stages in flight the limit: the operand ring takes five
+    // stages (32 KB each), six for W4A8, whose epilogue's per-warp Y staging tile is then
+    // 32 x 32 bf16 (64-byte rows, 64-byte swizzle) to make room.
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int SC_BYTES = RSFA_BYTES + RSFB_BYTES;
+    // NVFP4 (four atoms per stage, two TMEM scale buffers) measured 10 % slower with the
+    // separate scale ring, so its scale atoms ride in the operand ring as before: the
+    // operand producer loads them with the stage's tiles (SC_STAGES == STAGES, slot s of the
+    // scale area belongs to operand stage s and is recycled with it).
+    static constexpr bool SEP_SC = (KIND != G_NVFP4);
     static constexpr int STAGES = (KIND == G_W4A8) ? 6 : 5;
+    static constexpr int SC_STAGES = SEP_SC ? 4 : STAGES;
     static constexpr int EPI_COLS = (STAGES == 6) ? 32 : 64;
     static constexpr int EPI_TILE = 32 * EPI_COLS * 2;
     static constexpr int EPI_BYTES = 8 * EPI_TILE;
     // the dynamic shared array is declared 1024-byte aligned (checked at run time), so the
     // layout needs no alignment slack
     // + barriers; NVFP4 also keeps the fused epilogue's 128-entry reciprocal table after them
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 512 + (KIND == G_NVFP4 ? 512 : 0);
+    static constexpr int SMEM_BYTES =
+        STAGES * STAGE_BYTES + EPI_BYTES + SC_STAGES * SC_BYTES + 512 + (KIND == G_NVFP4 ? 512 : 0);
     static constexpr uint32_t AB_TX = A_BYTES + ((KIND == G_W4A8) ? B_BYTES / 2 : B_BYTES);
     static constexpr uint32_t SF_TX = RSFA_BYTES + RSFB_BYTES;
     // TMEM columns: two accumulators overlapping by OVL columns, the shared columns drained
@@ -445,7 +466,12 @@ struct Gemm2Cfg {
     // plain bf16 output (HOLD_ALL) its holders copy all four chunks to registers before
     // converting any, so the overlap is released after the copy rather than after a pair
     // has been written; the fused epilogues need those registers for their arithmetic.
-    static constexpr int ACC1_COL = (KIND == G_NVFP4) ? 160 : 192;
+    // The plain-output MXFP4 and W4A4 SVDQuant kernels (two atoms, 24 columns per scale
+    // buffer) overlap by 96 too, which leaves room for four scale buffers: the writers then
+    // refill a buffer four stages after its MMAs were issued rather than two.  The fused
+    // GELU epilogues keep a 64-column overlap (their holders convert before releasing it)
+    // and two buffers; W4A8 (one atom, 12 columns) fits four buffers beside a 64 overlap.
+    static constexpr int ACC1_COL = (KIND == G_NVFP4) ? 160 : (KIND == G_W4A8 || OUTQ != 0) ? 192 : 160;
     static constexpr int SF_COL0 = ACC1_COL + 256;
     static constexpr int OVL = 256 - ACC1_COL;
     static constexpr bool HOLD_ALL = (OUTQ == 0) && (OVL > 64);
@@ -640,22 +666,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
     extern __shared__ __align__(1024) uint8_t smem2_raw[];
     // 128-byte-swizzled operand tiles need 1024-byte alignment; both CTAs see the same
     // layout, so both leave here together, before any barrier
-    if ((smem_u32(smem2_raw) & 1023u) != 0) {
+    // and the launch must have provided the whole layout: a kernel launched with less
+    // dynamic shared memory than its configuration needs writes nothing and reports it
+    uint32_t dyn_smem;
+    asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_smem));
+    if ((smem_u32(smem2_raw) & 1023u) != 0 || dyn_smem < (uint32_t)C::SMEM_BYTES) {
         if (threadIdx.x == 0) atomicCAS(p.status, 0, STATUS_LAYOUT);
         return;
     }
     uint8_t* sA = smem2_raw;
     uint8_t* sB = sA + S * C::A_BYTES;
     uint8_t* sEpi = sB + S * C::B_BYTES;                  // 8 per-warp Y staging tiles
-    uint8_t* sRSFA = sEpi + C::EPI_BYTES;
-    uint8_t* sRSFB = sRSFA + S * C::RSFA_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sRSFB + S * C::RSFB_BYTES);
+    uint8_t* sSC = sEpi + C::EPI_BYTES;                   // scale ring: per slot A atoms, then B atoms
+    constexpr int SJ = C::SC_STAGES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sSC + SJ * C::SC_BYTES);
     // fused NVFP4 epilogue: reciprocals of the decoded scales, 128 floats after the barriers
     float* rcp_tab = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 512);
     uint64_t* full = bars;
-    uint64_t* sf_full = full + S;
-    uint64_t* empty = sf_full + S;
-    uint64_t* sf_ready = empty + S;                       // [TB]
+    uint64_t* empty = full + S;
+    uint64_t* sc_full = empty + S;                        // [SJ] scale ring slot loaded (local)
+    uint64_t* sc_empty = sc_full + SJ;                    // [SJ] scale ring slot read by the 4 writers (local)
+    uint64_t* sf_ready = sc_empty + SJ;                   // [TB]
     uint64_t* tmem_full = sf_ready + TB;                  // [2]
     uint64_t* acc_free = tmem_full + 2;                   // [2]
     uint64_t* ovl_free = acc_free + 2;
@@ -671,8 +702,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&sf_full[s], 1);
             mbar_init(&empty[s], 1);
+        }
+        for (int j = 0; j < SJ; ++j) {
+            mbar_init(&sc_full[j], 1);
+            mbar_init(&sc_empty[j], 4);
         }
         for (int t = 0; t < TB; ++t) mbar_init(&sf_ready[t], 8);
         for (int b = 0; b < 2; ++b) {
@@ -937,10 +971,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                         // A/B of both CTAs land on the leader's barrier; only the leader expects them
                         const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
                         if (HAS_LR && kb == num_kb) {
-                            // low-rank stage: u pair rows and packed-L2 rows; no scale atoms, but
-                            // sf_full still completes a phase so its parity keeps counting stages
+                            // low-rank stage: u pair rows and the L2 columns
                             if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::LR_TX);
-                            mbar_arrive(&sf_full[s]);
                             tma_load_2d_pair(sA + s * C::A_BYTES, &tmU, bar, 0, mb * 256 + (int)rank * 128, pol_a);
                             // L2 [32][N]: this CTA's 128 columns as two 64-column boxes of 32 rows
                             tma_load_2d_pair(sB + s * C::B_BYTES, &tmL, bar, nb * 256 + (int)rank * 128, 0, pol_b);
@@ -949,29 +981,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                             continue;
                         }
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::AB_TX);
-                        mbar_arrive_expect_tx(&sf_full[s], C::SF_TX);
                         // x: bytes of the row for packed FP4 and E4M3, elements for the W4A8 unpacking map
                         const int ax = kb * C::ROW_BYTES;
                         const int bx = (KIND == G_W4A8) ? kb * C::BK : kb * C::ROW_BYTES;
                         tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, bar, ax, mb * 256 + (int)rank * 128, pol_a);
                         tma_load_2d_pair(sB + s * C::B_BYTES, &tmB, bar, bx, nb * 256 + (int)rank * 128, pol_b);
-                        tma_load_2d(sRSFA + s * C::RSFA_BYTES, &tmSFA, &sf_full[s], 0,
-                                    (mb * 2 + (int)rank) * apr + kb * C::ATOMS, pol_a);
+                        if constexpr (!C::SEP_SC) {
+                            // this CTA's raw scale atoms of the stage, into the stage's scale slot
+                            uint8_t* slot = sSC + s * C::SC_BYTES;
+                            mbar_arrive_expect_tx(&sc_full[s], C::SF_TX);
+                            tma_load_2d(slot, &tmSFA, &sc_full[s], 0, (mb * 2 + (int)rank) * apr + kb * C::ATOMS, pol_a);
     #pragma unroll
-                        for (int j = 0; j < 2; ++j)
-                            tma_load_2d(sRSFB + s * C::RSFB_BYTES + j * C::ATOMS * 512, &tmSFB, &sf_full[s], 0,
-                                        (nb * 2 + j) * apr + kb * C::ATOMS, pol_b);
+                            for (int r = 0; r < 2; ++r)
+                                tma_load_2d(slot + C::RSFA_BYTES + r * C::ATOMS * 512, &tmSFB, &sc_full[s], 0,
+                                            (nb * 2 + r) * apr + kb * C::ATOMS, pol_b);
+                        }
                     }
                     sc.step(kb0, kb1);
                 }
-                // drain what this CTA issued: its scale loads, and (leader) both CTAs' A/B
+                // drain what was issued into this pair's ring: (leader) both CTAs' A/B, and the
+                // scale atoms when they ride in the operand ring
                 for (int j = max(0, it - S); j < it; ++j) {
                     if (j == p.skip_iter) continue;
-                    if (!mbar_wait_drain(&sf_full[j % S], (uint32_t)(j / S) & 1u, p.timeout_ns))
+                    if (!C::SEP_SC && !mbar_wait_drain(&sc_full[j % S], (uint32_t)(j / S) & 1u, p.timeout_ns))
                         gemm2_fail(p, abort, peer_abort);
                     if (rank == 0 && !mbar_wait_drain(&full[j % S], (uint32_t)(j / S) & 1u, p.timeout_ns))
                         gemm2_fail(p, abort, peer_abort);
                 }
+            }
+        } else if (warp == 3) {
+            // ============================================================ scale producer (both CTAs)
+            // This CTA's raw scale atoms of every stage into the scale ring; a slot is reused
+            // once the four writer warps have read it.  The W4A8 / W4A4 SVDQuant low-rank stage
+            // has no scales: its slot turn completes with a plain arrive, so the ring counters
+            // stay in step with the stages.
+            if (C::SEP_SC && lane == 0) {
+                griddep_wait();
+                const uint64_t pol_a = policy_evict_normal();
+                const uint64_t pol_b = policy_evict_last();
+                int it = 0;
+                bool ok = true;
+                Sched sc = sched0;
+                sc.begin();
+                int tile, kb0, kb1;
+                while (ok && sc.get(tile, kb0, kb1)) {
+                    const int mb = tile / num_n, nb = tile % num_n;
+                    for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
+                        const int j = it % SJ;
+                        if (!mbar_wait(&sc_empty[j], ((uint32_t)(it / SJ) & 1u) ^ 1u, p.timeout_ns, abort)) {
+                            gemm2_fail(p, abort, peer_abort);
+                            ok = false;
+                            break;
+                        }
+                        if (HAS_LR && kb == num_kb) {
+                            mbar_arrive(&sc_full[j]);
+                            continue;
+                        }
+                        uint8_t* slot = sSC + j * C::SC_BYTES;
+                        mbar_arrive_expect_tx(&sc_full[j], C::SF_TX);
+                        tma_load_2d(slot, &tmSFA, &sc_full[j], 0, (mb * 2 + (int)rank) * apr + kb * C::ATOMS, pol_a);
+    #pragma unroll
+                        for (int r = 0; r < 2; ++r)
+                            tma_load_2d(slot + C::RSFA_BYTES + r * C::ATOMS * 512, &tmSFB, &sc_full[j], 0,
+                                        (nb * 2 + r) * apr + kb * C::ATOMS, pol_b);
+                    }
+                    sc.step(kb0, kb1);
+                }
+                // drain this CTA's scale loads still in flight
+                for (int q = max(0, it - SJ); q < it; ++q)
+                    if (!mbar_wait_drain(&sc_full[q % SJ], (uint32_t)(q / SJ) & 1u, p.timeout_ns))
+                        gemm2_fail(p, abort, peer_abort);
             }
         } else if (warp >= 4) {
             // ============================================================ scale writers (both CTAs)
@@ -984,16 +1063,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
             int tile, kb0, kb1;
             while (ok && sc.get(tile, kb0, kb1)) {
                 for (int kb = kb0; kb < kb1 + (HAS_LR ? 1 : 0); ++kb, ++it) {
-                    const int s = it % S;
+                    const int j = it % SJ;
                     const int t = it % TB;
-                    bool got = mbar_wait(&sf_full[s], (uint32_t)(it / S) & 1u, p.timeout_ns, abort);
+                    bool got = mbar_wait(&sc_full[j], (uint32_t)(it / SJ) & 1u, p.timeout_ns, abort);
                     if (!__all_sync(0xffffffffu, got)) {
                         if (lane == 0) gemm2_fail(p, abort, peer_abort);
                         ok = false;
                         break;
                     }
-                    const uint4* rsfa = reinterpret_cast<const uint4*>(sRSFA + s * C::RSFA_BYTES);
-                    const uint4* rsfb = reinterpret_cast<const uint4*>(sRSFB + s * C::RSFB_BYTES);
+                    const uint4* rsfa = reinterpret_cast<const uint4*>(sSC + j * C::SC_BYTES);
+                    const uint4* rsfb = reinterpret_cast<const uint4*>(sSC + j * C::SC_BYTES + C::RSFA_BYTES);
                     // lane i takes row i of every atom: words 0-3 = the scales of rows i, 32+i, 64+i, 96+i
                     uint32_t va[4 * C::ATOMS];
                     uint32_t vb[8 * C::ATOMS];
@@ -1015,6 +1094,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                         ok = false;
                         break;
                     }
+                    // order the TMEM stores after the MMAs that read the buffer (their commit,
+                    // observed through the mbarrier)
+                    tc_fence_after();
                     const uint32_t xa = C::SF_COL0 + (uint32_t)(t * C::SF_COLS);
                     const uint32_t xb = xa + C::SFA_COLS;
                     // the W4A8 low-rank stage reads no scales: its buffer turn passes unwritten
@@ -1034,6 +1116,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) arrive_leader_relaxed(&sf_ready[t], rank);
+                    // the slot's words have been consumed by the TMEM stores: hand the slot back
+                    // to the scale producer (a slot that rides in the operand ring is recycled
+                    // with its stage instead)
+                    if (C::SEP_SC && lane == 0) mbar_arrive(&sc_empty[j]);
                 }
                 sc.step(kb0, kb1);
             }

@@ -324,8 +324,8 @@ fp4_status_t w4a4_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N
 /* Synchronizes `stream`, then returns and clears the device status word of the current
  * GPU: FP4_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call,
  * FP4_ERR_ARCH if a GEMM kernel found its shared memory placed without the 1024-byte
- * alignment it is built for (it then wrote no output), FP4_ERR_CUDA if the
- * synchronization failed, FP4_OK otherwise. */
+ * alignment it is built for, or smaller than its layout (it then wrote no output),
+ * FP4_ERR_CUDA if the synchronization failed, FP4_OK otherwise. */
 fp4_status_t fp4_sync_status(void* stream);
 
 /* Static, human-readable name of a status code. */
