@@ -34,6 +34,7 @@ EXPORTS = [
     "fp4_set_wait_timeout_ns", "fp4_linear_noalloc",
     "w4a4_workspace_bytes", "w4a4_quantize_act", "w4a4_gemm", "w4a4_svd_linear",
     "fp4_gelu_quantize_act", "fp4_gemm_gelu_quant", "fp4_linear_gelu_quant", "fp4_calibrate_act_global",
+    "fp4_heads_codes_bytes", "fp4_heads_sf_bytes", "fp4_quantize_heads", "fp4_attn_scores",
 ]
 
 
@@ -77,6 +78,10 @@ def lib():
             "w4a4_svd_linear": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, P, SZ, P]),
             "w4a8_gemm": (I, [P, P, P, I64, I64, I64, P, P, P, I, P, P, P]),
             "w4a8_svd_linear": (I, [P, I64, I64, I64, P, P, P, P, I, P, P, P, SZ, P]),
+            "fp4_heads_codes_bytes": (SZ, [I, I64, I64, I64]),
+            "fp4_heads_sf_bytes": (SZ, [I, I64, I64, I64]),
+            "fp4_quantize_heads": (I, [I, P, I64, I64, I64, P, P, P, P]),
+            "fp4_attn_scores": (I, [I, P, P, I64, P, P, I64, I64, I64, I64, P, P, P, P]),
             "fp4_sync_status": (I, [P]),
             "fp4_status_string": (ctypes.c_char_p, [I]),
             "fp4_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
@@ -241,6 +246,25 @@ def w4a4_svd_linear(x, M: int, K: int, N: int, r_codes, r_sf, l1, l2, rank: int,
            "w4a4_svd_linear")
 
 
+def fp4_heads_codes_bytes(fmt, T: int, H: int, D: int = 128) -> int:
+    return lib().fp4_heads_codes_bytes(_fmt(fmt), T, H, D)
+
+
+def fp4_heads_sf_bytes(fmt, T: int, H: int, D: int = 128) -> int:
+    return lib().fp4_heads_sf_bytes(_fmt(fmt), T, H, D)
+
+
+def fp4_quantize_heads(fmt, x, T: int, H: int, D: int, g, codes, sf, stream=None):
+    _check(lib().fp4_quantize_heads(_fmt(fmt), _ptr(x), T, H, D, _ptr(g), _ptr(codes), _ptr(sf), _stream(stream)),
+           "fp4_quantize_heads")
+
+
+def fp4_attn_scores(fmt, q_codes, q_sf, T_q: int, k_codes, k_sf, T_kv: int, H: int, D: int, head: int, g_q, g_k,
+                    s, stream=None):
+    _check(lib().fp4_attn_scores(_fmt(fmt), _ptr(q_codes), _ptr(q_sf), T_q, _ptr(k_codes), _ptr(k_sf), T_kv, H, D,
+                                 head, _ptr(g_q), _ptr(g_k), _ptr(s), _stream(stream)), "fp4_attn_scores")
+
+
 def fp4_sync_status(stream=None) -> int:
     return lib().fp4_sync_status(_stream(stream))
 
@@ -313,6 +337,35 @@ def quantize_act(x, fmt="mxfp4", a_global=None, stream=None):
     sf = torch.empty(fp4_sf_bytes(f, M, K), dtype=torch.uint8, device=x.device)
     fp4_quantize_act(f, x, M, K, a_global, codes, sf, stream)
     return codes, sf
+
+
+def quantize_heads(x, H: int, fmt="mxfp4", g=None, stream=None):
+    """bf16 [T, H * 128] (CUDA) -> head-major (codes [H, Tpad, 64], scales [H, sf bytes per head])."""
+    import torch
+
+    f = _fmt(fmt)
+    T, HD = x.shape
+    D = HD // H
+    Tpad = (T + 127) // 128 * 128
+    codes = torch.empty((H, Tpad, D // 2), dtype=torch.uint8, device=x.device)
+    sf = torch.empty((H, fp4_heads_sf_bytes(f, T, H, D) // H), dtype=torch.uint8, device=x.device)
+    fp4_quantize_heads(f, x, T, H, D, g, codes, sf, stream)
+    return codes, sf
+
+
+def attn_scores(q_heads, k_heads, T_q: int, T_kv: int, head: int, fmt="mxfp4", g_q=None, g_k=None, s=None,
+                stream=None):
+    """Scores of one head from quantize_heads outputs: bf16 [T_q, T_kv rounded up to 128]."""
+    import torch
+
+    f = _fmt(fmt)
+    qc, qs = q_heads
+    kc, ks = k_heads
+    H, _, half_d = qc.shape
+    if s is None:
+        s = torch.empty((T_q, (T_kv + 127) // 128 * 128), dtype=torch.bfloat16, device=qc.device)
+    fp4_attn_scores(f, qc, qs, T_q, kc, ks, T_kv, H, 2 * half_d, head, g_q, g_k, s, stream)
+    return s
 
 
 def linear(x, pw: PackedWeight, bias=None, a_global=None, y=None, workspace=None, stream=None):

@@ -174,11 +174,16 @@ int quant_blocks(const DeviceState* ds, int kind, int64_t M, int64_t K) {
 }
 
 // gelu: quantize bf16_rn(gelu_tanh(x)) instead of x (MXFP4 / NVFP4 only)
+// heads: x is [M tokens, K = heads x 128], written head-major (MXFP4 / NVFP4 only)
 fp4_status_t launch_quant(const DeviceState* ds, int kind, const void* x, int64_t M, int64_t K, const float* g,
-                          uint8_t* out, uint8_t* sf, cudaStream_t st, bool gelu = false) {
+                          uint8_t* out, uint8_t* sf, cudaStream_t st, bool gelu = false, bool heads = false) {
     const int blocks = quant_blocks(ds, kind, M, K);
     const uint4* xv = static_cast<const uint4*>(x);
-    if (gelu && kind == Q_MXFP4)
+    if (heads && kind == Q_MXFP4)
+        quant_kernel<Q_MXFP4, false, true><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
+    else if (heads)
+        quant_kernel<Q_NVFP4, false, true><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
+    else if (gelu && kind == Q_MXFP4)
         quant_kernel<Q_MXFP4, true><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
     else if (gelu)
         quant_kernel<Q_NVFP4, true><<<blocks, QUANT_THREADS, 0, st>>>(xv, M, K, g, out, sf);
@@ -492,6 +497,31 @@ fp4_status_t fp4_gelu_quantize_act(fp4_fmt_t fmt, const void* z_bf16, int64_t M,
                         static_cast<cudaStream_t>(stream), true);
 }
 
+size_t fp4_heads_codes_bytes(fp4_fmt_t fmt, int64_t T, int64_t H, int64_t D) {
+    if (!fmt_ok(fmt) || T < 0 || H < 0 || D != FP4_HEAD_DIM) return 0;
+    return (size_t)H * (size_t)((T + 127) / 128 * 128) * (size_t)(D / 2);
+}
+
+size_t fp4_heads_sf_bytes(fp4_fmt_t fmt, int64_t T, int64_t H, int64_t D) {
+    if (!fmt_ok(fmt) || T < 0 || H < 0 || D != FP4_HEAD_DIM) return 0;
+    return (size_t)H * fp4_sf_bytes(fmt, T, D);
+}
+
+fp4_status_t fp4_quantize_heads(fp4_fmt_t fmt, const void* x_bf16, int64_t T, int64_t H, int64_t D,
+                                const float* g, uint8_t* codes, uint8_t* sf, void* stream) {
+    if (!fmt_ok(fmt) || !x_bf16 || !codes || !sf || T < 1 || H < 1) return FP4_ERR_INVALID_ARG;
+    if ((fmt == FP4_FMT_NVFP4) != (g != nullptr)) return FP4_ERR_INVALID_ARG;
+    if (D != FP4_HEAD_DIM || H >= kMaxDim / D) return FP4_ERR_UNSUPPORTED_SHAPE;
+    fp4_status_t s = check_shape(T, H * D, 128);
+    if (s != FP4_OK) return s;
+    if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(sf) || (reinterpret_cast<uintptr_t>(g) & 3u))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    if ((s = device_state(&ds)) != FP4_OK) return s;
+    return launch_quant(ds, fmt == FP4_FMT_MXFP4 ? Q_MXFP4 : Q_NVFP4, x_bf16, T, H * D, g, codes, sf,
+                        static_cast<cudaStream_t>(stream), false, true);
+}
+
 fp4_status_t fp4_pack_weight(fp4_fmt_t fmt, const void* w_bf16, int64_t N, int64_t K, uint8_t* w_codes,
                              uint8_t* w_sf, float* w_global, void* stream) {
     if (!fmt_ok(fmt) || !w_bf16 || !w_codes || !w_sf) return FP4_ERR_INVALID_ARG;
@@ -582,6 +612,23 @@ fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf
                       const void* bias_f16, void* y_bf16, void* stream) {
     return gemm_impl(fmt, a_codes, a_sf, M, K, N, w_codes, w_sf, w_global, a_global, bias_f16, y_bf16, stream,
                      nullptr, 0);
+}
+
+fp4_status_t fp4_attn_scores(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,
+                             const uint8_t* k_codes, const uint8_t* k_sf, int64_t T_kv, int64_t H, int64_t D,
+                             int64_t head, const float* g_q, const float* g_k, void* s_bf16, void* stream) {
+    if (!fmt_ok(fmt) || !q_codes || !q_sf || !k_codes || !k_sf || !s_bf16) return FP4_ERR_INVALID_ARG;
+    if (T_q < 1 || T_kv < 1 || H < 1 || head < 0 || head >= H) return FP4_ERR_INVALID_ARG;
+    if (D != FP4_HEAD_DIM) return FP4_ERR_UNSUPPORTED_SHAPE;
+    const int64_t tq_pad = (T_q + 127) / 128 * 128, tk_pad = (T_kv + 127) / 128 * 128;
+    // head `head` of the head-major buffers: its codes, then its scale atoms
+    const uint8_t* qc = q_codes + (size_t)head * tq_pad * (D / 2);
+    const uint8_t* kc = k_codes + (size_t)head * tk_pad * (D / 2);
+    const uint8_t* qs = q_sf + (size_t)head * fp4_sf_bytes(fmt, T_q, D);
+    const uint8_t* ks = k_sf + (size_t)head * fp4_sf_bytes(fmt, T_kv, D);
+    // S = Q_h K_h^T: Q_h is the activation operand (M = T_q), K_h the weight operand over
+    // all T_kv_pad key rows (padding keys have zero codes, so their columns hold 0)
+    return gemm_impl(fmt, qc, qs, T_q, D, tk_pad, kc, ks, g_k, g_q, nullptr, s_bf16, stream, nullptr, 0);
 }
 
 fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K, int64_t N, const uint8_t* w_codes,

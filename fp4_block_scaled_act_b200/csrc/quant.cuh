@@ -48,7 +48,12 @@ FP4_DEV float mx_inv_scale(uint32_t byte) { return __uint_as_float((254u - byte)
 
 // GELU = true: the input is the bf16 up-projection output z and the quantized value is
 // bf16_rn(gelu_tanh(z)) (gelu.cuh), the down projection's activation.
-template <int KIND, bool GELU = false>
+// HEADS = true: x is [M tokens, H heads x 128] (attention Q or K, head_dim 128), so a unit
+// is one token's head (chunk = head), and the output is head-major: codes
+// [H][Mpad][64 bytes] (padding tokens get zero codes) and per head the scale atoms of a
+// [Mpad, 128] matrix, heads one after another.  Each head's codes and scales are then the
+// A or B operand layout of a GEMM with K = head_dim.
+template <int KIND, bool GELU = false, bool HEADS = false>
 __global__ void __launch_bounds__(QUANT_THREADS, 4) quant_kernel(const uint4* __restrict__ x, int64_t M, int64_t K,
                                                               const float* __restrict__ g_ptr,
                                                               uint8_t* __restrict__ out, uint8_t* __restrict__ sf) {
@@ -141,7 +146,10 @@ __global__ void __launch_bounds__(QUANT_THREADS, 4) quant_kernel(const uint4* __
                 for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], inv);
             }
 
-            if (rows[it] < (uint32_t)M) {
+            if (HEADS) {
+                static_assert(!HEADS || KIND != Q_MXFP8, "head-major output is FP4 only");
+                reinterpret_cast<uint32_t*>(out)[((size_t)chunks[it] * Mpad + rows[it]) * 16 + part] = cvt_e2m1x8(v);
+            } else if (rows[it] < (uint32_t)M) {
                 if (KIND == Q_MXFP8) {
                     uint2 w;
                     w.x = cvt_e4m3x2(v[0], v[1]) | (cvt_e4m3x2(v[2], v[3]) << 16);
@@ -160,15 +168,25 @@ __global__ void __launch_bounds__(QUANT_THREADS, 4) quant_kernel(const uint4* __
                 word = sfb << (8 * ((part >> 1) & 3));  // groups of 2 lanes, words of 8 lanes
                 word |= __shfl_xor_sync(0xffffffffu, word, 2);
                 word |= __shfl_xor_sync(0xffffffffu, word, 4);
-                if ((part & 7) == 0)
-                    *reinterpret_cast<uint32_t*>(sf + sf_word_offset(rows[it], chunks[it] * 2 + (part >> 3), apr)) =
-                        word;
+                if ((part & 7) == 0) {
+                    if (HEADS)  // head chunks[it]: two atoms per row block
+                        *reinterpret_cast<uint32_t*>(sf + (size_t)chunks[it] * (Mpad >> 7) * 1024 +
+                                                     sf_word_offset(rows[it], part >> 3, 2)) = word;
+                    else
+                        *reinterpret_cast<uint32_t*>(sf + sf_word_offset(rows[it], chunks[it] * 2 + (part >> 3), apr)) =
+                            word;
+                }
             } else {
                 word = sfb << (8 * (part >> 2));        // groups of 4 lanes, one word per unit
                 word |= __shfl_xor_sync(0xffffffffu, word, 4);
                 word |= __shfl_xor_sync(0xffffffffu, word, 8);
-                if (part == 0)
-                    *reinterpret_cast<uint32_t*>(sf + sf_word_offset(rows[it], chunks[it], apr)) = word;
+                if (part == 0) {
+                    if (HEADS)  // head chunks[it]: one atom per row block
+                        *reinterpret_cast<uint32_t*>(sf + (size_t)chunks[it] * (Mpad >> 7) * 512 +
+                                                     sf_word_offset(rows[it], 0, 1)) = word;
+                    else
+                        *reinterpret_cast<uint32_t*>(sf + sf_word_offset(rows[it], chunks[it], apr)) = word;
+                }
             }
         }
     }

@@ -316,6 +316,50 @@ fp4_status_t w4a4_svd_linear(const void* x_bf16, int64_t M, int64_t K, int64_t N
                              const void* l2_bf16, int rank, const void* bias_f16, void* y_bf16,
                              void* workspace, size_t ws_bytes, void* stream);
 
+/* ----------------------------------------------------------------- FP4 attention operands */
+
+/* First slice of microscaling FP4 attention: the attention backends the Wan2.2-Animate-14B
+ * MXFP4 card compares ("Results") include SageAttention v3, which it describes as
+ * Blackwell microscaling FP4 attention.  The card gives no algorithm; this library reads
+ * it as Q and K quantized per token and head in blocks along head_dim by the same MXFP4 /
+ * NVFP4 rules as the linear's activations, and the scores S = deq(Q_h) deq(K_h)^T of one
+ * head computed by the block-scaled GEMM (fp32 accumulation, bf16 out).  Softmax and the
+ * P V product are not part of this interface.
+ *
+ * Head-major layout of a quantized [T tokens, H heads x D] tensor (D = FP4_HEAD_DIM):
+ *   codes  [H][Tpad][D/2] bytes, Tpad = T rounded up to 128; tokens in [T, Tpad) hold
+ *          zero codes;
+ *   sf     H consecutive blocks of fp4_sf_bytes(fmt, T, D) bytes: head h's scales in the
+ *          sf layout above for a [T, D] matrix (K = D).
+ * Head h's codes and scales are thus exactly fp4_quantize_act of columns h*D .. h*D+D-1
+ * of x (with T rows), the codes padded to Tpad rows with zeros. */
+#define FP4_HEAD_DIM 128
+
+/* Bytes of the head-major codes / scales of a [T, H x D] tensor (0 if invalid: D must be
+ * FP4_HEAD_DIM). */
+size_t fp4_heads_codes_bytes(fp4_fmt_t fmt, int64_t T, int64_t H, int64_t D);
+size_t fp4_heads_sf_bytes(fp4_fmt_t fmt, int64_t T, int64_t H, int64_t D);
+
+/* Quantize x_bf16 (device) [T, H*D] bf16, row-major (token-major, heads contiguous within
+ * a token, as a linear projection writes them), into the head-major layout above.
+ *   g      (device) NVFP4: the tensor's fp32 global (e.g. fp4_calibrate_act_global over x
+ *          itself); MXFP4: must be NULL
+ *   codes  (device, out) fp4_heads_codes_bytes(fmt, T, H, D)
+ *   sf     (device, out) fp4_heads_sf_bytes(fmt, T, H, D)
+ * D other than FP4_HEAD_DIM returns FP4_ERR_UNSUPPORTED_SHAPE. */
+fp4_status_t fp4_quantize_heads(fp4_fmt_t fmt, const void* x_bf16, int64_t T, int64_t H, int64_t D,
+                                const float* g, uint8_t* codes, uint8_t* sf, void* stream);
+
+/* Scores of head `head`: s_bf16 (device, out) [T_q][T_kv_pad] bf16, row-major, T_kv_pad =
+ * T_kv rounded up to 128, s[i][j] = bf16_rn( sum_d deq(q)[i][d] deq(k)[j][d] ) with the
+ * NVFP4 globals g_q g_k applied (device fp32, NULL for MXFP4); columns j >= T_kv are 0.
+ * q_codes / q_sf and k_codes / k_sf are the whole head-major buffers of fp4_quantize_heads
+ * (T_q resp. T_kv tokens, H heads).  No softmax scaling is applied. */
+fp4_status_t fp4_attn_scores(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,
+                             const uint8_t* k_codes, const uint8_t* k_sf, int64_t T_kv, int64_t H,
+                             int64_t D, int64_t head, const float* g_q, const float* g_k, void* s_bf16,
+                             void* stream);
+
 /* ----------------------------------------------------------------- status */
 
 /* The status calls below are part of this library's error model, not of the method: the

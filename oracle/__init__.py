@@ -257,6 +257,42 @@ def svd_linear_rows(act: str, x_bf16, r_packed, l1_bf16, l2_bf16, bias_f16, rows
     return Y + LR, S + LS
 
 
+# ----------------------------------------------------------------------------- FP4 attention operands
+# Wan2.2-Animate-14B MXFP4 card, "Results": SageAttention v3 is Blackwell microscaling FP4
+# attention.  The card gives no algorithm; the reading followed here quantizes Q and K per
+# token and head in blocks of G along head_dim with the activation rules above (a head of
+# D = 128 is a whole number of groups, so no group spans two heads) and takes the scores
+# of one head as the fp64 product of the dequantized operands.
+def quantize_heads(fmt: int, x_bf16: np.ndarray, H: int, g: float | None = None):
+    """bf16 [T, H*128] -> head-major (codes [H, Tpad, 64] uint8, sf [H, sf_bytes(Tpad, 128/G)]):
+    head h is `quantize` of columns h*128 .. h*128+127, its codes padded with zero rows."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    T, HD = x.shape
+    D = HD // H
+    assert D * H == HD and D == 128
+    Tpad = (T + 127) // 128 * 128
+    codes = np.zeros((H, Tpad, D // 2), dtype=np.uint8)
+    sfs = np.zeros((H, sf_bytes(Tpad, D // group_size(fmt))), dtype=np.uint8)
+    for h in range(H):
+        c, s = quantize(fmt, np.ascontiguousarray(x[:, h * D:(h + 1) * D]), g)
+        codes[h, :T] = c
+        sfs[h] = s
+    return codes, sfs
+
+
+def attn_scores_rows(fmt: int, q_heads, k_heads, head: int, rows, g_q: float | None = None,
+                     g_k: float | None = None):
+    """(Y, S) of rows `rows` of head `head`'s scores: Y[i, j] = sum_d deq(q)[i, d] deq(k)[j, d]
+    over every key row j of the head-major buffers (padding keys give 0), in fp64;
+    S = sum_d |deq(q) deq(k)| for the tolerance."""
+    qc, qs = q_heads
+    kc, ks = k_heads
+    D = 2 * qc.shape[2]
+    a = dequant_fp4(fmt, qc[head], qs[head], D, 1.0 if fmt == MX else g_q, rows=rows)
+    w = dequant_fp4(fmt, kc[head], ks[head], D, 1.0 if fmt == MX else g_k)
+    return linear_fp64(a, w, None)
+
+
 def num_threads() -> int:
     return lib().orc_num_threads()
 

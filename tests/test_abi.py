@@ -55,6 +55,11 @@ def test_size_queries(fb):
     assert fb.w4a4_workspace_bytes(75600, 5120, 13824, 32) == (
         a256(75600 * 2560) + a256(fb.fp4_sf_bytes(MX, 75600, 5120)) + a256(75600 * 32 * 4))
     assert fb.w4a4_workspace_bytes(4290, 3072, 14336, 16) == 0
+    # head-major attention operands: [H][Tpad][64] codes, H blocks of [Tpad, 128] scales
+    assert fb.fp4_heads_codes_bytes(MX, 75600, 40) == 40 * 75648 * 64
+    assert fb.fp4_heads_sf_bytes(MX, 75600, 40) == 40 * fb.fp4_sf_bytes(MX, 75600, 128) == 40 * 75648 * 4
+    assert fb.fp4_heads_sf_bytes(NV, 130, 3) == 3 * 256 * 8
+    assert fb.fp4_heads_codes_bytes(MX, 130, 3, 64) == 0                # head_dim 128 only
 
 
 def test_bytes_per_weight_match_format(fb):
@@ -117,6 +122,16 @@ def test_invalid_calls_rejected_before_launch(fb):
     # weight pack: MXFP4 must not get a global
     assert L.fp4_pack_weight(0, A, 256, 256, A, A, A, st) == 1
     assert L.fp4_tensor_amax(A, 0, A, st) == 1
+    # FP4 attention operands: head_dim, format / global pairing, alignment, head index
+    assert L.fp4_quantize_heads(0, A, 16, 2, 64, None, A, A, st) == 2
+    assert L.fp4_quantize_heads(1, A, 16, 2, 128, None, A, A, st) == 1
+    assert L.fp4_quantize_heads(0, A, 16, 2, 128, A, A, A, st) == 1
+    assert L.fp4_quantize_heads(0, bad, 16, 2, 128, None, A, A, st) == 3
+    assert L.fp4_quantize_heads(0, A, 0, 2, 128, None, A, A, st) == 1
+    assert L.fp4_attn_scores(0, A, A, 16, A, A, 16, 2, 128, 2, None, None, A, st) == 1
+    assert L.fp4_attn_scores(0, A, A, 16, A, A, 16, 2, 64, 0, None, None, A, st) == 2
+    assert L.fp4_attn_scores(1, A, A, 16, A, A, 16, 2, 128, 0, None, None, A, st) == 1
+    assert L.fp4_attn_scores(0, A, A, 16, A, A, 16, 2, 128, 0, None, None, bad, st) == 3
 
 
 def test_product_path_has_no_oracle_import():
