@@ -422,6 +422,29 @@ def extra_workloads(fb, torch, args, steps: int = 20, warmup: int = 3):
         call_t()
     out["mxfp4_text_kv_512x5120x5120_graph"] = timed(graph.replay, 2.0 * 512 * 5120 * 5120, n=200)
     del graph
+    # FP4 attention operands at the Wan2.2 sequence length: the head-major K quantizer
+    # (40 heads of 128) and one head's 75600 x 75648 score GEMM (bound by writing S)
+    Ta, Ha = 75600, 40
+    for fmt in ("mxfp4", "nvfp4"):
+        f = fb.MXFP4 if fmt == "mxfp4" else fb.NVFP4
+        qa, ka = act(Ta, Ha * 128), act(Ta, Ha * 128)
+        g_q = g_k = None
+        if fmt == "nvfp4":
+            g_q, _ = fb.calibrate_act_global(qa)
+            g_k, _ = fb.calibrate_act_global(ka)
+        qh = fb.quantize_heads(qa, Ha, fmt, g_q)
+        kh = fb.quantize_heads(ka, Ha, fmt, g_k)
+        qb = Ta * Ha * 128 * 2 + fb.fp4_heads_codes_bytes(f, Ta, Ha) + fb.fp4_heads_sf_bytes(f, Ta, Ha)
+        kc_buf, ks_buf = kh
+        r_q = timed(lambda: fb.fp4_quantize_heads(f, ka, Ta, Ha, 128, g_k, kc_buf, ks_buf), 0.0)
+        r_q["gbs"] = qb / (r_q["ms"] / 1e3) / 1e9
+        out[f"{fmt}_attn_quantize_heads_75600x40x128"] = r_q
+        s_buf = torch.empty((Ta, (Ta + 127) // 128 * 128), dtype=torch.bfloat16, device="cuda")
+        r_s = timed(lambda: fb.attn_scores(qh, kh, Ta, Ta, 17, fmt, g_q, g_k, s_buf), 2.0 * Ta * s_buf.shape[1] * 128,
+                    n=10)
+        r_s["s_write_gbs"] = s_buf.numel() * 2 / (r_s["ms"] / 1e3) / 1e9
+        out[f"{fmt}_attn_scores_head_75600x75648x128"] = r_s
+        del qa, ka, qh, kh, kc_buf, ks_buf, s_buf
     # W4A8 SVDQuant linear at the TI2V-5B shape (MXFP8 activations, rank 32)
     Mw, Kw, Nw, r = 4290, 3072, 14336, 32
     xw = act(Mw, Kw)
@@ -442,6 +465,10 @@ def extra_workloads(fb, torch, args, steps: int = 20, warmup: int = 3):
     for k, v in out.items():
         v["note"] = "pct_nominal: of 9 PFLOP/s dense FP4" + (" (W4A8 runs at the FP8 rate, nominal 4.5)"
                                                              if k.startswith("w4a8") else "")
+        if "quantize_heads" in k:
+            v["note"] = "HBM-bound: gbs = bf16 read + codes and scales written, per second"
+        elif "attn_scores" in k:
+            v["note"] = "bound by writing S (bf16): s_write_gbs; pct_nominal of 9 PFLOP/s dense FP4"
     return out
 
 
