@@ -406,6 +406,32 @@ def extra_workloads(fb, torch, args, steps: int = 20, warmup: int = 3):
         lambda: fb.fp4_linear("mxfp4", x, Mx, 5120, 5120, pw_a.codes, pw_a.sf, None, None, b_a, ya, ws,
                               ws.numel()), 2.0 * Mx * 5120 * 5120)
     del ya, x
+    # the rest of the Wan2.2 block's linears and the M sweep, in both formats (quantize +
+    # GEMM through fp4_linear; NVFP4 activation globals calibrated once on a separate batch)
+    def linear_case(fmt, M, K, N, kind="act"):
+        if kind == "gelu":  # the down projection's input: GELU-tanh of an N(0,1) tensor
+            z = torch.randn(M, K, generator=gen, device="cuda")
+            xs = torch.nn.functional.gelu(z, approximate="tanh").to(torch.bfloat16)
+            del z
+        else:
+            xs = act(M, K)
+        pw_c = fb.pack_weight(wgt(N, K), fmt)
+        g_c = fb.calibrate_act_global(act(4096, K))[0] if fmt == "nvfp4" else None
+        y_c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        ws_c = torch.empty(fb.fp4_linear_workspace_bytes(fmt, M, K, N), dtype=torch.uint8, device="cuda")
+        b_c = bias(N)
+        r = timed(lambda: fb.fp4_linear(fmt, xs, M, K, N, pw_c.codes, pw_c.sf, pw_c.w_global, g_c, b_c, y_c, ws_c,
+                                        ws_c.numel()), 2.0 * M * K * N)
+        del xs, pw_c, y_c, ws_c
+        return r
+
+    for fmt in ("mxfp4", "nvfp4"):
+        out[f"{fmt}_ffn_down_75600x13824x5120"] = linear_case(fmt, Mx, 13824, 5120, "gelu")
+        if fmt == "nvfp4":
+            out["nvfp4_attn_75600x5120x5120"] = linear_case(fmt, Mx, 5120, 5120)
+            out["nvfp4_text_kv_512x5120x5120_eager"] = linear_case(fmt, 512, 5120, 5120)
+        for Ms in (512, 4096, 16384):
+            out[f"{fmt}_m_sweep_{Ms}x5120x13824"] = linear_case(fmt, Ms, 5120, 13824)
     xt = act(512, 5120)
     yt = torch.empty((512, 5120), dtype=torch.bfloat16, device="cuda")
     wst = torch.empty(fb.fp4_linear_workspace_bytes("mxfp4", 512, 5120, 5120), dtype=torch.uint8, device="cuda")
