@@ -58,7 +58,50 @@ def parse():
     ap.add_argument("--fmt", default="mxfp4", choices=["mxfp4", "nvfp4"])
     ap.add_argument("--m", type=int, default=75600,
                     help="tokens; smaller values run a reduced case of the same kernels (profiling only)")
+    ap.add_argument("--attn-tokens", type=int, default=0,
+                    help="profiling only: run the FP4 attention operands (K quantizer over 40 heads of 128 and "
+                         "head 17's score GEMM) at this many tokens for --steps iterations, print timings, exit")
     return ap.parse_args()
+
+
+def attn_profile(args):
+    """The FP4 attention-operand kernels alone (a case for ncu): quantize_heads of Q and K
+    ([T, 40 x 128] bf16), then per step the K quantizer and head 17's score GEMM."""
+    import torch
+
+    import fp4_block_scaled_act_b200 as fb
+
+    fb.lib()
+    T, Hn, fmt = args.attn_tokens, 40, args.fmt
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(20261203)
+    q = torch.randn(T, Hn * 128, generator=gen, device="cuda").to(torch.bfloat16)
+    k = torch.randn(T, Hn * 128, generator=gen, device="cuda").to(torch.bfloat16)
+    gq = gk = None
+    if fmt == "nvfp4":
+        gq, _ = fb.calibrate_act_global(q)
+        gk, _ = fb.calibrate_act_global(k)
+    qh = fb.quantize_heads(q, Hn, fmt, gq)
+    kh = fb.quantize_heads(k, Hn, fmt, gk)
+    s_buf = torch.empty((T, (T + 127) // 128 * 128), dtype=torch.bfloat16, device="cuda")
+    f = fb.MXFP4 if fmt == "mxfp4" else fb.NVFP4
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    tq = ts = 0.0
+    for _ in range(args.steps):
+        e[0].record()
+        fb.fp4_quantize_heads(f, k, T, Hn, 128, gk, kh[0], kh[1])
+        e[1].record()
+        fb.attn_scores(qh, kh, T, T, 17, fmt, gq, gk, s_buf)
+        e[2].record()
+        torch.cuda.synchronize()
+        tq += e[0].elapsed_time(e[1])
+        ts += e[1].elapsed_time(e[2])
+    st = fb.fp4_sync_status()
+    if st != 0:
+        raise RuntimeError(f"device status: {fb.fp4_status_string(st)}")
+    print(json.dumps({"attn_tokens": T, "heads": Hn, "fmt": fmt, "quantize_heads_ms": tq / args.steps,
+                      "scores_ms": ts / args.steps, "s_bytes": s_buf.numel() * 2}), flush=True)
+    return 0
 
 
 def dist_env():
@@ -676,6 +719,8 @@ def main():
         M = args.m
         WORKLOAD = f"ffn_up_{FMT}_m{M}"
         FLOP_PER_STEP = 2.0 * M * K * N
+    if args.attn_tokens:
+        return attn_profile(args)
     if args.impl == "reference":
         return reference_arm(args)
     return native_arm(args)
