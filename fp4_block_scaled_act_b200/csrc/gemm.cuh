@@ -392,8 +392,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 //
 // Warps (512 threads, four warpgroups): 0 operand TMA producer, 1 TMEM owner + MMA issuer
 // (leader), 2 stage coordinator (leader), 3 scale TMA producer, 4-7 scale writers, 8-15
-// epilogue.  The
-// control warpgroups (0-7) drop to REG_LO registers per thread with setmaxnreg and the
+// epilogue.  The control warpgroups (0-7) drop to REG_LO registers per thread with setmaxnreg and the
 // epilogue warpgroups rise to REG_HI: the fused epilogues run without spilling, and an
 // NVFP4 overlap holder can copy its whole 128-column share before converting any.
 // The tensor pipe queues very little ahead of the issuing thread, so every cycle that
@@ -404,7 +403,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 //   full[s]      (leader)  A/B bytes of both CTAs; the leader alone expects them
 //   empty[s]     (both)    the leader's commit (MMAs of stage s done)
 //   sc_full[j]   (local)   this CTA's raw scale atoms in scale-ring slot j
-//   sc_empty[j]  (local)   slot j read by this CTA's 4 writer warps (separate scale ring;
+//   sc_empty[j]  (local)   slot j stored into TMEM by this CTA's 4 writer warps (separate scale ring;
 //                          NVFP4's scale slots ride in the operand ring and are recycled
 //                          with empty[s], loaded by the operand producer)
 //   sf_ready[t]  (leader)  scale buffer t written in both CTAs (8 writer warps)
@@ -943,7 +942,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<KIND>::THRE
         if (lane == 0) bulk_wait_group0();
         __syncwarp();
     } else {
-        // warps 0-7: producer, MMA issuer, coordinator, an idle warp and the scale writers
+        // warps 0-7: operand producer, MMA issuer, coordinator, scale producer and the scale writers
         setmaxnreg_dec<C::REG_LO>();
         if (warp == 0) {
             // ============================================================ producer (both CTAs)
