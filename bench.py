@@ -288,6 +288,17 @@ def kernel_code_digest() -> str:
 
 
 # ----------------------------------------------------------------------------- cpu baseline
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), recorded beside the core count."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(x_bits, w_bits, b_bits, target_s: float = 15.0):
     """The oracle, as it stands, on a bounded row sample of the same workload."""
     import oracle
@@ -311,10 +322,19 @@ def cpu_baseline(x_bits, w_bits, b_bits, target_s: float = 15.0):
     t = time.perf_counter()
     run(rows)
     dt = time.perf_counter() - t
+    # the activation quantizer alone over a row sample of its own, as a bandwidth
+    qrows = np.arange(min(M, 8192))
+    xq = np.ascontiguousarray(x_bits[qrows])
+    t = time.perf_counter()
+    oracle.quantize(f, xq, g_a)
+    dq = time.perf_counter() - t
+    q_bytes = qrows.size * K * 2 + qrows.size * K // 2 + oracle.sf_bytes(qrows.size, K // oracle.group_size(f))
     return {"value": 2.0 * nrows * K * N / dt / 1e12, "unit": "TFLOPS", "cores": oracle.num_threads(),
-            "kind": "oracle",
+            "cpu": cpu_model(), "kind": "oracle",
+            "quantize_gbs": q_bytes / dq / 1e9,
             "sample": f"{nrows} of {M} rows: {FMT.upper()} quantize + dequantize + fp64 GEMM over full K={K}, N={N} "
-                      f"({dt:.1f} s); weight pack and dequantize excluded (offline)"}
+                      f"({dt:.1f} s); weight pack and dequantize excluded (offline); quantize_gbs: the quantizer "
+                      f"alone on {qrows.size} rows ({dq:.2f} s)"}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -365,8 +385,8 @@ def reference_arm(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / max(args.steps, 1) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_dict(args.gpus),
-        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": oracle.num_threads(), "cpu": cpu_model(),
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
