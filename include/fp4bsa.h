@@ -360,6 +360,51 @@ fp4_status_t fp4_attn_scores(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_
                              int64_t D, int64_t head, const float* g_q, const float* g_k, void* s_bf16,
                              void* stream);
 
+/* The rest of one head's attention (MXFP4 only), read the same way: P = softmax(S * scale)
+ * per query row over the T_kv keys, quantized in MXFP4 blocks of 32 consecutive keys; V of
+ * the head quantized per head-dim channel in MXFP4 blocks of 32 consecutive tokens; and
+ * O = deq(P) deq(V) by the block-scaled GEMM, whose K is then the key axis.  fp4_attn_scores,
+ * fp4_attn_softmax_quant and fp4_attn_pv in sequence give one head's attention output.
+ *
+ * Head-major layout of V^T, quantized from v [T tokens, H heads x D]:
+ *   codes  [H][D][Tpad/2] bytes (head h, channel d: its Tpad tokens as packed E2M1; padding
+ *          tokens hold zero codes);
+ *   sf     H consecutive blocks of fp4_sf_bytes(MXFP4, D, Tpad) bytes: head h's scales in the
+ *          sf layout above for the [D, Tpad] matrix (rows = channels, K = tokens). */
+size_t fp4_heads_vt_codes_bytes(fp4_fmt_t fmt, int64_t T, int64_t H, int64_t D);
+size_t fp4_heads_vt_sf_bytes(fp4_fmt_t fmt, int64_t T, int64_t H, int64_t D);
+
+/* Quantize v_bf16 (device) [T, H*D] bf16, row-major, into the V^T layout above (codes and
+ * sf device, out).  fmt must be FP4_FMT_MXFP4 (else FP4_ERR_INVALID_ARG); D must be
+ * FP4_HEAD_DIM (else FP4_ERR_UNSUPPORTED_SHAPE); H < 65536. */
+fp4_status_t fp4_quantize_heads_vt(fp4_fmt_t fmt, const void* v_bf16, int64_t T, int64_t H, int64_t D,
+                                   uint8_t* codes, uint8_t* sf, void* stream);
+
+/* Softmax of scores and its MXFP4 quantization.
+ *   s_bf16  (device) [T_q][T_kv_pad] bf16 scores (fp4_attn_scores' output; columns >= T_kv
+ *           are ignored)
+ *   scale   the softmax scale (e.g. 1/sqrt(D)), > 0 and finite; the kernels use
+ *           c = fp32(scale * log2 e), t_j = fl(fl(s_j c) - m), m = max_j fl(s_j c) over
+ *           j < T_kv, l = sum_j exp2(t_j) (fp32, a fixed order per row), p_j = fl(exp2(t_j) *
+ *           fl(1/l)); exp2 is CUDA's exp2f (within 2 ulp), so p is the softmax within
+ *           a relative 2e-4 (the bound the tests apply)
+ *   stats   (device, out) [T_q] pairs of fp32 (m, l)
+ *   p_codes (device, out) [T_q][T_kv_pad/2]; p_sf (device, out) fp4_sf_bytes(MXFP4, T_q,
+ *           T_kv_pad): p quantized by the MXFP4 rules above; keys >= T_kv hold p = 0 and
+ *           padding rows zero scale bytes.
+ * fmt must be FP4_FMT_MXFP4. */
+fp4_status_t fp4_attn_softmax_quant(fp4_fmt_t fmt, const void* s_bf16, int64_t T_q, int64_t T_kv, float scale,
+                                    void* stats, uint8_t* p_codes, uint8_t* p_sf, void* stream);
+
+/* O = deq(P) deq(V_head) for head `head`: the block-scaled GEMM with K = T_kv_pad.
+ *   p_codes, p_sf      fp4_attn_softmax_quant's output (T_q rows)
+ *   vt_codes, vt_sf    fp4_quantize_heads_vt's output (T_kv tokens, H heads)
+ *   o_bf16  (device, out) [T_q][D] bf16
+ * fmt must be FP4_FMT_MXFP4. */
+fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p_sf, int64_t T_q, int64_t T_kv,
+                         const uint8_t* vt_codes, const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head,
+                         void* o_bf16, void* stream);
+
 /* ----------------------------------------------------------------- status */
 
 /* The status calls below are part of this library's error model, not of the method: the

@@ -293,6 +293,72 @@ def attn_scores_rows(fmt: int, q_heads, k_heads, head: int, rows, g_q: float | N
     return linear_fp64(a, w, None)
 
 
+def quantize_heads_vt(x_bf16: np.ndarray, H: int):
+    """V bf16 [T, H*128] -> head-major V^T in MXFP4 (codes [H, 128, Tpad/2], sf [H, sf_bytes(128, Tpad/32)]):
+    head h is `quantize` of the [128, Tpad] matrix whose column t is token t of the head
+    (tokens >= T zero), i.e. the scales run along the tokens, the GEMM's K of P V."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    T, HD = x.shape
+    D = HD // H
+    assert D * H == HD and D == 128
+    Tpad = (T + 127) // 128 * 128
+    codes = np.zeros((H, D, Tpad // 2), dtype=np.uint8)
+    sfs = np.zeros((H, sf_bytes(D, Tpad // 32)), dtype=np.uint8)
+    for h in range(H):
+        vt = np.zeros((D, Tpad), dtype=np.uint16)
+        vt[:, :T] = x[:, h * D:(h + 1) * D].T
+        codes[h], sfs[h] = quantize(MX, vt)
+    return codes, sfs
+
+
+LOG2E = 1.4426950408889634
+
+
+def softmax_c(scale: float) -> float:
+    """The exponent multiplier as the library states it: c = fp32(scale * log2 e)."""
+    return float(np.float32(scale * LOG2E))
+
+
+def softmax_rows(s_bf16, T_kv: int, scale: float):
+    """Row softmax of bf16 scores [R, T_kv_pad] over the first T_kv keys, in fp64:
+    p_j = 2^(s_j c - max) / sum_k 2^(s_k c - max) with c = softmax_c(scale); keys >= T_kv get 0.
+    Returns (p, t_max_abs) where t_max_abs[r] = max_j |s_j c| (for the error bound)."""
+    s = synth_bits_to_f64(s_bf16)
+    c = softmax_c(scale)
+    u = s[:, :T_kv] * c
+    m = u.max(axis=1, keepdims=True)
+    e = np.exp2(u - m)
+    p = np.zeros_like(s)
+    p[:, :T_kv] = e / e.sum(axis=1, keepdims=True)
+    return p, np.abs(u).max(axis=1)
+
+
+def softmax_bound(T_kv_pad: int, t_max_abs):
+    """Relative bound on the library's fp32 p (per row): argument rounding of fl(fl(s c) - m)
+    (two roundings of terms up to 2 max|s c|, through 2^t: ln2 * 4 max|s c| 2^-24), exp2f
+    within 2 ulp (2^-22), the sum l of positive terms in fp32 (each of a row's 256 threads adds
+    at most 8 ceil(T_kv_pad / 2048) terms in order, then a 5-step warp tree and 7 more
+    additions, plus the terms' own errors), and fl(1/l) and the product (2^-23); doubled for
+    margin."""
+    u = 2.0 ** -24
+    term = np.log(2.0) * 4.0 * np.asarray(t_max_abs) * u + 2.0 ** -22
+    n = 8 * -(-T_kv_pad // 2048) + 12
+    return 2.0 * (2.0 * term + n * u + 2.0 * u)
+
+
+def pv_rows(p_codes, p_sf, vt_heads, head: int, T_kv_pad: int, rows):
+    """(Y, S) of rows `rows` of O = deq(P) deq(V_head) (MXFP4), in fp64."""
+    vc, vs = vt_heads
+    a = dequant_fp4(MX, p_codes, p_sf, T_kv_pad, rows=rows)
+    w = dequant_fp4(MX, vc[head], vs[head], T_kv_pad)
+    return linear_fp64(a, w, None)
+
+
+def synth_bits_to_f64(b) -> np.ndarray:
+    b = np.ascontiguousarray(b, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
 def num_threads() -> int:
     return lib().orc_num_threads()
 

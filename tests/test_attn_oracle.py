@@ -89,3 +89,105 @@ def test_scores_select_the_head_and_rows():
     rows = np.array([3, 1])
     Y, _ = oracle.attn_scores_rows(MX, qh, kh, 2, rows)
     np.testing.assert_array_equal(Y[:, :7], q[rows, 256:384] @ k[:, 256:384].T)
+
+
+# ------------------------------------------------------------------ V^T, softmax, P V
+@pytest.mark.parametrize("T,H", [(1, 1), (130, 2), (257, 3)])
+def test_quantize_heads_vt_is_the_row_quantizer_of_the_transpose(T, H):
+    """Head h's V^T is the pinned row quantizer applied to the explicit transpose of its 128
+    columns, zero-padded to Tpad tokens: codes and every scale byte."""
+    x = _x(900 + T + H, T, H)
+    codes, sfs = oracle.quantize_heads_vt(x, H)
+    Tpad = (T + 127) // 128 * 128
+    assert codes.shape == (H, D, Tpad // 2)
+    for h in range(H):
+        vt = np.zeros((D, Tpad), dtype=np.uint16)
+        for t in range(T):
+            for d in range(D):
+                vt[d, t] = x[t, h * D + d]
+        c, s = oracle.quantize(MX, vt)
+        np.testing.assert_array_equal(codes[h], c)
+        np.testing.assert_array_equal(sfs[h], s)
+        assert not codes[h][:, (T + 1) // 2:].any(), "padding tokens hold zero codes"
+
+
+def test_quantize_heads_vt_single_token_worked():
+    """One token, one head: each channel's first group holds the token's value and 31 zero
+    tokens, so its scale comes from |v_d| alone and the code is e2m1(v_d / 2^e)."""
+    v = np.array([[6.0, -3.0, 0.5, 0.0] + [1.0] * 124], dtype=np.float32)
+    codes, sfs = oracle.quantize_heads_vt(synth.f32_to_bf16_bits(v), 1)
+    # channel 0: amax 6 -> e = 0, code 6 = 0x7; channel 1: amax 3 -> e = -1, -3 / 2^-1 = -6 -> 0xF;
+    # channel 2: 0.5 -> e = -3, 4 -> 0x6; channel 3: zero group -> byte 0, code 0
+    assert [codes[0, d, 0] & 0xF for d in range(4)] == [0x7, 0xF, 0x6, 0x0]
+    assert [sfs[0, oracle.sf_offset(d, 0, 128 // 32)] for d in range(4)] == [127, 126, 124, 0]
+    assert not codes[0, :, 1:].any(), "padding tokens hold zero codes"
+
+
+def test_softmax_oracle_against_closed_forms_and_scipy():
+    from scipy.special import softmax
+
+    rng = np.random.default_rng(3)
+    s = synth.f32_to_bf16_bits(rng.normal(0, 4, size=(5, 384)).astype(np.float32))
+    p, tmax = oracle.softmax_rows(s, 300, 0.125)
+    sf = oracle.synth_bits_to_f64(s)
+    c = oracle.softmax_c(0.125)
+    ref = softmax(sf[:, :300] * c * np.log(2.0), axis=1)    # 2^(s c) = e^(s c ln 2)
+    np.testing.assert_allclose(p[:, :300], ref, rtol=1e-12, atol=0)
+    assert not p[:, 300:].any()
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=1e-14)
+    # a constant row is uniform; a row with one score far above the rest is one-hot
+    const = np.full((1, 128), synth.f32_to_bf16_bits(np.float32([2.5]))[0], dtype=np.uint16)
+    pc, _ = oracle.softmax_rows(const, 100, 1.0)
+    np.testing.assert_allclose(pc[0, :100], 1.0 / 100, rtol=1e-15)
+    hot = np.zeros((1, 128), dtype=np.uint16)
+    hot[0, 7] = synth.f32_to_bf16_bits(np.float32([1000.0]))[0]
+    ph, _ = oracle.softmax_rows(hot, 128, 1.0)
+    assert ph[0, 7] == 1.0 and ph[0, :7].max() < 1e-290
+
+
+def test_softmax_bound_covers_an_fp32_evaluation():
+    """numpy float32 steps as the library states them (fl(fl(s c) - m), exp2, sequential sums
+    per thread stride, 1/l, product) stay inside softmax_bound of the fp64 softmax."""
+    rng = np.random.default_rng(4)
+    kpad, T_kv = 2048, 1990
+    s = synth.f32_to_bf16_bits(rng.normal(0, 6, size=(3, kpad)).astype(np.float32))
+    p, tmax = oracle.softmax_rows(s, T_kv, 0.088388)
+    eps = oracle.softmax_bound(kpad, tmax)
+    c = np.float32(oracle.softmax_c(0.088388))
+    sf = oracle.synth_bits_to_f64(s).astype(np.float32)
+    for r in range(3):
+        u = (sf[r, :T_kv] * c).astype(np.float32)
+        m = u.max()
+        e = np.exp2((u - m).astype(np.float32)).astype(np.float32)
+        lanes = np.zeros(256 * 8, dtype=np.float32)
+        ee = np.zeros(kpad, dtype=np.float32)
+        ee[:T_kv] = e
+        part = np.zeros(256, dtype=np.float32)
+        for i in range(kpad // 8):                 # thread i % 256 takes 8-element vector i
+            for k in range(8):
+                part[i % 256] = np.float32(part[i % 256] + ee[i * 8 + k])
+        l = np.float32(0.0)
+        for v in part:
+            l = np.float32(l + v)
+        p32 = (e * np.float32(np.float32(1.0) / l)).astype(np.float32)
+        rel = np.abs(p32.astype(np.float64) - p[r, :T_kv]) / p[r, :T_kv]
+        assert rel.max() <= eps[r], (rel.max(), eps[r])
+        del lanes
+
+
+def test_pv_oracle_exact_on_representable_blocks():
+    """P V on losslessly representable operands (P blocks of 32 keys and V blocks of 32 tokens
+    on the E2M1 grid times the block's power of two, each block's amax 6 * 2^e) equals numpy's
+    exact product of the original values, for each head; padding keys and tokens give 0."""
+    rng = np.random.default_rng(6)
+    Tq, Tk, H = 3, 160, 2                                    # 160 tokens = 5 whole groups
+    kpad = 256
+    pvals = _representable(rng, Tq, 2, 32)[:, :kpad]         # [Tq, 256] exact MX blocks
+    pvals[:, Tk:] = 0.0
+    pc, ps = oracle.quantize(MX, synth.f32_to_bf16_bits(pvals.astype(np.float32)))
+    vtv = _representable(rng, H * D, 2, 32)[:, :Tk]          # [H*128 channels, Tk tokens]: blocks along tokens
+    v = np.ascontiguousarray(vtv.T)                          # [Tk, H*128]
+    vt = oracle.quantize_heads_vt(synth.f32_to_bf16_bits(v.astype(np.float32)), H)
+    for head in range(H):
+        Y, _ = oracle.pv_rows(pc, ps, vt, head, kpad, np.arange(Tq))
+        np.testing.assert_array_equal(Y, pvals[:, :Tk] @ v[:, head * D:(head + 1) * D])

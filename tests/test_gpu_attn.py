@@ -91,3 +91,172 @@ def test_attn_scores_full_size_sampled(fb, orc, fmt):
     T = 75600
     rows = H.sample_rows(T, n_random=16, seed=17 + fmt)
     _scores_case(fb, orc, fmt, T, T, 40, 17, seed=3500 + fmt, rows=rows)
+
+
+# ------------------------------------------------------------------ V^T, softmax + P quantize, P V
+SCALE = 1.0 / np.sqrt(128.0)
+
+
+@pytest.mark.parametrize("T,Hn", [(1, 1), (130, 3), (300, 40), (75600, 40)])
+def test_quantize_heads_vt_bit_exact(fb, orc, T, Hn):
+    import torch
+
+    v = synth.activation(3700 + T + Hn, T, Hn * D, "lognormal", gain_seed=3701)
+    c_ref, s_ref = orc.quantize_heads_vt(v, Hn)
+    codes, sf = fb.quantize_heads_vt(H.dev_bf16(v), Hn)
+    st = fb.fp4_sync_status()
+    assert st == 0, fb.fp4_status_string(st)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(H.host_u8(codes), c_ref)
+    np.testing.assert_array_equal(H.host_u8(sf), s_ref)
+
+
+def _scores_bits(seed, Tq, kpad, T_kv, sigma=4.0):
+    """Seeded bf16 scores [Tq, kpad]; the padding keys hold large values the softmax must ignore."""
+    rng = np.random.default_rng(seed)
+    s = rng.normal(0.0, sigma, size=(Tq, kpad)).astype(np.float32)
+    s[:, T_kv:] = 1.0e4
+    return synth.f32_to_bf16_bits(s)
+
+
+def _check_p(orc, s_bits, T_kv, p_codes_h, p_sf_h, stats_h, rows, what):
+    """P codes / scales admissible for the fp64 softmax within the library's bound; stats'
+    m exact (the fp32 maximum of fl(s c)), l within the bound of the exact sum."""
+    from oracle import oracle_np as onp
+
+    kpad = s_bits.shape[1]
+    p, tmax = orc.softmax_rows(s_bits, T_kv, SCALE)
+    eps = orc.softmax_bound(kpad, tmax)[:, None]
+    tiny = 2.0 ** -125
+    lo = np.maximum(p * (1 - eps) - tiny, 0.0)
+    hi = p * (1 + eps) + tiny
+    lo[:, T_kv:] = 0.0
+    hi[:, T_kv:] = 0.0
+    H.check_quant_of_interval(MX, p_codes_h, p_sf_h, lo, hi, None, what, row_ids=rows)
+    c = np.float32(orc.softmax_c(SCALE))
+    u = (orc.synth_bits_to_f64(s_bits)[:, :T_kv].astype(np.float32) * c).astype(np.float32)
+    np.testing.assert_array_equal(stats_h[:, 0], u.max(axis=1))
+    e_exact = np.exp2(u.astype(np.float64) - u.max(axis=1, keepdims=True).astype(np.float64)).sum(axis=1)
+    assert (np.abs(stats_h[:, 1] - e_exact) <= eps[:, 0] * e_exact).all(), what
+
+
+@pytest.mark.parametrize("Tq,T_kv", [(1, 1), (130, 200), (300, 257), (64, 75600), (8, 102500)])
+def test_softmax_quant_admissible(fb, orc, Tq, T_kv):
+    import torch
+
+    from oracle import oracle_np as onp
+
+    kpad = (T_kv + 127) // 128 * 128
+    s_bits = _scores_bits(3800 + Tq + T_kv, Tq, kpad, T_kv)
+    pc, ps, stats = fb.attn_softmax_quant(H.dev_bf16(s_bits), Tq, T_kv, SCALE)
+    st = fb.fp4_sync_status()
+    assert st == 0, fb.fp4_status_string(st)
+    torch.cuda.synchronize()
+    qpad = (Tq + 127) // 128 * 128
+    sf_all = onp.unswizzle_sf(H.host_u8(ps), qpad, kpad // 32)
+    assert not sf_all[Tq:].any(), "padding query rows hold zero scale bytes"
+    _check_p(orc, s_bits, T_kv, H.host_u8(pc), sf_all[:Tq], stats.cpu().numpy(), np.arange(Tq),
+             f"softmax Tq={Tq} T_kv={T_kv}")
+
+
+def _pv_case(fb, orc, Tq, T_kv, Hn, head, seed, rows=None):
+    import torch
+
+    from oracle import oracle_np as onp
+
+    kpad = (T_kv + 127) // 128 * 128
+    s_bits = _scores_bits(seed, Tq, kpad, T_kv, sigma=2.0)
+    v = synth.activation(seed + 1, T_kv, Hn * D, "lognormal", gain_seed=seed + 2)
+    pc, ps, _ = fb.attn_softmax_quant(H.dev_bf16(s_bits), Tq, T_kv, SCALE)
+    vt = fb.quantize_heads_vt(H.dev_bf16(v), Hn)
+    o = fb.attn_pv((pc, ps), vt, Tq, T_kv, head)
+    st = fb.fp4_sync_status()
+    assert st == 0, fb.fp4_status_string(st)
+    torch.cuda.synchronize()
+    rows = np.arange(Tq) if rows is None else rows
+    vt_ref = orc.quantize_heads_vt(v, Hn)
+    np.testing.assert_array_equal(H.host_u8(vt[0][head]), vt_ref[0][head])
+    pc_h = H.host_u8(pc)[rows]
+    qpad = (Tq + 127) // 128 * 128
+    ps_rows = onp.unswizzle_sf(H.host_u8(ps), qpad, kpad // 32)[rows]
+    # re-swizzle the sampled rows as a small [len(rows), kpad] operand for the oracle
+    ps_small = np.zeros(orc.sf_bytes(len(rows), kpad // 32), dtype=np.uint8)
+    for i in range(len(rows)):
+        for j in range(kpad // 32):
+            ps_small[orc.sf_offset(i, j, kpad // 32)] = ps_rows[i, j]
+    Y, S = orc.pv_rows(pc_h, ps_small, vt_ref, head, kpad, np.arange(len(rows)))
+    H.check_linear(o[torch.as_tensor(rows, device="cuda")], Y, S, np.arange(len(rows)),
+                   f"P V Tq={Tq} T_kv={T_kv} H={Hn} head={head}")
+    return o
+
+
+@pytest.mark.parametrize("Tq,T_kv,Hn,head", [(1, 1, 1, 0), (130, 200, 3, 2), (300, 257, 2, 1), (200, 4096, 40, 39)])
+def test_attn_pv_all_elements(fb, orc, Tq, T_kv, Hn, head):
+    _pv_case(fb, orc, Tq, T_kv, Hn, head, seed=3900 + Tq + T_kv)
+
+
+def test_attn_chain_full_size_sampled(fb, orc):
+    """The whole head at 75600 tokens, 40 heads, head 17: scores -> softmax + P quantize ->
+    P V, each stage checked on sampled query rows against the oracle fed that stage's GPU input."""
+    import torch
+
+    from oracle import oracle_np as onp
+
+    T, Hn, head = 75600, 40, 17
+    kpad = 75648
+    rows = H.sample_rows(T, n_random=12, seed=21)
+    q = synth.activation(4100, T, Hn * D, "lognormal", gain_seed=4101)
+    k = synth.activation(4102, T, Hn * D, "lognormal", gain_seed=4103)
+    v = synth.activation(4104, T, Hn * D, "lognormal", gain_seed=4105)
+    qh = fb.quantize_heads(H.dev_bf16(q), Hn)
+    kh = fb.quantize_heads(H.dev_bf16(k), Hn)
+    s = fb.attn_scores(qh, kh, T, T, head)
+    pc, ps, stats = fb.attn_softmax_quant(s, T, T, SCALE)
+    vt = fb.quantize_heads_vt(H.dev_bf16(v), Hn)
+    o = fb.attn_pv((pc, ps), vt, T, T, head)
+    st = fb.fp4_sync_status()
+    assert st == 0, fb.fp4_status_string(st)
+    torch.cuda.synchronize()
+    idx = torch.as_tensor(rows, device="cuda")
+    s_bits = s[idx].contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+    sf_all = onp.unswizzle_sf(H.host_u8(ps), kpad, kpad // 32)
+    _check_p(orc, s_bits, T, H.host_u8(pc[idx]), sf_all[rows], stats[idx].cpu().numpy(), rows,
+             "softmax full size")
+    vt_ref = orc.quantize_heads_vt(v, Hn)
+    np.testing.assert_array_equal(H.host_u8(vt[0][head]), vt_ref[0][head])
+    np.testing.assert_array_equal(H.host_u8(vt[1][head]), vt_ref[1][head])
+    ps_small = np.zeros(orc.sf_bytes(len(rows), kpad // 32), dtype=np.uint8)
+    for i in range(len(rows)):
+        for j in range(kpad // 32):
+            ps_small[orc.sf_offset(i, j, kpad // 32)] = sf_all[rows[i], j]
+    Y, S = orc.pv_rows(H.host_u8(pc[idx]), ps_small, vt_ref, head, kpad, np.arange(len(rows)))
+    H.check_linear(o[idx], Y, S, np.arange(len(rows)), "P V full size")
+
+
+def test_attn_chain_close_to_unquantized_attention(fb, orc):
+    """Sanity of the wiring, not a parity claim: the FP4 chain's O against fp64 attention on
+    the unquantized bf16 inputs (q, k ~ N(0, 1), so the softmax is not one-hot and FP4 noise
+    in S cannot move its argmax).  The same chain emulated with the oracle (P rounded to
+    bf16 before its quantization) gives row cosines of median 0.968, minimum 0.835 here;
+    FP4 attention is coarse, as the card says of SageAttention v3."""
+    import torch
+
+    T, Hn, head = 1000, 2, 1
+    rng = np.random.default_rng(4200)
+    q = synth.f32_to_bf16_bits(rng.normal(size=(T, Hn * D)).astype(np.float32))
+    k = synth.f32_to_bf16_bits(rng.normal(size=(T, Hn * D)).astype(np.float32))
+    v = synth.activation(4202, T, Hn * D, "lognormal")
+    qh = fb.quantize_heads(H.dev_bf16(q), Hn)
+    kh = fb.quantize_heads(H.dev_bf16(k), Hn)
+    s = fb.attn_scores(qh, kh, T, T, head)
+    pc, ps, _ = fb.attn_softmax_quant(s, T, T, SCALE)
+    o = fb.attn_pv((pc, ps), fb.quantize_heads_vt(H.dev_bf16(v), Hn), T, T, head)
+    torch.cuda.synchronize()
+    of = H.host_bf16_as_f64(o)
+    qf, kf, vf = (orc.synth_bits_to_f64(a)[:, head * D:(head + 1) * D] for a in (q, k, v))
+    sc = qf @ kf.T * SCALE
+    pr = np.exp(sc - sc.max(axis=1, keepdims=True))
+    pr /= pr.sum(axis=1, keepdims=True)
+    ref = pr @ vf
+    cos = (of * ref).sum(1) / np.linalg.norm(of, axis=1) / np.linalg.norm(ref, axis=1)
+    assert np.median(cos) > 0.95 and cos.min() > 0.7, (np.median(cos), cos.min())
