@@ -385,9 +385,11 @@ fp4_status_t fp4_quantize_heads_vt(fp4_fmt_t fmt, const void* v_bf16, int64_t T,
  *           are ignored)
  *   scale   the softmax scale (e.g. 1/sqrt(D)), > 0 and finite; the kernels use
  *           c = fp32(scale * log2 e), t_j = fl(fl(s_j c) - m), m = max_j fl(s_j c) over
- *           j < T_kv, l = sum_j exp2(t_j) (fp32, a fixed order per row), p_j = fl(exp2(t_j) *
- *           fl(1/l)); exp2 is CUDA's exp2f (within 2 ulp), so p is the softmax within
- *           a relative 2e-4 (the bound the tests apply)
+ *           j < T_kv, l = sum_j exp2(t_j) (fp32; each of a row's 256 threads adds its keys in
+ *           order, then a fixed tree), p_j = fl(exp2(t_j) * fl(1/l)); exp2 is CUDA's exp2f
+ *           (within 2 ulp).  p is then the exact softmax of s * scale within a relative
+ *           2 (2 (ln2 * 4 max|s c| + 4) + 8 ceil(T_kv_pad / 2048) + 14) 2^-24 (about 7e-5
+ *           at 75648 keys and max|s c| = 50), the bound the tests hold it to
  *   stats   (device, out) [T_q] pairs of fp32 (m, l)
  *   p_codes (device, out) [T_q][T_kv_pad/2]; p_sf (device, out) fp4_sf_bytes(MXFP4, T_q,
  *           T_kv_pad): p quantized by the MXFP4 rules above; keys >= T_kv hold p = 0 and
