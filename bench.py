@@ -533,24 +533,25 @@ def extra_workloads(fb, torch, args, steps: int = 20, warmup: int = 3):
                     n=10)
         r_s["s_write_gbs"] = s_buf.numel() * 2 / (r_s["ms"] / 1e3) / 1e9
         out[f"{fmt}_attn_scores_head_75600x75648x128"] = r_s
-        if fmt == "mxfp4":
-            # the rest of the head (MXFP4): V^T quantizer (all 40 heads), softmax + P quantize,
-            # and O = P V (K = the 75648 padded keys)
-            va = act(Ta, Ha * 128)
-            vt = fb.quantize_heads_vt(va, Ha)
-            kp = s_buf.shape[1]
-            r_v = timed(lambda: fb.fp4_quantize_heads_vt(f, va, Ta, Ha, 128, vt[0], vt[1]), 0.0)
-            r_v["gbs"] = (Ta * Ha * 128 * 2 + vt[0].numel() + vt[1].numel()) / (r_v["ms"] / 1e3) / 1e9
-            out["mxfp4_attn_quantize_heads_vt_75600x40x128"] = r_v
-            pc, ps, st = fb.attn_softmax_quant(s_buf, Ta, Ta, 128 ** -0.5)
-            r_m = timed(lambda: fb.fp4_attn_softmax_quant(f, s_buf, Ta, Ta, 128 ** -0.5, st, pc, ps), 0.0, n=10)
-            # S read three times (row max, row sum, quantize), P codes and scales written
-            r_m["gbs"] = (3 * s_buf.numel() * 2 + pc.numel() + ps.numel()) / (r_m["ms"] / 1e3) / 1e9
-            out["mxfp4_attn_softmax_quant_head_75600x75648"] = r_m
-            o_buf = fb.attn_pv((pc, ps), vt, Ta, Ta, 17)
-            out["mxfp4_attn_pv_head_75600x128x75648"] = timed(
-                lambda: fb.attn_pv((pc, ps), vt, Ta, Ta, 17, o=o_buf), 2.0 * Ta * kp * 128, n=10)
-            del va, vt, pc, ps, st, o_buf
+        # the rest of the head: V^T quantizer (all 40 heads), softmax + P quantize, and O = P V
+        # (K = the 75648 padded keys); NVFP4 with V's global and P's constant 1/2688
+        va = act(Ta, Ha * 128)
+        g_v = fb.calibrate_act_global(va)[0] if fmt == "nvfp4" else None
+        g_p = torch.tensor([fb.P_GLOBAL_NVFP4], dtype=torch.float32, device="cuda") if fmt == "nvfp4" else None
+        vt = fb.quantize_heads_vt(va, Ha, fmt, g_v)
+        kp = s_buf.shape[1]
+        r_v = timed(lambda: fb.fp4_quantize_heads_vt(f, va, Ta, Ha, 128, g_v, vt[0], vt[1]), 0.0)
+        r_v["gbs"] = (Ta * Ha * 128 * 2 + vt[0].numel() + vt[1].numel()) / (r_v["ms"] / 1e3) / 1e9
+        out[f"{fmt}_attn_quantize_heads_vt_75600x40x128"] = r_v
+        pc, ps, st = fb.attn_softmax_quant(s_buf, Ta, Ta, 128 ** -0.5, fmt, g_p)
+        r_m = timed(lambda: fb.fp4_attn_softmax_quant(f, s_buf, Ta, Ta, 128 ** -0.5, g_p, st, pc, ps), 0.0, n=10)
+        # S read three times (row max, row sum, quantize), P codes and scales written
+        r_m["gbs"] = (3 * s_buf.numel() * 2 + pc.numel() + ps.numel()) / (r_m["ms"] / 1e3) / 1e9
+        out[f"{fmt}_attn_softmax_quant_head_75600x75648"] = r_m
+        o_buf = fb.attn_pv((pc, ps), vt, Ta, Ta, 17, fmt, g_p, g_v)
+        out[f"{fmt}_attn_pv_head_75600x128x75648"] = timed(
+            lambda: fb.attn_pv((pc, ps), vt, Ta, Ta, 17, fmt, g_p, g_v, o=o_buf), 2.0 * Ta * kp * 128, n=10)
+        del va, vt, pc, ps, st, o_buf
         del qa, ka, qh, kh, kc_buf, ks_buf, s_buf
     # W4A8 SVDQuant linear at the TI2V-5B shape (MXFP8 activations, rank 32)
     Mw, Kw, Nw, r = 4290, 3072, 14336, 32

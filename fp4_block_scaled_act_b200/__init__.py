@@ -86,9 +86,9 @@ def lib():
             "fp4_attn_scores": (I, [I, P, P, I64, P, P, I64, I64, I64, I64, P, P, P, P]),
             "fp4_heads_vt_codes_bytes": (SZ, [I, I64, I64, I64]),
             "fp4_heads_vt_sf_bytes": (SZ, [I, I64, I64, I64]),
-            "fp4_quantize_heads_vt": (I, [I, P, I64, I64, I64, P, P, P]),
-            "fp4_attn_softmax_quant": (I, [I, P, I64, I64, ctypes.c_float, P, P, P, P]),
-            "fp4_attn_pv": (I, [I, P, P, I64, I64, P, P, I64, I64, I64, P, P]),
+            "fp4_quantize_heads_vt": (I, [I, P, I64, I64, I64, P, P, P, P]),
+            "fp4_attn_softmax_quant": (I, [I, P, I64, I64, ctypes.c_float, P, P, P, P, P]),
+            "fp4_attn_pv": (I, [I, P, P, P, I64, I64, P, P, P, I64, I64, I64, P, P]),
             "fp4_sync_status": (I, [P]),
             "fp4_status_string": (ctypes.c_char_p, [I]),
             "fp4_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
@@ -280,20 +280,21 @@ def fp4_heads_vt_sf_bytes(fmt, T: int, H: int, D: int = 128) -> int:
     return lib().fp4_heads_vt_sf_bytes(_fmt(fmt), T, H, D)
 
 
-def fp4_quantize_heads_vt(fmt, v, T: int, H: int, D: int, codes, sf, stream=None):
-    _check(lib().fp4_quantize_heads_vt(_fmt(fmt), _ptr(v), T, H, D, _ptr(codes), _ptr(sf), _stream(stream)),
-           "fp4_quantize_heads_vt")
+def fp4_quantize_heads_vt(fmt, v, T: int, H: int, D: int, g, codes, sf, stream=None):
+    _check(lib().fp4_quantize_heads_vt(_fmt(fmt), _ptr(v), T, H, D, _ptr(g), _ptr(codes), _ptr(sf),
+                                       _stream(stream)), "fp4_quantize_heads_vt")
 
 
-def fp4_attn_softmax_quant(fmt, s, T_q: int, T_kv: int, scale: float, stats, p_codes, p_sf, stream=None):
-    _check(lib().fp4_attn_softmax_quant(_fmt(fmt), _ptr(s), T_q, T_kv, float(scale), _ptr(stats), _ptr(p_codes),
-                                        _ptr(p_sf), _stream(stream)), "fp4_attn_softmax_quant")
+def fp4_attn_softmax_quant(fmt, s, T_q: int, T_kv: int, scale: float, p_global, stats, p_codes, p_sf,
+                           stream=None):
+    _check(lib().fp4_attn_softmax_quant(_fmt(fmt), _ptr(s), T_q, T_kv, float(scale), _ptr(p_global), _ptr(stats),
+                                        _ptr(p_codes), _ptr(p_sf), _stream(stream)), "fp4_attn_softmax_quant")
 
 
-def fp4_attn_pv(fmt, p_codes, p_sf, T_q: int, T_kv: int, vt_codes, vt_sf, H: int, D: int, head: int, o,
-                stream=None):
-    _check(lib().fp4_attn_pv(_fmt(fmt), _ptr(p_codes), _ptr(p_sf), T_q, T_kv, _ptr(vt_codes), _ptr(vt_sf), H, D,
-                             head, _ptr(o), _stream(stream)), "fp4_attn_pv")
+def fp4_attn_pv(fmt, p_codes, p_sf, p_global, T_q: int, T_kv: int, vt_codes, vt_sf, v_global, H: int, D: int,
+                head: int, o, stream=None):
+    _check(lib().fp4_attn_pv(_fmt(fmt), _ptr(p_codes), _ptr(p_sf), _ptr(p_global), T_q, T_kv, _ptr(vt_codes),
+                             _ptr(vt_sf), _ptr(v_global), H, D, head, _ptr(o), _stream(stream)), "fp4_attn_pv")
 
 
 def fp4_sync_status(stream=None) -> int:
@@ -399,41 +400,49 @@ def attn_scores(q_heads, k_heads, T_q: int, T_kv: int, head: int, fmt="mxfp4", g
     return s
 
 
-def quantize_heads_vt(v, H: int, stream=None):
-    """bf16 [T, H * 128] (CUDA) -> head-major V^T in MXFP4 (codes [H, 128, Tpad/2], scales [H, bytes per head])."""
+P_GLOBAL_NVFP4 = 1.0 / 2688.0   # P's NVFP4 global: p <= 1, so T / (6 * 448) with T = 1
+
+
+def quantize_heads_vt(v, H: int, fmt="mxfp4", g=None, stream=None):
+    """bf16 [T, H * 128] (CUDA) -> head-major V^T (codes [H, 128, Tpad/2], scales [H, bytes per head])."""
     import torch
 
+    f = _fmt(fmt)
     T, HD = v.shape
     D = HD // H
     Tpad = (T + 127) // 128 * 128
     codes = torch.empty((H, D, Tpad // 2), dtype=torch.uint8, device=v.device)
-    sf = torch.empty((H, fp4_heads_vt_sf_bytes(MXFP4, T, H, D) // H), dtype=torch.uint8, device=v.device)
-    fp4_quantize_heads_vt(MXFP4, v, T, H, D, codes, sf, stream)
+    sf = torch.empty((H, fp4_heads_vt_sf_bytes(f, T, H, D) // H), dtype=torch.uint8, device=v.device)
+    fp4_quantize_heads_vt(f, v, T, H, D, g, codes, sf, stream)
     return codes, sf
 
 
-def attn_softmax_quant(s, T_q: int, T_kv: int, scale: float, stream=None):
-    """Scores bf16 [T_q, T_kv_pad] (CUDA) -> (P codes [T_q, T_kv_pad/2], P scales, (m, l) stats [T_q, 2]) in MXFP4."""
+def attn_softmax_quant(s, T_q: int, T_kv: int, scale: float, fmt="mxfp4", p_global=None, stream=None):
+    """Scores bf16 [T_q, T_kv_pad] (CUDA) -> (P codes [T_q, T_kv_pad/2], P scales, (m, l) stats [T_q, 2]).
+    NVFP4 needs p_global (a one-element fp32 device tensor, P_GLOBAL_NVFP4)."""
     import torch
 
+    f = _fmt(fmt)
     kpad = s.shape[1]
     p_codes = torch.empty((T_q, kpad // 2), dtype=torch.uint8, device=s.device)
-    p_sf = torch.empty(fp4_sf_bytes(MXFP4, T_q, kpad), dtype=torch.uint8, device=s.device)
+    p_sf = torch.empty(fp4_sf_bytes(f, T_q, kpad), dtype=torch.uint8, device=s.device)
     stats = torch.empty((T_q, 2), dtype=torch.float32, device=s.device)
-    fp4_attn_softmax_quant(MXFP4, s, T_q, T_kv, scale, stats, p_codes, p_sf, stream)
+    fp4_attn_softmax_quant(f, s, T_q, T_kv, scale, p_global, stats, p_codes, p_sf, stream)
     return p_codes, p_sf, stats
 
 
-def attn_pv(p, vt_heads, T_q: int, T_kv: int, head: int, o=None, stream=None):
+def attn_pv(p, vt_heads, T_q: int, T_kv: int, head: int, fmt="mxfp4", p_global=None, v_global=None, o=None,
+            stream=None):
     """O = deq(P) deq(V_head) -> bf16 [T_q, 128] from attn_softmax_quant's P and quantize_heads_vt's V^T."""
     import torch
 
+    f = _fmt(fmt)
     p_codes, p_sf = p[0], p[1]
     vc, vs = vt_heads
     H, D, _ = vc.shape
     if o is None:
         o = torch.empty((T_q, D), dtype=torch.bfloat16, device=p_codes.device)
-    fp4_attn_pv(MXFP4, p_codes, p_sf, T_q, T_kv, vc, vs, H, D, head, o, stream)
+    fp4_attn_pv(f, p_codes, p_sf, p_global, T_q, T_kv, vc, vs, v_global, H, D, head, o, stream)
     return o
 
 

@@ -3,10 +3,12 @@
 //
 // Reading followed (the Wan2.2-Animate-14B MXFP4 card, "Results", names SageAttention v3 as
 // Blackwell microscaling FP4 attention without giving its algorithm): P = softmax(S * scale)
-// per query row over the T_kv keys, quantized in MXFP4 blocks of 32 consecutive keys; V of a
-// head quantized per head-dim channel in MXFP4 blocks of 32 consecutive tokens; O = deq(P)
-// deq(V) by the block-scaled GEMM (its K is the key axis, so both operands carry their
-// scales along the keys).
+// per query row over the T_kv keys, quantized in blocks of G consecutive keys; V of a head
+// quantized per head-dim channel in blocks of G consecutive tokens; O = deq(P) deq(V) by the
+// block-scaled GEMM (its K is the key axis, so both operands carry their scales along the
+// keys).  MXFP4: G = 32, E8M0 scales.  NVFP4: G = 16, E4M3 scales under one fp32 global per
+// tensor (V's from its amax; P's is a caller's constant, 1 / 2688 for p <= 1), by the same
+// steps as the activation quantizer.
 //
 // Layouts (head-major, as the score operands):
 //   V^T  codes [H][128 dims][Tpad/2] bytes (tokens along K; padding tokens hold zero codes),
@@ -26,15 +28,26 @@ constexpr int VT_PITCH = 136;   // bf16 elements per staged token row (16 bytes 
 constexpr int SOFTMAX_THREADS = 256;
 
 // V^T quantizer: block (token block tb, head h) stages V[tb*128 .. +127][h*128 .. +127] in
-// shared memory; thread d (a head-dim channel) quantizes the four 32-token groups of its
-// column and writes their 64 code bytes and one scale word.
+// shared memory; thread d (a head-dim channel) quantizes the 128 / G groups of its column
+// and writes their 64 code bytes and its scale word(s) (one MXFP4 atom, two NVFP4 atoms).
+template <int KIND>
 __global__ void __launch_bounds__(128) quant_vt_kernel(const __nv_bfloat16* __restrict__ v, int64_t T, int H,
-                                                       int64_t tpad, uint8_t* __restrict__ codes,
-                                                       uint8_t* __restrict__ sf) {
+                                                       int64_t tpad, const float* __restrict__ g_ptr,
+                                                       uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+    constexpr int G = (KIND == Q_NVFP4) ? 16 : 32;
     __shared__ __align__(16) __nv_bfloat16 tile[VT_TOKENS * VT_PITCH];
+    __shared__ float nv_rcp[128];
     const int tb = blockIdx.x, h = blockIdx.y;
     const int64_t t0 = (int64_t)tb * VT_TOKENS;
     const int64_t row_elems = (int64_t)H * 128;
+    float six_g = 6.0f;
+    if (KIND == Q_NVFP4) {
+        // 1 / (e4m3(sf) * g) for every scale byte, by the activation quantizer's operations
+        const float g = *g_ptr;
+        six_g = __fmul_rn(6.0f, g);
+        const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
+        nv_rcp[threadIdx.x] = d == 0.0f ? 0.0f : __frcp_rn(d);
+    }
     // 128 token rows x 256 bytes as 16-byte chunks: 2048 chunks over 128 threads
     for (int c = threadIdx.x; c < VT_TOKENS * 16; c += 128) {
         const int r = c >> 4, q = c & 15;
@@ -44,33 +57,45 @@ __global__ void __launch_bounds__(128) quant_vt_kernel(const __nv_bfloat16* __re
     }
     __syncthreads();
     const int d = threadIdx.x;
-    uint32_t word = 0;
+    uint32_t words[2] = {0u, 0u};
     uint8_t* crow = codes + ((int64_t)h * 128 + d) * (tpad / 2) + t0 / 2;
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-        float x[32];
+    for (int g = 0; g < 128 / G; ++g) {
+        float x[G];
         float amax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            x[i] = __bfloat162float(tile[(g * 32 + i) * VT_PITCH + d]);
+        for (int i = 0; i < G; ++i) {
+            x[i] = __bfloat162float(tile[(g * G + i) * VT_PITCH + d]);
             amax = fmaxf(amax, fabsf(x[i]));
         }
-        const uint32_t sfb = mx_scale_byte<2>(amax);
-        const float inv = mx_inv_scale(sfb);
-        uint32_t cw[4];
+        uint32_t sfb;
+        if (KIND == Q_NVFP4) {
+            sfb = cvt_e4m3x2(__fdiv_rn(amax, six_g), 0.0f) & 0xFFu;
+            const float r = nv_rcp[sfb & 0x7Fu];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float e[8];
+            for (int i = 0; i < G; ++i) x[i] = (r == 0.0f) ? 0.0f : __fmul_rn(x[i], r);
+        } else {
+            sfb = mx_scale_byte<2>(amax);
+            const float inv = mx_inv_scale(sfb);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) e[i] = __fmul_rn(x[q * 8 + i], inv);
-            cw[q] = cvt_e2m1x8(e);
+            for (int i = 0; i < G; ++i) x[i] = __fmul_rn(x[i], inv);
         }
-        *reinterpret_cast<uint4*>(crow + g * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        word |= sfb << (8 * g);
+        uint32_t cw[G / 8];
+#pragma unroll
+        for (int q = 0; q < G / 8; ++q) cw[q] = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(x + 8 * q));
+        if constexpr (G == 32)
+            *reinterpret_cast<uint4*>(crow + g * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        else
+            *reinterpret_cast<uint2*>(crow + g * 8) = make_uint2(cw[0], cw[1]);
+        words[g >> 2] |= sfb << (8 * (g & 3));
     }
     // head h's scales: rows = the 128 channels (one row block), atoms along the Tpad tokens
-    const int64_t apr = tpad / 128;
-    *reinterpret_cast<uint32_t*>(sf + (int64_t)h * apr * 512 + sf_word_offset(d, tb, apr)) = word;
+    constexpr int ATOMS = 128 / (G * 4);  // atoms per 128 tokens: MXFP4 1, NVFP4 2
+    const int64_t apr = tpad / (G * 4);
+#pragma unroll
+    for (int a = 0; a < ATOMS; ++a)
+        *reinterpret_cast<uint32_t*>(sf + (int64_t)h * apr * 512 + sf_word_offset(d, (int64_t)tb * ATOMS + a, apr)) =
+            words[a];
 }
 
 // The softmax argument of a score in fp32, the same two roundings in both softmax kernels:
@@ -124,19 +149,34 @@ __global__ void __launch_bounds__(SOFTMAX_THREADS) softmax_stats_kernel(const __
     if (threadIdx.x == 0) stats[blockIdx.x] = make_float2(m, l);
 }
 
-// P = exp2(t_j) * (1 / l), quantized in MXFP4 groups of 32 keys.  One block per query row
-// of the padded [T_q_pad, T_kv_pad] layout; its 8 warps take 256-key chunks in turn, a lane
-// 8 keys (16-byte load, 4-byte code store), 4 lanes a group.  Keys j >= T_kv give p = 0;
-// rows >= T_q write only zero scale bytes (the layout's padding).
+// P = exp2(t_j) * (1 / l), quantized in groups of G keys (MXFP4 32, NVFP4 16 under the
+// global *g_ptr).  One block per query row of the padded [T_q_pad, T_kv_pad] layout; its 8
+// warps take 256-key chunks in turn, a lane 8 keys (16-byte load, 4-byte code store), G / 8
+// lanes a group.  Keys j >= T_kv give p = 0; rows >= T_q write only zero scale bytes (the
+// layout's padding).
+template <int KIND>
 __global__ void __launch_bounds__(SOFTMAX_THREADS) softmax_quant_kernel(const __nv_bfloat16* __restrict__ s,
                                                                        int64_t T_q, int64_t kpad, int64_t T_kv,
                                                                        float c, const float2* __restrict__ stats,
+                                                                       const float* __restrict__ g_ptr,
                                                                        uint8_t* __restrict__ p_codes,
                                                                        uint8_t* __restrict__ p_sf) {
+    constexpr int G = (KIND == Q_NVFP4) ? 16 : 32;
+    __shared__ float nv_rcp[128];
     const int64_t r = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t apr = kpad / 128;
+    const int64_t apr = kpad / (G * 4);
     const bool real = r < T_q;
+    float six_g = 6.0f;
+    if (KIND == Q_NVFP4) {
+        const float g = *g_ptr;
+        six_g = __fmul_rn(6.0f, g);
+        if (threadIdx.x < 128) {
+            const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
+            nv_rcp[threadIdx.x] = d == 0.0f ? 0.0f : __frcp_rn(d);
+        }
+        __syncthreads();
+    }
     float m = 0.0f, inv_l = 0.0f;
     if (real) {
         const float2 st = stats[r];
@@ -161,21 +201,27 @@ __global__ void __launch_bounds__(SOFTMAX_THREADS) softmax_quant_kernel(const __
             for (int k = 0; k < 8; ++k) p[k] = 0.0f;
         }
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        const uint32_t sfb = mx_scale_byte<2>(amax);
-        if (real && in) {
+        if (G == 32) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        uint32_t sfb;
+        if (KIND == Q_NVFP4) {
+            sfb = cvt_e4m3x2(__fdiv_rn(amax, six_g), 0.0f) & 0xFFu;
+            const float rr = nv_rcp[sfb & 0x7Fu];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) p[k] = (rr == 0.0f) ? 0.0f : __fmul_rn(p[k], rr);
+        } else {
+            sfb = mx_scale_byte<2>(amax);
             const float inv = mx_inv_scale(sfb);
 #pragma unroll
             for (int k = 0; k < 8; ++k) p[k] = __fmul_rn(p[k], inv);
-            *reinterpret_cast<uint32_t*>(p_codes + r * (kpad / 2) + col / 2) = cvt_e2m1x8(p);
         }
-        // the 4 group bytes of each 128-key unit into one word (lanes 0-15: unit 2 chunk,
-        // lanes 16-31: unit 2 chunk + 1)
-        uint32_t word = sfb << (8 * ((lane & 15) >> 2));
-        word |= __shfl_xor_sync(0xffffffffu, word, 4);
-        word |= __shfl_xor_sync(0xffffffffu, word, 8);
-        if ((lane & 15) == 0 && in)
-            *reinterpret_cast<uint32_t*>(p_sf + sf_word_offset(r, chunk * 2 + (lane >> 4), apr)) = word;
+        if (real && in) *reinterpret_cast<uint32_t*>(p_codes + r * (kpad / 2) + col / 2) = cvt_e2m1x8(p);
+        // the 4 group bytes of each atom word: MXFP4 16 lanes (128 keys) per word, NVFP4 8 (64)
+        constexpr int LW = G / 2;  // lanes per word
+        uint32_t word = sfb << (8 * ((lane % LW) / (G / 8)));
+        word |= __shfl_xor_sync(0xffffffffu, word, G / 8);
+        word |= __shfl_xor_sync(0xffffffffu, word, G / 4);
+        if (lane % LW == 0 && in)
+            *reinterpret_cast<uint32_t*>(p_sf + sf_word_offset(r, (chunk * 256 + lane * 8) / (G * 4), apr)) = word;
     }
 }
 

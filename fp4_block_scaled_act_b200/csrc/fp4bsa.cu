@@ -616,33 +616,43 @@ fp4_status_t fp4_gemm(fp4_fmt_t fmt, const uint8_t* a_codes, const uint8_t* a_sf
 }
 
 size_t fp4_heads_vt_codes_bytes(fp4_fmt_t fmt, int64_t T, int64_t H, int64_t D) {
-    if (fmt != FP4_FMT_MXFP4 || T < 0 || H < 0 || D != FP4_HEAD_DIM) return 0;
+    if (!fmt_ok(fmt) || T < 0 || H < 0 || D != FP4_HEAD_DIM) return 0;
     return (size_t)H * (size_t)D * (size_t)((T + 127) / 128 * 128 / 2);
 }
 
 size_t fp4_heads_vt_sf_bytes(fp4_fmt_t fmt, int64_t T, int64_t H, int64_t D) {
-    if (fmt != FP4_FMT_MXFP4 || T < 0 || H < 0 || D != FP4_HEAD_DIM) return 0;
+    if (!fmt_ok(fmt) || T < 0 || H < 0 || D != FP4_HEAD_DIM) return 0;
     return (size_t)H * fp4_sf_bytes(fmt, D, (T + 127) / 128 * 128);
 }
 
 fp4_status_t fp4_quantize_heads_vt(fp4_fmt_t fmt, const void* v_bf16, int64_t T, int64_t H, int64_t D,
-                                   uint8_t* codes, uint8_t* sf, void* stream) {
-    if (fmt != FP4_FMT_MXFP4 || !v_bf16 || !codes || !sf || T < 1 || H < 1) return FP4_ERR_INVALID_ARG;
+                                   const float* g, uint8_t* codes, uint8_t* sf, void* stream) {
+    if (!fmt_ok(fmt) || !v_bf16 || !codes || !sf || T < 1 || H < 1) return FP4_ERR_INVALID_ARG;
+    if ((fmt == FP4_FMT_NVFP4) != (g != nullptr)) return FP4_ERR_INVALID_ARG;
     if (D != FP4_HEAD_DIM || H >= kMaxDim / D || T >= kMaxDim || H >= 65536) return FP4_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(v_bf16) || !aligned16(codes) || !aligned16(sf)) return FP4_ERR_MISALIGNED;
+    if (!aligned16(v_bf16) || !aligned16(codes) || !aligned16(sf) || (reinterpret_cast<uintptr_t>(g) & 3u))
+        return FP4_ERR_MISALIGNED;
     DeviceState* ds;
     fp4_status_t s = device_state(&ds);
     if (s != FP4_OK) return s;
     const int64_t tpad = (T + 127) / 128 * 128;
-    quant_vt_kernel<<<dim3((unsigned)(tpad / 128), (unsigned)H), 128, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const __nv_bfloat16*>(v_bf16), T, (int)H, tpad, codes, sf);
+    const dim3 grid((unsigned)(tpad / 128), (unsigned)H);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (fmt == FP4_FMT_NVFP4)
+        quant_vt_kernel<Q_NVFP4><<<grid, 128, 0, cs>>>(static_cast<const __nv_bfloat16*>(v_bf16), T, (int)H, tpad, g,
+                                                       codes, sf);
+    else
+        quant_vt_kernel<Q_MXFP4><<<grid, 128, 0, cs>>>(static_cast<const __nv_bfloat16*>(v_bf16), T, (int)H, tpad,
+                                                       nullptr, codes, sf);
     return launched();
 }
 
 fp4_status_t fp4_attn_softmax_quant(fp4_fmt_t fmt, const void* s_bf16, int64_t T_q, int64_t T_kv, float scale,
-                                    void* stats, uint8_t* p_codes, uint8_t* p_sf, void* stream) {
-    if (fmt != FP4_FMT_MXFP4 || !s_bf16 || !stats || !p_codes || !p_sf || T_q < 1 || T_kv < 1)
-        return FP4_ERR_INVALID_ARG;
+                                    const float* p_global, void* stats, uint8_t* p_codes, uint8_t* p_sf,
+                                    void* stream) {
+    if (!fmt_ok(fmt) || !s_bf16 || !stats || !p_codes || !p_sf || T_q < 1 || T_kv < 1) return FP4_ERR_INVALID_ARG;
+    if ((fmt == FP4_FMT_NVFP4) != (p_global != nullptr)) return FP4_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(p_global) & 3u) return FP4_ERR_MISALIGNED;
     if (!(scale > 0.0f) || !(scale < 3.0e38f)) return FP4_ERR_INVALID_ARG;
     if (T_q >= kMaxDim || T_kv >= kMaxDim || T_q >= (int64_t)1 << 31) return FP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(s_bf16) || !aligned16(stats) || !aligned16(p_codes) || !aligned16(p_sf))
@@ -657,16 +667,21 @@ fp4_status_t fp4_attn_softmax_quant(fp4_fmt_t fmt, const void* s_bf16, int64_t T
     softmax_stats_kernel<<<(unsigned)T_q, SOFTMAX_THREADS, 0, cs>>>(static_cast<const __nv_bfloat16*>(s_bf16), kpad,
                                                                      T_kv, c, static_cast<float2*>(stats));
     if ((st = launched()) != FP4_OK) return st;
-    softmax_quant_kernel<<<(unsigned)qpad, SOFTMAX_THREADS, 0, cs>>>(static_cast<const __nv_bfloat16*>(s_bf16), T_q,
-                                                                      kpad, T_kv, c,
-                                                                      static_cast<const float2*>(stats), p_codes, p_sf);
+    const auto sb = static_cast<const __nv_bfloat16*>(s_bf16);
+    const auto sp = static_cast<const float2*>(stats);
+    if (fmt == FP4_FMT_NVFP4)
+        softmax_quant_kernel<Q_NVFP4><<<(unsigned)qpad, SOFTMAX_THREADS, 0, cs>>>(sb, T_q, kpad, T_kv, c, sp, p_global,
+                                                                                 p_codes, p_sf);
+    else
+        softmax_quant_kernel<Q_MXFP4><<<(unsigned)qpad, SOFTMAX_THREADS, 0, cs>>>(sb, T_q, kpad, T_kv, c, sp, nullptr,
+                                                                                 p_codes, p_sf);
     return launched();
 }
 
-fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p_sf, int64_t T_q, int64_t T_kv,
-                         const uint8_t* vt_codes, const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head,
-                         void* o_bf16, void* stream) {
-    if (fmt != FP4_FMT_MXFP4 || !p_codes || !p_sf || !vt_codes || !vt_sf || !o_bf16) return FP4_ERR_INVALID_ARG;
+fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p_sf, const float* p_global,
+                         int64_t T_q, int64_t T_kv, const uint8_t* vt_codes, const uint8_t* vt_sf, const float* v_global,
+                         int64_t H, int64_t D, int64_t head, void* o_bf16, void* stream) {
+    if (!fmt_ok(fmt) || !p_codes || !p_sf || !vt_codes || !vt_sf || !o_bf16) return FP4_ERR_INVALID_ARG;
     if (T_q < 1 || T_kv < 1 || H < 1 || head < 0 || head >= H) return FP4_ERR_INVALID_ARG;
     if (D != FP4_HEAD_DIM) return FP4_ERR_UNSUPPORTED_SHAPE;
     const int64_t kpad = (T_kv + 127) / 128 * 128;
@@ -674,7 +689,8 @@ fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p
     const uint8_t* vc = vt_codes + (size_t)head * D * (kpad / 2);
     const uint8_t* vs = vt_sf + (size_t)head * fp4_sf_bytes(fmt, D, kpad);
     // O = P V_h: P is the activation operand (M = T_q, K = the padded keys), V_h^T the weight
-    return gemm_impl(fmt, p_codes, p_sf, T_q, kpad, D, vc, vs, nullptr, nullptr, nullptr, o_bf16, stream, nullptr, 0);
+    // (NVFP4: the epilogue applies g_P g_V; gemm_impl checks that both are given)
+    return gemm_impl(fmt, p_codes, p_sf, T_q, kpad, D, vc, vs, v_global, p_global, nullptr, o_bf16, stream, nullptr, 0);
 }
 
 fp4_status_t fp4_attn_scores(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,

@@ -360,25 +360,28 @@ fp4_status_t fp4_attn_scores(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_
                              int64_t D, int64_t head, const float* g_q, const float* g_k, void* s_bf16,
                              void* stream);
 
-/* The rest of one head's attention (MXFP4 only), read the same way: P = softmax(S * scale)
- * per query row over the T_kv keys, quantized in MXFP4 blocks of 32 consecutive keys; V of
- * the head quantized per head-dim channel in MXFP4 blocks of 32 consecutive tokens; and
- * O = deq(P) deq(V) by the block-scaled GEMM, whose K is then the key axis.  fp4_attn_scores,
- * fp4_attn_softmax_quant and fp4_attn_pv in sequence give one head's attention output.
+/* The rest of one head's attention, read the same way: P = softmax(S * scale) per query row
+ * over the T_kv keys, quantized in blocks of G consecutive keys; V of the head quantized per
+ * head-dim channel in blocks of G consecutive tokens; and O = deq(P) deq(V) by the
+ * block-scaled GEMM, whose K is then the key axis.  MXFP4: G = 32; NVFP4: G = 16 with E4M3
+ * scales under one fp32 global per tensor (V: from its amax, e.g. fp4_calibrate_act_global
+ * over v; P: a constant the caller provides, 1/2688 = 1/(6*448) since p <= 1).
+ * fp4_attn_scores, fp4_attn_softmax_quant and fp4_attn_pv in sequence give one head's
+ * attention output.
  *
  * Head-major layout of V^T, quantized from v [T tokens, H heads x D]:
  *   codes  [H][D][Tpad/2] bytes (head h, channel d: its Tpad tokens as packed E2M1; padding
  *          tokens hold zero codes);
- *   sf     H consecutive blocks of fp4_sf_bytes(MXFP4, D, Tpad) bytes: head h's scales in the
+ *   sf     H consecutive blocks of fp4_sf_bytes(fmt, D, Tpad) bytes: head h's scales in the
  *          sf layout above for the [D, Tpad] matrix (rows = channels, K = tokens). */
 size_t fp4_heads_vt_codes_bytes(fp4_fmt_t fmt, int64_t T, int64_t H, int64_t D);
 size_t fp4_heads_vt_sf_bytes(fp4_fmt_t fmt, int64_t T, int64_t H, int64_t D);
 
 /* Quantize v_bf16 (device) [T, H*D] bf16, row-major, into the V^T layout above (codes and
- * sf device, out).  fmt must be FP4_FMT_MXFP4 (else FP4_ERR_INVALID_ARG); D must be
+ * sf device, out).  g (device): NVFP4, V's fp32 global; MXFP4, must be NULL.  D must be
  * FP4_HEAD_DIM (else FP4_ERR_UNSUPPORTED_SHAPE); H < 65536. */
 fp4_status_t fp4_quantize_heads_vt(fp4_fmt_t fmt, const void* v_bf16, int64_t T, int64_t H, int64_t D,
-                                   uint8_t* codes, uint8_t* sf, void* stream);
+                                   const float* g, uint8_t* codes, uint8_t* sf, void* stream);
 
 /* Softmax of scores and its MXFP4 quantization.
  *   s_bf16  (device) [T_q][T_kv_pad] bf16 scores (fp4_attn_scores' output; columns >= T_kv
@@ -390,22 +393,23 @@ fp4_status_t fp4_quantize_heads_vt(fp4_fmt_t fmt, const void* v_bf16, int64_t T,
  *           (within 2 ulp).  p is then the exact softmax of s * scale within a relative
  *           2 (2 (ln2 * 4 max|s c| + 4) + 8 ceil(T_kv_pad / 2048) + 14) 2^-24 (about 7e-5
  *           at 75648 keys and max|s c| = 50), the bound the tests hold it to
+ *   p_global (device) NVFP4: P's fp32 global (1/2688 for p <= 1); MXFP4: must be NULL
  *   stats   (device, out) [T_q] pairs of fp32 (m, l)
- *   p_codes (device, out) [T_q][T_kv_pad/2]; p_sf (device, out) fp4_sf_bytes(MXFP4, T_q,
- *           T_kv_pad): p quantized by the MXFP4 rules above; keys >= T_kv hold p = 0 and
- *           padding rows zero scale bytes.
- * fmt must be FP4_FMT_MXFP4. */
+ *   p_codes (device, out) [T_q][T_kv_pad/2]; p_sf (device, out) fp4_sf_bytes(fmt, T_q,
+ *           T_kv_pad): p quantized by the format's rules above; keys >= T_kv hold p = 0 and
+ *           padding rows zero scale bytes. */
 fp4_status_t fp4_attn_softmax_quant(fp4_fmt_t fmt, const void* s_bf16, int64_t T_q, int64_t T_kv, float scale,
-                                    void* stats, uint8_t* p_codes, uint8_t* p_sf, void* stream);
+                                    const float* p_global, void* stats, uint8_t* p_codes, uint8_t* p_sf,
+                                    void* stream);
 
 /* O = deq(P) deq(V_head) for head `head`: the block-scaled GEMM with K = T_kv_pad.
- *   p_codes, p_sf      fp4_attn_softmax_quant's output (T_q rows)
- *   vt_codes, vt_sf    fp4_quantize_heads_vt's output (T_kv tokens, H heads)
- *   o_bf16  (device, out) [T_q][D] bf16
- * fmt must be FP4_FMT_MXFP4. */
-fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p_sf, int64_t T_q, int64_t T_kv,
-                         const uint8_t* vt_codes, const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head,
-                         void* o_bf16, void* stream);
+ *   p_codes, p_sf      fp4_attn_softmax_quant's output (T_q rows); p_global its NVFP4 global
+ *   vt_codes, vt_sf    fp4_quantize_heads_vt's output (T_kv tokens, H heads); v_global its
+ *                      NVFP4 global (both globals device pointers, NULL for MXFP4)
+ *   o_bf16  (device, out) [T_q][D] bf16 */
+fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p_sf, const float* p_global,
+                         int64_t T_q, int64_t T_kv, const uint8_t* vt_codes, const uint8_t* vt_sf,
+                         const float* v_global, int64_t H, int64_t D, int64_t head, void* o_bf16, void* stream);
 
 /* ----------------------------------------------------------------- status */
 

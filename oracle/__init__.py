@@ -293,21 +293,22 @@ def attn_scores_rows(fmt: int, q_heads, k_heads, head: int, rows, g_q: float | N
     return linear_fp64(a, w, None)
 
 
-def quantize_heads_vt(x_bf16: np.ndarray, H: int):
-    """V bf16 [T, H*128] -> head-major V^T in MXFP4 (codes [H, 128, Tpad/2], sf [H, sf_bytes(128, Tpad/32)]):
+def quantize_heads_vt(x_bf16: np.ndarray, H: int, fmt: int = MX, g: float | None = None):
+    """V bf16 [T, H*128] -> head-major V^T (codes [H, 128, Tpad/2], sf [H, sf_bytes(128, Tpad/G)]):
     head h is `quantize` of the [128, Tpad] matrix whose column t is token t of the head
-    (tokens >= T zero), i.e. the scales run along the tokens, the GEMM's K of P V."""
+    (tokens >= T zero), i.e. the scales run along the tokens, the GEMM's K of P V (NVFP4
+    under V's global g)."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     T, HD = x.shape
     D = HD // H
     assert D * H == HD and D == 128
     Tpad = (T + 127) // 128 * 128
     codes = np.zeros((H, D, Tpad // 2), dtype=np.uint8)
-    sfs = np.zeros((H, sf_bytes(D, Tpad // 32)), dtype=np.uint8)
+    sfs = np.zeros((H, sf_bytes(D, Tpad // group_size(fmt))), dtype=np.uint8)
     for h in range(H):
         vt = np.zeros((D, Tpad), dtype=np.uint16)
         vt[:, :T] = x[:, h * D:(h + 1) * D].T
-        codes[h], sfs[h] = quantize(MX, vt)
+        codes[h], sfs[h] = quantize(fmt, vt, g)
     return codes, sfs
 
 
@@ -346,11 +347,15 @@ def softmax_bound(T_kv_pad: int, t_max_abs):
     return 2.0 * (2.0 * term + n * u + 2.0 * u)
 
 
-def pv_rows(p_codes, p_sf, vt_heads, head: int, T_kv_pad: int, rows):
-    """(Y, S) of rows `rows` of O = deq(P) deq(V_head) (MXFP4), in fp64."""
+P_GLOBAL_NVFP4 = 1.0 / 2688.0  # the NVFP4 global of P (p <= 1): T / (6 * 448) with T = 1
+
+
+def pv_rows(p_codes, p_sf, vt_heads, head: int, T_kv_pad: int, rows, fmt: int = MX, g_p: float | None = None,
+            g_v: float | None = None):
+    """(Y, S) of rows `rows` of O = deq(P) deq(V_head), in fp64 (NVFP4 with the globals g_p, g_v)."""
     vc, vs = vt_heads
-    a = dequant_fp4(MX, p_codes, p_sf, T_kv_pad, rows=rows)
-    w = dequant_fp4(MX, vc[head], vs[head], T_kv_pad)
+    a = dequant_fp4(fmt, p_codes, p_sf, T_kv_pad, 1.0 if fmt == MX else g_p, rows=rows)
+    w = dequant_fp4(fmt, vc[head], vs[head], T_kv_pad, 1.0 if fmt == MX else g_v)
     return linear_fp64(a, w, None)
 
 

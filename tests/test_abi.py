@@ -60,6 +60,10 @@ def test_size_queries(fb):
     assert fb.fp4_heads_sf_bytes(MX, 75600, 40) == 40 * fb.fp4_sf_bytes(MX, 75600, 128) == 40 * 75648 * 4
     assert fb.fp4_heads_sf_bytes(NV, 130, 3) == 3 * 256 * 8
     assert fb.fp4_heads_codes_bytes(MX, 130, 3, 64) == 0                # head_dim 128 only
+    # V^T: [H][128][Tpad/2] codes, H blocks of [128, Tpad] scales (along the tokens)
+    assert fb.fp4_heads_vt_codes_bytes(MX, 75600, 40) == 40 * 128 * 75648 // 2
+    assert fb.fp4_heads_vt_sf_bytes(MX, 75600, 40) == 40 * fb.fp4_sf_bytes(MX, 128, 75648) == 40 * 128 * 75648 // 32
+    assert fb.fp4_heads_vt_sf_bytes(NV, 130, 3) == 3 * 128 * 256 // 16
 
 
 def test_bytes_per_weight_match_format(fb):
@@ -132,6 +136,19 @@ def test_invalid_calls_rejected_before_launch(fb):
     assert L.fp4_attn_scores(0, A, A, 16, A, A, 16, 2, 64, 0, None, None, A, st) == 2
     assert L.fp4_attn_scores(1, A, A, 16, A, A, 16, 2, 128, 0, None, None, A, st) == 1
     assert L.fp4_attn_scores(0, A, A, 16, A, A, 16, 2, 128, 0, None, None, bad, st) == 3
+    # V^T, softmax + P quantize, P V: format / global pairing, shape, alignment, head index
+    assert L.fp4_quantize_heads_vt(1, A, 16, 2, 128, None, A, A, st) == 1
+    assert L.fp4_quantize_heads_vt(0, A, 16, 2, 128, A, A, A, st) == 1
+    assert L.fp4_quantize_heads_vt(0, A, 16, 2, 96, None, A, A, st) == 2
+    assert L.fp4_quantize_heads_vt(0, A, 16, 70000, 128, None, A, A, st) == 2
+    assert L.fp4_quantize_heads_vt(0, bad, 16, 2, 128, None, A, A, st) == 3
+    assert L.fp4_attn_softmax_quant(1, A, 16, 16, 0.1, None, A, A, A, st) == 1
+    assert L.fp4_attn_softmax_quant(0, A, 16, 16, 0.0, None, A, A, A, st) == 1
+    assert L.fp4_attn_softmax_quant(0, A, 0, 16, 0.1, None, A, A, A, st) == 1
+    assert L.fp4_attn_softmax_quant(0, A, 16, 16, 0.1, None, A, bad, A, st) == 3
+    assert L.fp4_attn_pv(0, A, A, None, 16, 16, A, A, None, 2, 128, 2, A, st) == 1
+    assert L.fp4_attn_pv(1, A, A, None, 16, 16, A, A, A, 2, 128, 0, A, st) == 1
+    assert L.fp4_attn_pv(0, A, A, None, 16, 16, A, A, None, 2, 64, 0, A, st) == 2
 
 
 def test_product_path_has_no_oracle_import():

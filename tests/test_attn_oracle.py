@@ -92,12 +92,14 @@ def test_scores_select_the_head_and_rows():
 
 
 # ------------------------------------------------------------------ V^T, softmax, P V
+@pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("T,H", [(1, 1), (130, 2), (257, 3)])
-def test_quantize_heads_vt_is_the_row_quantizer_of_the_transpose(T, H):
+def test_quantize_heads_vt_is_the_row_quantizer_of_the_transpose(fmt, T, H):
     """Head h's V^T is the pinned row quantizer applied to the explicit transpose of its 128
-    columns, zero-padded to Tpad tokens: codes and every scale byte."""
+    columns, zero-padded to Tpad tokens: codes and every scale byte (NVFP4 under V's global)."""
     x = _x(900 + T + H, T, H)
-    codes, sfs = oracle.quantize_heads_vt(x, H)
+    g = oracle.nv_global(oracle.tensor_amax(x)) if fmt == NV else None
+    codes, sfs = oracle.quantize_heads_vt(x, H, fmt, g)
     Tpad = (T + 127) // 128 * 128
     assert codes.shape == (H, D, Tpad // 2)
     for h in range(H):
@@ -105,7 +107,7 @@ def test_quantize_heads_vt_is_the_row_quantizer_of_the_transpose(T, H):
         for t in range(T):
             for d in range(D):
                 vt[d, t] = x[t, h * D + d]
-        c, s = oracle.quantize(MX, vt)
+        c, s = oracle.quantize(fmt, vt, g)
         np.testing.assert_array_equal(codes[h], c)
         np.testing.assert_array_equal(sfs[h], s)
         assert not codes[h][:, (T + 1) // 2:].any(), "padding tokens hold zero codes"
@@ -173,6 +175,27 @@ def test_softmax_bound_covers_an_fp32_evaluation():
         rel = np.abs(p32.astype(np.float64) - p[r, :T_kv]) / p[r, :T_kv]
         assert rel.max() <= eps[r], (rel.max(), eps[r])
         del lanes
+
+
+def test_pv_oracle_nvfp4_exact_on_representable_blocks():
+    """NVFP4 P V on operands exact under global 1 (E2M1 values times the block's power of two,
+    each 16-block's amax 6 * 2^e, so the E4M3 block scale is 2^e) equals numpy's product of
+    the original values; a P global of 1/2 halves it exactly (the globals are applied)."""
+    rng = np.random.default_rng(7)
+    Tq, Tk, H = 2, 64, 2
+    kpad = 128
+    pv = _representable(rng, Tq, 1, 16)[:, :kpad]
+    pv[:, Tk:] = 0.0
+    pc, ps = oracle.quantize(NV, synth.f32_to_bf16_bits(pv.astype(np.float32)), 1.0)
+    vtv = _representable(rng, H * D, 1, 16)[:, :Tk]          # blocks of 16 tokens
+    v = np.ascontiguousarray(vtv.T)
+    vt = oracle.quantize_heads_vt(synth.f32_to_bf16_bits(v.astype(np.float32)), H, NV, 1.0)
+    for head in range(H):
+        ref = pv[:, :Tk] @ v[:, head * D:(head + 1) * D]
+        Y, _ = oracle.pv_rows(pc, ps, vt, head, kpad, np.arange(Tq), NV, 1.0, 1.0)
+        np.testing.assert_array_equal(Y, ref)
+        Yh, _ = oracle.pv_rows(pc, ps, vt, head, kpad, np.arange(Tq), NV, 0.5, 1.0)
+        np.testing.assert_array_equal(Yh, 0.5 * ref)
 
 
 def test_pv_oracle_exact_on_representable_blocks():

@@ -97,13 +97,19 @@ def test_attn_scores_full_size_sampled(fb, orc, fmt):
 SCALE = 1.0 / np.sqrt(128.0)
 
 
+def _fmt_name(fmt):
+    return "mxfp4" if fmt == MX else "nvfp4"
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("T,Hn", [(1, 1), (130, 3), (300, 40), (75600, 40)])
-def test_quantize_heads_vt_bit_exact(fb, orc, T, Hn):
+def test_quantize_heads_vt_bit_exact(fb, orc, fmt, T, Hn):
     import torch
 
     v = synth.activation(3700 + T + Hn, T, Hn * D, "lognormal", gain_seed=3701)
-    c_ref, s_ref = orc.quantize_heads_vt(v, Hn)
-    codes, sf = fb.quantize_heads_vt(H.dev_bf16(v), Hn)
+    g = orc.nv_global(orc.tensor_amax(v)) if fmt == NV else None
+    c_ref, s_ref = orc.quantize_heads_vt(v, Hn, fmt, g)
+    codes, sf = fb.quantize_heads_vt(H.dev_bf16(v), Hn, _fmt_name(fmt), H.dev_f32([g]) if fmt == NV else None)
     st = fb.fp4_sync_status()
     assert st == 0, fb.fp4_status_string(st)
     torch.cuda.synchronize()
@@ -119,7 +125,7 @@ def _scores_bits(seed, Tq, kpad, T_kv, sigma=4.0):
     return synth.f32_to_bf16_bits(s)
 
 
-def _check_p(orc, s_bits, T_kv, p_codes_h, p_sf_h, stats_h, rows, what):
+def _check_p(orc, s_bits, T_kv, p_codes_h, p_sf_h, stats_h, rows, what, fmt=MX):
     """P codes / scales admissible for the fp64 softmax within the library's bound; stats'
     m exact (the fp32 maximum of fl(s c)), l within the bound of the exact sum."""
     from oracle import oracle_np as onp
@@ -132,7 +138,7 @@ def _check_p(orc, s_bits, T_kv, p_codes_h, p_sf_h, stats_h, rows, what):
     hi = p * (1 + eps) + tiny
     lo[:, T_kv:] = 0.0
     hi[:, T_kv:] = 0.0
-    H.check_quant_of_interval(MX, p_codes_h, p_sf_h, lo, hi, None, what, row_ids=rows)
+    H.check_quant_of_interval(fmt, p_codes_h, p_sf_h, lo, hi, np.float32(orc.P_GLOBAL_NVFP4), what, row_ids=rows)
     c = np.float32(orc.softmax_c(SCALE))
     u = (orc.synth_bits_to_f64(s_bits)[:, :T_kv].astype(np.float32) * c).astype(np.float32)
     np.testing.assert_array_equal(stats_h[:, 0], u.max(axis=1))
@@ -140,62 +146,80 @@ def _check_p(orc, s_bits, T_kv, p_codes_h, p_sf_h, stats_h, rows, what):
     assert (np.abs(stats_h[:, 1] - e_exact) <= eps[:, 0] * e_exact).all(), what
 
 
+def _p_global(orc, fmt):
+    return H.dev_f32([orc.P_GLOBAL_NVFP4]) if fmt == NV else None
+
+
+@pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("Tq,T_kv", [(1, 1), (130, 200), (300, 257), (64, 75600), (8, 102500)])
-def test_softmax_quant_admissible(fb, orc, Tq, T_kv):
+def test_softmax_quant_admissible(fb, orc, fmt, Tq, T_kv):
     import torch
 
     from oracle import oracle_np as onp
 
     kpad = (T_kv + 127) // 128 * 128
     s_bits = _scores_bits(3800 + Tq + T_kv, Tq, kpad, T_kv)
-    pc, ps, stats = fb.attn_softmax_quant(H.dev_bf16(s_bits), Tq, T_kv, SCALE)
+    pc, ps, stats = fb.attn_softmax_quant(H.dev_bf16(s_bits), Tq, T_kv, SCALE, _fmt_name(fmt), _p_global(orc, fmt))
     st = fb.fp4_sync_status()
     assert st == 0, fb.fp4_status_string(st)
     torch.cuda.synchronize()
     qpad = (Tq + 127) // 128 * 128
-    sf_all = onp.unswizzle_sf(H.host_u8(ps), qpad, kpad // 32)
+    sf_all = onp.unswizzle_sf(H.host_u8(ps), qpad, kpad // orc.group_size(fmt))
     assert not sf_all[Tq:].any(), "padding query rows hold zero scale bytes"
     _check_p(orc, s_bits, T_kv, H.host_u8(pc), sf_all[:Tq], stats.cpu().numpy(), np.arange(Tq),
-             f"softmax Tq={Tq} T_kv={T_kv}")
+             f"softmax fmt={fmt} Tq={Tq} T_kv={T_kv}", fmt)
 
 
-def _pv_case(fb, orc, Tq, T_kv, Hn, head, seed, rows=None):
+def _resquare(orc, sf_rows, Kg):
+    """Unswizzled scale bytes of R rows -> the atom layout of an [R, Kg * G] operand."""
+    out = np.zeros(orc.sf_bytes(sf_rows.shape[0], Kg), dtype=np.uint8)
+    for i in range(sf_rows.shape[0]):
+        for j in range(Kg):
+            out[orc.sf_offset(i, j, Kg)] = sf_rows[i, j]
+    return out
+
+
+def _pv_case(fb, orc, fmt, Tq, T_kv, Hn, head, seed, rows=None):
     import torch
 
     from oracle import oracle_np as onp
 
     kpad = (T_kv + 127) // 128 * 128
+    G = orc.group_size(fmt)
     s_bits = _scores_bits(seed, Tq, kpad, T_kv, sigma=2.0)
     v = synth.activation(seed + 1, T_kv, Hn * D, "lognormal", gain_seed=seed + 2)
-    pc, ps, _ = fb.attn_softmax_quant(H.dev_bf16(s_bits), Tq, T_kv, SCALE)
-    vt = fb.quantize_heads_vt(H.dev_bf16(v), Hn)
-    o = fb.attn_pv((pc, ps), vt, Tq, T_kv, head)
+    g_v = orc.nv_global(orc.tensor_amax(v)) if fmt == NV else None
+    gvd = H.dev_f32([g_v]) if fmt == NV else None
+    gpd = _p_global(orc, fmt)
+    pc, ps, _ = fb.attn_softmax_quant(H.dev_bf16(s_bits), Tq, T_kv, SCALE, _fmt_name(fmt), gpd)
+    vt = fb.quantize_heads_vt(H.dev_bf16(v), Hn, _fmt_name(fmt), gvd)
+    o = fb.attn_pv((pc, ps), vt, Tq, T_kv, head, _fmt_name(fmt), gpd, gvd)
     st = fb.fp4_sync_status()
     assert st == 0, fb.fp4_status_string(st)
     torch.cuda.synchronize()
     rows = np.arange(Tq) if rows is None else rows
-    vt_ref = orc.quantize_heads_vt(v, Hn)
+    vt_ref = orc.quantize_heads_vt(v, Hn, fmt, g_v)
     np.testing.assert_array_equal(H.host_u8(vt[0][head]), vt_ref[0][head])
+    np.testing.assert_array_equal(H.host_u8(vt[1][head]), vt_ref[1][head])
     pc_h = H.host_u8(pc)[rows]
     qpad = (Tq + 127) // 128 * 128
-    ps_rows = onp.unswizzle_sf(H.host_u8(ps), qpad, kpad // 32)[rows]
-    # re-swizzle the sampled rows as a small [len(rows), kpad] operand for the oracle
-    ps_small = np.zeros(orc.sf_bytes(len(rows), kpad // 32), dtype=np.uint8)
-    for i in range(len(rows)):
-        for j in range(kpad // 32):
-            ps_small[orc.sf_offset(i, j, kpad // 32)] = ps_rows[i, j]
-    Y, S = orc.pv_rows(pc_h, ps_small, vt_ref, head, kpad, np.arange(len(rows)))
+    ps_rows = onp.unswizzle_sf(H.host_u8(ps), qpad, kpad // G)[rows]
+    # the sampled rows' scales as a small [len(rows), kpad] operand for the oracle
+    Y, S = orc.pv_rows(pc_h, _resquare(orc, ps_rows, kpad // G), vt_ref, head, kpad, np.arange(len(rows)), fmt,
+                       float(np.float32(orc.P_GLOBAL_NVFP4)), g_v)
     H.check_linear(o[torch.as_tensor(rows, device="cuda")], Y, S, np.arange(len(rows)),
-                   f"P V Tq={Tq} T_kv={T_kv} H={Hn} head={head}")
+                   f"P V fmt={fmt} Tq={Tq} T_kv={T_kv} H={Hn} head={head}")
     return o
 
 
+@pytest.mark.parametrize("fmt", [MX, NV])
 @pytest.mark.parametrize("Tq,T_kv,Hn,head", [(1, 1, 1, 0), (130, 200, 3, 2), (300, 257, 2, 1), (200, 4096, 40, 39)])
-def test_attn_pv_all_elements(fb, orc, Tq, T_kv, Hn, head):
-    _pv_case(fb, orc, Tq, T_kv, Hn, head, seed=3900 + Tq + T_kv)
+def test_attn_pv_all_elements(fb, orc, fmt, Tq, T_kv, Hn, head):
+    _pv_case(fb, orc, fmt, Tq, T_kv, Hn, head, seed=3900 + Tq + T_kv)
 
 
-def test_attn_chain_full_size_sampled(fb, orc):
+@pytest.mark.parametrize("fmt", [MX, NV])
+def test_attn_chain_full_size_sampled(fb, orc, fmt):
     """The whole head at 75600 tokens, 40 heads, head 17: scores -> softmax + P quantize ->
     P V, each stage checked on sampled query rows against the oracle fed that stage's GPU input."""
     import torch
@@ -204,33 +228,35 @@ def test_attn_chain_full_size_sampled(fb, orc):
 
     T, Hn, head = 75600, 40, 17
     kpad = 75648
+    G = orc.group_size(fmt)
+    name = _fmt_name(fmt)
     rows = H.sample_rows(T, n_random=12, seed=21)
     q = synth.activation(4100, T, Hn * D, "lognormal", gain_seed=4101)
     k = synth.activation(4102, T, Hn * D, "lognormal", gain_seed=4103)
     v = synth.activation(4104, T, Hn * D, "lognormal", gain_seed=4105)
-    qh = fb.quantize_heads(H.dev_bf16(q), Hn)
-    kh = fb.quantize_heads(H.dev_bf16(k), Hn)
-    s = fb.attn_scores(qh, kh, T, T, head)
-    pc, ps, stats = fb.attn_softmax_quant(s, T, T, SCALE)
-    vt = fb.quantize_heads_vt(H.dev_bf16(v), Hn)
-    o = fb.attn_pv((pc, ps), vt, T, T, head)
+    g = {n: (orc.nv_global(orc.tensor_amax(a)) if fmt == NV else None) for n, a in (("q", q), ("k", k), ("v", v))}
+    gd = {n: (H.dev_f32([x]) if x is not None else None) for n, x in g.items()}
+    gpd = _p_global(orc, fmt)
+    qh = fb.quantize_heads(H.dev_bf16(q), Hn, name, gd["q"])
+    kh = fb.quantize_heads(H.dev_bf16(k), Hn, name, gd["k"])
+    s = fb.attn_scores(qh, kh, T, T, head, name, gd["q"], gd["k"])
+    pc, ps, stats = fb.attn_softmax_quant(s, T, T, SCALE, name, gpd)
+    vt = fb.quantize_heads_vt(H.dev_bf16(v), Hn, name, gd["v"])
+    o = fb.attn_pv((pc, ps), vt, T, T, head, name, gpd, gd["v"])
     st = fb.fp4_sync_status()
     assert st == 0, fb.fp4_status_string(st)
     torch.cuda.synchronize()
     idx = torch.as_tensor(rows, device="cuda")
     s_bits = s[idx].contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
-    sf_all = onp.unswizzle_sf(H.host_u8(ps), kpad, kpad // 32)
+    sf_all = onp.unswizzle_sf(H.host_u8(ps), kpad, kpad // G)
     _check_p(orc, s_bits, T, H.host_u8(pc[idx]), sf_all[rows], stats[idx].cpu().numpy(), rows,
-             "softmax full size")
-    vt_ref = orc.quantize_heads_vt(v, Hn)
+             f"softmax full size fmt={fmt}", fmt)
+    vt_ref = orc.quantize_heads_vt(v, Hn, fmt, g["v"])
     np.testing.assert_array_equal(H.host_u8(vt[0][head]), vt_ref[0][head])
     np.testing.assert_array_equal(H.host_u8(vt[1][head]), vt_ref[1][head])
-    ps_small = np.zeros(orc.sf_bytes(len(rows), kpad // 32), dtype=np.uint8)
-    for i in range(len(rows)):
-        for j in range(kpad // 32):
-            ps_small[orc.sf_offset(i, j, kpad // 32)] = sf_all[rows[i], j]
-    Y, S = orc.pv_rows(H.host_u8(pc[idx]), ps_small, vt_ref, head, kpad, np.arange(len(rows)))
-    H.check_linear(o[idx], Y, S, np.arange(len(rows)), "P V full size")
+    Y, S = orc.pv_rows(H.host_u8(pc[idx]), _resquare(orc, sf_all[rows], kpad // G), vt_ref, head, kpad,
+                       np.arange(len(rows)), fmt, float(np.float32(orc.P_GLOBAL_NVFP4)), g["v"])
+    H.check_linear(o[idx], Y, S, np.arange(len(rows)), f"P V full size fmt={fmt}")
 
 
 def test_attn_chain_close_to_unquantized_attention(fb, orc):
