@@ -88,7 +88,7 @@ def lib():
             "fp4_heads_vt_sf_bytes": (SZ, [I, I64, I64, I64]),
             "fp4_quantize_heads_vt": (I, [I, P, I64, I64, I64, P, P, P, P]),
             "fp4_attn_softmax_quant": (I, [I, P, I64, I64, ctypes.c_float, P, P, P, P, P]),
-            "fp4_attn_pv": (I, [I, P, P, P, I64, I64, P, P, P, I64, I64, I64, P, P]),
+            "fp4_attn_pv": (I, [I, P, P, P, I64, I64, P, P, P, I64, I64, I64, P, P, P]),
             "fp4_sync_status": (I, [P]),
             "fp4_status_string": (ctypes.c_char_p, [I]),
             "fp4_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
@@ -292,9 +292,10 @@ def fp4_attn_softmax_quant(fmt, s, T_q: int, T_kv: int, scale: float, p_global, 
 
 
 def fp4_attn_pv(fmt, p_codes, p_sf, p_global, T_q: int, T_kv: int, vt_codes, vt_sf, v_global, H: int, D: int,
-                head: int, o, stream=None):
+                head: int, stats, o, stream=None):
     _check(lib().fp4_attn_pv(_fmt(fmt), _ptr(p_codes), _ptr(p_sf), _ptr(p_global), T_q, T_kv, _ptr(vt_codes),
-                             _ptr(vt_sf), _ptr(v_global), H, D, head, _ptr(o), _stream(stream)), "fp4_attn_pv")
+                             _ptr(vt_sf), _ptr(v_global), H, D, head, _ptr(stats), _ptr(o), _stream(stream)),
+           "fp4_attn_pv")
 
 
 def fp4_sync_status(stream=None) -> int:
@@ -432,17 +433,19 @@ def attn_softmax_quant(s, T_q: int, T_kv: int, scale: float, fmt="mxfp4", p_glob
 
 
 def attn_pv(p, vt_heads, T_q: int, T_kv: int, head: int, fmt="mxfp4", p_global=None, v_global=None, o=None,
-            stream=None):
-    """O = deq(P) deq(V_head) -> bf16 [T_q, 128] from attn_softmax_quant's P and quantize_heads_vt's V^T."""
+            normalize=True, stream=None):
+    """O -> bf16 [T_q, 128] from attn_softmax_quant's (codes, scales, stats) and quantize_heads_vt's V^T:
+    deq(P~) deq(V_head), each row divided by its softmax sum unless normalize is False."""
     import torch
 
     f = _fmt(fmt)
     p_codes, p_sf = p[0], p[1]
+    stats = p[2] if (normalize and len(p) > 2) else None
     vc, vs = vt_heads
     H, D, _ = vc.shape
     if o is None:
         o = torch.empty((T_q, D), dtype=torch.bfloat16, device=p_codes.device)
-    fp4_attn_pv(f, p_codes, p_sf, p_global, T_q, T_kv, vc, vs, v_global, H, D, head, o, stream)
+    fp4_attn_pv(f, p_codes, p_sf, p_global, T_q, T_kv, vc, vs, v_global, H, D, head, stats, o, stream)
     return o
 
 

@@ -2,13 +2,14 @@
 // the row softmax of the scores and its MXFP4 quantization (the P operand), all HBM-bound.
 //
 // Reading followed (the Wan2.2-Animate-14B MXFP4 card, "Results", names SageAttention v3 as
-// Blackwell microscaling FP4 attention without giving its algorithm): P = softmax(S * scale)
-// per query row over the T_kv keys, quantized in blocks of G consecutive keys; V of a head
-// quantized per head-dim channel in blocks of G consecutive tokens; O = deq(P) deq(V) by the
-// block-scaled GEMM (its K is the key axis, so both operands carry their scales along the
-// keys).  MXFP4: G = 32, E8M0 scales.  NVFP4: G = 16, E4M3 scales under one fp32 global per
-// tensor (V's from its amax; P's is a caller's constant, 1 / 2688 for p <= 1), by the same
-// steps as the activation quantizer.
+// Blackwell microscaling FP4 attention without giving its algorithm): per query row, the
+// unnormalized softmax weights P~ = 2^(s c - max) (c = scale log2 e; the largest is exactly
+// 1) over the T_kv keys, quantized in blocks of G consecutive keys, and their fp32 sum l; V of
+// a head quantized per head-dim channel in blocks of G consecutive tokens; O = deq(P~) deq(V)
+// by the block-scaled GEMM (its K is the key axis, so both operands carry their scales along
+// the keys), then each row divided by its l.  MXFP4: G = 32, E8M0 scales.  NVFP4: G = 16,
+// E4M3 scales under one fp32 global per tensor (V's from its amax; P~'s is a caller's
+// constant, 1 / 2688 for p <= 1), by the same steps as the activation quantizer.
 //
 // Layouts (head-major, as the score operands):
 //   V^T  codes [H][128 dims][Tpad/2] bytes (tokens along K; padding tokens hold zero codes),
@@ -119,50 +120,42 @@ FP4_DEV float block_reduce(float v, float* red) {
     return r;
 }
 
-// Row statistics of the softmax: m = max_j fl(s_j c) over the T_kv valid keys and
-// l = sum_j exp2(t_j), each thread summing its columns in order, then the fixed block tree.
-// One block per query row; the row (T_kv_pad bf16) is read twice, the second time from L2.
-__global__ void __launch_bounds__(SOFTMAX_THREADS) softmax_stats_kernel(const __nv_bfloat16* __restrict__ s,
-                                                                       int64_t kpad, int64_t T_kv, float c,
-                                                                       float2* __restrict__ stats) {
+// Row maximum of the softmax argument: m = max_j fl(s_j c) over the T_kv valid keys (one
+// block per query row; a maximum is exact, so the order does not matter).
+__global__ void __launch_bounds__(SOFTMAX_THREADS) softmax_max_kernel(const __nv_bfloat16* __restrict__ s,
+                                                                     int64_t kpad, int64_t T_kv, float c,
+                                                                     float2* __restrict__ stats) {
     __shared__ float red[SOFTMAX_THREADS / 32];
     const __nv_bfloat16* row = s + (int64_t)blockIdx.x * kpad;
     const int64_t nvec = kpad / 8;
     float m = -INFINITY;
     for (int64_t i = threadIdx.x; i < nvec; i += SOFTMAX_THREADS) {
         float v[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + i * 8), v);
+        bf16x8_to_f32(__ldcs(reinterpret_cast<const uint4*>(row + i * 8)), v);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
             if (i * 8 + k < T_kv) m = fmaxf(m, __fmul_rn(v[k], c));
     }
     m = block_reduce<true>(m, red);
-    float l = 0.0f;
-    for (int64_t i = threadIdx.x; i < nvec; i += SOFTMAX_THREADS) {
-        float v[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + i * 8), v);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-            if (i * 8 + k < T_kv) l = __fadd_rn(l, exp2f(softmax_t(v[k], c, m)));
-    }
-    l = block_reduce<false>(l, red);
-    if (threadIdx.x == 0) stats[blockIdx.x] = make_float2(m, l);
+    if (threadIdx.x == 0) stats[blockIdx.x] = make_float2(m, 0.0f);
 }
 
-// P = exp2(t_j) * (1 / l), quantized in groups of G keys (MXFP4 32, NVFP4 16 under the
-// global *g_ptr).  One block per query row of the padded [T_q_pad, T_kv_pad] layout; its 8
-// warps take 256-key chunks in turn, a lane 8 keys (16-byte load, 4-byte code store), G / 8
-// lanes a group.  Keys j >= T_kv give p = 0; rows >= T_q write only zero scale bytes (the
-// layout's padding).
+// P~ = exp2(t_j), quantized in groups of G keys (MXFP4 32, NVFP4 16 under the global
+// *g_ptr), and the row sum l = sum_j P~_j in fp32 (each thread adds its keys in order, then
+// the fixed block tree) into stats[r].y.  One block per query row of the padded
+// [T_q_pad, T_kv_pad] layout; its 8 warps take 256-key chunks in turn, a lane 8 keys
+// (16-byte load, 4-byte code store), G / 8 lanes a group.  Keys j >= T_kv give p = 0; rows
+// >= T_q write only zero scale bytes (the layout's padding).
 template <int KIND>
 __global__ void __launch_bounds__(SOFTMAX_THREADS) softmax_quant_kernel(const __nv_bfloat16* __restrict__ s,
                                                                        int64_t T_q, int64_t kpad, int64_t T_kv,
-                                                                       float c, const float2* __restrict__ stats,
+                                                                       float c, float2* __restrict__ stats,
                                                                        const float* __restrict__ g_ptr,
                                                                        uint8_t* __restrict__ p_codes,
                                                                        uint8_t* __restrict__ p_sf) {
     constexpr int G = (KIND == Q_NVFP4) ? 16 : 32;
     __shared__ float nv_rcp[128];
+    __shared__ float red[SOFTMAX_THREADS / 32];
     const int64_t r = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t apr = kpad / (G * 4);
@@ -177,12 +170,8 @@ __global__ void __launch_bounds__(SOFTMAX_THREADS) softmax_quant_kernel(const __
         }
         __syncthreads();
     }
-    float m = 0.0f, inv_l = 0.0f;
-    if (real) {
-        const float2 st = stats[r];
-        m = st.x;
-        inv_l = __frcp_rn(st.y);
-    }
+    const float m = real ? stats[r].x : 0.0f;
+    float l = 0.0f;
     for (int64_t chunk = warp; chunk * 256 < kpad; chunk += SOFTMAX_THREADS / 32) {
         const int64_t col = chunk * 256 + lane * 8;
         const bool in = col < kpad;  // T_kv_pad = 128 (mod 256): the last chunk's upper half is absent
@@ -193,7 +182,8 @@ __global__ void __launch_bounds__(SOFTMAX_THREADS) softmax_quant_kernel(const __
             bf16x8_to_f32(*reinterpret_cast<const uint4*>(s + r * kpad + col), v);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                p[k] = (col + k < T_kv) ? __fmul_rn(exp2f(softmax_t(v[k], c, m)), inv_l) : 0.0f;
+                p[k] = (col + k < T_kv) ? exp2f(softmax_t(v[k], c, m)) : 0.0f;
+                l = __fadd_rn(l, p[k]);
                 amax = fmaxf(amax, p[k]);
             }
         } else {
@@ -223,6 +213,27 @@ __global__ void __launch_bounds__(SOFTMAX_THREADS) softmax_quant_kernel(const __
         if (lane % LW == 0 && in)
             *reinterpret_cast<uint32_t*>(p_sf + sf_word_offset(r, (chunk * 256 + lane * 8) / (G * 4), apr)) = word;
     }
+    l = block_reduce<false>(l, red);  // uniform per block: real is the same for every thread
+    if (real && threadIdx.x == 0) stats[r].y = l;
+}
+
+// O's rows divided by their softmax sums, in place: o = bf16_rn(o * fl(1 / l)).
+__global__ void __launch_bounds__(256) attn_row_scale_kernel(__nv_bfloat16* __restrict__ o, int64_t rows, int D,
+                                                             const float2* __restrict__ stats) {
+    const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;  // one 8-element vector
+    const int64_t per_row = D / 8;
+    if (i >= rows * per_row) return;
+    const float inv = __frcp_rn(stats[i / per_row].y);
+    uint4 w = *reinterpret_cast<uint4*>(o + i * 8);
+    float v[8];
+    bf16x8_to_f32(w, v);
+    uint32_t out[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(v[2 * k], inv), __fmul_rn(v[2 * k + 1], inv));
+        out[k] = *reinterpret_cast<uint32_t*>(&b);
+    }
+    *reinterpret_cast<uint4*>(o + i * 8) = make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 }  // namespace fp4

@@ -664,11 +664,11 @@ fp4_status_t fp4_attn_softmax_quant(fp4_fmt_t fmt, const void* s_bf16, int64_t T
     // c = scale * log2(e), rounded once to fp32; both kernels take exp2 of fl(fl(s c) - m)
     const float c = (float)((double)scale * 1.4426950408889634);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    softmax_stats_kernel<<<(unsigned)T_q, SOFTMAX_THREADS, 0, cs>>>(static_cast<const __nv_bfloat16*>(s_bf16), kpad,
-                                                                     T_kv, c, static_cast<float2*>(stats));
+    softmax_max_kernel<<<(unsigned)T_q, SOFTMAX_THREADS, 0, cs>>>(static_cast<const __nv_bfloat16*>(s_bf16), kpad,
+                                                                   T_kv, c, static_cast<float2*>(stats));
     if ((st = launched()) != FP4_OK) return st;
     const auto sb = static_cast<const __nv_bfloat16*>(s_bf16);
-    const auto sp = static_cast<const float2*>(stats);
+    const auto sp = static_cast<float2*>(stats);
     if (fmt == FP4_FMT_NVFP4)
         softmax_quant_kernel<Q_NVFP4><<<(unsigned)qpad, SOFTMAX_THREADS, 0, cs>>>(sb, T_q, kpad, T_kv, c, sp, p_global,
                                                                                  p_codes, p_sf);
@@ -680,8 +680,9 @@ fp4_status_t fp4_attn_softmax_quant(fp4_fmt_t fmt, const void* s_bf16, int64_t T
 
 fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p_sf, const float* p_global,
                          int64_t T_q, int64_t T_kv, const uint8_t* vt_codes, const uint8_t* vt_sf, const float* v_global,
-                         int64_t H, int64_t D, int64_t head, void* o_bf16, void* stream) {
+                         int64_t H, int64_t D, int64_t head, const void* stats, void* o_bf16, void* stream) {
     if (!fmt_ok(fmt) || !p_codes || !p_sf || !vt_codes || !vt_sf || !o_bf16) return FP4_ERR_INVALID_ARG;
+    if (!aligned16(stats)) return FP4_ERR_MISALIGNED;
     if (T_q < 1 || T_kv < 1 || H < 1 || head < 0 || head >= H) return FP4_ERR_INVALID_ARG;
     if (D != FP4_HEAD_DIM) return FP4_ERR_UNSUPPORTED_SHAPE;
     const int64_t kpad = (T_kv + 127) / 128 * 128;
@@ -690,7 +691,14 @@ fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p
     const uint8_t* vs = vt_sf + (size_t)head * fp4_sf_bytes(fmt, D, kpad);
     // O = P V_h: P is the activation operand (M = T_q, K = the padded keys), V_h^T the weight
     // (NVFP4: the epilogue applies g_P g_V; gemm_impl checks that both are given)
-    return gemm_impl(fmt, p_codes, p_sf, T_q, kpad, D, vc, vs, v_global, p_global, nullptr, o_bf16, stream, nullptr, 0);
+    fp4_status_t s = gemm_impl(fmt, p_codes, p_sf, T_q, kpad, D, vc, vs, v_global, p_global, nullptr, o_bf16, stream,
+                               nullptr, 0);
+    if (s != FP4_OK || !stats) return s;
+    // then each row of O divided by its softmax sum
+    const int64_t vecs = T_q * (D / 8);
+    attn_row_scale_kernel<<<(unsigned)((vecs + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<__nv_bfloat16*>(o_bf16), T_q, (int)D, static_cast<const float2*>(stats));
+    return launched();
 }
 
 fp4_status_t fp4_attn_scores(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,

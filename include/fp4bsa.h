@@ -360,12 +360,14 @@ fp4_status_t fp4_attn_scores(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_
                              int64_t D, int64_t head, const float* g_q, const float* g_k, void* s_bf16,
                              void* stream);
 
-/* The rest of one head's attention, read the same way: P = softmax(S * scale) per query row
- * over the T_kv keys, quantized in blocks of G consecutive keys; V of the head quantized per
- * head-dim channel in blocks of G consecutive tokens; and O = deq(P) deq(V) by the
- * block-scaled GEMM, whose K is then the key axis.  MXFP4: G = 32; NVFP4: G = 16 with E4M3
- * scales under one fp32 global per tensor (V: from its amax, e.g. fp4_calibrate_act_global
- * over v; P: a constant the caller provides, 1/2688 = 1/(6*448) since p <= 1).
+/* The rest of one head's attention, read the same way: per query row the unnormalized
+ * softmax weights P~_j = 2^(s_j c - max) over the T_kv keys (c = scale * log2 e; the largest
+ * is exactly 1), quantized in blocks of G consecutive keys, and their sum l; V of the head
+ * quantized per head-dim channel in blocks of G consecutive tokens; O = deq(P~) deq(V) by
+ * the block-scaled GEMM, whose K is then the key axis, each row then divided by its l.
+ * MXFP4: G = 32; NVFP4: G = 16 with E4M3 scales under one fp32 global per tensor (V: from its
+ * amax, e.g. fp4_calibrate_act_global over v; P~: a constant the caller provides, 1/2688 =
+ * 1/(6*448) since p <= 1).
  * fp4_attn_scores, fp4_attn_softmax_quant and fp4_attn_pv in sequence give one head's
  * attention output.
  *
@@ -383,33 +385,36 @@ size_t fp4_heads_vt_sf_bytes(fp4_fmt_t fmt, int64_t T, int64_t H, int64_t D);
 fp4_status_t fp4_quantize_heads_vt(fp4_fmt_t fmt, const void* v_bf16, int64_t T, int64_t H, int64_t D,
                                    const float* g, uint8_t* codes, uint8_t* sf, void* stream);
 
-/* Softmax of scores and its MXFP4 quantization.
+/* Softmax weights of scores and their quantization.
  *   s_bf16  (device) [T_q][T_kv_pad] bf16 scores (fp4_attn_scores' output; columns >= T_kv
  *           are ignored)
  *   scale   the softmax scale (e.g. 1/sqrt(D)), > 0 and finite; the kernels use
- *           c = fp32(scale * log2 e), t_j = fl(fl(s_j c) - m), m = max_j fl(s_j c) over
- *           j < T_kv, l = sum_j exp2(t_j) (fp32; each of a row's 256 threads adds its keys in
- *           order, then a fixed tree), p_j = fl(exp2(t_j) * fl(1/l)); exp2 is CUDA's exp2f
- *           (within 2 ulp).  p is then the exact softmax of s * scale within a relative
- *           2 (2 (ln2 * 4 max|s c| + 4) + 8 ceil(T_kv_pad / 2048) + 14) 2^-24 (about 7e-5
- *           at 75648 keys and max|s c| = 50), the bound the tests hold it to
+ *           c = fp32(scale * log2 e), m = max_j fl(s_j c) over j < T_kv, t_j = fl(fl(s_j c)
+ *           - m), p~_j = exp2(t_j) with CUDA's exp2f (within 2 ulp), so p~ is 2^(s_j c - max)
+ *           within a relative 2 (ln2 * 4 max|s c| + 4) 2^-24; and l = sum_j p~_j in fp32 (each
+ *           of a row's 256 threads adds its keys in order, then a fixed tree), within a
+ *           relative (8 ceil(T_kv_pad / 2048) + 12) 2^-24 more of the sum of the p~ it adds
  *   p_global (device) NVFP4: P's fp32 global (1/2688 for p <= 1); MXFP4: must be NULL
  *   stats   (device, out) [T_q] pairs of fp32 (m, l)
  *   p_codes (device, out) [T_q][T_kv_pad/2]; p_sf (device, out) fp4_sf_bytes(fmt, T_q,
- *           T_kv_pad): p quantized by the format's rules above; keys >= T_kv hold p = 0 and
+ *           T_kv_pad): p~ quantized by the format's rules above; keys >= T_kv hold 0 and
  *           padding rows zero scale bytes. */
 fp4_status_t fp4_attn_softmax_quant(fp4_fmt_t fmt, const void* s_bf16, int64_t T_q, int64_t T_kv, float scale,
                                     const float* p_global, void* stats, uint8_t* p_codes, uint8_t* p_sf,
                                     void* stream);
 
-/* O = deq(P) deq(V_head) for head `head`: the block-scaled GEMM with K = T_kv_pad.
+/* O for head `head`: bf16 [T_q][D] = deq(P~) deq(V_head) by the block-scaled GEMM with
+ * K = T_kv_pad, then, when stats is given, each row o = bf16_rn(o * fl(1 / l)).
  *   p_codes, p_sf      fp4_attn_softmax_quant's output (T_q rows); p_global its NVFP4 global
  *   vt_codes, vt_sf    fp4_quantize_heads_vt's output (T_kv tokens, H heads); v_global its
  *                      NVFP4 global (both globals device pointers, NULL for MXFP4)
+ *   stats   (device) fp4_attn_softmax_quant's (m, l) pairs, or NULL for the unnormalized
+ *           product
  *   o_bf16  (device, out) [T_q][D] bf16 */
 fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p_sf, const float* p_global,
                          int64_t T_q, int64_t T_kv, const uint8_t* vt_codes, const uint8_t* vt_sf,
-                         const float* v_global, int64_t H, int64_t D, int64_t head, void* o_bf16, void* stream);
+                         const float* v_global, int64_t H, int64_t D, int64_t head, const void* stats,
+                         void* o_bf16, void* stream);
 
 /* ----------------------------------------------------------------- status */
 

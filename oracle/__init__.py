@@ -320,31 +320,34 @@ def softmax_c(scale: float) -> float:
     return float(np.float32(scale * LOG2E))
 
 
-def softmax_rows(s_bf16, T_kv: int, scale: float):
-    """Row softmax of bf16 scores [R, T_kv_pad] over the first T_kv keys, in fp64:
-    p_j = 2^(s_j c - max) / sum_k 2^(s_k c - max) with c = softmax_c(scale); keys >= T_kv get 0.
-    Returns (p, t_max_abs) where t_max_abs[r] = max_j |s_j c| (for the error bound)."""
+def softmax_weights(s_bf16, T_kv: int, scale: float):
+    """Unnormalized softmax weights of bf16 scores [R, T_kv_pad] over the first T_kv keys, in
+    fp64: p~_j = 2^(s_j c - max_k s_k c) with c = softmax_c(scale) (the largest is 1), keys >=
+    T_kv 0.  Returns (p~, l, t_max_abs): l[r] = sum_j p~_j, t_max_abs[r] = max_j |s_j c| (for
+    the error bounds)."""
     s = synth_bits_to_f64(s_bf16)
     c = softmax_c(scale)
     u = s[:, :T_kv] * c
     m = u.max(axis=1, keepdims=True)
-    e = np.exp2(u - m)
     p = np.zeros_like(s)
-    p[:, :T_kv] = e / e.sum(axis=1, keepdims=True)
-    return p, np.abs(u).max(axis=1)
+    p[:, :T_kv] = np.exp2(u - m)
+    return p, p.sum(axis=1), np.abs(u).max(axis=1)
 
 
-def softmax_bound(T_kv_pad: int, t_max_abs):
-    """Relative bound on the library's fp32 p (per row): argument rounding of fl(fl(s c) - m)
-    (two roundings of terms up to 2 max|s c|, through 2^t: ln2 * 4 max|s c| 2^-24), exp2f
-    within 2 ulp (2^-22), the sum l of positive terms in fp32 (each of a row's 256 threads adds
-    at most 8 ceil(T_kv_pad / 2048) terms in order, then a 5-step warp tree and 7 more
-    additions, plus the terms' own errors), and fl(1/l) and the product (2^-23); doubled for
-    margin."""
-    u = 2.0 ** -24
-    term = np.log(2.0) * 4.0 * np.asarray(t_max_abs) * u + 2.0 ** -22
+def softmax_weight_bound(t_max_abs):
+    """Relative bound on the library's fp32 p~ (per row): the two roundings of fl(fl(s c) - m)
+    (terms up to 2 max|s c|, through 2^t: ln2 * 4 max|s c| 2^-24) and exp2f within 2 ulp
+    (2^-22); doubled for margin."""
+    return 2.0 * (np.log(2.0) * 4.0 * np.asarray(t_max_abs) * 2.0 ** -24 + 2.0 ** -22)
+
+
+def softmax_sum_bound(T_kv_pad: int, t_max_abs):
+    """Relative bound on the library's fp32 l against the exact sum of the exact p~: the
+    terms' own error (softmax_weight_bound) plus the fp32 sum of positive terms (each of a
+    row's 256 threads adds at most 8 ceil(T_kv_pad / 2048) terms in order, then a 5-step warp
+    tree and 7 more additions); doubled for margin."""
     n = 8 * -(-T_kv_pad // 2048) + 12
-    return 2.0 * (2.0 * term + n * u + 2.0 * u)
+    return softmax_weight_bound(t_max_abs) + 2.0 * n * 2.0 ** -24
 
 
 P_GLOBAL_NVFP4 = 1.0 / 2688.0  # the NVFP4 global of P (p <= 1): T / (6 * 448) with T = 1

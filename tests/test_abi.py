@@ -146,9 +146,10 @@ def test_invalid_calls_rejected_before_launch(fb):
     assert L.fp4_attn_softmax_quant(0, A, 16, 16, 0.0, None, A, A, A, st) == 1
     assert L.fp4_attn_softmax_quant(0, A, 0, 16, 0.1, None, A, A, A, st) == 1
     assert L.fp4_attn_softmax_quant(0, A, 16, 16, 0.1, None, A, bad, A, st) == 3
-    assert L.fp4_attn_pv(0, A, A, None, 16, 16, A, A, None, 2, 128, 2, A, st) == 1
-    assert L.fp4_attn_pv(1, A, A, None, 16, 16, A, A, A, 2, 128, 0, A, st) == 1
-    assert L.fp4_attn_pv(0, A, A, None, 16, 16, A, A, None, 2, 64, 0, A, st) == 2
+    assert L.fp4_attn_pv(0, A, A, None, 16, 16, A, A, None, 2, 128, 2, None, A, st) == 1
+    assert L.fp4_attn_pv(1, A, A, None, 16, 16, A, A, A, 2, 128, 0, None, A, st) == 1
+    assert L.fp4_attn_pv(0, A, A, None, 16, 16, A, A, None, 2, 64, 0, None, A, st) == 2
+    assert L.fp4_attn_pv(0, A, A, None, 16, 16, A, A, None, 2, 128, 0, bad, A, st) == 3
 
 
 def test_product_path_has_no_oracle_import():

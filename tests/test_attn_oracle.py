@@ -130,51 +130,54 @@ def test_softmax_oracle_against_closed_forms_and_scipy():
 
     rng = np.random.default_rng(3)
     s = synth.f32_to_bf16_bits(rng.normal(0, 4, size=(5, 384)).astype(np.float32))
-    p, tmax = oracle.softmax_rows(s, 300, 0.125)
+    p, l, tmax = oracle.softmax_weights(s, 300, 0.125)
     sf = oracle.synth_bits_to_f64(s)
     c = oracle.softmax_c(0.125)
     ref = softmax(sf[:, :300] * c * np.log(2.0), axis=1)    # 2^(s c) = e^(s c ln 2)
-    np.testing.assert_allclose(p[:, :300], ref, rtol=1e-12, atol=0)
+    np.testing.assert_allclose(p[:, :300] / l[:, None], ref, rtol=1e-12, atol=0)
     assert not p[:, 300:].any()
-    np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=1e-14)
-    # a constant row is uniform; a row with one score far above the rest is one-hot
+    np.testing.assert_array_equal(p.max(axis=1), 1.0)      # the largest weight is exactly 1
+    np.testing.assert_allclose(tmax, np.abs(sf[:, :300] * c).max(axis=1), rtol=0)
+    # a constant row: every weight 1, l = T_kv; a row with one score far above the rest: l = 1
     const = np.full((1, 128), synth.f32_to_bf16_bits(np.float32([2.5]))[0], dtype=np.uint16)
-    pc, _ = oracle.softmax_rows(const, 100, 1.0)
-    np.testing.assert_allclose(pc[0, :100], 1.0 / 100, rtol=1e-15)
+    pc, lc, _ = oracle.softmax_weights(const, 100, 1.0)
+    assert (pc[0, :100] == 1.0).all() and lc[0] == 100.0
     hot = np.zeros((1, 128), dtype=np.uint16)
     hot[0, 7] = synth.f32_to_bf16_bits(np.float32([1000.0]))[0]
-    ph, _ = oracle.softmax_rows(hot, 128, 1.0)
-    assert ph[0, 7] == 1.0 and ph[0, :7].max() < 1e-290
+    ph, lh, _ = oracle.softmax_weights(hot, 128, 1.0)
+    assert ph[0, 7] == 1.0 and lh[0] == 1.0
 
 
-def test_softmax_bound_covers_an_fp32_evaluation():
-    """numpy float32 steps as the library states them (fl(fl(s c) - m), exp2, sequential sums
-    per thread stride, 1/l, product) stay inside softmax_bound of the fp64 softmax."""
+def test_softmax_bounds_cover_an_fp32_evaluation():
+    """numpy float32 steps as the library states them (fl(fl(s c) - m), exp2, sums per thread
+    in the library's key order, then the block tree) stay inside the stated bounds of the
+    fp64 weights and sum."""
     rng = np.random.default_rng(4)
     kpad, T_kv = 2048, 1990
     s = synth.f32_to_bf16_bits(rng.normal(0, 6, size=(3, kpad)).astype(np.float32))
-    p, tmax = oracle.softmax_rows(s, T_kv, 0.088388)
-    eps = oracle.softmax_bound(kpad, tmax)
+    p, l, tmax = oracle.softmax_weights(s, T_kv, 0.088388)
+    ew = oracle.softmax_weight_bound(tmax)
+    el = oracle.softmax_sum_bound(kpad, tmax)
     c = np.float32(oracle.softmax_c(0.088388))
     sf = oracle.synth_bits_to_f64(s).astype(np.float32)
     for r in range(3):
-        u = (sf[r, :T_kv] * c).astype(np.float32)
-        m = u.max()
-        e = np.exp2((u - m).astype(np.float32)).astype(np.float32)
-        lanes = np.zeros(256 * 8, dtype=np.float32)
-        ee = np.zeros(kpad, dtype=np.float32)
-        ee[:T_kv] = e
+        u = (sf[r] * c).astype(np.float32)
+        m = u[:T_kv].max()
+        e = np.zeros(kpad, dtype=np.float32)
+        e[:T_kv] = np.exp2((u[:T_kv] - m).astype(np.float32)).astype(np.float32)
+        rel = np.abs(e[:T_kv].astype(np.float64) - p[r, :T_kv]) / p[r, :T_kv]
+        assert rel.max() <= ew[r], (rel.max(), ew[r])
+        # thread t = 32 w + lane takes keys 256 (w + 8 k) + 8 lane .. + 7 in order
         part = np.zeros(256, dtype=np.float32)
-        for i in range(kpad // 8):                 # thread i % 256 takes 8-element vector i
-            for k in range(8):
-                part[i % 256] = np.float32(part[i % 256] + ee[i * 8 + k])
-        l = np.float32(0.0)
+        for chunk in range(kpad // 256):
+            for lane in range(32):
+                t = 32 * (chunk % 8) + lane
+                for k in range(8):
+                    part[t] = np.float32(part[t] + e[chunk * 256 + lane * 8 + k])
+        tot = np.float32(0.0)
         for v in part:
-            l = np.float32(l + v)
-        p32 = (e * np.float32(np.float32(1.0) / l)).astype(np.float32)
-        rel = np.abs(p32.astype(np.float64) - p[r, :T_kv]) / p[r, :T_kv]
-        assert rel.max() <= eps[r], (rel.max(), eps[r])
-        del lanes
+            tot = np.float32(tot + v)
+        assert abs(float(tot) - l[r]) <= el[r] * l[r], (abs(float(tot) - l[r]) / l[r], el[r])
 
 
 def test_pv_oracle_nvfp4_exact_on_representable_blocks():
