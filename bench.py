@@ -59,14 +59,15 @@ def parse():
     ap.add_argument("--m", type=int, default=75600,
                     help="tokens; smaller values run a reduced case of the same kernels (profiling only)")
     ap.add_argument("--attn-tokens", type=int, default=0,
-                    help="profiling only: run the FP4 attention operands (K quantizer over 40 heads of 128 and "
-                         "head 17's score GEMM) at this many tokens for --steps iterations, print timings, exit")
+                    help="profiling only: run one head of FP4 attention (K quantizer over 40 heads of 128, head 17's "
+                         "scores, softmax weights + quantize, P V) at this many tokens for --steps iterations, print "
+                         "timings, exit")
     return ap.parse_args()
 
 
 def attn_profile(args):
-    """The FP4 attention-operand kernels alone (a case for ncu): quantize_heads of Q and K
-    ([T, 40 x 128] bf16), then per step the K quantizer and head 17's score GEMM."""
+    """One head of FP4 attention alone (a case for ncu): Q, K, V quantized ([T, 40 x 128] bf16),
+    then per step the K quantizer, head 17's scores, the softmax weights + quantize and P V."""
     import torch
 
     import fp4_block_scaled_act_b200 as fb
@@ -81,26 +82,37 @@ def attn_profile(args):
     if fmt == "nvfp4":
         gq, _ = fb.calibrate_act_global(q)
         gk, _ = fb.calibrate_act_global(k)
+    v = torch.randn(T, Hn * 128, generator=gen, device="cuda").to(torch.bfloat16)
+    gv = fb.calibrate_act_global(v)[0] if fmt == "nvfp4" else None
+    gp = torch.tensor([fb.P_GLOBAL_NVFP4], dtype=torch.float32, device="cuda") if fmt == "nvfp4" else None
     qh = fb.quantize_heads(q, Hn, fmt, gq)
     kh = fb.quantize_heads(k, Hn, fmt, gk)
+    vt = fb.quantize_heads_vt(v, Hn, fmt, gv)
     s_buf = torch.empty((T, (T + 127) // 128 * 128), dtype=torch.bfloat16, device="cuda")
+    p = fb.attn_softmax_quant(s_buf.zero_(), T, T, 128 ** -0.5, fmt, gp)
+    o = torch.empty((T, 128), dtype=torch.bfloat16, device="cuda")
     f = fb.MXFP4 if fmt == "mxfp4" else fb.NVFP4
-    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    tq = ts = 0.0
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    t = [0.0] * 4
     for _ in range(args.steps):
         e[0].record()
         fb.fp4_quantize_heads(f, k, T, Hn, 128, gk, kh[0], kh[1])
         e[1].record()
         fb.attn_scores(qh, kh, T, T, 17, fmt, gq, gk, s_buf)
         e[2].record()
+        fb.fp4_attn_softmax_quant(f, s_buf, T, T, 128 ** -0.5, gp, p[2], p[0], p[1])
+        e[3].record()
+        fb.attn_pv(p, vt, T, T, 17, fmt, gp, gv, o=o)
+        e[4].record()
         torch.cuda.synchronize()
-        tq += e[0].elapsed_time(e[1])
-        ts += e[1].elapsed_time(e[2])
+        for i in range(4):
+            t[i] += e[i].elapsed_time(e[i + 1])
     st = fb.fp4_sync_status()
     if st != 0:
         raise RuntimeError(f"device status: {fb.fp4_status_string(st)}")
-    print(json.dumps({"attn_tokens": T, "heads": Hn, "fmt": fmt, "quantize_heads_ms": tq / args.steps,
-                      "scores_ms": ts / args.steps, "s_bytes": s_buf.numel() * 2}), flush=True)
+    print(json.dumps({"attn_tokens": T, "heads": Hn, "fmt": fmt, "quantize_heads_ms": t[0] / args.steps,
+                      "scores_ms": t[1] / args.steps, "softmax_quant_ms": t[2] / args.steps,
+                      "pv_ms": t[3] / args.steps, "s_bytes": s_buf.numel() * 2}), flush=True)
     return 0
 
 
