@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(128) quant_vt_kernel(const __nv_bfloat16* __re
             words[a];
 }
 
-// The softmax argument of a score in fp32, the same two roundings in both softmax kernels:
-// t = fl(fl(s * c) - m), c = scale * log2(e), m = the row maximum of fl(s * c).
+// The softmax argument of a score in fp32: t = fl(fl(s * c) - m), c = scale * log2(e), m =
+// the row maximum of fl(s * c) (softmax_max_kernel), so the largest score gives t = 0.
 FP4_DEV float softmax_t(float s, float c, float m) { return __fsub_rn(__fmul_rn(s, c), m); }
 
 // Block reduction in a fixed order (warp shuffles, then the warp results in index order).
