@@ -299,3 +299,59 @@ def test_attn_chain_close_to_unquantized_attention(fb, orc):
     ref = pr @ vf
     cos = (of * ref).sum(1) / np.linalg.norm(of, axis=1) / np.linalg.norm(ref, axis=1)
     assert np.median(cos) > 0.95 and cos.min() > 0.7, (np.median(cos), cos.min())
+
+
+def test_attn_chain_is_deterministic_and_replays_in_a_cuda_graph(fb, orc):
+    """The head's kernels (quantizers, scores, softmax, P V, row scaling) allocate nothing
+    and never synchronize: captured once in a CUDA graph and replayed on new inputs copied
+    into the same buffers, they give bit for bit the eager results, which are themselves
+    identical from run to run (every sum in a fixed order)."""
+    import torch
+
+    T, Hn, head = 700, 2, 1
+    bufs = {n: torch.empty((T, Hn * D), dtype=torch.bfloat16, device="cuda") for n in "qkv"}
+    qh = fb.quantize_heads(bufs["q"], Hn)
+    kh = fb.quantize_heads(bufs["k"], Hn)
+    vt = fb.quantize_heads_vt(bufs["v"], Hn)
+    s = fb.attn_scores(qh, kh, T, T, head)
+    p = fb.attn_softmax_quant(s, T, T, SCALE)
+    o = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
+
+    def chain():
+        fb.fp4_quantize_heads(MX, bufs["q"], T, Hn, D, None, qh[0], qh[1])
+        fb.fp4_quantize_heads(MX, bufs["k"], T, Hn, D, None, kh[0], kh[1])
+        fb.fp4_quantize_heads_vt(MX, bufs["v"], T, Hn, D, None, vt[0], vt[1])
+        fb.attn_scores(qh, kh, T, T, head, s=s)
+        fb.fp4_attn_softmax_quant(MX, s, T, T, SCALE, None, p[2], p[0], p[1])
+        fb.attn_pv(p, vt, T, T, head, o=o)
+
+    def load(seed):
+        for i, n in enumerate("qkv"):
+            bufs[n].copy_(H.dev_bf16(synth.activation(seed + i, T, Hn * D, "lognormal")))
+
+    load(4300)
+    chain()
+    torch.cuda.synchronize()
+    first = o.clone()
+    chain()
+    torch.cuda.synchronize()
+    assert torch.equal(first.view(torch.int16), o.view(torch.int16)), "two eager runs differ"
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        chain()
+        side.synchronize()
+        with torch.cuda.graph(graph, stream=side):
+            chain()
+    for seed in (4400, 4500):
+        load(seed)
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        replay = o.clone()
+        chain()
+        torch.cuda.synchronize()
+        assert torch.equal(replay.view(torch.int16), o.view(torch.int16)), f"graph replay differs (seed {seed})"
+    assert fb.fp4_sync_status() == 0
+    del graph
