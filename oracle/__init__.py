@@ -379,3 +379,91 @@ def tolerance(Y_ref: np.ndarray, S: np.ndarray) -> np.ndarray:
     _, ex = np.frexp(np.where(a > 0, a, 1.0))
     ulp = np.where(a > 0, np.ldexp(1.0, np.maximum(ex - 1 - 7, -133)), 2.0 ** -133)
     return ulp + 1e-5 * S
+
+
+# ----------------------------------------------------------------------------- streaming attention
+# The streaming (flash) form of one head's attention (the Wan2.2-Animate-14B MXFP4 card,
+# "Results", names FP4 attention with microscaling on Blackwell; no page gives its
+# algorithm): keys in blocks of FLASH_BLOCK; block j's weights are taken against the running
+# maximum m_j of the blocks seen so far, and the partial outputs are brought to the final
+# maximum by the factors 2^(m_j - m_last).
+
+FLASH_BLOCK = 256
+_E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0])
+
+
+def dequant_mx_rows(codes, sf_rows) -> np.ndarray:
+    """MXFP4 rows in fp64 from codes [R, K/2] (two E2M1 codes per byte, low nibble first) and
+    their E8M0 scale bytes [R, K/32] in row order: value = e2m1(code) 2^(byte - 127)."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    sf_rows = np.asarray(sf_rows, dtype=np.int64)
+    nib = np.stack([codes & 15, codes >> 4], axis=-1).reshape(codes.shape[0], -1)
+    vals = _E2M1[nib]
+    R, K = vals.shape
+    return (vals.reshape(R, K // 32, 32) * np.ldexp(1.0, sf_rows - 127)[..., None]).reshape(R, K)
+
+
+def flash_maxima(s: np.ndarray, T_kv: int, scale: float, block: int = FLASH_BLOCK) -> np.ndarray:
+    """Running maxima [R, nblk] (nblk = ceil(T_kv / block)) of exact scores s [R, >= T_kv]:
+    m[r, j] = max of s[r, k] c over the keys k < min(T_kv, (j + 1) block), c = softmax_c(scale)."""
+    u = np.asarray(s, dtype=np.float64)[:, :T_kv] * softmax_c(scale)
+    nb = -(-T_kv // block)
+    full = np.full((u.shape[0], nb * block), -np.inf)
+    full[:, :T_kv] = u
+    return np.maximum.accumulate(full.reshape(u.shape[0], nb, block).max(axis=2), axis=1)
+
+
+def flash_weights(s: np.ndarray, T_kv: int, scale: float, m: np.ndarray, block: int = FLASH_BLOCK) -> np.ndarray:
+    """Block j's weights against its own maximum, fp64 [R, nblk * block]: p[r, k] = 2^(s c - m[r, j])
+    for the keys k < T_kv of block j = k // block, 0 for the rest."""
+    nb = m.shape[1]
+    u = np.asarray(s, dtype=np.float64)[:, :T_kv] * softmax_c(scale)
+    p = np.zeros((u.shape[0], nb * block))
+    p[:, :T_kv] = np.exp2(u - np.repeat(m, block, axis=1)[:, :T_kv])
+    return p
+
+
+def flash_combine(p_vals: np.ndarray, m: np.ndarray, w: np.ndarray, block: int = FLASH_BLOCK):
+    """(Y, S) of the unnormalized streaming output: Y = sum_j 2^(m_j - m_last) P_j W_j^T in fp64,
+    P_j block j's columns of p_vals [R, nblk * block], W [N, nblk * block] (columns beyond W's
+    width are zero); S the same sum of absolute terms (for the tolerance)."""
+    nb = m.shape[1]
+    f = np.exp2(m - m[:, -1:])
+    a = p_vals[:, :nb * block] * np.repeat(f, block, axis=1)
+    wf = np.zeros((w.shape[0], nb * block))
+    wf[:, :min(w.shape[1], nb * block)] = w[:, :nb * block]
+    return linear_fp64(a, wf, None)
+
+
+def flash_pv_rows(p_codes, p_sf_rows, m: np.ndarray, vt_heads, head: int, T_kv_pad: int,
+                  block: int = FLASH_BLOCK):
+    """flash_combine of the MXFP4 weights (codes [R, nblk * block / 2], scale bytes
+    [R, nblk * block / 32] in row order) with V_head^T dequantized from quantize_heads_vt."""
+    vc, vs = vt_heads
+    w = dequant_fp4(MX, vc[head], vs[head], T_kv_pad, 1.0)
+    return flash_combine(dequant_mx_rows(p_codes, p_sf_rows), m, w, block)
+
+
+def flash_sum(s: np.ndarray, T_kv: int, scale: float, m_last: np.ndarray) -> np.ndarray:
+    """l[r] = sum over keys k < T_kv of 2^(s[r, k] c - m_last[r]), fp64: the streaming sum
+    sum_j 2^(m_j - m_last) sum_{k in j} 2^(s c - m_j), whose factors telescope."""
+    u = np.asarray(s, dtype=np.float64)[:, :T_kv] * softmax_c(scale)
+    return np.exp2(u - np.asarray(m_last, dtype=np.float64)[:, None]).sum(axis=1)
+
+
+def flash_weight_interval(s: np.ndarray, es: np.ndarray, T_kv: int, scale: float, m: np.ndarray,
+                          block: int = FLASH_BLOCK):
+    """(lo, hi) [R, nblk * block] holding the fp32 weight exp2(fl(fl(s' c) - m_j)) for any fp32
+    score s' with |s' - s| <= es (the exponent off by at most c es + 2^-23 (|s c| + |m_j|): the
+    score's error and the two roundings) and exp2f within 2 ulp (relative 2^-22, taken as
+    2^-21); keys >= T_kv give [0, 0]."""
+    nb = m.shape[1]
+    c = softmax_c(scale)
+    u = np.asarray(s, dtype=np.float64)[:, :T_kv] * c
+    mj = np.repeat(m, block, axis=1)[:, :T_kv]
+    d = c * np.asarray(es, dtype=np.float64)[:, :T_kv] + 2.0 ** -23 * (np.abs(u) + np.abs(mj))
+    lo = np.zeros((u.shape[0], nb * block))
+    hi = np.zeros((u.shape[0], nb * block))
+    lo[:, :T_kv] = np.exp2(u - mj - d) * (1.0 - 2.0 ** -21)
+    hi[:, :T_kv] = np.exp2(u - mj + d) * (1.0 + 2.0 ** -21)
+    return lo, hi

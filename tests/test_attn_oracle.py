@@ -217,3 +217,102 @@ def test_pv_oracle_exact_on_representable_blocks():
     for head in range(H):
         Y, _ = oracle.pv_rows(pc, ps, vt, head, kpad, np.arange(Tq))
         np.testing.assert_array_equal(Y, pvals[:, :Tk] @ v[:, head * D:(head + 1) * D])
+
+
+# ------------------------------------------------------------------ streaming (flash) form
+
+
+def test_dequant_mx_rows_matches_the_atom_layout_dequantizer():
+    """Row-order MXFP4 dequantization equals the pinned dequantizer fed the same bytes in the
+    128x4 atom layout."""
+    rng = np.random.default_rng(11)
+    R, K = 130, 512
+    codes = rng.integers(0, 256, size=(R, K // 2), dtype=np.uint8)
+    sf = rng.integers(100, 150, size=(R, K // 32), dtype=np.uint8)
+    atoms = np.zeros(oracle.sf_bytes(R, K // 32), dtype=np.uint8)
+    for i in range(R):
+        for j in range(K // 32):
+            atoms[oracle.sf_offset(i, j, K // 32)] = sf[i, j]
+    np.testing.assert_array_equal(oracle.dequant_mx_rows(codes, sf), oracle.dequant_fp4(MX, codes, atoms, K))
+
+
+def test_flash_maxima_and_sum_reduce_to_the_plain_softmax():
+    """The last running maximum is the row maximum of s c, the maxima never fall, a block's
+    maximum is reached inside it or before; with m_last the flash sum is the plain softmax
+    oracle's l (which scipy pins)."""
+    rng = np.random.default_rng(12)
+    T_kv, scale = 1000, 0.0883883
+    s = rng.normal(0.0, 4.0, size=(5, 1024)).astype(np.float32).astype(np.float64)
+    m = oracle.flash_maxima(s, T_kv, scale)
+    c = oracle.softmax_c(scale)
+    assert m.shape == (5, 4)
+    np.testing.assert_array_equal(m[:, -1], (s[:, :T_kv] * c).max(axis=1))
+    assert (np.diff(m, axis=1) >= 0).all()
+    np.testing.assert_array_equal(m[:, 0], (s[:, :256] * c).max(axis=1))
+    bits = synth.f32_to_bf16_bits(s.astype(np.float32))
+    sb = oracle.synth_bits_to_f64(bits)
+    _, l_plain, _ = oracle.softmax_weights(bits, T_kv, scale)
+    l_flash = oracle.flash_sum(sb, T_kv, scale, oracle.flash_maxima(sb, T_kv, scale)[:, -1])
+    np.testing.assert_allclose(l_flash, l_plain, rtol=1e-13)
+
+
+def test_flash_combine_is_softmax_attention_without_quantization():
+    """Unquantized streaming weights combined by flash_combine and divided by flash_sum equal
+    softmax(s scale) V computed by scipy, for a key count with a ragged last block."""
+    from scipy.special import softmax
+
+    rng = np.random.default_rng(13)
+    T_kv, scale, R = 700, 0.125, 6
+    s = rng.normal(0.0, 6.0, size=(R, T_kv))
+    # a late key with a much larger score forces the maxima to grow block by block
+    s[:, 650] += 30.0
+    v = rng.normal(size=(T_kv, 128))
+    m = oracle.flash_maxima(s, T_kv, scale)
+    p = oracle.flash_weights(s, T_kv, scale, m)
+    Y, _ = oracle.flash_combine(p, m, v.T)
+    l = oracle.flash_sum(s, T_kv, scale, m[:, -1])
+    c = oracle.softmax_c(scale)
+    ref = softmax(s * c * np.log(2.0), axis=1) @ v
+    np.testing.assert_allclose(Y / l[:, None], ref, rtol=1e-10, atol=1e-12)
+
+
+def test_flash_combine_worked_two_blocks():
+    """Block 0 of ones against m_0 = m_1 - 1, block 1 of halves, V of ones: each output is
+    2^-1 * 256 + 0.5 * 256 = 256 (a reversed factor 2^(m_last - m_j) would give 640)."""
+    p = np.concatenate([np.ones((2, 256)), np.full((2, 256), 0.5)], axis=1)
+    m = np.array([[3.0, 4.0], [-7.5, -6.5]])
+    Y, S = oracle.flash_combine(p, m, np.ones((128, 512)))
+    np.testing.assert_array_equal(Y, np.full((2, 128), 256.0))
+    np.testing.assert_array_equal(S, Y)
+
+
+def test_flash_weight_interval_holds_an_fp32_evaluation():
+    """For fp32 scores s' within es of s and m_j the fp32 running maxima of fl(s' c) (what a
+    kernel computes), the fp32 weights exp2(fl(fl(s' c) - m_j)) lie in the interval built on
+    the exact s (numpy's exp2 in fp64 rounded to fp32 stands in for a 2-ulp exp2f)."""
+    rng = np.random.default_rng(14)
+    T_kv, scale, R = 600, 0.0883883, 4
+    s = rng.normal(0.0, 8.0, size=(R, 768))
+    es = np.abs(s) * 1e-5 + 1e-3
+    c = np.float32(oracle.softmax_c(scale))
+    for pert in (-es, es, es * rng.uniform(-1, 1, size=s.shape), 0.0 * es):
+        s32 = (s + pert).astype(np.float32)
+        u = (s32[:, :T_kv] * c).astype(np.float32)
+        full = np.full((R, 768), -np.inf, dtype=np.float32)
+        full[:, :T_kv] = u
+        mj = np.maximum.accumulate(full.reshape(R, 3, 256).max(axis=2), axis=1)
+        lo, hi = oracle.flash_weight_interval(s, es, T_kv, scale, mj.astype(np.float64))
+        t = (u - np.repeat(mj, 256, axis=1)[:, :T_kv]).astype(np.float32)
+        w = np.exp2(t.astype(np.float64)).astype(np.float32).astype(np.float64)
+        assert (w >= lo[:, :T_kv]).all() and (w <= hi[:, :T_kv]).all()
+        assert (lo[:, T_kv:] == 0).all() and (hi[:, T_kv:] == 0).all()
+    # an interval without the score error misses some of the perturbed weights
+    s32 = (s + es).astype(np.float32)
+    u = (s32[:, :T_kv] * c).astype(np.float32)
+    full = np.full((R, 768), -np.inf, dtype=np.float32)
+    full[:, :T_kv] = u
+    mj = np.maximum.accumulate(full.reshape(R, 3, 256).max(axis=2), axis=1)
+    lo, hi = oracle.flash_weight_interval(s, 0.0 * es, T_kv, scale, mj.astype(np.float64))
+    t = (u - np.repeat(mj, 256, axis=1)[:, :T_kv]).astype(np.float32)
+    w = np.exp2(t.astype(np.float64)).astype(np.float32).astype(np.float64)
+    assert not ((w >= lo[:, :T_kv]).all() and (w <= hi[:, :T_kv]).all())
