@@ -60,8 +60,8 @@ def parse():
                     help="tokens; smaller values run a reduced case of the same kernels (profiling only)")
     ap.add_argument("--attn-tokens", type=int, default=0,
                     help="profiling only: run one head of FP4 attention (K quantizer over 40 heads of 128, head 17's "
-                         "scores, softmax weights + quantize, P V) at this many tokens for --steps iterations, print "
-                         "timings, exit")
+                         "scores, softmax weights + quantize, P V; MXFP4: then the fused head) at this many "
+                         "tokens for --steps iterations, print timings, exit")
     return ap.parse_args()
 
 
@@ -92,8 +92,8 @@ def attn_profile(args):
     p = fb.attn_softmax_quant(s_buf.zero_(), T, T, 128 ** -0.5, fmt, gp)
     o = torch.empty((T, 128), dtype=torch.bfloat16, device="cuda")
     f = fb.MXFP4 if fmt == "mxfp4" else fb.NVFP4
-    e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
-    t = [0.0] * 4
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    t = [0.0] * 5
     for _ in range(args.steps):
         e[0].record()
         fb.fp4_quantize_heads(f, k, T, Hn, 128, gk, kh[0], kh[1])
@@ -104,15 +104,19 @@ def attn_profile(args):
         e[3].record()
         fb.attn_pv(p, vt, T, T, 17, fmt, gp, gv, o=o)
         e[4].record()
+        if fmt == "mxfp4":
+            fb.attn_fused(qh, kh, vt, T, T, 17, 128 ** -0.5, o=o)
+        e[5].record()
         torch.cuda.synchronize()
-        for i in range(4):
+        for i in range(5):
             t[i] += e[i].elapsed_time(e[i + 1])
     st = fb.fp4_sync_status()
     if st != 0:
         raise RuntimeError(f"device status: {fb.fp4_status_string(st)}")
     print(json.dumps({"attn_tokens": T, "heads": Hn, "fmt": fmt, "quantize_heads_ms": t[0] / args.steps,
                       "scores_ms": t[1] / args.steps, "softmax_quant_ms": t[2] / args.steps,
-                      "pv_ms": t[3] / args.steps, "s_bytes": s_buf.numel() * 2}), flush=True)
+                      "pv_ms": t[3] / args.steps, "fused_ms": t[4] / args.steps, "s_bytes": s_buf.numel() * 2}),
+          flush=True)
     return 0
 
 
@@ -563,6 +567,13 @@ def extra_workloads(fb, torch, args, steps: int = 20, warmup: int = 3):
         o_buf = fb.attn_pv((pc, ps, st), vt, Ta, Ta, 17, fmt, g_p, g_v)
         out[f"{fmt}_attn_pv_head_75600x128x75648"] = timed(
             lambda: fb.attn_pv((pc, ps, st), vt, Ta, Ta, 17, fmt, g_p, g_v, o=o_buf), 2.0 * Ta * kp * 128, n=10)
+        if fmt == "mxfp4":
+            # the same head in one kernel (streaming form): S and P~ never leave the SM
+            st_f = torch.empty((Ta, 2), dtype=torch.float32, device="cuda")
+            out["mxfp4_attn_fused_head_75600x75648x128"] = timed(
+                lambda: fb.attn_fused(qh, kh, vt, Ta, Ta, 17, 128 ** -0.5, o=o_buf, stats=st_f), 4.0 * Ta * kp * 128,
+                n=10)
+            del st_f
         del va, vt, pc, ps, st, o_buf
         del qa, ka, qh, kh, kc_buf, ks_buf, s_buf
     # W4A8 SVDQuant linear at the TI2V-5B shape (MXFP8 activations, rank 32)
@@ -591,6 +602,9 @@ def extra_workloads(fb, torch, args, steps: int = 20, warmup: int = 3):
             v["note"] = "HBM- and exp2-bound: gbs = S read twice + P codes and scales written, per second"
         elif "attn_pv" in k:
             v["note"] = "P V with N = 128 (half of each 256-wide pair MMA); pct_nominal of 9 PFLOP/s dense FP4"
+        elif "attn_fused" in k:
+            v["note"] = ("one head in one kernel: S = Q K^T and O = P~ V on the tensor cores, softmax + P~ quantize "
+                         "on the SM; pct_nominal of 9 PFLOP/s dense FP4 over both products")
         elif "attn_scores" in k:
             v["note"] = "bound by writing S (bf16): s_write_gbs; pct_nominal of 9 PFLOP/s dense FP4"
     return out

@@ -1,0 +1,381 @@
+// attn_fused.cuh -- one head of MXFP4 attention in one kernel: S, the softmax weights and
+// their quantization stay on the SM (TMEM and shared memory), O accumulates in TMEM.
+//
+// Reading (the Wan2.2-Animate-14B MXFP4 card, "Results", names SageAttention v3 as Blackwell
+// microscaling FP4 attention; no page gives its algorithm): the keys are taken in blocks of
+// 256.  For block j and each query row, S_j = deq(Q) deq(K_j)^T (fp32, in TMEM), the running
+// maximum m_j = max(m_{j-1}, max_k fl(s_k c)) (c = scale log2 e), the weights
+// P~_j = 2^(fl(fl(s c) - m_j)) quantized in MXFP4 blocks of 32 keys (the same rule as the
+// activations), O_j = O_{j-1} 2^(m_{j-1} - m_j) + deq(P~_j) deq(V_j) (fp32, in TMEM) and
+// l_j = l_{j-1} 2^(m_{j-1} - m_j) + sum P~_j; the output is bf16_rn(O / l).  The weights are
+// thus quantized against the running maximum of the blocks seen so far, as a streaming
+// (flash) attention must, not against the row's final maximum as the separate-kernel path
+// (fp4_attn_softmax_quant) does.
+//
+// One CTA per 128 query rows of one head; 256 threads: warp 0 TMA producer, warp 1 TMEM
+// owner and MMA issuer, warps 4-7 the softmax (thread = query row = TMEM lane), warps 2-3
+// idle.  Per key block: S_j = Q K_j^T (two 128x256x64 block32 MMAs), the softmax warps read
+// S_j from TMEM twice (block maximum, then the weights), rescale their O row in TMEM when the
+// maximum grew (after the previous P~ V is done), write P~_j into a 128-byte-swizzled shared
+// tile and its scale atoms into shared memory; then O += P~_j V_j (four 128x128x64 MMAs,
+// the P~ atoms copied into TMEM by tcgen05.cp).  K_j, V_j and their atoms come through a
+// two-slot TMA ring.  Every wait is bounded (status FP4_ERR_TIMEOUT).
+#pragma once
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+#include "quant.cuh"
+
+namespace fp4 {
+
+struct AttnParams {
+    int64_t T_q, T_kv, tq_pad, tk_pad;
+    int head, nblk;  // head index; key blocks of 256 (the last may hold 128 padded keys)
+    float c;         // scale * log2(e), fp32
+    const uint8_t* q_sf;  // this head's Q scale atoms (q tile t at t * 512)
+    const uint8_t* k_sf;  // this head's K scale atoms (128-key row block b at b * 512)
+    const uint8_t* v_sf;  // this head's V^T scale atoms (128-key atom a at a * 512)
+    __nv_bfloat16* o;     // [T_q][128]
+    float2* stats;        // [T_q] (final running maximum, l) or null
+    // test hook (null in the product path): for query tile trace_tile only, per key block j
+    // the running maximum m_j of each of its 128 rows ([nblk][128] floats), the P~_j codes
+    // ([nblk][128][128 bytes]) and scale bytes ([nblk][128][8]), padding rows included
+    int trace_tile;
+    float* dbg_m;
+    uint8_t* dbg_codes;
+    uint8_t* dbg_sf;
+    uint64_t timeout_ns;
+    int* status;
+};
+
+constexpr int ATT_THREADS = 256;
+constexpr int ATT_Q_BYTES = 128 * 128;  // 128 rows x 128 bytes (the 64 bytes of a head, zero-filled to 128)
+constexpr int ATT_K_BYTES = 256 * 128;
+constexpr int ATT_V_BYTES = 128 * 128;
+constexpr int ATT_P_BYTES = 128 * 128;
+constexpr int ATT_OFF_K = ATT_Q_BYTES;
+constexpr int ATT_OFF_V = ATT_OFF_K + 2 * ATT_K_BYTES;
+constexpr int ATT_OFF_P = ATT_OFF_V + 2 * ATT_V_BYTES;
+constexpr int ATT_OFF_QSF = ATT_OFF_P + ATT_P_BYTES;
+constexpr int ATT_OFF_KSF = ATT_OFF_QSF + 512;    // [2] x 1024
+constexpr int ATT_OFF_VSF = ATT_OFF_KSF + 2048;   // [2] x 1024
+constexpr int ATT_OFF_PSF = ATT_OFF_VSF + 2048;   // 1024
+constexpr int ATT_OFF_BAR = ATT_OFF_PSF + 1024;
+constexpr int ATT_SMEM = ATT_OFF_BAR + 256;
+static_assert(ATT_OFF_QSF % 1024 == 0, "operand tiles 1024-byte aligned");
+// TMEM columns: S [0, 256), O [256, 384), then the scale buffers
+constexpr uint32_t ATT_T_S = 0, ATT_T_O = 256, ATT_T_QSF = 384;
+constexpr uint32_t ATT_T_KSF = 388;  // [2] x 8: row block 0 at +0, row block 1 at +4
+constexpr uint32_t ATT_T_VSF = 404;  // [2] x 16: atom a at +8a
+constexpr uint32_t ATT_T_PSF = 436;  // [2] x 8: atom a at +4a
+// instruction descriptors: E2M1 x E2M1, UE8M0 scales, M = 128; N = 256 (S) or 128 (P~ V)
+constexpr uint32_t ATT_IDESC = (1u << 7) | (1u << 10) | (1u << 23) | ((uint32_t)(128 >> 4) << 24);
+constexpr uint32_t ATT_IDESC_S = ATT_IDESC | ((uint32_t)(256 >> 3) << 17);
+constexpr uint32_t ATT_IDESC_PV = ATT_IDESC | ((uint32_t)(128 >> 3) << 17);
+
+FP4_DEV void attn_fail(const AttnParams& p, volatile int* abort) {
+    *abort = 1;
+    atomicCAS(p.status, 0, STATUS_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(ATT_THREADS, 1)
+    attn_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, AttnParams p) {
+    extern __shared__ __align__(1024) uint8_t sm[];
+    uint32_t dyn_smem;
+    asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_smem));
+    if ((smem_u32(sm) & 1023u) != 0 || dyn_smem < (uint32_t)ATT_SMEM) {
+        if (threadIdx.x == 0) atomicCAS(p.status, 0, STATUS_LAYOUT);
+        return;
+    }
+    uint8_t* sQ = sm;
+    uint8_t* sK = sm + ATT_OFF_K;
+    uint8_t* sV = sm + ATT_OFF_V;
+    uint8_t* sP = sm + ATT_OFF_P;
+    uint8_t* sQSF = sm + ATT_OFF_QSF;
+    uint8_t* sKSF = sm + ATT_OFF_KSF;
+    uint8_t* sVSF = sm + ATT_OFF_VSF;
+    uint8_t* sPSF = sm + ATT_OFF_PSF;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + ATT_OFF_BAR);
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = bars + 1;   // [2]
+    uint64_t* kv_empty = bars + 3;  // [2]
+    uint64_t* s_full = bars + 5;    // S_j in TMEM (MMA commit)
+    uint64_t* s_free = bars + 6;    // S_j read by the 4 softmax warps
+    uint64_t* p_full = bars + 7;    // P~_j tile and atoms written (4 softmax warps)
+    uint64_t* o_done = bars + 8;    // P~_j V_j done (MMA commit)
+    uint64_t* mma_done = bars + 9;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 10);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qt = blockIdx.x, nb = p.nblk;
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(s_free, 4);
+        mbar_init(p_full, 4);
+        mbar_init(o_done, 1);
+        mbar_init(mma_done, 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    // the scale slots of a partial last key block are not all loaded: start them at zero
+    for (int i = threadIdx.x; i < (2048 + 2048) / 16; i += ATT_THREADS)
+        *reinterpret_cast<uint4*>(sKSF + i * 16) = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ============================================================ producer
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_normal();
+            mbar_arrive_expect_tx(q_full, ATT_Q_BYTES + 512);
+            tma_load_2d(sQ, &tmQ, q_full, 0, (int)(p.head * p.tq_pad + (int64_t)qt * 128), pol);
+            bulk_load(sQSF, p.q_sf + (int64_t)qt * 512, 512, q_full, pol);
+            int j = 0;
+            for (; j < nb; ++j) {
+                const int s = j & 1;
+                if (!mbar_wait(&kv_empty[s], (uint32_t)((j >> 1) & 1) ^ 1u, p.timeout_ns, abort)) {
+                    attn_fail(p, abort);
+                    break;
+                }
+                const int64_t key0 = (int64_t)j * 256;
+                const int rbs = (key0 + 128 < p.tk_pad) ? 2 : 1;  // 128-key row blocks present
+                mbar_arrive_expect_tx(&kv_full[s], ATT_K_BYTES + ATT_V_BYTES + 2 * rbs * 512);
+                tma_load_2d(sK + s * ATT_K_BYTES, &tmK, &kv_full[s], 0, (int)(p.head * p.tk_pad + key0), pol);
+                bulk_load(sKSF + s * 1024, p.k_sf + (int64_t)(2 * j) * 512, rbs * 512, &kv_full[s], pol);
+                tma_load_2d(sV + s * ATT_V_BYTES, &tmV, &kv_full[s], j * 128, p.head * 128, pol);
+                bulk_load(sVSF + s * 1024, p.v_sf + (int64_t)(2 * j) * 512, rbs * 512, &kv_full[s], pol);
+            }
+            // every copy issued must land before the CTA exits
+            for (int i = max(0, j - 2); i < j; ++i)
+                if (!mbar_wait_drain(&kv_full[i & 1], (uint32_t)((i >> 1) & 1), p.timeout_ns)) attn_fail(p, abort);
+            if (!mbar_wait_drain(q_full, 0, p.timeout_ns)) attn_fail(p, abort);
+        }
+    } else if (warp == 1) {
+        // ============================================================ MMA issuer
+        if (lane == 0) {
+            bool ok = mbar_wait(q_full, 0, p.timeout_ns, abort);
+            tc_fence_after();
+            if (ok) tmem_cp_sf_atom(tmem + ATT_T_QSF, smem_desc(smem_u32(sQSF), 0, 128, 0));
+            const uint64_t qdesc = smem_desc(smem_u32(sQ), 0, 1024, 2);
+            const uint64_t pdesc = smem_desc(smem_u32(sP), 0, 1024, 2);
+            auto issue_s = [&](int j) -> bool {
+                const int s = j & 1;
+                if (!mbar_wait(&kv_full[s], (uint32_t)((j >> 1) & 1), p.timeout_ns, abort)) return false;
+                tc_fence_after();
+                tmem_cp_sf_atom(tmem + ATT_T_KSF + s * 8, smem_desc(smem_u32(sKSF + s * 1024), 0, 128, 0));
+                tmem_cp_sf_atom(tmem + ATT_T_KSF + s * 8 + 4, smem_desc(smem_u32(sKSF + s * 1024 + 512), 0, 128, 0));
+                tmem_cp_sf_atom(tmem + ATT_T_VSF + s * 16, smem_desc(smem_u32(sVSF + s * 1024), 0, 128, 0));
+                tmem_cp_sf_atom(tmem + ATT_T_VSF + s * 16 + 8, smem_desc(smem_u32(sVSF + s * 1024 + 512), 0, 128, 0));
+                const uint64_t kdesc = smem_desc(smem_u32(sK + s * ATT_K_BYTES), 0, 1024, 2);
+                // K = 128 dims: MMAs 0 and 1 read bytes 0-31 and 32-63 of each row, scale atom 0
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const uint32_t sf_id = (uint32_t)k * 2u;
+                    mma_mxf4nvf4_block32(tmem + ATT_T_S, qdesc + (uint64_t)(k * 2), kdesc + (uint64_t)(k * 2),
+                                         ATT_IDESC_S | (sf_id << 29) | (sf_id << 4), k > 0 ? 1u : 0u,
+                                         tmem + ATT_T_QSF, tmem + ATT_T_KSF + s * 8);
+                }
+                tc_commit(s_full);
+                return true;
+            };
+            auto issue_pv = [&](int j) -> bool {
+                const int s = j & 1;
+                if (!mbar_wait(p_full, (uint32_t)(j & 1), p.timeout_ns, abort)) return false;
+                tc_fence_after();
+                tmem_cp_sf_atom(tmem + ATT_T_PSF + s * 8, smem_desc(smem_u32(sPSF), 0, 128, 0));
+                tmem_cp_sf_atom(tmem + ATT_T_PSF + s * 8 + 4, smem_desc(smem_u32(sPSF + 512), 0, 128, 0));
+                const uint64_t vdesc = smem_desc(smem_u32(sV + s * ATT_V_BYTES), 0, 1024, 2);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int atom = k >> 1;
+                    const uint32_t sf_id = (uint32_t)(k & 1) * 2u;
+                    mma_mxf4nvf4_block32(tmem + ATT_T_O, pdesc + (uint64_t)(k * 2), vdesc + (uint64_t)(k * 2),
+                                         ATT_IDESC_PV | (sf_id << 29) | (sf_id << 4), (j > 0 || k > 0) ? 1u : 0u,
+                                         tmem + ATT_T_PSF + s * 8 + atom * 4, tmem + ATT_T_VSF + s * 16 + atom * 8);
+                }
+                tc_commit(o_done);
+                tc_commit(&kv_empty[s]);
+                return true;
+            };
+            // from the scale copy on, tensor-core work may be in flight: drain it before exit
+            const bool issued = ok;
+            if (ok) ok = issue_s(0);
+            for (int j = 0; ok && j < nb; ++j) {
+                if (j + 1 < nb) {
+                    // S_{j+1} overwrites S_j: the softmax warps must have read it
+                    ok = mbar_wait(s_free, (uint32_t)(j & 1), p.timeout_ns, abort);
+                    if (ok) tc_fence_after();
+                    if (ok) ok = issue_s(j + 1);
+                }
+                if (ok) ok = issue_pv(j);
+            }
+            if (!ok) attn_fail(p, abort);
+            if (issued) {
+                tc_commit(mma_done);
+                if (!mbar_wait_drain(mma_done, 0, p.timeout_ns)) attn_fail(p, abort);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ============================================================ softmax (thread = query row)
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        const int64_t row = (int64_t)qt * 128 + r;
+        const bool real = row < p.T_q;
+        const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+        const float c = p.c;
+        const bool tracing = p.dbg_m != nullptr && qt == p.trace_tile;
+        float m_run = -INFINITY, l = 0.0f;
+        bool ok = true;
+        for (int j = 0; j < nb && ok; ++j) {
+            ok = __all_sync(0xffffffffu, mbar_wait(s_full, (uint32_t)(j & 1), p.timeout_ns, abort));
+            if (!ok) break;
+            tc_fence_after();
+            const int64_t key0 = (int64_t)j * 256;
+            // pass 1: the block maximum of fl(s c) over the valid keys
+            float mb = -INFINITY;
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tl + ATT_T_S + ch * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (key0 + ch * 32 + i < p.T_kv) mb = fmaxf(mb, __fmul_rn(__uint_as_float(v[i]), c));
+            }
+            const float m_new = fmaxf(m_run, mb);
+            // P~_{j-1} V_{j-1} must be done before the P~ tile, its atoms or O are touched
+            if (j > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)((j - 1) & 1), p.timeout_ns, abort));
+                if (!ok) break;
+                tc_fence_after();
+            }
+            // O and l follow the new maximum: O *= 2^(m_prev - m_new) (whole warp, a factor of 1
+            // for rows whose maximum did not grow)
+            const bool grow = (j > 0) && (m_new > m_run);
+            const bool warp_grow = __any_sync(0xffffffffu, grow);
+            if (warp_grow) {
+                const float f = grow ? exp2f(__fsub_rn(m_run, m_new)) : 1.0f;
+                l = __fmul_rn(l, f);
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld_32x32b_x32(tl + ATT_T_O + ch * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), f));
+                    tmem_st_32x32b_x16(tl + ATT_T_O + ch * 32, *reinterpret_cast<const uint32_t(*)[16]>(o));
+                    tmem_st_32x32b_x16(tl + ATT_T_O + ch * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(o + 16));
+                }
+            }
+            // pass 2: P~ = exp2(fl(fl(s c) - m_new)), MXFP4 groups of 32 keys, into row r of the
+            // 128-byte-swizzled P~ tile (16-byte granule g at g ^ (r % 8))
+            uint32_t words[2] = {0u, 0u};
+            float lb = 0.0f;
+            const uint32_t prow = smem_u32(sP) + (uint32_t)r * 128u;
+            for (int ch = 0; ch < 8; ++ch) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tl + ATT_T_S + ch * 32, v);
+                tmem_wait_ld();
+                float pv[32], part[16];
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const bool valid = key0 + ch * 32 + i < p.T_kv;
+                    pv[i] = valid ? exp2f(__fsub_rn(__fmul_rn(__uint_as_float(v[i]), c), m_new)) : 0.0f;
+                    amax = fmaxf(amax, pv[i]);
+                }
+                // the 32 weights summed as a pairwise tree, then added to the block's sum in order
+#pragma unroll
+                for (int i = 0; i < 16; ++i) part[i] = __fadd_rn(pv[2 * i], pv[2 * i + 1]);
+#pragma unroll
+                for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int i = 0; i < w; ++i) part[i] = __fadd_rn(part[i], part[i + w]);
+                lb = __fadd_rn(lb, part[0]);
+                const uint32_t sfb = mx_scale_byte<2>(amax);
+                const float inv = mx_inv_scale(sfb);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) pv[i] = __fmul_rn(pv[i], inv);
+                uint32_t cw[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) cw[q] = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(pv + 8 * q));
+                st_shared_v4(prow + (uint32_t)((ch ^ (r & 7)) * 16), cw[0], cw[1], cw[2], cw[3]);
+                words[ch >> 2] |= sfb << (8 * (ch & 3));
+                if (tracing) {
+                    const int64_t d = (int64_t)j * 128 + r;
+                    *reinterpret_cast<uint4*>(p.dbg_codes + d * 128 + ch * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                    p.dbg_sf[d * 8 + ch] = (uint8_t)sfb;
+                }
+            }
+            l = __fadd_rn(l, lb);
+            // S_j is read: the MMA warp may compute S_{j+1}
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_free);
+            // the row's scale words into the two P~ atoms (keys 0-127, 128-255)
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+                *reinterpret_cast<uint32_t*>(sPSF + a * 512 + (r & 31) * 16 + (r >> 5) * 4) = words[a];
+            if (warp_grow) tmem_wait_st();
+            if (tracing) p.dbg_m[(int64_t)j * 128 + r] = m_new;
+            // the tile and atoms are written by threads and read by the tensor core
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+            m_run = m_new;
+        }
+        // O / l, rounded once to bf16
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)((nb - 1) & 1), p.timeout_ns, abort));
+        if (ok) {
+            tc_fence_after();
+            const float inv_l = __frcp_rn(l);
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t o[32];
+                tmem_ld_32x32b_x32(tl + ATT_T_O + ch * 32, o);
+                tmem_wait_ld();
+                if (real) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(o[2 * i]), inv_l),
+                                                                 __fmul_rn(__uint_as_float(o[2 * i + 1]), inv_l));
+                        w[i] = *reinterpret_cast<uint32_t*>(&b);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(p.o + row * 128 + ch * 32);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                }
+            }
+            if (p.stats != nullptr && real) p.stats[row] = make_float2(m_run, l);
+        } else if (lane == 0) {
+            attn_fail(p, abort);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace fp4

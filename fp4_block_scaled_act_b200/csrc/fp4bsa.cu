@@ -9,6 +9,7 @@
 
 #include "fp4bsa.h"
 #include "attn.cuh"
+#include "attn_fused.cuh"
 #include "gemm.cuh"
 #include "quant.cuh"
 
@@ -100,7 +101,9 @@ fp4_status_t device_state(DeviceState** out) {
                 cudaFuncSetAttribute(gemm2_kernel<G_MXFP4, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Gemm2Cfg<G_MXFP4>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm2_kernel<G_NVFP4, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     Gemm2Cfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess)
+                                     Gemm2Cfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(attn_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM) !=
+                    cudaSuccess)
                 return FP4_ERR_CUDA;
             {
                 constexpr int R = (int)Gemm2Cfg<G_MXFP4>::REG_LAUNCH;
@@ -716,6 +719,84 @@ fp4_status_t fp4_attn_scores(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_
     // S = Q_h K_h^T: Q_h is the activation operand (M = T_q), K_h the weight operand over
     // all T_kv_pad key rows (padding keys have zero codes, so their columns hold 0)
     return gemm_impl(fmt, qc, qs, T_q, D, tk_pad, kc, ks, g_k, g_q, nullptr, s_bf16, stream, nullptr, 0);
+}
+
+}  // extern "C"
+
+namespace {
+fp4_status_t attn_fused_impl(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,
+                             const uint8_t* k_codes, const uint8_t* k_sf, int64_t T_kv, const uint8_t* vt_codes,
+                             const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale, void* stats,
+                             void* o_bf16, int64_t trace_tile, float* trace_m, uint8_t* trace_codes,
+                             uint8_t* trace_sf, void* stream) {
+    if (fmt != FP4_FMT_MXFP4 || !q_codes || !q_sf || !k_codes || !k_sf || !vt_codes || !vt_sf || !o_bf16)
+        return FP4_ERR_INVALID_ARG;
+    if (T_q < 1 || T_kv < 1 || H < 1 || head < 0 || head >= H) return FP4_ERR_INVALID_ARG;
+    if (!(scale > 0.0f) || !(scale < 3.0e38f)) return FP4_ERR_INVALID_ARG;
+    if (D != FP4_HEAD_DIM) return FP4_ERR_UNSUPPORTED_SHAPE;
+    const int64_t tq_pad = (T_q + 127) / 128 * 128, tk_pad = (T_kv + 127) / 128 * 128;
+    // TMA row coordinates are 32-bit: every head's padded rows must stay below 2^31
+    if (T_q >= kMaxDim || T_kv >= kMaxDim || H * tq_pad >= ((int64_t)1 << 31) || H * tk_pad >= ((int64_t)1 << 31))
+        return FP4_ERR_UNSUPPORTED_SHAPE;
+    const bool tracing = trace_m || trace_codes || trace_sf;
+    if (tracing && (!trace_m || !trace_codes || !trace_sf || trace_tile < 0 || trace_tile >= tq_pad / 128))
+        return FP4_ERR_INVALID_ARG;
+    if (!aligned16(q_codes) || !aligned16(q_sf) || !aligned16(k_codes) || !aligned16(k_sf) || !aligned16(vt_codes) ||
+        !aligned16(vt_sf) || !aligned16(stats) || !aligned16(o_bf16) || !aligned16(trace_m) ||
+        !aligned16(trace_codes) || !aligned16(trace_sf))
+        return FP4_ERR_MISALIGNED;
+    DeviceState* ds;
+    fp4_status_t s = device_state(&ds);
+    if (s != FP4_OK) return s;
+    // Q and K: all heads' rows of 64 bytes (zero-filled to the 128-byte box); V^T: H * 128
+    // rows of T_kv_pad / 2 bytes, one 256-key box per block
+    CUtensorMap tq, tk, tv;
+    if ((s = encode_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_codes, D / 2, (uint64_t)(H * tq_pad), D / 2, 128, 128)) !=
+        FP4_OK)
+        return s;
+    if ((s = encode_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_codes, D / 2, (uint64_t)(H * tk_pad), D / 2, 128, 256)) !=
+        FP4_OK)
+        return s;
+    if ((s = encode_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, vt_codes, (uint64_t)(tk_pad / 2), (uint64_t)(H * D),
+                       (uint64_t)(tk_pad / 2), 128, 128)) != FP4_OK)
+        return s;
+    AttnParams p{};
+    p.T_q = T_q, p.T_kv = T_kv, p.tq_pad = tq_pad, p.tk_pad = tk_pad;
+    p.head = (int)head;
+    p.nblk = (int)((tk_pad + 255) / 256);
+    p.c = (float)((double)scale * 1.4426950408889634);
+    p.q_sf = q_sf + (size_t)head * fp4_sf_bytes(fmt, T_q, D);
+    p.k_sf = k_sf + (size_t)head * fp4_sf_bytes(fmt, T_kv, D);
+    p.v_sf = vt_sf + (size_t)head * fp4_sf_bytes(fmt, D, tk_pad);
+    p.o = static_cast<__nv_bfloat16*>(o_bf16);
+    p.stats = static_cast<float2*>(stats);
+    p.trace_tile = tracing ? (int)trace_tile : -1;
+    p.dbg_m = trace_m, p.dbg_codes = trace_codes, p.dbg_sf = trace_sf;
+    p.timeout_ns = g_timeout_ns;
+    p.status = ds->status;
+    attn_fused_kernel<<<(unsigned)(tq_pad / 128), ATT_THREADS, ATT_SMEM, static_cast<cudaStream_t>(stream)>>>(tq, tk,
+                                                                                                         tv, p);
+    return launched();
+}
+}  // namespace
+
+extern "C" {
+
+fp4_status_t fp4_attn_fused(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,
+                            const uint8_t* k_codes, const uint8_t* k_sf, int64_t T_kv, const uint8_t* vt_codes,
+                            const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale, void* stats,
+                            void* o_bf16, void* stream) {
+    return attn_fused_impl(fmt, q_codes, q_sf, T_q, k_codes, k_sf, T_kv, vt_codes, vt_sf, H, D, head, scale, stats,
+                           o_bf16, -1, nullptr, nullptr, nullptr, stream);
+}
+
+fp4_status_t fp4_attn_fused_trace(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,
+                                  const uint8_t* k_codes, const uint8_t* k_sf, int64_t T_kv, const uint8_t* vt_codes,
+                                  const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale, void* stats,
+                                  void* o_bf16, int64_t trace_tile, float* trace_m, uint8_t* trace_codes,
+                                  uint8_t* trace_sf, void* stream) {
+    return attn_fused_impl(fmt, q_codes, q_sf, T_q, k_codes, k_sf, T_kv, vt_codes, vt_sf, H, D, head, scale, stats,
+                           o_bf16, trace_tile, trace_m, trace_codes, trace_sf, stream);
 }
 
 fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K, int64_t N, const uint8_t* w_codes,
