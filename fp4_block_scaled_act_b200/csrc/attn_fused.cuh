@@ -12,16 +12,21 @@
 // (flash) attention must, not against the row's final maximum as the separate-kernel path
 // (fp4_attn_softmax_quant) does.
 //
-// One CTA per 128 query rows of one head; 256 threads: warp 0 TMA producer, warp 1 TMEM
-// owner and MMA issuer, warps 4-7 the softmax (thread = query row = TMEM lane), warps 2-3
-// idle.  Per key block: S_j = Q K_j^T (two 128x256x64 block32 MMAs), the softmax warps read
-// S_j from TMEM twice (block maximum, then the weights), rescale their O row in TMEM when the
-// maximum grew (after the previous P~ V is done), write P~_j into a 128-byte-swizzled shared
-// tile and its scale atoms into shared memory; then O += P~_j V_j (four 128x128x64 MMAs,
-// the P~ atoms copied into TMEM by tcgen05.cp).  K_j, V_j and their atoms come through a
-// two-slot TMA ring.  Every wait is bounded (status FP4_ERR_TIMEOUT).
+// One CTA per 128 query rows of one head; 384 threads: warp 0 TMA producer, warp 1 TMEM
+// owner and MMA issuer, warps 2-3 idle, warps 4-11 the softmax (a thread is one query row,
+// its TMEM lane, in one half of the key block: warps 4-7 keys 0-127, warps 8-11 keys 128-255).
+// Per key block: S_j = Q K_j^T (two 128x256x64 block32 MMAs); each softmax thread reads its
+// half of S_j from TMEM twice (the half's maximum, exchanged with the other half through
+// shared memory and a pair mbarrier; then the weights), rescales its 64 columns of O in TMEM
+// when the maximum grew (after the previous P~ V is done), writes its P~_j codes into a
+// 128-byte-swizzled shared tile and its scale word into the half's atom; then O += P~_j V_j
+// (four 128x128x64 MMAs, the P~ atoms copied into TMEM by tcgen05.cp).  Each half keeps its
+// own l (scaled by the same factors); the two are added at the end.  K_j, V_j and their atoms
+// come through a two-slot TMA ring.  Every wait is bounded (status FP4_ERR_TIMEOUT).
 #pragma once
 #include <cuda_bf16.h>
+
+#include <type_traits>
 
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -48,7 +53,7 @@ struct AttnParams {
     int* status;
 };
 
-constexpr int ATT_THREADS = 256;
+constexpr int ATT_THREADS = 384;
 constexpr int ATT_Q_BYTES = 128 * 128;  // 128 rows x 128 bytes (the 64 bytes of a head, zero-filled to 128)
 constexpr int ATT_K_BYTES = 256 * 128;
 constexpr int ATT_V_BYTES = 128 * 128;
@@ -60,7 +65,8 @@ constexpr int ATT_OFF_QSF = ATT_OFF_P + ATT_P_BYTES;
 constexpr int ATT_OFF_KSF = ATT_OFF_QSF + 512;    // [2] x 1024
 constexpr int ATT_OFF_VSF = ATT_OFF_KSF + 2048;   // [2] x 1024
 constexpr int ATT_OFF_PSF = ATT_OFF_VSF + 2048;   // 1024
-constexpr int ATT_OFF_BAR = ATT_OFF_PSF + 1024;
+constexpr int ATT_OFF_RED = ATT_OFF_PSF + 1024;    // [2][2][128] floats
+constexpr int ATT_OFF_BAR = ATT_OFF_RED + 2048;
 constexpr int ATT_SMEM = ATT_OFF_BAR + 256;
 static_assert(ATT_OFF_QSF % 1024 == 0, "operand tiles 1024-byte aligned");
 // TMEM columns: S [0, 256), O [256, 384), then the scale buffers
@@ -105,7 +111,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     uint64_t* p_full = bars + 7;    // P~_j tile and atoms written (4 softmax warps)
     uint64_t* o_done = bars + 8;    // P~_j V_j done (MMA commit)
     uint64_t* mma_done = bars + 9;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 10);
+    uint64_t* pair_bar = bars + 10;  // [4]: the two softmax warps on rows 32 q .. 32 q + 31
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -117,8 +124,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             mbar_init(&kv_empty[i], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(s_free, 4);
-        mbar_init(p_full, 4);
+        mbar_init(s_free, 8);
+        mbar_init(p_full, 8);
+        for (int i = 0; i < 4; ++i) mbar_init(&pair_bar[i], 2);
         mbar_init(o_done, 1);
         mbar_init(mma_done, 1);
         *abort = 0;
@@ -236,32 +244,71 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         __syncwarp();
     } else if (warp >= 4) {
-        // ============================================================ softmax (thread = query row)
+        // ============================================================ softmax
+        // warps 4-7 take keys 0-127 of every block, warps 8-11 keys 128-255; a thread is one
+        // query row (its TMEM lane) in one half; the two warps on the same rows exchange their
+        // maxima and, at the end, their sums through shared memory and a pair mbarrier
         const int q4 = warp & 3;
+        const int h = (warp - 4) >> 2;
         const int r = q4 * 32 + lane;
         const int64_t row = (int64_t)qt * 128 + r;
         const bool real = row < p.T_q;
         const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+        const uint32_t t_s = tl + ATT_T_S + (uint32_t)h * 128u;  // this half's S columns
+        const uint32_t t_o = tl + ATT_T_O + (uint32_t)h * 64u;   // this half's O columns
+        float* red = reinterpret_cast<float*>(sm + ATT_OFF_RED);  // [2 phases][2 halves][128 rows]
+        uint64_t* pair = &pair_bar[q4];
         const float c = p.c;
         const bool tracing = p.dbg_m != nullptr && qt == p.trace_tile;
-        float m_run = -INFINITY, l = 0.0f;
+        float m_run = -INFINITY, l = 0.0f;  // l: this half's sum
         bool ok = true;
-        for (int j = 0; j < nb && ok; ++j) {
+        int j = 0;
+        for (; j < nb && ok; ++j) {
             ok = __all_sync(0xffffffffu, mbar_wait(s_full, (uint32_t)(j & 1), p.timeout_ns, abort));
             if (!ok) break;
             tc_fence_after();
-            const int64_t key0 = (int64_t)j * 256;
-            // pass 1: the block maximum of fl(s c) over the valid keys
-            float mb = -INFINITY;
-            for (int ch = 0; ch < 8; ++ch) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tl + ATT_T_S + ch * 32, v);
-                tmem_wait_ld();
+            const int64_t k0 = (int64_t)j * 256 + h * 128;  // this half's first key
+            const int nvalid = (int)(p.T_kv - k0 >= 128 ? 128 : (p.T_kv > k0 ? p.T_kv - k0 : 0));
+            // pass 1: the half's maximum of s over its valid keys; c > 0, so the block's
+            // max fl(s c) is fl(max s * c)
+            float mx = -INFINITY;
+            if (nvalid == 128) {
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ch += 2) {
+                    uint32_t v[32], w[32];
+                    tmem_ld_32x32b_x32(t_s + ch * 32, v);
+                    tmem_ld_32x32b_x32(t_s + ch * 32 + 32, w);
+                    tmem_wait_ld();
+                    tmem_tie(v);
+                    tmem_tie(w);
+                    float t[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (key0 + ch * 32 + i < p.T_kv) mb = fmaxf(mb, __fmul_rn(__uint_as_float(v[i]), c));
+                    for (int i = 0; i < 32; ++i) t[i] = fmaxf(__uint_as_float(v[i]), __uint_as_float(w[i]));
+#pragma unroll
+                    for (int n = 16; n >= 1; n >>= 1)
+#pragma unroll
+                        for (int i = 0; i < n; ++i) t[i] = fmaxf(t[i], t[i + n]);
+                    mx = fmaxf(mx, t[0]);
+                }
+            } else {
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(t_s + ch * 32, v);
+                    tmem_wait_ld();
+                    tmem_tie(v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (ch * 32 + i < nvalid) mx = fmaxf(mx, __uint_as_float(v[i]));
+                }
             }
-            const float m_new = fmaxf(m_run, mb);
+            red[((j & 1) * 2 + h) * 128 + r] = mx;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pair);
+            ok = __all_sync(0xffffffffu, mbar_wait(pair, (uint32_t)(j & 1), p.timeout_ns, abort));
+            if (!ok) break;
+            const float mb = fmaxf(mx, red[((j & 1) * 2 + (h ^ 1)) * 128 + r]);
+            const float m_new = fmaxf(m_run, __fmul_rn(mb, c));
             // P~_{j-1} V_{j-1} must be done before the P~ tile, its atoms or O are touched
             if (j > 0) {
                 ok = __all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)((j - 1) & 1), p.timeout_ns, abort));
@@ -269,47 +316,57 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 tc_fence_after();
             }
             // O and l follow the new maximum: O *= 2^(m_prev - m_new) (whole warp, a factor of 1
-            // for rows whose maximum did not grow)
+            // for rows whose maximum did not grow); each half rescales its 64 columns of O
             const bool grow = (j > 0) && (m_new > m_run);
             const bool warp_grow = __any_sync(0xffffffffu, grow);
             if (warp_grow) {
                 const float f = grow ? exp2f(__fsub_rn(m_run, m_new)) : 1.0f;
                 l = __fmul_rn(l, f);
-                for (int ch = 0; ch < 4; ++ch) {
+#pragma unroll 1
+                for (int ch = 0; ch < 2; ++ch) {
                     uint32_t o[32];
-                    tmem_ld_32x32b_x32(tl + ATT_T_O + ch * 32, o);
+                    tmem_ld_32x32b_x32(t_o + ch * 32, o);
                     tmem_wait_ld();
+                    tmem_tie(o);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), f));
-                    tmem_st_32x32b_x16(tl + ATT_T_O + ch * 32, *reinterpret_cast<const uint32_t(*)[16]>(o));
-                    tmem_st_32x32b_x16(tl + ATT_T_O + ch * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(o + 16));
+                    tmem_st_32x32b_x16(t_o + ch * 32, *reinterpret_cast<const uint32_t(*)[16]>(o));
+                    tmem_st_32x32b_x16(t_o + ch * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(o + 16));
                 }
             }
             // pass 2: P~ = exp2(fl(fl(s c) - m_new)), MXFP4 groups of 32 keys, into row r of the
             // 128-byte-swizzled P~ tile (16-byte granule g at g ^ (r % 8))
-            uint32_t words[2] = {0u, 0u};
+            uint32_t word = 0u;
             float lb = 0.0f;
             const uint32_t prow = smem_u32(sP) + (uint32_t)r * 128u;
-            for (int ch = 0; ch < 8; ++ch) {
+            auto chunk = [&](int ch, auto full_tag) {
+                constexpr bool FULL = decltype(full_tag)::value;
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tl + ATT_T_S + ch * 32, v);
+                tmem_ld_32x32b_x32(t_s + ch * 32, v);
                 tmem_wait_ld();
-                float pv[32], part[16];
-                float amax = 0.0f;
+                tmem_tie(v);
+                float pv[32], part[16], mxp[16];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const bool valid = key0 + ch * 32 + i < p.T_kv;
+                    const bool valid = FULL || ch * 32 + i < nvalid;
                     pv[i] = valid ? exp2f(__fsub_rn(__fmul_rn(__uint_as_float(v[i]), c), m_new)) : 0.0f;
-                    amax = fmaxf(amax, pv[i]);
                 }
-                // the 32 weights summed as a pairwise tree, then added to the block's sum in order
+                // the 32 weights summed as a pairwise tree, then added to the half's block sum in
+                // order; their maximum by the same tree
 #pragma unroll
-                for (int i = 0; i < 16; ++i) part[i] = __fadd_rn(pv[2 * i], pv[2 * i + 1]);
+                for (int i = 0; i < 16; ++i) {
+                    part[i] = __fadd_rn(pv[2 * i], pv[2 * i + 1]);
+                    mxp[i] = fmaxf(pv[2 * i], pv[2 * i + 1]);
+                }
 #pragma unroll
                 for (int w = 8; w >= 1; w >>= 1)
 #pragma unroll
-                    for (int i = 0; i < w; ++i) part[i] = __fadd_rn(part[i], part[i + w]);
+                    for (int i = 0; i < w; ++i) {
+                        part[i] = __fadd_rn(part[i], part[i + w]);
+                        mxp[i] = fmaxf(mxp[i], mxp[i + w]);
+                    }
                 lb = __fadd_rn(lb, part[0]);
+                const float amax = mxp[0];
                 const uint32_t sfb = mx_scale_byte<2>(amax);
                 const float inv = mx_inv_scale(sfb);
 #pragma unroll
@@ -317,25 +374,31 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 uint32_t cw[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) cw[q] = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(pv + 8 * q));
-                st_shared_v4(prow + (uint32_t)((ch ^ (r & 7)) * 16), cw[0], cw[1], cw[2], cw[3]);
-                words[ch >> 2] |= sfb << (8 * (ch & 3));
+                const int gch = h * 4 + ch;  // the chunk's 16-byte granule in the 256-key row
+                st_shared_v4(prow + (uint32_t)((gch ^ (r & 7)) * 16), cw[0], cw[1], cw[2], cw[3]);
+                word |= sfb << (8 * ch);
                 if (tracing) {
                     const int64_t d = (int64_t)j * 128 + r;
-                    *reinterpret_cast<uint4*>(p.dbg_codes + d * 128 + ch * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-                    p.dbg_sf[d * 8 + ch] = (uint8_t)sfb;
+                    *reinterpret_cast<uint4*>(p.dbg_codes + d * 128 + gch * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                    p.dbg_sf[d * 8 + gch] = (uint8_t)sfb;
                 }
+            };
+            if (nvalid == 128) {
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) chunk(ch, std::true_type{});
+            } else {
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) chunk(ch, std::false_type{});
             }
             l = __fadd_rn(l, lb);
             // S_j is read: the MMA warp may compute S_{j+1}
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_free);
-            // the row's scale words into the two P~ atoms (keys 0-127, 128-255)
-#pragma unroll
-            for (int a = 0; a < 2; ++a)
-                *reinterpret_cast<uint32_t*>(sPSF + a * 512 + (r & 31) * 16 + (r >> 5) * 4) = words[a];
+            // the row's scale word into this half's P~ atom (keys 0-127 or 128-255)
+            *reinterpret_cast<uint32_t*>(sPSF + h * 512 + (r & 31) * 16 + (r >> 5) * 4) = word;
             if (warp_grow) tmem_wait_st();
-            if (tracing) p.dbg_m[(int64_t)j * 128 + r] = m_new;
+            if (tracing && h == 0) p.dbg_m[(int64_t)j * 128 + r] = m_new;
             // the tile and atoms are written by threads and read by the tensor core
             fence_proxy_async_smem();
             tc_fence_before();
@@ -343,15 +406,24 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             if (lane == 0) mbar_arrive(p_full);
             m_run = m_new;
         }
-        // O / l, rounded once to bf16
+        // the two halves' sums added in a fixed order, then O / l rounded once to bf16
+        if (ok) {
+            red[((nb & 1) * 2 + h) * 128 + r] = l;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pair);
+            ok = __all_sync(0xffffffffu, mbar_wait(pair, (uint32_t)(nb & 1), p.timeout_ns, abort));
+        }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)((nb - 1) & 1), p.timeout_ns, abort));
         if (ok) {
             tc_fence_after();
-            const float inv_l = __frcp_rn(l);
-            for (int ch = 0; ch < 4; ++ch) {
+            const float lt = __fadd_rn(red[((nb & 1) * 2) * 128 + r], red[((nb & 1) * 2 + 1) * 128 + r]);
+            const float inv_l = __frcp_rn(lt);
+#pragma unroll 1
+            for (int ch = 0; ch < 2; ++ch) {
                 uint32_t o[32];
-                tmem_ld_32x32b_x32(tl + ATT_T_O + ch * 32, o);
+                tmem_ld_32x32b_x32(t_o + ch * 32, o);
                 tmem_wait_ld();
+                tmem_tie(o);
                 if (real) {
                     uint32_t w[16];
 #pragma unroll
@@ -360,12 +432,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                                                  __fmul_rn(__uint_as_float(o[2 * i + 1]), inv_l));
                         w[i] = *reinterpret_cast<uint32_t*>(&b);
                     }
-                    uint4* dst = reinterpret_cast<uint4*>(p.o + row * 128 + ch * 32);
+                    uint4* dst = reinterpret_cast<uint4*>(p.o + row * 128 + h * 64 + ch * 32);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
                 }
             }
-            if (p.stats != nullptr && real) p.stats[row] = make_float2(m_run, l);
+            if (p.stats != nullptr && real && h == 0) p.stats[row] = make_float2(m_run, lt);
         } else if (lane == 0) {
             attn_fail(p, abort);
         }

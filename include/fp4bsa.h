@@ -422,11 +422,12 @@ fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p
  * query row and block j: s = deq(q) deq(k)^T in fp32 (never rounded to bf16), the running
  * maximum m_j = max(m_{j-1}, max fl(s c)) over the block's keys < T_kv (c = fp32(scale *
  * log2 e)), the weights p~ = exp2(fl(fl(s c) - m_j)) quantized as MXFP4 in groups of 32 keys,
- * O_j = O_{j-1} f_j + deq(P~_j) deq(V_j) and l_j = fl(fl(l_{j-1} f_j) + the block's sum of
- * p~) with f_j = exp2(fl(m_{j-1} - m_j)) (1 when the maximum did not grow); each block's sum
- * adds, in key order, eight pairwise-tree sums of 32 weights.  The output is o = bf16_rn(O
- * fl(1 / l)).  The weights are thus quantized against the running maximum, not the row's
- * final one as fp4_attn_softmax_quant does, and S stays in fp32.
+ * O_j = O_{j-1} f_j + deq(P~_j) deq(V_j) with f_j = exp2(fl(m_{j-1} - m_j)) (1 when the
+ * maximum did not grow); the sum is kept per half block (keys 0-127 and 128-255 of every
+ * block): l_h = fl(fl(l_h f_j) + the half's four pairwise-tree sums of 32 weights, added in key
+ * order), and l = fl(l_0 + l_1).  The output is o = bf16_rn(O fl(1 / l)).  The weights are
+ * thus quantized against the running maximum, not the row's final one as
+ * fp4_attn_softmax_quant does, and S stays in fp32.
  *   q_codes / q_sf, k_codes / k_sf   fp4_quantize_heads' buffers (T_q resp. T_kv tokens)
  *   vt_codes / vt_sf                 fp4_quantize_heads_vt's buffers (T_kv tokens)
  *   scale   the softmax scale, > 0 and finite
