@@ -12,17 +12,19 @@
 // (flash) attention must, not against the row's final maximum as the separate-kernel path
 // (fp4_attn_softmax_quant) does.
 //
-// One CTA per 128 query rows of one head; 384 threads: warp 0 TMA producer, warp 1 TMEM
-// owner and MMA issuer, warps 2-3 idle, warps 4-11 the softmax (a thread is one query row,
-// its TMEM lane, in one half of the key block: warps 4-7 keys 0-127, warps 8-11 keys 128-255).
+// One CTA per 128 query rows of one head; 640 threads: warp 0 TMA producer, warp 1 TMEM
+// owner and MMA issuer, warps 2-3 idle, warps 4-19 the softmax (a thread is one query row,
+// its TMEM lane, in one quarter of the key block: warp w takes keys 64 qq .. 64 qq + 63 with
+// qq = (w - 4) / 4, four warps per SM sub-partition to hide the latency of TMEM loads and exp2).
 // Per key block: S_j = Q K_j^T (two 128x256x64 block32 MMAs); each softmax thread reads its
-// half of S_j from TMEM twice (the half's maximum, exchanged with the other half through
-// shared memory and a pair mbarrier; then the weights), rescales its 64 columns of O in TMEM
-// when the maximum grew (after the previous P~ V is done), writes its P~_j codes into a
-// 128-byte-swizzled shared tile and its scale word into the half's atom; then O += P~_j V_j
-// (four 128x128x64 MMAs, the P~ atoms copied into TMEM by tcgen05.cp).  Each half keeps its
-// own l (scaled by the same factors); the two are added at the end.  K_j, V_j and their atoms
-// come through a two-slot TMA ring.  Every wait is bounded (status FP4_ERR_TIMEOUT).
+// quarter of S_j from TMEM twice (the quarter's maximum, exchanged with the other quarters
+// through shared memory and a bounded mbarrier; then the weights), rescales its 32 columns of
+// O in TMEM when the maximum grew (after the previous P~ V is done), writes its P~_j codes into
+// a 128-byte-swizzled shared tile and its two scale bytes into the P~ atom; then
+// O += P~_j V_j (four 128x128x64 MMAs, the P~ atoms copied into TMEM by tcgen05.cp).  Each
+// quarter keeps its own l (scaled by the same factors); they are added at the end.  K_j, V_j
+// and their atoms come through a two-slot TMA ring.  Every wait is bounded (status
+// FP4_ERR_TIMEOUT).
 #pragma once
 #include <cuda_bf16.h>
 
@@ -53,7 +55,7 @@ struct AttnParams {
     int* status;
 };
 
-constexpr int ATT_THREADS = 384;
+constexpr int ATT_THREADS = 640;
 constexpr int ATT_Q_BYTES = 128 * 128;  // 128 rows x 128 bytes (the 64 bytes of a head, zero-filled to 128)
 constexpr int ATT_K_BYTES = 256 * 128;
 constexpr int ATT_V_BYTES = 128 * 128;
@@ -65,8 +67,8 @@ constexpr int ATT_OFF_QSF = ATT_OFF_P + ATT_P_BYTES;
 constexpr int ATT_OFF_KSF = ATT_OFF_QSF + 512;    // [2] x 1024
 constexpr int ATT_OFF_VSF = ATT_OFF_KSF + 2048;   // [2] x 1024
 constexpr int ATT_OFF_PSF = ATT_OFF_VSF + 2048;   // 1024
-constexpr int ATT_OFF_RED = ATT_OFF_PSF + 1024;    // [2][2][128] floats
-constexpr int ATT_OFF_BAR = ATT_OFF_RED + 2048;
+constexpr int ATT_OFF_RED = ATT_OFF_PSF + 1024;    // [2][4][128] floats
+constexpr int ATT_OFF_BAR = ATT_OFF_RED + 4096;
 constexpr int ATT_SMEM = ATT_OFF_BAR + 256;
 static_assert(ATT_OFF_QSF % 1024 == 0, "operand tiles 1024-byte aligned");
 // TMEM columns: S [0, 256), O [256, 384), then the scale buffers
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     uint64_t* p_full = bars + 7;    // P~_j tile and atoms written (4 softmax warps)
     uint64_t* o_done = bars + 8;    // P~_j V_j done (MMA commit)
     uint64_t* mma_done = bars + 9;
-    uint64_t* pair_bar = bars + 10;  // [4]: the two softmax warps on rows 32 q .. 32 q + 31
+    uint64_t* pair_bar = bars + 10;  // [4]: the four softmax warps on rows 32 q .. 32 q + 31
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -124,9 +126,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             mbar_init(&kv_empty[i], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(s_free, 8);
-        mbar_init(p_full, 8);
-        for (int i = 0; i < 4; ++i) mbar_init(&pair_bar[i], 2);
+        mbar_init(s_free, 16);
+        mbar_init(p_full, 16);
+        for (int i = 0; i < 4; ++i) mbar_init(&pair_bar[i], 4);
         mbar_init(o_done, 1);
         mbar_init(mma_done, 1);
         *abort = 0;
@@ -245,69 +247,63 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         __syncwarp();
     } else if (warp >= 4) {
         // ============================================================ softmax
-        // warps 4-7 take keys 0-127 of every block, warps 8-11 keys 128-255; a thread is one
-        // query row (its TMEM lane) in one half; the two warps on the same rows exchange their
-        // maxima and, at the end, their sums through shared memory and a pair mbarrier
+        // warps 4-19: warp w takes keys 64 qq .. 64 qq + 63 of every block (qq = (w - 4) / 4)
+        // for the 32 query rows of TMEM lanes 32 (w % 4) ..; a thread is one query row in one
+        // quarter.  The four warps on the same rows exchange their maxima and, at the end,
+        // their sums through shared memory and a bounded mbarrier.
         const int q4 = warp & 3;
-        const int h = (warp - 4) >> 2;
+        const int qq = (warp - 4) >> 2;
         const int r = q4 * 32 + lane;
         const int64_t row = (int64_t)qt * 128 + r;
         const bool real = row < p.T_q;
         const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
-        const uint32_t t_s = tl + ATT_T_S + (uint32_t)h * 128u;  // this half's S columns
-        const uint32_t t_o = tl + ATT_T_O + (uint32_t)h * 64u;   // this half's O columns
-        float* red = reinterpret_cast<float*>(sm + ATT_OFF_RED);  // [2 phases][2 halves][128 rows]
+        const uint32_t t_s = tl + ATT_T_S + (uint32_t)qq * 64u;  // this quarter's S columns
+        const uint32_t t_o = tl + ATT_T_O + (uint32_t)qq * 32u;  // this quarter's O columns
+        float* red = reinterpret_cast<float*>(sm + ATT_OFF_RED);  // [2 phases][4 quarters][128 rows]
         uint64_t* pair = &pair_bar[q4];
         const float c = p.c;
         const bool tracing = p.dbg_m != nullptr && qt == p.trace_tile;
-        float m_run = -INFINITY, l = 0.0f;  // l: this half's sum
+        float m_run = -INFINITY, l = 0.0f;  // l: this quarter's sum
         bool ok = true;
-        int j = 0;
-        for (; j < nb && ok; ++j) {
+        for (int j = 0; j < nb && ok; ++j) {
             ok = __all_sync(0xffffffffu, mbar_wait(s_full, (uint32_t)(j & 1), p.timeout_ns, abort));
             if (!ok) break;
             tc_fence_after();
-            const int64_t k0 = (int64_t)j * 256 + h * 128;  // this half's first key
-            const int nvalid = (int)(p.T_kv - k0 >= 128 ? 128 : (p.T_kv > k0 ? p.T_kv - k0 : 0));
-            // pass 1: the half's maximum of s over its valid keys; c > 0, so the block's
+            const int64_t k0 = (int64_t)j * 256 + qq * 64;  // this quarter's first key
+            const int nvalid = (int)(p.T_kv - k0 >= 64 ? 64 : (p.T_kv > k0 ? p.T_kv - k0 : 0));
+            // pass 1: the quarter's maximum of s over its valid keys; c > 0, so the block's
             // max fl(s c) is fl(max s * c)
             float mx = -INFINITY;
-            if (nvalid == 128) {
-#pragma unroll 1
-                for (int ch = 0; ch < 4; ch += 2) {
-                    uint32_t v[32], w[32];
-                    tmem_ld_32x32b_x32(t_s + ch * 32, v);
-                    tmem_ld_32x32b_x32(t_s + ch * 32 + 32, w);
-                    tmem_wait_ld();
-                    tmem_tie(v);
-                    tmem_tie(w);
-                    float t[32];
+            {
+                uint32_t v[32], w[32];
+                tmem_ld_32x32b_x32(t_s, v);
+                tmem_ld_32x32b_x32(t_s + 32, w);
+                tmem_wait_ld();
+                tmem_tie(v);
+                tmem_tie(w);
+                float t[32];
+                if (nvalid == 64) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) t[i] = fmaxf(__uint_as_float(v[i]), __uint_as_float(w[i]));
-#pragma unroll
-                    for (int n = 16; n >= 1; n >>= 1)
-#pragma unroll
-                        for (int i = 0; i < n; ++i) t[i] = fmaxf(t[i], t[i + n]);
-                    mx = fmaxf(mx, t[0]);
-                }
-            } else {
-#pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(t_s + ch * 32, v);
-                    tmem_wait_ld();
-                    tmem_tie(v);
+                } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
-                        if (ch * 32 + i < nvalid) mx = fmaxf(mx, __uint_as_float(v[i]));
+                        t[i] = fmaxf(i < nvalid ? __uint_as_float(v[i]) : -INFINITY,
+                                     32 + i < nvalid ? __uint_as_float(w[i]) : -INFINITY);
                 }
+#pragma unroll
+                for (int n = 16; n >= 1; n >>= 1)
+#pragma unroll
+                    for (int i = 0; i < n; ++i) t[i] = fmaxf(t[i], t[i + n]);
+                mx = t[0];
             }
-            red[((j & 1) * 2 + h) * 128 + r] = mx;
+            red[((j & 1) * 4 + qq) * 128 + r] = mx;
             __syncwarp();
             if (lane == 0) mbar_arrive(pair);
             ok = __all_sync(0xffffffffu, mbar_wait(pair, (uint32_t)(j & 1), p.timeout_ns, abort));
             if (!ok) break;
-            const float mb = fmaxf(mx, red[((j & 1) * 2 + (h ^ 1)) * 128 + r]);
+            const float* rj = red + (j & 1) * 512 + r;
+            const float mb = fmaxf(fmaxf(rj[0], rj[128]), fmaxf(rj[256], rj[384]));
             const float m_new = fmaxf(m_run, __fmul_rn(mb, c));
             // P~_{j-1} V_{j-1} must be done before the P~ tile, its atoms or O are touched
             if (j > 0) {
@@ -316,27 +312,24 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 tc_fence_after();
             }
             // O and l follow the new maximum: O *= 2^(m_prev - m_new) (whole warp, a factor of 1
-            // for rows whose maximum did not grow); each half rescales its 64 columns of O
+            // for rows whose maximum did not grow); each quarter rescales its 32 columns of O
             const bool grow = (j > 0) && (m_new > m_run);
             const bool warp_grow = __any_sync(0xffffffffu, grow);
             if (warp_grow) {
                 const float f = grow ? exp2f(__fsub_rn(m_run, m_new)) : 1.0f;
                 l = __fmul_rn(l, f);
-#pragma unroll 1
-                for (int ch = 0; ch < 2; ++ch) {
-                    uint32_t o[32];
-                    tmem_ld_32x32b_x32(t_o + ch * 32, o);
-                    tmem_wait_ld();
-                    tmem_tie(o);
+                uint32_t o[32];
+                tmem_ld_32x32b_x32(t_o, o);
+                tmem_wait_ld();
+                tmem_tie(o);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), f));
-                    tmem_st_32x32b_x16(t_o + ch * 32, *reinterpret_cast<const uint32_t(*)[16]>(o));
-                    tmem_st_32x32b_x16(t_o + ch * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(o + 16));
-                }
+                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), f));
+                tmem_st_32x32b_x16(t_o, *reinterpret_cast<const uint32_t(*)[16]>(o));
+                tmem_st_32x32b_x16(t_o + 16, *reinterpret_cast<const uint32_t(*)[16]>(o + 16));
             }
             // pass 2: P~ = exp2(fl(fl(s c) - m_new)), MXFP4 groups of 32 keys, into row r of the
             // 128-byte-swizzled P~ tile (16-byte granule g at g ^ (r % 8))
-            uint32_t word = 0u;
+            uint32_t bytes2 = 0u;
             float lb = 0.0f;
             const uint32_t prow = smem_u32(sP) + (uint32_t)r * 128u;
             auto chunk = [&](int ch, auto full_tag) {
@@ -351,8 +344,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                     const bool valid = FULL || ch * 32 + i < nvalid;
                     pv[i] = valid ? exp2f(__fsub_rn(__fmul_rn(__uint_as_float(v[i]), c), m_new)) : 0.0f;
                 }
-                // the 32 weights summed as a pairwise tree, then added to the half's block sum in
-                // order; their maximum by the same tree
+                // the 32 weights summed as a pairwise tree, then added to the quarter's block sum
+                // in order; their maximum by the same tree
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     part[i] = __fadd_rn(pv[2 * i], pv[2 * i + 1]);
@@ -366,39 +359,40 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                         mxp[i] = fmaxf(mxp[i], mxp[i + w]);
                     }
                 lb = __fadd_rn(lb, part[0]);
-                const float amax = mxp[0];
-                const uint32_t sfb = mx_scale_byte<2>(amax);
+                const uint32_t sfb = mx_scale_byte<2>(mxp[0]);
                 const float inv = mx_inv_scale(sfb);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) pv[i] = __fmul_rn(pv[i], inv);
                 uint32_t cw[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) cw[q] = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(pv + 8 * q));
-                const int gch = h * 4 + ch;  // the chunk's 16-byte granule in the 256-key row
+                const int gch = qq * 2 + ch;  // the chunk's 16-byte granule in the 256-key row
                 st_shared_v4(prow + (uint32_t)((gch ^ (r & 7)) * 16), cw[0], cw[1], cw[2], cw[3]);
-                word |= sfb << (8 * ch);
+                bytes2 |= sfb << (8 * ch);
                 if (tracing) {
                     const int64_t d = (int64_t)j * 128 + r;
                     *reinterpret_cast<uint4*>(p.dbg_codes + d * 128 + gch * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
                     p.dbg_sf[d * 8 + gch] = (uint8_t)sfb;
                 }
             };
-            if (nvalid == 128) {
-#pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) chunk(ch, std::true_type{});
+            if (nvalid == 64) {
+                chunk(0, std::true_type{});
+                chunk(1, std::true_type{});
             } else {
-#pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) chunk(ch, std::false_type{});
+                chunk(0, std::false_type{});
+                chunk(1, std::false_type{});
             }
             l = __fadd_rn(l, lb);
             // S_j is read: the MMA warp may compute S_{j+1}
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_free);
-            // the row's scale word into this half's P~ atom (keys 0-127 or 128-255)
-            *reinterpret_cast<uint32_t*>(sPSF + h * 512 + (r & 31) * 16 + (r >> 5) * 4) = word;
+            // the row's two scale bytes into its P~ atom (keys 0-127 or 128-255): bytes
+            // 2 (qq % 2) and 2 (qq % 2) + 1 of the row's word
+            *reinterpret_cast<uint16_t*>(sPSF + (qq >> 1) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (qq & 1) * 2) =
+                (uint16_t)bytes2;
             if (warp_grow) tmem_wait_st();
-            if (tracing && h == 0) p.dbg_m[(int64_t)j * 128 + r] = m_new;
+            if (tracing && qq == 0) p.dbg_m[(int64_t)j * 128 + r] = m_new;
             // the tile and atoms are written by threads and read by the tensor core
             fence_proxy_async_smem();
             tc_fence_before();
@@ -406,9 +400,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             if (lane == 0) mbar_arrive(p_full);
             m_run = m_new;
         }
-        // the two halves' sums added in a fixed order, then O / l rounded once to bf16
+        // the four quarters' sums added in a fixed order, then O / l rounded once to bf16
         if (ok) {
-            red[((nb & 1) * 2 + h) * 128 + r] = l;
+            red[((nb & 1) * 4 + qq) * 128 + r] = l;
             __syncwarp();
             if (lane == 0) mbar_arrive(pair);
             ok = __all_sync(0xffffffffu, mbar_wait(pair, (uint32_t)(nb & 1), p.timeout_ns, abort));
@@ -416,28 +410,26 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)((nb - 1) & 1), p.timeout_ns, abort));
         if (ok) {
             tc_fence_after();
-            const float lt = __fadd_rn(red[((nb & 1) * 2) * 128 + r], red[((nb & 1) * 2 + 1) * 128 + r]);
+            const float* rl = red + (nb & 1) * 512 + r;
+            const float lt = __fadd_rn(__fadd_rn(rl[0], rl[128]), __fadd_rn(rl[256], rl[384]));
             const float inv_l = __frcp_rn(lt);
-#pragma unroll 1
-            for (int ch = 0; ch < 2; ++ch) {
-                uint32_t o[32];
-                tmem_ld_32x32b_x32(t_o + ch * 32, o);
-                tmem_wait_ld();
-                tmem_tie(o);
-                if (real) {
-                    uint32_t w[16];
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(t_o, o);
+            tmem_wait_ld();
+            tmem_tie(o);
+            if (real) {
+                uint32_t w[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(o[2 * i]), inv_l),
-                                                                 __fmul_rn(__uint_as_float(o[2 * i + 1]), inv_l));
-                        w[i] = *reinterpret_cast<uint32_t*>(&b);
-                    }
-                    uint4* dst = reinterpret_cast<uint4*>(p.o + row * 128 + h * 64 + ch * 32);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                for (int i = 0; i < 16; ++i) {
+                    __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(o[2 * i]), inv_l),
+                                                             __fmul_rn(__uint_as_float(o[2 * i + 1]), inv_l));
+                    w[i] = *reinterpret_cast<uint32_t*>(&b);
                 }
+                uint4* dst = reinterpret_cast<uint4*>(p.o + row * 128 + qq * 32);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
             }
-            if (p.stats != nullptr && real && h == 0) p.stats[row] = make_float2(m_run, lt);
+            if (p.stats != nullptr && real && qq == 0) p.stats[row] = make_float2(m_run, lt);
         } else if (lane == 0) {
             attn_fail(p, abort);
         }

@@ -423,9 +423,10 @@ fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p
  * maximum m_j = max(m_{j-1}, max fl(s c)) over the block's keys < T_kv (c = fp32(scale *
  * log2 e)), the weights p~ = exp2(fl(fl(s c) - m_j)) quantized as MXFP4 in groups of 32 keys,
  * O_j = O_{j-1} f_j + deq(P~_j) deq(V_j) with f_j = exp2(fl(m_{j-1} - m_j)) (1 when the
- * maximum did not grow); the sum is kept per half block (keys 0-127 and 128-255 of every
- * block): l_h = fl(fl(l_h f_j) + the half's four pairwise-tree sums of 32 weights, added in key
- * order), and l = fl(l_0 + l_1).  The output is o = bf16_rn(O fl(1 / l)).  The weights are
+ * maximum did not grow); the sum is kept per quarter block (keys 64 q .. 64 q + 63 of every
+ * block): l_q = fl(fl(l_q f_j) + the quarter's two pairwise-tree sums of 32 weights, added in
+ * key order), and l = fl(fl(l_0 + l_1) + fl(l_2 + l_3)).  The output is o = bf16_rn(O fl(1 /
+ * l)).  The weights are
  * thus quantized against the running maximum, not the row's final one as
  * fp4_attn_softmax_quant does, and S stays in fp32.
  *   q_codes / q_sf, k_codes / k_sf   fp4_quantize_heads' buffers (T_q resp. T_kv tokens)
