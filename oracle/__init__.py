@@ -403,6 +403,18 @@ def dequant_mx_rows(codes, sf_rows) -> np.ndarray:
     return (vals.reshape(R, K // 32, 32) * np.ldexp(1.0, sf_rows - 127)[..., None]).reshape(R, K)
 
 
+def dequant_nv_rows(codes, sf_rows, g: float) -> np.ndarray:
+    """NVFP4 rows in fp64 from codes [R, K/2] (low nibble first) and their E4M3 scale bytes
+    [R, K/16] in row order: value = e2m1(code) dec(byte) g."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    sf_rows = np.asarray(sf_rows, dtype=np.uint8)
+    dec = np.array([e4m3_decode(b) for b in range(256)])
+    nib = np.stack([codes & 15, codes >> 4], axis=-1).reshape(codes.shape[0], -1)
+    vals = _E2M1[nib]
+    R, K = vals.shape
+    return (vals.reshape(R, K // 16, 16) * (dec[sf_rows] * float(g))[..., None]).reshape(R, K)
+
+
 def flash_maxima(s: np.ndarray, T_kv: int, scale: float, block: int = FLASH_BLOCK) -> np.ndarray:
     """Running maxima [R, nblk] (nblk = ceil(T_kv / block)) of exact scores s [R, >= T_kv]:
     m[r, j] = max of s[r, k] c over the keys k < min(T_kv, (j + 1) block), c = softmax_c(scale)."""
@@ -436,12 +448,14 @@ def flash_combine(p_vals: np.ndarray, m: np.ndarray, w: np.ndarray, block: int =
 
 
 def flash_pv_rows(p_codes, p_sf_rows, m: np.ndarray, vt_heads, head: int, T_kv_pad: int,
-                  block: int = FLASH_BLOCK):
-    """flash_combine of the MXFP4 weights (codes [R, nblk * block / 2], scale bytes
-    [R, nblk * block / 32] in row order) with V_head^T dequantized from quantize_heads_vt."""
+                  block: int = FLASH_BLOCK, fmt: int = MX, g_p: float | None = None, g_v: float | None = None):
+    """flash_combine of the quantized weights (codes [R, nblk * block / 2], scale bytes
+    [R, nblk * block / G] in row order; NVFP4 under the global g_p) with V_head^T dequantized
+    from quantize_heads_vt (NVFP4 under g_v)."""
     vc, vs = vt_heads
-    w = dequant_fp4(MX, vc[head], vs[head], T_kv_pad, 1.0)
-    return flash_combine(dequant_mx_rows(p_codes, p_sf_rows), m, w, block)
+    w = dequant_fp4(fmt, vc[head], vs[head], T_kv_pad, 1.0 if fmt == MX else g_v)
+    a = dequant_mx_rows(p_codes, p_sf_rows) if fmt == MX else dequant_nv_rows(p_codes, p_sf_rows, g_p)
+    return flash_combine(a, m, w, block)
 
 
 def flash_sum(s: np.ndarray, T_kv: int, scale: float, m_last: np.ndarray) -> np.ndarray:
@@ -452,16 +466,17 @@ def flash_sum(s: np.ndarray, T_kv: int, scale: float, m_last: np.ndarray) -> np.
 
 
 def flash_weight_interval(s: np.ndarray, es: np.ndarray, T_kv: int, scale: float, m: np.ndarray,
-                          block: int = FLASH_BLOCK):
+                          block: int = FLASH_BLOCK, rel: float = 2.0 ** -23):
     """(lo, hi) [R, nblk * block] holding the fp32 weight exp2(fl(fl(s' c) - m_j)) for any fp32
-    score s' with |s' - s| <= es (the exponent off by at most c es + 2^-23 (|s c| + |m_j|): the
-    score's error and the two roundings) and exp2f within 2 ulp (relative 2^-22, taken as
-    2^-21); keys >= T_kv give [0, 0]."""
+    score s' with |s' - s| <= es (the exponent off by at most c es + rel (|s c| + |m_j|): the
+    score's error and the roundings, rel = 2^-23 for the two of fl(fl(s c) - m), 2^-22 when
+    the scores' NVFP4 globals are folded into c as well) and exp2f within 2 ulp (relative
+    2^-22, taken as 2^-21); keys >= T_kv give [0, 0]."""
     nb = m.shape[1]
     c = softmax_c(scale)
     u = np.asarray(s, dtype=np.float64)[:, :T_kv] * c
     mj = np.repeat(m, block, axis=1)[:, :T_kv]
-    d = c * np.asarray(es, dtype=np.float64)[:, :T_kv] + 2.0 ** -23 * (np.abs(u) + np.abs(mj))
+    d = c * np.asarray(es, dtype=np.float64)[:, :T_kv] + rel * (np.abs(u) + np.abs(mj))
     lo = np.zeros((u.shape[0], nb * block))
     hi = np.zeros((u.shape[0], nb * block))
     lo[:, :T_kv] = np.exp2(u - mj - d) * (1.0 - 2.0 ** -21)

@@ -236,6 +236,20 @@ def test_dequant_mx_rows_matches_the_atom_layout_dequantizer():
     np.testing.assert_array_equal(oracle.dequant_mx_rows(codes, sf), oracle.dequant_fp4(MX, codes, atoms, K))
 
 
+def test_dequant_nv_rows_matches_the_atom_layout_dequantizer():
+    """Row-order NVFP4 dequantization (E4M3 scales, a global) equals the pinned dequantizer
+    fed the same bytes in the 128x4 atom layout."""
+    rng = np.random.default_rng(15)
+    R, K, g = 130, 256, 0.0123
+    codes = rng.integers(0, 256, size=(R, K // 2), dtype=np.uint8)
+    sf = rng.integers(0, 127, size=(R, K // 16), dtype=np.uint8)
+    atoms = np.zeros(oracle.sf_bytes(R, K // 16), dtype=np.uint8)
+    for i in range(R):
+        for j in range(K // 16):
+            atoms[oracle.sf_offset(i, j, K // 16)] = sf[i, j]
+    np.testing.assert_array_equal(oracle.dequant_nv_rows(codes, sf, g), oracle.dequant_fp4(NV, codes, atoms, K, g))
+
+
 def test_flash_maxima_and_sum_reduce_to_the_plain_softmax():
     """The last running maximum is the row maximum of s c, the maxima never fall, a block's
     maximum is reached inside it or before; with m_last the flash sum is the plain softmax
