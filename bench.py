@@ -60,7 +60,7 @@ def parse():
                     help="tokens; smaller values run a reduced case of the same kernels (profiling only)")
     ap.add_argument("--attn-tokens", type=int, default=0,
                     help="profiling only: run one head of FP4 attention (K quantizer over 40 heads of 128, head 17's "
-                         "scores, softmax weights + quantize, P V; MXFP4: then the fused head) at this many "
+                         "scores, softmax weights + quantize, P V, then the fused head) at this many "
                          "tokens for --steps iterations, print timings, exit")
     return ap.parse_args()
 
@@ -104,8 +104,7 @@ def attn_profile(args):
         e[3].record()
         fb.attn_pv(p, vt, T, T, 17, fmt, gp, gv, o=o)
         e[4].record()
-        if fmt == "mxfp4":
-            fb.attn_fused(qh, kh, vt, T, T, 17, 128 ** -0.5, o=o)
+        fb.attn_fused(qh, kh, vt, T, T, 17, 128 ** -0.5, fmt, gq, gk, gv, gp, o=o)
         e[5].record()
         torch.cuda.synchronize()
         for i in range(5):
@@ -567,13 +566,12 @@ def extra_workloads(fb, torch, args, steps: int = 20, warmup: int = 3):
         o_buf = fb.attn_pv((pc, ps, st), vt, Ta, Ta, 17, fmt, g_p, g_v)
         out[f"{fmt}_attn_pv_head_75600x128x75648"] = timed(
             lambda: fb.attn_pv((pc, ps, st), vt, Ta, Ta, 17, fmt, g_p, g_v, o=o_buf), 2.0 * Ta * kp * 128, n=10)
-        if fmt == "mxfp4":
-            # the same head in one kernel (streaming form): S and P~ never leave the SM
-            st_f = torch.empty((Ta, 2), dtype=torch.float32, device="cuda")
-            out["mxfp4_attn_fused_head_75600x75648x128"] = timed(
-                lambda: fb.attn_fused(qh, kh, vt, Ta, Ta, 17, 128 ** -0.5, o=o_buf, stats=st_f), 4.0 * Ta * kp * 128,
-                n=10)
-            del st_f
+        # the same head in one kernel (streaming form): S and P~ never leave the SM
+        st_f = torch.empty((Ta, 2), dtype=torch.float32, device="cuda")
+        out[f"{fmt}_attn_fused_head_75600x75648x128"] = timed(
+            lambda: fb.attn_fused(qh, kh, vt, Ta, Ta, 17, 128 ** -0.5, fmt, g_q, g_k, g_v, g_p, o=o_buf, stats=st_f),
+            4.0 * Ta * kp * 128, n=10)
+        del st_f
         del va, vt, pc, ps, st, o_buf
         del qa, ka, qh, kh, kc_buf, ks_buf, s_buf
     # W4A8 SVDQuant linear at the TI2V-5B shape (MXFP8 activations, rank 32)

@@ -91,9 +91,10 @@ def lib():
             "fp4_quantize_heads_vt": (I, [I, P, I64, I64, I64, P, P, P, P]),
             "fp4_attn_softmax_quant": (I, [I, P, I64, I64, ctypes.c_float, P, P, P, P, P]),
             "fp4_attn_pv": (I, [I, P, P, P, I64, I64, P, P, P, I64, I64, I64, P, P, P]),
-            "fp4_attn_fused": (I, [I, P, P, I64, P, P, I64, P, P, I64, I64, I64, ctypes.c_float, P, P, P]),
-            "fp4_attn_fused_trace": (I, [I, P, P, I64, P, P, I64, P, P, I64, I64, I64, ctypes.c_float, P, P, I64,
-                                         P, P, P, P]),
+            "fp4_attn_fused": (I, [I, P, P, I64, P, P, I64, P, P, I64, I64, I64, ctypes.c_float, P, P, P, P, P, P,
+                                   P]),
+            "fp4_attn_fused_trace": (I, [I, P, P, I64, P, P, I64, P, P, I64, I64, I64, ctypes.c_float, P, P, P, P, P,
+                                         P, I64, P, P, P, P]),
             "fp4_sync_status": (I, [P]),
             "fp4_status_string": (ctypes.c_char_p, [I]),
             "fp4_set_wait_timeout_ns": (None, [ctypes.c_uint64]),
@@ -304,19 +305,19 @@ def fp4_attn_pv(fmt, p_codes, p_sf, p_global, T_q: int, T_kv: int, vt_codes, vt_
 
 
 def fp4_attn_fused(fmt, q_codes, q_sf, T_q: int, k_codes, k_sf, T_kv: int, vt_codes, vt_sf, H: int, D: int,
-                   head: int, scale: float, stats, o, stream=None):
+                   head: int, scale: float, g_q, g_k, g_v, p_global, stats, o, stream=None):
     _check(lib().fp4_attn_fused(_fmt(fmt), _ptr(q_codes), _ptr(q_sf), T_q, _ptr(k_codes), _ptr(k_sf), T_kv,
-                                _ptr(vt_codes), _ptr(vt_sf), H, D, head, scale, _ptr(stats), _ptr(o),
-                                _stream(stream)), "fp4_attn_fused")
+                                _ptr(vt_codes), _ptr(vt_sf), H, D, head, scale, _ptr(g_q), _ptr(g_k), _ptr(g_v),
+                                _ptr(p_global), _ptr(stats), _ptr(o), _stream(stream)), "fp4_attn_fused")
 
 
 def fp4_attn_fused_trace(fmt, q_codes, q_sf, T_q: int, k_codes, k_sf, T_kv: int, vt_codes, vt_sf, H: int, D: int,
-                         head: int, scale: float, stats, o, trace_tile: int, trace_m, trace_codes, trace_sf,
-                         stream=None):
+                         head: int, scale: float, g_q, g_k, g_v, p_global, stats, o, trace_tile: int, trace_m,
+                         trace_codes, trace_sf, stream=None):
     _check(lib().fp4_attn_fused_trace(_fmt(fmt), _ptr(q_codes), _ptr(q_sf), T_q, _ptr(k_codes), _ptr(k_sf), T_kv,
-                                      _ptr(vt_codes), _ptr(vt_sf), H, D, head, scale, _ptr(stats), _ptr(o),
-                                      trace_tile, _ptr(trace_m), _ptr(trace_codes), _ptr(trace_sf),
-                                      _stream(stream)), "fp4_attn_fused_trace")
+                                      _ptr(vt_codes), _ptr(vt_sf), H, D, head, scale, _ptr(g_q), _ptr(g_k),
+                                      _ptr(g_v), _ptr(p_global), _ptr(stats), _ptr(o), trace_tile, _ptr(trace_m),
+                                      _ptr(trace_codes), _ptr(trace_sf), _stream(stream)), "fp4_attn_fused_trace")
 
 
 def fp4_sync_status(stream=None) -> int:
@@ -470,13 +471,13 @@ def attn_pv(p, vt_heads, T_q: int, T_kv: int, head: int, fmt="mxfp4", p_global=N
     return o
 
 
-def attn_fused(q_heads, k_heads, vt_heads, T_q: int, T_kv: int, head: int, scale: float, o=None, stats=None,
-               trace_tile=None, stream=None):
-    """One head's MXFP4 attention in one kernel (streaming form) from quantize_heads' Q and K and
-    quantize_heads_vt's V^T: bf16 [T_q, 128].  stats: an fp32 [T_q, 2] tensor to receive (final
-    running maximum, l), or None.  trace_tile: a query tile whose per-block running maxima, P~
-    codes and scale bytes are returned too, as (o, (m [nblk, 128], codes [nblk, 128, 128],
-    sf [nblk, 128, 8]))."""
+def attn_fused(q_heads, k_heads, vt_heads, T_q: int, T_kv: int, head: int, scale: float, fmt="mxfp4", g_q=None,
+               g_k=None, g_v=None, p_global=None, o=None, stats=None, trace_tile=None, stream=None):
+    """One head's FP4 attention in one kernel (streaming form) from quantize_heads' Q and K and
+    quantize_heads_vt's V^T: bf16 [T_q, 128].  NVFP4: the device fp32 globals of Q, K, V and P~
+    (P_GLOBAL_NVFP4).  stats: an fp32 [T_q, 2] tensor to receive (final running maximum, l), or
+    None.  trace_tile: a query tile whose per-block running maxima, P~ codes and scale bytes are
+    returned too, as (o, (m [nblk, 128], codes [nblk, 128, 128], sf [nblk, 128, 256 / G]))."""
     import torch
 
     qc, qs = q_heads
@@ -487,14 +488,16 @@ def attn_fused(q_heads, k_heads, vt_heads, T_q: int, T_kv: int, head: int, scale
     if o is None:
         o = torch.empty((T_q, D), dtype=torch.bfloat16, device=qc.device)
     if trace_tile is None:
-        fp4_attn_fused("mxfp4", qc, qs, T_q, kc, ks, T_kv, vc, vs, H, D, head, scale, stats, o, stream)
+        fp4_attn_fused(fmt, qc, qs, T_q, kc, ks, T_kv, vc, vs, H, D, head, scale, g_q, g_k, g_v, p_global, stats, o,
+                       stream)
         return o
     nblk = ((T_kv + 127) // 128 * 128 + 255) // 256
+    G = 32 if _fmt(fmt) == MXFP4 else 16
     tm = torch.empty((nblk, 128), dtype=torch.float32, device=qc.device)
     tc = torch.empty((nblk, 128, 128), dtype=torch.uint8, device=qc.device)
-    ts = torch.empty((nblk, 128, 8), dtype=torch.uint8, device=qc.device)
-    fp4_attn_fused_trace("mxfp4", qc, qs, T_q, kc, ks, T_kv, vc, vs, H, D, head, scale, stats, o, trace_tile, tm,
-                         tc, ts, stream)
+    ts = torch.empty((nblk, 128, 256 // G), dtype=torch.uint8, device=qc.device)
+    fp4_attn_fused_trace(fmt, qc, qs, T_q, kc, ks, T_kv, vc, vs, H, D, head, scale, g_q, g_k, g_v, p_global, stats, o,
+                         trace_tile, tm, tc, ts, stream)
     return o, (tm, tc, ts)
 
 

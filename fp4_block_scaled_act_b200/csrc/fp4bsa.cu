@@ -102,8 +102,10 @@ fp4_status_t device_state(DeviceState** out) {
                                      Gemm2Cfg<G_MXFP4>::SMEM_BYTES) != cudaSuccess ||
                 cudaFuncSetAttribute(gemm2_kernel<G_NVFP4, 0, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Gemm2Cfg<G_NVFP4>::SMEM_BYTES) != cudaSuccess ||
-                cudaFuncSetAttribute(attn_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM) !=
-                    cudaSuccess)
+                cudaFuncSetAttribute(attn_fused_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     ATT_SMEM) != cudaSuccess ||
+                cudaFuncSetAttribute(attn_fused_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     ATT_SMEM) != cudaSuccess)
                 return FP4_ERR_CUDA;
             {
                 constexpr int R = (int)Gemm2Cfg<G_MXFP4>::REG_LAUNCH;
@@ -726,11 +728,19 @@ fp4_status_t fp4_attn_scores(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_
 namespace {
 fp4_status_t attn_fused_impl(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,
                              const uint8_t* k_codes, const uint8_t* k_sf, int64_t T_kv, const uint8_t* vt_codes,
-                             const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale, void* stats,
-                             void* o_bf16, int64_t trace_tile, float* trace_m, uint8_t* trace_codes,
+                             const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale,
+                             const float* g_q, const float* g_k, const float* g_v, const float* p_global,
+                             void* stats, void* o_bf16, int64_t trace_tile, float* trace_m, uint8_t* trace_codes,
                              uint8_t* trace_sf, void* stream) {
-    if (fmt != FP4_FMT_MXFP4 || !q_codes || !q_sf || !k_codes || !k_sf || !vt_codes || !vt_sf || !o_bf16)
+    if (!fmt_ok(fmt) || !q_codes || !q_sf || !k_codes || !k_sf || !vt_codes || !vt_sf || !o_bf16)
         return FP4_ERR_INVALID_ARG;
+    const bool nv = fmt == FP4_FMT_NVFP4;
+    // NVFP4 takes all four globals, MXFP4 none
+    if ((nv && (!g_q || !g_k || !g_v || !p_global)) || (!nv && (g_q || g_k || g_v || p_global)))
+        return FP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(g_q) | reinterpret_cast<uintptr_t>(g_k) | reinterpret_cast<uintptr_t>(g_v) |
+         reinterpret_cast<uintptr_t>(p_global)) & 3u)
+        return FP4_ERR_MISALIGNED;
     if (T_q < 1 || T_kv < 1 || H < 1 || head < 0 || head >= H) return FP4_ERR_INVALID_ARG;
     if (!(scale > 0.0f) || !(scale < 3.0e38f)) return FP4_ERR_INVALID_ARG;
     if (D != FP4_HEAD_DIM) return FP4_ERR_UNSUPPORTED_SHAPE;
@@ -770,12 +780,16 @@ fp4_status_t attn_fused_impl(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_
     p.v_sf = vt_sf + (size_t)head * fp4_sf_bytes(fmt, D, tk_pad);
     p.o = static_cast<__nv_bfloat16*>(o_bf16);
     p.stats = static_cast<float2*>(stats);
+    p.g_q = g_q, p.g_k = g_k, p.g_v = g_v, p.g_p = p_global;
     p.trace_tile = tracing ? (int)trace_tile : -1;
     p.dbg_m = trace_m, p.dbg_codes = trace_codes, p.dbg_sf = trace_sf;
     p.timeout_ns = g_timeout_ns;
     p.status = ds->status;
-    attn_fused_kernel<<<(unsigned)(tq_pad / 128), ATT_THREADS, ATT_SMEM, static_cast<cudaStream_t>(stream)>>>(tq, tk,
-                                                                                                         tv, p);
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (nv)
+        attn_fused_kernel<true><<<(unsigned)(tq_pad / 128), ATT_THREADS, ATT_SMEM, cs>>>(tq, tk, tv, p);
+    else
+        attn_fused_kernel<false><<<(unsigned)(tq_pad / 128), ATT_THREADS, ATT_SMEM, cs>>>(tq, tk, tv, p);
     return launched();
 }
 }  // namespace
@@ -784,19 +798,21 @@ extern "C" {
 
 fp4_status_t fp4_attn_fused(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,
                             const uint8_t* k_codes, const uint8_t* k_sf, int64_t T_kv, const uint8_t* vt_codes,
-                            const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale, void* stats,
-                            void* o_bf16, void* stream) {
-    return attn_fused_impl(fmt, q_codes, q_sf, T_q, k_codes, k_sf, T_kv, vt_codes, vt_sf, H, D, head, scale, stats,
-                           o_bf16, -1, nullptr, nullptr, nullptr, stream);
+                            const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale, const float* g_q,
+                            const float* g_k, const float* g_v, const float* p_global, void* stats, void* o_bf16,
+                            void* stream) {
+    return attn_fused_impl(fmt, q_codes, q_sf, T_q, k_codes, k_sf, T_kv, vt_codes, vt_sf, H, D, head, scale, g_q, g_k,
+                           g_v, p_global, stats, o_bf16, -1, nullptr, nullptr, nullptr, stream);
 }
 
 fp4_status_t fp4_attn_fused_trace(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,
                                   const uint8_t* k_codes, const uint8_t* k_sf, int64_t T_kv, const uint8_t* vt_codes,
-                                  const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale, void* stats,
-                                  void* o_bf16, int64_t trace_tile, float* trace_m, uint8_t* trace_codes,
-                                  uint8_t* trace_sf, void* stream) {
-    return attn_fused_impl(fmt, q_codes, q_sf, T_q, k_codes, k_sf, T_kv, vt_codes, vt_sf, H, D, head, scale, stats,
-                           o_bf16, trace_tile, trace_m, trace_codes, trace_sf, stream);
+                                  const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale,
+                                  const float* g_q, const float* g_k, const float* g_v, const float* p_global,
+                                  void* stats, void* o_bf16, int64_t trace_tile, float* trace_m,
+                                  uint8_t* trace_codes, uint8_t* trace_sf, void* stream) {
+    return attn_fused_impl(fmt, q_codes, q_sf, T_q, k_codes, k_sf, T_kv, vt_codes, vt_sf, H, D, head, scale, g_q, g_k,
+                           g_v, p_global, stats, o_bf16, trace_tile, trace_m, trace_codes, trace_sf, stream);
 }
 
 fp4_status_t fp4_linear(fp4_fmt_t fmt, const void* x_bf16, int64_t M, int64_t K, int64_t N, const uint8_t* w_codes,

@@ -416,12 +416,13 @@ fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p
                          const float* v_global, int64_t H, int64_t D, int64_t head, const void* stats,
                          void* o_bf16, void* stream);
 
-/* One head's MXFP4 attention in one kernel, in the streaming (flash) form of the reading
+/* One head's FP4 attention in one kernel, in the streaming (flash) form of the reading
  * above (the Wan2.2-Animate-14B MXFP4 card, "Results": FP4 attention on Blackwell with
  * microscaling; the page gives no algorithm).  The keys are taken in blocks of 256; per
  * query row and block j: s = deq(q) deq(k)^T in fp32 (never rounded to bf16), the running
  * maximum m_j = max(m_{j-1}, max fl(s c)) over the block's keys < T_kv (c = fp32(scale *
- * log2 e)), the weights p~ = exp2(fl(fl(s c) - m_j)) quantized as MXFP4 in groups of 32 keys,
+ * log2 e)), the weights p~ = exp2(fl(fl(s c) - m_j)) quantized in groups of G keys (MXFP4:
+ * 32, E8M0 scales; NVFP4: 16, E4M3 scales under P~'s global p_global, 1/2688 for p <= 1),
  * O_j = O_{j-1} f_j + deq(P~_j) deq(V_j) with f_j = exp2(fl(m_{j-1} - m_j)) (1 when the
  * maximum did not grow); the sum is kept per quarter block (keys 64 q .. 64 q + 63 of every
  * block): l_q = fl(fl(l_q f_j) + the quarter's two pairwise-tree sums of 32 weights, added in
@@ -432,27 +433,33 @@ fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p
  *   q_codes / q_sf, k_codes / k_sf   fp4_quantize_heads' buffers (T_q resp. T_kv tokens)
  *   vt_codes / vt_sf                 fp4_quantize_heads_vt's buffers (T_kv tokens)
  *   scale   the softmax scale, > 0 and finite
+ *   g_q, g_k, g_v, p_global  (device) NVFP4: the fp32 globals of Q, K, V and P~; the scores'
+ *           pair is folded into the exponent multiplier, c' = fl(c fl(g_q g_k)) and
+ *           fl(s c) = fl(acc c'), and the output is o = bf16_rn(O fl(fl(p_global g_v) fl(1 / l)));
+ *           MXFP4: all four must be NULL
  *   stats   (device, out) [T_q] pairs of fp32 (final running maximum, l), or NULL
  *   o_bf16  (device, out) [T_q][D] bf16
- * MXFP4 only: fmt NVFP4 returns FP4_ERR_INVALID_ARG.  D = FP4_HEAD_DIM; H times T_q or T_kv
+ * Globals given for MXFP4 or missing for NVFP4 return FP4_ERR_INVALID_ARG.  D = FP4_HEAD_DIM; H times T_q or T_kv
  * rounded up to 128 must stay below 2^31 (else FP4_ERR_UNSUPPORTED_SHAPE).  One CTA per 128
  * query rows; a wait that runs out of time records FP4_ERR_TIMEOUT. */
 fp4_status_t fp4_attn_fused(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,
                             const uint8_t* k_codes, const uint8_t* k_sf, int64_t T_kv, const uint8_t* vt_codes,
-                            const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale, void* stats,
-                            void* o_bf16, void* stream);
+                            const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale, const float* g_q,
+                            const float* g_k, const float* g_v, const float* p_global, void* stats, void* o_bf16,
+                            void* stream);
 
 /* fp4_attn_fused that also records, for the 128 query rows of tile trace_tile (rows
  * 128 trace_tile ...), every block's intermediate values: trace_m [nblk][128] fp32 running
  * maxima, trace_codes [nblk][128][128] the P~_j codes (256 keys per row, two per byte, low
- * nibble first), trace_sf [nblk][128][8] their E8M0 scale bytes; nblk = ceil(T_kv_pad / 256).
+ * nibble first), trace_sf [nblk][128][256 / G] their scale bytes; nblk = ceil(T_kv_pad / 256).
  * A test hook with no counterpart on the pages: all three device pointers or none (then it
  * is fp4_attn_fused), 0 <= trace_tile < T_q_pad / 128. */
 fp4_status_t fp4_attn_fused_trace(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,
                                   const uint8_t* k_codes, const uint8_t* k_sf, int64_t T_kv, const uint8_t* vt_codes,
-                                  const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale, void* stats,
-                                  void* o_bf16, int64_t trace_tile, float* trace_m, uint8_t* trace_codes,
-                                  uint8_t* trace_sf, void* stream);
+                                  const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale,
+                                  const float* g_q, const float* g_k, const float* g_v, const float* p_global,
+                                  void* stats, void* o_bf16, int64_t trace_tile, float* trace_m,
+                                  uint8_t* trace_codes, uint8_t* trace_sf, void* stream);
 
 /* ----------------------------------------------------------------- status */
 

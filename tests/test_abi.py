@@ -151,18 +151,26 @@ def test_invalid_calls_rejected_before_launch(fb):
     assert L.fp4_attn_pv(0, A, A, None, 16, 16, A, A, None, 2, 64, 0, None, A, st) == 2
     assert L.fp4_attn_pv(0, A, A, None, 16, 16, A, A, None, 2, 128, 0, bad, A, st) == 3
     F = ctypes.c_float
-    # fused head: MXFP4 only, head < H, D = 128, scale > 0, aligned, 32-bit TMA rows
-    assert L.fp4_attn_fused(1, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), None, A, st) == 1
-    assert L.fp4_attn_fused(0, A, A, 16, A, A, 16, A, A, 2, 128, 2, F(0.1), None, A, st) == 1
-    assert L.fp4_attn_fused(0, A, A, 16, A, A, 16, A, A, 2, 64, 0, F(0.1), None, A, st) == 2
-    assert L.fp4_attn_fused(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.0), None, A, st) == 1
-    assert L.fp4_attn_fused(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), None, bad, st) == 3
-    assert L.fp4_attn_fused(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), bad, A, st) == 3
-    assert L.fp4_attn_fused(0, A, A, 16, A, A, 60000, A, A, 40000, 128, 0, F(0.1), None, A, st) == 2
+    # fused head: globals all (NVFP4) or none (MXFP4), head < H, D = 128, scale > 0, aligned,
+    # 32-bit TMA rows
+    N4 = (None, None, None, None)
+    G4 = (A, A, A, A)
+    assert L.fp4_attn_fused(1, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), *N4, None, A, st) == 1
+    assert L.fp4_attn_fused(1, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), A, A, A, None, None, A, st) == 1
+    assert L.fp4_attn_fused(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), *G4, None, A, st) == 1
+    assert L.fp4_attn_fused(1, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), A, A, A, A + 2, None, A, st) == 3
+    assert L.fp4_attn_fused(0, A, A, 16, A, A, 16, A, A, 2, 128, 2, F(0.1), *N4, None, A, st) == 1
+    assert L.fp4_attn_fused(0, A, A, 16, A, A, 16, A, A, 2, 64, 0, F(0.1), *N4, None, A, st) == 2
+    assert L.fp4_attn_fused(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.0), *N4, None, A, st) == 1
+    assert L.fp4_attn_fused(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), *N4, None, bad, st) == 3
+    assert L.fp4_attn_fused(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), *N4, bad, A, st) == 3
+    assert L.fp4_attn_fused(0, A, A, 16, A, A, 60000, A, A, 40000, 128, 0, F(0.1), *N4, None, A, st) == 2
     # trace: all three buffers or none, the tile inside the query rows
-    assert L.fp4_attn_fused_trace(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), None, A, 1, A, A, A, st) == 1
-    assert L.fp4_attn_fused_trace(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), None, A, 0, A, None, A, st) == 1
-    assert L.fp4_attn_fused_trace(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), None, A, 0, A, A, bad, st) == 3
+    assert L.fp4_attn_fused_trace(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), *N4, None, A, 1, A, A, A, st) == 1
+    assert L.fp4_attn_fused_trace(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), *N4, None, A, 0, A, None, A,
+                                  st) == 1
+    assert L.fp4_attn_fused_trace(0, A, A, 16, A, A, 16, A, A, 2, 128, 0, F(0.1), *N4, None, A, 0, A, A, bad,
+                                  st) == 3
 
 
 def test_product_path_has_no_oracle_import():
