@@ -387,6 +387,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 tmem_ld_32x32b_x32(t_s + ch * 32, v);
                 tmem_wait_ld();
                 tmem_tie(v);
+                if (ch == 1) {
+                    // the quarter's last read of S_j has landed: the MMA warp may compute S_{j+1}
+                    // while this chunk's weights are made
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(s_free);
+                }
                 float pv[32], part[16], mxp[16];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -453,10 +460,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 chunk(1, std::false_type{});
             }
             l = __fadd_rn(l, lb);
-            // S_j is read: the MMA warp may compute S_{j+1}
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_free);
             // the row's scale bytes into the P~ atoms: MXFP4 bytes 2 (qq % 2), +1 of the row's
             // word in atom qq / 2 (128 keys per atom); NVFP4 the whole word of atom qq (64 keys)
             if (NV)
