@@ -426,22 +426,21 @@ fp4_status_t fp4_attn_pv(fp4_fmt_t fmt, const uint8_t* p_codes, const uint8_t* p
  * O_j = O_{j-1} f_j + deq(P~_j) deq(V_j) with f_j = exp2(fl(m_{j-1} - m_j)) (1 when the
  * maximum did not grow); the sum is kept per quarter block (keys 64 q .. 64 q + 63 of every
  * block): l_q = fl(fl(l_q f_j) + the quarter's two pairwise-tree sums of 32 weights, added in
- * key order), and l = fl(fl(l_0 + l_1) + fl(l_2 + l_3)).  The output is o = bf16_rn(O fl(1 /
- * l)).  The weights are
- * thus quantized against the running maximum, not the row's final one as
- * fp4_attn_softmax_quant does, and S stays in fp32.
+ * key order), and l = fl(fl(l_0 + l_1) + fl(l_2 + l_3)).  The output is
+ * o = bf16_rn(O fl(1 / l)).  The weights are thus quantized against the running maximum,
+ * not the row's final one as fp4_attn_softmax_quant does, and S stays in fp32.
  *   q_codes / q_sf, k_codes / k_sf   fp4_quantize_heads' buffers (T_q resp. T_kv tokens)
  *   vt_codes / vt_sf                 fp4_quantize_heads_vt's buffers (T_kv tokens)
  *   scale   the softmax scale, > 0 and finite
  *   g_q, g_k, g_v, p_global  (device) NVFP4: the fp32 globals of Q, K, V and P~; the scores'
  *           pair is folded into the exponent multiplier, c' = fl(c fl(g_q g_k)) and
- *           fl(s c) = fl(acc c'), and the output is o = bf16_rn(O fl(fl(p_global g_v) fl(1 / l)));
- *           MXFP4: all four must be NULL
+ *           fl(s c) = fl(acc c') for the raw block-scaled product acc, and the output is
+ *           o = bf16_rn(O fl(fl(p_global g_v) fl(1 / l))); MXFP4: all four must be NULL
  *   stats   (device, out) [T_q] pairs of fp32 (final running maximum, l), or NULL
  *   o_bf16  (device, out) [T_q][D] bf16
- * Globals given for MXFP4 or missing for NVFP4 return FP4_ERR_INVALID_ARG.  D = FP4_HEAD_DIM; H times T_q or T_kv
- * rounded up to 128 must stay below 2^31 (else FP4_ERR_UNSUPPORTED_SHAPE).  One CTA per 128
- * query rows; a wait that runs out of time records FP4_ERR_TIMEOUT. */
+ * Globals given for MXFP4 or missing for NVFP4 return FP4_ERR_INVALID_ARG.  D = FP4_HEAD_DIM;
+ * H times T_q or T_kv rounded up to 128 must stay below 2^31 (else FP4_ERR_UNSUPPORTED_SHAPE).
+ * One CTA per 128 query rows; a wait that runs out of time records FP4_ERR_TIMEOUT. */
 fp4_status_t fp4_attn_fused(fp4_fmt_t fmt, const uint8_t* q_codes, const uint8_t* q_sf, int64_t T_q,
                             const uint8_t* k_codes, const uint8_t* k_sf, int64_t T_kv, const uint8_t* vt_codes,
                             const uint8_t* vt_sf, int64_t H, int64_t D, int64_t head, float scale, const float* g_q,
